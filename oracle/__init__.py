@@ -1,0 +1,180 @@
+"""float64 CPU oracle for causal linear attention -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The product
+path (the CUDA library and its Python binding) never imports it, and this
+package imports nothing from the product.
+
+The arithmetic lives in ``la_oracle.c`` (plain C, float64, OpenMP over
+independent (sequence, head, state-row) tasks); this module builds it with gcc
+and marshals numpy arrays to it.  What each function computes, and the passage
+it follows, is stated in the C file's header:
+
+* ``recurrent`` -- the token-by-token recurrence of "1.6 长上下文与高效注意力",
+  section 线性注意力 (displayed equation for o_t, S_t, z_t), with a per-head
+  constant decay gamma on the old state and the normaliser.
+* ``chunked``   -- the same result regrouped into chunks (a restatement used to
+  pin chunk-size invariance).
+* ``step``      -- one decode token on a given state.
+
+Inputs may be numpy float32, float64, or bfloat16 given as raw ``uint16`` bits
+(use :func:`bf16_bits`); they are upcast to float64 exactly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "la_oracle.c")
+_LIB = os.path.join(_HERE, "liblaoracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+PHI_IDENTITY, PHI_ELU1 = 0, 1
+_PHI = {"identity": PHI_IDENTITY, "elu1": PHI_ELU1, PHI_IDENTITY: PHI_IDENTITY, PHI_ELU1: PHI_ELU1}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile la_oracle.c into liblaoracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, i32, vp, dp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+        lib.oracle_recurrent.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, i32, dp, dp, i32]
+        lib.oracle_recurrent.restype = i32
+        lib.oracle_chunked.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i64, i32, i32, dp, dp, i32]
+        lib.oracle_chunked.restype = i32
+        lib.oracle_step.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, i32, i32]
+        lib.oracle_step.restype = i32
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def bf16_bits(x) -> np.ndarray:
+    """Raw bfloat16 bits (uint16) of a torch bfloat16 tensor, for the oracle."""
+    import torch  # local: only used to view torch bf16 storage
+
+    assert x.dtype == torch.bfloat16
+    return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _as_input(a):
+    """(contiguous array, oracle dtype code) for a numpy array or torch tensor."""
+    try:
+        import torch
+
+        if isinstance(a, torch.Tensor):
+            if a.dtype == torch.bfloat16:
+                return bf16_bits(a), BF16
+            a = a.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.float64:
+        return a, F64
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError("oracle inputs must be float32, float64 or bfloat16 bits, got %s" % a.dtype)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _prep(q, k, v, gamma, cu_seqlens):
+    q, dq = _as_input(q)
+    k, dk_ = _as_input(k)
+    v, dv_ = _as_input(v)
+    if not (dq == dk_ == dv_):
+        raise TypeError("q, k, v must share one dtype")
+    if q.ndim != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B, T, H, d_k] and v [B, T, H, d_v]")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(-1))
+    if g.size == 1 and H > 1:
+        g = np.full(H, g[0])
+    if g.size != H:
+        raise ValueError("gamma must have H entries")
+    cu = None
+    n_seqs = B
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n_seqs = cu.size - 1
+    return q, k, v, dq, B, T, H, dk, dv, g, cu, n_seqs
+
+
+def recurrent(q, k, v, gamma, cu_seqlens=None, phi="identity", normalize=False, nthreads=0):
+    """Token-by-token recurrence; returns (out [B,T,H,d_v], final_state [N,H,d_k,d_v]) in float64."""
+    q, k, v, dt, B, T, H, dk, dv, g, cu, n = _prep(q, k, v, gamma, cu_seqlens)
+    out = np.zeros((B, T, H, dv), np.float64)
+    fs = np.zeros((n, H, dk, dv), np.float64)
+    rc = _load().oracle_recurrent(
+        _ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(g), _ptr(cu), n,
+        _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), int(nthreads),
+    )
+    if rc != 0:
+        raise ValueError("oracle_recurrent rejected its arguments (code %d)" % rc)
+    return out, fs
+
+
+def chunked(q, k, v, gamma, chunk, cu_seqlens=None, phi="identity", normalize=False, nthreads=0):
+    """Chunked restatement (float64); same outputs as :func:`recurrent` up to rounding."""
+    q, k, v, dt, B, T, H, dk, dv, g, cu, n = _prep(q, k, v, gamma, cu_seqlens)
+    out = np.zeros((B, T, H, dv), np.float64)
+    fs = np.zeros((n, H, dk, dv), np.float64)
+    rc = _load().oracle_chunked(
+        _ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(g), _ptr(cu), n, int(chunk),
+        _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), int(nthreads),
+    )
+    if rc != 0:
+        raise ValueError("oracle_chunked rejected its arguments (code %d)" % rc)
+    return out, fs
+
+
+def step(q, k, v, gamma, state, phi="identity", nthreads=0):
+    """One decode token.  q,k [N,H,d_k], v [N,H,d_v], state [N,H,d_k,d_v] (S^T).
+
+    Returns (out [N,H,d_v], new_state) in float64; the input state is not modified.
+    """
+    q, dq = _as_input(q)
+    k, _ = _as_input(k)
+    v, _ = _as_input(v)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    if st.shape != (N, H, dk, dv):
+        raise ValueError("state must be [N, H, d_k, d_v]")
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(-1))
+    if g.size == 1 and H > 1:
+        g = np.full(H, g[0])
+    out = np.zeros((N, H, dv), np.float64)
+    rc = _load().oracle_step(
+        _ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(g), _ptr(st), _ptr(out), _PHI[phi], int(nthreads)
+    )
+    if rc != 0:
+        raise ValueError("oracle_step rejected its arguments (code %d)" % rc)
+    return out, st

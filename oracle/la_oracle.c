@@ -1,0 +1,316 @@
+/*
+ * la_oracle.c -- float64 CPU oracle for causal linear attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path loads this library:
+ * only the test suite, the smoke check in __graft_entry__.py and the
+ * cpu_baseline / reference legs of bench.py may load or call it.  It shares no
+ * code, header, table or helper with the CUDA library.
+ *
+ * What it computes (the plain definition, no blocking or reordering):
+ *   "1.6 长上下文与高效注意力" (long context and efficient attention), section
+ *   线性注意力 (linear attention), the displayed equation
+ *       o_t = S_t phi(q_t) / (z_t^T phi(q_t)),
+ *       S_t = S_{t-1} + v_t phi(k_t)^T,   z_t = z_{t-1} + phi(k_t),
+ *   with S a d_v x d_k matrix started at zero, phi(x) = elu(x) + 1 or the
+ *   identity, and a per-head constant decay gamma multiplying the old state:
+ *       S_t = gamma S_{t-1} + v_t phi(k_t)^T,  z_t = gamma z_{t-1} + phi(k_t).
+ *   gamma = 1 is the page's equation exactly.  The state includes token t
+ *   before o_t is read (the sum in the displayed equation runs over j <= t).
+ *
+ * Functions:
+ *   oracle_recurrent  -- the token-by-token recurrence above (prefill).
+ *   oracle_chunked    -- the same result regrouped into chunks of C tokens;
+ *                        the chunk form is derived in the header comment of
+ *                        that function.  It exists to pin the derivation that
+ *                        a chunked implementation relies on (results must not
+ *                        depend on C beyond rounding).
+ *   oracle_step       -- one decode token on a given state, in place.
+ *
+ * Layouts (all row-major, last dimension contiguous):
+ *   q, k  [B, T, H, d_k];  v  [B, T, H, d_v];  out  [B, T, H, d_v] (double)
+ *   with cu_seqlens != NULL: B must be 1 and sequence n occupies tokens
+ *   cu_seqlens[n] .. cu_seqlens[n+1]-1 of the packed T axis.
+ *   final_state [n_seqs, H, d_k, d_v] (double) holds S^T (entry [c][r] is
+ *   S[r][c]); NULL skips it.
+ *   Inputs may be float32, bfloat16 (raw uint16 bits) or float64; they are
+ *   upcast to double exactly on every read.
+ *
+ * Return value: 0 on success, a negative number for a bad argument.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_F32 0
+#define ORC_BF16 1
+#define ORC_F64 2
+
+#define ORC_PHI_IDENTITY 0
+#define ORC_PHI_ELU1 1
+
+#define ROWS_PER_TASK 8
+
+static double orc_load(const void *p, int dtype, int64_t i) {
+  if (dtype == ORC_F32) return (double)((const float *)p)[i];
+  if (dtype == ORC_BF16) {
+    uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+  }
+  return ((const double *)p)[i];
+}
+
+/* elu with alpha = 1, plus one: x + 1 for x > 0, exp(x) otherwise. */
+static double orc_phi(double x, int phi) {
+  if (phi == ORC_PHI_ELU1) return x > 0.0 ? x + 1.0 : exp(x);
+  return x;
+}
+
+static int orc_check(int dtype, int64_t B, int64_t T, int64_t H, int64_t dk,
+                     int64_t dv, const int32_t *cu, int64_t n_seqs, int phi) {
+  if (dtype < ORC_F32 || dtype > ORC_F64) return -1;
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return -2;
+  if (phi != ORC_PHI_IDENTITY && phi != ORC_PHI_ELU1) return -3;
+  if (cu) {
+    if (B != 1 || n_seqs < 0) return -4;
+    if (cu[0] != 0) return -5;
+    for (int64_t n = 0; n < n_seqs; ++n)
+      if (cu[n + 1] < cu[n]) return -6;
+    if ((int64_t)cu[n_seqs] > T) return -7;
+  } else if (n_seqs != B) {
+    return -8;
+  }
+  return 0;
+}
+
+static void orc_seq(const int32_t *cu, int64_t T, int64_t n, int64_t *start,
+                    int64_t *len) {
+  if (cu) {
+    *start = cu[n];
+    *len = (int64_t)cu[n + 1] - cu[n];
+  } else {
+    *start = n * T;
+    *len = T;
+  }
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/*
+ * The recurrence, token by token.  Row r of S depends only on column r of v
+ * and on phi(k), so the work splits into independent tasks over
+ * (sequence, head, block of rows of S); z is recomputed inside each task.
+ */
+int oracle_recurrent(const void *q, const void *k, const void *v, int dtype,
+                     int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                     const double *gamma, const int32_t *cu_seqlens,
+                     int64_t n_seqs, int phi, int normalize, double *out,
+                     double *final_state, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  const int64_t nblk = (dv + ROWS_PER_TASK - 1) / ROWS_PER_TASK;
+  const int64_t ntask = n_seqs * H * nblk;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < ntask; ++task) {
+    const int64_t n = task / (H * nblk);
+    const int64_t h = (task / nblk) % H;
+    const int64_t r0 = (task % nblk) * ROWS_PER_TASK;
+    const int64_t nr = dv - r0 < ROWS_PER_TASK ? dv - r0 : ROWS_PER_TASK;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const double g = gamma[h];
+
+    double *S = (double *)calloc((size_t)(ROWS_PER_TASK * dk), sizeof(double));
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t tok = start + t;
+      const int64_t qk_base = (tok * H + h) * dk;
+      const int64_t v_base = (tok * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk_base + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk_base + c), phi);
+      }
+      double den = 1.0;
+      if (normalize) {
+        den = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          z[c] = g * z[c] + kh[c];
+          den += z[c] * qh[c];
+        }
+      }
+      for (int64_t i = 0; i < nr; ++i) {
+        const double vr = orc_load(v, dtype, v_base + r0 + i);
+        double *Sr = S + i * dk;
+        double num = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          Sr[c] = g * Sr[c] + vr * kh[c];
+          num += Sr[c] * qh[c];
+        }
+        out[v_base + r0 + i] = num / den;
+      }
+    }
+    if (final_state) {
+      double *F = final_state + (n * H + h) * dk * dv;
+      for (int64_t i = 0; i < nr; ++i)
+        for (int64_t c = 0; c < dk; ++c) F[c * dv + r0 + i] = S[i * dk + c];
+    }
+    free(S);
+    free(z);
+    free(qh);
+    free(kh);
+  }
+  return 0;
+}
+
+/*
+ * The chunked form.  Unrolling the recurrence from a chunk whose first token
+ * sees the state S_p (and z_p), for positions i, j = 0 .. C'-1 inside a chunk
+ * of C' tokens:
+ *   S after token i   = gamma^(i+1) S_p + sum_{j<=i} gamma^(i-j) v_j kh_j^T
+ *   o_i (numerator)   = gamma^(i+1) S_p qh_i + sum_{j<=i} gamma^(i-j) (qh_i.kh_j) v_j
+ *   den_i             = gamma^(i+1) z_p.qh_i + sum_{j<=i} gamma^(i-j) (qh_i.kh_j)
+ *   S_next            = gamma^C' S_p + sum_j gamma^(C'-1-j) v_j kh_j^T
+ *   z_next            = gamma^C' z_p + sum_j gamma^(C'-1-j) kh_j
+ * Chunks restart at each sequence start; the last chunk of a sequence holds
+ * the remaining len mod C tokens when that is not zero.
+ */
+int oracle_chunked(const void *q, const void *k, const void *v, int dtype,
+                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                   const double *gamma, const int32_t *cu_seqlens,
+                   int64_t n_seqs, int64_t chunk, int phi, int normalize,
+                   double *out, double *final_state, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (chunk <= 0) return -9;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const double g = gamma[h];
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double)); /* S[r][c] */
+    double *Sn = (double *)malloc((size_t)(dv * dk) * sizeof(double));
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *zn = (double *)malloc((size_t)dk * sizeof(double));
+    double *qh = (double *)malloc((size_t)(chunk * dk) * sizeof(double));
+    double *kh = (double *)malloc((size_t)(chunk * dk) * sizeof(double));
+    double *vv = (double *)malloc((size_t)(chunk * dv) * sizeof(double));
+
+    for (int64_t c0 = 0; c0 < len; c0 += chunk) {
+      const int64_t Cp = len - c0 < chunk ? len - c0 : chunk;
+      for (int64_t i = 0; i < Cp; ++i) {
+        const int64_t tok = start + c0 + i;
+        for (int64_t c = 0; c < dk; ++c) {
+          qh[i * dk + c] = orc_phi(orc_load(q, dtype, (tok * H + h) * dk + c), phi);
+          kh[i * dk + c] = orc_phi(orc_load(k, dtype, (tok * H + h) * dk + c), phi);
+        }
+        for (int64_t r = 0; r < dv; ++r)
+          vv[i * dv + r] = orc_load(v, dtype, (tok * H + h) * dv + r);
+      }
+      /* outputs of the chunk */
+      for (int64_t i = 0; i < Cp; ++i) {
+        const double gi1 = pow(g, (double)(i + 1));
+        double den = 0.0;
+        for (int64_t c = 0; c < dk; ++c) den += z[c] * qh[i * dk + c];
+        den *= gi1;
+        double *o = out + ((start + c0 + i) * H + h) * dv;
+        for (int64_t r = 0; r < dv; ++r) {
+          double acc = 0.0;
+          for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * qh[i * dk + c];
+          o[r] = gi1 * acc;
+        }
+        for (int64_t j = 0; j <= i; ++j) {
+          double a = 0.0;
+          for (int64_t c = 0; c < dk; ++c) a += qh[i * dk + c] * kh[j * dk + c];
+          const double p = pow(g, (double)(i - j)) * a;
+          den += p;
+          for (int64_t r = 0; r < dv; ++r) o[r] += p * vv[j * dv + r];
+        }
+        if (normalize)
+          for (int64_t r = 0; r < dv; ++r) o[r] /= den;
+      }
+      /* state carried to the next chunk */
+      const double gC = pow(g, (double)Cp);
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) Sn[r * dk + c] = gC * S[r * dk + c];
+      for (int64_t c = 0; c < dk; ++c) zn[c] = gC * z[c];
+      for (int64_t j = 0; j < Cp; ++j) {
+        const double w = pow(g, (double)(Cp - 1 - j));
+        for (int64_t c = 0; c < dk; ++c) zn[c] += w * kh[j * dk + c];
+        for (int64_t r = 0; r < dv; ++r) {
+          const double wv = w * vv[j * dv + r];
+          for (int64_t c = 0; c < dk; ++c) Sn[r * dk + c] += wv * kh[j * dk + c];
+        }
+      }
+      memcpy(S, Sn, (size_t)(dv * dk) * sizeof(double));
+      memcpy(z, zn, (size_t)dk * sizeof(double));
+    }
+    if (final_state) {
+      double *F = final_state + (n * H + h) * dk * dv;
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) F[c * dv + r] = S[r * dk + c];
+    }
+    free(S);
+    free(Sn);
+    free(z);
+    free(zn);
+    free(qh);
+    free(kh);
+    free(vv);
+  }
+  return 0;
+}
+
+/*
+ * One decode token: the recurrence applied once to a given state.
+ *   q, k [N, H, d_k];  v [N, H, d_v] (any input dtype above)
+ *   state [N, H, d_k, d_v] double, holding S^T, updated in place:
+ *       S^T[c][r] <- gamma S^T[c][r] + kh_c v_r
+ *   out [N, H, d_v] double:  o_r = sum_c S^T[c][r] qh_c   (after the update)
+ */
+int oracle_step(const void *q, const void *k, const void *v, int dtype,
+                int64_t N, int64_t H, int64_t dk, int64_t dv,
+                const double *gamma, double *state, double *out, int phi,
+                int nthreads) {
+  int rc = orc_check(dtype, 1, 1, H, dk, dv, NULL, 1, phi);
+  if (rc) return rc;
+  if (N < 0) return -2;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+  for (int64_t task = 0; task < N * H; ++task) {
+    const int64_t h = task % H;
+    const double g = gamma[h];
+    double *St = state + task * dk * dv;
+    double *o = out + task * dv;
+    for (int64_t r = 0; r < dv; ++r) o[r] = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+      const double qc = orc_phi(orc_load(q, dtype, task * dk + c), phi);
+      const double kc = orc_phi(orc_load(k, dtype, task * dk + c), phi);
+      for (int64_t r = 0; r < dv; ++r) {
+        const double s = g * St[c * dv + r] + kc * orc_load(v, dtype, task * dv + r);
+        St[c * dv + r] = s;
+        o[r] += s * qc;
+      }
+    }
+  }
+  return 0;
+}

@@ -1,0 +1,266 @@
+"""Pins for the float64 oracle (CPU only).
+
+Each test pins the oracle to something other than itself:
+  * the quadratic (parallel) masked form written out here by brute force --
+    a different formula for the same result ("1.6 长上下文与高效注意力",
+    section 线性注意力: training may run in parallel form; the page's listing
+    asserts parallel form == recurrent form);
+  * hand-derived values (tests/golden/*.json, derivations inside);
+  * closed forms for constant inputs, and special cases (T = 1, gamma = 0,
+    d = 1, varlen == independent runs, prefill + one decode step == prefill
+    of one more token);
+  * invariance of the chunked restatement to the chunk size.
+A plausible slip anywhere -- a dropped decay, the diagonal excluded, S used
+transposed, the normaliser taken before the update, a wrong power of gamma in
+the chunk carry -- fails at least one of these.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+TOL = 1e-12
+
+
+def phi_np(x, kind):
+    if kind == "elu1":
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    return x
+
+
+def quadratic_form(q, k, v, gamma, phi, normalize):
+    """O = ((phi(Q) phi(K)^T) * M_gamma) V [/ row sums], M[i,j] = gamma^(i-j) for i >= j.
+
+    One sequence, one head: q, k [T, d_k], v [T, d_v] (float64).
+    """
+    T = q.shape[0]
+    A = phi_np(q, phi) @ phi_np(k, phi).T
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        M = np.where(i >= j, np.power(float(gamma), np.maximum(i - j, 0).astype(np.float64)), 0.0)
+    P = A * M
+    O = P @ v
+    if normalize:
+        O = O / P.sum(axis=1, keepdims=True)
+    return O
+
+
+def rel(x, ref):
+    den = np.max(np.abs(ref))
+    return float(np.max(np.abs(x - ref)) / (den if den > 0 else 1.0))
+
+
+def rand_qkv(B, T, H, dk, dv, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, dk)) * scale
+    k = rng.standard_normal((B, T, H, dk)) * scale
+    v = rng.standard_normal((B, T, H, dv))
+    return q, k, v
+
+
+# ---------------------------------------------------------------- brute force
+@pytest.mark.parametrize("T", [1, 2, 3, 17, 64])
+@pytest.mark.parametrize("d", [1, 4, 16])
+@pytest.mark.parametrize("gamma", [0.0, 0.5, 0.9, 1.0])
+@pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", False), ("elu1", True)])
+def test_recurrent_equals_quadratic(oracle_mod, T, d, gamma, phi, normalize):
+    B, H = 2, 2
+    q, k, v = rand_qkv(B, T, H, d, d + 1, seed=T * 131 + d)
+    out, _ = oracle_mod.recurrent(q, k, v, [gamma] * H, phi=phi, normalize=normalize)
+    for b in range(B):
+        for h in range(H):
+            ref = quadratic_form(q[b, :, h], k[b, :, h], v[b, :, h], gamma, phi, normalize)
+            assert rel(out[b, :, h], ref) < TOL
+
+
+def test_final_state_equals_weighted_outer_sum(oracle_mod):
+    """S_T = sum_j gamma^(T-1-j) v_j phi(k_j)^T, stored transposed ([d_k][d_v])."""
+    T, dk, dv, g = 37, 5, 3, 0.8
+    q, k, v = rand_qkv(1, T, 1, dk, dv, seed=3)
+    _, fs = oracle_mod.recurrent(q, k, v, [g], phi="elu1")
+    kh = phi_np(k[0, :, 0], "elu1")
+    S = sum(g ** (T - 1 - j) * np.outer(v[0, j, 0], kh[j]) for j in range(T))
+    assert rel(fs[0, 0], S.T) < TOL
+
+
+def test_page_listing_check(oracle_mod):
+    """The page's listing compares parallel and recurrent forms at T=50, d=16,
+    phi = elu+1, normalised, gamma = 1, and reports agreement within atol 1e-5.
+    Here the parallel form is computed independently (float64) and compared
+    with the oracle on inputs drawn the same way (torch.manual_seed(0), three
+    standard-normal [T, d] tensors)."""
+    torch.manual_seed(0)
+    qt, kt, vt = (torch.randn(50, 16) for _ in range(3))
+    q, k, v = (x.double().numpy() for x in (qt, kt, vt))
+    par = quadratic_form(q, k, v, 1.0, "elu1", True)
+    out, _ = oracle_mod.recurrent(q[None, :, None], k[None, :, None], v[None, :, None], [1.0],
+                                  phi="elu1", normalize=True)
+    assert np.max(np.abs(out[0, :, 0] - par)) < 1e-5
+    assert rel(out[0, :, 0], par) < TOL
+
+
+# ---------------------------------------------------------------- hand values
+def test_golden_hand_d2(oracle_mod):
+    with open(os.path.join(GOLD, "hand_d2_T2.json")) as f:
+        G = json.load(f)
+    q = np.array(G["q"], float)[None, :, None]
+    k = np.array(G["k"], float)[None, :, None]
+    v = np.array(G["v"], float)[None, :, None]
+    out, fs = oracle_mod.recurrent(q, k, v, [G["gamma"]])
+    np.testing.assert_allclose(out[0, :, 0], G["out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(fs[0, 0], G["final_state"], rtol=0, atol=1e-15)
+    outn, _ = oracle_mod.recurrent(q, k, v, [G["gamma"]], normalize=True)
+    np.testing.assert_allclose(outn[0, :, 0], G["out_normalized"], rtol=0, atol=1e-15)
+    s = G["step"]
+    o, st = oracle_mod.step(np.array(s["q"], float)[None, None], np.array(s["k"], float)[None, None],
+                            np.array(s["v"], float)[None, None], [G["gamma"]], fs)
+    np.testing.assert_allclose(st[0, 0], s["state_out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(o[0, 0], s["out"], rtol=0, atol=1e-15)
+
+
+def test_golden_hand_d1_elu(oracle_mod):
+    with open(os.path.join(GOLD, "hand_d1_elu.json")) as f:
+        G = json.load(f)
+    ev = lambda e: eval(e, {"exp": math.exp})  # noqa: E731  (expressions from the fixture)
+    q = np.array(G["q"], float)[None, :, None, None]
+    k = np.array(G["k"], float)[None, :, None, None]
+    v = np.array(G["v"], float)[None, :, None, None]
+    out, fs = oracle_mod.recurrent(q, k, v, [G["gamma"]], phi="elu1")
+    np.testing.assert_allclose(out.reshape(-1), [ev(e) for e in G["expr_out"]], rtol=1e-15)
+    np.testing.assert_allclose(fs.reshape(-1), [ev(G["expr_final_state"])], rtol=1e-15)
+    outn, _ = oracle_mod.recurrent(q, k, v, [G["gamma"]], phi="elu1", normalize=True)
+    np.testing.assert_allclose(outn.reshape(-1), [ev(e) for e in G["expr_out_normalized"]], rtol=1e-15)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+@pytest.mark.parametrize("gamma", [1.0, 0.9, 0.3])
+def test_constant_inputs_closed_form(oracle_mod, phi, gamma):
+    T, dk, dv = 40, 6, 4
+    rng = np.random.default_rng(11)
+    qv, kv, vv = rng.standard_normal(dk), np.abs(rng.standard_normal(dk)), rng.standard_normal(dv)
+    q = np.broadcast_to(qv, (1, T, 1, dk)).copy()
+    k = np.broadcast_to(kv, (1, T, 1, dk)).copy()
+    v = np.broadcast_to(vv, (1, T, 1, dv)).copy()
+    out, fs = oracle_mod.recurrent(q, k, v, [gamma], phi=phi)
+    qh, kh = phi_np(qv, phi), phi_np(kv, phi)
+    t = np.arange(1, T + 1, dtype=np.float64)
+    w = t if gamma == 1.0 else (1 - gamma ** t) / (1 - gamma)  # sum_{j<t} gamma^j
+    ref = w[:, None] * (qh @ kh) * vv[None, :]
+    assert rel(out[0, :, 0], ref) < TOL
+    assert rel(fs[0, 0], w[-1] * np.outer(kh, vv)) < TOL
+    if phi == "elu1":  # normalised: every output equals v exactly
+        outn, _ = oracle_mod.recurrent(q, k, v, [gamma], phi=phi, normalize=True)
+        assert np.max(np.abs(outn[0, :, 0] - vv[None, :])) < 1e-13
+
+
+# ---------------------------------------------------------------- special cases
+def test_single_token_and_gamma_zero(oracle_mod):
+    q, k, v = rand_qkv(1, 30, 2, 8, 5, seed=5)
+    for phi in ("identity", "elu1"):
+        qh, kh = phi_np(q, phi), phi_np(k, phi)
+        o1, _ = oracle_mod.recurrent(q[:, :1], k[:, :1], v[:, :1], [0.7, 1.0], phi=phi)
+        ref1 = np.einsum("bthc,bthc->bth", qh[:, :1], kh[:, :1])[..., None] * v[:, :1]
+        assert rel(o1, ref1) < TOL
+        o0, fs0 = oracle_mod.recurrent(q, k, v, [0.0, 0.0], phi=phi)
+        ref0 = np.einsum("bthc,bthc->bth", qh, kh)[..., None] * v
+        assert rel(o0, ref0) < TOL
+        assert rel(fs0[0], np.einsum("hc,hr->hcr", kh[0, -1], v[0, -1])) < TOL
+
+
+def test_d1_scalar_ewma(oracle_mod):
+    T, g = 25, 0.75
+    q, k, v = rand_qkv(1, T, 1, 1, 1, seed=9)
+    out, _ = oracle_mod.recurrent(q, k, v, [g])
+    s, ref = 0.0, []
+    for t in range(T):
+        s = g * s + v[0, t, 0, 0] * k[0, t, 0, 0]
+        ref.append(s * q[0, t, 0, 0])
+    assert rel(out.reshape(-1), np.array(ref)) < TOL
+
+
+def test_varlen_equals_independent_runs(oracle_mod):
+    lengths = [5, 0, 17, 1, 64, 33]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 3, 8, 6
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=21)
+    gam = [1.0, 0.95, 0.5]
+    for phi, norm in (("identity", False), ("elu1", True)):
+        out, fs = oracle_mod.recurrent(q, k, v, gam, cu_seqlens=cu, phi=phi, normalize=norm)
+        for n, L in enumerate(lengths):
+            s, e = cu[n], cu[n + 1]
+            o1, f1 = oracle_mod.recurrent(q[:, s:e], k[:, s:e], v[:, s:e], gam, phi=phi, normalize=norm)
+            assert np.array_equal(out[:, s:e], o1)
+            assert np.array_equal(fs[n], f1[0])
+            if L == 0:
+                assert not fs[n].any()
+
+
+def test_prefill_then_step_equals_longer_prefill(oracle_mod):
+    T, H, dk, dv = 20, 2, 8, 8
+    q, k, v = rand_qkv(3, T + 1, H, dk, dv, seed=31)
+    gam = [0.9, 0.99]
+    for phi in ("identity", "elu1"):
+        _, fsT = oracle_mod.recurrent(q[:, :T], k[:, :T], v[:, :T], gam, phi=phi)
+        oT1, fsT1 = oracle_mod.recurrent(q, k, v, gam, phi=phi)
+        o, st = oracle_mod.step(q[:, T], k[:, T], v[:, T], gam, fsT, phi=phi)
+        assert rel(o, oT1[:, T]) < TOL
+        assert rel(st, fsT1) < TOL
+
+
+# ---------------------------------------------------------------- chunked form
+@pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
+@pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
+def test_chunk_invariance(oracle_mod, chunk, phi, normalize):
+    T, H, dk, dv = 130, 3, 6, 5
+    q, k, v = rand_qkv(2, T, H, dk, dv, seed=chunk)
+    gam = [1.0, 0.93, 0.0]
+    ref, fref = oracle_mod.recurrent(q, k, v, gam, phi=phi, normalize=normalize)
+    out, fs = oracle_mod.chunked(q, k, v, gam, chunk, phi=phi, normalize=normalize)
+    assert rel(out, ref) < TOL
+    assert rel(fs, fref) < TOL
+
+
+def test_chunk_invariance_varlen(oracle_mod):
+    lengths = [64, 65, 1, 0, 130, 63]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    q, k, v = rand_qkv(1, int(cu[-1]), 2, 8, 8, seed=77)
+    gam = [0.97, 1.0]
+    ref, fref = oracle_mod.recurrent(q, k, v, gam, cu_seqlens=cu, phi="elu1", normalize=True)
+    for chunk in (16, 64):
+        out, fs = oracle_mod.chunked(q, k, v, gam, chunk, cu_seqlens=cu, phi="elu1", normalize=True)
+        assert rel(out, ref) < TOL and rel(fs, fref) < TOL
+
+
+# ---------------------------------------------------------------- input types
+def test_bf16_and_f32_inputs_upcast_exactly(oracle_mod):
+    qf, kf, vf = (torch.randn(1, 33, 2, 8, dtype=torch.float32) for _ in range(3))
+    qb, kb, vb = (x.to(torch.bfloat16) for x in (qf, kf, vf))
+    o_b, f_b = oracle_mod.recurrent(qb, kb, vb, [0.9, 1.0])
+    o_d, f_d = oracle_mod.recurrent(*(x.double().numpy() for x in (qb, kb, vb)), [0.9, 1.0])
+    assert np.array_equal(o_b, o_d) and np.array_equal(f_b, f_d)
+    o_f, _ = oracle_mod.recurrent(qf.numpy(), kf.numpy(), vf.numpy(), [0.9, 1.0])
+    o_f64, _ = oracle_mod.recurrent(*(x.double().numpy() for x in (qf, kf, vf)), [0.9, 1.0])
+    assert np.array_equal(o_f, o_f64)
+
+
+def test_rejects_bad_arguments(oracle_mod):
+    q, k, v = rand_qkv(2, 4, 1, 2, 2, seed=1)
+    with pytest.raises(ValueError):
+        oracle_mod.recurrent(q, k, v, [1.0], cu_seqlens=[0, 2, 4])  # B must be 1 with cu_seqlens
+    with pytest.raises(ValueError):
+        oracle_mod.recurrent(q[:1], k[:1], v[:1], [1.0], cu_seqlens=[0, 3, 2])  # decreasing
+    with pytest.raises(ValueError):
+        oracle_mod.chunked(q, k, v, [1.0], 0)
+
+
+def test_oracle_is_independent_of_the_product():
+    """The oracle package imports nothing from the CUDA library's package."""
+    src = open(os.path.join(os.path.dirname(__file__), "..", "oracle", "__init__.py")).read()
+    src += open(os.path.join(os.path.dirname(__file__), "..", "oracle", "la_oracle.c")).read()
+    assert "chunkwise_causal_linear_la_b200" not in src

@@ -1,0 +1,89 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case copies oracle/la_oracle.c to a temporary directory, plants one
+mistake in the copy (the committed oracle is untouched), compiles it with gcc
+and checks that the pins of test_oracle.py reject the mutant: the brute-force
+quadratic form and the hand-derived fixture.
+"""
+import ctypes
+import json
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from test_oracle import GOLD, quadratic_form, rand_qkv, rel
+
+SRC = os.path.join(os.path.dirname(__file__), "..", "oracle", "la_oracle.c")
+
+MUTATIONS = {
+    "decay dropped from the state": (
+        "Sr[c] = g * Sr[c] + vr * kh[c];", "Sr[c] = Sr[c] + vr * kh[c];"),
+    "decay dropped from the normaliser": (
+        "z[c] = g * z[c] + kh[c];", "z[c] = z[c] + kh[c];"),
+    "output read before the update (diagonal excluded)": (
+        "Sr[c] = g * Sr[c] + vr * kh[c];\n          num += Sr[c] * qh[c];",
+        "num += Sr[c] * qh[c];\n          Sr[c] = g * Sr[c] + vr * kh[c];"),
+    "elu+1 missing the +1": (
+        "return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x);"),
+    "final state stored untransposed": (
+        "F[c * dv + r0 + i] = S[i * dk + c];", "F[(r0 + i) * dk + c] = S[i * dk + c];"),
+    "decay applied twice": (
+        "Sr[c] = g * Sr[c] + vr * kh[c];", "Sr[c] = g * g * Sr[c] + vr * kh[c];"),
+}
+
+
+def _build(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    mpath = tmp_path / "mut.c"
+    mpath.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(mpath), "-o", str(so), "-lm"])
+    lib = ctypes.CDLL(str(so))
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.oracle_recurrent.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, vp, vp, i64, i32, i32, vp, vp, i32]
+    lib.oracle_recurrent.restype = i32
+    return lib
+
+
+def _run(lib, q, k, v, gamma, phi, normalize):
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    g = np.ascontiguousarray(gamma, dtype=np.float64)
+    out = np.zeros((B, T, H, dv))
+    fs = np.zeros((B, H, dk, dv))
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = lib.oracle_recurrent(p(q), p(k), p(v), 2, B, T, H, dk, dv, p(g), None, B,
+                              1 if phi == "elu1" else 0, int(normalize), p(out), p(fs), 1)
+    assert rc == 0
+    return out, fs
+
+
+def _pins_pass(lib):
+    """True when the mutant passes every pin used here."""
+    ok = True
+    q, k, v = rand_qkv(1, 24, 1, 4, 4, seed=4)
+    for gamma, phi, norm in ((0.9, "identity", False), (1.0, "elu1", True), (0.8, "elu1", True)):
+        out, _ = _run(lib, q, k, v, [gamma], phi, norm)
+        ok &= rel(out[0, :, 0], quadratic_form(q[0, :, 0], k[0, :, 0], v[0, :, 0], gamma, phi, norm)) < 1e-12
+    with open(os.path.join(GOLD, "hand_d2_T2.json")) as f:
+        G = json.load(f)
+    qg, kg, vg = (np.array(G[x], float)[None, :, None] for x in "qkv")
+    out, fs = _run(lib, qg, kg, vg, [G["gamma"]], "identity", False)
+    ok &= np.allclose(out[0, :, 0], G["out"], atol=1e-15) and np.allclose(fs[0, 0], G["final_state"], atol=1e-15)
+    return bool(ok)
+
+
+def test_unmutated_copy_passes(tmp_path):
+    lib = _build(tmp_path, "none", "#define ROWS_PER_TASK 8", "#define ROWS_PER_TASK 8")
+    assert _pins_pass(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTATIONS[name]
+    lib = _build(tmp_path, name, old, new)
+    assert not _pins_pass(lib), name
