@@ -1,1 +1,20 @@
-"""Chunkwise causal linear attention on NVIDIA B200 (sm_100a)."""
+"""Chunkwise causal linear attention on NVIDIA B200 (sm_100a).
+
+The compute lives in the C-ABI library libla_b200.so (include/la_b200.h);
+this package is its Python binding:
+
+    from chunkwise_causal_linear_la_b200 import la_fwd_chunk, la_step
+    out, final_state = la_fwd_chunk(q, k, v, gamma, chunk=64, phi="identity")
+    o = la_step(q1, k1, v1, gamma, final_state)   # decode one more token
+
+``workloads`` draws the seeded synthetic inputs of the standard workloads.
+"""
+from .binding import (  # noqa: F401
+    LA_FLAG_NONE,
+    LA_FLAG_SIMT,
+    LaError,
+    la_fwd_chunk,
+    la_step,
+    load_library,
+    workspace_size,
+)

@@ -1,0 +1,164 @@
+"""Thin ctypes binding of libla_b200.so (include/la_b200.h).
+
+Argument marshalling only: torch tensors are described to the C ABI by data
+pointer, shape, strides and dtype, outputs and workspace are allocated with
+torch (device memory plumbing), and the call is enqueued on the current torch
+stream.  Every step of the computation runs in the library's CUDA kernels; if
+the library is missing this module raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libla_b200.so")
+
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE, LA_ERR_CUDA = range(5)
+LA_PHI_IDENTITY, LA_PHI_ELU1 = 0, 1
+LA_F32, LA_BF16 = 0, 1
+LA_FLAG_NONE, LA_FLAG_SIMT = 0, 1
+
+_PHI = {"identity": LA_PHI_IDENTITY, "elu1": LA_PHI_ELU1, LA_PHI_IDENTITY: LA_PHI_IDENTITY,
+        LA_PHI_ELU1: LA_PHI_ELU1}
+_DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
+
+# Every function include/la_b200.h declares.
+EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_workspace_size", "la_step", "la_status_string",
+           "la_last_error", "la_version")
+
+
+class LaTensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64), ("D", ctypes.c_int64),
+        ("stride_b", ctypes.c_int64), ("stride_t", ctypes.c_int64), ("stride_h", ctypes.c_int64),
+    ]
+
+
+class LaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libla_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            "libla_b200.so is not built (%s); run `python -c 'import __graft_entry__ as g; g.build()'`" % path)
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(LaTensor)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.la_fwd_chunk.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, i32, vp, sz, vp]
+    lib.la_fwd_chunk.restype = i32
+    lib.la_fwd_chunk_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32, i32]
+    lib.la_fwd_chunk_workspace_size.restype = sz
+    lib.la_step.argtypes = [P, P, P, vp, vp, P, i32, vp]
+    lib.la_step.restype = i32
+    lib.la_status_string.argtypes = [i32]
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_last_error.argtypes = []
+    lib.la_last_error.restype = ctypes.c_char_p
+    lib.la_version.argtypes = []
+    lib.la_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def describe(t: torch.Tensor) -> LaTensor:
+    """la_tensor for a [B, T, H, D] torch tensor whose last dim is contiguous."""
+    if t.dim() != 4:
+        raise ValueError("expected a [B, T, H, D] tensor, got shape %s" % (tuple(t.shape),))
+    if t.dtype not in _DT:
+        raise TypeError("dtype %s not supported (float32 or bfloat16)" % t.dtype)
+    if t.shape[3] > 1 and t.stride(3) != 1:
+        raise ValueError("the head dim must be contiguous")
+    B, T, H, D = t.shape
+    return LaTensor(t.data_ptr(), _DT[t.dtype], B, T, H, D, t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(lib, status: int, what: str):
+    if status != LA_OK:
+        detail = lib.la_last_error().decode(errors="replace")
+        raise LaError(status, "%s failed: %s (%s)" % (what, lib.la_status_string(status).decode(), detail))
+
+
+def workspace_size(B, T, H, d_k, d_v, n_seqs, varlen, chunk, dtype=torch.bfloat16, flags=0) -> int:
+    lib = load_library()
+    n = lib.la_fwd_chunk_workspace_size(B, T, H, d_k, d_v, n_seqs, int(bool(varlen)), chunk, _DT[dtype], flags)
+    if n == ctypes.c_size_t(-1).value:
+        raise LaError(LA_ERR_INVALID_ARG, "la_fwd_chunk_workspace_size rejected the arguments")
+    return int(n)
+
+
+def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", normalize=False,
+                 out=None, final_state=None, return_final_state=True, flags=LA_FLAG_NONE,
+                 workspace=None, stream=None):
+    """Chunkwise causal linear attention forward (see la_fwd_chunk in include/la_b200.h).
+
+    q, k [B,T,H,d_k], v [B,T,H,d_v] (CUDA, float32 or bfloat16); gamma float32 [H];
+    cu_seqlens int32 [N+1] or None.  Returns (out, final_state or None).
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if gamma.dtype != torch.float32 or gamma.numel() != H:
+        raise TypeError("gamma must be float32 with H entries")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = workspace_size(B, T, H, dk, dv, n_seqs, cu_seqlens is not None, chunk, q.dtype, flags)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    tq, tk, tv, to = describe(q), describe(k), describe(v), describe(out)
+    st = lib.la_fwd_chunk(
+        ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
+        None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
+        int(bool(normalize)), ctypes.byref(to), None if final_state is None else final_state.data_ptr(),
+        int(flags), None if workspace is None else workspace.data_ptr(),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(lib, st, "la_fwd_chunk")
+    return out, final_state
+
+
+def la_step(q, k, v, gamma, state, out=None, phi="identity", stream=None):
+    """One decode token (see la_step in include/la_b200.h).
+
+    q, k [N,H,d_k] or [N,1,H,d_k]; v [N,H,d_v] likewise; state float32 [N,H,d_k,d_v]
+    updated in place.  Returns out shaped like v.
+    """
+    lib = load_library()
+    squeeze = q.dim() == 3
+    q4, k4, v4 = (x.unsqueeze(1) if squeeze else x for x in (q, k, v))
+    if out is None:
+        out = torch.empty_like(v4)
+    o4 = out.unsqueeze(1) if out.dim() == 3 else out
+    if state.dtype != torch.float32 or not state.is_contiguous():
+        raise TypeError("state must be a contiguous float32 tensor")
+    tq, tk, tv, to = describe(q4), describe(k4), describe(v4), describe(o4)
+    st = lib.la_step(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(), state.data_ptr(),
+                     ctypes.byref(to), _PHI[phi], _stream(stream))
+    _check(lib, st, "la_step")
+    return o4.squeeze(1) if squeeze else o4

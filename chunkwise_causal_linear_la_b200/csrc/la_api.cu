@@ -1,0 +1,249 @@
+// la_api.cu -- the C ABI of include/la_b200.h: argument validation, kernel
+// selection and launch.  No allocation, no synchronisation, no exceptions.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+thread_local char g_msg[512];
+
+la_status fail(la_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+la_status ok() {
+  g_msg[0] = 0;
+  return LA_OK;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_smem_optin[kMaxDevices];
+
+int elem_size(int dtype) { return dtype == LA_F32 ? 4 : 2; }
+
+bool head_dim_ok(int64_t d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
+
+// Shape, stride and alignment checks common to every tensor argument.
+la_status check_tensor(const la_tensor *t, const char *name) {
+  if (!t) return fail(LA_ERR_INVALID_ARG, "%s: NULL tensor descriptor", name);
+  if (t->dtype != LA_F32 && t->dtype != LA_BF16)
+    return fail(LA_ERR_INVALID_ARG, "%s: dtype %d is not LA_F32 or LA_BF16", name, t->dtype);
+  if (t->B < 0 || t->T < 0 || t->H < 0 || t->D <= 0)
+    return fail(LA_ERR_INVALID_ARG, "%s: negative or zero size", name);
+  if (t->stride_b < 0 || t->stride_t < 0 || t->stride_h < 0)
+    return fail(LA_ERR_INVALID_ARG, "%s: negative stride", name);
+  const int64_t numel = t->B * t->T * t->H;
+  if (numel > 0 && !t->data) return fail(LA_ERR_INVALID_ARG, "%s: NULL data pointer", name);
+  const int es = elem_size(t->dtype);
+  if (((uintptr_t)t->data) % 16 != 0)
+    return fail(LA_ERR_INVALID_ARG, "%s: data pointer not 16-byte aligned", name);
+  if ((t->stride_b * es) % 16 || (t->stride_t * es) % 16 || (t->stride_h * es) % 16)
+    return fail(LA_ERR_INVALID_ARG, "%s: strides must be multiples of 16 bytes", name);
+  return LA_OK;
+}
+
+TensorView view(const la_tensor *t) { return TensorView{t->data, t->stride_b, t->stride_t, t->stride_h}; }
+
+}  // namespace
+
+int sm_count(int device) {
+  if (device < 0 || device >= kMaxDevices) return 148;
+  int v = g_sm_count[device].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || v <= 0) v = 148;
+    g_sm_count[device].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+int max_smem_optin(int device) {
+  if (device < 0 || device >= kMaxDevices) return 232448;
+  int v = g_smem_optin[device].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess || v <= 0)
+      v = 232448;
+    g_smem_optin[device].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+const char *la_status_string(int32_t status) {
+  switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: valid but not implemented";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or launch failed";
+    default: return "unknown la_status";
+  }
+}
+
+const char *la_last_error(void) { return g_msg; }
+
+int32_t la_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                   int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
+                                   int32_t dtype, int32_t flags) {
+  if (B < 0 || T < 0 || H <= 0 || n_seqs < 0 || !head_dim_ok(d_k) || !head_dim_ok(d_v))
+    return (size_t)-1;
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return (size_t)-1;
+  if (dtype != LA_F32 && dtype != LA_BF16) return (size_t)-1;
+  if (dtype == LA_F32 || (flags & LA_FLAG_SIMT)) return 0;
+  return tc_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0, chunk);
+}
+
+la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                       const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                       int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+  la_status s;
+  if ((s = check_tensor(q, "q")) != LA_OK) return s;
+  if ((s = check_tensor(k, "k")) != LA_OK) return s;
+  if ((s = check_tensor(v, "v")) != LA_OK) return s;
+  if ((s = check_tensor(out, "out")) != LA_OK) return s;
+  if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype)
+    return fail(LA_ERR_INVALID_ARG, "q, k, v and out must share one dtype");
+  if (k->B != q->B || v->B != q->B || out->B != q->B || k->T != q->T || v->T != q->T ||
+      out->T != q->T || k->H != q->H || v->H != q->H || out->H != q->H)
+    return fail(LA_ERR_INVALID_ARG, "q, k, v, out disagree on B, T or H");
+  if (k->D != q->D) return fail(LA_ERR_INVALID_ARG, "q and k must have the same head dim d_k");
+  if (out->D != v->D) return fail(LA_ERR_INVALID_ARG, "out and v must have the same head dim d_v");
+  if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
+  if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (cu_seqlens) {
+    if (q->B != 1) return fail(LA_ERR_INVALID_ARG, "packed batches (cu_seqlens) need B == 1");
+    if (n_seqs < 0) return fail(LA_ERR_INVALID_ARG, "n_seqs is negative");
+  } else if (n_seqs != q->B) {
+    return fail(LA_ERR_INVALID_ARG, "n_seqs must equal B when cu_seqlens is NULL");
+  }
+  if (((uintptr_t)final_state) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "final_state not 16-byte aligned");
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128)
+    return fail(LA_ERR_UNSUPPORTED, "chunk %d not in {16, 32, 64, 128}", chunk);
+  if (!head_dim_ok(q->D) || !head_dim_ok(v->D))
+    return fail(LA_ERR_UNSUPPORTED, "head dims (%lld, %lld) not in {16, 32, 64, 128, 256}",
+                (long long)q->D, (long long)v->D);
+
+  ChunkArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.out = out->data;
+  a.o_sb = out->stride_b;
+  a.o_st = out->stride_t;
+  a.o_sh = out->stride_h;
+  a.gamma = gamma;
+  a.cu_seqlens = cu_seqlens;
+  a.final_state = final_state;
+  a.B = q->B;
+  a.T = q->T;
+  a.n_seqs = n_seqs;
+  a.H = (int)q->H;
+  a.dk = (int)q->D;
+  a.dv = (int)v->D;
+  a.chunk = chunk;
+  a.phi = phi;
+  a.normalize = normalize ? 1 : 0;
+  a.dtype = q->dtype;
+
+  const size_t need = la_fwd_chunk_workspace_size(a.B, a.T, a.H, a.dk, a.dv, n_seqs, cu_seqlens != nullptr,
+                                                  chunk, a.dtype, flags);
+  if (need > 0 && (workspace_bytes < need || !workspace))
+    return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if (workspace && ((uintptr_t)workspace) % 256 != 0)
+    return fail(LA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+
+  cudaStream_t st = (cudaStream_t)stream;
+  int device = 0;
+  cudaError_t err = cudaGetDevice(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+
+  // No token to process: only the final states (all zero) remain to be written.
+  if (a.n_seqs == 0) return ok();
+  if (a.T == 0 || a.B == 0) {
+    if (final_state) {
+      err = cudaMemsetAsync(final_state, 0, (size_t)a.n_seqs * a.H * a.dk * a.dv * sizeof(float), st);
+      if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    }
+    return ok();
+  }
+
+  const bool use_tc = a.dtype == LA_BF16 && !(flags & LA_FLAG_SIMT) && tc_supported(a);
+  if (use_tc) {
+    const char *why = nullptr;
+    err = launch_chunk_tc(a, workspace, workspace_bytes, st, &why);
+    if (err != cudaSuccess)
+      return fail(LA_ERR_CUDA, "tensor-core chunk kernel: %s%s%s", cudaGetErrorString(err), why ? ": " : "",
+                  why ? why : "");
+    return ok();
+  }
+  if (!simt_supported(a, device))
+    return fail(LA_ERR_UNSUPPORTED, "chunk %d with d_k %d does not fit the CUDA-core kernel's shared memory",
+                chunk, a.dk);
+  err = launch_chunk_simt(a, st);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "CUDA-core chunk kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
+                  const la_tensor *out, int32_t phi, void *stream) {
+  la_status s;
+  if ((s = check_tensor(q, "q")) != LA_OK) return s;
+  if ((s = check_tensor(k, "k")) != LA_OK) return s;
+  if ((s = check_tensor(v, "v")) != LA_OK) return s;
+  if ((s = check_tensor(out, "out")) != LA_OK) return s;
+  if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype)
+    return fail(LA_ERR_INVALID_ARG, "q, k, v and out must share one dtype");
+  if (q->T != 1 || k->T != 1 || v->T != 1 || out->T != 1)
+    return fail(LA_ERR_INVALID_ARG, "la_step takes exactly one token (T == 1)");
+  if (k->B != q->B || v->B != q->B || out->B != q->B || k->H != q->H || v->H != q->H || out->H != q->H)
+    return fail(LA_ERR_INVALID_ARG, "q, k, v, out disagree on N or H");
+  if (k->D != q->D || out->D != v->D) return fail(LA_ERR_INVALID_ARG, "head dims disagree");
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (q->B * q->H > 0 && !state) return fail(LA_ERR_INVALID_ARG, "state is NULL");
+  if (((uintptr_t)state) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "state not 16-byte aligned");
+  if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
+
+  StepArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.out = out->data;
+  a.o_sb = out->stride_b;
+  a.o_sh = out->stride_h;
+  a.gamma = gamma;
+  a.state = state;
+  a.N = q->B;
+  a.H = (int)q->H;
+  a.dk = (int)q->D;
+  a.dv = (int)v->D;
+  a.phi = phi;
+  a.dtype = q->dtype;
+  if (a.dk > 256 || a.dv > 256 || !step_supported(a))
+    return fail(LA_ERR_UNSUPPORTED, "la_step needs d_k <= 256 and d_v a power of two in [4, 256]");
+  cudaError_t err = launch_step(a, (cudaStream_t)stream);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "decode kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+}  // extern "C"

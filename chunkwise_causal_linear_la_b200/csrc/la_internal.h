@@ -1,0 +1,62 @@
+// la_internal.h -- host-side interface between the C-ABI layer (la_api.cu)
+// and the kernel files.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/la_b200.h"
+
+namespace la {
+
+// Device-side view of one strided activation tensor [B, T, H, D] (D contiguous).
+struct TensorView {
+  const void *data;
+  int64_t sb, st, sh;  // element strides of B, T, H
+};
+
+// Everything a chunked-prefill kernel needs.  Sequence n covers tokens
+// [start, start + len) of batch row b:  dense  -> b = n, start = 0, len = T;
+// packed (cu_seqlens) -> b = 0, start = cu[n], len = cu[n+1] - cu[n].
+struct ChunkArgs {
+  TensorView q, k, v;
+  void *out;
+  int64_t o_sb, o_st, o_sh;
+  const float *gamma;
+  const int32_t *cu_seqlens;  // NULL for dense batches
+  float *final_state;         // NULL allowed
+  int64_t B, T, n_seqs;
+  int H, dk, dv, chunk, phi, normalize;
+  int dtype;  // la_dtype of q, k, v, out
+};
+
+struct StepArgs {
+  TensorView q, k, v;
+  void *out;
+  int64_t o_sb, o_sh;
+  const float *gamma;
+  float *state;
+  int64_t N;
+  int H, dk, dv, phi, dtype;
+};
+
+// Per-device properties, cached on first use.
+int sm_count(int device);
+int max_smem_optin(int device);
+
+// SIMT (CUDA-core, fp32 arithmetic) chunked forward.
+bool simt_supported(const ChunkArgs &a, int device);
+cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
+
+// One-token decode step.
+bool step_supported(const StepArgs &a);
+cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
+
+// Tensor-core (tcgen05 / TMA / TMEM) chunked forward for bf16.
+bool tc_supported(const ChunkArgs &a);
+size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs,
+                          bool varlen, int chunk);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream, const char **why);
+
+}  // namespace la

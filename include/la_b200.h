@@ -1,0 +1,177 @@
+/*
+ * la_b200.h -- causal linear attention on NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The method.  "1.6 长上下文与高效注意力" (long context and efficient
+ * attention), section 线性注意力 (linear attention), displayed equation:
+ * causal attention with sim(q, k) = phi(q)^T phi(k) collapses into a state
+ * S_t (d_v x d_k) and a normaliser z_t (d_k) updated once per token,
+ *     S_t = gamma S_{t-1} + v_t phi(k_t)^T,     z_t = gamma z_{t-1} + phi(k_t),
+ *     o_t = S_t phi(q_t)        or, normalised,  o_t = S_t phi(q_t) / (z_t^T phi(q_t)),
+ * with S_0 = 0, z_0 = 0.  phi is elu(x)+1 (the page's positive feature map)
+ * or the identity.  gamma is a constant decay per head (gamma = 1 is the
+ * page's equation; gamma < 1 is the decay-masked form the same chapter
+ * describes under 状态空间模型与 Mamba as linear attention with a decay mask).
+ * The same section notes that training runs in parallel or in chunks and that
+ * inference keeps O(1) state per token; "Triton fused linear attention
+ * kernels" (hotdry blog, 2025-09-14) names the chunk mode.  la_fwd_chunk is the
+ * chunk-mode prefill and la_step the one-token recurrent update.
+ *
+ * Conventions shared by every call.
+ *   Memory.  Every pointer given to a compute call is DEVICE memory on the
+ *     current CUDA device, owned by the caller.  The library allocates and
+ *     frees no device memory; scratch space is passed in as `workspace`.
+ *   Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  Calls enqueue work and return without synchronising;
+ *     a returned LA_OK means the arguments were valid and the launches were
+ *     accepted, not that the kernels have finished.
+ *   Errors.  Every call returns an la_status; nothing aborts, throws or exits
+ *     across this interface.  On an error no kernel has been launched (for
+ *     LA_ERR_CUDA, a launch itself failed).  la_last_error() gives a message
+ *     for the calling thread's last failure.
+ *   Thread safety.  Calls may come from several host threads; the only state
+ *     kept between calls is a per-thread error message and per-device
+ *     attribute caches.
+ */
+#ifndef LA_B200_H
+#define LA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported entry points (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1, /* a pointer, size, stride or value is invalid */
+  LA_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels implement */
+  LA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+  LA_ERR_CUDA = 4         /* a CUDA runtime/driver call or launch failed */
+} la_status;
+
+typedef enum { LA_PHI_IDENTITY = 0, LA_PHI_ELU1 = 1 } la_phi;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/* Flags for la_fwd_chunk. */
+#define LA_FLAG_NONE 0
+/* Run the CUDA-core (SIMT, fp32 arithmetic) chunk kernel even where the
+ * tensor-core kernel applies.  Both are CUDA kernels; there is no CPU path. */
+#define LA_FLAG_SIMT 1
+
+/*
+ * A strided 4-D activation tensor [B, T, H, D] in device memory.
+ *   data      pointer to element [0,0,0,0]; 16-byte aligned
+ *   dtype     la_dtype of every element
+ *   B,T,H,D   logical shape (batch, tokens, heads, head dim)
+ *   stride_*  element strides of the B, T and H axes; the D axis is
+ *             contiguous (stride 1).  Strides must be >= 0.
+ * [B, T, hidden] activations with hidden = H*D are this layout with
+ * stride_h = D, stride_t = H*D, stride_b = T*H*D.
+ */
+typedef struct {
+  void *data;
+  int32_t dtype;
+  int64_t B, T, H, D;
+  int64_t stride_b, stride_t, stride_h;
+} la_tensor;
+
+/*
+ * la_fwd_chunk -- chunkwise-parallel causal linear attention forward
+ * (prefill) over a dense batch or a packed variable-length batch.
+ *
+ *   q, k        [B, T, H, d_k]; v [B, T, H, d_v]; one dtype for all three.
+ *   gamma       device float[H]: the decay of each head, 0 <= gamma <= 1.
+ *   cu_seqlens  NULL for a dense batch (n_seqs = B sequences of T tokens), or
+ *               device int32[n_seqs + 1] for a packed batch: B must be 1,
+ *               sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1,
+ *               cu_seqlens[0] = 0, entries non-decreasing, last entry <= T.
+ *               The state and normaliser restart at zero for each sequence;
+ *               a zero-length sequence yields a zero final state.  The entries
+ *               are read on the device only; violating these rules gives
+ *               undefined results (the call cannot check them without a
+ *               device-to-host copy).
+ *   n_seqs      number of sequences (B when cu_seqlens is NULL).
+ *   chunk       tile length along T: 16, 32, 64 or 128.  The result does not
+ *               depend on it beyond floating-point rounding.
+ *   phi         la_phi applied to q and k (never to v).
+ *   normalize   nonzero: divide each output row by z_t^T phi(q_t).  No epsilon
+ *               is added; with phi = identity the denominator can vanish.
+ *   out         [B, T, H, d_v], same dtype as q; written for every token that
+ *               belongs to a sequence (others are left untouched).
+ *   final_state NULL, or device float[n_seqs, H, d_k, d_v] receiving S^T of
+ *               each sequence after its last token, row-major: entry
+ *               [n][h][c][r] = S[r][c].  This is the `state` la_step takes.
+ *   flags       LA_FLAG_NONE or LA_FLAG_SIMT.
+ *   workspace   device scratch of at least la_fwd_chunk_workspace_size(...)
+ *               bytes (NULL allowed when that size is 0), 256-byte aligned.
+ *               Its contents need not be initialised and are undefined after.
+ *   stream      cudaStream_t as void*.
+ *
+ * Arithmetic: bf16 inputs are read as bf16, phi is evaluated in fp32 and the
+ * tensor-core operands (phi(q), phi(k), decayed phi(k), the masked score tile
+ * and the carried state) are rounded to bf16; all accumulation, the carried
+ * state and the normaliser are fp32; `out` is rounded to its dtype once.
+ * f32 inputs run entirely in fp32 on CUDA cores (no TF32).
+ *
+ * Errors: LA_ERR_INVALID_ARG for NULL required pointers, inconsistent shapes,
+ * dtype mismatch, negative sizes, a bad phi, misaligned pointers;
+ * LA_ERR_UNSUPPORTED for a chunk outside {16,32,64,128} or head dims outside
+ * {16, 32, 64, 128, 256}; LA_ERR_WORKSPACE when the workspace is too small.
+ */
+LA_API la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                       const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs,
+                       int32_t chunk, int32_t phi, int32_t normalize, const la_tensor *out,
+                       float *final_state, int32_t flags, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace la_fwd_chunk needs for this problem: B, T, H, d_k, d_v
+ * and n_seqs as they will be passed, has_cu_seqlens nonzero for a packed
+ * batch.  Returns 0 when no workspace is needed and (size_t)-1 for arguments
+ * la_fwd_chunk would reject.  Host-only; touches no device.
+ */
+LA_API size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                   int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
+                                   int32_t dtype, int32_t flags);
+
+/*
+ * la_step -- one decode token per sequence: the recurrence applied once.
+ *   q, k   [N, 1, H, d_k]; v [N, 1, H, d_v] (la_tensor with T = 1); f32 or
+ *          bf16, one dtype for all three.
+ *   gamma  device float[H].
+ *   state  device float[N, H, d_k, d_v], S^T as la_fwd_chunk writes it,
+ *          updated in place:  S^T[c][r] <- gamma S^T[c][r] + phi(k)_c v_r.
+ *   out    [N, 1, H, d_v], q's dtype:  o_r = sum_c S^T[c][r] phi(q)_c,
+ *          read after the update (the token sees itself, as in prefill).
+ *   phi    la_phi.  No normaliser: the state carries no z.
+ * The state is read and written exactly once (fp32 arithmetic); the kernel is
+ * bound by HBM bandwidth.  Errors as for la_fwd_chunk; LA_ERR_UNSUPPORTED
+ * unless d_k <= 256 and d_v is a power of two in [4, 256]; state must be
+ * 16-byte aligned.
+ */
+LA_API la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                  float *state, const la_tensor *out, int32_t phi, void *stream);
+
+/* Static description of a status code. */
+LA_API const char *la_status_string(int32_t status);
+
+/* Message describing the calling thread's most recent failed call ("" if none). */
+LA_API const char *la_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+LA_API int32_t la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_B200_H */

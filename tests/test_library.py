@@ -1,0 +1,101 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the public
+header declares, and its host-side logic (validation, workspace sizing, status
+strings) behaves as documented.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from chunkwise_causal_linear_la_b200 import build, binding
+
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("la_fwd_chunk", "la_step", "la_fwd_chunk_workspace_size", "la_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from chunkwise_causal_linear_la_b200 import binding
+
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in binding.EXPORTS, name
+
+
+def test_library_exports_nothing_else():
+    import subprocess
+
+    from chunkwise_causal_linear_la_b200 import binding
+
+    out = subprocess.check_output(["nm", "-D", "--defined-only", binding.LIB_PATH]).decode()
+    exported = sorted(l.split()[-1] for l in out.splitlines() if l.split()[1] == "T")
+    assert exported == declared_functions()
+
+
+def test_status_strings_and_version(lib):
+    for s in range(5):
+        assert lib.la_status_string(s).startswith(b"LA_")
+    assert lib.la_status_string(99) == b"unknown la_status"
+    assert lib.la_version() >= 10000
+
+
+def test_workspace_size_host_logic(lib):
+    ws = lib.la_fwd_chunk_workspace_size
+    bad = ctypes.c_size_t(-1).value
+    assert ws(8, 128, 16, 128, 128, 8, 0, 63, 1, 0) == bad  # chunk not supported
+    assert ws(8, 128, 16, 96, 128, 8, 0, 64, 1, 0) == bad  # head dim not supported
+    assert ws(8, 128, 0, 128, 128, 8, 0, 64, 1, 0) == bad  # H = 0
+    assert ws(1, 256, 2, 64, 64, 1, 0, 64, 0, 0) == 0  # f32 runs on CUDA cores, no workspace
+    assert ws(8, 128, 16, 128, 128, 8, 0, 64, 1, 1) == 0  # forced SIMT
+
+
+def _t(B=1, T=4, H=2, D=64, dtype=1, ptr=0x1000):
+    from chunkwise_causal_linear_la_b200.binding import LaTensor
+
+    return LaTensor(ptr, dtype, B, T, H, D, T * H * D, H * D, D)
+
+
+def _call(lib, q=None, k=None, v=None, out=None, gamma=0x2000, cu=None, n=1, chunk=64, phi=0, flags=0):
+    q = q or _t()
+    k = k or _t()
+    v = v or _t()
+    out = out or _t()
+    return lib.la_fwd_chunk(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), gamma, cu, n, chunk, phi, 0,
+                            ctypes.byref(out), None, flags, None, 0, None)
+
+
+def test_validation_rejects_bad_arguments_before_any_device_call(lib):
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    assert _call(lib, gamma=None) == b.LA_ERR_INVALID_ARG
+    assert _call(lib, k=_t(dtype=0)) == b.LA_ERR_INVALID_ARG  # dtype mismatch
+    assert _call(lib, v=_t(T=5)) == b.LA_ERR_INVALID_ARG  # shape mismatch
+    assert _call(lib, q=_t(ptr=0x1004)) == b.LA_ERR_INVALID_ARG  # misaligned
+    assert _call(lib, phi=7) == b.LA_ERR_INVALID_ARG
+    assert _call(lib, flags=4) == b.LA_ERR_INVALID_ARG
+    assert _call(lib, n=2) == b.LA_ERR_INVALID_ARG  # n_seqs != B without cu_seqlens
+    assert _call(lib, q=_t(B=2), k=_t(B=2), v=_t(B=2), out=_t(B=2), cu=0x3000, n=1) == b.LA_ERR_INVALID_ARG
+    assert _call(lib, chunk=48) == b.LA_ERR_UNSUPPORTED
+    assert _call(lib, q=_t(D=96), k=_t(D=96)) == b.LA_ERR_UNSUPPORTED
+    assert b"chunk" in lib.la_last_error() or b"head dims" in lib.la_last_error()
+    null = _t(ptr=0)
+    assert _call(lib, q=null) == b.LA_ERR_INVALID_ARG
