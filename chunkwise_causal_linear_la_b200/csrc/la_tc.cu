@@ -1,10 +1,634 @@
-// la_tc.cu -- tensor-core chunk kernel (placeholder until the tcgen05 path lands).
+// la_tc.cu -- chunkwise causal linear attention forward on the sm_100a tensor
+// cores (tcgen05 + TMA + TMEM), bf16 inputs, fp32 accumulation and state.
+//
+// The method: "1.6 长上下文与高效注意力", section 线性注意力 (state S_t = gamma S_{t-1}
+// + v_t phi(k_t)^T, output o_t = S_t phi(q_t), optional normaliser z_t), run in
+// chunk mode ("Triton fused linear attention kernels", hotdry blog: chunk-mode
+// forward).  Unrolling the recurrence over a chunk of C' <= C tokens that
+// starts from state S_p gives, for i, j < C':
+//   o_i   = gamma^(i+1) S_p qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j) v_j
+//   den_i = gamma^(i+1) z_p . qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j)
+//   S'    = gamma^C' S_p + sum_j gamma^(C'-1-j) v_j kh_j^T,   z' likewise.
+//
+// One CTA owns one (sequence, head, slice of DVT value columns) and walks its
+// chunks in order with S^T[:, slice] (fp32) resident in tensor memory:
+//   warp 0      TMA producer: Q, K, V chunk tiles into an NS-deep ring.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
+//   warps 4-7   transform: phi(q), and kd_j = w_j phi(k_j) with
+//               w_j = gamma^(C'-1-j) (0 past the sequence end), in place.
+//   warps 8-11  state: S (TMEM) -> bf16 copy in shared memory for the next
+//               chunk's inter-chunk product, then S <- gamma^C'' S in TMEM;
+//               the final S^T goes to global memory.
+//   warps 12-15 output: scores -> masked, decayed bf16 tile P; then
+//               o = gamma^(i+1) (qh S_p^T) + P V, normalised, cast, stored.
+// Per chunk, four MMAs (M1..M4):
+//   M1  A  = qh kd^T                 (M=C, N=C,   K=d_k)
+//   M2  Oe = qh S_p^T                (M=C, N=DVT, K=d_k)  [skipped on chunk 0]
+//   M4  S  = (accumulate) kd^T V     (M=128 per d_k block, N=DVT, K=C)
+//   M3  Oa = P V                     (M=C, N=DVT, K=C)
+// Because kd carries gamma^(C'-1-j), A_ij = gamma^(C'-1-j) (qh_i.kh_j) and the
+// decay mask becomes one per-row factor: P_ij = A_ij / gamma^(C'-1-i) for
+// j <= i.  That needs gamma^(C-1) well inside the normal range; heads with a
+// smaller gamma ("small-gamma mode", gamma^(C-1) < 2^-64) instead keep phi(k)
+// undecayed in place, write kd to a separate tile, and take
+// P_ij = A_ij gamma^(i-j) from a table.
+//
+// Every wait is bounded: on a timeout the CTA raises an abort flag, records
+// the failure in a device error word, drains and frees its tensor memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "la_common.cuh"
 #include "la_internal.h"
+#include "la_sm100.cuh"
 
 namespace la {
-bool tc_supported(const ChunkArgs &) { return false; }
-size_t tc_workspace_bytes(int64_t, int64_t, int64_t, int, int, int64_t, bool, int) { return 0; }
-cudaError_t launch_chunk_tc(const ChunkArgs &, void *, size_t, cudaStream_t, const char **) {
-  return cudaErrorNotSupported;
+
+__device__ unsigned int g_tc_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 512;
+constexpr long long kTimeoutCycles = 4000000000LL;  // about two seconds
+constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64
+
+struct TcArgs {
+  void *out;
+  int64_t o_sb, o_st, o_sh;
+  const float *gamma;
+  const int32_t *cu_seqlens;
+  float *final_state;
+  int64_t T;
+  int H, dv, phi, normalize;
+};
+
+template <int DK, int DVT, int C, int NS>
+struct Cfg {
+  static constexpr int KB = DK / 64;    // 64-column slabs of a q/k tile
+  static constexpr int VB = DVT / 64;   // 64-column slabs of a v tile
+  static constexpr int SLAB = C * 128;  // bytes of one [C rows x 64 bf16] slab
+  static constexpr int QK_BYTES = KB * SLAB;
+  static constexpr int V_BYTES = VB * SLAB;
+  static constexpr int STAGE_BYTES = 2 * QK_BYTES + V_BYTES;
+  static constexpr int P_SLABS = C / 64;
+  static constexpr int P_BYTES = P_SLABS * SLAB;  // [C rows x C cols] bf16, K-major
+  static constexpr int SB_SLAB = DK * 128;        // [DK rows x 64 cols] bf16
+  static constexpr int SB_BYTES = VB * SB_SLAB;
+
+  static constexpr int OFF_STAGE = 0;
+  static constexpr int OFF_KX = NS * STAGE_BYTES;
+  static constexpr int OFF_P = OFF_KX + QK_BYTES;
+  static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_Z = OFF_SB + SB_BYTES;
+  static constexpr int OFF_PW = OFF_Z + DK * 4;
+  static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
+  // barriers
+  static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_AEMPTY = 3 * NS + 2,
+                       B_PFULL = 3 * NS + 4, B_SFULL = 3 * NS + 6, B_SREADY = 3 * NS + 7, B_OFULL = 3 * NS + 8,
+                       B_OEMPTY = 3 * NS + 9, NBAR = 3 * NS + 10;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+
+  // tensor memory columns
+  static constexpr int T_S = 0;                      // S^T: DK/128 blocks of DVT columns
+  static constexpr int T_A = (DK / 128) * DVT;       // two score tiles of C columns
+  static constexpr int T_OE = T_A + 2 * C;           // inter-chunk output
+  static constexpr int T_OA = T_OE + DVT;            // intra-chunk output
+  static constexpr int T_COLS_USED = T_OA + DVT;
+  static constexpr int T_COLS = T_COLS_USED <= 32 ? 32 : T_COLS_USED <= 64 ? 64 : T_COLS_USED <= 128 ? 128
+                                : T_COLS_USED <= 256 ? 256 : 512;
+
+  static_assert(C == 64, "score tiles use the M=64 tensor-memory layout");
+  static_assert(DK % 128 == 0 && DVT % 64 == 0, "tile shape");
+  static_assert(T_COLS_USED <= 512, "tensor memory");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+struct Sync {
+  uint64_t *bar;
+  volatile int *abort;
+};
+
+__device__ __forceinline__ bool wait_bar(const Sync &sy, int idx, uint32_t parity) {
+  uint64_t *b = sy.bar + idx;
+  if (mbar_test(b, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_test(b, parity)) return true;
+    if ((spin & 255) == 0) {
+      if (*sy.abort) return false;
+      if (clock64() - t0 > kTimeoutCycles) {
+        *sy.abort = 1;
+        atomicOr(&g_tc_error, 1u);
+        return false;
+      }
+    }
+  }
 }
+
+// Wait that ignores the abort flag (used to drain asynchronous arrivals).
+__device__ __forceinline__ void drain_bar(const Sync &sy, int idx, uint32_t parity) {
+  uint64_t *b = sy.bar + idx;
+  const long long t0 = clock64();
+  while (!mbar_test(b, parity)) {
+    if (clock64() - t0 > kTimeoutCycles) {
+      atomicOr(&g_tc_error, 2u);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&p);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+template <int DK, int DVT, int C, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
+  using G = Cfg<DK, DVT, C, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
+  float *pw = reinterpret_cast<float *>(sm + G::OFF_PW);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + G::OFF_MISC + 4);
+  const Sync sy{bars, abort_flag};
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- the unit this CTA owns
+  const int NVT = a.dv / DVT;
+  const int vt = blockIdx.x % NVT;
+  const int h = (blockIdx.x / NVT) % a.H;
+  const int n = blockIdx.x / (NVT * a.H);
+  int64_t start, len;
+  int bidx;
+  if (a.cu_seqlens) {
+    bidx = 0;
+    start = a.cu_seqlens[n];
+    len = (int64_t)a.cu_seqlens[n + 1] - start;
+  } else {
+    bidx = n;
+    start = 0;
+    len = a.T;
+  }
+  const int nchunks = (int)((len + C - 1) / C);
+  const float g = a.gamma[h];
+
+  // ---- setup
+  if (tid <= C) pw[tid] = decay_pow(g, tid);
+  for (int i = tid; i < DK; i += kThreads) z[i] = 0.f;
+  if (tid == 0) {
+    for (int i = 0; i < G::NBAR; ++i) {
+      uint32_t cnt = 1;
+      if ((i >= G::B_XFORM && i < G::B_XFORM + NS) || (i >= G::B_AEMPTY && i < G::B_AEMPTY + 2) ||
+          (i >= G::B_PFULL && i < G::B_PFULL + 2) || i == G::B_SREADY || i == G::B_OEMPTY)
+        cnt = 128;
+      mbar_init(bars + i, cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, G::T_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const bool small_gamma = (g < 1.f) && (pw[C - 1] < kSmallGammaLimit);
+
+  auto chunk_len = [&](int c) -> int { return (int)min((int64_t)C, len - (int64_t)c * C); };
+  auto q_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES; };
+  auto k_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + G::QK_BYTES; };
+  auto v_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + 2 * G::QK_BYTES; };
+  uint8_t *kx_tile = sm + G::OFF_KX;
+  uint8_t *sb_tile = sm + G::OFF_SB;
+  auto p_tile = [&](int b) { return sm + G::OFF_P + b * G::P_BYTES; };
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS;
+        if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1)) break;
+        mbar_arrive_expect_tx(bars + G::B_FULL + s, G::STAGE_BYTES);
+        const int t0 = (int)(start + (int64_t)c * C);
+        for (int kb = 0; kb < G::KB; ++kb) {
+          tma_load_4d(q_tile(s) + kb * G::SLAB, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
+          tma_load_4d(k_tile(s) + kb * G::SLAB, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
+        }
+        for (int vb = 0; vb < G::VB; ++vb)
+          tma_load_4d(v_tile(s) + vb * G::SLAB, &tm_v, bars + G::B_FULL + s, vt * DVT + vb * 64, h, t0, bidx);
+        issued = c + 1;
+      }
+      if (*abort_flag) {  // let every issued copy land before the CTA exits
+        for (int c = max(0, issued - NS); c < issued; ++c) drain_bar(sy, G::B_FULL + c % NS, (c / NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_M1 = idesc_bf16_f32(C, C, 0, 0);
+      constexpr uint32_t ID_M2 = idesc_bf16_f32(C, DVT, 0, 1);
+      constexpr uint32_t ID_M3 = idesc_bf16_f32(C, DVT, 0, 1);
+      constexpr uint32_t ID_M4 = idesc_bf16_f32(128, DVT, 1, 1);
+      int done = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS, b = c & 1;
+        if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) break;
+        if (!wait_bar(sy, G::B_AEMPTY + b, ((c >> 1) & 1) ^ 1)) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(q_tile(s)), ka = smem_u32(k_tile(s)), va = smem_u32(v_tile(s));
+        // M1: scores
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
+          umma_bf16(tbase + G::T_A + b * C, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                    ID_M1, kk > 0);
+        }
+        umma_commit(bars + G::B_AFULL + b);
+        if (c > 0) {
+          if (!wait_bar(sy, G::B_SREADY, (c - 1) & 1)) break;
+          if (!wait_bar(sy, G::B_OEMPTY, (c - 1) & 1)) break;
+          tc_fence_after();
+          // M2: inter-chunk output from the bf16 copy of S_p
+          const uint32_t sba = smem_u32(sb_tile);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
+            umma_bf16(tbase + G::T_OE, smem_desc_sw128(qa + off, 16, 1024),
+                      smem_desc_sw128(sba + kk * 2048, G::SB_SLAB, 1024), ID_M2, kk > 0);
+          }
+        }
+        // M4: state update S += kd^T V
+        const uint32_t kda = small_gamma ? smem_u32(kx_tile) : ka;
+#pragma unroll
+        for (int mb = 0; mb < DK / 128; ++mb) {
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) {
+            umma_bf16(tbase + G::T_S + mb * DVT, smem_desc_sw128(kda + 2 * mb * G::SLAB + kk * 2048, G::SLAB, 1024),
+                      smem_desc_sw128(va + kk * 2048, G::SLAB, 1024), ID_M4, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(bars + G::B_SFULL);
+        // M3: intra-chunk output
+        if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(p_tile(b));
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
+          umma_bf16(tbase + G::T_OA, smem_desc_sw128(pa + off, 16, 1024), smem_desc_sw128(va + kk * 2048, G::SLAB, 1024),
+                    ID_M3, kk > 0);
+        }
+        umma_commit(bars + G::B_OFULL);
+        umma_commit(bars + G::B_EMPTY + s);
+        done = c + 1;
+      }
+      // the last commits arrive asynchronously: wait for them before tensor memory is freed
+      for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ================================================================ transform
+    const int tt = tid - 128;
+    const bool elu = a.phi != 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % NS, k = c / NS;
+      if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
+      const int Cp = chunk_len(c);
+      if (small_gamma && c > 0 && !wait_bar(sy, G::B_SFULL, (c - 1) & 1)) break;
+      const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
+      if (need_k) {
+        uint8_t *kt = k_tile(s);
+        for (int e = tt; e < G::QK_BYTES / 16; e += 128) {
+          const int off = e * 16;
+          const int j = (off % G::SLAB) >> 7;
+          const float w = j < Cp ? pw[Cp - 1 - j] : 0.f;
+          float f[8];
+          unpack8(*reinterpret_cast<const uint4 *>(kt + off), f);
+          if (elu) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = feature_map(f[u], 1);
+          }
+          if (small_gamma) {
+            float d[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) d[u] = f[u] * w;
+            *reinterpret_cast<uint4 *>(kx_tile + off) = pack8(d);
+            if (elu) *reinterpret_cast<uint4 *>(kt + off) = pack8(f);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] *= w;
+            *reinterpret_cast<uint4 *>(kt + off) = pack8(f);
+          }
+        }
+      }
+      if (elu) {
+        uint8_t *qt = q_tile(s);
+        for (int e = tt; e < G::QK_BYTES / 16; e += 128) {
+          float f[8];
+          unpack8(*reinterpret_cast<const uint4 *>(qt + e * 16), f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = feature_map(f[u], 1);
+          *reinterpret_cast<uint4 *>(qt + e * 16) = pack8(f);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_XFORM + s);
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ================================================================ state
+    const int sp = warp & 3;
+    float *F = a.final_state ? a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT : nullptr;
+    if (nchunks == 0 && F) {
+      for (int mb = 0; mb < DK / 128; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;
+        for (int col = 0; col < DVT; col += 4)
+          *reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv + col) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      if (!wait_bar(sy, G::B_SFULL, c & 1)) break;
+      tc_fence_after();
+      const bool last = c == nchunks - 1;
+      const float gsc = last ? 1.f : pw[chunk_len(c + 1)];
+#pragma unroll 1
+      for (int mb = 0; mb < DK / 128; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
+#pragma unroll 1
+        for (int grp = 0; grp < DVT / 32; ++grp) {
+          const uint32_t taddr = tbase + ((uint32_t)(sp * 32) << 16) + G::T_S + mb * DVT + grp * 32;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr, r);
+          tmem_wait_ld();
+          if (last) {
+            if (F) {
+              float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv + grp * 32);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                     __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            }
+          } else {
+            const int slab = (grp * 32) >> 6;
+            const int ch0 = ((grp * 32) & 63) >> 3;
+            uint8_t *row = sb_tile + slab * G::SB_SLAB + kr * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                                         pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                                         pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                                         pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+              *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) = v;
+            }
+            if (gsc != 1.f) {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * gsc);
+              tmem_st_32x32b_x32(taddr, r);
+            }
+          }
+        }
+      }
+      if (!last) {
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bars + G::B_SREADY);
+      }
+    }
+  } else if (warp >= 12) {
+    // ================================================================ output
+    const int sp = warp & 3;
+    const int ot = tid - 384;
+    const int i = sp * 16 + (lane & 15);  // chunk row held by this thread
+    const int hf = lane >> 4;             // which half of the columns
+    uint8_t *obase = reinterpret_cast<uint8_t *>(a.out) +
+                     2 * ((int64_t)bidx * a.o_sb + (int64_t)h * a.o_sh + vt * DVT);
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % NS, k = c / NS, b = c & 1;
+      const int Cp = chunk_len(c);
+      if (!wait_bar(sy, G::B_AFULL + b, (c >> 1) & 1)) break;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bars + G::B_AEMPTY + b);
+
+      float den = 1.f;
+      float zq = 0.f;
+      if (a.normalize) {
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) break;
+        // zq = z_p . qh_i over this thread's half of d_k
+        const uint8_t *qt = q_tile(s);
+#pragma unroll 1
+        for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
+          const uint8_t *row = qt + kb * G::SLAB + i * 128;
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(row + p * 16), f);
+            const int col = kb * 64 + ((p ^ (i & 7)) << 3);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) zq = fmaf(z[col + u], f[u], zq);
+          }
+        }
+        zq += __shfl_xor_sync(0xffffffffu, zq, 16);
+        named_bar_sync(1, 128);
+        // z <- gamma^C' z + sum_j kd_j
+        const uint8_t *kt = k_tile(s);
+        for (int col = ot; col < DK; col += 128) {
+          const int slab = col >> 6, lc = (col & 63) >> 3, e = col & 7;
+          float acc = 0.f;
+          for (int j = 0; j < Cp; ++j) {
+            const uint16_t bits =
+                *reinterpret_cast<const uint16_t *>(kt + slab * G::SLAB + j * 128 + ((lc ^ (j & 7)) << 4) + 2 * e);
+            const float x = __uint_as_float((uint32_t)bits << 16);
+            acc = small_gamma ? fmaf(pw[Cp - 1 - j], x, acc) : acc + x;
+          }
+          z[col] = fmaf(pw[Cp], z[col], acc);
+        }
+        named_bar_sync(1, 128);
+      }
+
+      // P: decay mask applied to the score tile, rounded to bf16
+      const float rs = (i < Cp && !small_gamma) ? 1.f / pw[Cp - 1 - i] : 0.f;
+      float f[32];
+      float rowsum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = hf * 32 + e;
+        const float x = __uint_as_float(r[e]);
+        float p = 0.f;
+        if (j <= i && i < Cp) p = small_gamma ? x * pw[i - j] : x * rs;
+        f[e] = p;
+        rowsum += p;
+      }
+      {
+        uint8_t *prow = p_tile(b) + i * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
+                                     pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
+          *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
+        }
+      }
+      rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
+      if (a.normalize) den = fmaf(pw[i + 1], zq, rowsum);
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_PFULL + b);
+
+      // output epilogue
+      if (!wait_bar(sy, G::B_OFULL, c & 1)) break;
+      tc_fence_after();
+      const float gi = pw[i + 1];
+      const float inv = 1.f / den;
+      uint8_t *orow = obase + 2 * ((start + (int64_t)c * C + i) * a.o_st);
+#pragma unroll 1
+      for (int pass = 0; pass < DVT / 64; ++pass) {
+        uint32_t ra[32], re[32];
+        tmem_ld_16x32bx2_x32<DVT / 2>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_OA + pass * 32, ra);
+        if (c > 0) tmem_ld_16x32bx2_x32<DVT / 2>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_OE + pass * 32, re);
+        tmem_wait_ld();
+        if (pass == DVT / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(bars + G::B_OEMPTY);
+        }
+        if (i < Cp) {
+          float o[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float inter = c > 0 ? __uint_as_float(re[e]) : 0.f;
+            o[e] = fmaf(gi, inter, __uint_as_float(ra[e])) * inv;
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + 2 * (hf * (DVT / 2) + pass * 32));
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack2(o[8 * q], o[8 * q + 1]), pack2(o[8 * q + 2], o[8 * q + 3]),
+                                pack2(o[8 * q + 4], o[8 * q + 5]), pack2(o[8 * q + 6], o[8 * q + 7]));
+        }
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    tmem_dealloc(tbase, G::T_COLS);
+    tmem_relinquish();
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, T, H, D] bf16 view as a 4-D TMA map with dims (D, H, T, B) and a
+// (64, 1, C, 1) box, 128-byte swizzle: one box is a [C rows x 64 cols] slab.
+bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t H, int64_t D, int C) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sh * 2, (cuuint64_t)t.st * 2, (cuuint64_t)t.sb * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (B == 1) strides[2] = (cuuint64_t)T * t.st * 2 > 0 ? ((cuuint64_t)T * t.st * 2 + 15) / 16 * 16 : 16;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(t.data), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int DK, int DVT, int C, int NS>
+cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why) {
+  using G = Cfg<DK, DVT, C, NS>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.B, a.T, a.H, a.dk, C) || !make_map(&mk, a.k, a.B, a.T, a.H, a.dk, C) ||
+      !make_map(&mv, a.v, a.B, a.T, a.H, a.dv, C)) {
+    if (why) *why = "cuTensorMapEncodeTiled rejected a tensor";
+    return cudaErrorInvalidValue;
+  }
+  TcArgs t;
+  t.out = a.out;
+  t.o_sb = a.o_sb;
+  t.o_st = a.o_st;
+  t.o_sh = a.o_sh;
+  t.gamma = a.gamma;
+  t.cu_seqlens = a.cu_seqlens;
+  t.final_state = a.final_state;
+  t.T = a.T;
+  t.H = a.H;
+  t.dv = a.dv;
+  t.phi = a.phi;
+  t.normalize = a.normalize;
+  const int64_t grid = a.n_seqs * a.H * (a.dv / DVT);
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  kern<<<(unsigned)grid, kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mv, t);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const ChunkArgs &a) {
+  if (a.dtype != LA_BF16 || a.chunk != 64 || a.dk != 128) return false;
+  if (a.dv != 128 && a.dv != 256) return false;
+  if (a.T > 0x7fffffffLL || a.H > 0xffff) return false;
+  return encode_fn() != nullptr;
+}
+
+size_t tc_workspace_bytes(int64_t, int64_t, int64_t, int, int, int64_t, bool, int) { return 0; }
+
+cudaError_t launch_chunk_tc(const ChunkArgs &a, void *, size_t, cudaStream_t stream, const char **why) {
+  return launch_cfg<128, 128, 64, 3>(a, stream, why);
+}
+
 }  // namespace la

@@ -1,0 +1,129 @@
+"""GPU parity of the tensor-core (tcgen05) chunk kernel against the float64 oracle.
+
+bf16 inputs, tolerance 2e-2 (slice-relative, see parity_util), for outputs and
+final states.  Shapes span several chunks and ragged tails; gammas cover the
+normal decay path (gamma^(C-1) >= 2^-64), the small-gamma path (gamma = 0,
+0.3) and gamma = 1; both feature maps; with and without the normaliser;
+dense and packed (cu_seqlens) batches.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import TOL, seq_slices, slice_rel_err, state_rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+BF = torch.bfloat16
+
+
+@pytest.fixture(scope="module")
+def la():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import chunkwise_causal_linear_la_b200 as la
+
+    la.load_library()
+    return la
+
+
+def _inputs(B, T, H, dk, dv, scale, seed):
+    from chunkwise_causal_linear_la_b200.workloads import make_qkv
+
+    return make_qkv(B, T, H, dk, dv, BF, scale, seed=seed)
+
+
+def _check(la, oracle_mod, q, k, v, gamma, cu=None, phi="identity", normalize=False, chunk=64):
+    dev = torch.device("cuda")
+    out, fs = la.la_fwd_chunk(q.to(dev), k.to(dev), v.to(dev), gamma.to(dev),
+                              cu_seqlens=None if cu is None else cu.to(dev), chunk=chunk, phi=phi,
+                              normalize=normalize)
+    torch.cuda.synchronize()
+    ref, fref = oracle_mod.recurrent(q, k, v, gamma.double().numpy(), cu_seqlens=None if cu is None else cu.numpy(),
+                                     phi=phi, normalize=normalize)
+    B, T = q.shape[:2]
+    e1 = slice_rel_err(to_np(out), ref, seq_slices(B, T, None if cu is None else cu.tolist()))
+    e2 = state_rel_err(to_np(fs), fref)
+    assert np.isfinite(to_np(out)).all()
+    assert e1 < TOL[BF] and e2 < TOL[BF], (e1, e2)
+    return e1, e2
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 4 * 64 + 17])
+def test_tc_lengths(la, oracle_mod, T):
+    q, k, v = _inputs(2, T, 3, 128, 128, 128 ** -0.5, seed=T)
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.9, 0.999, 1.0]))
+
+
+@pytest.mark.parametrize("gamma", [0.0, 0.3, 0.5, 0.9, 0.97, 1.0])
+def test_tc_gammas(la, oracle_mod, gamma):
+    q, k, v = _inputs(1, 300, 2, 128, 128, 128 ** -0.5, seed=7)
+    _check(la, oracle_mod, q, k, v, torch.tensor([gamma, gamma]))
+
+
+@pytest.mark.parametrize("phi,normalize", [("elu1", True), ("elu1", False), ("identity", False)])
+@pytest.mark.parametrize("gamma", [1.0, 0.95, 0.2])
+def test_tc_feature_maps(la, oracle_mod, phi, normalize, gamma):
+    q, k, v = _inputs(2, 333, 2, 128, 128, 128 ** -0.5, seed=3)
+    _check(la, oracle_mod, q, k, v, torch.tensor([gamma, 1.0]), phi=phi, normalize=normalize)
+
+
+def test_tc_dv256(la, oracle_mod):
+    q, k, _ = _inputs(2, 150, 2, 128, 128, 128 ** -0.5, seed=9)
+    _, _, v = _inputs(2, 150, 2, 128, 256, 128 ** -0.5, seed=10)
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.98, 1.0]))
+
+
+def test_tc_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    lengths = [130, 0, 1, 64, 65, 300, 17, 128]
+    cu = cu_seqlens_from_lengths(lengths)
+    q, k, v = _inputs(1, int(cu[-1]), 4, 128, 128, 128 ** -0.5, seed=5)
+    _check(la, oracle_mod, q, k, v, torch.tensor([1.0, 0.9, 0.99, 0.0]), cu=cu, phi="elu1", normalize=True)
+    _check(la, oracle_mod, q, k, v, torch.tensor([1.0, 0.9, 0.99, 0.0]), cu=cu)
+
+
+def test_tc_varlen_config_sample(la, oracle_mod):
+    """The packed-batch workload (64 sequences, lengths U[128, 2048], H=8, d=128,
+    elu+1 with normaliser, gamma=1) at full size; the oracle checks 2 heads."""
+    from chunkwise_causal_linear_la_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS["varlen"]
+    x = make_inputs(w, seed=0)
+    dev = torch.device("cuda")
+    out, fs = la.la_fwd_chunk(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), x["gamma"].to(dev),
+                              cu_seqlens=x["cu_seqlens"].to(dev), chunk=64, phi="elu1", normalize=True)
+    torch.cuda.synchronize()
+    heads = [0, 5]
+    cu = x["cu_seqlens"]
+    ref, fref = oracle_mod.recurrent(x["q"][:, :, heads], x["k"][:, :, heads], x["v"][:, :, heads],
+                                     np.ones(len(heads)), cu_seqlens=cu.numpy(), phi="elu1", normalize=True)
+    o = to_np(out[:, :, heads])
+    assert slice_rel_err(o, ref, seq_slices(1, 0, cu.tolist())) < TOL[BF]
+    assert state_rel_err(to_np(fs[:, heads]), fref) < TOL[BF]
+
+
+def test_tc_matches_simt(la):
+    """Tensor-core and CUDA-core kernels agree on the same bf16 inputs."""
+    q, k, v = _inputs(2, 500, 4, 128, 128, 128 ** -0.5, seed=1)
+    dev = torch.device("cuda")
+    g = torch.tensor([0.9, 0.95, 0.99, 1.0], device=dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o1, f1 = la.la_fwd_chunk(qd, kd, vd, g, chunk=64)
+    o2, f2 = la.la_fwd_chunk(qd, kd, vd, g, chunk=64, flags=la.LA_FLAG_SIMT)
+    torch.cuda.synchronize()
+    assert slice_rel_err(to_np(o1), to_np(o2), seq_slices(2, 500)) < TOL[BF]
+    assert state_rel_err(to_np(f1), to_np(f2)) < TOL[BF]
+
+
+def test_tc_repeatable(la):
+    """Two runs on the same inputs give bit-identical results (no races)."""
+    q, k, v = _inputs(2, 700, 4, 128, 128, 128 ** -0.5, seed=2)
+    dev = torch.device("cuda")
+    g = torch.tensor([0.9, 0.95, 0.99, 1.0], device=dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o1, f1 = la.la_fwd_chunk(qd, kd, vd, g, phi="elu1", normalize=True)
+    o2, f2 = la.la_fwd_chunk(qd, kd, vd, g, phi="elu1", normalize=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(f1, f2)
