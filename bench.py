@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark: chunkwise causal linear attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la|reference]
+                    [--workload NAME]
+
+One step = one la_fwd_chunk call (the whole hot path: phi, intra-chunk
+products, inter-chunk state carry, normaliser, epilogue) over one batch of the
+workload, inputs resident in HBM.  Default workload: B=8, H=16, d_k=d_v=128,
+T=16384, bf16, gamma_h evenly spaced in [0.9, 0.999], phi=identity, chunk=64,
+unnormalised.  The inputs (2.15 GB per step) are larger than L2, so no flush
+is needed between steps.
+
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun, one rank per GPU): every
+rank runs its own batch (independent sequences -> weak scaling, no collective
+on the data path); the time is the maximum over ranks of the device time.
+
+--impl reference times the float64 CPU oracle (the only reference that
+exists) on a bounded prefix sample of the same workload per step, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal linear-attn fwd tokens/s and % of roofline (bf16, B200)"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons, sampled every 50 ms in a thread."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.samples = []  # (t, sm, smmax, [reason flags])
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm, smax = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            flags = [p.lower().startswith("active") for p in parts[3:7]]
+            self.samples.append((time.time(), sm, smax, flags))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        win = [s for s in self.samples if t0 - 0.05 <= s[0] <= t1 + 0.05]
+        if not win and self.samples:  # region shorter than the sampling period: nearest samples
+            win = sorted(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))[:3]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({n for s in win for n, f in zip(self.NAMES, s[3]) if f})
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": max(s[2] for s in win),
+                "reasons": reasons, "samples": len(win)}
+
+
+def _algorithmic(w, n_seqs, tokens):
+    """Bytes and flops one launch must move / perform (per rank)."""
+    e = 2 if w.dtype == "bf16" else 4
+    bytes_ = tokens * w.H * e * (2 * w.d_k + 2 * w.d_v) + n_seqs * w.H * w.d_k * w.d_v * 4
+    C = w.chunk
+    flops = tokens * w.H * ((C + 1) * (w.d_k + w.d_v) + 4 * w.d_k * w.d_v)
+    return bytes_, flops
+
+
+def _kernel_sources_sha():
+    h = hashlib.sha256()
+    for fn in ("la_tc.cu", "la_sm100.cuh", "la_common.cuh"):
+        with open(os.path.join(ROOT, "chunkwise_causal_linear_la_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload_name, units_scale):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        ent = t["chunk_tc_kernel"]
+        if ent.get("source_sha") != _kernel_sources_sha():
+            return None
+        if ent.get("workload") == workload_name:
+            return float(ent["dram_bytes_per_launch"])
+        if "dram_bytes_per_unit" in ent:
+            return float(ent["dram_bytes_per_unit"]) * units_scale
+    except Exception:
+        return None
+    return None
+
+
+def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1):
+    """Time the float64 oracle on a prefix of the first nseq sequences (all heads).
+
+    Returns (tokens/s, tokens per sequence, secs, threads)."""
+    import oracle
+
+    oracle.build()
+    T = int(x["q"].shape[1]) if w.varlen is None else int(x["cu_seqlens"][1])
+    if w.varlen is not None:
+        nseq = 1
+    q, k, v = (t[:nseq] for t in (x["q"], x["k"], x["v"]))
+    g = x["gamma"].double().cpu().numpy()
+    # calibrate on a short prefix
+    n0 = min(T, 64)
+    t0 = time.perf_counter()
+    oracle.recurrent(q[:, :n0].cpu(), k[:, :n0].cpu(), v[:, :n0].cpu(), g, phi=w.phi, normalize=w.normalize)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(T, max(n0, n0 * budget_s / dt)))
+    if max_tokens:
+        n = min(n, max_tokens)
+    qs, ks, vs = (t[:, :n].cpu().contiguous() for t in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.recurrent(qs, ks, vs, g, phi=w.phi, normalize=w.normalize)
+    secs = time.perf_counter() - t0
+    return nseq * n / secs, n, secs, oracle.max_threads()
+
+
+def run_reference(args):
+    """The reference arm: the float64 oracle timed on host cores, rank 0 only."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import torch
+
+    from chunkwise_causal_linear_la_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, seed=0, device="cpu", B=1, T=min(w.T, 4096) if w.varlen is None else None)
+    # per step: a prefix sample sized so that all steps fit in about two minutes
+    per_step = max(0.02, 120.0 / max(1, args.steps + args.warmup))
+    import oracle
+
+    oracle.build()
+    _, n, _, threads = _oracle_rate(w, x, per_step)
+    q, k, v = (t[:1, :n].contiguous() for t in (x["q"], x["k"], x["v"]))
+    g = x["gamma"].double().numpy()
+    for _ in range(args.warmup):
+        oracle.recurrent(q, k, v, g, phi=w.phi, normalize=w.normalize)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrent(q, k, v, g, phi=w.phi, normalize=w.normalize)
+    secs = time.perf_counter() - t0
+    value = n * args.steps / secs
+    sample = "sequence 0 of %s, all %d heads, first %d tokens per step (float64 recurrence)" % (w.name, w.H, n)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w, ws),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, ws):
+    return {
+        "workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "B_per_gpu": w.B, "H": w.H,
+        "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk, "phi": w.phi, "normalize": w.normalize,
+        "gamma": "evenly spaced in [%.3g, %.3g]" % (min(w.gamma), max(w.gamma)),
+        "parallelism": "dp%d" % ws, "l2": "inputs larger than L2 (no flush needed)",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="la", choices=["la", "reference"])
+    ap.add_argument("--workload", default="sweep_T16384")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import chunkwise_causal_linear_la_b200 as la
+    from chunkwise_causal_linear_la_b200.workloads import DECODE, WORKLOADS, make_decode_inputs, make_inputs
+
+    ws, rank, local = _dist()
+    if ws != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, ws))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    hbm_peak, tc_peak, peak_kind = _peaks()
+
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, seed=rank, device=dev)
+    q, k, v, g, cu = x["q"], x["k"], x["v"], x["gamma"], x["cu_seqlens"]
+    B, T = q.shape[:2]
+    n_seqs = B if cu is None else cu.numel() - 1
+    tokens = B * T if cu is None else int(cu[-1])
+    out = torch.empty((B, T, w.H, w.d_v), dtype=q.dtype, device=dev)
+    fs = torch.empty((n_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
+    nws = la.workspace_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, w.chunk, q.dtype)
+    wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        la.la_fwd_chunk(q, k, v, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
+                        out=out, final_state=fs, workspace=wsbuf, stream=stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev).uuid and
+                           "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)).start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_wall0 = time.time()
+    e_all0, e_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_all0.record(stream)
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    e_all1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    torch.cuda.synchronize()
+    time.sleep(0.1)
+    sampler.stop()
+    elapsed_ms = e_all0.elapsed_time(e_all1)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    if ws > 1:
+        t = torch.tensor([elapsed_ms, launch_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, launch_ms = float(t[0]), float(t[1])
+    value = tokens * args.steps * ws / (elapsed_ms / 1e3)
+    alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
+    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # ---- parity on sampled (sequence, head) slices, float64 oracle (rank 0)
+    parity = None
+    if rank == 0 and not args.no_extra:
+        import numpy as np
+
+        import oracle
+
+        oracle.build()
+        torch.cuda.synchronize()
+        sl = [(0, 0), (B - 1, w.H - 1)] if cu is None else [(0, 0)]
+        worst = 0.0
+        for b, h in sl:
+            if cu is None:
+                qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
+                ref, fref = oracle.recurrent(qs, ks, vs, [float(g[h])], phi=w.phi, normalize=w.normalize)
+                o = out[b:b + 1, :, h:h + 1].float().cpu().numpy()
+                f = fs[b:b + 1, h:h + 1].cpu().numpy()
+            else:
+                s, e = int(cu[0]), int(cu[1])
+                qs, ks, vs = (t[:, s:e, h:h + 1].cpu() for t in (q, k, v))
+                ref, fref = oracle.recurrent(qs, ks, vs, [float(g[h])], phi=w.phi, normalize=w.normalize)
+                o = out[:, s:e, h:h + 1].float().cpu().numpy()
+                f = fs[0:1, h:h + 1].cpu().numpy()
+            worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))),
+                        float(np.max(np.abs(f - fref)) / np.max(np.abs(fref))))
+        parity = {"max_rel_err": worst, "tolerance": 2e-2 if w.dtype == "bf16" else 1e-4,
+                  "slices": "(sequence, head) = %s vs float64 oracle, full length" % sl}
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    fh = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(out, non_blocking=True)
+        fh.copy_(fs, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = out.numel() * out.element_size() + fs.numel() * fs.element_size()
+    e2e = {"value": tokens * args.e2e_steps * ws / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    # ---- decode step (la_step), HBM-bound: achieved GB/s
+    extra = {}
+    if not args.no_extra:
+        d = make_decode_inputs(DECODE["N"], DECODE["H"], DECODE["d_k"], DECODE["d_v"], DECODE["scale"],
+                               DECODE["state_std"], DECODE["gamma"], seed=rank, device=dev)
+        # four state batches used in turn: each step's 67 MB state was last touched three
+        # steps (~200 MB of traffic) earlier, so it is not served from the 126 MB L2
+        states = [d["state"]] + [d["state"].clone() for _ in range(3)]
+        st = states[0]
+        dq, dk_, dv_, dg = d["q"], d["k"], d["v"], d["gamma"]
+        do = torch.empty_like(dv_)
+        for i in range(12):
+            la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"])
+        torch.cuda.synchronize()
+        nrep = 400
+        evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nrep)]
+        for i in range(nrep):
+            evd[i][0].record(stream)
+            la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"])
+            evd[i][1].record(stream)
+        torch.cuda.synchronize()
+        us = statistics.mean(a.elapsed_time(b) for a, b in evd) * 1e3
+        dbytes = 2 * st.numel() * 4 + (dq.numel() + dk_.numel() + dv_.numel() + do.numel()) * 4
+        extra["decode"] = {"workload": DECODE["name"], "us_per_step": us, "alg_bytes": dbytes,
+                           "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
+                           "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "step_kernel",
+                           "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
+
+    # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        nseq = 1 if cu is not None else B
+        rate, n, secs, threads = _oracle_rate(w, x, budget_s=12.0 / nseq, nseq=nseq)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "%d sequence(s) of %s, all %d heads, first %d tokens each (float64 recurrence, %.1f s)"
+                         % (nseq, w.name, w.H, n, secs)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype), "data": "synthetic",
+            "config": _config(w, ws),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": _traffic(w.name, 1.0),
+                         "peak_kind": "%s (burst copy bandwidth)" % peak_kind,
+                         "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
+                         "launch_ms": launch_ms, "kernel": "chunk_tc_kernel"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+            "parity": parity, "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -183,3 +183,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 
 }  // namespace sm100
 }  // namespace la
+
+namespace la {
+namespace sm100 {
+// Warpgroup-wide register reallocation (all 128 threads of a warpgroup).
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+}  // namespace sm100
+}  // namespace la

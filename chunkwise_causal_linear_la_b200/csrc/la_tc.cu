@@ -9,29 +9,34 @@
 //   o_i   = gamma^(i+1) S_p qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j) v_j
 //   den_i = gamma^(i+1) z_p . qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j)
 //   S'    = gamma^C' S_p + sum_j gamma^(C'-1-j) v_j kh_j^T,   z' likewise.
+// With the decayed keys kd_j = gamma^(C'-1-j) kh_j every decay factor becomes
+// a per-row factor: multiplying o_i by gamma^(C'-1-i),
+//   o_i gamma^(C'-1-i)   = qh_i (gamma^C' S_p)^T + sum_{j<=i} (qh_i . kd_j) v_j
+//   den_i gamma^(C'-1-i) = qh_i . (gamma^C' z_p) + sum_{j<=i} (qh_i . kd_j),
+// so one accumulator O = qh Sb^T + P V, with Sb = gamma^C' S_p (bf16) and
+// P = tril(qh kd^T) (bf16, no per-element scaling), gives o_i = O_i / den'_i
+// when normalised and o_i = O_i / gamma^(C'-1-i) otherwise.  This needs
+// gamma^(C-1) well inside the normal range; heads with gamma^(C-1) < 2^-64
+// ("small-gamma mode") keep phi(k) undecayed for the scores, use a separate
+// decayed key tile for the state, P_ij = (qh_i.kh_j) gamma^(i-j) from a table,
+// and two accumulators O_inter = qh S_p^T and O_intra = P V combined as
+// o_i = gamma^(i+1) O_inter_i + O_intra_i.
 //
 // One CTA owns one (sequence, head, slice of DVT value columns) and walks its
-// chunks in order with S^T[:, slice] (fp32) resident in tensor memory:
+// chunks in order; the fp32 state S^T[:, slice] lives in the registers of the
+// state warpgroup:
 //   warp 0      TMA producer: Q, K, V chunk tiles into an NS-deep ring.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 4-7   transform: phi(q), and kd_j = w_j phi(k_j) with
-//               w_j = gamma^(C'-1-j) (0 past the sequence end), in place.
-//   warps 8-11  state: S (TMEM) -> bf16 copy in shared memory for the next
-//               chunk's inter-chunk product, then S <- gamma^C'' S in TMEM;
-//               the final S^T goes to global memory.
-//   warps 12-15 output: scores -> masked, decayed bf16 tile P; then
-//               o = gamma^(i+1) (qh S_p^T) + P V, normalised, cast, stored.
-// Per chunk, four MMAs (M1..M4):
-//   M1  A  = qh kd^T                 (M=C, N=C,   K=d_k)
-//   M2  Oe = qh S_p^T                (M=C, N=DVT, K=d_k)  [skipped on chunk 0]
-//   M4  S  = (accumulate) kd^T V     (M=128 per d_k block, N=DVT, K=C)
-//   M3  Oa = P V                     (M=C, N=DVT, K=C)
-// Because kd carries gamma^(C'-1-j), A_ij = gamma^(C'-1-j) (qh_i.kh_j) and the
-// decay mask becomes one per-row factor: P_ij = A_ij / gamma^(C'-1-i) for
-// j <= i.  That needs gamma^(C-1) well inside the normal range; heads with a
-// smaller gamma ("small-gamma mode", gamma^(C-1) < 2^-64) instead keep phi(k)
-// undecayed in place, write kd to a separate tile, and take
-// P_ij = A_ij gamma^(i-j) from a table.
+//   warps 4-7   transform: phi(q) and the decayed keys, in place.
+//   warps 8-11  state: S <- gamma^C' S + U (U from tensor memory), the bf16
+//               operand Sb for the next chunk, and the final state.
+//   warps 12-15 output: score tile -> P (one chunk ahead), then the epilogue
+//               (row factor, cast, store) of the previous chunk.
+// Per chunk, four MMAs:
+//   M1  A = qh kd^T          (M=C, N=C,   K=d_k)     -> A[c%2]
+//   M4  U = kd^T V           (M=128 per d_k block, N=DVT, K=C)
+//   M2  O = qh Sb^T          (M=C, N=DVT, K=d_k)     [skipped on chunk 0]
+//   M3  O += P V             (M=C, N=DVT, K=C)       -> O[c%2]
 //
 // Every wait is bounded: on a timeout the CTA raises an abort flag, records
 // the failure in a device error word, drains and frees its tensor memory.
@@ -71,13 +76,13 @@ template <int DK, int DVT, int C, int NS>
 struct Cfg {
   static constexpr int KB = DK / 64;    // 64-column slabs of a q/k tile
   static constexpr int VB = DVT / 64;   // 64-column slabs of a v tile
+  static constexpr int MB = DK / 128;   // 128-row blocks of the state
   static constexpr int SLAB = C * 128;  // bytes of one [C rows x 64 bf16] slab
   static constexpr int QK_BYTES = KB * SLAB;
   static constexpr int V_BYTES = VB * SLAB;
   static constexpr int STAGE_BYTES = 2 * QK_BYTES + V_BYTES;
-  static constexpr int P_SLABS = C / 64;
-  static constexpr int P_BYTES = P_SLABS * SLAB;  // [C rows x C cols] bf16, K-major
-  static constexpr int SB_SLAB = DK * 128;        // [DK rows x 64 cols] bf16
+  static constexpr int P_BYTES = (C / 64) * SLAB;  // [C rows x C cols] bf16, K-major
+  static constexpr int SB_SLAB = DK * 128;         // [DK rows x 64 cols] bf16
   static constexpr int SB_BYTES = VB * SB_SLAB;
 
   static constexpr int OFF_STAGE = 0;
@@ -89,23 +94,24 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
   // barriers
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_AEMPTY = 3 * NS + 2,
-                       B_PFULL = 3 * NS + 4, B_SFULL = 3 * NS + 6, B_SREADY = 3 * NS + 7, B_OFULL = 3 * NS + 8,
-                       B_OEMPTY = 3 * NS + 9, NBAR = 3 * NS + 10;
+                       B_PFULL = 3 * NS + 4, B_UFULL = 3 * NS + 6, B_UEMPTY = 3 * NS + 7, B_SBFULL = 3 * NS + 8,
+                       B_SBEMPTY = 3 * NS + 9, B_OFULL = 3 * NS + 10, B_OEMPTY = 3 * NS + 12, NBAR = 3 * NS + 14;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
   // tensor memory columns
-  static constexpr int T_S = 0;                      // S^T: DK/128 blocks of DVT columns
-  static constexpr int T_A = (DK / 128) * DVT;       // two score tiles of C columns
-  static constexpr int T_OE = T_A + 2 * C;           // inter-chunk output
-  static constexpr int T_OA = T_OE + DVT;            // intra-chunk output
-  static constexpr int T_COLS_USED = T_OA + DVT;
+  static constexpr int T_U = 0;                // per-chunk state update: MB blocks of DVT columns
+  static constexpr int T_A = MB * DVT;         // two score tiles of C columns
+  static constexpr int T_O = T_A + 2 * C;      // two output tiles of DVT columns
+  static constexpr int T_COLS_USED = T_O + 2 * DVT;
   static constexpr int T_COLS = T_COLS_USED <= 32 ? 32 : T_COLS_USED <= 64 ? 64 : T_COLS_USED <= 128 ? 128
                                 : T_COLS_USED <= 256 ? 256 : 512;
+  static constexpr int RPT = MB * DVT;  // state values held per state-warpgroup thread
 
   static_assert(C == 64, "score tiles use the M=64 tensor-memory layout");
   static_assert(DK % 128 == 0 && DVT % 64 == 0, "tile shape");
+  static_assert(RPT <= 128, "state registers");
   static_assert(T_COLS_USED <= 512, "tensor memory");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -205,7 +211,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = 0; i < G::NBAR; ++i) {
       uint32_t cnt = 1;
       if ((i >= G::B_XFORM && i < G::B_XFORM + NS) || (i >= G::B_AEMPTY && i < G::B_AEMPTY + 2) ||
-          (i >= G::B_PFULL && i < G::B_PFULL + 2) || i == G::B_SREADY || i == G::B_OEMPTY)
+          (i >= G::B_PFULL && i < G::B_PFULL + 2) || i == G::B_UEMPTY || i == G::B_SBFULL ||
+          (i >= G::B_OEMPTY && i < G::B_OEMPTY + 2))
         cnt = 128;
       mbar_init(bars + i, cnt);
     }
@@ -232,9 +239,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t *sb_tile = sm + G::OFF_SB;
   auto p_tile = [&](int b) { return sm + G::OFF_P + b * G::P_BYTES; };
 
-  if (warp == 0) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
+  if (warp < 4) {
+    reg_dealloc<56>();
+    if (warp == 0 && lane == 0) {
+      // ============================================================ TMA producer
       int issued = 0;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
@@ -252,17 +260,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (*abort_flag) {  // let every issued copy land before the CTA exits
         for (int c = max(0, issued - NS); c < issued; ++c) drain_bar(sy, G::B_FULL + c % NS, (c / NS) & 1);
       }
-    }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ============================================================ MMA issuer
       constexpr uint32_t ID_M1 = idesc_bf16_f32(C, C, 0, 0);
       constexpr uint32_t ID_M2 = idesc_bf16_f32(C, DVT, 0, 1);
       constexpr uint32_t ID_M3 = idesc_bf16_f32(C, DVT, 0, 1);
       constexpr uint32_t ID_M4 = idesc_bf16_f32(128, DVT, 1, 1);
+      const uint32_t sba = smem_u32(sb_tile);
       int done = 0;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS, b = c & 1;
+        const int ob = small_gamma ? 0 : b;
+        const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
         if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
         if (!wait_bar(sy, G::B_XFORM + s, k & 1)) break;
         if (!wait_bar(sy, G::B_AEMPTY + b, ((c >> 1) & 1) ^ 1)) break;
@@ -272,60 +281,67 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-          umma_bf16(tbase + G::T_A + b * C, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                    ID_M1, kk > 0);
+          umma_bf16(tbase + G::T_A + b * C, smem_desc_sw128(qa + off, 16, 1024),
+                    smem_desc_sw128(ka + off, 16, 1024), ID_M1, kk > 0);
         }
         umma_commit(bars + G::B_AFULL + b);
+        // M4: this chunk's state update U = kd^T V
         if (c > 0) {
-          if (!wait_bar(sy, G::B_SREADY, (c - 1) & 1)) break;
-          if (!wait_bar(sy, G::B_OEMPTY, (c - 1) & 1)) break;
+          if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1)) break;
           tc_fence_after();
-          // M2: inter-chunk output from the bf16 copy of S_p
-          const uint32_t sba = smem_u32(sb_tile);
+        }
+        const uint32_t kda = small_gamma ? smem_u32(kx_tile) : ka;
+#pragma unroll
+        for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk)
+            umma_bf16(tbase + G::T_U + mb * DVT,
+                      smem_desc_sw128(kda + 2 * mb * G::SLAB + kk * 2048, G::SLAB, 1024),
+                      smem_desc_sw128(va + kk * 2048, G::SLAB, 1024), ID_M4, kk > 0);
+        }
+        umma_commit(bars + G::B_UFULL);
+        // M2 / M3: output accumulators
+        if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1)) break;
+        tc_fence_after();
+        const uint32_t o_inter = tbase + G::T_O + ob * DVT;
+        const uint32_t o_intra = small_gamma ? tbase + G::T_O + DVT : o_inter;
+        if (c > 0) {
+          if (!wait_bar(sy, G::B_SBFULL, (c - 1) & 1)) break;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk) {
             const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-            umma_bf16(tbase + G::T_OE, smem_desc_sw128(qa + off, 16, 1024),
+            umma_bf16(o_inter, smem_desc_sw128(qa + off, 16, 1024),
                       smem_desc_sw128(sba + kk * 2048, G::SB_SLAB, 1024), ID_M2, kk > 0);
           }
+          umma_commit(bars + G::B_SBEMPTY);
         }
-        // M4: state update S += kd^T V
-        const uint32_t kda = small_gamma ? smem_u32(kx_tile) : ka;
-#pragma unroll
-        for (int mb = 0; mb < DK / 128; ++mb) {
-#pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk) {
-            umma_bf16(tbase + G::T_S + mb * DVT, smem_desc_sw128(kda + 2 * mb * G::SLAB + kk * 2048, G::SLAB, 1024),
-                      smem_desc_sw128(va + kk * 2048, G::SLAB, 1024), ID_M4, (c > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        umma_commit(bars + G::B_SFULL);
-        // M3: intra-chunk output
         if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t pa = smem_u32(p_tile(b));
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-          umma_bf16(tbase + G::T_OA, smem_desc_sw128(pa + off, 16, 1024), smem_desc_sw128(va + kk * 2048, G::SLAB, 1024),
-                    ID_M3, kk > 0);
+          umma_bf16(o_intra, smem_desc_sw128(pa + off, 16, 1024), smem_desc_sw128(va + kk * 2048, G::SLAB, 1024),
+                    ID_M3, ((!small_gamma && c > 0) || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bars + G::B_OFULL);
+        umma_commit(bars + G::B_OFULL + ob);
         umma_commit(bars + G::B_EMPTY + s);
         done = c + 1;
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
       for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp < 8) {
     // ================================================================ transform
+    reg_dealloc<80>();
     const int tt = tid - 128;
     const bool elu = a.phi != 0;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % NS, k = c / NS;
       if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
       const int Cp = chunk_len(c);
-      if (small_gamma && c > 0 && !wait_bar(sy, G::B_SFULL, (c - 1) & 1)) break;
+      if (small_gamma && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1)) break;  // M4(c-1) read kx
       const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
       if (need_k) {
         uint8_t *kt = k_tile(s);
@@ -365,89 +381,94 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       fence_proxy_async_smem();
       mbar_arrive(bars + G::B_XFORM + s);
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp < 12) {
     // ================================================================ state
+    reg_alloc<232>();
     const int sp = warp & 3;
+    float S[G::RPT];
+#pragma unroll
+    for (int u = 0; u < G::RPT; ++u) S[u] = 0.f;
     float *F = a.final_state ? a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT : nullptr;
-    if (nchunks == 0 && F) {
-      for (int mb = 0; mb < DK / 128; ++mb) {
-        const int kr = mb * 128 + sp * 32 + lane;
-        for (int col = 0; col < DVT; col += 4)
-          *reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv + col) = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
     for (int c = 0; c < nchunks; ++c) {
-      if (!wait_bar(sy, G::B_SFULL, c & 1)) break;
+      const int Cp = chunk_len(c);
+      if (!wait_bar(sy, G::B_UFULL, c & 1)) break;
       tc_fence_after();
-      const bool last = c == nchunks - 1;
-      const float gsc = last ? 1.f : pw[chunk_len(c + 1)];
-#pragma unroll 1
-      for (int mb = 0; mb < DK / 128; ++mb) {
-        const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
-#pragma unroll 1
+      const float gdec = pw[Cp];
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
         for (int grp = 0; grp < DVT / 32; ++grp) {
-          const uint32_t taddr = tbase + ((uint32_t)(sp * 32) << 16) + G::T_S + mb * DVT + grp * 32;
           uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr, r);
+          tmem_ld_32x32b_x32(tbase + ((uint32_t)(sp * 32) << 16) + G::T_U + mb * DVT + grp * 32, r);
           tmem_wait_ld();
-          if (last) {
-            if (F) {
-              float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv + grp * 32);
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                     __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-            }
-          } else {
-            const int slab = (grp * 32) >> 6;
-            const int ch0 = ((grp * 32) & 63) >> 3;
-            uint8_t *row = sb_tile + slab * G::SB_SLAB + kr * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 v = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                                         pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                                         pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                                         pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
-              *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) = v;
-            }
-            if (gsc != 1.f) {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * gsc);
-              tmem_st_32x32b_x32(taddr, r);
-            }
+          for (int e = 0; e < 32; ++e) {
+            float &x = S[mb * DVT + grp * 32 + e];
+            x = fmaf(gdec, x, __uint_as_float(r[e]));
           }
         }
       }
-      if (!last) {
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(bars + G::B_SREADY);
+      tc_fence_before();
+      mbar_arrive(bars + G::B_UEMPTY);
+      if (c == nchunks - 1) break;
+      // bf16 operand for the next chunk's inter-chunk product
+      const float sc = small_gamma ? 1.f : pw[chunk_len(c + 1)];
+      if (c >= 1 && !wait_bar(sy, G::B_SBEMPTY, (c - 1) & 1)) break;
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
+#pragma unroll
+        for (int grp = 0; grp < DVT / 32; ++grp) {
+          uint8_t *row = sb_tile + ((grp * 32) >> 6) * G::SB_SLAB + kr * 128;
+          const int ch0 = ((grp * 32) & 63) >> 3;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float *x = &S[mb * DVT + grp * 32 + 8 * q];
+            const uint4 v = make_uint4(pack2(sc * x[0], sc * x[1]), pack2(sc * x[2], sc * x[3]),
+                                       pack2(sc * x[4], sc * x[5]), pack2(sc * x[6], sc * x[7]));
+            *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) = v;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_SBFULL);
+    }
+    if (F) {  // S after the last chunk (zero for an empty sequence)
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;
+        float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv);
+#pragma unroll
+        for (int q = 0; q < DVT / 4; ++q)
+          dst[q] = make_float4(S[mb * DVT + 4 * q], S[mb * DVT + 4 * q + 1], S[mb * DVT + 4 * q + 2],
+                               S[mb * DVT + 4 * q + 3]);
       }
     }
-  } else if (warp >= 12) {
+  } else {
     // ================================================================ output
+    reg_alloc<136>();
     const int sp = warp & 3;
     const int ot = tid - 384;
     const int i = sp * 16 + (lane & 15);  // chunk row held by this thread
     const int hf = lane >> 4;             // which half of the columns
     uint8_t *obase = reinterpret_cast<uint8_t *>(a.out) +
                      2 * ((int64_t)bidx * a.o_sb + (int64_t)h * a.o_sh + vt * DVT);
-    for (int c = 0; c < nchunks; ++c) {
+
+    // scores of chunk c -> P tile; returns this row's output factor
+    auto scores = [&](int c, bool &ok) -> float {
       const int s = c % NS, k = c / NS, b = c & 1;
       const int Cp = chunk_len(c);
-      if (!wait_bar(sy, G::B_AFULL + b, (c >> 1) & 1)) break;
+      ok = false;
+      if (!wait_bar(sy, G::B_AFULL + b, (c >> 1) & 1)) return 0.f;
       tc_fence_after();
       uint32_t r[32];
       tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, r);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bars + G::B_AEMPTY + b);
-
-      float den = 1.f;
       float zq = 0.f;
       if (a.normalize) {
-        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) break;
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) return 0.f;
         // zq = z_p . qh_i over this thread's half of d_k
         const uint8_t *qt = q_tile(s);
 #pragma unroll 1
@@ -464,14 +485,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         zq += __shfl_xor_sync(0xffffffffu, zq, 16);
         named_bar_sync(1, 128);
-        // z <- gamma^C' z + sum_j kd_j
+        // z <- gamma^C' z + sum_j gamma^(C'-1-j) kh_j
         const uint8_t *kt = k_tile(s);
         for (int col = ot; col < DK; col += 128) {
           const int slab = col >> 6, lc = (col & 63) >> 3, e = col & 7;
           float acc = 0.f;
           for (int j = 0; j < Cp; ++j) {
-            const uint16_t bits =
-                *reinterpret_cast<const uint16_t *>(kt + slab * G::SLAB + j * 128 + ((lc ^ (j & 7)) << 4) + 2 * e);
+            const uint16_t bits = *reinterpret_cast<const uint16_t *>(kt + slab * G::SLAB + j * 128 +
+                                                                      ((lc ^ (j & 7)) << 4) + 2 * e);
             const float x = __uint_as_float((uint32_t)bits << 16);
             acc = small_gamma ? fmaf(pw[Cp - 1 - j], x, acc) : acc + x;
           }
@@ -479,9 +500,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         named_bar_sync(1, 128);
       }
-
-      // P: decay mask applied to the score tile, rounded to bf16
-      const float rs = (i < Cp && !small_gamma) ? 1.f / pw[Cp - 1 - i] : 0.f;
       float f[32];
       float rowsum = 0.f;
 #pragma unroll
@@ -489,47 +507,58 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int j = hf * 32 + e;
         const float x = __uint_as_float(r[e]);
         float p = 0.f;
-        if (j <= i && i < Cp) p = small_gamma ? x * pw[i - j] : x * rs;
+        if (j <= i && i < Cp) p = small_gamma ? x * pw[i - j] : x;
         f[e] = p;
         rowsum += p;
       }
-      {
-        uint8_t *prow = p_tile(b) + i * 128;
+      uint8_t *prow = p_tile(b) + i * 128;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
-                                     pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
-          *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
-        }
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
+                                   pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
+        *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
       }
-      rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
-      if (a.normalize) den = fmaf(pw[i + 1], zq, rowsum);
       fence_proxy_async_smem();
       mbar_arrive(bars + G::B_PFULL + b);
+      rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
+      ok = true;
+      if (i >= Cp) return 0.f;
+      if (small_gamma) return a.normalize ? 1.f / fmaf(pw[i + 1], zq, rowsum) : 1.f;
+      return a.normalize ? 1.f / fmaf(pw[Cp], zq, rowsum) : 1.f / pw[Cp - 1 - i];
+    };
 
-      // output epilogue
-      if (!wait_bar(sy, G::B_OFULL, c & 1)) break;
+    // epilogue of chunk c
+    auto epilogue = [&](int c, float fac) -> bool {
+      const int Cp = chunk_len(c);
+      const int ob = small_gamma ? 0 : (c & 1);
+      const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
+      if (!wait_bar(sy, G::B_OFULL + ob, oph)) return false;
       tc_fence_after();
       const float gi = pw[i + 1];
-      const float inv = 1.f / den;
       uint8_t *orow = obase + 2 * ((start + (int64_t)c * C + i) * a.o_st);
+      const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
 #pragma unroll 1
       for (int pass = 0; pass < DVT / 64; ++pass) {
         uint32_t ra[32], re[32];
-        tmem_ld_16x32bx2_x32<DVT / 2>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_OA + pass * 32, ra);
-        if (c > 0) tmem_ld_16x32bx2_x32<DVT / 2>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_OE + pass * 32, re);
-        tmem_wait_ld();
+        float o[32];
+        if (small_gamma) {
+          tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + DVT + pass * 32, ra);
+          if (c > 0) tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + pass * 32, re);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            o[e] = fmaf(gi, c > 0 ? __uint_as_float(re[e]) : 0.f, __uint_as_float(ra[e])) * fac;
+        } else {
+          tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + ob * DVT + pass * 32, ra);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ra[e]) * fac;
+        }
         if (pass == DVT / 64 - 1) {
           tc_fence_before();
-          mbar_arrive(bars + G::B_OEMPTY);
+          mbar_arrive(bars + G::B_OEMPTY + ob);
         }
         if (i < Cp) {
-          float o[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float inter = c > 0 ? __uint_as_float(re[e]) : 0.f;
-            o[e] = fmaf(gi, inter, __uint_as_float(ra[e])) * inv;
-          }
           uint4 *dst = reinterpret_cast<uint4 *>(orow + 2 * (hf * (DVT / 2) + pass * 32));
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -537,6 +566,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 pack2(o[8 * q + 4], o[8 * q + 5]), pack2(o[8 * q + 6], o[8 * q + 7]));
         }
       }
+      return true;
+    };
+
+    // scores run one chunk ahead of the epilogue
+    bool ok = true;
+    float fac_cur = 0.f, fac_next = 0.f;
+    if (nchunks > 0) fac_cur = scores(0, ok);
+    for (int c = 0; c < nchunks && ok; ++c) {
+      if (c + 1 < nchunks) {
+        fac_next = scores(c + 1, ok);
+        if (!ok) break;
+      }
+      if (!epilogue(c, fac_cur)) break;
+      fac_cur = fac_next;
     }
   }
 
