@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     LA_FLAG_NONE,
     LA_FLAG_SIMT,
     LaError,
+    device_error,
     la_fwd_chunk,
     la_step,
     load_library,

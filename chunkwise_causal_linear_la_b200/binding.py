@@ -28,7 +28,7 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 
 # Every function include/la_b200.h declares.
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_workspace_size", "la_step", "la_status_string",
-           "la_last_error", "la_version")
+           "la_last_error", "la_version", "la_device_error")
 
 
 class LaTensor(ctypes.Structure):
@@ -72,6 +72,8 @@ def load_library(path: str = LIB_PATH):
     lib.la_last_error.restype = ctypes.c_char_p
     lib.la_version.argtypes = []
     lib.la_version.restype = i32
+    lib.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32), i32]
+    lib.la_device_error.restype = i32
     _lib = lib
     return lib
 
@@ -141,6 +143,14 @@ def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", norm
     )
     _check(lib, st, "la_fwd_chunk")
     return out, final_state
+
+
+def device_error(reset: bool = True):
+    """(flags, detail) of the tensor-core kernel's bounded-wait error word (synchronises the device)."""
+    lib = load_library()
+    f, d = ctypes.c_uint32(0), ctypes.c_uint32(0)
+    _check(lib, lib.la_device_error(ctypes.byref(f), ctypes.byref(d), int(reset)), "la_device_error")
+    return int(f.value), int(d.value)
 
 
 def la_step(q, k, v, gamma, state, out=None, phi="identity", stream=None):

@@ -100,6 +100,16 @@ const char *la_last_error(void) { return g_msg; }
 
 int32_t la_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
+la_status la_device_error(uint32_t *flags, uint32_t *detail, int32_t reset) {
+  if (!flags || !detail) return fail(LA_ERR_INVALID_ARG, "flags and detail must not be NULL");
+  unsigned int f = 0, w = 0;
+  cudaError_t err = tc_device_error(&f, &w, reset != 0);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(err));
+  *flags = f;
+  *detail = w;
+  return ok();
+}
+
 size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
                                    int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
                                    int32_t dtype, int32_t flags) {

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/la_b200.h"
+#include "la_b200.h"
 
 namespace la {
 
@@ -58,5 +58,7 @@ size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64
                           bool varlen, int chunk);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t workspace_bytes,
                             cudaStream_t stream, const char **why);
+// Device error words of the tensor-core kernel (timeouts of bounded waits).
+cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset);
 
 }  // namespace la

@@ -39,7 +39,22 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
       : "memory");
 }
 
-// One non-blocking probe: true once the phase with the given parity has completed.
+// Probe that may suspend the calling thread for up to `hint_ns` nanoseconds
+// (the hardware resumes it as soon as the phase completes): true once the
+// phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// One probe without a suspend hint: true once the phase with the given parity has completed.
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -27,10 +27,10 @@
 // state warpgroup:
 //   warp 0      TMA producer: Q, K, V chunk tiles into an NS-deep ring.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 4-7   transform: phi(q) and the decayed keys, in place.
-//   warps 8-11  state: S <- gamma^C' S + U (U from tensor memory), the bf16
+//   warps 2-3   transform: phi(q) and the decayed keys, in place.
+//   warps 4-7   state: S <- gamma^C' S + U (U from tensor memory), the bf16
 //               operand Sb for the next chunk, and the final state.
-//   warps 12-15 output: score tile -> P (one chunk ahead), then the epilogue
+//   warps 8-11  output: score tile -> P (one chunk ahead), then the epilogue
 //               (row factor, cast, store) of the previous chunk.
 // Per chunk, four MMAs:
 //   M1  A = qh kd^T          (M=C, N=C,   K=d_k)     -> A[c%2]
@@ -53,13 +53,16 @@
 namespace la {
 
 __device__ unsigned int g_tc_error = 0;
+// First wait that gave up: 0x80000000 | chunk << 8 | barrier index.
+__device__ unsigned int g_tc_where = 0;
 
 namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about two seconds
+constexpr uint32_t kSuspendHintNs = 20000;
 constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64
 
 struct TcArgs {
@@ -91,11 +94,12 @@ struct Cfg {
   static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_Z = OFF_SB + SB_BYTES;
   static constexpr int OFF_PW = OFF_Z + DK * 4;
-  static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
+  static constexpr int OFF_ZRED = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;  // normaliser partial sums
+  static constexpr int OFF_BAR = OFF_ZRED + 128 * 8 * 4;
   // barriers
-  static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_AEMPTY = 3 * NS + 2,
-                       B_PFULL = 3 * NS + 4, B_UFULL = 3 * NS + 6, B_UEMPTY = 3 * NS + 7, B_SBFULL = 3 * NS + 8,
-                       B_SBEMPTY = 3 * NS + 9, B_OFULL = 3 * NS + 10, B_OEMPTY = 3 * NS + 12, NBAR = 3 * NS + 14;
+  static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_PFULL = 3 * NS + 2,
+                       B_UFULL = 3 * NS + 4, B_UEMPTY = 3 * NS + 5, B_SBFULL = 3 * NS + 6, B_SBEMPTY = 3 * NS + 7,
+                       B_OFULL = 3 * NS + 8, B_OEMPTY = 3 * NS + 10, B_OSYNC = 3 * NS + 12, NBAR = 3 * NS + 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -121,21 +125,28 @@ struct Sync {
   volatile int *abort;
 };
 
-__device__ __forceinline__ bool wait_bar(const Sync &sy, int idx, uint32_t parity) {
+// Waiting threads sleep in the barrier (suspend hint) instead of polling, so
+// they leave issue slots to the warps that share their SM sub-partition.
+__device__ __forceinline__ bool wait_bar(const Sync &sy, int idx, uint32_t parity, int chunk = 0) {
   uint64_t *b = sy.bar + idx;
   if (mbar_test(b, parity)) return true;
   const long long t0 = clock64();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_test(b, parity)) return true;
-    if ((spin & 255) == 0) {
-      if (*sy.abort) return false;
-      if (clock64() - t0 > kTimeoutCycles) {
-        *sy.abort = 1;
-        atomicOr(&g_tc_error, 1u);
-        return false;
-      }
+  while (true) {
+    if (mbar_wait_hint(b, parity, kSuspendHintNs)) return true;
+    if (*sy.abort) return false;
+    if (clock64() - t0 > kTimeoutCycles) {
+      *sy.abort = 1;
+      atomicOr(&g_tc_error, 1u);
+      atomicCAS(&g_tc_where, 0u, 0x80000000u | ((uint32_t)(chunk & 0x7FFFFF) << 8) | (uint32_t)idx);
+      return false;
     }
   }
+}
+
+// Warp-uniform wait for warps that go on to execute warp-collective or
+// .sync.aligned instructions: every lane takes the same path even on abort.
+__device__ __forceinline__ bool wait_bar_warp(const Sync &sy, int idx, uint32_t parity, int chunk = 0) {
+  return __all_sync(0xffffffffu, wait_bar(sy, idx, parity, chunk));
 }
 
 // Wait that ignores the abort flag (used to drain asynchronous arrivals).
@@ -149,6 +160,11 @@ __device__ __forceinline__ void drain_bar(const Sync &sy, int idx, uint32_t pari
     }
   }
 }
+
+// phi for the bf16 tensor-core operands: elu(x) + 1 with the hardware
+// exponential (__expf); its relative error (~1e-6 near 0) is far below the
+// bf16 rounding (2^-9) the operand gets right after.
+__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -168,7 +184,7 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
-template <int DK, int DVT, int C, int NS>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
@@ -177,6 +193,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
   float *pw = reinterpret_cast<float *>(sm + G::OFF_PW);
+  float *zred = reinterpret_cast<float *>(sm + G::OFF_ZRED);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + G::OFF_MISC + 4);
@@ -210,8 +227,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < G::NBAR; ++i) {
       uint32_t cnt = 1;
-      if ((i >= G::B_XFORM && i < G::B_XFORM + NS) || (i >= G::B_AEMPTY && i < G::B_AEMPTY + 2) ||
-          (i >= G::B_PFULL && i < G::B_PFULL + 2) || i == G::B_UEMPTY || i == G::B_SBFULL ||
+      if (i >= G::B_XFORM && i < G::B_XFORM + NS)
+        cnt = 64;
+      else if ((i >= G::B_PFULL && i < G::B_PFULL + 2) ||
+          i == G::B_UEMPTY || i == G::B_SBFULL || i == G::B_OSYNC ||
           (i >= G::B_OEMPTY && i < G::B_OEMPTY + 2))
         cnt = 128;
       mbar_init(bars + i, cnt);
@@ -240,13 +259,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto p_tile = [&](int b) { return sm + G::OFF_P + b * G::P_BYTES; };
 
   if (warp < 4) {
-    reg_dealloc<56>();
+    reg_dealloc<104>();
     if (warp == 0 && lane == 0) {
       // ============================================================ TMA producer
       int issued = 0;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
-        if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1)) break;
+        if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1, c)) break;
         mbar_arrive_expect_tx(bars + G::B_FULL + s, G::STAGE_BYTES);
         const int t0 = (int)(start + (int64_t)c * C);
         for (int kb = 0; kb < G::KB; ++kb) {
@@ -266,64 +285,77 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       constexpr uint32_t ID_M2 = idesc_bf16_f32(C, DVT, 0, 1);
       constexpr uint32_t ID_M3 = idesc_bf16_f32(C, DVT, 0, 1);
       constexpr uint32_t ID_M4 = idesc_bf16_f32(128, DVT, 1, 1);
-      const uint32_t sba = smem_u32(sb_tile);
-      int done = 0;
-      for (int c = 0; c < nchunks; ++c) {
+      const uint64_t dsb = smem_desc_sw128(smem_u32(sb_tile), G::SB_SLAB, 1024);
+      int m1_issued = 0;
+      // M1 of chunk c: scores A[c%2] = qh kd^T
+      auto issue_scores = [&](int c) -> bool {
         const int s = c % NS, k = c / NS, b = c & 1;
-        const int ob = small_gamma ? 0 : b;
-        const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
-        if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
-        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) break;
-        if (!wait_bar(sy, G::B_AEMPTY + b, ((c >> 1) & 1) ^ 1)) break;
+        // the transform warps saw the tile land before arriving; A[b] was last read
+        // by the score step of chunk c-2, whose P tile this thread already waited for
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(q_tile(s)), ka = smem_u32(k_tile(s)), va = smem_u32(v_tile(s));
-        // M1: scores
+        const uint64_t dq = smem_desc_sw128(smem_u32(q_tile(s)), 16, 1024);
+        const uint64_t dk = smem_desc_sw128(smem_u32(k_tile(s)), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-          umma_bf16(tbase + G::T_A + b * C, smem_desc_sw128(qa + off, 16, 1024),
-                    smem_desc_sw128(ka + off, 16, 1024), ID_M1, kk > 0);
+          const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+          umma_bf16(tbase + G::T_A + b * C, dq + off, dk + off, ID_M1, kk > 0);
         }
         umma_commit(bars + G::B_AFULL + b);
+        m1_issued = c + 1;
+        return true;
+      };
+      // Issue order per chunk c: M4(c), M1(c+1), M2(c), M3(c).  The next chunk's
+      // scores are queued before waiting for this chunk's P tile, so the score
+      // step of chunk c+1 overlaps the P V product of chunk c.
+      int done = 0;
+      bool ok = nchunks == 0 || issue_scores(0);
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int s = c % NS, b = c & 1;
+        const int ob = small_gamma ? 0 : b;
+        const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
+        const uint64_t dq = smem_desc_sw128(smem_u32(q_tile(s)), 16, 1024);
+        const uint64_t dv = smem_desc_sw128(smem_u32(v_tile(s)), G::SLAB, 1024);
+        const uint64_t dkd = small_gamma ? smem_desc_sw128(smem_u32(kx_tile), G::SLAB, 1024)
+                                         : smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
         // M4: this chunk's state update U = kd^T V
         if (c > 0) {
-          if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1)) break;
+          if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
           tc_fence_after();
         }
-        const uint32_t kda = small_gamma ? smem_u32(kx_tile) : ka;
 #pragma unroll
         for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk)
-            umma_bf16(tbase + G::T_U + mb * DVT,
-                      smem_desc_sw128(kda + 2 * mb * G::SLAB + kk * 2048, G::SLAB, 1024),
-                      smem_desc_sw128(va + kk * 2048, G::SLAB, 1024), ID_M4, kk > 0);
+            umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
+                      dv + ((kk * 2048) >> 4), ID_M4, kk > 0);
         }
         umma_commit(bars + G::B_UFULL);
+        // M1 of the next chunk
+        if (c + 1 < nchunks && !issue_scores(c + 1)) break;
         // M2 / M3: output accumulators
-        if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1)) break;
+        if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1, c)) break;
         tc_fence_after();
         const uint32_t o_inter = tbase + G::T_O + ob * DVT;
         const uint32_t o_intra = small_gamma ? tbase + G::T_O + DVT : o_inter;
         if (c > 0) {
-          if (!wait_bar(sy, G::B_SBFULL, (c - 1) & 1)) break;
+          if (!wait_bar(sy, G::B_SBFULL, (c - 1) & 1, c)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-            umma_bf16(o_inter, smem_desc_sw128(qa + off, 16, 1024),
-                      smem_desc_sw128(sba + kk * 2048, G::SB_SLAB, 1024), ID_M2, kk > 0);
+            const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+            umma_bf16(o_inter, dq + off, dsb + ((kk * 2048) >> 4), ID_M2, kk > 0);
           }
           umma_commit(bars + G::B_SBEMPTY);
         }
-        if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1)) break;
+        if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
         tc_fence_after();
-        const uint32_t pa = smem_u32(p_tile(b));
+        const uint64_t dp = smem_desc_sw128(smem_u32(p_tile(b)), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * G::SLAB + (kk & 3) * 32;
-          umma_bf16(o_intra, smem_desc_sw128(pa + off, 16, 1024), smem_desc_sw128(va + kk * 2048, G::SLAB, 1024),
-                    ID_M3, ((!small_gamma && c > 0) || kk > 0) ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+          umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
+                    ((!small_gamma && c > 0) || kk > 0) ? 1u : 0u);
         }
         umma_commit(bars + G::B_OFULL + ob);
         umma_commit(bars + G::B_EMPTY + s);
@@ -331,57 +363,66 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
       for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
+      if (m1_issued > done) {  // a score MMA issued ahead of an aborted chunk
+        const int c = m1_issued - 1;
+        drain_bar(sy, G::B_AFULL + (c & 1), (c >> 1) & 1);
+      }
+    } else if (warp >= 2) {
+      // ========================================================== transform
+      // 64 threads; thread tt owns the 16-byte vectors tt + 64 m of a tile.  A
+      // vector v sits in row (v mod 8C) / 8 of its [C x 64] slab.
+      const int tt = tid - 64;
+      constexpr bool elu = ELU;
+      constexpr int NV = G::QK_BYTES / 16 / 64;  // vectors per thread per tile
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS;
+        if (!wait_bar(sy, G::B_FULL + s, k & 1, c)) break;
+        const int Cp = chunk_len(c);
+        if (small_gamma && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1, c)) break;  // M4(c-1) read kx
+        const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
+#pragma unroll 1
+        for (int tile = 0; tile < 2; ++tile) {  // 0: keys (phi, decay), 1: queries (phi)
+          if (tile == 0 ? !need_k : !elu) continue;
+          uint8_t *base = tile == 0 ? k_tile(s) : q_tile(s);
+#pragma unroll 1
+          for (int m0 = 0; m0 < NV; m0 += 4) {
+            uint4 x[4];
+            float wv[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int v = tt + 64 * (m0 + m);
+              x[m] = *reinterpret_cast<const uint4 *>(base + v * 16);
+              const int j = (v % (G::SLAB / 16)) >> 3;
+              wv[m] = tile == 1 ? 1.f : (j < Cp ? pw[Cp - 1 - j] : 0.f);
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int off = (tt + 64 * (m0 + m)) * 16;
+              float f[8];
+              unpack8(x[m], f);
+              if (elu) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) f[u] = phi_fast(f[u]);
+              }
+              if (tile == 0 && small_gamma) {
+                float d[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) d[u] = f[u] * wv[m];
+                *reinterpret_cast<uint4 *>(kx_tile + off) = pack8(d);
+                if (elu) *reinterpret_cast<uint4 *>(base + off) = pack8(f);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) f[u] *= wv[m];
+                *reinterpret_cast<uint4 *>(base + off) = pack8(f);
+              }
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bars + G::B_XFORM + s);
+      }
     }
   } else if (warp < 8) {
-    // ================================================================ transform
-    reg_dealloc<80>();
-    const int tt = tid - 128;
-    const bool elu = a.phi != 0;
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c % NS, k = c / NS;
-      if (!wait_bar(sy, G::B_FULL + s, k & 1)) break;
-      const int Cp = chunk_len(c);
-      if (small_gamma && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1)) break;  // M4(c-1) read kx
-      const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
-      if (need_k) {
-        uint8_t *kt = k_tile(s);
-        for (int e = tt; e < G::QK_BYTES / 16; e += 128) {
-          const int off = e * 16;
-          const int j = (off % G::SLAB) >> 7;
-          const float w = j < Cp ? pw[Cp - 1 - j] : 0.f;
-          float f[8];
-          unpack8(*reinterpret_cast<const uint4 *>(kt + off), f);
-          if (elu) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = feature_map(f[u], 1);
-          }
-          if (small_gamma) {
-            float d[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) d[u] = f[u] * w;
-            *reinterpret_cast<uint4 *>(kx_tile + off) = pack8(d);
-            if (elu) *reinterpret_cast<uint4 *>(kt + off) = pack8(f);
-          } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] *= w;
-            *reinterpret_cast<uint4 *>(kt + off) = pack8(f);
-          }
-        }
-      }
-      if (elu) {
-        uint8_t *qt = q_tile(s);
-        for (int e = tt; e < G::QK_BYTES / 16; e += 128) {
-          float f[8];
-          unpack8(*reinterpret_cast<const uint4 *>(qt + e * 16), f);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = feature_map(f[u], 1);
-          *reinterpret_cast<uint4 *>(qt + e * 16) = pack8(f);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bars + G::B_XFORM + s);
-    }
-  } else if (warp < 12) {
     // ================================================================ state
     reg_alloc<232>();
     const int sp = warp & 3;
@@ -391,7 +432,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *F = a.final_state ? a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT : nullptr;
     for (int c = 0; c < nchunks; ++c) {
       const int Cp = chunk_len(c);
-      if (!wait_bar(sy, G::B_UFULL, c & 1)) break;
+      if (!wait_bar_warp(sy, G::B_UFULL, c & 1, c)) break;
       tc_fence_after();
       const float gdec = pw[Cp];
 #pragma unroll
@@ -413,7 +454,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (c == nchunks - 1) break;
       // bf16 operand for the next chunk's inter-chunk product
       const float sc = small_gamma ? 1.f : pw[chunk_len(c + 1)];
-      if (c >= 1 && !wait_bar(sy, G::B_SBEMPTY, (c - 1) & 1)) break;
+      if (c >= 1 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1) & 1, c)) break;
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
         const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
@@ -446,70 +487,111 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ================================================================ output
-    reg_alloc<136>();
+    reg_alloc<168>();
     const int sp = warp & 3;
-    const int ot = tid - 384;
+    const int ot = tid - 256;
     const int i = sp * 16 + (lane & 15);  // chunk row held by this thread
     const int hf = lane >> 4;             // which half of the columns
     uint8_t *obase = reinterpret_cast<uint8_t *>(a.out) +
                      2 * ((int64_t)bidx * a.o_sb + (int64_t)h * a.o_sh + vt * DVT);
 
-    // scores of chunk c -> P tile; returns this row's output factor
-    auto scores = [&](int c, bool &ok) -> float {
-      const int s = c % NS, k = c / NS, b = c & 1;
+    // bounded barrier among the 128 output threads (an mbarrier used as a barrier)
+    uint32_t osync_phase = 0;
+    auto group_sync = [&](int c) -> bool {
+      mbar_arrive(bars + G::B_OSYNC);
+      const bool r = wait_bar_warp(sy, G::B_OSYNC, osync_phase, c);
+      osync_phase ^= 1;
+      return r;
+    };
+
+    // normaliser pieces of chunk c (before its scores): zq = z_p . qh_i, then
+    // z <- gamma^C' z + sum_j gamma^(C'-1-j) kh_j.  Loads are issued in batches.
+    auto normaliser = [&](int c, bool &ok) -> float {
+      const int s = c % NS, k = c / NS;
       const int Cp = chunk_len(c);
       ok = false;
-      if (!wait_bar(sy, G::B_AFULL + b, (c >> 1) & 1)) return 0.f;
+      if (!wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) return 0.f;
+      float zq = 0.f;
+      const uint8_t *qt = q_tile(s);
+#pragma unroll
+      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
+        const uint8_t *row = qt + kb * G::SLAB + i * 128;
+        uint4 qv[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) qv[p] = *reinterpret_cast<const uint4 *>(row + p * 16);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const float *zc = z + kb * 64 + ((p ^ (i & 7)) << 3);
+          const float4 z0 = *reinterpret_cast<const float4 *>(zc);
+          const float4 z1 = *reinterpret_cast<const float4 *>(zc + 4);
+          float f[8];
+          unpack8(qv[p], f);
+          zq = fmaf(z0.x, f[0], zq); zq = fmaf(z0.y, f[1], zq); zq = fmaf(z0.z, f[2], zq);
+          zq = fmaf(z0.w, f[3], zq); zq = fmaf(z1.x, f[4], zq); zq = fmaf(z1.y, f[5], zq);
+          zq = fmaf(z1.z, f[6], zq); zq = fmaf(z1.w, f[7], zq);
+        }
+      }
+      zq += __shfl_xor_sync(0xffffffffu, zq, 16);
+      // column sums of the decayed keys: thread ot sums 8 columns over a group of rows
+      constexpr int NCH = DK / 8;         // 8-column chunks
+      constexpr int RG = 128 / NCH;       // row groups
+      constexpr int RPG = C / RG;         // rows per group
+      const int cc = ot % NCH, rg = ot / NCH;
+      const uint8_t *kt = k_tile(s);
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = 0; r < RPG; ++r) {
+        const int j = rg * RPG + r;
+        const uint4 kv = *reinterpret_cast<const uint4 *>(kt + (cc >> 3) * G::SLAB + j * 128 +
+                                                           (((cc & 7) ^ (j & 7)) << 4));
+        float f[8];
+        unpack8(kv, f);
+        const float wj = small_gamma ? (j < Cp ? pw[Cp - 1 - j] : 0.f) : 1.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[u] = fmaf(wj, f[u], part[u]);
+      }
+      if (!group_sync(c)) return 0.f;  // every thread has read z_p
+      float *red = zred;
+      *reinterpret_cast<float4 *>(red + rg * DK + cc * 8) = make_float4(part[0], part[1], part[2], part[3]);
+      *reinterpret_cast<float4 *>(red + rg * DK + cc * 8 + 4) = make_float4(part[4], part[5], part[6], part[7]);
+      if (!group_sync(c)) return 0.f;
+      for (int col = ot; col < DK; col += 128) {
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) acc += red[r * DK + col];
+        z[col] = fmaf(pw[Cp], z[col], acc);
+      }
+      if (!group_sync(c)) return 0.f;  // z updated before the next chunk reads it
+      ok = true;
+      return zq;
+    };
+
+    // scores of chunk c -> P tile; returns this row's output factor
+    auto scores = [&](int c, bool &ok) -> float {
+      const int b = c & 1;
+      const int Cp = chunk_len(c);
+      float zq = 0.f;
+      if (NORM) {
+        zq = normaliser(c, ok);
+        if (!ok) return 0.f;
+      }
+      ok = false;
+      if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return 0.f;
       tc_fence_after();
       uint32_t r[32];
       tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, r);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bars + G::B_AEMPTY + b);
-      float zq = 0.f;
-      if (a.normalize) {
-        if (!wait_bar(sy, G::B_XFORM + s, k & 1)) return 0.f;
-        // zq = z_p . qh_i over this thread's half of d_k
-        const uint8_t *qt = q_tile(s);
-#pragma unroll 1
-        for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
-          const uint8_t *row = qt + kb * G::SLAB + i * 128;
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            float f[8];
-            unpack8(*reinterpret_cast<const uint4 *>(row + p * 16), f);
-            const int col = kb * 64 + ((p ^ (i & 7)) << 3);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) zq = fmaf(z[col + u], f[u], zq);
-          }
-        }
-        zq += __shfl_xor_sync(0xffffffffu, zq, 16);
-        named_bar_sync(1, 128);
-        // z <- gamma^C' z + sum_j gamma^(C'-1-j) kh_j
-        const uint8_t *kt = k_tile(s);
-        for (int col = ot; col < DK; col += 128) {
-          const int slab = col >> 6, lc = (col & 63) >> 3, e = col & 7;
-          float acc = 0.f;
-          for (int j = 0; j < Cp; ++j) {
-            const uint16_t bits = *reinterpret_cast<const uint16_t *>(kt + slab * G::SLAB + j * 128 +
-                                                                      ((lc ^ (j & 7)) << 4) + 2 * e);
-            const float x = __uint_as_float((uint32_t)bits << 16);
-            acc = small_gamma ? fmaf(pw[Cp - 1 - j], x, acc) : acc + x;
-          }
-          z[col] = fmaf(pw[Cp], z[col], acc);
-        }
-        named_bar_sync(1, 128);
-      }
       float f[32];
-      float rowsum = 0.f;
+      const bool row_ok = i < Cp;
+      if (!small_gamma) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = hf * 32 + e;
-        const float x = __uint_as_float(r[e]);
-        float p = 0.f;
-        if (j <= i && i < Cp) p = small_gamma ? x * pw[i - j] : x;
-        f[e] = p;
-        rowsum += p;
+        for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e <= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = hf * 32 + e;
+          f[e] = (j <= i && row_ok) ? __uint_as_float(r[e]) * pw[i - j] : 0.f;
+        }
       }
       uint8_t *prow = p_tile(b) + i * 128;
 #pragma unroll
@@ -519,12 +601,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
-      mbar_arrive(bars + G::B_PFULL + b);
-      rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
+      tc_fence_before();
+      mbar_arrive(bars + G::B_PFULL + b);  // also tells the MMA issuer that A[b] has been read
       ok = true;
-      if (i >= Cp) return 0.f;
-      if (small_gamma) return a.normalize ? 1.f / fmaf(pw[i + 1], zq, rowsum) : 1.f;
-      return a.normalize ? 1.f / fmaf(pw[Cp], zq, rowsum) : 1.f / pw[Cp - 1 - i];
+      float rowsum = 0.f;
+      if (NORM) {  // warp-wide: every lane takes part, including rows past the chunk end
+#pragma unroll
+        for (int e = 0; e < 32; ++e) rowsum += f[e];
+        rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
+      }
+      if (!row_ok) return 0.f;
+      if (!NORM) return small_gamma ? 1.f : 1.f / pw[Cp - 1 - i];
+      return 1.f / fmaf(small_gamma ? pw[i + 1] : pw[Cp], zq, rowsum);
     };
 
     // epilogue of chunk c
@@ -532,7 +620,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int Cp = chunk_len(c);
       const int ob = small_gamma ? 0 : (c & 1);
       const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
-      if (!wait_bar(sy, G::B_OFULL + ob, oph)) return false;
+      if (!wait_bar_warp(sy, G::B_OFULL + ob, oph, c)) return false;
       tc_fence_after();
       const float gi = pw[i + 1];
       uint8_t *orow = obase + 2 * ((start + (int64_t)c * C + i) * a.o_st);
@@ -569,17 +657,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       return true;
     };
 
-    // scores run one chunk ahead of the epilogue
-    bool ok = true;
-    float fac_cur = 0.f, fac_next = 0.f;
-    if (nchunks > 0) fac_cur = scores(0, ok);
-    for (int c = 0; c < nchunks && ok; ++c) {
-      if (c + 1 < nchunks) {
-        fac_next = scores(c + 1, ok);
+    // scores run one chunk ahead of the epilogue: step t does scores(t), epilogue(t-1)
+    float fac_even = 0.f, fac_odd = 0.f;
+    for (int t = 0; t <= nchunks; ++t) {
+      if (t < nchunks) {
+        bool ok = true;
+        const float f = scores(t, ok);
         if (!ok) break;
+        if (t & 1) fac_odd = f; else fac_even = f;
       }
-      if (!epilogue(c, fac_cur)) break;
-      fac_cur = fac_next;
+      if (t >= 1 && !epilogue(t - 1, ((t - 1) & 1) ? fac_odd : fac_even)) break;
     }
   }
 
@@ -627,7 +714,7 @@ bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t
   return r == CUDA_SUCCESS;
 }
 
-template <int DK, int DVT, int C, int NS>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU>
 cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why) {
   using G = Cfg<DK, DVT, C, NS>;
   CUtensorMap mq, mk, mv;
@@ -652,7 +739,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why
   const int64_t grid = a.n_seqs * a.H * (a.dv / DVT);
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  auto kern = chunk_tc_kernel<DK, DVT, C, NS>;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   kern<<<(unsigned)grid, kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mv, t);
@@ -660,6 +747,17 @@ cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why
 }
 
 }  // namespace
+
+cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_tc_error, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(where, g_tc_where, sizeof(unsigned int));
+  if (e == cudaSuccess && reset) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(zero));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tc_where, &zero, sizeof(zero));
+  }
+  return e;
+}
 
 bool tc_supported(const ChunkArgs &a) {
   if (a.dtype != LA_BF16 || a.chunk != 64 || a.dk != 128) return false;
@@ -671,7 +769,13 @@ bool tc_supported(const ChunkArgs &a) {
 size_t tc_workspace_bytes(int64_t, int64_t, int64_t, int, int, int64_t, bool, int) { return 0; }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *, size_t, cudaStream_t stream, const char **why) {
-  return launch_cfg<128, 128, 64, 3>(a, stream, why);
+  // one instantiation per (normaliser, feature map): each carries only its own code path
+  if (a.normalize) {
+    return a.phi ? launch_cfg<128, 128, 64, 3, true, true>(a, stream, why)
+                 : launch_cfg<128, 128, 64, 3, true, false>(a, stream, why);
+  }
+  return a.phi ? launch_cfg<128, 128, 64, 3, false, true>(a, stream, why)
+               : launch_cfg<128, 128, 64, 3, false, false>(a, stream, why);
 }
 
 }  // namespace la

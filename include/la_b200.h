@@ -161,6 +161,23 @@ LA_API size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64
 LA_API la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                   float *state, const la_tensor *out, int32_t phi, void *stream);
 
+/*
+ * la_device_error -- read the device-side error word of the tensor-core
+ * kernel.  Every wait inside that kernel is bounded (about two seconds); a
+ * wait that runs out makes the CTA give up, drain its asynchronous copies, free
+ * its tensor memory and return, and records the failure here instead of
+ * hanging or trapping.
+ *   flags   receives a bit set: 1 = a wait timed out, 2 = draining timed out
+ *           (0 = no failure since the last reset)
+ *   detail  receives the first failed wait: bit 31 set, chunk index << 8,
+ *           barrier index in the low 8 bits (0 if none)
+ *   reset   nonzero: clear both words after reading
+ * Synchronous: waits for all work on the current device to finish (it copies
+ * from a device symbol).  Host pointers.  Errors: LA_ERR_INVALID_ARG for NULL
+ * pointers, LA_ERR_CUDA if the copy fails.
+ */
+LA_API la_status la_device_error(uint32_t *flags, uint32_t *detail, int32_t reset);
+
 /* Static description of a status code. */
 LA_API const char *la_status_string(int32_t status);
 
