@@ -46,6 +46,25 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+# The tensor-core kernel re-splits its registers between warpgroups with
+# setmaxnreg (.dec to 120 and 152, .inc to 232), which is only valid if the
+# kernel launches with exactly this many registers per thread.
+TC_LAUNCH_REGS = 168
+
+
+def _check_tc_registers(ptxas_log: str) -> None:
+    regs, entry = [], None
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            entry = line
+        elif "Used" in line and "registers" in line and entry and "chunk_tc_kernel" in entry:
+            regs.append(int(line.split("Used")[1].split("registers")[0]))
+            entry = None
+    if not regs or any(r != TC_LAUNCH_REGS for r in regs):
+        raise RuntimeError("tensor-core kernel launch registers %s != %d: the setmaxnreg split in la_tc.cu "
+                           "must be revised" % (regs, TC_LAUNCH_REGS))
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     """Compile and link libla_b200.so if any source is newer; returns its path."""
     if not force and not _stale():
@@ -58,16 +77,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
         objs.append(obj)
         cmd = [nv, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
+        if src.endswith("la_tc.cu"):
+            cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
     failed = []
     for src, p in procs:
         out, _ = p.communicate()
+        text = out.decode(errors="replace")
         if verbose or p.returncode:
-            sys.stderr.write(out.decode(errors="replace"))
+            sys.stderr.write(text)
         if p.returncode:
             failed.append(os.path.basename(src))
+        elif src.endswith("la_tc.cu"):
+            _check_tc_registers(text)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
     tmp = LIB + ".tmp.%d" % os.getpid()

@@ -384,19 +384,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int tile = 0; tile < 2; ++tile) {  // 0: keys (phi, decay), 1: queries (phi)
           if (tile == 0 ? !need_k : !elu) continue;
           uint8_t *base = tile == 0 ? k_tile(s) : q_tile(s);
+          // vector tt + 64 m is in row tt/8 + 8 (m mod 8) of slab m / 8
+          static_assert(G::SLAB / 16 == 8 * 64, "row mapping assumes C = 64");
+          float wv[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int j = (tt >> 3) + 8 * m;
+            wv[m] = tile == 1 ? 1.f : (j < Cp ? pw[Cp - 1 - j] : 0.f);
+          }
 #pragma unroll 1
-          for (int m0 = 0; m0 < NV; m0 += 4) {
-            uint4 x[4];
-            float wv[4];
+          for (int m0 = 0; m0 < NV; m0 += 8) {  // one slab per batch; its 8 loads in flight together
+            uint4 x[8];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const int v = tt + 64 * (m0 + m);
-              x[m] = *reinterpret_cast<const uint4 *>(base + v * 16);
-              const int j = (v % (G::SLAB / 16)) >> 3;
-              wv[m] = tile == 1 ? 1.f : (j < Cp ? pw[Cp - 1 - j] : 0.f);
-            }
+            for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4 *>(base + (tt + 64 * (m0 + m)) * 16);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
+            for (int m = 0; m < 8; ++m) {
               const int off = (tt + 64 * (m0 + m)) * 16;
               float f[8];
               unpack8(x[m], f);
@@ -487,7 +489,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ================================================================ output
-    reg_alloc<168>();
+    // The kernel launches with 168 registers per thread (384 threads); the
+    // warpgroups re-split them as 104 (producer, MMA, transform), 232 (state)
+    // and 168 (output), 504 x 128 in total.  setmaxnreg.inc may only raise and
+    // .dec only lower a warp's count; the output warpgroup keeps the launch count.
     const int sp = warp & 3;
     const int ot = tid - 256;
     const int i = sp * 16 + (lane & 15);  // chunk row held by this thread
