@@ -113,6 +113,27 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(win)}
 
 
+def max_over_ranks(values, device, dist_mod=None):
+    """Element-wise maximum of a list of floats over all ranks (identity on one rank)."""
+    import torch
+
+    if dist_mod is None or not dist_mod.is_initialized() or dist_mod.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_rate(units_per_rank_per_step, steps, world, max_ms):
+    """Whole-job throughput: units every rank processed over the slowest rank's time."""
+    return units_per_rank_per_step * steps * world / (max_ms / 1e3)
+
+
+def rank_seed(rank):
+    """Each rank draws its own batch (independent sequences: weak scaling)."""
+    return rank
+
+
 def _algorithmic(w, n_seqs, tokens):
     """Bytes and flops one launch must move / perform (per rank)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -254,7 +275,7 @@ def main():
     hbm_peak, tc_peak, peak_kind = _peaks()
 
     w = WORKLOADS[args.workload]
-    x = make_inputs(w, seed=rank, device=dev)
+    x = make_inputs(w, seed=rank_seed(rank), device=dev)
     q, k, v, g, cu = x["q"], x["k"], x["v"], x["gamma"], x["cu_seqlens"]
     B, T = q.shape[:2]
     n_seqs = B if cu is None else cu.numel() - 1
@@ -297,13 +318,9 @@ def main():
     torch.cuda.synchronize()
     time.sleep(0.1)
     sampler.stop()
-    elapsed_ms = e_all0.elapsed_time(e_all1)
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    if ws > 1:
-        t = torch.tensor([elapsed_ms, launch_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, launch_ms = float(t[0]), float(t[1])
-    value = tokens * args.steps * ws / (elapsed_ms / 1e3)
+    elapsed_ms, launch_ms = max_over_ranks(
+        [e_all0.elapsed_time(e_all1), statistics.mean(a.elapsed_time(b) for a, b in evs)], dev, dist)
+    value = aggregate_rate(tokens, args.steps, ws, elapsed_ms)
     alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -359,14 +376,10 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev, dist)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = out.numel() * out.element_size() + fs.numel() * fs.element_size()
-    e2e = {"value": tokens * args.e2e_steps * ws / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e = {"value": aggregate_rate(tokens, args.e2e_steps, ws, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
     # ---- decode step (la_step), HBM-bound: achieved GB/s
