@@ -73,6 +73,14 @@ struct TcArgs {
   float *final_state;
   int64_t T;
   int H, dv, phi, normalize;
+  // Segmentation of long sequences (G = 1: none).  A sequence is split into G
+  // segments of segC chunks.  The state pass (MODE 1, Gp = G - 1 CTAs per unit)
+  // writes each segment's end state from a zero start to ws_s / ws_z; a scan
+  // turns slot g - 1 into the start state of segment g; the output pass (MODE 0,
+  // Gp = G) seeds segment g >= 1 with it.
+  int G, Gp, segC;
+  float *ws_s;  // [units][G-1][DK][DVT] (S^T rows)
+  float *ws_z;  // [units][G-1][DK]
 };
 
 template <int DK, int DVT, int C, int NS>
@@ -99,7 +107,7 @@ struct Cfg {
   // barriers
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_PFULL = 3 * NS + 2,
                        B_UFULL = 3 * NS + 4, B_UEMPTY = 3 * NS + 5, B_SBFULL = 3 * NS + 6, B_SBEMPTY = 3 * NS + 7,
-                       B_OFULL = 3 * NS + 8, B_OEMPTY = 3 * NS + 10, B_OSYNC = 3 * NS + 12, NBAR = 3 * NS + 13;
+                       B_OFULL = 3 * NS + 8, B_OEMPTY = 3 * NS + 10, B_OSYNC = 3 * NS + 12, B_ZDONE = 3 * NS + 13, NBAR = 4 * NS + 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -184,7 +192,7 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
@@ -204,9 +212,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   // ---- the unit this CTA owns
   const int NVT = a.dv / DVT;
-  const int vt = blockIdx.x % NVT;
-  const int h = (blockIdx.x / NVT) % a.H;
-  const int n = blockIdx.x / (NVT * a.H);
+  const int unit = blockIdx.x / a.Gp;  // (sequence, head, value slice)
+  const int seg = blockIdx.x % a.Gp;
+  const int vt = unit % NVT;
+  const int h = (unit / NVT) % a.H;
+  const int n = unit / (NVT * a.H);
   int64_t start, len;
   int bidx;
   if (a.cu_seqlens) {
@@ -218,19 +228,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     start = 0;
     len = a.T;
   }
+  if (a.G > 1) {  // this CTA's segment of the sequence
+    const int64_t c0 = (int64_t)seg * a.segC * C;
+    start += c0;
+    len = max((int64_t)0, min(len - c0, (int64_t)a.segC * C));
+  }
+  const bool has_init = MODE == 0 && a.G > 1 && seg > 0;  // start state from the scan
+  const bool last_seg = a.G == 1 || seg == a.G - 1;
+  const int64_t ws_slot = (int64_t)unit * (a.G - 1) + (MODE == 1 ? seg : seg - 1);
   const int nchunks = (int)((len + C - 1) / C);
   const float g = a.gamma[h];
 
   // ---- setup
   if (tid <= C) pw[tid] = decay_pow(g, tid);
-  for (int i = tid; i < DK; i += kThreads) z[i] = 0.f;
+  for (int i = tid; i < DK; i += kThreads) z[i] = (NORM && has_init) ? a.ws_z[ws_slot * DK + i] : 0.f;
   if (tid == 0) {
     for (int i = 0; i < G::NBAR; ++i) {
       uint32_t cnt = 1;
       if (i >= G::B_XFORM && i < G::B_XFORM + NS)
         cnt = 64;
       else if ((i >= G::B_PFULL && i < G::B_PFULL + 2) ||
-          i == G::B_UEMPTY || i == G::B_SBFULL || i == G::B_OSYNC ||
+          i == G::B_UEMPTY || i == G::B_SBFULL || i == G::B_OSYNC || (i >= G::B_ZDONE && i < G::B_ZDONE + NS) ||
           (i >= G::B_OEMPTY && i < G::B_OEMPTY + 2))
         cnt = 128;
       mbar_init(bars + i, cnt);
@@ -266,10 +284,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
         if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1, c)) break;
-        mbar_arrive_expect_tx(bars + G::B_FULL + s, G::STAGE_BYTES);
+        mbar_arrive_expect_tx(bars + G::B_FULL + s, MODE == 1 ? G::STAGE_BYTES - G::QK_BYTES : G::STAGE_BYTES);
         const int t0 = (int)(start + (int64_t)c * C);
         for (int kb = 0; kb < G::KB; ++kb) {
-          tma_load_4d(q_tile(s) + kb * G::SLAB, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
+          if (MODE == 0) tma_load_4d(q_tile(s) + kb * G::SLAB, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
           tma_load_4d(k_tile(s) + kb * G::SLAB, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
         }
         for (int vb = 0; vb < G::VB; ++vb)
@@ -309,8 +327,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // scores are queued before waiting for this chunk's P tile, so the score
       // step of chunk c+1 overlaps the P V product of chunk c.
       int done = 0;
-      bool ok = nchunks == 0 || issue_scores(0);
-      for (int c = 0; c < nchunks && ok; ++c) {
+      if (MODE == 1) {
+        // state pass: U = kd^T V per chunk; the stage is released once the state
+        // update (and, normalised, the output warps' column sums) have read it
+        for (int c = 0; c < nchunks; ++c) {
+          const int s = c % NS, k = c / NS;
+          if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) break;
+          if (c > 0 && !wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
+          tc_fence_after();
+          const uint64_t dv = smem_desc_sw128(smem_u32(v_tile(s)), G::SLAB, 1024);
+          const uint64_t dkd = small_gamma ? smem_desc_sw128(smem_u32(kx_tile), G::SLAB, 1024)
+                                           : smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
+#pragma unroll
+          for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+              umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
+                        dv + ((kk * 2048) >> 4), ID_M4, kk > 0);
+          }
+          umma_commit(bars + G::B_UFULL);
+          if (NORM && !wait_bar(sy, G::B_ZDONE + s, k & 1, c)) break;
+          umma_commit(bars + G::B_EMPTY + s);
+          done = c + 1;
+        }
+      }
+      const int sbo = has_init ? 1 : 0;  // an initial state adds one Sb hand-over before chunk 0
+      bool ok = MODE == 1 || nchunks == 0 || issue_scores(0);
+      for (int c = 0; c < nchunks && ok && MODE == 0; ++c) {
         const int s = c % NS, b = c & 1;
         const int ob = small_gamma ? 0 : b;
         const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
@@ -338,8 +381,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         const uint32_t o_inter = tbase + G::T_O + ob * DVT;
         const uint32_t o_intra = small_gamma ? tbase + G::T_O + DVT : o_inter;
-        if (c > 0) {
-          if (!wait_bar(sy, G::B_SBFULL, (c - 1) & 1, c)) break;
+        if (c > 0 || has_init) {
+          if (!wait_bar(sy, G::B_SBFULL, (c - 1 + sbo) & 1, c)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk) {
@@ -355,7 +398,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
           umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
-                    ((!small_gamma && c > 0) || kk > 0) ? 1u : 0u);
+                    ((!small_gamma && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
         }
         umma_commit(bars + G::B_OFULL + ob);
         umma_commit(bars + G::B_EMPTY + s);
@@ -382,7 +425,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
 #pragma unroll 1
         for (int tile = 0; tile < 2; ++tile) {  // 0: keys (phi, decay), 1: queries (phi)
-          if (tile == 0 ? !need_k : !elu) continue;
+          if (tile == 0 ? !need_k : (!elu || MODE == 1)) continue;  // no queries in the state pass
           uint8_t *base = tile == 0 ? k_tile(s) : q_tile(s);
           // vector tt + 64 m is in row tt/8 + 8 (m mod 8) of slab m / 8
           static_assert(G::SLAB / 16 == 8 * 64, "row mapping assumes C = 64");
@@ -429,9 +472,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     reg_alloc<232>();
     const int sp = warp & 3;
     float S[G::RPT];
+    if (has_init) {  // start state of this segment, from the scan (S^T rows)
+      const float *W = a.ws_s + ws_slot * DK * DVT;
 #pragma unroll
-    for (int u = 0; u < G::RPT; ++u) S[u] = 0.f;
-    float *F = a.final_state ? a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT : nullptr;
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const float4 *src = reinterpret_cast<const float4 *>(W + (mb * 128 + sp * 32 + lane) * DVT);
+#pragma unroll
+        for (int q = 0; q < DVT / 4; ++q) {
+          const float4 x = src[q];
+          S[mb * DVT + 4 * q] = x.x;
+          S[mb * DVT + 4 * q + 1] = x.y;
+          S[mb * DVT + 4 * q + 2] = x.z;
+          S[mb * DVT + 4 * q + 3] = x.w;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < G::RPT; ++u) S[u] = 0.f;
+    }
+    // bf16 operand Sb = sc * S for the next chunk's inter-chunk product
+    auto write_sb = [&](float sc) {
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
+#pragma unroll
+        for (int grp = 0; grp < DVT / 32; ++grp) {
+          uint8_t *row = sb_tile + ((grp * 32) >> 6) * G::SB_SLAB + kr * 128;
+          const int ch0 = ((grp * 32) & 63) >> 3;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float *x = &S[mb * DVT + grp * 32 + 8 * q];
+            const uint4 v = make_uint4(pack2(sc * x[0], sc * x[1]), pack2(sc * x[2], sc * x[3]),
+                                       pack2(sc * x[4], sc * x[5]), pack2(sc * x[6], sc * x[7]));
+            *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) = v;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_SBFULL);
+    };
+    const int sbo = has_init ? 1 : 0;
+    if (has_init && nchunks > 0) write_sb(small_gamma ? 1.f : pw[chunk_len(0)]);
     for (int c = 0; c < nchunks; ++c) {
       const int Cp = chunk_len(c);
       if (!wait_bar_warp(sy, G::B_UFULL, c & 1, c)) break;
@@ -453,34 +534,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       tc_fence_before();
       mbar_arrive(bars + G::B_UEMPTY);
-      if (c == nchunks - 1) break;
-      // bf16 operand for the next chunk's inter-chunk product
-      const float sc = small_gamma ? 1.f : pw[chunk_len(c + 1)];
-      if (c >= 1 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1) & 1, c)) break;
-#pragma unroll
-      for (int mb = 0; mb < G::MB; ++mb) {
-        const int kr = mb * 128 + sp * 32 + lane;  // d_k index held by this thread
-#pragma unroll
-        for (int grp = 0; grp < DVT / 32; ++grp) {
-          uint8_t *row = sb_tile + ((grp * 32) >> 6) * G::SB_SLAB + kr * 128;
-          const int ch0 = ((grp * 32) & 63) >> 3;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float *x = &S[mb * DVT + grp * 32 + 8 * q];
-            const uint4 v = make_uint4(pack2(sc * x[0], sc * x[1]), pack2(sc * x[2], sc * x[3]),
-                                       pack2(sc * x[4], sc * x[5]), pack2(sc * x[6], sc * x[7]));
-            *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) = v;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bars + G::B_SBFULL);
+      if (MODE == 1 || c == nchunks - 1) continue;
+      // the previous Sb has been read once M2 of chunk c is done
+      if (c - 1 + sbo >= 0 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1 + sbo) & 1, c)) break;
+      write_sb(small_gamma ? 1.f : pw[chunk_len(c + 1)]);
     }
-    if (F) {  // S after the last chunk (zero for an empty sequence)
+    // S after the last chunk: the segment's end state (state pass) or the final
+    // state of the sequence (zero for an empty sequence)
+    float *F = nullptr;
+    int64_t ld = a.dv;
+    if (MODE == 1) {
+      F = a.ws_s + ws_slot * DK * DVT;
+      ld = DVT;
+    } else if (a.final_state && last_seg) {
+      F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT;
+    }
+    if (F) {
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
         const int kr = mb * 128 + sp * 32 + lane;
-        float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * a.dv);
+        float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * ld);
 #pragma unroll
         for (int q = 0; q < DVT / 4; ++q)
           dst[q] = make_float4(S[mb * DVT + 4 * q], S[mb * DVT + 4 * q + 1], S[mb * DVT + 4 * q + 2],
@@ -511,7 +584,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // normaliser pieces of chunk c (before its scores): zq = z_p . qh_i, then
     // z <- gamma^C' z + sum_j gamma^(C'-1-j) kh_j.  Loads are issued in batches.
-    auto normaliser = [&](int c, bool &ok) -> float {
+    auto normaliser = [&](int c, bool &ok, bool want_zq) -> float {
       const int s = c % NS, k = c / NS;
       const int Cp = chunk_len(c);
       ok = false;
@@ -519,7 +592,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float zq = 0.f;
       const uint8_t *qt = q_tile(s);
 #pragma unroll
-      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
+      for (int kb = hf * (G::KB / 2); want_zq && kb < (hf + 1) * (G::KB / 2); ++kb) {
         const uint8_t *row = qt + kb * G::SLAB + i * 128;
         uint4 qv[8];
 #pragma unroll
@@ -577,7 +650,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int Cp = chunk_len(c);
       float zq = 0.f;
       if (NORM) {
-        zq = normaliser(c, ok);
+        zq = normaliser(c, ok, true);
         if (!ok) return 0.f;
       }
       ok = false;
@@ -662,9 +735,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       return true;
     };
 
+    if (MODE == 1) {
+      // state pass: only the normaliser's running key sum, then its end value
+      if (NORM) {
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
+          normaliser(c, ok, false);
+          if (ok) mbar_arrive(bars + G::B_ZDONE + c % NS);  // the column sums have read the stage
+        }
+        if (ok)
+          for (int col = ot; col < DK; col += 128) a.ws_z[ws_slot * DK + col] = z[col];
+      }
+    }
     // scores run one chunk ahead of the epilogue: step t does scores(t), epilogue(t-1)
     float fac_even = 0.f, fac_odd = 0.f;
-    for (int t = 0; t <= nchunks; ++t) {
+    for (int t = 0; t <= nchunks && MODE == 0; ++t) {
       if (t < nchunks) {
         bool ok = true;
         const float f = scores(t, ok);
@@ -719,8 +804,69 @@ bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t
   return r == CUDA_SUCCESS;
 }
 
+// Segmentation plan for the tensor-core path: when a dense batch has too few
+// (sequence, head, value-slice) units to fill the GPU, every sequence is split
+// into G segments of segC chunks so that units * G CTAs run in one wave.  The
+// plan depends only on the problem shape (not on the device), so the workspace
+// size a caller queries matches what the launch uses.
+constexpr int kPlanSMs = 148;         // B200 streaming multiprocessors
+constexpr int kMinSegmentChunks = 16;  // below this the two extra passes do not pay
+
+struct SegPlan {
+  int G = 1, segC = 0;
+  int64_t units = 0;
+};
+
+SegPlan seg_plan(int64_t n_seqs, int64_t T, int64_t H, int dv, bool varlen, int chunk) {
+  SegPlan p;
+  p.units = n_seqs * H * (dv / 128);
+  if (varlen || p.units <= 0 || T <= 0) return p;
+  const int64_t nch = (T + chunk - 1) / chunk;
+  int64_t G = kPlanSMs / p.units;
+  if (nch / kMinSegmentChunks < G) G = nch / kMinSegmentChunks;
+  if (G < 2) return p;
+  const int64_t segC = (nch + G - 1) / G;
+  p.G = (int)((nch + segC - 1) / segC);
+  p.segC = (int)segC;
+  if (p.G < 2) p.G = 1;
+  return p;
+}
+
+size_t seg_ws_bytes(const SegPlan &p, int dk, int dvt) {
+  if (p.G < 2) return 0;
+  return (size_t)p.units * (p.G - 1) * ((size_t)dk * dvt + dk) * sizeof(float);
+}
+
+// Segment start states from segment end states, in place: slot g-1 of a unit
+// ends up holding W_g = gamma^L W_{g-1} + E_{g-1} (W_0 = 0), L = tokens of a
+// full segment; the same recurrence runs on the normaliser sums.
+__global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *gamma, int G, int64_t seg_tokens,
+                                int H, int nvt, int elems_s, int elems_z) {
+  const int64_t unit = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= elems_s + elems_z) return;
+  const int h = (int)((unit / nvt) % H);
+  const float gL = powf(gamma[h], (float)seg_tokens);
+  float *base;
+  int64_t stride;
+  if (e < elems_s) {
+    base = ws_s + unit * (int64_t)(G - 1) * elems_s + e;
+    stride = elems_s;
+  } else {
+    if (!ws_z) return;
+    base = ws_z + unit * (int64_t)(G - 1) * elems_z + (e - elems_s);
+    stride = elems_z;
+  }
+  float w = 0.f;
+  for (int g = 1; g < G; ++g) {
+    float *slot = base + (int64_t)(g - 1) * stride;
+    w = fmaf(gL, w, *slot);
+    *slot = w;
+  }
+}
+
 template <int DK, int DVT, int C, int NS, bool NORM, bool ELU>
-cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why) {
+cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   using G = Cfg<DK, DVT, C, NS>;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, a.B, a.T, a.H, a.dk, C) || !make_map(&mk, a.k, a.B, a.T, a.H, a.dk, C) ||
@@ -741,13 +887,41 @@ cudaError_t launch_cfg(const ChunkArgs &a, cudaStream_t stream, const char **why
   t.dv = a.dv;
   t.phi = a.phi;
   t.normalize = a.normalize;
-  const int64_t grid = a.n_seqs * a.H * (a.dv / DVT);
-  if (grid == 0) return cudaSuccess;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU>;
+  const SegPlan plan = seg_plan(a.n_seqs, a.T, a.H, a.dv, a.cu_seqlens != nullptr, C);
+  const int64_t units = a.n_seqs * a.H * (a.dv / DVT);
+  if (units == 0) return cudaSuccess;
+  if (units * plan.G > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  t.G = plan.G;
+  t.segC = plan.segC;
+  t.ws_s = nullptr;
+  t.ws_z = nullptr;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  kern<<<(unsigned)grid, kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mv, t);
+  if (plan.G > 1) {
+    if (!workspace) {
+      if (why) *why = "segmented launch without workspace";
+      return cudaErrorInvalidValue;
+    }
+    t.ws_s = static_cast<float *>(workspace);
+    t.ws_z = NORM ? t.ws_s + units * (plan.G - 1) * DK * DVT : nullptr;
+    // pass 1: end state of every segment but the last, from a zero start
+    auto kst = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 1>;
+    err = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    t.Gp = plan.G - 1;
+    kst<<<(unsigned)(units * t.Gp), kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mv, t);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // scan: start states of segments 1 .. G-1
+    const int elems_s = DK * DVT, elems_z = NORM ? DK : 0;
+    dim3 sgrid((unsigned)((elems_s + elems_z + 255) / 256), (unsigned)units);
+    seg_scan_kernel<<<sgrid, 256, 0, stream>>>(t.ws_s, t.ws_z, a.gamma, plan.G, (int64_t)plan.segC * C, a.H,
+                                               a.dv / DVT, elems_s, elems_z);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  // output pass: every segment, seeded with its start state
+  t.Gp = plan.G;
+  kern<<<(unsigned)(units * plan.G), kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mv, t);
   return cudaGetLastError();
 }
 
@@ -771,16 +945,20 @@ bool tc_supported(const ChunkArgs &a) {
   return encode_fn() != nullptr;
 }
 
-size_t tc_workspace_bytes(int64_t, int64_t, int64_t, int, int, int64_t, bool, int) { return 0; }
+size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen, int chunk) {
+  (void)B;
+  if (chunk != 64 || dk != 128 || (dv != 128 && dv != 256)) return 0;  // not a tensor-core shape
+  return seg_ws_bytes(seg_plan(n_seqs, T, H, dv, varlen, chunk), dk, 128);
+}
 
-cudaError_t launch_chunk_tc(const ChunkArgs &a, void *, size_t, cudaStream_t stream, const char **why) {
+cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t, cudaStream_t stream, const char **why) {
   // one instantiation per (normaliser, feature map): each carries only its own code path
   if (a.normalize) {
-    return a.phi ? launch_cfg<128, 128, 64, 3, true, true>(a, stream, why)
-                 : launch_cfg<128, 128, 64, 3, true, false>(a, stream, why);
+    return a.phi ? launch_cfg<128, 128, 64, 3, true, true>(a, workspace, stream, why)
+                 : launch_cfg<128, 128, 64, 3, true, false>(a, workspace, stream, why);
   }
-  return a.phi ? launch_cfg<128, 128, 64, 3, false, true>(a, stream, why)
-               : launch_cfg<128, 128, 64, 3, false, false>(a, stream, why);
+  return a.phi ? launch_cfg<128, 128, 64, 3, false, true>(a, workspace, stream, why)
+               : launch_cfg<128, 128, 64, 3, false, false>(a, workspace, stream, why);
 }
 
 }  // namespace la

@@ -127,3 +127,36 @@ def test_tc_repeatable(la):
     o2, f2 = la.la_fwd_chunk(qd, kd, vd, g, phi="elu1", normalize=True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(f1, f2)
+
+
+# ---------------------------------------------------------------- segmented sequences
+@pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
+@pytest.mark.parametrize("gamma", [1.0, 0.995, 0.9, 0.0])
+def test_tc_segmented_long_sequence(la, oracle_mod, phi, normalize, gamma):
+    """Few (sequence, head) units and a long sequence: the sequence is split into
+    segments (state pass, scan, output pass) -- 79 chunks with a ragged tail."""
+    B, T, H = 1, 5000, 2
+    q, k, v = _inputs(B, T, H, 128, 128, 128 ** -0.5, seed=17)
+    need = la.workspace_size(B, T, H, 128, 128, B, False, 64)
+    assert need > 0  # this shape is segmented
+    _check(la, oracle_mod, q, k, v, torch.tensor([gamma, 0.97]), phi=phi, normalize=normalize)
+
+
+def test_tc_segmented_matches_unsegmented(la):
+    """The same sequences with and without segmentation agree (the 4-unit batch is
+    segmented, the 160-unit batch with the same first sequences is not)."""
+    dev = torch.device("cuda")
+    q, k, v = _inputs(40, 2048, 4, 128, 128, 128 ** -0.5, seed=23)
+    g = torch.tensor([0.99, 0.9, 1.0, 0.95], device=dev)
+    assert la.workspace_size(1, 2048, 4, 128, 128, 1, False, 64) > 0
+    assert la.workspace_size(40, 2048, 4, 128, 128, 40, False, 64) == 0
+    o_all, f_all = la.la_fwd_chunk(q.to(dev), k.to(dev), v.to(dev), g)
+    o_one, f_one = la.la_fwd_chunk(q[:1].to(dev), k[:1].to(dev), v[:1].to(dev), g)
+    torch.cuda.synchronize()
+    assert slice_rel_err(to_np(o_one), to_np(o_all[:1]), seq_slices(1, 2048)) < TOL[BF]
+    assert state_rel_err(to_np(f_one), to_np(f_all[:1])) < TOL[BF]
+
+
+def test_tc_device_error_word_clear(la):
+    """After every tensor-core launch above, no bounded wait timed out."""
+    assert la.device_error(reset=True) == (0, 0)
