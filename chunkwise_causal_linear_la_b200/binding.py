@@ -28,7 +28,7 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 
 # Every function include/la_b200.h declares.
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_workspace_size", "la_step", "la_status_string",
-           "la_last_error", "la_version", "la_device_error")
+           "la_last_error", "la_version", "la_device_error", "la_fwd_chunk_noalloc")
 
 
 class LaTensor(ctypes.Structure):
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.la_version.restype = i32
     lib.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32), i32]
     lib.la_device_error.restype = i32
+    lib.la_fwd_chunk_noalloc.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, i32, vp]
+    lib.la_fwd_chunk_noalloc.restype = i32
     _lib = lib
     return lib
 

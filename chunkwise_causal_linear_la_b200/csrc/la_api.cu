@@ -58,6 +58,11 @@ TensorView view(const la_tensor *t) { return TensorView{t->data, t->stride_b, t-
 
 }  // namespace
 
+la_status report_error(la_status status, const char *msg) {
+  snprintf(g_msg, sizeof g_msg, "%s", msg);
+  return status;
+}
+
 int sm_count(int device) {
   if (device < 0 || device >= kMaxDevices) return 148;
   int v = g_sm_count[device].load(std::memory_order_relaxed);

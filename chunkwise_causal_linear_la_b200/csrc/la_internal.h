@@ -40,6 +40,9 @@ struct StepArgs {
   int H, dk, dv, phi, dtype;
 };
 
+// Sets the calling thread's la_last_error() message and returns `status`.
+la_status report_error(la_status status, const char *msg);
+
 // Per-device properties, cached on first use.
 int sm_count(int device);
 int max_smem_optin(int device);

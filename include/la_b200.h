@@ -162,6 +162,36 @@ LA_API la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor
                   float *state, const la_tensor *out, int32_t phi, void *stream);
 
 /*
+ * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device
+ * memory.  (An addition of this library; the pages have no counterpart.)
+ *
+ * Some callers may not allocate: a plugin running inside a framework that owns
+ * all device memory and hands out none at execution time, or a latency-bound
+ * serving loop in which cudaMalloc could synchronise the device.  la_fwd_chunk
+ * needs scratch memory for long sequences (the segment states); this variant
+ * takes no workspace and uses instead one array of LA_NOALLOC_SCRATCH_BYTES
+ * that the library keeps in the memory of every device it is loaded on, until
+ * the process exits.  It allocates nothing and frees nothing.
+ *
+ *   Arguments, layouts, results and errors are those of la_fwd_chunk without
+ *   `workspace` / `workspace_bytes`.  LA_ERR_WORKSPACE if the problem needs more
+ *   than LA_NOALLOC_SCRATCH_BYTES of scratch (la_fwd_chunk_workspace_size tells;
+ *   every problem the current kernels segment fits).
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: all calls on a device use the same array and it keeps the previous
+ *   call's contents (nothing in it needs to start at zero).  Calls whose work
+ *   overlaps on the GPU (different streams, or several host threads on one
+ *   device) race on it: order them.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (10u << 20)
+LA_API la_status la_fwd_chunk_noalloc(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                      const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs,
+                                      int32_t chunk, int32_t phi, int32_t normalize, const la_tensor *out,
+                                      float *final_state, int32_t flags, void *stream);
+
+/*
  * la_device_error -- read the device-side error word of the tensor-core
  * kernel.  Every wait inside that kernel is bounded (about two seconds); a
  * wait that runs out makes the CTA give up, drain its asynchronous copies, free
