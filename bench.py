@@ -244,6 +244,37 @@ def _config(w, ws):
     }
 
 
+def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400):
+    """Times la_step on the decode workload: per-launch CUDA events, four state
+    batches used in turn so that each step's 67 MB state was last touched three
+    steps (~200 MB of traffic) earlier and is not served from the 126 MB L2."""
+    import torch
+
+    from chunkwise_causal_linear_la_b200.workloads import DECODE, make_decode_inputs
+
+    d = make_decode_inputs(DECODE["N"], DECODE["H"], DECODE["d_k"], DECODE["d_v"], DECODE["scale"],
+                           DECODE["state_std"], DECODE["gamma"], seed=rank, device=dev)
+    states = [d["state"]] + [d["state"].clone() for _ in range(3)]
+    st = states[0]
+    dq, dk_, dv_, dg = d["q"], d["k"], d["v"], d["gamma"]
+    do = torch.empty_like(dv_)
+    for i in range(12):
+        la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"], stream=stream)
+    torch.cuda.synchronize()
+    evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nrep)]
+    for i in range(nrep):
+        evd[i][0].record(stream)
+        la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"], stream=stream)
+        evd[i][1].record(stream)
+    torch.cuda.synchronize()
+    us = statistics.mean(a.elapsed_time(b) for a, b in evd) * 1e3
+    dbytes = 2 * st.numel() * 4 + (dq.numel() + dk_.numel() + dv_.numel() + do.numel()) * 4
+    return {"workload": DECODE["name"], "us_per_step": us, "alg_bytes": dbytes,
+            "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
+            "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "step_kernel", "launches": nrep,
+            "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -254,6 +285,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step (la_step) and print its JSON object")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -263,7 +296,7 @@ def main():
     import torch.distributed as dist
 
     import chunkwise_causal_linear_la_b200 as la
-    from chunkwise_causal_linear_la_b200.workloads import DECODE, WORKLOADS, make_decode_inputs, make_inputs
+    from chunkwise_causal_linear_la_b200.workloads import WORKLOADS, make_inputs
 
     ws, rank, local = _dist()
     if ws != args.gpus:
@@ -273,6 +306,15 @@ def main():
     if ws > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     hbm_peak, tc_peak, peak_kind = _peaks()
+    stream = torch.cuda.current_stream()
+    if args.decode_only:
+        res = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1))
+        if rank == 0:
+            print(json.dumps({"impl": "la", "decode": res, "peak_kind": peak_kind}), flush=True)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     w = WORKLOADS[args.workload]
     x = make_inputs(w, seed=rank_seed(rank), device=dev)
@@ -284,7 +326,6 @@ def main():
     fs = torch.empty((n_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
     nws = la.workspace_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, w.chunk, q.dtype)
     wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
 
     def step():
         la.la_fwd_chunk(q, k, v, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
@@ -385,30 +426,7 @@ def main():
     # ---- decode step (la_step), HBM-bound: achieved GB/s
     extra = {}
     if not args.no_extra:
-        d = make_decode_inputs(DECODE["N"], DECODE["H"], DECODE["d_k"], DECODE["d_v"], DECODE["scale"],
-                               DECODE["state_std"], DECODE["gamma"], seed=rank, device=dev)
-        # four state batches used in turn: each step's 67 MB state was last touched three
-        # steps (~200 MB of traffic) earlier, so it is not served from the 126 MB L2
-        states = [d["state"]] + [d["state"].clone() for _ in range(3)]
-        st = states[0]
-        dq, dk_, dv_, dg = d["q"], d["k"], d["v"], d["gamma"]
-        do = torch.empty_like(dv_)
-        for i in range(12):
-            la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"])
-        torch.cuda.synchronize()
-        nrep = 400
-        evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nrep)]
-        for i in range(nrep):
-            evd[i][0].record(stream)
-            la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"])
-            evd[i][1].record(stream)
-        torch.cuda.synchronize()
-        us = statistics.mean(a.elapsed_time(b) for a, b in evd) * 1e3
-        dbytes = 2 * st.numel() * 4 + (dq.numel() + dk_.numel() + dv_.numel() + do.numel()) * 4
-        extra["decode"] = {"workload": DECODE["name"], "us_per_step": us, "alg_bytes": dbytes,
-                           "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
-                           "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "step_kernel",
-                           "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
+        extra["decode"] = _decode_leg(la, dev, stream, hbm_peak, rank)
 
     # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
     cpu = None

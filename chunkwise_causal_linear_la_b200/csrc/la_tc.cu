@@ -16,15 +16,19 @@
 // so one accumulator O = qh Sb^T + P V, with Sb = gamma^C' S_p (bf16) and
 // P = tril(qh kd^T) (bf16, no per-element scaling), gives o_i = O_i / den'_i
 // when normalised and o_i = O_i / gamma^(C'-1-i) otherwise.  This needs
-// gamma^(C-1) well inside the normal range; heads with gamma^(C-1) < 2^-64
-// ("small-gamma mode") keep phi(k) undecayed for the scores, use a separate
-// decayed key tile for the state, P_ij = (qh_i.kh_j) gamma^(i-j) from a table,
-// and two accumulators O_inter = qh S_p^T and O_intra = P V combined as
-// o_i = gamma^(i+1) O_inter_i + O_intra_i.
+// gamma^(C-1) well inside the normal range.  The other form ("value-decay
+// mode") keeps phi(k) undecayed, moves the state decay onto a separate tile of
+// decayed values vd_j = gamma^(C'-1-j) v_j (U = kh^T vd), takes
+// P_ij = (qh_i.kh_j) gamma^(i-j) from a table, and uses two accumulators
+// O_inter = qh S_p^T and O_intra = P V combined as o_i = gamma^(i+1) O_inter_i +
+// O_intra_i.  It runs for heads with gamma^(C-1) < 2^-64 and always at
+// d_k = 256, where it transforms the 8 KB value slice instead of the 32 KB key
+// tile per chunk.
 //
 // One CTA owns one (sequence, head, slice of DVT value columns) and walks its
 // chunks in order; the fp32 state S^T[:, slice] lives in the registers of the
-// state warpgroup:
+// state warpgroup (d_k = 128: DVT = 128; d_k = 256: DVT = 64, so that each of
+// the 128 state threads holds 128 values either way):
 //   warp 0      TMA producer: Q, K, V chunk tiles into an NS-deep ring.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
 //   warps 2-3   transform: phi(q) and the decayed keys, in place.
@@ -34,7 +38,7 @@
 //               (row factor, cast, store) of the previous chunk.
 // Per chunk, four MMAs:
 //   M1  A = qh kd^T          (M=C, N=C,   K=d_k)     -> A[c%2]
-//   M4  U = kd^T V           (M=128 per d_k block, N=DVT, K=C)
+//   M4  U = kd^T V           (M=128 per d_k block, N=DVT, K=C)  [value decay: kh^T vd]
 //   M2  O = qh Sb^T          (M=C, N=DVT, K=d_k)     [skipped on chunk 0]
 //   M3  O += P V             (M=C, N=DVT, K=C)       -> O[c%2]
 //
@@ -63,7 +67,7 @@ using namespace sm100;
 constexpr int kThreads = 384;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about two seconds
 constexpr uint32_t kSuspendHintNs = 20000;
-constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64
+constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64: below, value-decay mode
 
 struct TcArgs {
   void *out;
@@ -97,8 +101,8 @@ struct Cfg {
   static constexpr int SB_BYTES = VB * SB_SLAB;
 
   static constexpr int OFF_STAGE = 0;
-  static constexpr int OFF_KX = NS * STAGE_BYTES;
-  static constexpr int OFF_P = OFF_KX + QK_BYTES;
+  static constexpr int OFF_VD = NS * STAGE_BYTES;  // decayed values (value-decay mode)
+  static constexpr int OFF_P = OFF_VD + V_BYTES;
   static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_Z = OFF_SB + SB_BYTES;
   static constexpr int OFF_PW = OFF_Z + DK * 4;
@@ -115,8 +119,12 @@ struct Cfg {
   // tensor memory columns
   static constexpr int T_U = 0;                // per-chunk state update: MB blocks of DVT columns
   static constexpr int T_A = MB * DVT;         // two score tiles of C columns
-  static constexpr int T_O = T_A + 2 * C;      // two output tiles of DVT columns
-  static constexpr int T_COLS_USED = T_O + 2 * DVT;
+  static constexpr int T_O = T_A + 2 * C;      // output tiles of DVT columns (below)
+  // Decayed-key mode double-buffers one accumulator per chunk: O[b] at T_O +
+  // b DVT.  Value-decay mode needs two (inter, intra); they are double-buffered
+  // too (pair b at T_O + 2 b DVT) when four tiles fit, else one pair is reused.
+  static constexpr bool VD_DB = T_O + 4 * DVT <= 512;
+  static constexpr int T_COLS_USED = T_O + (VD_DB ? 4 : 2) * DVT;
   static constexpr int T_COLS = T_COLS_USED <= 32 ? 32 : T_COLS_USED <= 64 ? 64 : T_COLS_USED <= 128 ? 128
                                 : T_COLS_USED <= 256 ? 256 : 512;
   static constexpr int RPT = MB * DVT;  // state values held per state-warpgroup thread
@@ -190,6 +198,32 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+// Transform of one [C x 64k] tile by the 64 transform threads: dst = w_row *
+// (FEAT ? phi(src) : src), bf16 in and out.  Thread tt owns the 16-byte vectors
+// tt + 64 m; vector tt + 64 m sits in row tt/8 + 8 (m mod 8) of slab m / 8, so
+// wv[m mod 8] is its row weight.  Each batch keeps one slab's 8 loads in flight.
+template <bool FEAT>
+__device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int tt, int nv, const float (&wv)[8]) {
+#pragma unroll 1
+  for (int m0 = 0; m0 < nv; m0 += 8) {
+    uint4 x[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4 *>(src + (tt + 64 * (m0 + m)) * 16);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      float f[8];
+      unpack8(x[m], f);
+      if (FEAT) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] = phi_fast(f[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] *= wv[m];
+      *reinterpret_cast<uint4 *>(dst + (tt + 64 * (m0 + m)) * 16) = pack8(f);
+    }
+  }
 }
 
 template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE>
@@ -266,13 +300,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const bool small_gamma = (g < 1.f) && (pw[C - 1] < kSmallGammaLimit);
+  const bool vd_mode = DK == 256 || ((g < 1.f) && (pw[C - 1] < kSmallGammaLimit));
+  // output accumulators of chunk c: buffer ob(c), completion parity oph(c)
+  auto out_buf = [&](int c) -> int { return (vd_mode && !G::VD_DB) ? 0 : (c & 1); };
+  auto out_phase = [&](int c) -> uint32_t { return (vd_mode && !G::VD_DB) ? (c & 1) : ((c >> 1) & 1); };
 
   auto chunk_len = [&](int c) -> int { return (int)min((int64_t)C, len - (int64_t)c * C); };
   auto q_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES; };
   auto k_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + G::QK_BYTES; };
   auto v_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + 2 * G::QK_BYTES; };
-  uint8_t *kx_tile = sm + G::OFF_KX;
+  uint8_t *vd_tile = sm + G::OFF_VD;
   uint8_t *sb_tile = sm + G::OFF_SB;
   auto p_tile = [&](int b) { return sm + G::OFF_P + b * G::P_BYTES; };
 
@@ -323,9 +360,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         m1_issued = c + 1;
         return true;
       };
-      // Issue order per chunk c: M4(c), M1(c+1), M2(c), M3(c).  The next chunk's
-      // scores are queued before waiting for this chunk's P tile, so the score
-      // step of chunk c+1 overlaps the P V product of chunk c.
+      // Issue order per chunk c with three stages: M4(c), M1(c+1), M2(c), M3(c).
+      // The next chunk's scores are queued before waiting for this chunk's P
+      // tile, so the score step of chunk c+1 overlaps the P V product of chunk c.
+      // With two stages the tiles of chunk c+1 wait for the release of chunk
+      // c-1's stage, so M1(c+1) goes last: M4(c), M2(c), M3(c), M1(c+1).
+      constexpr bool kScoresAhead = NS >= 3;
       int done = 0;
       if (MODE == 1) {
         // state pass: U = kd^T V per chunk; the stage is released once the state
@@ -335,15 +375,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) break;
           if (c > 0 && !wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
           tc_fence_after();
-          const uint64_t dv = smem_desc_sw128(smem_u32(v_tile(s)), G::SLAB, 1024);
-          const uint64_t dkd = small_gamma ? smem_desc_sw128(smem_u32(kx_tile), G::SLAB, 1024)
-                                           : smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
+          const uint64_t dvu = smem_desc_sw128(smem_u32(vd_mode ? vd_tile : v_tile(s)), G::SLAB, 1024);
+          const uint64_t dkd = smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
 #pragma unroll
           for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
               umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
-                        dv + ((kk * 2048) >> 4), ID_M4, kk > 0);
+                        dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
           }
           umma_commit(bars + G::B_UFULL);
           if (NORM && !wait_bar(sy, G::B_ZDONE + s, k & 1, c)) break;
@@ -355,32 +394,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = MODE == 1 || nchunks == 0 || issue_scores(0);
       for (int c = 0; c < nchunks && ok && MODE == 0; ++c) {
         const int s = c % NS, b = c & 1;
-        const int ob = small_gamma ? 0 : b;
-        const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
+        const int ob = out_buf(c);
+        const uint32_t oph = out_phase(c);
         const uint64_t dq = smem_desc_sw128(smem_u32(q_tile(s)), 16, 1024);
         const uint64_t dv = smem_desc_sw128(smem_u32(v_tile(s)), G::SLAB, 1024);
-        const uint64_t dkd = small_gamma ? smem_desc_sw128(smem_u32(kx_tile), G::SLAB, 1024)
-                                         : smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
-        // M4: this chunk's state update U = kd^T V
+        const uint64_t dkd = smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
+        // M4: this chunk's state update U = kd^T V (value decay: kh^T vd)
         if (c > 0) {
           if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
           tc_fence_after();
         }
+        const uint64_t dvu = smem_desc_sw128(smem_u32(vd_mode ? vd_tile : v_tile(s)), G::SLAB, 1024);
 #pragma unroll
         for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk)
             umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
-                      dv + ((kk * 2048) >> 4), ID_M4, kk > 0);
+                      dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
         }
         umma_commit(bars + G::B_UFULL);
-        // M1 of the next chunk
-        if (c + 1 < nchunks && !issue_scores(c + 1)) break;
+        // M1 of the next chunk, ahead of M2 / M3 when three stages are in flight
+        if (kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
         // M2 / M3: output accumulators
         if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1, c)) break;
         tc_fence_after();
-        const uint32_t o_inter = tbase + G::T_O + ob * DVT;
-        const uint32_t o_intra = small_gamma ? tbase + G::T_O + DVT : o_inter;
+        const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
+        const uint32_t o_intra = vd_mode ? o_inter + DVT : o_inter;
         if (c > 0 || has_init) {
           if (!wait_bar(sy, G::B_SBFULL, (c - 1 + sbo) & 1, c)) break;
           tc_fence_after();
@@ -398,11 +437,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
           umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
-                    ((!small_gamma && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+                    ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
         }
         umma_commit(bars + G::B_OFULL + ob);
         umma_commit(bars + G::B_EMPTY + s);
         done = c + 1;
+        // with two stages, chunk c+1's tiles land only after chunk c-1's stage is
+        // released: its scores follow this chunk's products instead
+        if (!kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
       for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
@@ -416,52 +458,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // vector v sits in row (v mod 8C) / 8 of its [C x 64] slab.
       const int tt = tid - 64;
       constexpr bool elu = ELU;
-      constexpr int NV = G::QK_BYTES / 16 / 64;  // vectors per thread per tile
+      constexpr int NV = G::QK_BYTES / 16 / 64;   // vectors per thread of a q or k tile
+      constexpr int NVV = G::V_BYTES / 16 / 64;   // ... of a v tile
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
         if (!wait_bar(sy, G::B_FULL + s, k & 1, c)) break;
         const int Cp = chunk_len(c);
-        if (small_gamma && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1, c)) break;  // M4(c-1) read kx
-        const bool need_k = elu || small_gamma || g != 1.f || Cp != C;
-#pragma unroll 1
-        for (int tile = 0; tile < 2; ++tile) {  // 0: keys (phi, decay), 1: queries (phi)
-          if (tile == 0 ? !need_k : (!elu || MODE == 1)) continue;  // no queries in the state pass
-          uint8_t *base = tile == 0 ? k_tile(s) : q_tile(s);
-          // vector tt + 64 m is in row tt/8 + 8 (m mod 8) of slab m / 8
-          static_assert(G::SLAB / 16 == 8 * 64, "row mapping assumes C = 64");
-          float wv[8];
+        if (vd_mode && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1, c)) break;  // M4(c-1) read vd
+        static_assert(G::SLAB / 16 == 8 * 64, "row mapping assumes C = 64");
+        // row weights of this thread's vectors: gamma^(C'-1-j), zero past the chunk end
+        auto decay_weights = [&](float (&wv)[8]) {
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             const int j = (tt >> 3) + 8 * m;
-            wv[m] = tile == 1 ? 1.f : (j < Cp ? pw[Cp - 1 - j] : 0.f);
+            wv[m] = j < Cp ? pw[Cp - 1 - j] : 0.f;
           }
+        };
+        float wv[8];
+        // keys (phi, and the decay unless small gamma, which keeps phi(k) as is),
+        // then queries (phi; the state pass loads none)
+        const bool need_k = elu || (!vd_mode && (g != 1.f || Cp != C));
 #pragma unroll 1
-          for (int m0 = 0; m0 < NV; m0 += 8) {  // one slab per batch; its 8 loads in flight together
-            uint4 x[8];
+        for (int tile = need_k ? 0 : 1; tile < ((elu && MODE == 0) ? 2 : 1); ++tile) {
+          uint8_t *t = tile == 0 ? k_tile(s) : q_tile(s);
+          if (tile == 0 && !vd_mode) {
+            decay_weights(wv);
+          } else {
 #pragma unroll
-            for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4 *>(base + (tt + 64 * (m0 + m)) * 16);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-              const int off = (tt + 64 * (m0 + m)) * 16;
-              float f[8];
-              unpack8(x[m], f);
-              if (elu) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) f[u] = phi_fast(f[u]);
-              }
-              if (tile == 0 && small_gamma) {
-                float d[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) d[u] = f[u] * wv[m];
-                *reinterpret_cast<uint4 *>(kx_tile + off) = pack8(d);
-                if (elu) *reinterpret_cast<uint4 *>(base + off) = pack8(f);
-              } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) f[u] *= wv[m];
-                *reinterpret_cast<uint4 *>(base + off) = pack8(f);
-              }
-            }
+            for (int m = 0; m < 8; ++m) wv[m] = 1.f;
           }
+          xform_tile<ELU>(t, t, tt, NV, wv);
+        }
+        // small gamma: decayed values vd for the state update
+        if (vd_mode) {
+          decay_weights(wv);
+          xform_tile<false>(v_tile(s), vd_tile, tt, NVV, wv);
         }
         fence_proxy_async_smem();
         mbar_arrive(bars + G::B_XFORM + s);
@@ -512,7 +543,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_arrive(bars + G::B_SBFULL);
     };
     const int sbo = has_init ? 1 : 0;
-    if (has_init && nchunks > 0) write_sb(small_gamma ? 1.f : pw[chunk_len(0)]);
+    if (has_init && nchunks > 0) write_sb(vd_mode ? 1.f : pw[chunk_len(0)]);
     for (int c = 0; c < nchunks; ++c) {
       const int Cp = chunk_len(c);
       if (!wait_bar_warp(sy, G::B_UFULL, c & 1, c)) break;
@@ -537,7 +568,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (MODE == 1 || c == nchunks - 1) continue;
       // the previous Sb has been read once M2 of chunk c is done
       if (c - 1 + sbo >= 0 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1 + sbo) & 1, c)) break;
-      write_sb(small_gamma ? 1.f : pw[chunk_len(c + 1)]);
+      write_sb(vd_mode ? 1.f : pw[chunk_len(c + 1)]);
     }
     // S after the last chunk: the segment's end state (state pass) or the final
     // state of the sequence (zero for an empty sequence)
@@ -624,7 +655,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                            (((cc & 7) ^ (j & 7)) << 4));
         float f[8];
         unpack8(kv, f);
-        const float wj = small_gamma ? (j < Cp ? pw[Cp - 1 - j] : 0.f) : 1.f;
+        const float wj = vd_mode ? (j < Cp ? pw[Cp - 1 - j] : 0.f) : 1.f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) part[u] = fmaf(wj, f[u], part[u]);
       }
@@ -661,7 +692,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_wait_ld();
       float f[32];
       const bool row_ok = i < Cp;
-      if (!small_gamma) {
+      if (!vd_mode) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e <= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
       } else {
@@ -689,15 +720,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
       }
       if (!row_ok) return 0.f;
-      if (!NORM) return small_gamma ? 1.f : 1.f / pw[Cp - 1 - i];
-      return 1.f / fmaf(small_gamma ? pw[i + 1] : pw[Cp], zq, rowsum);
+      if (!NORM) return vd_mode ? 1.f : 1.f / pw[Cp - 1 - i];
+      return 1.f / fmaf(vd_mode ? pw[i + 1] : pw[Cp], zq, rowsum);
     };
 
     // epilogue of chunk c
     auto epilogue = [&](int c, float fac) -> bool {
       const int Cp = chunk_len(c);
-      const int ob = small_gamma ? 0 : (c & 1);
-      const uint32_t oph = small_gamma ? (c & 1) : ((c >> 1) & 1);
+      const int ob = out_buf(c);
+      const uint32_t oph = out_phase(c);
       if (!wait_bar_warp(sy, G::B_OFULL + ob, oph, c)) return false;
       tc_fence_after();
       const float gi = pw[i + 1];
@@ -707,13 +738,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int pass = 0; pass < DVT / 64; ++pass) {
         uint32_t ra[32], re[32];
         float o[32];
-        if (small_gamma) {
-          tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + DVT + pass * 32, ra);
-          if (c > 0) tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + pass * 32, re);
+        if (vd_mode) {  // o = gamma^(i+1) O_inter + O_intra; no inter term without a prior state
+          const bool inter = c > 0 || has_init;
+          const uint32_t pair = lane_base + G::T_O + ob * 2 * DVT + pass * 32;
+          tmem_ld_16x32bx2_x32<DVT / 2>(pair + DVT, ra);
+          if (inter) tmem_ld_16x32bx2_x32<DVT / 2>(pair, re);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            o[e] = fmaf(gi, c > 0 ? __uint_as_float(re[e]) : 0.f, __uint_as_float(ra[e])) * fac;
+            o[e] = fmaf(gi, inter ? __uint_as_float(re[e]) : 0.f, __uint_as_float(ra[e])) * fac;
         } else {
           tmem_ld_16x32bx2_x32<DVT / 2>(lane_base + G::T_O + ob * DVT + pass * 32, ra);
           tmem_wait_ld();
@@ -817,9 +850,13 @@ struct SegPlan {
   int64_t units = 0;
 };
 
-SegPlan seg_plan(int64_t n_seqs, int64_t T, int64_t H, int dv, bool varlen, int chunk) {
+// Value-slice width of the tensor-core kernel for a key head dim: the state
+// warpgroup holds d_k x DVT fp32 values, 128 per thread.
+constexpr int tc_dvt(int dk) { return dk == 256 ? 64 : 128; }
+
+SegPlan seg_plan(int64_t n_seqs, int64_t T, int64_t H, int nvt, bool varlen, int chunk) {
   SegPlan p;
-  p.units = n_seqs * H * (dv / 128);
+  p.units = n_seqs * H * nvt;
   if (varlen || p.units <= 0 || T <= 0) return p;
   const int64_t nch = (T + chunk - 1) / chunk;
   int64_t G = kPlanSMs / p.units;
@@ -887,7 +924,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.dv = a.dv;
   t.phi = a.phi;
   t.normalize = a.normalize;
-  const SegPlan plan = seg_plan(a.n_seqs, a.T, a.H, a.dv, a.cu_seqlens != nullptr, C);
+  const SegPlan plan = seg_plan(a.n_seqs, a.T, a.H, a.dv / DVT, a.cu_seqlens != nullptr, C);
   const int64_t units = a.n_seqs * a.H * (a.dv / DVT);
   if (units == 0) return cudaSuccess;
   if (units * plan.G > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -939,26 +976,36 @@ cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset
 }
 
 bool tc_supported(const ChunkArgs &a) {
-  if (a.dtype != LA_BF16 || a.chunk != 64 || a.dk != 128) return false;
-  if (a.dv != 128 && a.dv != 256) return false;
+  if (a.dtype != LA_BF16 || a.chunk != 64) return false;
+  if (a.dk != 128 && a.dk != 256) return false;
+  if (a.dv < tc_dvt(a.dk) || a.dv % tc_dvt(a.dk) != 0) return false;
   if (a.T > 0x7fffffffLL || a.H > 0xffff) return false;
   return encode_fn() != nullptr;
 }
 
 size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen, int chunk) {
   (void)B;
-  if (chunk != 64 || dk != 128 || (dv != 128 && dv != 256)) return 0;  // not a tensor-core shape
-  return seg_ws_bytes(seg_plan(n_seqs, T, H, dv, varlen, chunk), dk, 128);
+  if (chunk != 64 || (dk != 128 && dk != 256) || dv < tc_dvt(dk) || dv % tc_dvt(dk) != 0)
+    return 0;  // not a tensor-core shape
+  const int dvt = tc_dvt(dk);
+  return seg_ws_bytes(seg_plan(n_seqs, T, H, dv / dvt, varlen, chunk), dk, dvt);
+}
+
+template <int DK, int DVT, int NS>
+cudaError_t launch_shape(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
+  // one instantiation per (normaliser, feature map): each carries only its own code path
+  if (a.normalize) {
+    return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true>(a, workspace, stream, why)
+                 : launch_cfg<DK, DVT, 64, NS, true, false>(a, workspace, stream, why);
+  }
+  return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true>(a, workspace, stream, why)
+               : launch_cfg<DK, DVT, 64, NS, false, false>(a, workspace, stream, why);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t, cudaStream_t stream, const char **why) {
-  // one instantiation per (normaliser, feature map): each carries only its own code path
-  if (a.normalize) {
-    return a.phi ? launch_cfg<128, 128, 64, 3, true, true>(a, workspace, stream, why)
-                 : launch_cfg<128, 128, 64, 3, true, false>(a, workspace, stream, why);
-  }
-  return a.phi ? launch_cfg<128, 128, 64, 3, false, true>(a, workspace, stream, why)
-               : launch_cfg<128, 128, 64, 3, false, false>(a, workspace, stream, why);
+  static_assert(tc_dvt(128) == 128 && tc_dvt(256) == 64, "value-slice widths");
+  if (a.dk == 256) return launch_shape<256, 64, 2>(a, workspace, stream, why);
+  return launch_shape<128, 128, 3>(a, workspace, stream, why);
 }
 
 }  // namespace la

@@ -131,7 +131,7 @@ def test_tc_repeatable(la):
 
 # ---------------------------------------------------------------- segmented sequences
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
-@pytest.mark.parametrize("gamma", [1.0, 0.995, 0.9, 0.0])
+@pytest.mark.parametrize("gamma", [1.0, 0.995, 0.9, 0.3, 0.0])
 def test_tc_segmented_long_sequence(la, oracle_mod, phi, normalize, gamma):
     """Few (sequence, head) units and a long sequence: the sequence is split into
     segments (state pass, scan, output pass) -- 79 chunks with a ragged tail."""
@@ -159,4 +159,71 @@ def test_tc_segmented_matches_unsegmented(la):
 
 def test_tc_device_error_word_clear(la):
     """After every tensor-core launch above, no bounded wait timed out."""
+    assert la.device_error(reset=True) == (0, 0)
+
+
+# ---------------------------------------------------------------- d_k = 256
+# d_k = 256 runs with 64-wide value slices (each CTA's state is 256 x 64 fp32)
+@pytest.mark.parametrize("dv", [64, 128, 256])
+@pytest.mark.parametrize("T", [1, 65, 200])
+def test_tc_dk256_shapes(la, oracle_mod, dv, T):
+    q, k, v = _inputs(2, T, 3, 256, dv, 256 ** -0.5, seed=T + dv)
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.97, 1.0, 0.3]))
+
+
+@pytest.mark.parametrize("phi,normalize", [("elu1", True), ("elu1", False), ("identity", False)])
+@pytest.mark.parametrize("gamma", [1.0, 0.96875, 0.2, 0.0])
+def test_tc_dk256_feature_maps(la, oracle_mod, phi, normalize, gamma):
+    q, k, v = _inputs(1, 333, 2, 256, 256, 256 ** -0.5, seed=11)
+    _check(la, oracle_mod, q, k, v, torch.tensor([gamma, 0.99]), phi=phi, normalize=normalize)
+
+
+def test_tc_dk256_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300])
+    q, k, v = _inputs(1, int(cu[-1]), 2, 256, 256, 256 ** -0.5, seed=13)
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.9, 1.0]), cu=cu, phi="elu1", normalize=True)
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.99, 0.1]), cu=cu)
+
+
+@pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
+def test_tc_dk256_segmented(la, oracle_mod, phi, normalize):
+    """One long sequence at d = 256: 8 (head, value-slice) units, split into segments."""
+    q, k, v = _inputs(1, 5000, 2, 256, 256, 256 ** -0.5, seed=19)
+    assert la.workspace_size(1, 5000, 2, 256, 256, 1, False, 64) > 0
+    _check(la, oracle_mod, q, k, v, torch.tensor([0.995, 0.9]), phi=phi, normalize=normalize)
+
+
+def test_tc_retnet_config_sample(la, oracle_mod):
+    """The RetNet-style workload (B=32, H=4, T=2048, d_k=d_v=256, gamma_h = 1-2^(-5-h))
+    at full size; the oracle checks the first and last (sequence, head) slices."""
+    from chunkwise_causal_linear_la_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS["retnet_d256"]
+    x = make_inputs(w, seed=0)
+    dev = torch.device("cuda")
+    out, fs = la.la_fwd_chunk(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), x["gamma"].to(dev), chunk=w.chunk,
+                              phi=w.phi, normalize=w.normalize)
+    torch.cuda.synchronize()
+    for b, h in [(0, 0), (31, 3)]:
+        qs, ks, vs = (x[n][b:b + 1, :, h:h + 1] for n in ("q", "k", "v"))
+        ref, fref = oracle_mod.recurrent(qs, ks, vs, [float(x["gamma"][h])], phi=w.phi, normalize=w.normalize)
+        assert slice_rel_err(to_np(out[b:b + 1, :, h:h + 1]), ref, seq_slices(1, 2048)) < TOL[BF]
+        assert state_rel_err(to_np(fs[b:b + 1, h:h + 1]), fref) < TOL[BF]
+
+
+def test_tc_dk256_matches_simt(la):
+    q, k, v = _inputs(2, 300, 2, 256, 256, 256 ** -0.5, seed=21)
+    dev = torch.device("cuda")
+    g = torch.tensor([0.97, 1.0], device=dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o1, f1 = la.la_fwd_chunk(qd, kd, vd, g)
+    o2, f2 = la.la_fwd_chunk(qd, kd, vd, g, flags=la.LA_FLAG_SIMT)
+    torch.cuda.synchronize()
+    assert slice_rel_err(to_np(o1), to_np(o2), seq_slices(2, 300)) < TOL[BF]
+    assert state_rel_err(to_np(f1), to_np(f2)) < TOL[BF]
+
+
+def test_tc_device_error_word_clear_after_dk256(la):
     assert la.device_error(reset=True) == (0, 0)
