@@ -104,14 +104,14 @@ struct Cfg {
   static constexpr int OFF_VD = NS * STAGE_BYTES;  // decayed values (value-decay mode)
   static constexpr int OFF_P = OFF_VD + V_BYTES;
   static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_Z = OFF_SB + SB_BYTES;
-  static constexpr int OFF_PW = OFF_Z + DK * 4;
-  static constexpr int OFF_ZRED = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;  // normaliser partial sums
-  static constexpr int OFF_BAR = OFF_ZRED + 128 * 8 * 4;
+  static constexpr int OFF_Z = OFF_SB + SB_BYTES;  // normaliser key sums z, two buffers of DK floats
+  static constexpr int OFF_KSUM = OFF_Z + 2 * DK * 4;  // per stage, per transform warp: chunk key column sums
+  static constexpr int OFF_PW = OFF_KSUM + NS * 2 * DK * 4;
+  static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
   // barriers
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_PFULL = 3 * NS + 2,
                        B_UFULL = 3 * NS + 4, B_UEMPTY = 3 * NS + 5, B_SBFULL = 3 * NS + 6, B_SBEMPTY = 3 * NS + 7,
-                       B_OFULL = 3 * NS + 8, B_OEMPTY = 3 * NS + 10, B_OSYNC = 3 * NS + 12, B_ZDONE = 3 * NS + 13, NBAR = 4 * NS + 13;
+                       B_OFULL = 3 * NS + 8, B_OEMPTY = 3 * NS + 10, B_ZFULL = 3 * NS + 12, NBAR = 3 * NS + 14;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -177,10 +177,17 @@ __device__ __forceinline__ void drain_bar(const Sync &sy, int idx, uint32_t pari
   }
 }
 
-// phi for the bf16 tensor-core operands: elu(x) + 1 with the hardware
-// exponential (__expf); its relative error (~1e-6 near 0) is far below the
-// bf16 rounding (2^-9) the operand gets right after.
-__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+// phi for the bf16 tensor-core operands: elu(x) + 1, with e^x = 2^(x log2 e)
+// on the PTX ex2.approx.ftz instruction (one multiply and one special-function
+// op; relative error ~2^-22, far below the bf16 rounding (2^-9) the operand
+// gets right after).  Branch-free: the exponential is taken for every lane (of
+// min(x, 0), so it cannot overflow) and the result is a select.
+__device__ __forceinline__ float phi_fast(float x) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fminf(x, 0.f) * kLog2e));
+  return x > 0.f ? x + 1.f : e;
+}
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -200,17 +207,24 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
-// Transform of one [C x 64k] tile by the 64 transform threads: dst = w_row *
-// (FEAT ? phi(src) : src), bf16 in and out.  Thread tt owns the 16-byte vectors
-// tt + 64 m; vector tt + 64 m sits in row tt/8 + 8 (m mod 8) of slab m / 8, so
-// wv[m mod 8] is its row weight.  Each batch keeps one slab's 8 loads in flight.
-template <bool FEAT>
-__device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int tt, int nv, const float (&wv)[8]) {
+// Transform of one [C x 64k] tile by the 64 transform threads (bf16 in and out):
+// with STORE, dst = wv[row] * (FEAT ? phi(src) : src); with SUM, also the column
+// sums sum_rows wsum[row] * (FEAT ? phi(src) : src), one fp32 [64k] row per warp
+// in ksum.  Thread tt owns the 16-byte vectors tt + 64 m; vector tt + 64 m sits
+// in row tt/8 + 8 (m mod 8) of slab m / 8 and physical 16-byte chunk tt mod 8,
+// which under the 128-byte swizzle holds the logical 8-column block
+// (tt mod 8) ^ (tt/8 mod 8) in every row this thread visits.  The four lanes of
+// a warp holding the same block are lane ^ 9, ^ 18, ^ 27, so two shuffle rounds
+// finish the warp's sums.  Each batch keeps one slab's 8 loads in flight.
+template <bool FEAT, bool STORE, bool SUM>
+__device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int tt, int nv, const float (&wv)[8],
+                                           const float (&wsum)[8], float *ksum) {
 #pragma unroll 1
   for (int m0 = 0; m0 < nv; m0 += 8) {
     uint4 x[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint4 *>(src + (tt + 64 * (m0 + m)) * 16);
+    float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       float f[8];
@@ -219,9 +233,27 @@ __device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int
 #pragma unroll
         for (int u = 0; u < 8; ++u) f[u] = phi_fast(f[u]);
       }
+      if (SUM) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] *= wv[m];
-      *reinterpret_cast<uint4 *>(dst + (tt + 64 * (m0 + m)) * 16) = pack8(f);
+        for (int u = 0; u < 8; ++u) part[u] = fmaf(wsum[m], f[u], part[u]);
+      }
+      if (STORE) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] *= wv[m];
+        *reinterpret_cast<uint4 *>(dst + (tt + 64 * (m0 + m)) * 16) = pack8(f);
+      }
+    }
+    if (SUM) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        part[u] += __shfl_xor_sync(0xffffffffu, part[u], 9);
+        part[u] += __shfl_xor_sync(0xffffffffu, part[u], 18);
+      }
+      if ((tt & 31) < 8) {
+        float *o = ksum + (m0 / 8) * 64 + (((tt & 7) ^ ((tt >> 3) & 7)) << 3);
+        *reinterpret_cast<float4 *>(o) = make_float4(part[0], part[1], part[2], part[3]);
+        *reinterpret_cast<float4 *>(o + 4) = make_float4(part[4], part[5], part[6], part[7]);
+      }
     }
   }
 }
@@ -234,8 +266,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
+  float *ksum = reinterpret_cast<float *>(sm + G::OFF_KSUM);
   float *pw = reinterpret_cast<float *>(sm + G::OFF_PW);
-  float *zred = reinterpret_cast<float *>(sm + G::OFF_ZRED);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + G::OFF_MISC + 4);
@@ -243,6 +275,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  // elu + 1: the output warps apply phi to the query tiles (they are idle most of
+  // a chunk), so the two transform warps only handle keys and values
+  constexpr bool kQByOutput = ELU && MODE == 0;
 
   // ---- the unit this CTA owns
   const int NVT = a.dv / DVT;
@@ -275,14 +310,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   // ---- setup
   if (tid <= C) pw[tid] = decay_pow(g, tid);
-  for (int i = tid; i < DK; i += kThreads) z[i] = (NORM && has_init) ? a.ws_z[ws_slot * DK + i] : 0.f;
+  // z buffer (c & 1) holds z after chunk c; buffer 1 starts with the z before chunk 0
+  for (int i = tid; i < DK; i += kThreads) z[DK + i] = (NORM && has_init) ? a.ws_z[ws_slot * DK + i] : 0.f;
   if (tid == 0) {
     for (int i = 0; i < G::NBAR; ++i) {
       uint32_t cnt = 1;
       if (i >= G::B_XFORM && i < G::B_XFORM + NS)
-        cnt = 64;
+        cnt = kQByOutput ? 64 + 128 : 64;  // transform warps (keys, values) [+ output warps (queries)]
       else if ((i >= G::B_PFULL && i < G::B_PFULL + 2) ||
-          i == G::B_UEMPTY || i == G::B_SBFULL || i == G::B_OSYNC || (i >= G::B_ZDONE && i < G::B_ZDONE + NS) ||
+          i == G::B_UEMPTY || i == G::B_SBFULL || (i >= G::B_ZFULL && i < G::B_ZFULL + 2) ||
           (i >= G::B_OEMPTY && i < G::B_OEMPTY + 2))
         cnt = 128;
       mbar_init(bars + i, cnt);
@@ -385,7 +421,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
           }
           umma_commit(bars + G::B_UFULL);
-          if (NORM && !wait_bar(sy, G::B_ZDONE + s, k & 1, c)) break;
+          // normalised: the state warps' key sums read the stage too
+          if (NORM && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;
           umma_commit(bars + G::B_EMPTY + s);
           done = c + 1;
         }
@@ -440,6 +477,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
         }
         umma_commit(bars + G::B_OFULL + ob);
+        if (NORM && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // key sums read the stage
         umma_commit(bars + G::B_EMPTY + s);
         done = c + 1;
         // with two stages, chunk c+1's tiles land only after chunk c-1's stage is
@@ -474,25 +512,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             wv[m] = j < Cp ? pw[Cp - 1 - j] : 0.f;
           }
         };
-        float wv[8];
-        // keys (phi, and the decay unless small gamma, which keeps phi(k) as is),
-        // then queries (phi; the state pass loads none)
-        const bool need_k = elu || (!vd_mode && (g != 1.f || Cp != C));
-#pragma unroll 1
-        for (int tile = need_k ? 0 : 1; tile < ((elu && MODE == 0) ? 2 : 1); ++tile) {
-          uint8_t *t = tile == 0 ? k_tile(s) : q_tile(s);
-          if (tile == 0 && !vd_mode) {
-            decay_weights(wv);
-          } else {
+        float wv[8], wsum[8];
+        // keys: phi, and the decay unless in value-decay mode (which keeps phi(k)
+        // as is); the queries are the output warps' part.  Normalised, the pass
+        // also leaves the chunk's weighted key column sums (gamma^(C'-1-j) on row
+        // j, zero past the chunk end) in ksum[s], one row per warp.
+        float *ks = ksum + (s * 2 + (tt >> 5)) * DK;
+        const bool store_k = elu || (!vd_mode && (g != 1.f || Cp != C));
+        if (vd_mode) {
 #pragma unroll
-            for (int m = 0; m < 8; ++m) wv[m] = 1.f;
-          }
-          xform_tile<ELU>(t, t, tt, NV, wv);
+          for (int m = 0; m < 8; ++m) wv[m] = 1.f;
+          decay_weights(wsum);
+        } else {
+          decay_weights(wv);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) wsum[m] = wv[m];
         }
-        // small gamma: decayed values vd for the state update
+        if (store_k)
+          xform_tile<ELU, true, NORM>(k_tile(s), k_tile(s), tt, NV, wv, wsum, ks);
+        else if (NORM)
+          xform_tile<false, false, true>(k_tile(s), k_tile(s), tt, NV, wv, wsum, ks);
+        // value-decay mode: decayed values vd for the state update
         if (vd_mode) {
           decay_weights(wv);
-          xform_tile<false>(v_tile(s), vd_tile, tt, NVV, wv);
+          xform_tile<false, true, false>(v_tile(s), vd_tile, tt, NVV, wv, wv, ks);
         }
         fence_proxy_async_smem();
         mbar_arrive(bars + G::B_XFORM + s);
@@ -521,6 +564,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int u = 0; u < G::RPT; ++u) S[u] = 0.f;
     }
+    // normaliser key sums z[kr] for the rows this thread holds
+    float zr[G::MB];
+#pragma unroll
+    for (int mb = 0; mb < G::MB; ++mb)
+      zr[mb] = (NORM && has_init) ? a.ws_z[ws_slot * DK + mb * 128 + sp * 32 + lane] : 0.f;
+    // z <- gamma^C' z + (chunk c's weighted key column sums, from the transform
+    // warps), published in z buffer (c & 1) for the output warps
+    auto key_sums = [&](int c, int Cp) -> bool {
+      const int s = c % NS;
+      if (!wait_bar_warp(sy, G::B_XFORM + s, (c / NS) & 1, c)) return false;
+      const float *ks = ksum + s * 2 * DK;
+      float *zb = z + (c & 1) * DK;
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;
+        zr[mb] = fmaf(pw[Cp], zr[mb], ks[kr] + ks[DK + kr]);
+        zb[kr] = zr[mb];
+      }
+      mbar_arrive(bars + G::B_ZFULL + (c & 1));
+      return true;
+    };
     // bf16 operand Sb = sc * S for the next chunk's inter-chunk product
     auto write_sb = [&](float sc) {
 #pragma unroll
@@ -565,6 +629,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       tc_fence_before();
       mbar_arrive(bars + G::B_UEMPTY);
+      if (NORM && !key_sums(c, Cp)) break;
       if (MODE == 1 || c == nchunks - 1) continue;
       // the previous Sb has been read once M2 of chunk c is done
       if (c - 1 + sbo >= 0 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1 + sbo) & 1, c)) break;
@@ -577,6 +642,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (MODE == 1) {
       F = a.ws_s + ws_slot * DK * DVT;
       ld = DVT;
+      if (NORM) {
+#pragma unroll
+        for (int mb = 0; mb < G::MB; ++mb) a.ws_z[ws_slot * DK + mb * 128 + sp * 32 + lane] = zr[mb];
+      }
     } else if (a.final_state && last_seg) {
       F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT;
     }
@@ -598,39 +667,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // and 168 (output), 504 x 128 in total.  setmaxnreg.inc may only raise and
     // .dec only lower a warp's count; the output warpgroup keeps the launch count.
     const int sp = warp & 3;
-    const int ot = tid - 256;
     const int i = sp * 16 + (lane & 15);  // chunk row held by this thread
     const int hf = lane >> 4;             // which half of the columns
     uint8_t *obase = reinterpret_cast<uint8_t *>(a.out) +
                      2 * ((int64_t)bidx * a.o_sb + (int64_t)h * a.o_sh + vt * DVT);
 
-    // bounded barrier among the 128 output threads (an mbarrier used as a barrier)
-    uint32_t osync_phase = 0;
-    auto group_sync = [&](int c) -> bool {
-      mbar_arrive(bars + G::B_OSYNC);
-      const bool r = wait_bar_warp(sy, G::B_OSYNC, osync_phase, c);
-      osync_phase ^= 1;
-      return r;
-    };
-
-    // normaliser pieces of chunk c (before its scores): zq = z_p . qh_i, then
-    // z <- gamma^C' z + sum_j gamma^(C'-1-j) kh_j.  Loads are issued in batches.
-    auto normaliser = [&](int c, bool &ok, bool want_zq) -> float {
-      const int s = c % NS, k = c / NS;
-      const int Cp = chunk_len(c);
+    // zq = z_p . qh_i over this thread's row and column half, z_p = z before chunk c
+    // (z buffer (c - 1) & 1; for c = 0 buffer 1 holds the initial z).  The q tile
+    // is final: the score MMA of chunk c has read it.
+    auto z_dot_q = [&](int c, bool &ok) -> float {
       ok = false;
-      if (!wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) return 0.f;
+      if (c > 0 && !wait_bar_warp(sy, G::B_ZFULL + ((c - 1) & 1), ((c - 1) >> 1) & 1, c)) return 0.f;
+      const float *zp = z + ((c - 1) & 1) * DK;
+      const uint8_t *qt = q_tile(c % NS);
       float zq = 0.f;
-      const uint8_t *qt = q_tile(s);
+      // columns in logical order (8-column block p sits in 16-byte chunk p ^ (i & 7)
+      // of the row): every lane of a half-warp reads the same z values
 #pragma unroll
-      for (int kb = hf * (G::KB / 2); want_zq && kb < (hf + 1) * (G::KB / 2); ++kb) {
+      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
         const uint8_t *row = qt + kb * G::SLAB + i * 128;
         uint4 qv[8];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) qv[p] = *reinterpret_cast<const uint4 *>(row + p * 16);
+        for (int p = 0; p < 8; ++p) qv[p] = *reinterpret_cast<const uint4 *>(row + ((p ^ (i & 7)) << 4));
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          const float *zc = z + kb * 64 + ((p ^ (i & 7)) << 3);
+          const float *zc = zp + kb * 64 + p * 8;
           const float4 z0 = *reinterpret_cast<const float4 *>(zc);
           const float4 z1 = *reinterpret_cast<const float4 *>(zc + 4);
           float f[8];
@@ -641,36 +702,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       zq += __shfl_xor_sync(0xffffffffu, zq, 16);
-      // column sums of the decayed keys: thread ot sums 8 columns over a group of rows
-      constexpr int NCH = DK / 8;         // 8-column chunks
-      constexpr int RG = 128 / NCH;       // row groups
-      constexpr int RPG = C / RG;         // rows per group
-      const int cc = ot % NCH, rg = ot / NCH;
-      const uint8_t *kt = k_tile(s);
-      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int r = 0; r < RPG; ++r) {
-        const int j = rg * RPG + r;
-        const uint4 kv = *reinterpret_cast<const uint4 *>(kt + (cc >> 3) * G::SLAB + j * 128 +
-                                                           (((cc & 7) ^ (j & 7)) << 4));
-        float f[8];
-        unpack8(kv, f);
-        const float wj = vd_mode ? (j < Cp ? pw[Cp - 1 - j] : 0.f) : 1.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) part[u] = fmaf(wj, f[u], part[u]);
-      }
-      if (!group_sync(c)) return 0.f;  // every thread has read z_p
-      float *red = zred;
-      *reinterpret_cast<float4 *>(red + rg * DK + cc * 8) = make_float4(part[0], part[1], part[2], part[3]);
-      *reinterpret_cast<float4 *>(red + rg * DK + cc * 8 + 4) = make_float4(part[4], part[5], part[6], part[7]);
-      if (!group_sync(c)) return 0.f;
-      for (int col = ot; col < DK; col += 128) {
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < RG; ++r) acc += red[r * DK + col];
-        z[col] = fmaf(pw[Cp], z[col], acc);
-      }
-      if (!group_sync(c)) return 0.f;  // z updated before the next chunk reads it
       ok = true;
       return zq;
     };
@@ -679,14 +710,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto scores = [&](int c, bool &ok) -> float {
       const int b = c & 1;
       const int Cp = chunk_len(c);
-      float zq = 0.f;
-      if (NORM) {
-        zq = normaliser(c, ok, true);
-        if (!ok) return 0.f;
-      }
       ok = false;
       if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return 0.f;
       tc_fence_after();
+      float zq = 0.f;
+      if (NORM) {
+        zq = z_dot_q(c, ok);
+        if (!ok) return 0.f;
+        ok = false;
+      }
       uint32_t r[32];
       tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, r);
       tmem_wait_ld();
@@ -768,21 +800,40 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       return true;
     };
 
-    if (MODE == 1) {
-      // state pass: only the normaliser's running key sum, then its end value
-      if (NORM) {
-        bool ok = true;
-        for (int c = 0; c < nchunks && ok; ++c) {
-          normaliser(c, ok, false);
-          if (ok) mbar_arrive(bars + G::B_ZDONE + c % NS);  // the column sums have read the stage
+    // elu + 1 on chunk c's query tile: this thread's row and column half, in place
+    // (chunks in the same conflict-free order as above)
+    auto q_xform = [&](int c) -> bool {
+      const int s = c % NS;
+      if (!wait_bar_warp(sy, G::B_FULL + s, (c / NS) & 1, c)) return false;
+#pragma unroll 1
+      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
+        uint8_t *row = q_tile(s) + kb * G::SLAB + i * 128;
+        uint4 x[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) x[p] = *reinterpret_cast<const uint4 *>(row + ((p ^ (i & 7)) << 4));
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          float f[8];
+          unpack8(x[p], f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = phi_fast(f[u]);
+          *reinterpret_cast<uint4 *>(row + ((p ^ (i & 7)) << 4)) = pack8(f);
         }
-        if (ok)
-          for (int col = ot; col < DK; col += 128) a.ws_z[ws_slot * DK + col] = z[col];
       }
-    }
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_XFORM + s);
+      return true;
+    };
+
     // scores run one chunk ahead of the epilogue: step t does scores(t), epilogue(t-1)
+    // and, with elu + 1, the query transform of chunk t + NS - 1 (the first NS - 1
+    // before the loop), so that the score MMA never waits for it
+    constexpr int QLA = NS - 1;
+    bool qok = true;
+    if (kQByOutput)
+      for (int c = 0; c < QLA && c < nchunks && qok; ++c) qok = q_xform(c);
     float fac_even = 0.f, fac_odd = 0.f;
-    for (int t = 0; t <= nchunks && MODE == 0; ++t) {
+    for (int t = 0; t <= nchunks && MODE == 0 && qok; ++t) {
       if (t < nchunks) {
         bool ok = true;
         const float f = scores(t, ok);
@@ -790,6 +841,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (t & 1) fac_odd = f; else fac_even = f;
       }
       if (t >= 1 && !epilogue(t - 1, ((t - 1) & 1) ? fac_odd : fac_even)) break;
+      if (kQByOutput && t + QLA < nchunks && !q_xform(t + QLA)) break;
     }
   }
 
