@@ -116,10 +116,14 @@ typedef struct {
  *               Its contents need not be initialised and are undefined after.
  *   stream      cudaStream_t as void*.
  *
+ * Kernels: bf16 with chunk 64 and d_k = 128 (d_v = 128 or 256) or d_k = 256
+ * (d_v = 64, 128 or 256) runs on the tensor cores; every other valid shape,
+ * f32, and LA_FLAG_SIMT run on the CUDA-core kernel.
+ *
  * Arithmetic: bf16 inputs are read as bf16, phi is evaluated in fp32 and the
- * tensor-core operands (phi(q), phi(k), decayed phi(k), the masked score tile
- * and the carried state) are rounded to bf16; all accumulation, the carried
- * state and the normaliser are fp32; `out` is rounded to its dtype once.
+ * tensor-core operands (phi(q), phi(k), decayed phi(k) or decayed v, the masked
+ * score tile and the carried state) are rounded to bf16; all accumulation, the
+ * carried state and the normaliser are fp32; `out` is rounded to its dtype once.
  * f32 inputs run entirely in fp32 on CUDA cores (no TF32).
  *
  * Errors: LA_ERR_INVALID_ARG for NULL required pointers, inconsistent shapes,
