@@ -246,10 +246,11 @@ def _config(w, ws):
     }
 
 
-def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400):
-    """Times la_step on the decode workload: per-launch CUDA events, four state
-    batches used in turn so that each step's 67 MB state was last touched three
-    steps (~200 MB of traffic) earlier and is not served from the 126 MB L2."""
+def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False):
+    """Times la_step (norm: la_step_norm, which also carries z) on the decode
+    workload: per-launch CUDA events, four state batches used in turn so that
+    each step's 67 MB state was last touched three steps (~200 MB of traffic)
+    earlier and is not served from the 126 MB L2."""
     import torch
 
     from chunkwise_causal_linear_la_b200.workloads import DECODE, make_decode_inputs
@@ -260,18 +261,29 @@ def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400):
     st = states[0]
     dq, dk_, dv_, dg = d["q"], d["k"], d["v"], d["gamma"]
     do = torch.empty_like(dv_)
+    phi = "elu1" if norm else DECODE["phi"]
+    zs = [torch.ones(st.shape[:3], dtype=torch.float32, device=dev) for _ in range(4)] if norm else None
+
+    def call(i):
+        if norm:
+            la.la_step_norm(dq, dk_, dv_, dg, states[i % 4], zs[i % 4], out=do, phi=phi, stream=stream)
+        else:
+            la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=phi, stream=stream)
+
     for i in range(12):
-        la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"], stream=stream)
+        call(i)
     torch.cuda.synchronize()
     evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nrep)]
     for i in range(nrep):
         evd[i][0].record(stream)
-        la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=DECODE["phi"], stream=stream)
+        call(i)
         evd[i][1].record(stream)
     torch.cuda.synchronize()
     us = statistics.mean(a.elapsed_time(b) for a, b in evd) * 1e3
     dbytes = 2 * st.numel() * 4 + (dq.numel() + dk_.numel() + dv_.numel() + do.numel()) * 4
-    return {"workload": DECODE["name"], "us_per_step": us, "alg_bytes": dbytes,
+    if norm:
+        dbytes += 2 * zs[0].numel() * 4
+    return {"workload": DECODE["name"] + ("_normalised" if norm else ""), "us_per_step": us, "alg_bytes": dbytes,
             "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
             "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "step_kernel", "launches": nrep,
             "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
@@ -311,8 +323,9 @@ def main():
     stream = torch.cuda.current_stream()
     if args.decode_only:
         res = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1))
+        resn = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1), norm=True)
         if rank == 0:
-            print(json.dumps({"impl": "la", "decode": res, "peak_kind": peak_kind}), flush=True)
+            print(json.dumps({"impl": "la", "decode": res, "decode_norm": resn, "peak_kind": peak_kind}), flush=True)
         if ws > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -429,6 +442,7 @@ def main():
     extra = {}
     if not args.no_extra:
         extra["decode"] = _decode_leg(la, dev, stream, hbm_peak, rank)
+        extra["decode_norm"] = _decode_leg(la, dev, stream, hbm_peak, rank, norm=True)
 
     # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
     cpu = None

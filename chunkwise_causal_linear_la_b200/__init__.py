@@ -7,6 +7,10 @@ this package is its Python binding:
     out, final_state = la_fwd_chunk(q, k, v, gamma, chunk=64, phi="identity")
     o = la_step(q1, k1, v1, gamma, final_state)   # decode one more token
 
+    # normalised: the prefill also hands over z
+    out, final_state, z = la_fwd_chunk_z(q, k, v, gamma, phi="elu1")
+    o = la_step_norm(q1, k1, v1, gamma, final_state, z, phi="elu1")
+
 ``workloads`` draws the seeded synthetic inputs of the standard workloads.
 """
 from .binding import (  # noqa: F401
@@ -15,7 +19,9 @@ from .binding import (  # noqa: F401
     LaError,
     device_error,
     la_fwd_chunk,
+    la_fwd_chunk_z,
     la_step,
+    la_step_norm,
     load_library,
     workspace_size,
 )

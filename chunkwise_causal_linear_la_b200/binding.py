@@ -27,8 +27,8 @@ _PHI = {"identity": LA_PHI_IDENTITY, "elu1": LA_PHI_ELU1, LA_PHI_IDENTITY: LA_PH
 _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 
 # Every function include/la_b200.h declares.
-EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_workspace_size", "la_step", "la_status_string",
-           "la_last_error", "la_version", "la_device_error", "la_fwd_chunk_noalloc")
+EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_workspace_size", "la_step", "la_step_norm",
+           "la_status_string", "la_last_error", "la_version", "la_device_error", "la_fwd_chunk_noalloc")
 
 
 class LaTensor(ctypes.Structure):
@@ -62,10 +62,14 @@ def load_library(path: str = LIB_PATH):
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.la_fwd_chunk.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, i32, vp, sz, vp]
     lib.la_fwd_chunk.restype = i32
+    lib.la_fwd_chunk_z.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, vp, i32, vp, sz, vp]
+    lib.la_fwd_chunk_z.restype = i32
     lib.la_fwd_chunk_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32, i32]
     lib.la_fwd_chunk_workspace_size.restype = sz
     lib.la_step.argtypes = [P, P, P, vp, vp, P, i32, vp]
     lib.la_step.restype = i32
+    lib.la_step_norm.argtypes = [P, P, P, vp, vp, vp, P, i32, vp]
+    lib.la_step_norm.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -120,6 +124,25 @@ def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", norm
     q, k [B,T,H,d_k], v [B,T,H,d_v] (CUDA, float32 or bfloat16); gamma float32 [H];
     cu_seqlens int32 [N+1] or None.  Returns (out, final_state or None).
     """
+    out, final_state, _ = _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, normalize, out, final_state,
+                               return_final_state, None, flags, workspace, stream)
+    return out, final_state
+
+
+def la_fwd_chunk_z(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="elu1", out=None, final_state=None,
+                   final_z=None, flags=LA_FLAG_NONE, workspace=None, stream=None):
+    """Normalised forward that also returns z after each sequence's last token
+    (see la_fwd_chunk_z in include/la_b200.h).  Returns (out, final_state, final_z)."""
+    B, T, H, dk = q.shape
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if final_z is None:
+        final_z = torch.empty((n_seqs, H, dk), dtype=torch.float32, device=q.device)
+    return _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, True, out, final_state, True, final_z, flags, workspace,
+                stream)
+
+
+def _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, normalize, out, final_state, return_final_state, final_z,
+         flags, workspace, stream):
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[3]
@@ -136,15 +159,18 @@ def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", norm
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     tq, tk, tv, to = describe(q), describe(k), describe(v), describe(out)
-    st = lib.la_fwd_chunk(
-        ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
-        None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
-        int(bool(normalize)), ctypes.byref(to), None if final_state is None else final_state.data_ptr(),
-        int(flags), None if workspace is None else workspace.data_ptr(),
-        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream),
-    )
-    _check(lib, st, "la_fwd_chunk")
-    return out, final_state
+    args = [ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
+            None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
+            int(bool(normalize)), ctypes.byref(to), None if final_state is None else final_state.data_ptr()]
+    tail = [int(flags), None if workspace is None else workspace.data_ptr(),
+            0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)]
+    if final_z is None:
+        _check(lib, lib.la_fwd_chunk(*args, *tail), "la_fwd_chunk")
+    else:
+        if final_z.dtype != torch.float32 or not final_z.is_contiguous():
+            raise TypeError("final_z must be a contiguous float32 tensor")
+        _check(lib, lib.la_fwd_chunk_z(*args, final_z.data_ptr(), *tail), "la_fwd_chunk_z")
+    return out, final_state, final_z
 
 
 def device_error(reset: bool = True):
@@ -173,4 +199,25 @@ def la_step(q, k, v, gamma, state, out=None, phi="identity", stream=None):
     st = lib.la_step(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(), state.data_ptr(),
                      ctypes.byref(to), _PHI[phi], _stream(stream))
     _check(lib, st, "la_step")
+    return o4.squeeze(1) if squeeze else o4
+
+
+def la_step_norm(q, k, v, gamma, state, z, out=None, phi="elu1", stream=None):
+    """One normalised decode token (see la_step_norm in include/la_b200.h).
+
+    As la_step, plus z float32 [N,H,d_k] updated in place; out = S phi(q) / (z . phi(q)).
+    """
+    lib = load_library()
+    squeeze = q.dim() == 3
+    q4, k4, v4 = (x.unsqueeze(1) if squeeze else x for x in (q, k, v))
+    if out is None:
+        out = torch.empty_like(v4)
+    o4 = out.unsqueeze(1) if out.dim() == 3 else out
+    for name, t in (("state", state), ("z", z)):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous float32 tensor" % name)
+    tq, tk, tv, to = describe(q4), describe(k4), describe(v4), describe(o4)
+    st = lib.la_step_norm(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
+                          state.data_ptr(), z.data_ptr(), ctypes.byref(to), _PHI[phi], _stream(stream))
+    _check(lib, st, "la_step_norm")
     return o4.squeeze(1) if squeeze else o4

@@ -130,6 +130,14 @@ la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
                        const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
                        int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,
                        void *workspace, size_t workspace_bytes, void *stream) {
+  return la_fwd_chunk_z(q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, nullptr,
+                        flags, workspace, workspace_bytes, stream);
+}
+
+la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                         const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                         int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
+                         int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
   la_status s;
   if ((s = check_tensor(q, "q")) != LA_OK) return s;
   if ((s = check_tensor(k, "k")) != LA_OK) return s;
@@ -153,6 +161,8 @@ la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
     return fail(LA_ERR_INVALID_ARG, "n_seqs must equal B when cu_seqlens is NULL");
   }
   if (((uintptr_t)final_state) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "final_state not 16-byte aligned");
+  if (((uintptr_t)final_z) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "final_z not 16-byte aligned");
+  if (final_z && !normalize) return fail(LA_ERR_INVALID_ARG, "final_z needs normalize");
   if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128)
     return fail(LA_ERR_UNSUPPORTED, "chunk %d not in {16, 32, 64, 128}", chunk);
   if (!head_dim_ok(q->D) || !head_dim_ok(v->D))
@@ -170,6 +180,7 @@ la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   a.gamma = gamma;
   a.cu_seqlens = cu_seqlens;
   a.final_state = final_state;
+  a.final_z = final_z;
   a.B = q->B;
   a.T = q->T;
   a.n_seqs = n_seqs;
@@ -200,6 +211,10 @@ la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
       err = cudaMemsetAsync(final_state, 0, (size_t)a.n_seqs * a.H * a.dk * a.dv * sizeof(float), st);
       if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     }
+    if (final_z) {
+      err = cudaMemsetAsync(final_z, 0, (size_t)a.n_seqs * a.H * a.dk * sizeof(float), st);
+      if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    }
     return ok();
   }
 
@@ -220,8 +235,14 @@ la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   return ok();
 }
 
-la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
-                  const la_tensor *out, int32_t phi, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by la_step and la_step_norm (z == NULL: no normaliser).
+la_status step_common(const char *name, const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                      const float *gamma, float *state, float *z, const la_tensor *out, int32_t phi,
+                      void *stream) {
   la_status s;
   if ((s = check_tensor(q, "q")) != LA_OK) return s;
   if ((s = check_tensor(k, "k")) != LA_OK) return s;
@@ -230,13 +251,14 @@ la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, co
   if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype)
     return fail(LA_ERR_INVALID_ARG, "q, k, v and out must share one dtype");
   if (q->T != 1 || k->T != 1 || v->T != 1 || out->T != 1)
-    return fail(LA_ERR_INVALID_ARG, "la_step takes exactly one token (T == 1)");
+    return fail(LA_ERR_INVALID_ARG, "%s takes exactly one token (T == 1)", name);
   if (k->B != q->B || v->B != q->B || out->B != q->B || k->H != q->H || v->H != q->H || out->H != q->H)
     return fail(LA_ERR_INVALID_ARG, "q, k, v, out disagree on N or H");
   if (k->D != q->D || out->D != v->D) return fail(LA_ERR_INVALID_ARG, "head dims disagree");
   if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
   if (q->B * q->H > 0 && !state) return fail(LA_ERR_INVALID_ARG, "state is NULL");
   if (((uintptr_t)state) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "state not 16-byte aligned");
+  if (((uintptr_t)z) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "z not 16-byte aligned");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
 
   StepArgs a;
@@ -248,6 +270,7 @@ la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, co
   a.o_sh = out->stride_h;
   a.gamma = gamma;
   a.state = state;
+  a.z = z;
   a.N = q->B;
   a.H = (int)q->H;
   a.dk = (int)q->D;
@@ -255,10 +278,25 @@ la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, co
   a.phi = phi;
   a.dtype = q->dtype;
   if (a.dk > 256 || a.dv > 256 || !step_supported(a))
-    return fail(LA_ERR_UNSUPPORTED, "la_step needs d_k <= 256 and d_v a power of two in [4, 256]");
+    return fail(LA_ERR_UNSUPPORTED, "%s needs d_k <= 256 and d_v a power of two in [4, 256]", name);
   cudaError_t err = launch_step(a, (cudaStream_t)stream);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "decode kernel: %s", cudaGetErrorString(err));
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
+                  const la_tensor *out, int32_t phi, void *stream) {
+  return step_common("la_step", q, k, v, gamma, state, nullptr, out, phi, stream);
+}
+
+la_status la_step_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                       float *state, float *z, const la_tensor *out, int32_t phi, void *stream) {
+  if (q && k && q->B * q->H > 0 && !z) return fail(LA_ERR_INVALID_ARG, "z is NULL");
+  return step_common("la_step_norm", q, k, v, gamma, state, z, out, phi, stream);
 }
 
 }  // extern "C"

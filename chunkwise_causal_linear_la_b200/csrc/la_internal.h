@@ -25,6 +25,7 @@ struct ChunkArgs {
   const float *gamma;
   const int32_t *cu_seqlens;  // NULL for dense batches
   float *final_state;         // NULL allowed
+  float *final_z;             // NULL allowed; only with normalize
   int64_t B, T, n_seqs;
   int H, dk, dv, chunk, phi, normalize;
   int dtype;  // la_dtype of q, k, v, out
@@ -36,6 +37,7 @@ struct StepArgs {
   int64_t o_sb, o_sh;
   const float *gamma;
   float *state;
+  float *z;  // normaliser state [N, H, d_k] (la_step_norm); NULL for la_step
   int64_t N;
   int H, dk, dv, phi, dtype;
 };

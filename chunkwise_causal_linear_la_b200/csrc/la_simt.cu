@@ -177,6 +177,10 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
     __syncthreads();
   }
 
+  if (a.final_z && v0 == 0) {  // z after the last token (kept only when normalising)
+    float *Zf = a.final_z + ((int64_t)n * a.H + h) * (int64_t)dk;
+    for (int c = tid; c < dk; c += kSimtThreads) Zf[c] = z[c];
+  }
   if (a.final_state) {
     float *F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)dk * a.dv + v0;
     for (int e = tid; e < dk * dvt; e += kSimtThreads) {

@@ -4,6 +4,9 @@
 // state and adds one outer product per token.  With the state stored as S^T
 // ([d_k][d_v], fp32) and the per-head decay gamma:
 //     S^T[c][r] <- gamma S^T[c][r] + phi(k)_c v_r,     o_r = sum_c S^T[c][r] phi(q)_c.
+// The normalised form (la_step_norm) also carries z, the running key sum of
+// the same section's displayed equation:
+//     z[c] <- gamma z[c] + phi(k)_c,     o_r /= sum_c z[c] phi(q)_c.
 // The state is read once and written once, so the kernel is bound by HBM
 // bandwidth: one CTA per (sequence, head) streams its d_k x d_v slab with
 // 16-byte loads and stores that bypass L1 and are marked for eviction first
@@ -20,7 +23,11 @@ namespace {
 constexpr int kStepThreads = 256;
 constexpr int kRowsUnroll = 8;
 
-template <typename Tin>
+// Shared memory: qh [dk], kh [dk], then (16-byte aligned) the row-group
+// partial outputs [nrg][ncg] float4, then one normaliser partial per warp.
+__host__ __device__ inline int step_red_offset(int dk) { return (2 * dk + 3) & ~3; }
+
+template <typename Tin, bool NORM>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel(StepArgs a) {
   extern __shared__ float sm[];
@@ -29,7 +36,8 @@ step_kernel(StepArgs a) {
   const int nrg = kStepThreads / ncg;   // row groups
   float *qh = sm;                       // [dk]
   float *kh = sm + dk;                  // [dk]
-  float4 *red = (float4 *)(sm + 2 * dk);  // [nrg][ncg]
+  float4 *red = (float4 *)(sm + step_red_offset(dk));  // [nrg][ncg]
+  float *zred = sm + step_red_offset(dk) + 4 * nrg * ncg;  // [kStepThreads / 32]
 
   const int64_t unit = blockIdx.x;  // n * H + h
   const int h = (int)(unit % a.H);
@@ -52,6 +60,19 @@ step_kernel(StepArgs a) {
     vr.w = to_f32<Tin>(V[4 * cg + 3]);
   }
   __syncthreads();
+
+  if (NORM) {  // z <- gamma z + kh, and this thread's share of z . qh
+    float *Z = a.z + unit * (int64_t)dk;
+    float part = 0.f;
+    for (int c = tid; c < dk; c += kStepThreads) {
+      const float zc = fmaf(g, Z[c], kh[c]);
+      Z[c] = zc;
+      part = fmaf(zc, qh[c], part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((tid & 31) == 0) zred[tid >> 5] = part;  // read after the barrier below
+  }
 
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   if (rg < nrg) {
@@ -90,6 +111,12 @@ step_kernel(StepArgs a) {
       const float4 y = red[r * ncg + tid];
       acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
     }
+    if (NORM) {
+      float den = 0.f;
+#pragma unroll
+      for (int w = 0; w < kStepThreads / 32; ++w) den += zred[w];
+      acc.x /= den; acc.y /= den; acc.z /= den; acc.w /= den;
+    }
     Tin *O = (Tin *)a.out + n * a.o_sb + h * a.o_sh + 4 * tid;
     O[0] = from_f32<Tin>(acc.x);
     O[1] = from_f32<Tin>(acc.y);
@@ -112,11 +139,20 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t stream) {
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int nrg = kStepThreads / (a.dv / 4);
-  const size_t smem = 2 * a.dk * sizeof(float) + (size_t)nrg * (a.dv / 4) * sizeof(float4);
-  if (a.dtype == LA_F32)
-    step_kernel<float><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
-  else
-    step_kernel<__nv_bfloat16><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
+  const size_t smem = step_red_offset(a.dk) * sizeof(float) + (size_t)nrg * (a.dv / 4) * sizeof(float4) +
+                      (kStepThreads / 32) * sizeof(float);
+  const bool norm = a.z != nullptr;
+  if (a.dtype == LA_F32) {
+    if (norm)
+      step_kernel<float, true><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
+    else
+      step_kernel<float, false><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
+  } else {
+    if (norm)
+      step_kernel<__nv_bfloat16, true><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
+    else
+      step_kernel<__nv_bfloat16, false><<<(unsigned)grid, kStepThreads, smem, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -75,6 +75,7 @@ struct TcArgs {
   const float *gamma;
   const int32_t *cu_seqlens;
   float *final_state;
+  float *final_z;  // NULL, or z after each sequence's last token (normalised only)
   int64_t T;
   int H, dv, phi, normalize;
   // Segmentation of long sequences (G = 1: none).  A sequence is split into G
@@ -649,6 +650,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } else if (a.final_state && last_seg) {
       F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT;
     }
+    if (MODE == 0 && NORM && a.final_z && last_seg && vt == 0) {  // z after the last token
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb)
+        a.final_z[((int64_t)n * a.H + h) * DK + mb * 128 + sp * 32 + lane] = zr[mb];
+    }
     if (F) {
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
@@ -971,6 +977,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.gamma = a.gamma;
   t.cu_seqlens = a.cu_seqlens;
   t.final_state = a.final_state;
+  t.final_z = a.final_z;
   t.T = a.T;
   t.H = a.H;
   t.dv = a.dv;

@@ -138,6 +138,25 @@ LA_API la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_t
                        size_t workspace_bytes, void *stream);
 
 /*
+ * la_fwd_chunk_z -- la_fwd_chunk that also returns the normaliser's state.
+ * "1.6 长上下文与高效注意力", section 线性注意力: the normalised output divides
+ * by z_t^T phi(q_t), where z_t = gamma z_{t-1} + phi(k_t) is carried beside S.
+ * A normalised decode (la_step_norm) continues from S and z, so a prefill that
+ * hands over to it needs z after the last token too.
+ *
+ *   final_z  NULL, or device float[n_seqs, H, d_k]: z of each sequence after
+ *            its last token (zero for a zero-length sequence).  Requires
+ *            normalize != 0 (LA_ERR_INVALID_ARG otherwise); 16-byte aligned.
+ *   Every other argument, layout, result and error is that of la_fwd_chunk,
+ *   which is this call with final_z = NULL.
+ */
+LA_API la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs,
+                                int32_t chunk, int32_t phi, int32_t normalize, const la_tensor *out,
+                                float *final_state, float *final_z, int32_t flags, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of workspace la_fwd_chunk needs for this problem: B, T, H, d_k, d_v
  * and n_seqs as they will be passed, has_cu_seqlens nonzero for a packed
  * batch.  Returns 0 when no workspace is needed and (size_t)-1 for arguments
@@ -164,6 +183,23 @@ LA_API size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64
  */
 LA_API la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                   float *state, const la_tensor *out, int32_t phi, void *stream);
+
+/*
+ * la_step_norm -- one normalised decode token per sequence: the displayed
+ * equation of "1.6 长上下文与高效注意力", section 线性注意力, applied once with
+ * the per-head decay:
+ *     z[c]      <- gamma z[c] + phi(k)_c
+ *     S^T[c][r] <- gamma S^T[c][r] + phi(k)_c v_r
+ *     o_r        = (sum_c S^T[c][r] phi(q)_c) / (sum_c z[c] phi(q)_c)
+ * (both sums after the update, as in prefill; no epsilon).
+ *   q, k, v, gamma, state, out, phi  as for la_step.
+ *   z      device float[N, H, d_k], updated in place; 16-byte aligned.  It
+ *          continues from la_fwd_chunk_z's final_z.
+ * The state and z are read and written once (fp32); HBM-bound.  Errors and
+ * supported sizes as for la_step.
+ */
+LA_API la_status la_step_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                              float *state, float *z, const la_tensor *out, int32_t phi, void *stream);
 
 /*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device

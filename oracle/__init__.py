@@ -16,6 +16,8 @@ it follows, is stated in the C file's header:
 * ``chunked``   -- the same result regrouped into chunks (a restatement used to
   pin chunk-size invariance).
 * ``step``      -- one decode token on a given state.
+* ``final_z``   -- the normaliser's key sum z after each sequence's last token.
+* ``step_norm`` -- one normalised decode token (state and z updated).
 
 Inputs may be numpy float32, float64, or bfloat16 given as raw ``uint16`` bits
 (use :func:`bf16_bits`); they are upcast to float64 exactly.
@@ -60,6 +62,10 @@ def _load():
         lib.oracle_chunked.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i64, i32, i32, dp, dp, i32]
         lib.oracle_chunked.restype = i32
         lib.oracle_step.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, i32, i32]
+        lib.oracle_final_z.argtypes = [vp, i32, i64, i64, i64, i64, dp, vp, i64, i32, dp, i32]
+        lib.oracle_final_z.restype = i32
+        lib.oracle_step_norm.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, dp, i32, i32]
+        lib.oracle_step_norm.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -178,3 +184,52 @@ def step(q, k, v, gamma, state, phi="identity", nthreads=0):
     if rc != 0:
         raise ValueError("oracle_step rejected its arguments (code %d)" % rc)
     return out, st
+
+
+def final_z(k, gamma, cu_seqlens=None, phi="identity", nthreads=0):
+    """z after the last token of each sequence: z_t = gamma z_{t-1} + phi(k_t).
+
+    k [B, T, H, d_k]; returns [N, H, d_k] float64.
+    """
+    k, dt = _as_input(k)
+    if k.ndim != 4:
+        raise ValueError("k must be [B, T, H, d_k]")
+    B, T, H, dk = k.shape
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(-1))
+    if g.size == 1 and H > 1:
+        g = np.full(H, g[0])
+    if g.size != H:
+        raise ValueError("gamma must have H entries")
+    cu, n = None, B
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n = cu.size - 1
+    z = np.zeros((n, H, dk), np.float64)
+    rc = _load().oracle_final_z(_ptr(k), dt, B, T, H, dk, _ptr(g), _ptr(cu), n, _PHI[phi], _ptr(z), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_final_z rejected its arguments (code %d)" % rc)
+    return z
+
+
+def step_norm(q, k, v, gamma, state, z, phi="identity", nthreads=0):
+    """One normalised decode token.  q,k [N,H,d_k], v [N,H,d_v], state [N,H,d_k,d_v]
+    (S^T), z [N,H,d_k].  Returns (out [N,H,d_v], new_state, new_z) in float64; the
+    inputs are not modified."""
+    q, dq = _as_input(q)
+    k, _ = _as_input(k)
+    v, _ = _as_input(v)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    zz = np.array(z, dtype=np.float64, copy=True, order="C")
+    if st.shape != (N, H, dk, dv) or zz.shape != (N, H, dk):
+        raise ValueError("state must be [N, H, d_k, d_v] and z [N, H, d_k]")
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(-1))
+    if g.size == 1 and H > 1:
+        g = np.full(H, g[0])
+    out = np.zeros((N, H, dv), np.float64)
+    rc = _load().oracle_step_norm(_ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(g), _ptr(st), _ptr(zz),
+                                  _ptr(out), _PHI[phi], int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_step_norm rejected its arguments (code %d)" % rc)
+    return out, st, zz

@@ -25,6 +25,11 @@
  *                        a chunked implementation relies on (results must not
  *                        depend on C beyond rounding).
  *   oracle_step       -- one decode token on a given state, in place.
+ *   oracle_final_z    -- the normaliser's key sum z after the last token of
+ *                        each sequence (the z a normalised decode continues
+ *                        from).
+ *   oracle_step_norm  -- one normalised decode token: S and z updated in
+ *                        place, o_t = S_t phi(q_t) / (z_t^T phi(q_t)).
  *
  * Layouts (all row-major, last dimension contiguous):
  *   q, k  [B, T, H, d_k];  v  [B, T, H, d_v];  out  [B, T, H, d_v] (double)
@@ -311,6 +316,74 @@ int oracle_step(const void *q, const void *k, const void *v, int dtype,
         o[r] += s * qc;
       }
     }
+  }
+  return 0;
+}
+
+/*
+ * z after the last token of each sequence, token by token:
+ *   z_t = gamma z_{t-1} + phi(k_t),  z_{-1} = 0.
+ *   k [B, T, H, d_k] (cu_seqlens as above);  final_z [n_seqs, H, d_k] double.
+ */
+int oracle_final_z(const void *k, int dtype, int64_t B, int64_t T, int64_t H, int64_t dk,
+                   const double *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int phi,
+                   double *final_z, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, 1, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    double *z = final_z + task * dk;
+    for (int64_t c = 0; c < dk; ++c) z[c] = 0.0;
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t base = ((start + t) * H + h) * dk;
+      for (int64_t c = 0; c < dk; ++c) z[c] = gamma[h] * z[c] + orc_phi(orc_load(k, dtype, base + c), phi);
+    }
+  }
+  return 0;
+}
+
+/*
+ * One normalised decode token (the displayed equation applied once):
+ *   z[c] <- gamma z[c] + kh_c,   S^T[c][r] <- gamma S^T[c][r] + kh_c v_r,
+ *   o_r = (sum_c S^T[c][r] qh_c) / (sum_c z[c] qh_c).
+ *   q, k [N, H, d_k]; v [N, H, d_v]; state [N, H, d_k, d_v] and z [N, H, d_k]
+ *   double, updated in place; out [N, H, d_v] double.
+ */
+int oracle_step_norm(const void *q, const void *k, const void *v, int dtype,
+                     int64_t N, int64_t H, int64_t dk, int64_t dv,
+                     const double *gamma, double *state, double *z, double *out, int phi,
+                     int nthreads) {
+  int rc = orc_check(dtype, 1, 1, H, dk, dv, NULL, 1, phi);
+  if (rc) return rc;
+  if (N < 0) return -2;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+  for (int64_t task = 0; task < N * H; ++task) {
+    const int64_t h = task % H;
+    const double g = gamma[h];
+    double *St = state + task * dk * dv;
+    double *zt = z + task * dk;
+    double *o = out + task * dv;
+    double den = 0.0;
+    for (int64_t r = 0; r < dv; ++r) o[r] = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+      const double qc = orc_phi(orc_load(q, dtype, task * dk + c), phi);
+      const double kc = orc_phi(orc_load(k, dtype, task * dk + c), phi);
+      zt[c] = g * zt[c] + kc;
+      den += zt[c] * qc;
+      for (int64_t r = 0; r < dv; ++r) {
+        const double s = g * St[c * dv + r] + kc * orc_load(v, dtype, task * dv + r);
+        St[c * dv + r] = s;
+        o[r] += s * qc;
+      }
+    }
+    for (int64_t r = 0; r < dv; ++r) o[r] /= den;
   }
   return 0;
 }

@@ -115,3 +115,24 @@ def test_validation_rejects_bad_arguments_before_any_device_call(lib):
     assert b"chunk" in lib.la_last_error() or b"head dims" in lib.la_last_error()
     null = _t(ptr=0)
     assert _call(lib, q=null) == b.LA_ERR_INVALID_ARG
+
+
+def test_normaliser_state_arguments_validated_on_host(lib):
+    """la_fwd_chunk_z needs normalize for final_z and a 16-byte aligned final_z;
+    la_step_norm needs a z pointer.  All rejected before any device call."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    q, k, v, o = _t(), _t(), _t(), _t()
+    def fz(normalize, final_z):
+        return lib.la_fwd_chunk_z(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), 0x2000, None, 1, 64, 1,
+                                  normalize, ctypes.byref(o), None, final_z, 0, None, 0, None)
+    assert fz(0, 0x4000) == b.LA_ERR_INVALID_ARG and b"normalize" in lib.la_last_error()
+    assert fz(1, 0x4004) == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()
+    one = lambda D: _t(T=1, D=D)  # noqa: E731
+    q1, k1, v1, o1 = one(64), one(64), one(64), one(64)
+    st = lib.la_step_norm(ctypes.byref(q1), ctypes.byref(k1), ctypes.byref(v1), 0x2000, 0x5000, None,
+                          ctypes.byref(o1), 1, None)
+    assert st == b.LA_ERR_INVALID_ARG and b"z" in lib.la_last_error()
+    st = lib.la_step_norm(ctypes.byref(q1), ctypes.byref(k1), ctypes.byref(v1), 0x2000, 0x5000, 0x6008,
+                          ctypes.byref(o1), 1, None)
+    assert st == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()

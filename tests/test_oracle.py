@@ -213,6 +213,51 @@ def test_prefill_then_step_equals_longer_prefill(oracle_mod):
         assert rel(st, fsT1) < TOL
 
 
+def test_final_z_closed_form_and_direct_sum(oracle_mod):
+    """z after the last token: with constant keys z_T = sum_{j<T} gamma^j phi(k);
+    for random keys it equals the direct weighted sum sum_t gamma^(T-1-t) phi(k_t)."""
+    T, dk = 37, 6
+    rng = np.random.default_rng(41)
+    kv = rng.standard_normal(dk)
+    for phi in ("identity", "elu1"):
+        for g in (1.0, 0.9, 0.0):
+            k = np.broadcast_to(kv, (1, T, 1, dk)).copy()
+            z = oracle_mod.final_z(k, [g], phi=phi)
+            w = float(T) if g == 1.0 else (1 - g ** T) / (1 - g)
+            assert rel(z[0, 0], w * phi_np(kv, phi)) < TOL
+    lengths = [9, 0, 30, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    _, k, _ = rand_qkv(1, int(cu[-1]), 2, dk, 1, seed=43)
+    gam = [0.8, 1.0]
+    for phi in ("identity", "elu1"):
+        z = oracle_mod.final_z(k, gam, cu_seqlens=cu, phi=phi)
+        for n, L in enumerate(lengths):
+            for h, g in enumerate(gam):
+                kh = phi_np(k[0, cu[n]:cu[n + 1], h], phi)
+                ref = (g ** np.arange(L - 1, -1, -1, dtype=np.float64))[:, None] * kh
+                assert rel(z[n, h], ref.sum(axis=0) if L else np.zeros(dk)) < TOL
+
+
+def test_prefill_then_normalised_step_equals_longer_prefill(oracle_mod):
+    """A normalised decode token continuing from (final state, final z) of a
+    prefill equals the normalised prefill of one more token."""
+    T, H, dk, dv = 20, 2, 8, 8
+    q, k, v = rand_qkv(3, T + 1, H, dk, dv, seed=33)
+    gam = [0.9, 1.0]
+    _, fsT = oracle_mod.recurrent(q[:, :T], k[:, :T], v[:, :T], gam, phi="elu1", normalize=True)
+    zT = oracle_mod.final_z(k[:, :T], gam, phi="elu1")
+    oT1, fsT1 = oracle_mod.recurrent(q, k, v, gam, phi="elu1", normalize=True)
+    o, st, z = oracle_mod.step_norm(q[:, T], k[:, T], v[:, T], gam, fsT, zT, phi="elu1")
+    assert rel(o, oT1[:, T]) < TOL
+    assert rel(st, fsT1) < TOL
+    assert rel(z, oracle_mod.final_z(k, gam, phi="elu1")) < TOL
+    # constant inputs: the normalised output is v exactly, from a zero start too
+    vv = v[:, 0]
+    o1, _, _ = oracle_mod.step_norm(q[:, 0], np.abs(k[:, 0]) + 0.1, vv, gam, np.zeros((3, H, dk, dv)),
+                                    np.zeros((3, H, dk)), phi="elu1")
+    assert np.max(np.abs(o1 - vv)) < 1e-13
+
+
 # ---------------------------------------------------------------- chunked form
 @pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
