@@ -18,6 +18,9 @@ it follows, is stated in the C file's header:
 * ``step``      -- one decode token on a given state.
 * ``final_z``   -- the normaliser's key sum z after each sequence's last token.
 * ``step_norm`` -- one normalised decode token (state and z updated).
+* ``recurrent_gated``, ``step_gated`` -- the same with a data-dependent decay
+  alpha_t = exp(g_t) per token and head (section 状态空间模型与 Mamba of the
+  same page: Mamba-2 as linear attention with a decay mask).
 
 Inputs may be numpy float32, float64, or bfloat16 given as raw ``uint16`` bits
 (use :func:`bf16_bits`); they are upcast to float64 exactly.
@@ -66,6 +69,11 @@ def _load():
         lib.oracle_final_z.restype = i32
         lib.oracle_step_norm.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, dp, i32, i32]
         lib.oracle_step_norm.restype = i32
+        lib.oracle_recurrent_gated.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, i32,
+                                               dp, dp, dp, i32]
+        lib.oracle_recurrent_gated.restype = i32
+        lib.oracle_step_gated.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, dp, i32, i32]
+        lib.oracle_step_gated.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -232,4 +240,48 @@ def step_norm(q, k, v, gamma, state, z, phi="identity", nthreads=0):
                                   _ptr(out), _PHI[phi], int(nthreads))
     if rc != 0:
         raise ValueError("oracle_step_norm rejected its arguments (code %d)" % rc)
+    return out, st, zz
+
+
+def recurrent_gated(q, k, v, g, cu_seqlens=None, phi="identity", normalize=False, nthreads=0):
+    """Token-by-token recurrence with a per-token decay exp(g[b, t, h]), g <= 0.
+
+    g [B, T, H].  Returns (out [B,T,H,d_v], final_state [N,H,d_k,d_v], final_z [N,H,d_k]) in float64.
+    """
+    q, k, v, dt, B, T, H, dk, dv, _, cu, n = _prep(q, k, v, np.ones(q.shape[2] if hasattr(q, "shape") else 1),
+                                                    cu_seqlens)
+    gg = np.ascontiguousarray(np.asarray(g, dtype=np.float64))
+    if gg.shape != (B, T, H):
+        raise ValueError("g must be [B, T, H]")
+    out = np.zeros((B, T, H, dv), np.float64)
+    fs = np.zeros((n, H, dk, dv), np.float64)
+    fz = np.zeros((n, H, dk), np.float64)
+    rc = _load().oracle_recurrent_gated(
+        _ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(gg), _ptr(cu), n,
+        _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), _ptr(fz), int(nthreads),
+    )
+    if rc != 0:
+        raise ValueError("oracle_recurrent_gated rejected its arguments (code %d)" % rc)
+    return out, fs, fz
+
+
+def step_gated(q, k, v, g, state, z=None, phi="identity", nthreads=0):
+    """One decode token with decay exp(g[n, h]).  z None: unnormalised; else normalised.
+
+    Returns (out, new_state, new_z or None) in float64; inputs are not modified."""
+    q, dq = _as_input(q)
+    k, _ = _as_input(k)
+    v, _ = _as_input(v)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    zz = None if z is None else np.array(z, dtype=np.float64, copy=True, order="C")
+    gg = np.ascontiguousarray(np.asarray(g, dtype=np.float64))
+    if st.shape != (N, H, dk, dv) or gg.shape != (N, H) or (zz is not None and zz.shape != (N, H, dk)):
+        raise ValueError("state [N,H,d_k,d_v], g [N,H], z [N,H,d_k] expected")
+    out = np.zeros((N, H, dv), np.float64)
+    rc = _load().oracle_step_gated(_ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(gg), _ptr(st), _ptr(zz),
+                                   _ptr(out), _PHI[phi], int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_step_gated rejected its arguments (code %d)" % rc)
     return out, st, zz

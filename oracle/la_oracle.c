@@ -30,6 +30,9 @@
  *                        from).
  *   oracle_step_norm  -- one normalised decode token: S and z updated in
  *                        place, o_t = S_t phi(q_t) / (z_t^T phi(q_t)).
+ *   oracle_recurrent_gated, oracle_step_gated -- the same with a per-token
+ *                        (per decode step) decay alpha_t = exp(g_t) in place
+ *                        of the per-head constant gamma.
  *
  * Layouts (all row-major, last dimension contiguous):
  *   q, k  [B, T, H, d_k];  v  [B, T, H, d_v];  out  [B, T, H, d_v] (double)
@@ -384,6 +387,117 @@ int oracle_step_norm(const void *q, const void *k, const void *v, int dtype,
       }
     }
     for (int64_t r = 0; r < dv; ++r) o[r] /= den;
+  }
+  return 0;
+}
+
+/*
+ * Data-dependent decay ("1.6 长上下文与高效注意力", section 状态空间模型与 Mamba:
+ * a state-space recurrence whose decay is a function of the input token, which
+ * Mamba-2 restricts to a scalar per step and shows to be linear attention with
+ * a decay mask).  The constant gamma of oracle_recurrent becomes a per-token,
+ * per-head factor alpha_t = exp(g_t), g_t <= 0 given in log space:
+ *     S_t = alpha_t S_{t-1} + v_t phi(k_t)^T,   z_t = alpha_t z_{t-1} + phi(k_t),
+ *     o_t = S_t phi(q_t)   [ / (z_t^T phi(q_t)) ].
+ *   g  [B, T, H] double (contiguous; packed batches as for q).
+ *   Other arguments as for oracle_recurrent; final_z [n_seqs, H, d_k] or NULL.
+ */
+int oracle_recurrent_gated(const void *q, const void *k, const void *v, int dtype,
+                           int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                           const double *g, const int32_t *cu_seqlens, int64_t n_seqs,
+                           int phi, int normalize, double *out, double *final_state,
+                           double *final_z, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (!g) return -10;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double));
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;  /* token row of the flattened [B * T] grid */
+      const double a = exp(g[row * H + h]);
+      const int64_t qk_base = (row * H + h) * dk;
+      const int64_t v_base = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk_base + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk_base + c), phi);
+      }
+      double den = 0.0;
+      for (int64_t c = 0; c < dk; ++c) {
+        z[c] = a * z[c] + kh[c];
+        den += z[c] * qh[c];
+      }
+      if (!normalize) den = 1.0;
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, v_base + r);
+        double *Sr = S + r * dk;
+        double num = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          Sr[c] = a * Sr[c] + vr * kh[c];
+          num += Sr[c] * qh[c];
+        }
+        out[v_base + r] = num / den;
+      }
+    }
+    if (final_state) {
+      double *F = final_state + task * dk * dv;
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) F[c * dv + r] = S[r * dk + c];
+    }
+    if (final_z)
+      for (int64_t c = 0; c < dk; ++c) final_z[task * dk + c] = z[c];
+    free(S);
+    free(z);
+    free(qh);
+    free(kh);
+  }
+  return 0;
+}
+
+/*
+ * One decode token with a per-(sequence, head) decay alpha = exp(g[n][h]):
+ * oracle_step (z == NULL) or oracle_step_norm (z != NULL) with gamma replaced
+ * by alpha.  g [N, H] double.
+ */
+int oracle_step_gated(const void *q, const void *k, const void *v, int dtype,
+                      int64_t N, int64_t H, int64_t dk, int64_t dv,
+                      const double *g, double *state, double *z, double *out, int phi,
+                      int nthreads) {
+  int rc = orc_check(dtype, 1, 1, H, dk, dv, NULL, 1, phi);
+  if (rc) return rc;
+  if (N < 0) return -2;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+  for (int64_t task = 0; task < N * H; ++task) {
+    const double a = exp(g[task]);
+    double *St = state + task * dk * dv;
+    double *o = out + task * dv;
+    double den = 0.0;
+    for (int64_t r = 0; r < dv; ++r) o[r] = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+      const double qc = orc_phi(orc_load(q, dtype, task * dk + c), phi);
+      const double kc = orc_phi(orc_load(k, dtype, task * dk + c), phi);
+      if (z) {
+        z[task * dk + c] = a * z[task * dk + c] + kc;
+        den += z[task * dk + c] * qc;
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        const double s = a * St[c * dv + r] + kc * orc_load(v, dtype, task * dv + r);
+        St[c * dv + r] = s;
+        o[r] += s * qc;
+      }
+    }
+    if (z)
+      for (int64_t r = 0; r < dv; ++r) o[r] /= den;
   }
   return 0;
 }

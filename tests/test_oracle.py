@@ -258,6 +258,73 @@ def test_prefill_then_normalised_step_equals_longer_prefill(oracle_mod):
     assert np.max(np.abs(o1 - vv)) < 1e-13
 
 
+# ---------------------------------------------------------------- data-dependent decay
+def gated_quadratic_form(q, k, v, g, phi, normalize):
+    """O = ((phi(Q) phi(K)^T) * M) V [/ row sums], M[i,j] = prod_{j<t<=i} exp(g_t) for i >= j
+    (the cumulative-product decay mask).  One sequence, one head."""
+    T = q.shape[0]
+    A = phi_np(q, phi) @ phi_np(k, phi).T
+    M = np.zeros((T, T))
+    for i in range(T):
+        for j in range(i + 1):
+            M[i, j] = math.exp(float(np.sum(g[j + 1:i + 1])))
+    P = A * M
+    O = P @ v
+    if normalize:
+        O = O / P.sum(axis=1, keepdims=True)
+    return O
+
+
+@pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", False), ("elu1", True)])
+def test_gated_equals_cumulative_mask_quadratic(oracle_mod, phi, normalize):
+    T, H, dk, dv = 40, 2, 6, 5
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=51)
+    g = -np.random.default_rng(52).uniform(0.0, 1.5, (1, T, H))
+    out, _, _ = oracle_mod.recurrent_gated(q, k, v, g, phi=phi, normalize=normalize)
+    for h in range(H):
+        ref = gated_quadratic_form(q[0, :, h], k[0, :, h], v[0, :, h], g[0, :, h], phi, normalize)
+        assert rel(out[0, :, h], ref) < 1e-11
+
+
+def test_gated_with_constant_gate_equals_per_head_decay(oracle_mod):
+    """g_t = log gamma_h for every token reproduces the per-head-decay oracle,
+    including the final state and z."""
+    T, H, dk, dv = 50, 3, 8, 4
+    q, k, v = rand_qkv(2, T, H, dk, dv, seed=53)
+    gam = np.array([0.9, 0.5, 1.0])
+    g = np.broadcast_to(np.log(gam), (2, T, H)).copy()
+    for phi, norm in (("identity", False), ("elu1", True)):
+        out, fs, fz = oracle_mod.recurrent_gated(q, k, v, g, phi=phi, normalize=norm)
+        ref, fref = oracle_mod.recurrent(q, k, v, gam, phi=phi, normalize=norm)
+        assert rel(out, ref) < TOL and rel(fs, fref) < TOL
+        assert rel(fz, oracle_mod.final_z(k, gam, phi=phi)) < TOL
+
+
+def test_gated_varlen_and_decode_handover(oracle_mod):
+    lengths = [7, 0, 30, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 2, 6, 6
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=55)
+    g = -np.random.default_rng(56).uniform(0.0, 0.5, (1, Tt, H))
+    out, fs, fz = oracle_mod.recurrent_gated(q, k, v, g, cu_seqlens=cu, phi="elu1", normalize=True)
+    for n, L in enumerate(lengths):
+        s_, e = cu[n], cu[n + 1]
+        o1, f1, z1 = oracle_mod.recurrent_gated(q[:, s_:e], k[:, s_:e], v[:, s_:e], g[:, s_:e], phi="elu1",
+                                                normalize=True)
+        assert np.array_equal(out[:, s_:e], o1) and np.array_equal(fs[n], f1[0]) and np.array_equal(fz[n], z1[0])
+    # prefill of T tokens + one gated decode step == prefill of T + 1 tokens
+    T = 25
+    q, k, v = rand_qkv(3, T + 1, H, dk, dv, seed=57)
+    g = -np.random.default_rng(58).uniform(0.0, 0.5, (3, T + 1, H))
+    for norm in (False, True):
+        _, fsT, fzT = oracle_mod.recurrent_gated(q[:, :T], k[:, :T], v[:, :T], g[:, :T], phi="elu1", normalize=norm)
+        oT1, fsT1, fzT1 = oracle_mod.recurrent_gated(q, k, v, g, phi="elu1", normalize=norm)
+        o, st, z = oracle_mod.step_gated(q[:, T], k[:, T], v[:, T], g[:, T], fsT, fzT if norm else None, phi="elu1")
+        assert rel(o, oT1[:, T]) < TOL and rel(st, fsT1) < TOL
+        if norm:
+            assert rel(z, fzT1) < TOL
+
+
 # ---------------------------------------------------------------- chunked form
 @pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
