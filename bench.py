@@ -138,6 +138,8 @@ def _algorithmic(w, n_seqs, tokens):
     """Bytes and flops one launch must move / perform (per rank)."""
     e = 2 if w.dtype == "bf16" else 4
     bytes_ = tokens * w.H * e * (2 * w.d_k + 2 * w.d_v) + n_seqs * w.H * w.d_k * w.d_v * 4
+    if w.gate is not None:  # the data-dependent log decay, fp32 per token and head
+        bytes_ += tokens * w.H * 4
     C = w.chunk
     flops = tokens * w.H * ((C + 1) * (w.d_k + w.d_v) + 4 * w.d_k * w.d_v)
     return bytes_, flops
@@ -169,6 +171,13 @@ def _traffic(workload_name, units_scale):
     return None
 
 
+def _oracle_run(oracle, w, q, k, v, gamma, g=None):
+    """The oracle's recurrence for workload w (per-head gamma, or the per-token log decay g)."""
+    if g is not None:
+        return oracle.recurrent_gated(q, k, v, g, phi=w.phi, normalize=w.normalize)[:2]
+    return oracle.recurrent(q, k, v, gamma, phi=w.phi, normalize=w.normalize)
+
+
 def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1):
     """Time the float64 oracle on a prefix of the first nseq sequences (all heads).
 
@@ -180,20 +189,26 @@ def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1):
     if w.varlen is not None:
         nseq = 1
     q, k, v = (t[:nseq] for t in (x["q"], x["k"], x["v"]))
+    gd = x["g"][:nseq] if "g" in x else None
     g = x["gamma"].double().cpu().numpy()
+
+    def sample(n):
+        qs, ks, vs = (t[:, :n].cpu().contiguous() for t in (q, k, v))
+        return qs, ks, vs, None if gd is None else gd[:, :n].double().cpu().numpy()
+
     # calibrate on short prefixes (the second sized to about a second), then size the sample to the budget
     n = min(T, 64)
     for target in (1.0, budget_s):
-        qs, ks, vs = (t[:, :n].cpu().contiguous() for t in (q, k, v))
+        qs, ks, vs, gs = sample(n)
         t0 = time.perf_counter()
-        oracle.recurrent(qs, ks, vs, g, phi=w.phi, normalize=w.normalize)
+        _oracle_run(oracle, w, qs, ks, vs, g, gs)
         dt = max(time.perf_counter() - t0, 1e-4)
         n = int(min(T, max(n, n * target / dt)))
     if max_tokens:
         n = min(n, max_tokens)
-    qs, ks, vs = (t[:, :n].cpu().contiguous() for t in (q, k, v))
+    qs, ks, vs, gs = sample(n)
     t0 = time.perf_counter()
-    oracle.recurrent(qs, ks, vs, g, phi=w.phi, normalize=w.normalize)
+    _oracle_run(oracle, w, qs, ks, vs, g, gs)
     secs = time.perf_counter() - t0
     return nseq * n / secs, n, secs, oracle.max_threads()
 
@@ -217,11 +232,12 @@ def run_reference(args):
     _, n, _, threads = _oracle_rate(w, x, per_step)
     q, k, v = (t[:1, :n].contiguous() for t in (x["q"], x["k"], x["v"]))
     g = x["gamma"].double().numpy()
+    gs = x["g"][:1, :n].double().numpy() if "g" in x else None
     for _ in range(args.warmup):
-        oracle.recurrent(q, k, v, g, phi=w.phi, normalize=w.normalize)
+        _oracle_run(oracle, w, q, k, v, g, gs)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.recurrent(q, k, v, g, phi=w.phi, normalize=w.normalize)
+        _oracle_run(oracle, w, q, k, v, g, gs)
     secs = time.perf_counter() - t0
     value = n * args.steps / secs
     sample = "sequence 0 of %s, all %d heads, first %d tokens per step (float64 recurrence)" % (w.name, w.H, n)
@@ -241,7 +257,8 @@ def _config(w, ws):
     return {
         "workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "B_per_gpu": w.B, "H": w.H,
         "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk, "phi": w.phi, "normalize": w.normalize,
-        "gamma": "evenly spaced in [%.3g, %.3g]" % (min(w.gamma), max(w.gamma)),
+        "gamma": ("per token: exp(g), g uniform in [ln %.3g, ln %.3g]" % w.gate) if w.gate else
+                 "evenly spaced in [%.3g, %.3g]" % (min(w.gamma), max(w.gamma)),
         "parallelism": "dp%d" % ws, "l2": "inputs larger than L2 (no flush needed)",
     }
 
@@ -342,9 +359,15 @@ def main():
     nws = la.workspace_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, w.chunk, q.dtype)
     wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
 
+    gd = x.get("g")  # data-dependent log decay (gated workloads)
+
     def step():
-        la.la_fwd_chunk(q, k, v, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
-                        out=out, final_state=fs, workspace=wsbuf, stream=stream)
+        if gd is not None:
+            la.la_fwd_chunk_gated(q, k, v, gd, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
+                                  out=out, final_state=fs, workspace=wsbuf, stream=stream)
+        else:
+            la.la_fwd_chunk(q, k, v, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
+                            out=out, final_state=fs, workspace=wsbuf, stream=stream)
 
     def barrier():
         if ws > 1:
@@ -395,13 +418,15 @@ def main():
         for b, h in sl:
             if cu is None:
                 qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
-                ref, fref = oracle.recurrent(qs, ks, vs, [float(g[h])], phi=w.phi, normalize=w.normalize)
+                gs = None if gd is None else gd[b:b + 1, :, h:h + 1].double().cpu().numpy()
+                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs)
                 o = out[b:b + 1, :, h:h + 1].float().cpu().numpy()
                 f = fs[b:b + 1, h:h + 1].cpu().numpy()
             else:
                 s, e = int(cu[0]), int(cu[1])
                 qs, ks, vs = (t[:, s:e, h:h + 1].cpu() for t in (q, k, v))
-                ref, fref = oracle.recurrent(qs, ks, vs, [float(g[h])], phi=w.phi, normalize=w.normalize)
+                gs = None if gd is None else gd[:, s:e, h:h + 1].double().cpu().numpy()
+                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs)
                 o = out[:, s:e, h:h + 1].float().cpu().numpy()
                 f = fs[0:1, h:h + 1].cpu().numpy()
             worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))),
@@ -410,14 +435,14 @@ def main():
                   "slices": "(sequence, head) = %s vs float64 oracle, full length" % sl}
 
     # ---- end to end: pinned host buffers, copies inside the timed region
-    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    inputs = (q, k, v) if gd is None else (q, k, v, gd)
+    hosts = [t.cpu().pin_memory() for t in inputs]
     oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     fh = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
 
     def e2e_step():
-        q.copy_(qh, non_blocking=True)
-        k.copy_(kh, non_blocking=True)
-        v.copy_(vh, non_blocking=True)
+        for dst, src in zip(inputs, hosts):
+            dst.copy_(src, non_blocking=True)
         step()
         oh.copy_(out, non_blocking=True)
         fh.copy_(fs, non_blocking=True)
@@ -433,7 +458,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev, dist)
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    h2d = sum(t.numel() * t.element_size() for t in inputs)
     d2h = out.numel() * out.element_size() + fs.numel() * fs.element_size()
     e2e = {"value": aggregate_rate(tokens, args.e2e_steps, ws, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}

@@ -19,8 +19,10 @@ from .binding import (  # noqa: F401
     LaError,
     device_error,
     la_fwd_chunk,
+    la_fwd_chunk_gated,
     la_fwd_chunk_z,
     la_step,
+    la_step_gated,
     la_step_norm,
     load_library,
     workspace_size,

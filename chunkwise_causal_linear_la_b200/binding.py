@@ -27,8 +27,9 @@ _PHI = {"identity": LA_PHI_IDENTITY, "elu1": LA_PHI_ELU1, LA_PHI_IDENTITY: LA_PH
 _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 
 # Every function include/la_b200.h declares.
-EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_workspace_size", "la_step", "la_step_norm",
-           "la_status_string", "la_last_error", "la_version", "la_device_error", "la_fwd_chunk_noalloc")
+EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
+           "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
+           "la_fwd_chunk_noalloc")
 
 
 class LaTensor(ctypes.Structure):
@@ -64,12 +65,16 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_chunk.restype = i32
     lib.la_fwd_chunk_z.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, vp, i32, vp, sz, vp]
     lib.la_fwd_chunk_z.restype = i32
+    lib.la_fwd_chunk_gated.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, vp, i32, vp, sz, vp]
+    lib.la_fwd_chunk_gated.restype = i32
     lib.la_fwd_chunk_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32, i32]
     lib.la_fwd_chunk_workspace_size.restype = sz
     lib.la_step.argtypes = [P, P, P, vp, vp, P, i32, vp]
     lib.la_step.restype = i32
     lib.la_step_norm.argtypes = [P, P, P, vp, vp, vp, P, i32, vp]
     lib.la_step_norm.restype = i32
+    lib.la_step_gated.argtypes = [P, P, P, vp, vp, vp, P, i32, vp]
+    lib.la_step_gated.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -129,6 +134,22 @@ def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", norm
     return out, final_state
 
 
+def la_fwd_chunk_gated(q, k, v, g, cu_seqlens=None, chunk=64, phi="identity", normalize=False, out=None,
+                       final_state=None, final_z=None, return_final_z=False, flags=LA_FLAG_NONE, workspace=None,
+                       stream=None):
+    """Forward with a data-dependent decay exp(g[b, t, h]) (see la_fwd_chunk_gated in
+    include/la_b200.h).  g float32 [B, T, H], <= 0.  Returns (out, final_state, final_z or None);
+    final_z needs normalize."""
+    B, T, H, dk = q.shape
+    if g.dtype != torch.float32 or tuple(g.shape) != (B, T, H) or not g.is_contiguous():
+        raise TypeError("g must be a contiguous float32 [B, T, H] tensor")
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if final_z is None and return_final_z:
+        final_z = torch.empty((n_seqs, H, dk), dtype=torch.float32, device=q.device)
+    return _fwd(q, k, v, None, cu_seqlens, chunk, phi, normalize, out, final_state, True, final_z, flags,
+                workspace, stream, g=g)
+
+
 def la_fwd_chunk_z(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="elu1", out=None, final_state=None,
                    final_z=None, flags=LA_FLAG_NONE, workspace=None, stream=None):
     """Normalised forward that also returns z after each sequence's last token
@@ -142,14 +163,14 @@ def la_fwd_chunk_z(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="elu1", out=No
 
 
 def _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, normalize, out, final_state, return_final_state, final_z,
-         flags, workspace, stream):
+         flags, workspace, stream, g=None):
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[3]
     n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
-    if gamma.dtype != torch.float32 or gamma.numel() != H:
+    if g is None and (gamma.dtype != torch.float32 or gamma.numel() != H):
         raise TypeError("gamma must be float32 with H entries")
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
@@ -159,17 +180,20 @@ def _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, normalize, out, final_state, re
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     tq, tk, tv, to = describe(q), describe(k), describe(v), describe(out)
-    args = [ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
+    args = [ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), (gamma if g is None else g).data_ptr(),
             None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
             int(bool(normalize)), ctypes.byref(to), None if final_state is None else final_state.data_ptr()]
     tail = [int(flags), None if workspace is None else workspace.data_ptr(),
             0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)]
-    if final_z is None:
+    fz = None if final_z is None else final_z.data_ptr()
+    if final_z is not None and (final_z.dtype != torch.float32 or not final_z.is_contiguous()):
+        raise TypeError("final_z must be a contiguous float32 tensor")
+    if g is not None:
+        _check(lib, lib.la_fwd_chunk_gated(*args, fz, *tail), "la_fwd_chunk_gated")
+    elif final_z is None:
         _check(lib, lib.la_fwd_chunk(*args, *tail), "la_fwd_chunk")
     else:
-        if final_z.dtype != torch.float32 or not final_z.is_contiguous():
-            raise TypeError("final_z must be a contiguous float32 tensor")
-        _check(lib, lib.la_fwd_chunk_z(*args, final_z.data_ptr(), *tail), "la_fwd_chunk_z")
+        _check(lib, lib.la_fwd_chunk_z(*args, fz, *tail), "la_fwd_chunk_z")
     return out, final_state, final_z
 
 
@@ -220,4 +244,25 @@ def la_step_norm(q, k, v, gamma, state, z, out=None, phi="elu1", stream=None):
     st = lib.la_step_norm(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
                           state.data_ptr(), z.data_ptr(), ctypes.byref(to), _PHI[phi], _stream(stream))
     _check(lib, st, "la_step_norm")
+    return o4.squeeze(1) if squeeze else o4
+
+
+def la_step_gated(q, k, v, g, state, z=None, out=None, phi="identity", stream=None):
+    """One decode token with decay exp(g[n, h]) (see la_step_gated in include/la_b200.h).
+
+    g float32 [N, H]; state [N,H,d_k,d_v] and, when given, z [N,H,d_k] (normalised) updated in place.
+    """
+    lib = load_library()
+    squeeze = q.dim() == 3
+    q4, k4, v4 = (x.unsqueeze(1) if squeeze else x for x in (q, k, v))
+    if out is None:
+        out = torch.empty_like(v4)
+    o4 = out.unsqueeze(1) if out.dim() == 3 else out
+    for name, t in (("state", state), ("z", z), ("g", g)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise TypeError("%s must be a contiguous float32 tensor" % name)
+    tq, tk, tv, to = describe(q4), describe(k4), describe(v4), describe(o4)
+    st = lib.la_step_gated(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), g.data_ptr(), state.data_ptr(),
+                           None if z is None else z.data_ptr(), ctypes.byref(to), _PHI[phi], _stream(stream))
+    _check(lib, st, "la_step_gated")
     return o4.squeeze(1) if squeeze else o4

@@ -88,56 +88,12 @@ int max_smem_optin(int device) {
 
 using namespace la;
 
-extern "C" {
+namespace {
 
-const char *la_status_string(int32_t status) {
-  switch (status) {
-    case LA_OK: return "LA_OK";
-    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
-    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: valid but not implemented";
-    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
-    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or launch failed";
-    default: return "unknown la_status";
-  }
-}
-
-const char *la_last_error(void) { return g_msg; }
-
-int32_t la_version(void) { return 1 * 10000 + 0 * 100 + 0; }
-
-la_status la_device_error(uint32_t *flags, uint32_t *detail, int32_t reset) {
-  if (!flags || !detail) return fail(LA_ERR_INVALID_ARG, "flags and detail must not be NULL");
-  unsigned int f = 0, w = 0;
-  cudaError_t err = tc_device_error(&f, &w, reset != 0);
-  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(err));
-  *flags = f;
-  *detail = w;
-  return ok();
-}
-
-size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
-                                   int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
-                                   int32_t dtype, int32_t flags) {
-  if (B < 0 || T < 0 || H <= 0 || n_seqs < 0 || !head_dim_ok(d_k) || !head_dim_ok(d_v))
-    return (size_t)-1;
-  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return (size_t)-1;
-  if (dtype != LA_F32 && dtype != LA_BF16) return (size_t)-1;
-  if (dtype == LA_F32 || (flags & LA_FLAG_SIMT)) return 0;
-  return tc_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0, chunk);
-}
-
-la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
-                       const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
-                       int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,
-                       void *workspace, size_t workspace_bytes, void *stream) {
-  return la_fwd_chunk_z(q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, nullptr,
-                        flags, workspace, workspace_bytes, stream);
-}
-
-la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
-                         const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
-                         int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
-                         int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                     const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                     int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
+                     int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
   la_status s;
   if ((s = check_tensor(q, "q")) != LA_OK) return s;
   if ((s = check_tensor(k, "k")) != LA_OK) return s;
@@ -151,7 +107,6 @@ la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor
   if (k->D != q->D) return fail(LA_ERR_INVALID_ARG, "q and k must have the same head dim d_k");
   if (out->D != v->D) return fail(LA_ERR_INVALID_ARG, "out and v must have the same head dim d_v");
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
-  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
   if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (cu_seqlens) {
@@ -178,6 +133,7 @@ la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor
   a.o_st = out->stride_t;
   a.o_sh = out->stride_h;
   a.gamma = gamma;
+  a.g = g;
   a.cu_seqlens = cu_seqlens;
   a.final_state = final_state;
   a.final_z = final_z;
@@ -235,14 +191,10 @@ la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor
   return ok();
 }
 
-}  // extern "C"
-
-namespace {
-
 // Shared by la_step and la_step_norm (z == NULL: no normaliser).
 la_status step_common(const char *name, const la_tensor *q, const la_tensor *k, const la_tensor *v,
-                      const float *gamma, float *state, float *z, const la_tensor *out, int32_t phi,
-                      void *stream) {
+                      const float *gamma, const float *g, float *state, float *z, const la_tensor *out,
+                      int32_t phi, void *stream) {
   la_status s;
   if ((s = check_tensor(q, "q")) != LA_OK) return s;
   if ((s = check_tensor(k, "k")) != LA_OK) return s;
@@ -255,7 +207,8 @@ la_status step_common(const char *name, const la_tensor *q, const la_tensor *k, 
   if (k->B != q->B || v->B != q->B || out->B != q->B || k->H != q->H || v->H != q->H || out->H != q->H)
     return fail(LA_ERR_INVALID_ARG, "q, k, v, out disagree on N or H");
   if (k->D != q->D || out->D != v->D) return fail(LA_ERR_INVALID_ARG, "head dims disagree");
-  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!gamma && !g) return fail(LA_ERR_INVALID_ARG, "%s is NULL", g ? "g" : "gamma");
+  if (((uintptr_t)g) % 4 != 0) return fail(LA_ERR_INVALID_ARG, "g not 4-byte aligned");
   if (q->B * q->H > 0 && !state) return fail(LA_ERR_INVALID_ARG, "state is NULL");
   if (((uintptr_t)state) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "state not 16-byte aligned");
   if (((uintptr_t)z) % 16 != 0) return fail(LA_ERR_INVALID_ARG, "z not 16-byte aligned");
@@ -269,6 +222,7 @@ la_status step_common(const char *name, const la_tensor *q, const la_tensor *k, 
   a.o_sb = out->stride_b;
   a.o_sh = out->stride_h;
   a.gamma = gamma;
+  a.g = g;
   a.state = state;
   a.z = z;
   a.N = q->B;
@@ -288,15 +242,84 @@ la_status step_common(const char *name, const la_tensor *q, const la_tensor *k, 
 
 extern "C" {
 
+const char *la_status_string(int32_t status) {
+  switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: valid but not implemented";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or launch failed";
+    default: return "unknown la_status";
+  }
+}
+
+const char *la_last_error(void) { return g_msg; }
+
+int32_t la_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+la_status la_device_error(uint32_t *flags, uint32_t *detail, int32_t reset) {
+  if (!flags || !detail) return fail(LA_ERR_INVALID_ARG, "flags and detail must not be NULL");
+  unsigned int f = 0, w = 0;
+  cudaError_t err = tc_device_error(&f, &w, reset != 0);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(err));
+  *flags = f;
+  *detail = w;
+  return ok();
+}
+
+size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                   int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
+                                   int32_t dtype, int32_t flags) {
+  if (B < 0 || T < 0 || H <= 0 || n_seqs < 0 || !head_dim_ok(d_k) || !head_dim_ok(d_v))
+    return (size_t)-1;
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return (size_t)-1;
+  if (dtype != LA_F32 && dtype != LA_BF16) return (size_t)-1;
+  if (dtype == LA_F32 || (flags & LA_FLAG_SIMT)) return 0;
+  return tc_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0, chunk);
+}
+
+la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                       const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                       int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+  return la_fwd_chunk_z(q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, nullptr,
+                        flags, workspace, workspace_bytes, stream);
+}
+
+la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                         const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                         int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
+                         int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  return fwd_common(q, k, v, gamma, nullptr, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, final_z,
+                    flags, workspace, workspace_bytes, stream);
+}
+
+la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                             const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                             int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
+                             int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!g && q && q->B * q->T * q->H > 0) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  if (((uintptr_t)g) % 4 != 0) return fail(LA_ERR_INVALID_ARG, "g not 4-byte aligned");
+  return fwd_common(q, k, v, nullptr, g, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, final_z,
+                    flags, workspace, workspace_bytes, stream);
+}
+
 la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
                   const la_tensor *out, int32_t phi, void *stream) {
-  return step_common("la_step", q, k, v, gamma, state, nullptr, out, phi, stream);
+  return step_common("la_step", q, k, v, gamma, nullptr, state, nullptr, out, phi, stream);
 }
 
 la_status la_step_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                        float *state, float *z, const la_tensor *out, int32_t phi, void *stream) {
   if (q && k && q->B * q->H > 0 && !z) return fail(LA_ERR_INVALID_ARG, "z is NULL");
-  return step_common("la_step_norm", q, k, v, gamma, state, z, out, phi, stream);
+  return step_common("la_step_norm", q, k, v, gamma, nullptr, state, z, out, phi, stream);
+}
+
+la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g, float *state,
+                        float *z, const la_tensor *out, int32_t phi, void *stream) {
+  if (!g && q && q->B * q->H > 0) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  return step_common("la_step_gated", q, k, v, nullptr, g, state, z, out, phi, stream);
 }
 
 }  // extern "C"

@@ -22,7 +22,8 @@ struct ChunkArgs {
   TensorView q, k, v;
   void *out;
   int64_t o_sb, o_st, o_sh;
-  const float *gamma;
+  const float *gamma;         // per-head decay [H] (ignored when g is set)
+  const float *g;             // NULL, or data-dependent log decay [B * T][H]
   const int32_t *cu_seqlens;  // NULL for dense batches
   float *final_state;         // NULL allowed
   float *final_z;             // NULL allowed; only with normalize
@@ -36,6 +37,7 @@ struct StepArgs {
   void *out;
   int64_t o_sb, o_sh;
   const float *gamma;
+  const float *g;  // NULL, or per-(sequence, head) log decay [N, H] replacing gamma
   float *state;
   float *z;  // normaliser state [N, H, d_k] (la_step_norm); NULL for la_step
   int64_t N;

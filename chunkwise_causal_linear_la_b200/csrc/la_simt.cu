@@ -7,6 +7,10 @@
 //   o_i   = gamma^(i+1) S_p qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j) v_j
 //   den_i = gamma^(i+1) z_p . qh_i + sum_{j<=i} gamma^(i-j) (qh_i . kh_j)
 //   S'    = gamma^C' S_p + sum_j gamma^(C'-1-j) v_j kh_j^T     (z' likewise)
+// With a data-dependent decay alpha_t = exp(g_t) (section 状态空间模型与 Mamba)
+// every gamma^n above becomes a product of the alphas it spans: with the chunk's
+// prefix sums b_i = sum_{t<=i} g_t, gamma^(i-j) -> exp(b_i - b_j), gamma^(i+1) ->
+// exp(b_i), gamma^C' -> exp(b_{C'-1}) and gamma^(C'-1-j) -> exp(b_{C'-1} - b_j).
 // This kernel is the exact-arithmetic path: f32 inputs (no TF32 anywhere) and
 // any shape the tensor-core kernel does not take.  One CTA owns one
 // (sequence, head, slice of d_v columns) and walks its chunks in order, with
@@ -26,7 +30,7 @@ struct SimtLayout {
   int n_vt;
   size_t smem;
   // float offsets
-  int off_st, off_z, off_q, off_k, off_v, off_p, off_pw, off_den;
+  int off_st, off_z, off_q, off_k, off_v, off_p, off_pw, off_den, off_b;
 };
 
 SimtLayout simt_layout(int dk, int dv, int C, int dvt) {
@@ -42,6 +46,7 @@ SimtLayout simt_layout(int dk, int dv, int C, int dvt) {
   L.off_p = o; o += C * (C + 1);
   L.off_pw = o; o += C + 1;
   L.off_den = o; o += C;
+  L.off_b = o; o += C;
   L.smem = (size_t)o * sizeof(float);
   return L;
 }
@@ -70,6 +75,7 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
   float *P = sm + L.off_p;      // [C][C+1]    decay-masked scores
   float *pw = sm + L.off_pw;    // [C+1]       gamma^n
   float *den = sm + L.off_den;  // [C]
+  float *bsum = sm + L.off_b;   // [C]         data-dependent decay: chunk prefix sums of g
 
   const int tid = threadIdx.x;
   const int C = a.chunk, dk = a.dk, dvt = L.dvt;
@@ -90,7 +96,8 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
     start = 0;
     len = a.T;
   }
-  const float g = a.gamma[h];
+  const float g = a.g ? 1.f : a.gamma[h];
+  const bool gated = a.g != nullptr;
   const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + h * a.q.sh;
   const Tin *K = (const Tin *)a.k.data + b * a.k.sb + h * a.k.sh;
   const Tin *V = (const Tin *)a.v.data + b * a.v.sb + h * a.v.sh + v0;
@@ -121,7 +128,20 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
       if (i < Cp && r < ncols) x = to_f32<Tin>(V[(start + c0 + i) * a.v.st + r]);
       vv[e] = x;
     }
+    if (gated && tid == 0) {  // prefix sums of the log decay over the chunk
+      float acc = 0.f;
+      const float *gp = a.g + (b * a.T + start + c0) * a.H + h;
+      for (int i = 0; i < C; ++i) {
+        if (i < Cp) acc += gp[(int64_t)i * a.H];
+        bsum[i] = acc;
+      }
+    }
     __syncthreads();
+    // decay factors of the chunk: D(i, j) = gamma^(i-j), E(i) = gamma^(i+1),
+    // W(j) = gamma^(Cp-1-j) (data-dependent: differences of the prefix sums)
+    auto Dij = [&](int i, int j) { return gated ? expf(bsum[i] - bsum[j]) : pw[i - j]; };
+    auto Ei = [&](int i) { return gated ? expf(bsum[i]) : pw[i + 1]; };
+    auto Wj = [&](int j) { return gated ? expf(bsum[Cp - 1] - bsum[j]) : pw[Cp - 1 - j]; };
     // ---- P = (qh kh^T) * D, D_ij = gamma^(i-j) for j <= i (diagonal kept)
     for (int e = tid; e < C * C; e += kSimtThreads) {
       const int i = e / C, j = e % C;
@@ -130,7 +150,7 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
         const float *qi = qh + i * (dk + 1);
         const float *kj = kh + j * (dk + 1);
         for (int c = 0; c < dk; ++c) acc = fmaf(qi[c], kj[c], acc);
-        acc *= pw[i - j];
+        acc *= Dij(i, j);
       }
       P[i * (C + 1) + j] = acc;
     }
@@ -142,7 +162,7 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
         const float *qi = qh + i * (dk + 1);
         for (int c = 0; c < dk; ++c) zq = fmaf(z[c], qi[c], zq);
         for (int j = 0; j <= i; ++j) ps += P[i * (C + 1) + j];
-        den[i] = fmaf(pw[i + 1], zq, ps);
+        den[i] = fmaf(Ei(i), zq, ps);
       }
       __syncthreads();
     }
@@ -154,23 +174,23 @@ chunk_simt_kernel(ChunkArgs a, SimtLayout L) {
       float inter = 0.f, intra = 0.f;
       for (int c = 0; c < dk; ++c) inter = fmaf(qi[c], St[c * dvt + r], inter);
       for (int j = 0; j <= i; ++j) intra = fmaf(P[i * (C + 1) + j], vv[j * dvt + r], intra);
-      float o = fmaf(pw[i + 1], inter, intra);
+      float o = fmaf(Ei(i), inter, intra);
       if (a.normalize) o = o / den[i];
       O[(start + c0 + i) * a.o_st + r] = from_f32<Tin>(o);
     }
     __syncthreads();
     // ---- carry: S^T <- gamma^Cp S^T + sum_j gamma^(Cp-1-j) kh_j v_j^T ; z likewise
-    const float gC = pw[Cp];
+    const float gC = gated ? expf(bsum[Cp - 1]) : pw[Cp];
     for (int e = tid; e < dk * dvt; e += kSimtThreads) {
       const int c = e / dvt, r = e % dvt;
       float acc = 0.f;
-      for (int j = 0; j < Cp; ++j) acc = fmaf(pw[Cp - 1 - j] * kh[j * (dk + 1) + c], vv[j * dvt + r], acc);
+      for (int j = 0; j < Cp; ++j) acc = fmaf(Wj(j) * kh[j * (dk + 1) + c], vv[j * dvt + r], acc);
       St[e] = fmaf(gC, St[e], acc);
     }
     if (a.normalize) {
       for (int c = tid; c < dk; c += kSimtThreads) {
         float acc = 0.f;
-        for (int j = 0; j < Cp; ++j) acc = fmaf(pw[Cp - 1 - j], kh[j * (dk + 1) + c], acc);
+        for (int j = 0; j < Cp; ++j) acc = fmaf(Wj(j), kh[j * (dk + 1) + c], acc);
         z[c] = fmaf(gC, z[c], acc);
       }
     }

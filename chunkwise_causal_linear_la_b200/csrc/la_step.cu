@@ -4,6 +4,8 @@
 // state and adds one outer product per token.  With the state stored as S^T
 // ([d_k][d_v], fp32) and the per-head decay gamma:
 //     S^T[c][r] <- gamma S^T[c][r] + phi(k)_c v_r,     o_r = sum_c S^T[c][r] phi(q)_c.
+// la_step_gated takes the decay per (sequence, head) as exp(g[n][h]) instead
+// (a data-dependent decay: "1.6 长上下文与高效注意力", section 状态空间模型与 Mamba).
 // The normalised form (la_step_norm) also carries z, the running key sum of
 // the same section's displayed equation:
 //     z[c] <- gamma z[c] + phi(k)_c,     o_r /= sum_c z[c] phi(q)_c.
@@ -50,7 +52,7 @@ step_kernel(StepArgs a) {
     qh[c] = feature_map(to_f32<Tin>(Q[c]), a.phi);
     kh[c] = feature_map(to_f32<Tin>(K[c]), a.phi);
   }
-  const float g = a.gamma[h];
+  const float g = a.g ? expf(a.g[unit]) : a.gamma[h];  // data-dependent decay: exp(g[n][h])
   const int cg = tid % ncg, rg = tid / ncg;
   float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
   if (rg < nrg) {

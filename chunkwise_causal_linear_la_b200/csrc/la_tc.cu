@@ -86,6 +86,9 @@ struct TcArgs {
   int G, Gp, segC;
   float *ws_s;  // [units][G-1][DK][DVT] (S^T rows)
   float *ws_z;  // [units][G-1][DK]
+  float *ws_g;  // [units][G-1]: log decay of each segment (data-dependent decay)
+  // Data-dependent decay: log alpha per token and head, [B * T][H] (NULL: gamma)
+  const float *g;
 };
 
 template <int DK, int DVT, int C, int NS>
@@ -107,7 +110,10 @@ struct Cfg {
   static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_Z = OFF_SB + SB_BYTES;  // normaliser key sums z, two buffers of DK floats
   static constexpr int OFF_KSUM = OFF_Z + 2 * DK * 4;  // per stage, per transform warp: chunk key column sums
-  static constexpr int OFF_PW = OFF_KSUM + NS * 2 * DK * 4;
+  // data-dependent decay, per stage: b_i = sum_{t<=i} log alpha_t over the chunk, i < C, and b_last at [C]
+  static constexpr int OFF_DT = OFF_KSUM + NS * 2 * DK * 4;
+  static constexpr int DT_STRIDE = C + 4;
+  static constexpr int OFF_PW = OFF_DT + NS * DT_STRIDE * 4;
   static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
   // barriers
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_PFULL = 3 * NS + 2,
@@ -190,6 +196,14 @@ __device__ __forceinline__ float phi_fast(float x) {
   return x > 0.f ? x + 1.f : e;
 }
 
+// e^x on the same instruction, for the data-dependent decay factors (x <= 0).
+__device__ __forceinline__ float exp_fast(float x) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * kLog2e));
+  return e;
+}
+
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -259,7 +273,7 @@ __device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int
   }
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
@@ -268,6 +282,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
   float *ksum = reinterpret_cast<float *>(sm + G::OFF_KSUM);
+  float *dtab = reinterpret_cast<float *>(sm + G::OFF_DT);  // [NS][DT_STRIDE]
   float *pw = reinterpret_cast<float *>(sm + G::OFF_PW);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
@@ -307,7 +322,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const bool last_seg = a.G == 1 || seg == a.G - 1;
   const int64_t ws_slot = (int64_t)unit * (a.G - 1) + (MODE == 1 ? seg : seg - 1);
   const int nchunks = (int)((len + C - 1) / C);
-  const float g = a.gamma[h];
+  const float g = GATED ? 1.f : a.gamma[h];
 
   // ---- setup
   if (tid <= C) pw[tid] = decay_pow(g, tid);
@@ -337,7 +352,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const bool vd_mode = DK == 256 || ((g < 1.f) && (pw[C - 1] < kSmallGammaLimit));
+  // value-decay mode: always with a data-dependent decay (its factors are all <= 1)
+  const bool vd_mode = GATED || DK == 256 || ((g < 1.f) && (pw[C - 1] < kSmallGammaLimit));
   // output accumulators of chunk c: buffer ob(c), completion parity oph(c)
   auto out_buf = [&](int c) -> int { return (vd_mode && !G::VD_DB) ? 0 : (c & 1); };
   auto out_phase = [&](int c) -> uint32_t { return (vd_mode && !G::VD_DB) ? (c & 1) : ((c >> 1) & 1); };
@@ -422,8 +438,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
           }
           umma_commit(bars + G::B_UFULL);
-          // normalised: the state warps' key sums read the stage too
-          if (NORM && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;
+          // normalised / data-dependent decay: the state warps read the stage's key
+          // sums and decay table too
+          if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;
           umma_commit(bars + G::B_EMPTY + s);
           done = c + 1;
         }
@@ -478,7 +495,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
         }
         umma_commit(bars + G::B_OFULL + ob);
-        if (NORM && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // key sums read the stage
+        if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
         umma_commit(bars + G::B_EMPTY + s);
         done = c + 1;
         // with two stages, chunk c+1's tiles land only after chunk c-1's stage is
@@ -505,12 +522,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int Cp = chunk_len(c);
         if (vd_mode && c > 0 && !wait_bar(sy, G::B_UFULL, (c - 1) & 1, c)) break;  // M4(c-1) read vd
         static_assert(G::SLAB / 16 == 8 * 64, "row mapping assumes C = 64");
-        // row weights of this thread's vectors: gamma^(C'-1-j), zero past the chunk end
+        // Data-dependent decay: prefix sums b_i = sum_{t<=i} log alpha_t over the
+        // chunk (tokens past its end count as alpha = 1).  Each warp computes all
+        // 64 (lane l holds b_l and b_{l+32}); the first warp publishes them with
+        // b_last = b_{C'-1} in the stage's table.
+        float blo = 0.f, bhi = 0.f, blast = 0.f;
+        if (GATED) {
+          const int ln = tt & 31;
+          const int64_t row0 = (int64_t)bidx * a.T + start + (int64_t)c * C;
+          blo = ln < Cp ? a.g[(row0 + ln) * a.H + h] : 0.f;
+          bhi = ln + 32 < Cp ? a.g[(row0 + ln + 32) * a.H + h] : 0.f;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, blo, o);
+            const float y1 = __shfl_up_sync(0xffffffffu, bhi, o);
+            if (ln >= o) {
+              blo += y0;
+              bhi += y1;
+            }
+          }
+          bhi += __shfl_sync(0xffffffffu, blo, 31);
+          blast = __shfl_sync(0xffffffffu, Cp <= 32 ? blo : bhi, (Cp - 1) & 31);
+          if (tt < 32) {
+            float *dt = dtab + s * G::DT_STRIDE;
+            dt[ln] = blo;
+            dt[ln + 32] = bhi;
+            if (ln == 0) dt[C] = blast;
+          }
+        }
+        // row weights of this thread's vectors: gamma^(C'-1-j) (data-dependent:
+        // exp(b_last - b_j)), zero past the chunk end
         auto decay_weights = [&](float (&wv)[8]) {
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             const int j = (tt >> 3) + 8 * m;
-            wv[m] = j < Cp ? pw[Cp - 1 - j] : 0.f;
+            if (GATED) {
+              const float b0 = __shfl_sync(0xffffffffu, blo, j & 31);
+              const float b1 = __shfl_sync(0xffffffffu, bhi, j & 31);
+              wv[m] = j < Cp ? exp_fast(blast - (j < 32 ? b0 : b1)) : 0.f;
+            } else {
+              wv[m] = j < Cp ? pw[Cp - 1 - j] : 0.f;
+            }
           }
         };
         float wv[8], wsum[8];
@@ -570,9 +622,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
     for (int mb = 0; mb < G::MB; ++mb)
       zr[mb] = (NORM && has_init) ? a.ws_z[ws_slot * DK + mb * 128 + sp * 32 + lane] : 0.f;
-    // z <- gamma^C' z + (chunk c's weighted key column sums, from the transform
-    // warps), published in z buffer (c & 1) for the output warps
-    auto key_sums = [&](int c, int Cp) -> bool {
+    // z <- gdec z + (chunk c's weighted key column sums, from the transform
+    // warps), published in z buffer (c & 1) for the output warps; gdec is the
+    // chunk's whole decay (gamma^C' or exp(b_last))
+    auto key_sums = [&](int c, float gdec) -> bool {
       const int s = c % NS;
       if (!wait_bar_warp(sy, G::B_XFORM + s, (c / NS) & 1, c)) return false;
       const float *ks = ksum + s * 2 * DK;
@@ -580,12 +633,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
         const int kr = mb * 128 + sp * 32 + lane;
-        zr[mb] = fmaf(pw[Cp], zr[mb], ks[kr] + ks[DK + kr]);
+        zr[mb] = fmaf(gdec, zr[mb], ks[kr] + ks[DK + kr]);
         zb[kr] = zr[mb];
       }
-      mbar_arrive(bars + G::B_ZFULL + (c & 1));
       return true;
     };
+    float seg_log = 0.f;  // data-dependent decay: log of this segment's whole decay (state pass)
     // bf16 operand Sb = sc * S for the next chunk's inter-chunk product
     auto write_sb = [&](float sc) {
 #pragma unroll
@@ -613,7 +666,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int Cp = chunk_len(c);
       if (!wait_bar_warp(sy, G::B_UFULL, c & 1, c)) break;
       tc_fence_after();
-      const float gdec = pw[Cp];
+      float gdec = pw[Cp];
+      if (GATED) {  // the chunk's decay from the transform warps' table
+        if (!wait_bar_warp(sy, G::B_XFORM + c % NS, (c / NS) & 1, c)) break;
+        const float bl = dtab[(c % NS) * G::DT_STRIDE + C];
+        gdec = exp_fast(bl);
+        seg_log += bl;
+      }
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
@@ -630,7 +689,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       tc_fence_before();
       mbar_arrive(bars + G::B_UEMPTY);
-      if (NORM && !key_sums(c, Cp)) break;
+      if (NORM && !key_sums(c, gdec)) break;
+      // this warpgroup is done with the stage's key sums and decay table
+      if (NORM || GATED) mbar_arrive(bars + G::B_ZFULL + (c & 1));
       if (MODE == 1 || c == nchunks - 1) continue;
       // the previous Sb has been read once M2 of chunk c is done
       if (c - 1 + sbo >= 0 && !wait_bar_warp(sy, G::B_SBEMPTY, (c - 1 + sbo) & 1, c)) break;
@@ -647,6 +708,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int mb = 0; mb < G::MB; ++mb) a.ws_z[ws_slot * DK + mb * 128 + sp * 32 + lane] = zr[mb];
       }
+      if (GATED && sp == 0 && lane == 0) a.ws_g[ws_slot] = seg_log;
     } else if (a.final_state && last_seg) {
       F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT;
     }
@@ -712,13 +774,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       return zq;
     };
 
-    // scores of chunk c -> P tile; returns this row's output factor
-    auto scores = [&](int c, bool &ok) -> float {
+    // scores of chunk c -> P tile; returns this row's output factor and, in
+    // value-decay mode, the inter-chunk factor gi (gamma^(i+1) or exp(b_i))
+    auto scores = [&](int c, bool &ok, float &gi) -> float {
       const int b = c & 1;
       const int Cp = chunk_len(c);
       ok = false;
       if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return 0.f;
       tc_fence_after();
+      const float *dt = dtab + (c % NS) * G::DT_STRIDE;
+      float bi = 0.f;
+      if (GATED) {  // the stage's decay table (published before the score MMA's inputs)
+        if (!wait_bar_warp(sy, G::B_XFORM + c % NS, (c / NS) & 1, c)) return 0.f;
+        bi = dt[i];
+        gi = exp_fast(bi);
+      } else {
+        gi = pw[i + 1];
+      }
       float zq = 0.f;
       if (NORM) {
         zq = z_dot_q(c, ok);
@@ -733,6 +805,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!vd_mode) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e <= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
+      } else if (GATED) {  // P_ij = A_ij exp(b_i - b_j)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = hf * 32 + e;
+          f[e] = (j <= i && row_ok) ? __uint_as_float(r[e]) * exp_fast(bi - dt[j]) : 0.f;
+        }
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -759,17 +837,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       if (!row_ok) return 0.f;
       if (!NORM) return vd_mode ? 1.f : 1.f / pw[Cp - 1 - i];
-      return 1.f / fmaf(vd_mode ? pw[i + 1] : pw[Cp], zq, rowsum);
+      return 1.f / fmaf(vd_mode ? gi : pw[Cp], zq, rowsum);
     };
 
     // epilogue of chunk c
-    auto epilogue = [&](int c, float fac) -> bool {
+    auto epilogue = [&](int c, float fac, float gi) -> bool {
       const int Cp = chunk_len(c);
       const int ob = out_buf(c);
       const uint32_t oph = out_phase(c);
       if (!wait_bar_warp(sy, G::B_OFULL + ob, oph, c)) return false;
       tc_fence_after();
-      const float gi = pw[i + 1];
       uint8_t *orow = obase + 2 * ((start + (int64_t)c * C + i) * a.o_st);
       const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
 #pragma unroll 1
@@ -838,15 +915,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool qok = true;
     if (kQByOutput)
       for (int c = 0; c < QLA && c < nchunks && qok; ++c) qok = q_xform(c);
-    float fac_even = 0.f, fac_odd = 0.f;
+    float fac_even = 0.f, fac_odd = 0.f, gi_even = 0.f, gi_odd = 0.f;
     for (int t = 0; t <= nchunks && MODE == 0 && qok; ++t) {
       if (t < nchunks) {
         bool ok = true;
-        const float f = scores(t, ok);
+        float gi = 0.f;
+        const float f = scores(t, ok, gi);
         if (!ok) break;
-        if (t & 1) fac_odd = f; else fac_even = f;
+        if (t & 1) {
+          fac_odd = f;
+          gi_odd = gi;
+        } else {
+          fac_even = f;
+          gi_even = gi;
+        }
       }
-      if (t >= 1 && !epilogue(t - 1, ((t - 1) & 1) ? fac_odd : fac_even)) break;
+      if (t >= 1 && !epilogue(t - 1, ((t - 1) & 1) ? fac_odd : fac_even, ((t - 1) & 1) ? gi_odd : gi_even)) break;
       if (kQByOutput && t + QLA < nchunks && !q_xform(t + QLA)) break;
     }
   }
@@ -927,21 +1011,25 @@ SegPlan seg_plan(int64_t n_seqs, int64_t T, int64_t H, int nvt, bool varlen, int
   return p;
 }
 
+// Workspace of a segmented launch: segment states S^T [units][G-1][dk][dvt],
+// normaliser sums [units][G-1][dk], segment log decays [units][G-1].
 size_t seg_ws_bytes(const SegPlan &p, int dk, int dvt) {
   if (p.G < 2) return 0;
-  return (size_t)p.units * (p.G - 1) * ((size_t)dk * dvt + dk) * sizeof(float);
+  return (size_t)p.units * (p.G - 1) * ((size_t)dk * dvt + dk + 1) * sizeof(float);
 }
 
 // Segment start states from segment end states, in place: slot g-1 of a unit
-// ends up holding W_g = gamma^L W_{g-1} + E_{g-1} (W_0 = 0), L = tokens of a
-// full segment; the same recurrence runs on the normaliser sums.
-__global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *gamma, int G, int64_t seg_tokens,
-                                int H, int nvt, int elems_s, int elems_z) {
+// ends up holding W_g = D_{g-1} W_{g-1} + E_{g-1} (W_0 = 0), where D is the
+// decay over a full segment: gamma^L (L tokens), or exp of the segment's summed
+// log decay (ws_g) with a data-dependent decay; the same recurrence runs on the
+// normaliser sums.
+__global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *ws_g, const float *gamma, int G,
+                                int64_t seg_tokens, int H, int nvt, int elems_s, int elems_z) {
   const int64_t unit = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= elems_s + elems_z) return;
   const int h = (int)((unit / nvt) % H);
-  const float gL = powf(gamma[h], (float)seg_tokens);
+  const float gL = ws_g ? 0.f : powf(gamma[h], (float)seg_tokens);
   float *base;
   int64_t stride;
   if (e < elems_s) {
@@ -955,12 +1043,13 @@ __global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *gamma, in
   float w = 0.f;
   for (int g = 1; g < G; ++g) {
     float *slot = base + (int64_t)(g - 1) * stride;
-    w = fmaf(gL, w, *slot);
+    const float d = ws_g ? expf(ws_g[unit * (G - 1) + (g - 1)]) : gL;
+    w = fmaf(d, w, *slot);
     *slot = w;
   }
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, bool GATED>
 cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   using G = Cfg<DK, DVT, C, NS>;
   CUtensorMap mq, mk, mv;
@@ -978,6 +1067,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.cu_seqlens = a.cu_seqlens;
   t.final_state = a.final_state;
   t.final_z = a.final_z;
+  t.g = a.g;
   t.T = a.T;
   t.H = a.H;
   t.dv = a.dv;
@@ -991,7 +1081,8 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.segC = plan.segC;
   t.ws_s = nullptr;
   t.ws_z = nullptr;
-  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0>;
+  t.ws_g = nullptr;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0, GATED>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   if (plan.G > 1) {
@@ -1001,8 +1092,9 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
     }
     t.ws_s = static_cast<float *>(workspace);
     t.ws_z = NORM ? t.ws_s + units * (plan.G - 1) * DK * DVT : nullptr;
+    t.ws_g = GATED ? t.ws_s + units * (plan.G - 1) * (DK * DVT + DK) : nullptr;
     // pass 1: end state of every segment but the last, from a zero start
-    auto kst = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 1>;
+    auto kst = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 1, GATED>;
     err = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     t.Gp = plan.G - 1;
@@ -1011,8 +1103,8 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
     // scan: start states of segments 1 .. G-1
     const int elems_s = DK * DVT, elems_z = NORM ? DK : 0;
     dim3 sgrid((unsigned)((elems_s + elems_z + 255) / 256), (unsigned)units);
-    seg_scan_kernel<<<sgrid, 256, 0, stream>>>(t.ws_s, t.ws_z, a.gamma, plan.G, (int64_t)plan.segC * C, a.H,
-                                               a.dv / DVT, elems_s, elems_z);
+    seg_scan_kernel<<<sgrid, 256, 0, stream>>>(t.ws_s, t.ws_z, t.ws_g, a.gamma, plan.G, (int64_t)plan.segC * C,
+                                               a.H, a.dv / DVT, elems_s, elems_z);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   // output pass: every segment, seeded with its start state
@@ -1050,15 +1142,21 @@ size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64
   return seg_ws_bytes(seg_plan(n_seqs, T, H, dv / dvt, varlen, chunk), dk, dvt);
 }
 
+template <int DK, int DVT, int NS, bool GATED>
+cudaError_t launch_shape_gated(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
+  // one instantiation per (normaliser, feature map, decay kind): each carries only its own code path
+  if (a.normalize) {
+    return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true, GATED>(a, workspace, stream, why)
+                 : launch_cfg<DK, DVT, 64, NS, true, false, GATED>(a, workspace, stream, why);
+  }
+  return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, GATED>(a, workspace, stream, why)
+               : launch_cfg<DK, DVT, 64, NS, false, false, GATED>(a, workspace, stream, why);
+}
+
 template <int DK, int DVT, int NS>
 cudaError_t launch_shape(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
-  // one instantiation per (normaliser, feature map): each carries only its own code path
-  if (a.normalize) {
-    return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true>(a, workspace, stream, why)
-                 : launch_cfg<DK, DVT, 64, NS, true, false>(a, workspace, stream, why);
-  }
-  return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true>(a, workspace, stream, why)
-               : launch_cfg<DK, DVT, 64, NS, false, false>(a, workspace, stream, why);
+  return a.g ? launch_shape_gated<DK, DVT, NS, true>(a, workspace, stream, why)
+             : launch_shape_gated<DK, DVT, NS, false>(a, workspace, stream, why);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t, cudaStream_t stream, const char **why) {

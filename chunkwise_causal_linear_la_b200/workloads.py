@@ -11,6 +11,8 @@ workload dtype.  Packed variable-length batches first draw their lengths on a
 CPU generator seeded the same way (``randint(lo, hi + 1, (n,))``), so the
 lengths do not depend on the device.  Decode workloads draw q, k, v of shape
 [N, H, d] and then the state [N, H, d_k, d_v] as ``state_std`` * N(0, 1).
+Workloads with a data-dependent decay then draw its log, g [B, T, H], uniform
+in [ln lo, ln hi] (``gate = (lo, hi)``), from a second generator seeded with seed + 1.
 """
 from __future__ import annotations
 
@@ -36,6 +38,7 @@ class Workload:
     normalize: bool
     chunk: int = 64
     varlen: Optional[tuple] = None  # (n_seqs, lo, hi) for packed batches
+    gate: Optional[tuple] = None  # (lo, hi): per-token decays in [lo, hi] (log drawn uniform)
 
     @property
     def torch_dtype(self):
@@ -77,6 +80,10 @@ WORKLOADS = {
         scale=1.0 / math.sqrt(128), gamma=(1.0,) * 8, phi="elu1", normalize=True,
         varlen=(64, 128, 2048),
     ),
+    "gated_T16384": Workload(
+        "gated_B8_H16_d128_T16384", B=8, T=16384, H=16, d_k=128, d_v=128, dtype="bf16",
+        scale=1.0 / math.sqrt(128), gamma=(1.0,) * 16, phi="identity", normalize=False, gate=(0.9, 0.999),
+    ),
     "long_1m": Workload(
         "long_B1_H4_T1048576_d128", B=1, T=1 << 20, H=4, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=retnet_gammas(4, 8), phi="identity", normalize=False,
@@ -114,8 +121,14 @@ def make_qkv(B, T, H, d_k, d_v, dtype, scale, seed=0, device="cpu"):
     return tuple(out)
 
 
+def make_log_decay(B, T, H, lo, hi, generator, device="cpu"):
+    """g [B, T, H] float32, uniform in [ln lo, ln hi] (decays exp(g) in [lo, hi])."""
+    a, b = math.log(lo), math.log(hi)
+    return torch.rand((B, T, H), generator=generator, device=device, dtype=torch.float32) * (b - a) + a
+
+
 def make_inputs(w: Workload, seed: int = 0, device="cpu", T: Optional[int] = None, B: Optional[int] = None):
-    """Inputs of workload ``w``: dict(q, k, v, gamma, cu_seqlens).
+    """Inputs of workload ``w``: dict(q, k, v, gamma, cu_seqlens[, g]).
 
     ``T`` / ``B`` override the sequence length / batch (used to shrink a
     workload for a quick check while keeping its distribution).
@@ -132,7 +145,12 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", T: Optional[int] = Non
     gamma = torch.tensor(w.gamma, dtype=torch.float32, device=device)
     if cu is not None:
         cu = cu.to(device)
-    return dict(q=q, k=k, v=v, gamma=gamma, cu_seqlens=cu)
+    x = dict(q=q, k=k, v=v, gamma=gamma, cu_seqlens=cu)
+    if w.gate is not None:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed + 1)
+        x["g"] = make_log_decay(Bq, Tq, w.H, w.gate[0], w.gate[1], gen, device)
+    return x
 
 
 def make_decode_inputs(N, H, d_k, d_v, scale, state_std, gamma, seed=0, device="cpu",

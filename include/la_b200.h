@@ -157,6 +157,25 @@ LA_API la_status la_fwd_chunk_z(const la_tensor *q, const la_tensor *k, const la
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * la_fwd_chunk_gated -- la_fwd_chunk_z with a data-dependent decay.
+ * "1.6 长上下文与高效注意力", section 状态空间模型与 Mamba: the decay of the state
+ * becomes a function of the input token (Mamba-2: a scalar per step, which is
+ * linear attention with a decay mask).  Here the decay of token t in head h is
+ * alpha = exp(g[t][h]):
+ *     S_t = alpha_t S_{t-1} + v_t phi(k_t)^T,   z_t = alpha_t z_{t-1} + phi(k_t).
+ *   g        device float[B, T, H], contiguous (token rows of the q layout; a
+ *            packed batch has B = 1): the log decay, finite and <= 0 (alpha in
+ *            (0, 1]); it takes the place of gamma.  4-byte aligned.
+ *   Every other argument, layout, result and error is that of la_fwd_chunk_z
+ *   (final_z may be NULL; it needs normalize).  The workspace size is
+ *   la_fwd_chunk_workspace_size's for the same shape.
+ */
+LA_API la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                                    const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                                    int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
+                                    int32_t flags, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of workspace la_fwd_chunk needs for this problem: B, T, H, d_k, d_v
  * and n_seqs as they will be passed, has_cu_seqlens nonzero for a packed
  * batch.  Returns 0 when no workspace is needed and (size_t)-1 for arguments
@@ -200,6 +219,16 @@ LA_API la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor
  */
 LA_API la_status la_step_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                               float *state, float *z, const la_tensor *out, int32_t phi, void *stream);
+
+/*
+ * la_step_gated -- one decode token with a data-dependent decay: la_step
+ * (z == NULL) or la_step_norm (z != NULL) with the decay of sequence n, head h
+ * equal to exp(g[n][h]) instead of gamma[h].
+ *   g  device float[N, H], contiguous: the log decay of this step, <= 0.
+ * Other arguments, sizes and errors as for la_step / la_step_norm.
+ */
+LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                               float *state, float *z, const la_tensor *out, int32_t phi, void *stream);
 
 /*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device

@@ -69,14 +69,15 @@ def test_workspace_size_host_logic(lib):
 
 
 def test_workspace_size_segment_plan(lib):
-    """Segment states are kept for all but the last segment of each unit, one
-    unit per (sequence, head, value slice); value slices are 128 columns wide at
-    d_k = 128 and 64 at d_k = 256."""
+    """Segment states (S^T, the normaliser sum and the log decay of a
+    data-dependent decay) are kept for all but the last segment of each unit,
+    one unit per (sequence, head, value slice); value slices are 128 columns
+    wide at d_k = 128 and 64 at d_k = 256."""
     ws = lib.la_fwd_chunk_workspace_size
     # d_k = 128: 2 units, 79 chunks -> G = min(148 // 2, 79 // 16) = 4 segments of 20 chunks
-    assert ws(1, 5000, 2, 128, 128, 1, 0, 64, 1, 0) == 2 * 3 * (128 * 128 + 128) * 4
+    assert ws(1, 5000, 2, 128, 128, 1, 0, 64, 1, 0) == 2 * 3 * (128 * 128 + 128 + 1) * 4
     # d_k = 256, d_v = 256: 8 units -> G = min(148 // 8, 4) = 4
-    assert ws(1, 5000, 2, 256, 256, 1, 0, 64, 1, 0) == 8 * 3 * (256 * 64 + 256) * 4
+    assert ws(1, 5000, 2, 256, 256, 1, 0, 64, 1, 0) == 8 * 3 * (256 * 64 + 256 + 1) * 4
     # enough units to fill the GPU (RetNet-style batch: 32 x 4 heads x 4 slices): none
     assert ws(32, 2048, 4, 256, 256, 32, 0, 64, 1, 0) == 0
     # packed batches are not segmented; nor are shapes the tensor cores do not run
