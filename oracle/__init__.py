@@ -18,6 +18,8 @@ it follows, is stated in the C file's header:
 * ``step``      -- one decode token on a given state.
 * ``final_z``   -- the normaliser's key sum z after each sequence's last token.
 * ``step_norm`` -- one normalised decode token (state and z updated).
+* ``backward``  -- dq, dk, dv of sum_t dout_t . o_t (unnormalised; the adjoint
+  of the recurrence, token by token).
 * ``recurrent_gated``, ``step_gated`` -- the same with a data-dependent decay
   alpha_t = exp(g_t) per token and head (section 状态空间模型与 Mamba of the
   same page: Mamba-2 as linear attention with a decay mask).
@@ -74,6 +76,9 @@ def _load():
         lib.oracle_recurrent_gated.restype = i32
         lib.oracle_step_gated.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, dp, dp, dp, dp, i32, i32]
         lib.oracle_step_gated.restype = i32
+        lib.oracle_backward.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, i32,
+                                        dp, dp, dp, i32]
+        lib.oracle_backward.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -285,3 +290,21 @@ def step_gated(q, k, v, g, state, z=None, phi="identity", nthreads=0):
     if rc != 0:
         raise ValueError("oracle_step_gated rejected its arguments (code %d)" % rc)
     return out, st, zz
+
+
+def backward(q, k, v, dout, gamma, cu_seqlens=None, phi="identity", nthreads=0):
+    """Gradients of L = sum(dout * o) for the unnormalised recurrence.
+
+    Returns (dq [B,T,H,d_k], dk [B,T,H,d_k], dv [B,T,H,d_v]) in float64."""
+    q, k, v, dt, B, T, H, dk, dv, g, cu, n = _prep(q, k, v, gamma, cu_seqlens)
+    do, ddt = _as_input(dout)
+    if ddt != dt or do.shape != v.shape:
+        raise ValueError("dout must be [B, T, H, d_v] of the inputs' dtype")
+    gq = np.zeros(q.shape, np.float64)
+    gk = np.zeros(k.shape, np.float64)
+    gv = np.zeros(v.shape, np.float64)
+    rc = _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), dt, B, T, H, dk, dv, _ptr(g), _ptr(cu), n,
+                                 _PHI[phi], 0, _ptr(gq), _ptr(gk), _ptr(gv), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_backward rejected its arguments (code %d)" % rc)
+    return gq, gk, gv

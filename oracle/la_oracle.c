@@ -30,6 +30,8 @@
  *                        from).
  *   oracle_step_norm  -- one normalised decode token: S and z updated in
  *                        place, o_t = S_t phi(q_t) / (z_t^T phi(q_t)).
+ *   oracle_backward   -- dq, dk, dv of sum_t dout_t . o_t for the unnormalised
+ *                        recurrence: the adjoint of the definition.
  *   oracle_recurrent_gated, oracle_step_gated -- the same with a per-token
  *                        (per decode step) decay alpha_t = exp(g_t) in place
  *                        of the per-head constant gamma.
@@ -498,6 +500,89 @@ int oracle_step_gated(const void *q, const void *k, const void *v, int dtype,
     }
     if (z)
       for (int64_t r = 0; r < dv; ++r) o[r] /= den;
+  }
+  return 0;
+}
+
+/*
+ * Backward of the unnormalised recurrence (per-head gamma), the adjoint of
+ * the definition token by token.  With L = sum_t dout_t . o_t:
+ *   forward:   S_t = gamma S_{t-1} + v_t kh_t^T,  o_t = S_t qh_t
+ *   dqh_t  = S_t^T dout_t
+ *   G_t    = dL/dS_t = dout_t qh_t^T + gamma G_{t+1}      (G_{len} = 0)
+ *   dkh_t  = G_t^T v_t,   dv_t = G_t kh_t
+ *   dq = dqh * phi'(q),   dk = dkh * phi'(k)   (phi' = 1, or for elu + 1:
+ *                                                1 if x > 0 else e^x)
+ *   dout [B, T, H, d_v]; dq, dk [B, T, H, d_k], dv [B, T, H, d_v] (double).
+ * The normalised form is not covered (returns -11 if normalize is set).
+ */
+static double orc_dphi(double x, int phi) {
+  if (phi == ORC_PHI_ELU1) return x > 0.0 ? 1.0 : exp(x);
+  return 1.0;
+}
+
+int oracle_backward(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                    int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                    const double *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int phi,
+                    int normalize, double *dq, double *dkk, double *dvv, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (normalize) return -11;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const double g = gamma[h];
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double));  /* S[r][c] */
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    /* forward in time: dqh_t = S_t^T dout_t */
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, vb + r);
+        for (int64_t c = 0; c < dk; ++c) S[r * dk + c] = g * S[r * dk + c] + vr * kh[c];
+      }
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * orc_load(dout, dtype, vb + r);
+        const double x = orc_load(q, dtype, qk + c);
+        dq[qk + c] = acc * orc_dphi(x, phi);
+      }
+    }
+    /* backward in time: G_t = dout_t qh_t^T + gamma G_{t+1} */
+    double *Gm = S;
+    memset(Gm, 0, (size_t)(dv * dk) * sizeof(double));
+    for (int64_t t = len - 1; t >= 0; --t) {
+      const int64_t row = start + t;
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        const double d = orc_load(dout, dtype, vb + r);
+        for (int64_t c = 0; c < dk; ++c) Gm[r * dk + c] = g * Gm[r * dk + c] + d * qh[c];
+      }
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < dv; ++r) acc += Gm[r * dk + c] * orc_load(v, dtype, vb + r);
+        dkk[qk + c] = acc * orc_dphi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += Gm[r * dk + c] * kh[c];
+        dvv[vb + r] = acc;
+      }
+    }
+    free(S);
+    free(qh);
+    free(kh);
   }
   return 0;
 }

@@ -325,6 +325,74 @@ def test_gated_varlen_and_decode_handover(oracle_mod):
             assert rel(z, fzT1) < TOL
 
 
+# ---------------------------------------------------------------- backward
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+@pytest.mark.parametrize("gamma", [0.8, 1.0, 0.0])
+def test_backward_matches_finite_differences(oracle_mod, phi, gamma):
+    """Central differences of L = sum(dout * o) through the forward oracle."""
+    B, T, H, dk, dv = 1, 7, 2, 3, 2
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=61)
+    dout = np.random.default_rng(62).standard_normal((B, T, H, dv))
+    gam = [gamma, 0.5]
+    gq, gk, gv = oracle_mod.backward(q, k, v, dout, gam, phi=phi)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle_mod.recurrent(q_, k_, v_, gam, phi=phi)
+        return float(np.sum(o * dout))
+
+    eps = 1e-6
+    for x, gref, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert rel(gref, fd) < 1e-7, which
+
+
+def test_backward_matches_autograd_of_quadratic_form(oracle_mod):
+    """torch autograd (float64) through the quadratic masked form, a different
+    formula for the same outputs."""
+    T, H, dk, dv = 30, 2, 5, 4
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=63)
+    dout = np.random.default_rng(64).standard_normal((1, T, H, dv))
+    gam = [0.9, 1.0]
+    for phi in ("identity", "elu1"):
+        gq, gk, gv = oracle_mod.backward(q, k, v, dout, gam, phi=phi)
+        for h in range(H):
+            qt, kt, vt = (torch.tensor(x[0, :, h], dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+            f = (lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))) if phi == "elu1" \
+                else (lambda x: x)
+            A = f(qt) @ f(kt).T
+            i = torch.arange(T)[:, None]
+            j = torch.arange(T)[None, :]
+            M = torch.where(i >= j, torch.tensor(gam[h], dtype=torch.float64) ** (i - j).clamp(min=0).double(),
+                            torch.zeros((), dtype=torch.float64))
+            O = (A * M) @ vt
+            (O * torch.tensor(dout[0, :, h])).sum().backward()
+            assert rel(gq[0, :, h], qt.grad.numpy()) < 1e-11
+            assert rel(gk[0, :, h], kt.grad.numpy()) < 1e-11
+            assert rel(gv[0, :, h], vt.grad.numpy()) < 1e-11
+
+
+def test_backward_varlen_equals_independent_runs(oracle_mod):
+    lengths = [5, 0, 17, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 2, 4, 3
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=65)
+    dout = np.random.default_rng(66).standard_normal((1, Tt, H, dv))
+    gam = [0.7, 1.0]
+    gq, gk, gv = oracle_mod.backward(q, k, v, dout, gam, cu_seqlens=cu, phi="elu1")
+    for n in range(len(lengths)):
+        s_, e = cu[n], cu[n + 1]
+        a, b, c = oracle_mod.backward(q[:, s_:e], k[:, s_:e], v[:, s_:e], dout[:, s_:e], gam, phi="elu1")
+        assert np.array_equal(gq[:, s_:e], a) and np.array_equal(gk[:, s_:e], b) and np.array_equal(gv[:, s_:e], c)
+
+
 # ---------------------------------------------------------------- chunked form
 @pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
