@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     LA_FLAG_SIMT,
     LaError,
     device_error,
+    la_bwd_chunk,
     la_fwd_chunk,
     la_fwd_chunk_gated,
     la_fwd_chunk_z,

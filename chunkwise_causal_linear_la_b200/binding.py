@@ -29,7 +29,7 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 # Every function include/la_b200.h declares.
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
-           "la_fwd_chunk_noalloc")
+           "la_fwd_chunk_noalloc", "la_bwd_chunk")
 
 
 class LaTensor(ctypes.Structure):
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.la_step_norm.restype = i32
     lib.la_step_gated.argtypes = [P, P, P, vp, vp, vp, P, i32, vp]
     lib.la_step_gated.restype = i32
+    lib.la_bwd_chunk.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, vp]
+    lib.la_bwd_chunk.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -266,3 +268,23 @@ def la_step_gated(q, k, v, g, state, z=None, out=None, phi="identity", stream=No
                            None if z is None else z.data_ptr(), ctypes.byref(to), _PHI[phi], _stream(stream))
     _check(lib, st, "la_step_gated")
     return o4.squeeze(1) if squeeze else o4
+
+
+def la_bwd_chunk(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="identity", dq=None, dk=None, dv=None,
+                 stream=None):
+    """Gradients (dq, dk, dv) of the unnormalised forward given dout (see la_bwd_chunk in
+    include/la_b200.h).  All tensors [B, T, H, d], one dtype."""
+    lib = load_library()
+    B, T, H, d_k = q.shape
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    t = [describe(x) for x in (q, k, v, dout, dq, dk, dv)]
+    st = lib.la_bwd_chunk(*(ctypes.byref(x) for x in t[:4]), gamma.data_ptr(),
+                          None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
+                          *(ctypes.byref(x) for x in t[4:]), _stream(stream))
+    _check(lib, st, "la_bwd_chunk")
+    return dq, dk, dv

@@ -305,6 +305,65 @@ la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
                     flags, workspace, workspace_bytes, stream);
 }
 
+la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                       const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                       const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, void *stream) {
+  la_status s;
+  const la_tensor *ts[7] = {q, k, v, dout, dq, dk, dv};
+  const char *names[7] = {"q", "k", "v", "dout", "dq", "dk", "dv"};
+  for (int i = 0; i < 7; ++i)
+    if ((s = check_tensor(ts[i], names[i])) != LA_OK) return s;
+  for (int i = 1; i < 7; ++i) {
+    if (ts[i]->dtype != q->dtype) return fail(LA_ERR_INVALID_ARG, "%s must have q's dtype", names[i]);
+    if (ts[i]->B != q->B || ts[i]->T != q->T || ts[i]->H != q->H)
+      return fail(LA_ERR_INVALID_ARG, "%s disagrees with q on B, T or H", names[i]);
+  }
+  if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
+  if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
+  if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
+  if (cu_seqlens) {
+    if (q->B != 1) return fail(LA_ERR_INVALID_ARG, "packed batches (cu_seqlens) need B == 1");
+    if (n_seqs < 0) return fail(LA_ERR_INVALID_ARG, "n_seqs is negative");
+  } else if (n_seqs != q->B) {
+    return fail(LA_ERR_INVALID_ARG, "n_seqs must equal B when cu_seqlens is NULL");
+  }
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128)
+    return fail(LA_ERR_UNSUPPORTED, "chunk %d not in {16, 32, 64, 128}", chunk);
+  if (!head_dim_ok(q->D) || !head_dim_ok(v->D))
+    return fail(LA_ERR_UNSUPPORTED, "head dims (%lld, %lld) not in {16, 32, 64, 128, 256}",
+                (long long)q->D, (long long)v->D);
+  BwdArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.dout = view(dout);
+  a.dq = view(dq);
+  a.dk_ = view(dk);
+  a.dv_ = view(dv);
+  a.gamma = gamma;
+  a.cu_seqlens = cu_seqlens;
+  a.T = q->T;
+  a.n_seqs = n_seqs;
+  a.H = (int)q->H;
+  a.dk = (int)q->D;
+  a.dv = (int)v->D;
+  a.chunk = chunk;
+  a.phi = phi;
+  a.dtype = q->dtype;
+  int device = 0;
+  cudaError_t err = cudaGetDevice(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  if (a.n_seqs == 0 || a.T == 0 || q->B == 0) return ok();
+  if (!bwd_supported(a, device))
+    return fail(LA_ERR_UNSUPPORTED, "d_k %d x d_v %d does not fit the backward kernel's shared memory", a.dk,
+                a.dv);
+  err = launch_bwd(a, (cudaStream_t)stream);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
 la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
                   const la_tensor *out, int32_t phi, void *stream) {
   return step_common("la_step", q, k, v, gamma, nullptr, state, nullptr, out, phi, stream);

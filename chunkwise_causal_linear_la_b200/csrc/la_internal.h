@@ -44,6 +44,14 @@ struct StepArgs {
   int H, dk, dv, phi, dtype;
 };
 
+struct BwdArgs {
+  TensorView q, k, v, dout, dq, dk_, dv_;
+  const float *gamma;
+  const int32_t *cu_seqlens;  // NULL for dense batches
+  int64_t T, n_seqs;
+  int H, dk, dv, chunk, phi, dtype;
+};
+
 // Sets the calling thread's la_last_error() message and returns `status`.
 la_status report_error(la_status status, const char *msg);
 
@@ -53,6 +61,8 @@ int max_smem_optin(int device);
 
 // SIMT (CUDA-core, fp32 arithmetic) chunked forward.
 bool simt_supported(const ChunkArgs &a, int device);
+bool bwd_supported(const BwdArgs &a, int device);
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 
 // One-token decode step.

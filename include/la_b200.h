@@ -231,6 +231,31 @@ LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_
                                float *state, float *z, const la_tensor *out, int32_t phi, void *stream);
 
 /*
+ * la_bwd_chunk -- backward of the unnormalised chunked forward: the gradients
+ * of a loss with respect to q, k, v, given its gradient dout at the output.
+ * The forward is the recurrence of "1.6 长上下文与高效注意力", section 线性注意力,
+ * with the per-head decay, S_t = gamma S_{t-1} + v_t phi(k_t)^T, o_t = S_t phi(q_t);
+ * its adjoint is
+ *     dphi(q)_t = S_t^T dout_t,   G_t = dout_t phi(q_t)^T + gamma G_{t+1},
+ *     dphi(k)_t = G_t^T v_t,      dv_t = G_t phi(k_t),
+ * and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k) (phi' = 1, or 1 / e^x for
+ * elu + 1 at x > 0 / x <= 0).
+ *   q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi  as for la_fwd_chunk (the
+ *               forward's inputs; states start at zero, gamma is not differentiated).
+ *   dout        [B, T, H, d_v], q's dtype: the gradient at `out`.
+ *   dq, dk      [B, T, H, d_k]; dv [B, T, H, d_v]; q's dtype; written for every
+ *               token that belongs to a sequence.
+ * Runs on CUDA cores in fp32 (bf16 or f32 inputs, results rounded once).
+ * LA_ERR_UNSUPPORTED when the state (d_k x d_v fp32) and one chunk's tiles do
+ * not fit in shared memory (d_k = d_v = 128 fits; 256 does not).  The
+ * normalised forward has no backward here.  Other errors as for la_fwd_chunk.
+ */
+LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                              const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
+                              int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv,
+                              void *stream);
+
+/*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device
  * memory.  (An addition of this library; the pages have no counterpart.)
  *
