@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "causal linear-attn fwd tokens/s and % of roofline (bf16, B200)"
+METRIC_BWD = "causal linear-attn bwd (dq, dk, dv) tokens/s and % of roofline (bf16, B200)"
 
 
 def _peaks():
@@ -171,14 +172,19 @@ def _traffic(workload_name, units_scale):
     return None
 
 
-def _oracle_run(oracle, w, q, k, v, gamma, g=None):
-    """The oracle's recurrence for workload w (per-head gamma, or the per-token log decay g)."""
+def _oracle_run(oracle, w, q, k, v, gamma, g=None, bwd=False):
+    """The oracle's recurrence for workload w (per-head gamma, or the per-token log decay g);
+    bwd: its adjoint for an all-ones output gradient."""
+    if bwd:
+        import torch
+
+        return oracle.backward(q, k, v, torch.ones_like(v), gamma, phi=w.phi)
     if g is not None:
         return oracle.recurrent_gated(q, k, v, g, phi=w.phi, normalize=w.normalize)[:2]
     return oracle.recurrent(q, k, v, gamma, phi=w.phi, normalize=w.normalize)
 
 
-def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1):
+def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1, bwd=False):
     """Time the float64 oracle on a prefix of the first nseq sequences (all heads).
 
     Returns (tokens/s, tokens per sequence, secs, threads)."""
@@ -201,14 +207,14 @@ def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1):
     for target in (1.0, budget_s):
         qs, ks, vs, gs = sample(n)
         t0 = time.perf_counter()
-        _oracle_run(oracle, w, qs, ks, vs, g, gs)
+        _oracle_run(oracle, w, qs, ks, vs, g, gs, bwd)
         dt = max(time.perf_counter() - t0, 1e-4)
         n = int(min(T, max(n, n * target / dt)))
     if max_tokens:
         n = min(n, max_tokens)
     qs, ks, vs, gs = sample(n)
     t0 = time.perf_counter()
-    _oracle_run(oracle, w, qs, ks, vs, g, gs)
+    _oracle_run(oracle, w, qs, ks, vs, g, gs, bwd)
     secs = time.perf_counter() - t0
     return nseq * n / secs, n, secs, oracle.max_threads()
 
@@ -316,6 +322,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward (la_bwd_chunk) on the workload instead of the forward")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (la_step) and print its JSON object")
     args = ap.parse_args()
@@ -360,9 +368,19 @@ def main():
     wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
 
     gd = x.get("g")  # data-dependent log decay (gated workloads)
+    if args.bwd:
+        if gd is not None or w.normalize:
+            raise SystemExit("--bwd covers the unnormalised per-head-decay workloads")
+        from chunkwise_causal_linear_la_b200.workloads import make_dout
+
+        dout = make_dout(v, seed=rank_seed(rank))
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
 
     def step():
-        if gd is not None:
+        if args.bwd:
+            la.la_bwd_chunk(q, k, v, dout, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0], dk=grads[1],
+                            dv=grads[2], stream=stream)
+        elif gd is not None:
             la.la_fwd_chunk_gated(q, k, v, gd, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize,
                                   out=out, final_state=fs, workspace=wsbuf, stream=stream)
         else:
@@ -401,7 +419,14 @@ def main():
         [e_all0.elapsed_time(e_all1), statistics.mean(a.elapsed_time(b) for a, b in evs)], dev, dist)
     value = aggregate_rate(tokens, args.steps, ws, elapsed_ms)
     alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
+    if args.bwd:  # read q, k, v, dout; write dq, dk, dv (no final state); three forward-shaped passes of flops
+        e_ = 2 if w.dtype == "bf16" else 4
+        alg_bytes = tokens * w.H * e_ * (4 * w.d_k + 3 * w.d_v)
+        alg_flops = 3 * alg_flops
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    # kernels launched per step: segmented sequences take a state pass, a scan and the output pass; the
+    # backward takes three forward-shaped passes (plus four elementwise kernels with elu + 1)
+    launches_per_step = (7 if w.phi == "elu1" else 3) if args.bwd else (3 if nws > 0 else 1)
     clocks = sampler.summary(t_wall0, t_wall1)
 
     # ---- parity on sampled (sequence, head) slices, float64 oracle (rank 0)
@@ -415,7 +440,15 @@ def main():
         torch.cuda.synchronize()
         sl = [(0, 0), (B - 1, w.H - 1)] if cu is None else [(0, 0)]
         worst = 0.0
-        for b, h in sl:
+        for b, h in sl if args.bwd else []:  # backward: dq, dk, dv against the oracle's adjoint
+            s0, e0_ = (0, T) if cu is None else (int(cu[0]), int(cu[1]))
+            bb = b if cu is None else 0
+            cut = lambda t: t[bb:bb + 1, s0:e0_, h:h + 1].cpu()  # noqa: E731
+            refs = oracle.backward(cut(q), cut(k), cut(v), cut(dout), [float(g[h])], phi=w.phi)
+            for got, ref in zip(grads, refs):
+                o = cut(got).float().numpy()
+                worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))))
+        for b, h in [] if args.bwd else sl:
             if cu is None:
                 qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
                 gs = None if gd is None else gd[b:b + 1, :, h:h + 1].double().cpu().numpy()
@@ -436,16 +469,18 @@ def main():
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     inputs = (q, k, v) if gd is None else (q, k, v, gd)
+    if args.bwd:
+        inputs = (q, k, v, dout)
+    outputs = grads if args.bwd else (out, fs)
     hosts = [t.cpu().pin_memory() for t in inputs]
-    oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    fh = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outputs]
 
     def e2e_step():
         for dst, src in zip(inputs, hosts):
             dst.copy_(src, non_blocking=True)
         step()
-        oh.copy_(out, non_blocking=True)
-        fh.copy_(fs, non_blocking=True)
+        for dst, src in zip(host_out, outputs):
+            dst.copy_(src, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -459,7 +494,7 @@ def main():
     torch.cuda.synchronize()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev, dist)
     h2d = sum(t.numel() * t.element_size() for t in inputs)
-    d2h = out.numel() * out.element_size() + fs.numel() * fs.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outputs)
     e2e = {"value": aggregate_rate(tokens, args.e2e_steps, ws, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
@@ -473,23 +508,25 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         nseq = 1 if cu is not None else B
-        rate, n, secs, threads = _oracle_rate(w, x, budget_s=15.0, nseq=nseq)
+        rate, n, secs, threads = _oracle_rate(w, x, budget_s=15.0, nseq=nseq, bwd=args.bwd)
         cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": "%d sequence(s) of %s, all %d heads, first %d tokens each (float64 recurrence, %.1f s)"
-                         % (nseq, w.name, w.H, n, secs)}
+               "sample": "%d sequence(s) of %s, all %d heads, first %d tokens each (float64 %s, %.1f s)"
+                         % (nseq, w.name, w.H, n, "adjoint of the recurrence" if args.bwd else "recurrence", secs)}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "metric": METRIC_BWD if args.bwd else METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype), "data": "synthetic",
             "config": _config(w, ws),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": _traffic(w.name, 1.0),
+                         "frac": achieved / hbm_peak, "traffic": None if args.bwd else _traffic(w.name, 1.0),
                          "peak_kind": "%s (burst copy bandwidth)" % peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
-                         "launch_ms": launch_ms, "kernel": "chunk_tc_kernel"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+                         "launch_ms": launch_ms,
+                         "kernel": "chunk_tc_kernel (3 passes: forward + 2 in reverse time)" if args.bwd
+                         else "chunk_tc_kernel"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
             "parity": parity, "extra": extra,
         }
         print(json.dumps(line), flush=True)

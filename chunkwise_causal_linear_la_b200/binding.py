@@ -75,7 +75,7 @@ def load_library(path: str = LIB_PATH):
     lib.la_step_norm.restype = i32
     lib.la_step_gated.argtypes = [P, P, P, vp, vp, vp, P, i32, vp]
     lib.la_step_gated.restype = i32
-    lib.la_bwd_chunk.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, vp]
+    lib.la_bwd_chunk.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, i32, vp]
     lib.la_bwd_chunk.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
@@ -271,7 +271,7 @@ def la_step_gated(q, k, v, g, state, z=None, out=None, phi="identity", stream=No
 
 
 def la_bwd_chunk(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="identity", dq=None, dk=None, dv=None,
-                 stream=None):
+                 flags=LA_FLAG_NONE, stream=None):
     """Gradients (dq, dk, dv) of the unnormalised forward given dout (see la_bwd_chunk in
     include/la_b200.h).  All tensors [B, T, H, d], one dtype."""
     lib = load_library()
@@ -285,6 +285,6 @@ def la_bwd_chunk(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="identity"
     t = [describe(x) for x in (q, k, v, dout, dq, dk, dv)]
     st = lib.la_bwd_chunk(*(ctypes.byref(x) for x in t[:4]), gamma.data_ptr(),
                           None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
-                          *(ctypes.byref(x) for x in t[4:]), _stream(stream))
+                          *(ctypes.byref(x) for x in t[4:]), int(flags), _stream(stream))
     _check(lib, st, "la_bwd_chunk")
     return dq, dk, dv

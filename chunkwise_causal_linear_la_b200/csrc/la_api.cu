@@ -147,6 +147,8 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
   a.phi = phi;
   a.normalize = normalize ? 1 : 0;
   a.dtype = q->dtype;
+  a.rev = 0;
+  a.noseg = 0;
 
   const size_t need = la_fwd_chunk_workspace_size(a.B, a.T, a.H, a.dk, a.dv, n_seqs, cu_seqlens != nullptr,
                                                   chunk, a.dtype, flags);
@@ -307,7 +309,8 @@ la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
 
 la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                        const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
-                       const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, void *stream) {
+                       const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
+                       void *stream) {
   la_status s;
   const la_tensor *ts[7] = {q, k, v, dout, dq, dk, dv};
   const char *names[7] = {"q", "k", "v", "dout", "dq", "dk", "dv"};
@@ -323,6 +326,7 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
   if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
+  if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (cu_seqlens) {
     if (q->B != 1) return fail(LA_ERR_INVALID_ARG, "packed batches (cu_seqlens) need B == 1");
     if (n_seqs < 0) return fail(LA_ERR_INVALID_ARG, "n_seqs is negative");
@@ -356,10 +360,76 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   cudaError_t err = cudaGetDevice(&device);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
   if (a.n_seqs == 0 || a.T == 0 || q->B == 0) return ok();
+  cudaStream_t st = (cudaStream_t)stream;
+
+  // Tensor cores: the backward is three forward passes on rearranged operands
+  // (each a sum of the forward's form, two of them anti-causal, run in reverse
+  // time):  dphi(q) = fwd(dout, v, phi(k));  dphi(k) = rev(v, dout, phi(q));
+  // dv = rev(phi(k), phi(q), dout).  With elu + 1 the operands the forward
+  // reads untransformed are made phi(x) first (in dq / dv, which are written
+  // after they are read), and phi' scales the q and k gradients.
+  const bool elu = phi == LA_PHI_ELU1;
+  ChunkArgs f;
+  f.gamma = gamma;
+  f.g = nullptr;
+  f.cu_seqlens = cu_seqlens;
+  f.final_state = nullptr;
+  f.final_z = nullptr;
+  f.B = q->B;
+  f.T = q->T;
+  f.n_seqs = n_seqs;
+  f.H = (int)q->H;
+  f.chunk = 64;
+  f.normalize = 0;
+  f.dtype = q->dtype;
+  f.noseg = 1;
+  auto setup = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
+                   int rev) {
+    f.q = view(qq);
+    f.k = view(kk);
+    f.v = view(vv);
+    f.out = oo->data;
+    f.o_sb = oo->stride_b;
+    f.o_st = oo->stride_t;
+    f.o_sh = oo->stride_h;
+    f.dk = (int)qq->D;
+    f.dv = (int)vv->D;
+    f.phi = ph;
+    f.rev = rev;
+    return tc_supported(f);
+  };
+  bool tc = q->dtype == LA_BF16 && chunk == 64 && !(flags & LA_FLAG_SIMT) && (!elu || q->D == v->D);
+  if (tc) tc = setup(v, dout, q, dk, 0, 1) && setup(dout, v, k, dq, 0, 0) && setup(k, q, dout, dv, 1, 1);
+  if (tc) {
+    const char *why = nullptr;
+    auto run = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
+                   int rev) -> cudaError_t {
+      setup(qq, kk, vv, oo, ph, rev);
+      return launch_chunk_tc(f, nullptr, 0, st, &why);
+    };
+    const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D;
+    if (elu) {
+      if ((err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
+          (err = run(v, dout, dq, dk, 0, 1)) != cudaSuccess ||
+          (err = launch_mul_dphi(view(k), view(dk), B, T, H, Dk, q->dtype, st)) != cudaSuccess ||
+          (err = launch_phi_copy(view(k), view(dv), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
+          (err = run(dout, v, dv, dq, 0, 0)) != cudaSuccess ||
+          (err = launch_mul_dphi(view(q), view(dq), B, T, H, Dk, q->dtype, st)) != cudaSuccess ||
+          (err = run(k, q, dout, dv, 1, 1)) != cudaSuccess)
+        return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
+                    why ? why : "");
+    } else {
+      if ((err = run(v, dout, q, dk, 0, 1)) != cudaSuccess || (err = run(dout, v, k, dq, 0, 0)) != cudaSuccess ||
+          (err = run(k, q, dout, dv, 0, 1)) != cudaSuccess)
+        return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
+                    why ? why : "");
+    }
+    return ok();
+  }
   if (!bwd_supported(a, device))
     return fail(LA_ERR_UNSUPPORTED, "d_k %d x d_v %d does not fit the backward kernel's shared memory", a.dk,
                 a.dv);
-  err = launch_bwd(a, (cudaStream_t)stream);
+  err = launch_bwd(a, st);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(err));
   return ok();
 }

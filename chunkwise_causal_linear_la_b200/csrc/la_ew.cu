@@ -1,0 +1,114 @@
+// la_ew.cu -- elementwise steps of the backward pass with phi = elu + 1.
+//
+// The backward runs on the forward kernel (see la_bwd_chunk): operands that
+// the forward kernel reads untransformed must hold phi(x) already, and the
+// gradients of phi(q), phi(k) are turned into those of q, k by phi'(x) = 1 for
+// x > 0 and e^x otherwise ("1.6 长上下文与高效注意力", section 线性注意力:
+// phi(x) = elu(x) + 1).  Both kernels stream a [B, T, H, D] tensor once.
+#include <cuda_bf16.h>
+
+#include "la_common.cuh"
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+constexpr int kEwThreads = 256;
+
+// One thread per 16-byte vector of a row (VW elements; D is a multiple of VW):
+// vector e is column block e mod (D / VW) of row e / (D / VW), rows ordered
+// (b, t, h).
+template <typename T>
+struct Vec {
+  static constexpr int VW = 16 / sizeof(T);
+};
+
+template <typename T>
+__device__ __forceinline__ void row_of(int64_t e, int64_t nvr, int64_t T_, int64_t H, int64_t &b, int64_t &t,
+                                       int64_t &h, int &col) {
+  const int64_t row = e / nvr;
+  col = (int)(e - row * nvr) * Vec<T>::VW;
+  h = row % H;
+  const int64_t bt = row / H;
+  t = bt % T_;
+  b = bt / T_;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) phi_kernel(TensorView src, TensorView dst, int64_t T_, int64_t H,
+                                                          int64_t D, int64_t nvec, int phi) {
+  constexpr int VW = Vec<T>::VW;
+  const int64_t nvr = D / VW;
+  for (int64_t e = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; e < nvec; e += (int64_t)gridDim.x * kEwThreads) {
+    int64_t b, t, h;
+    int col;
+    row_of<T>(e, nvr, T_, H, b, t, h, col);
+    const T *s = (const T *)src.data + b * src.sb + t * src.st + h * src.sh + col;
+    T *o = (T *)dst.data + b * dst.sb + t * dst.st + h * dst.sh + col;
+    uint4 x = *reinterpret_cast<const uint4 *>(s);
+    T *xv = reinterpret_cast<T *>(&x);
+#pragma unroll
+    for (int u = 0; u < VW; ++u) xv[u] = from_f32<T>(feature_map(to_f32<T>(xv[u]), phi));
+    *reinterpret_cast<uint4 *>(o) = x;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) mul_dphi_kernel(TensorView x, TensorView grad, int64_t T_, int64_t H,
+                                                               int64_t D, int64_t nvec) {
+  constexpr int VW = Vec<T>::VW;
+  const int64_t nvr = D / VW;
+  for (int64_t e = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; e < nvec; e += (int64_t)gridDim.x * kEwThreads) {
+    int64_t b, t, h;
+    int col;
+    row_of<T>(e, nvr, T_, H, b, t, h, col);
+    const uint4 xr = *reinterpret_cast<const uint4 *>((const T *)x.data + b * x.sb + t * x.st + h * x.sh + col);
+    uint4 *gp = reinterpret_cast<uint4 *>((T *)grad.data + b * grad.sb + t * grad.st + h * grad.sh + col);
+    uint4 gr = *gp;
+    const T *xv = reinterpret_cast<const T *>(&xr);
+    T *gv = reinterpret_cast<T *>(&gr);
+#pragma unroll
+    for (int u = 0; u < VW; ++u) {
+      const float xf = to_f32<T>(xv[u]);
+      gv[u] = from_f32<T>(to_f32<T>(gv[u]) * (xf > 0.f ? 1.f : expf(xf)));
+    }
+    *gp = gr;
+  }
+}
+
+unsigned ew_grid(int64_t n) {
+  const int64_t blocks = (n + kEwThreads - 1) / kEwThreads;
+  return (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
+}
+
+}  // namespace
+
+// Both need 16-byte aligned rows (la_tensor's pointer and stride rules) and
+// D a multiple of the vector width (every supported head dim is).
+cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T, int64_t H, int64_t D, int phi,
+                            int dtype, cudaStream_t stream) {
+  const int vw = dtype == LA_F32 ? 4 : 8;
+  if (D % vw) return cudaErrorInvalidValue;
+  const int64_t n = B * T * H * (D / vw);
+  if (n == 0) return cudaSuccess;
+  if (dtype == LA_F32)
+    phi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
+  else
+    phi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
+                            cudaStream_t stream) {
+  const int vw = dtype == LA_F32 ? 4 : 8;
+  if (D % vw) return cudaErrorInvalidValue;
+  const int64_t n = B * T * H * (D / vw);
+  if (n == 0) return cudaSuccess;
+  if (dtype == LA_F32)
+    mul_dphi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
+  else
+    mul_dphi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
+  return cudaGetLastError();
+}
+
+}  // namespace la

@@ -30,6 +30,8 @@ struct ChunkArgs {
   int64_t B, T, n_seqs;
   int H, dk, dv, chunk, phi, normalize;
   int dtype;  // la_dtype of q, k, v, out
+  int rev;    // 1: reverse time (tensor-core kernel only; used by the backward pass)
+  int noseg;  // 1: never split sequences into segments (no workspace)
 };
 
 struct StepArgs {
@@ -62,6 +64,10 @@ int max_smem_optin(int device);
 // SIMT (CUDA-core, fp32 arithmetic) chunked forward.
 bool simt_supported(const ChunkArgs &a, int device);
 bool bwd_supported(const BwdArgs &a, int device);
+cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T, int64_t H, int64_t D, int phi,
+                            int dtype, cudaStream_t stream);
+cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
+                            cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 

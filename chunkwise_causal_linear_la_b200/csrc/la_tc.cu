@@ -273,11 +273,19 @@ __device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int
   }
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED>
+// REV: reverse time.  The sequence is walked from its end: chunk c is the
+// window of C tokens ending (C c) tokens before the end, and inside it token
+// row i stands for position i' = C - 1 - i of the reversed sequence.  Every
+// formula of the forward then holds in the primed indices (valid rows
+// i' < C', causal j' <= i'); the tiles stay in natural row order, so the
+// products need no change.  This runs the anti-causal sums of the backward
+// pass (sum over i >= j) on the same kernel.
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED, bool REV>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
   using G = Cfg<DK, DVT, C, NS>;
+  static_assert(!(REV && (NORM || GATED)), "reverse time is built for the unnormalised per-head decay");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
@@ -313,9 +321,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     start = 0;
     len = a.T;
   }
+  // natural end of the walk (reverse time): the segment starts c0 tokens before the sequence end
+  int64_t rend = start + len;
   if (a.G > 1) {  // this CTA's segment of the sequence
     const int64_t c0 = (int64_t)seg * a.segC * C;
     start += c0;
+    rend -= c0;
     len = max((int64_t)0, min(len - c0, (int64_t)a.segC * C));
   }
   const bool has_init = MODE == 0 && a.G > 1 && seg > 0;  // start state from the scan
@@ -359,6 +370,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto out_phase = [&](int c) -> uint32_t { return (vd_mode && !G::VD_DB) ? (c & 1) : ((c >> 1) & 1); };
 
   auto chunk_len = [&](int c) -> int { return (int)min((int64_t)C, len - (int64_t)c * C); };
+  // first (natural) token of chunk c's window; in reverse time it may lie before
+  // the sequence start (those rows are masked, or read as zeros by TMA)
+  auto tok0 = [&](int c) -> int64_t { return REV ? rend - (int64_t)(c + 1) * C : start + (int64_t)c * C; };
+  // row of the (reversed) sequence that tile row r stands for
+  auto lrow = [&](int r) -> int { return REV ? C - 1 - r : r; };
   auto q_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES; };
   auto k_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + G::QK_BYTES; };
   auto v_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + 2 * G::QK_BYTES; };
@@ -375,7 +391,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int s = c % NS, k = c / NS;
         if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1, c)) break;
         mbar_arrive_expect_tx(bars + G::B_FULL + s, MODE == 1 ? G::STAGE_BYTES - G::QK_BYTES : G::STAGE_BYTES);
-        const int t0 = (int)(start + (int64_t)c * C);
+        const int t0 = (int)tok0(c);
         for (int kb = 0; kb < G::KB; ++kb) {
           if (MODE == 0) tma_load_4d(q_tile(s) + kb * G::SLAB, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
           tma_load_4d(k_tile(s) + kb * G::SLAB, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bidx);
@@ -561,7 +577,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               const float b1 = __shfl_sync(0xffffffffu, bhi, j & 31);
               wv[m] = j < Cp ? exp_fast(blast - (j < 32 ? b0 : b1)) : 0.f;
             } else {
-              wv[m] = j < Cp ? pw[Cp - 1 - j] : 0.f;
+              const int jl = lrow(j);
+              wv[m] = jl < Cp ? pw[Cp - 1 - jl] : 0.f;
             }
           }
         };
@@ -789,7 +806,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bi = dt[i];
         gi = exp_fast(bi);
       } else {
-        gi = pw[i + 1];
+        gi = pw[lrow(i) + 1];
       }
       float zq = 0.f;
       if (NORM) {
@@ -801,8 +818,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, r);
       tmem_wait_ld();
       float f[32];
-      const bool row_ok = i < Cp;
-      if (!vd_mode) {
+      const int il = lrow(i);  // row of the (reversed) sequence
+      const bool row_ok = il < Cp;
+      if (REV) {  // causal in the reversed order: j' <= i', i.e. j >= i
+        if (!vd_mode) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e >= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = hf * 32 + e;
+            f[e] = (j >= i && row_ok) ? __uint_as_float(r[e]) * pw[j - i] : 0.f;
+          }
+        }
+      } else if (!vd_mode) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e <= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
       } else if (GATED) {  // P_ij = A_ij exp(b_i - b_j)
@@ -836,7 +865,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
       }
       if (!row_ok) return 0.f;
-      if (!NORM) return vd_mode ? 1.f : 1.f / pw[Cp - 1 - i];
+      if (!NORM) return vd_mode ? 1.f : 1.f / pw[Cp - 1 - il];
       return 1.f / fmaf(vd_mode ? gi : pw[Cp], zq, rowsum);
     };
 
@@ -847,7 +876,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t oph = out_phase(c);
       if (!wait_bar_warp(sy, G::B_OFULL + ob, oph, c)) return false;
       tc_fence_after();
-      uint8_t *orow = obase + 2 * ((start + (int64_t)c * C + i) * a.o_st);
+      const int64_t otok = tok0(c) + i;  // natural token of this row (in reverse time, may precede the sequence)
       const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
 #pragma unroll 1
       for (int pass = 0; pass < DVT / 64; ++pass) {
@@ -872,8 +901,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc_fence_before();
           mbar_arrive(bars + G::B_OEMPTY + ob);
         }
-        if (i < Cp) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + 2 * (hf * (DVT / 2) + pass * 32));
+        if (lrow(i) < Cp) {
+          uint4 *dst = reinterpret_cast<uint4 *>(obase + 2 * (otok * a.o_st + hf * (DVT / 2) + pass * 32));
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             dst[q] = make_uint4(pack2(o[8 * q], o[8 * q + 1]), pack2(o[8 * q + 2], o[8 * q + 3]),
@@ -1049,7 +1078,7 @@ __global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *ws_g, con
   }
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, bool GATED>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, bool GATED, bool REV>
 cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   using G = Cfg<DK, DVT, C, NS>;
   CUtensorMap mq, mk, mv;
@@ -1073,7 +1102,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.dv = a.dv;
   t.phi = a.phi;
   t.normalize = a.normalize;
-  const SegPlan plan = seg_plan(a.n_seqs, a.T, a.H, a.dv / DVT, a.cu_seqlens != nullptr, C);
+  const SegPlan plan = a.noseg ? SegPlan{1, 0, 0} : seg_plan(a.n_seqs, a.T, a.H, a.dv / DVT, a.cu_seqlens != nullptr, C);
   const int64_t units = a.n_seqs * a.H * (a.dv / DVT);
   if (units == 0) return cudaSuccess;
   if (units * plan.G > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -1082,7 +1111,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.ws_s = nullptr;
   t.ws_z = nullptr;
   t.ws_g = nullptr;
-  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0, GATED>;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0, GATED, REV>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   if (plan.G > 1) {
@@ -1094,7 +1123,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
     t.ws_z = NORM ? t.ws_s + units * (plan.G - 1) * DK * DVT : nullptr;
     t.ws_g = GATED ? t.ws_s + units * (plan.G - 1) * (DK * DVT + DK) : nullptr;
     // pass 1: end state of every segment but the last, from a zero start
-    auto kst = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 1, GATED>;
+    auto kst = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 1, GATED, REV>;
     err = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     t.Gp = plan.G - 1;
@@ -1146,15 +1175,20 @@ template <int DK, int DVT, int NS, bool GATED>
 cudaError_t launch_shape_gated(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   // one instantiation per (normaliser, feature map, decay kind): each carries only its own code path
   if (a.normalize) {
-    return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true, GATED>(a, workspace, stream, why)
-                 : launch_cfg<DK, DVT, 64, NS, true, false, GATED>(a, workspace, stream, why);
+    return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true, GATED, false>(a, workspace, stream, why)
+                 : launch_cfg<DK, DVT, 64, NS, true, false, GATED, false>(a, workspace, stream, why);
   }
-  return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, GATED>(a, workspace, stream, why)
-               : launch_cfg<DK, DVT, 64, NS, false, false, GATED>(a, workspace, stream, why);
+  return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, GATED, false>(a, workspace, stream, why)
+               : launch_cfg<DK, DVT, 64, NS, false, false, GATED, false>(a, workspace, stream, why);
 }
 
 template <int DK, int DVT, int NS>
 cudaError_t launch_shape(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
+  if (a.rev) {  // reverse time (the backward pass): unnormalised, per-head decay
+    if (a.normalize || a.g) return cudaErrorInvalidValue;
+    return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, false, true>(a, workspace, stream, why)
+                 : launch_cfg<DK, DVT, 64, NS, false, false, false, true>(a, workspace, stream, why);
+  }
   return a.g ? launch_shape_gated<DK, DVT, NS, true>(a, workspace, stream, why)
              : launch_shape_gated<DK, DVT, NS, false>(a, workspace, stream, why);
 }

@@ -153,6 +153,13 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", T: Optional[int] = Non
     return x
 
 
+def make_dout(v: torch.Tensor, seed: int = 0) -> torch.Tensor:
+    """A seeded N(0, 1) output gradient shaped and typed like ``v`` (for the backward)."""
+    g = torch.Generator(device=v.device)
+    g.manual_seed(seed + 2)
+    return torch.randn(v.shape, generator=g, device=v.device, dtype=torch.float32).to(v.dtype)
+
+
 def make_decode_inputs(N, H, d_k, d_v, scale, state_std, gamma, seed=0, device="cpu",
                        dtype=torch.float32):
     """Decode inputs: q, k [N,H,d_k], v [N,H,d_v], state [N,H,d_k,d_v] fp32, gamma [H]."""

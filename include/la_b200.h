@@ -245,15 +245,26 @@ LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_
  *   dout        [B, T, H, d_v], q's dtype: the gradient at `out`.
  *   dq, dk      [B, T, H, d_k]; dv [B, T, H, d_v]; q's dtype; written for every
  *               token that belongs to a sequence.
- * Runs on CUDA cores in fp32 (bf16 or f32 inputs, results rounded once).
- * LA_ERR_UNSUPPORTED when the state (d_k x d_v fp32) and one chunk's tiles do
- * not fit in shared memory (d_k = d_v = 128 fits; 256 does not).  The
- * normalised forward has no backward here.  Other errors as for la_fwd_chunk.
+ *   flags       LA_FLAG_NONE or LA_FLAG_SIMT (force the CUDA-core kernel).
+ * Kernels: bf16 with chunk 64 and tensor-core head dims (as for la_fwd_chunk;
+ * with elu + 1 also d_k == d_v) runs as three tensor-core forward passes on
+ * rearranged operands:
+ *     dphi(q) = forward(q' = dout, k' = v, v' = phi(k))
+ *     dphi(k) = forward in reverse time (q' = v, k' = dout, v' = phi(q))
+ *     dv      = forward in reverse time (q' = phi(k), k' = phi(q), v' = dout)
+ * (each sum above has exactly that form; reverse time turns sum_{i>=j} into
+ * the forward's sum_{j<=i}); bf16 operands and fp32 accumulation as in the
+ * forward.  Every other shape, f32, and LA_FLAG_SIMT run one CUDA-core kernel
+ * in fp32; it needs the d_k x d_v fp32 state and one chunk's tiles to fit in
+ * shared memory (d_k = d_v = 128 fits; 256 does not: LA_ERR_UNSUPPORTED).
+ * Tokens outside every sequence of a packed batch may be overwritten in dq,
+ * dk, dv.  The normalised forward has no backward here.  Other errors as for
+ * la_fwd_chunk.
  */
 LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                               const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
                               int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv,
-                              void *stream);
+                              int32_t flags, void *stream);
 
 /*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device

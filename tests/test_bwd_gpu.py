@@ -80,10 +80,54 @@ def test_bwd_headline_shape_sample(la, oracle_mod):
     gen.manual_seed(3)
     dout = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16)
     dev = torch.device("cuda")
-    dq, dk, dv = la.la_bwd_chunk(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), dout.to(dev), x["gamma"].to(dev))
+    dq, dk, dv = la.la_bwd_chunk(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), dout.to(dev), x["gamma"].to(dev))  # tensor cores
     torch.cuda.synchronize()
     for b, h in [(0, 0), (7, 15)]:
         sl = lambda t: t[b:b + 1, :, h:h + 1]  # noqa: E731
         rq, rk, rv = oracle_mod.backward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(dout), [float(x["gamma"][h])])
         for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
             assert slice_rel_err(to_np(sl(got)), ref, seq_slices(1, 2048)) < TOL[torch.bfloat16]
+
+
+# ---------------------------------------------------------------- tensor-core backward
+# bf16, chunk 64, d_k = d_v in {128, 256}: three tensor-core forward passes,
+# two of them in reverse time (windows at negative token offsets, masked rows
+# of the previous sequence in packed batches).
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("T", [1, 65, 300])
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+def test_bwd_tc_shapes(la, oracle_mod, d, T, phi):
+    q, k, v, dout = _inputs(2, T, 2, d, d, torch.bfloat16, T + d)
+    _check(la, oracle_mod, q, k, v, dout, torch.tensor([0.97, 1.0]), phi=phi)
+
+
+@pytest.mark.parametrize("gamma", [0.0, 0.3, 0.9, 1.0])
+def test_bwd_tc_gammas(la, oracle_mod, gamma):
+    """gamma <= 0.3 takes the forward kernel's value-decay mode."""
+    q, k, v, dout = _inputs(1, 200, 2, 128, 128, torch.bfloat16, 11)
+    _check(la, oracle_mod, q, k, v, dout, torch.tensor([gamma, 0.99]), phi="elu1")
+
+
+def test_bwd_tc_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 2, 128, 128, torch.bfloat16, 13)
+    _check(la, oracle_mod, q, k, v, dout, torch.tensor([0.9, 1.0]), cu=cu)
+    _check(la, oracle_mod, q, k, v, dout, torch.tensor([0.99, 0.5]), cu=cu, phi="elu1")
+
+
+def test_bwd_tc_matches_simt(la):
+    q, k, v, dout = _inputs(2, 300, 2, 128, 128, torch.bfloat16, 15)
+    dev = torch.device("cuda")
+    g = torch.tensor([0.95, 1.0], device=dev)
+    args = [x.to(dev) for x in (q, k, v, dout)]
+    a = la.la_bwd_chunk(*args, g, phi="elu1")
+    b = la.la_bwd_chunk(*args, g, phi="elu1", flags=la.LA_FLAG_SIMT)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert slice_rel_err(to_np(x), to_np(y), seq_slices(2, 300)) < TOL[torch.bfloat16]
+
+
+def test_bwd_device_error_word_clear(la):
+    assert la.device_error(reset=True) == (0, 0)
