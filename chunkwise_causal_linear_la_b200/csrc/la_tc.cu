@@ -410,6 +410,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       constexpr uint32_t ID_M3 = idesc_bf16_f32(C, DVT, 0, 1);
       constexpr uint32_t ID_M4 = idesc_bf16_f32(128, DVT, 1, 1);
       const uint64_t dsb = smem_desc_sw128(smem_u32(sb_tile), G::SB_SLAB, 1024);
+      // operand descriptors of stage 0 (stage s adds s * STAGE_BYTES / 16 to the
+      // start-address field, which cannot carry: shared addresses are < 256 KB)
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(q_tile(0)), 16, 1024);          // K-major
+      const uint64_t dkk0 = smem_desc_sw128(smem_u32(k_tile(0)), 16, 1024);         // K-major (scores)
+      const uint64_t dkm0 = smem_desc_sw128(smem_u32(k_tile(0)), G::SLAB, 1024);    // MN-major (state update)
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(v_tile(0)), G::SLAB, 1024);
+      const uint64_t dvd = smem_desc_sw128(smem_u32(vd_tile), G::SLAB, 1024);
+      const uint64_t dp0 = smem_desc_sw128(smem_u32(p_tile(0)), 16, 1024);
+      auto stage_off = [](int s) -> uint64_t { return (uint64_t)(s * (G::STAGE_BYTES >> 4)); };
       int m1_issued = 0;
       // M1 of chunk c: scores A[c%2] = qh kd^T
       auto issue_scores = [&](int c) -> bool {
@@ -418,8 +427,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // by the score step of chunk c-2, whose P tile this thread already waited for
         if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) return false;
         tc_fence_after();
-        const uint64_t dq = smem_desc_sw128(smem_u32(q_tile(s)), 16, 1024);
-        const uint64_t dk = smem_desc_sw128(smem_u32(k_tile(s)), 16, 1024);
+        const uint64_t dq = dq0 + stage_off(s);
+        const uint64_t dk = dkk0 + stage_off(s);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
@@ -444,8 +453,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) break;
           if (c > 0 && !wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
           tc_fence_after();
-          const uint64_t dvu = smem_desc_sw128(smem_u32(vd_mode ? vd_tile : v_tile(s)), G::SLAB, 1024);
-          const uint64_t dkd = smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
+          const uint64_t dvu = vd_mode ? dvd : dv0 + stage_off(s);
+          const uint64_t dkd = dkm0 + stage_off(s);
 #pragma unroll
           for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
@@ -467,15 +476,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int s = c % NS, b = c & 1;
         const int ob = out_buf(c);
         const uint32_t oph = out_phase(c);
-        const uint64_t dq = smem_desc_sw128(smem_u32(q_tile(s)), 16, 1024);
-        const uint64_t dv = smem_desc_sw128(smem_u32(v_tile(s)), G::SLAB, 1024);
-        const uint64_t dkd = smem_desc_sw128(smem_u32(k_tile(s)), G::SLAB, 1024);
+        const uint64_t dq = dq0 + stage_off(s);
+        const uint64_t dv = dv0 + stage_off(s);
+        const uint64_t dkd = dkm0 + stage_off(s);
         // M4: this chunk's state update U = kd^T V (value decay: kh^T vd)
         if (c > 0) {
           if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
           tc_fence_after();
         }
-        const uint64_t dvu = smem_desc_sw128(smem_u32(vd_mode ? vd_tile : v_tile(s)), G::SLAB, 1024);
+        const uint64_t dvu = vd_mode ? dvd : dv;
 #pragma unroll
         for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
@@ -503,7 +512,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
         tc_fence_after();
-        const uint64_t dp = smem_desc_sw128(smem_u32(p_tile(b)), 16, 1024);
+        const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
