@@ -426,7 +426,9 @@ def main():
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
     # kernels launched per step: segmented sequences take a state pass, a scan and the output pass; the
     # backward takes three forward-shaped passes (plus four elementwise kernels with elu + 1)
-    launches_per_step = (7 if w.phi == "elu1" else 3) if args.bwd else (3 if nws > 0 else 1)
+    # (a packed batch with a workspace has its longest-first order computed first: 2 launches)
+    launches_per_step = (7 if w.phi == "elu1" else 3) if args.bwd else (
+        (2 if cu is not None else 3) if nws > 0 else 1)
     clocks = sampler.summary(t_wall0, t_wall1)
 
     # ---- parity on sampled (sequence, head) slices, float64 oracle (rank 0)

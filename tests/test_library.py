@@ -82,6 +82,10 @@ def test_workspace_size_segment_plan(lib):
     assert ws(32, 2048, 4, 256, 256, 32, 0, 64, 1, 0) == 0
     # packed batches are not segmented; nor are shapes the tensor cores do not run
     assert ws(1, 5000, 2, 128, 128, 1, 1, 64, 1, 0) == 0
+    # packed batches of 2 .. 4096 sequences keep their longest-first order (int32 each, 256-byte blocks)
+    assert ws(1, 77431, 8, 128, 128, 64, 1, 64, 1, 0) == 256
+    assert ws(1, 77431, 8, 128, 128, 65, 1, 64, 1, 0) == 512
+    assert ws(1, 77431, 8, 128, 128, 5000, 1, 64, 1, 0) == 0
     assert ws(1, 5000, 2, 64, 64, 1, 0, 64, 1, 0) == 0
 
 
