@@ -179,7 +179,10 @@ LA_API la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
  * Bytes of workspace la_fwd_chunk needs for this problem: B, T, H, d_k, d_v
  * and n_seqs as they will be passed, has_cu_seqlens nonzero for a packed
  * batch.  Returns 0 when no workspace is needed and (size_t)-1 for arguments
- * la_fwd_chunk would reject.  Host-only; touches no device.
+ * la_fwd_chunk would reject.  Host-only; touches no device.  On the tensor-core
+ * path the workspace holds the segment states of long sequences in batches too
+ * small to fill the GPU (each sequence then runs as several segments), and the
+ * longest-first order of a packed batch of 2 .. 4096 sequences.
  */
 LA_API size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
                                    int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
