@@ -20,6 +20,7 @@ it follows, is stated in the C file's header:
 * ``step_norm`` -- one normalised decode token (state and z updated).
 * ``backward``  -- dq, dk, dv of sum_t dout_t . o_t (unnormalised; the adjoint
   of the recurrence, token by token).
+* ``norm_gate``  -- y = RMSNorm(o) * w * swish(g) per (token, head) over d_v.
 * ``recurrent_gated``, ``step_gated`` -- the same with a data-dependent decay
   alpha_t = exp(g_t) per token and head (section 状态空间模型与 Mamba of the
   same page: Mamba-2 as linear attention with a decay mask).
@@ -79,6 +80,8 @@ def _load():
         lib.oracle_backward.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, i32,
                                         dp, dp, dp, i32]
         lib.oracle_backward.restype = i32
+        lib.oracle_norm_gate.argtypes = [dp, vp, i32, i64, i64, dp, ctypes.c_double, dp, i32]
+        lib.oracle_norm_gate.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -308,3 +311,21 @@ def backward(q, k, v, dout, gamma, cu_seqlens=None, phi="identity", nthreads=0):
     if rc != 0:
         raise ValueError("oracle_backward rejected its arguments (code %d)" % rc)
     return gq, gk, gv
+
+
+def norm_gate(o, g, w, eps=1e-5, nthreads=0):
+    """y = o / sqrt(mean(o^2) + eps) * w * g * sigmoid(g) over the last axis (d_v).
+
+    o float64 [..., d_v]; g [..., d_v] (float32 / float64 / bfloat16); w [d_v].  Returns float64."""
+    oo = np.ascontiguousarray(np.asarray(o, dtype=np.float64))
+    gg, dt = _as_input(g)
+    ww = np.ascontiguousarray(np.asarray(w, dtype=np.float64).reshape(-1))
+    dv = oo.shape[-1]
+    if gg.shape != oo.shape or ww.size != dv:
+        raise ValueError("g must match o and w must have d_v entries")
+    y = np.zeros_like(oo)
+    rc = _load().oracle_norm_gate(_ptr(oo), _ptr(gg), dt, oo.size // dv, dv, _ptr(ww), float(eps), _ptr(y),
+                                  int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_norm_gate rejected its arguments (code %d)" % rc)
+    return y

@@ -32,6 +32,7 @@
  *                        place, o_t = S_t phi(q_t) / (z_t^T phi(q_t)).
  *   oracle_backward   -- dq, dk, dv of sum_t dout_t . o_t for the unnormalised
  *                        recurrence: the adjoint of the definition.
+ *   oracle_norm_gate  -- RMSNorm over d_v times a Swish gate, per (token, head).
  *   oracle_recurrent_gated, oracle_step_gated -- the same with a per-token
  *                        (per decode step) decay alpha_t = exp(g_t) in place
  *                        of the per-head constant gamma.
@@ -583,6 +584,35 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
     free(S);
     free(qh);
     free(kh);
+  }
+  return 0;
+}
+
+/*
+ * Output norm and gate ("使用 FlashAttention 内核实现最先进的线性注意力", the
+ * paragraph on fused norm-gate operations: RMSNorm fused with a Swish gate;
+ * the formula is the plain reading of those two names):
+ *   y[r] = o[r] / sqrt(mean_r' o[r']^2 + eps) * w[r] * g[r] * sigmoid(g[r])
+ * per (token, head) over the d_v values of o; w [d_v] is shared by all heads.
+ *   o, y [rows, d_v] double (y may alias o); g [rows, d_v] (input dtype, see
+ *   orc_load); rows = B * T * H.
+ */
+int oracle_norm_gate(const double *o, const void *g, int dtype, int64_t rows, int64_t dv, const double *w,
+                     double eps, double *y, int nthreads) {
+  if (rows < 0 || dv <= 0 || !o || !g || !w || !y) return -1;
+  if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_F64) return -1;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+  for (int64_t row = 0; row < rows; ++row) {
+    const double *x = o + row * dv;
+    double ss = 0.0;
+    for (int64_t r = 0; r < dv; ++r) ss += x[r] * x[r];
+    const double rstd = 1.0 / sqrt(ss / (double)dv + eps);
+    for (int64_t r = 0; r < dv; ++r) {
+      const double gv = orc_load(g, dtype, row * dv + r);
+      y[row * dv + r] = x[r] * rstd * w[r] * gv / (1.0 + exp(-gv));
+    }
   }
   return 0;
 }

@@ -393,6 +393,28 @@ def test_backward_varlen_equals_independent_runs(oracle_mod):
         assert np.array_equal(gq[:, s_:e], a) and np.array_equal(gk[:, s_:e], b) and np.array_equal(gv[:, s_:e], c)
 
 
+# ---------------------------------------------------------------- output norm and gate
+def test_norm_gate_closed_forms(oracle_mod):
+    """Constant rows: o = c * 1 gives y = sign(c) * w * swish(g) (up to eps); scaling
+    o leaves y unchanged with eps = 0; g = 0 gives y = 0; a large gate passes
+    the normalised row times w (swish(g) -> g)."""
+    rng = np.random.default_rng(71)
+    dv = 16
+    w = rng.uniform(0.5, 1.5, dv)
+    g = rng.standard_normal((3, dv))
+    o = np.broadcast_to(np.array([2.0, -0.5, 3.0])[:, None], (3, dv)).copy()
+    y = oracle_mod.norm_gate(o, g, w, eps=0.0)
+    swish = g / (1.0 + np.exp(-g))
+    assert rel(y, np.sign(o) * w * swish) < TOL
+    x = rng.standard_normal((5, dv))
+    g2 = rng.standard_normal((5, dv))
+    assert rel(oracle_mod.norm_gate(7.5 * x, g2, w, eps=0.0), oracle_mod.norm_gate(x, g2, w, eps=0.0)) < TOL
+    assert not oracle_mod.norm_gate(x, np.zeros_like(x), w).any()
+    big = np.full_like(x, 40.0)
+    rms = np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-5)
+    assert rel(oracle_mod.norm_gate(x, big, w), x / rms * w * 40.0) < 1e-12
+
+
 # ---------------------------------------------------------------- chunked form
 @pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
