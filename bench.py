@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "causal linear-attn fwd tokens/s and % of roofline (bf16, B200)"
 METRIC_BWD = "causal linear-attn bwd (dq, dk, dv) tokens/s and % of roofline (bf16, B200)"
+METRIC_NG = "causal linear-attn fwd + output RMSNorm/Swish gate tokens/s and % of roofline (bf16, B200)"
 
 
 def _peaks():
@@ -322,6 +323,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--normgate", action="store_true",
+                    help="forward with the output RMSNorm and Swish gate (la_fwd_chunk_normgate)")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward (la_bwd_chunk) on the workload instead of the forward")
     ap.add_argument("--decode-only", action="store_true",
@@ -376,8 +379,18 @@ def main():
         dout = make_dout(v, seed=rank_seed(rank))
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
 
+    if args.normgate:
+        if gd is not None or args.bwd:
+            raise SystemExit("--normgate covers the per-head-decay forward")
+        from chunkwise_causal_linear_la_b200.workloads import make_norm_gate
+
+        ng_gate, ng_w = make_norm_gate(v, seed=rank_seed(rank))
+
     def step():
-        if args.bwd:
+        if args.normgate:
+            la.la_fwd_chunk_normgate(q, k, v, g, ng_gate, ng_w, eps=1e-5, cu_seqlens=cu, chunk=w.chunk, phi=w.phi,
+                                     normalize=w.normalize, out=out, final_state=fs, workspace=wsbuf, stream=stream)
+        elif args.bwd:
             la.la_bwd_chunk(q, k, v, dout, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0], dk=grads[1],
                             dv=grads[2], stream=stream)
         elif gd is not None:
@@ -419,6 +432,8 @@ def main():
         [e_all0.elapsed_time(e_all1), statistics.mean(a.elapsed_time(b) for a, b in evs)], dev, dist)
     value = aggregate_rate(tokens, args.steps, ws, elapsed_ms)
     alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
+    if args.normgate:  # the gate is read too
+        alg_bytes += tokens * w.H * (2 if w.dtype == "bf16" else 4) * w.d_v
     if args.bwd:  # read q, k, v, dout; write dq, dk, dv (no final state); three forward-shaped passes of flops
         e_ = 2 if w.dtype == "bf16" else 4
         alg_bytes = tokens * w.H * e_ * (4 * w.d_k + 3 * w.d_v)
@@ -455,6 +470,8 @@ def main():
                 qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
                 gs = None if gd is None else gd[b:b + 1, :, h:h + 1].double().cpu().numpy()
                 ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs)
+                if args.normgate:
+                    ref = oracle.norm_gate(ref, ng_gate[b:b + 1, :, h:h + 1].cpu(), ng_w.double().cpu().numpy())
                 o = out[b:b + 1, :, h:h + 1].float().cpu().numpy()
                 f = fs[b:b + 1, h:h + 1].cpu().numpy()
             else:
@@ -471,6 +488,8 @@ def main():
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     inputs = (q, k, v) if gd is None else (q, k, v, gd)
+    if args.normgate:
+        inputs = (q, k, v, ng_gate)
     if args.bwd:
         inputs = (q, k, v, dout)
     outputs = grads if args.bwd else (out, fs)
@@ -517,12 +536,13 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC_BWD if args.bwd else METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "metric": METRIC_BWD if args.bwd else (METRIC_NG if args.normgate else METRIC), "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype), "data": "synthetic",
             "config": _config(w, ws),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None if args.bwd else _traffic(w.name, 1.0),
+                         "frac": achieved / hbm_peak,
+                         "traffic": None if (args.bwd or args.normgate) else _traffic(w.name, 1.0),
                          "peak_kind": "%s (burst copy bandwidth)" % peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "launch_ms": launch_ms,

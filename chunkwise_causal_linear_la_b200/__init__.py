@@ -21,7 +21,9 @@ from .binding import (  # noqa: F401
     la_bwd_chunk,
     la_fwd_chunk,
     la_fwd_chunk_gated,
+    la_fwd_chunk_normgate,
     la_fwd_chunk_z,
+    la_norm_gate,
     la_step,
     la_step_gated,
     la_step_norm,

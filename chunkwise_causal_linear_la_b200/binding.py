@@ -29,7 +29,7 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 # Every function include/la_b200.h declares.
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
-           "la_fwd_chunk_noalloc", "la_bwd_chunk")
+           "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate")
 
 
 class LaTensor(ctypes.Structure):
@@ -77,6 +77,11 @@ def load_library(path: str = LIB_PATH):
     lib.la_step_gated.restype = i32
     lib.la_bwd_chunk.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, i32, vp]
     lib.la_bwd_chunk.restype = i32
+    lib.la_norm_gate.argtypes = [P, P, vp, ctypes.c_float, P, vp]
+    lib.la_norm_gate.restype = i32
+    lib.la_fwd_chunk_normgate.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, ctypes.c_float, P, vp, i32,
+                                          vp, sz, vp]
+    lib.la_fwd_chunk_normgate.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -288,3 +293,47 @@ def la_bwd_chunk(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="identity"
                           *(ctypes.byref(x) for x in t[4:]), int(flags), _stream(stream))
     _check(lib, st, "la_bwd_chunk")
     return dq, dk, dv
+
+
+def la_norm_gate(o, gate, w, eps=1e-5, y=None, stream=None):
+    """y = RMSNorm(o) * w * swish(gate) per (token, head) over d_v (see la_norm_gate in
+    include/la_b200.h).  y defaults to a new tensor; pass y=o to work in place."""
+    lib = load_library()
+    if y is None:
+        y = torch.empty_like(o)
+    if w.dtype != torch.float32 or w.numel() != o.shape[3]:
+        raise TypeError("w must be float32 with d_v entries")
+    to, tg, ty = describe(o), describe(gate), describe(y)
+    st = lib.la_norm_gate(ctypes.byref(to), ctypes.byref(tg), w.data_ptr(), float(eps), ctypes.byref(ty),
+                          _stream(stream))
+    _check(lib, st, "la_norm_gate")
+    return y
+
+
+def la_fwd_chunk_normgate(q, k, v, gamma, gate, w, eps=1e-5, cu_seqlens=None, chunk=64, phi="identity",
+                          normalize=False, out=None, final_state=None, flags=LA_FLAG_NONE, workspace=None,
+                          stream=None):
+    """Forward whose output is la_norm_gate(o, gate, w, eps) (see la_fwd_chunk_normgate in
+    include/la_b200.h).  Returns (out, final_state)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if w.dtype != torch.float32 or w.numel() != dv:
+        raise TypeError("w must be float32 with d_v entries")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = workspace_size(B, T, H, dk, dv, n_seqs, cu_seqlens is not None, chunk, q.dtype, flags)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    t = [describe(x) for x in (q, k, v, gate, out)]
+    st = lib.la_fwd_chunk_normgate(
+        ctypes.byref(t[0]), ctypes.byref(t[1]), ctypes.byref(t[2]), gamma.data_ptr(),
+        None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi], int(bool(normalize)),
+        ctypes.byref(t[3]), w.data_ptr(), float(eps), ctypes.byref(t[4]), final_state.data_ptr(), int(flags),
+        None if workspace is None else workspace.data_ptr(),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(lib, st, "la_fwd_chunk_normgate")
+    return out, final_state

@@ -90,10 +90,18 @@ using namespace la;
 
 namespace {
 
+// Output norm and gate requested by la_fwd_chunk_normgate (NULL w: none).
+struct NormGate {
+  const la_tensor *gate = nullptr;
+  const float *w = nullptr;
+  float eps = 0.f;
+};
+
 la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                      const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
                      int32_t normalize, const la_tensor *out, float *final_state, float *final_z,
-                     int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+                     int32_t flags, void *workspace, size_t workspace_bytes, void *stream,
+                     const NormGate &ng = NormGate()) {
   la_status s;
   if ((s = check_tensor(q, "q")) != LA_OK) return s;
   if ((s = check_tensor(k, "k")) != LA_OK) return s;
@@ -149,6 +157,16 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
   a.dtype = q->dtype;
   a.rev = 0;
   a.noseg = 0;
+  a.ng_w = nullptr;
+  a.ng_gate = TensorView{nullptr, 0, 0, 0};
+  a.ng_eps = 0.f;
+  if (ng.w) {
+    if ((s = check_tensor(ng.gate, "gate")) != LA_OK) return s;
+    if (ng.gate->dtype != q->dtype || ng.gate->B != out->B || ng.gate->T != out->T || ng.gate->H != out->H ||
+        ng.gate->D != out->D)
+      return fail(LA_ERR_INVALID_ARG, "gate must have out's shape and dtype");
+    if (!(ng.eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+  }
 
   const size_t need = la_fwd_chunk_workspace_size(a.B, a.T, a.H, a.dk, a.dv, n_seqs, cu_seqlens != nullptr,
                                                   chunk, a.dtype, flags);
@@ -177,19 +195,30 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
   }
 
   const bool use_tc = a.dtype == LA_BF16 && !(flags & LA_FLAG_SIMT) && tc_supported(a);
+  const bool fuse_ng = ng.w && use_tc && tc_can_fuse_norm_gate(a);
+  if (fuse_ng) {
+    a.ng_w = ng.w;
+    a.ng_gate = view(ng.gate);
+    a.ng_eps = ng.eps;
+  }
   if (use_tc) {
     const char *why = nullptr;
     err = launch_chunk_tc(a, workspace, workspace_bytes, st, &why);
     if (err != cudaSuccess)
       return fail(LA_ERR_CUDA, "tensor-core chunk kernel: %s%s%s", cudaGetErrorString(err), why ? ": " : "",
                   why ? why : "");
-    return ok();
+  } else {
+    if (!simt_supported(a, device))
+      return fail(LA_ERR_UNSUPPORTED, "chunk %d with d_k %d does not fit the CUDA-core kernel's shared memory",
+                  chunk, a.dk);
+    err = launch_chunk_simt(a, st);
+    if (err != cudaSuccess) return fail(LA_ERR_CUDA, "CUDA-core chunk kernel: %s", cudaGetErrorString(err));
   }
-  if (!simt_supported(a, device))
-    return fail(LA_ERR_UNSUPPORTED, "chunk %d with d_k %d does not fit the CUDA-core kernel's shared memory",
-                chunk, a.dk);
-  err = launch_chunk_simt(a, st);
-  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "CUDA-core chunk kernel: %s", cudaGetErrorString(err));
+  if (ng.w && !fuse_ng) {  // the norm and gate as a second pass over out, in place
+    err = launch_norm_gate(view(out), view(ng.gate), view(out), ng.w, ng.eps, out->B, out->T, out->H,
+                           (int)out->D, q->dtype, st);
+    if (err != cudaSuccess) return fail(LA_ERR_CUDA, "output norm kernel: %s", cudaGetErrorString(err));
+  }
   return ok();
 }
 
@@ -307,6 +336,39 @@ la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
                     flags, workspace, workspace_bytes, stream);
 }
 
+la_status la_fwd_chunk_normgate(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                                const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                                int32_t normalize, const la_tensor *gate, const float *w, float eps,
+                                const la_tensor *out, float *final_state, int32_t flags, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!w) return fail(LA_ERR_INVALID_ARG, "w is NULL");
+  if (!gate) return fail(LA_ERR_INVALID_ARG, "gate: NULL tensor descriptor");
+  NormGate ng;
+  ng.gate = gate;
+  ng.w = w;
+  ng.eps = eps;
+  return fwd_common(q, k, v, gamma, nullptr, cu_seqlens, n_seqs, chunk, phi, normalize, out, final_state, nullptr,
+                    flags, workspace, workspace_bytes, stream, ng);
+}
+
+la_status la_norm_gate(const la_tensor *o, const la_tensor *gate, const float *w, float eps, const la_tensor *y,
+                       void *stream) {
+  la_status s;
+  if ((s = check_tensor(o, "o")) != LA_OK) return s;
+  if ((s = check_tensor(gate, "gate")) != LA_OK) return s;
+  if ((s = check_tensor(y, "y")) != LA_OK) return s;
+  for (const la_tensor *t : {gate, y})
+    if (t->dtype != o->dtype || t->B != o->B || t->T != o->T || t->H != o->H || t->D != o->D)
+      return fail(LA_ERR_INVALID_ARG, "gate and y must have o's shape and dtype");
+  if (!w) return fail(LA_ERR_INVALID_ARG, "w is NULL");
+  if (!(eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+  const cudaError_t err = launch_norm_gate(view(o), view(gate), view(y), w, eps, o->B, o->T, o->H, (int)o->D,
+                                           o->dtype, (cudaStream_t)stream);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "output norm kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
 la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                        const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
                        const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
@@ -383,6 +445,9 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   f.normalize = 0;
   f.dtype = q->dtype;
   f.noseg = 1;
+  f.ng_w = nullptr;
+  f.ng_gate = TensorView{nullptr, 0, 0, 0};
+  f.ng_eps = 0.f;
   auto setup = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
                    int rev) {
     f.q = view(qq);

@@ -1,4 +1,5 @@
-// la_ew.cu -- elementwise steps of the backward pass with phi = elu + 1.
+// la_ew.cu -- elementwise kernels: the steps of the backward pass with
+// phi = elu + 1, and the output RMSNorm with a Swish gate.
 //
 // The backward runs on the forward kernel (see la_bwd_chunk): operands that
 // the forward kernel reads untransformed must hold phi(x) already, and the
@@ -108,6 +109,54 @@ cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T,
     mul_dphi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
   else
     mul_dphi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
+  return cudaGetLastError();
+}
+
+}  // namespace la
+
+namespace la {
+namespace {
+
+// y = o / sqrt(mean(o^2) + eps) * w * g * sigmoid(g) over the d_v values of one
+// (token, head): one warp per row, fp32 arithmetic, y may alias o.
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) norm_gate_kernel(TensorView o, TensorView g, TensorView y,
+                                                                const float *w, float eps, int64_t T_,
+                                                                int64_t H, int dv, int64_t rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kEwThreads / 32);
+  for (int64_t row = blockIdx.x * (int64_t)(kEwThreads / 32) + (threadIdx.x >> 5); row < rows; row += warps) {
+    const int64_t h = row % H, t = (row / H) % T_, b = row / (H * T_);
+    const T *op = (const T *)o.data + b * o.sb + t * o.st + h * o.sh;
+    const T *gp = (const T *)g.data + b * g.sb + t * g.st + h * g.sh;
+    T *yp = (T *)y.data + b * y.sb + t * y.st + h * y.sh;
+    float ss = 0.f;
+    for (int c = lane; c < dv; c += 32) {
+      const float x = to_f32<T>(op[c]);
+      ss = fmaf(x, x, ss);
+    }
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, k);
+    const float rstd = rsqrtf(ss / (float)dv + eps);
+    for (int c = lane; c < dv; c += 32) {
+      const float gv = to_f32<T>(gp[c]);
+      yp[c] = from_f32<T>(to_f32<T>(op[c]) * rstd * w[c] * (gv / (1.f + expf(-gv))));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,
+                             int64_t T, int64_t H, int dv, int dtype, cudaStream_t stream) {
+  const int64_t rows = B * T * H;
+  if (rows == 0) return cudaSuccess;
+  const int64_t blocks = (rows + kEwThreads / 32 - 1) / (kEwThreads / 32);
+  const unsigned grid = (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
+  if (dtype == LA_F32)
+    norm_gate_kernel<float><<<grid, kEwThreads, 0, stream>>>(o, g, y, w, eps, T, H, dv, rows);
+  else
+    norm_gate_kernel<__nv_bfloat16><<<grid, kEwThreads, 0, stream>>>(o, g, y, w, eps, T, H, dv, rows);
   return cudaGetLastError();
 }
 

@@ -30,6 +30,11 @@ struct ChunkArgs {
   int64_t B, T, n_seqs;
   int H, dk, dv, chunk, phi, normalize;
   int dtype;  // la_dtype of q, k, v, out
+  // Output norm and gate fused into the epilogue (tensor-core kernel, d_v equal
+  // to its value slice): out = RMSNorm(o) * ng_w * swish(gate); NULL ng_w: none
+  const float *ng_w;
+  TensorView ng_gate;
+  float ng_eps;
   int rev;    // 1: reverse time (tensor-core kernel only; used by the backward pass)
   int noseg;  // 1: never split sequences into segments (no workspace)
 };
@@ -68,6 +73,8 @@ cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T
                             int dtype, cudaStream_t stream);
 cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
                             cudaStream_t stream);
+cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,
+                             int64_t T, int64_t H, int dv, int dtype, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 
@@ -77,6 +84,7 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 
 // Tensor-core (tcgen05 / TMA / TMEM) chunked forward for bf16.
 bool tc_supported(const ChunkArgs &a);
+bool tc_can_fuse_norm_gate(const ChunkArgs &a);
 size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs,
                           bool varlen, int chunk);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t workspace_bytes,

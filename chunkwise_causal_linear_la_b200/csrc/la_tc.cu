@@ -91,6 +91,11 @@ struct TcArgs {
   const float *g;
   // Packed batches: sequence of each rank, longest first (NULL: natural order)
   const int32_t *order;
+  // Output norm and gate (NG): weights [DVT], gate [B, T, H, DVT] bf16 with element strides, eps
+  const float *ng_w;
+  const void *ng_gate;
+  int64_t ng_sb, ng_st, ng_sh;
+  float ng_eps;
 };
 
 template <int DK, int DVT, int C, int NS>
@@ -115,7 +120,8 @@ struct Cfg {
   // data-dependent decay, per stage: b_i = sum_{t<=i} log alpha_t over the chunk, i < C, and b_last at [C]
   static constexpr int OFF_DT = OFF_KSUM + NS * 2 * DK * 4;
   static constexpr int DT_STRIDE = C + 4;
-  static constexpr int OFF_PW = OFF_DT + NS * DT_STRIDE * 4;
+  static constexpr int OFF_NGW = OFF_DT + NS * DT_STRIDE * 4;  // output-norm weights [DVT]
+  static constexpr int OFF_PW = OFF_NGW + DVT * 4;
   static constexpr int OFF_BAR = OFF_PW + ((C + 1) * 4 + 15) / 16 * 16;
   // barriers
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_AFULL = 3 * NS, B_PFULL = 3 * NS + 2,
@@ -196,6 +202,15 @@ __device__ __forceinline__ float phi_fast(float x) {
   float e;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fminf(x, 0.f) * kLog2e));
   return x > 0.f ? x + 1.f : e;
+}
+
+// swish(g) = g sigmoid(g) with sigmoid(g) = (1 + tanh(g / 2)) / 2 on the PTX
+// tanh.approx instruction: one special-function op per element (relative
+// error ~2^-11, below the bf16 rounding of the output).
+__device__ __forceinline__ float swish_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return x * fmaf(0.5f, t, 0.5f);
 }
 
 // e^x on the same instruction, for the data-dependent decay factors (x <= 0).
@@ -282,7 +297,8 @@ __device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int
 // i' < C', causal j' <= i'); the tiles stay in natural row order, so the
 // products need no change.  This runs the anti-causal sums of the backward
 // pass (sum over i >= j) on the same kernel.
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED, bool REV>
+// NG: the output RMSNorm with a Swish gate in the epilogue (d_v == DVT).
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED, bool REV, bool NG = false>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
@@ -293,6 +309,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
   float *ksum = reinterpret_cast<float *>(sm + G::OFF_KSUM);
   float *dtab = reinterpret_cast<float *>(sm + G::OFF_DT);  // [NS][DT_STRIDE]
+  float *ngw = reinterpret_cast<float *>(sm + G::OFF_NGW);  // [DVT]
   float *pw = reinterpret_cast<float *>(sm + G::OFF_PW);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
@@ -339,6 +356,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   // ---- setup
   if (tid <= C) pw[tid] = decay_pow(g, tid);
+  if (NG)
+    for (int i = tid; i < DVT; i += kThreads) ngw[i] = a.ng_w[i];
   // z buffer (c & 1) holds z after chunk c; buffer 1 starts with the z before chunk 0
   for (int i = tid; i < DK; i += kThreads) z[DK + i] = (NORM && has_init) ? a.ws_z[ws_slot * DK + i] : 0.f;
   if (tid == 0) {
@@ -810,6 +829,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ok = false;
       if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return 0.f;
       tc_fence_after();
+      if (NG && lrow(i) < Cp) {  // warm L2 with this row's gate for the epilogue of chunk c (one step later)
+        const uint8_t *gp = reinterpret_cast<const uint8_t *>(a.ng_gate) +
+                            2 * ((int64_t)bidx * a.ng_sb + (int64_t)h * a.ng_sh + (tok0(c) + i) * a.ng_st +
+                                 hf * (DVT / 2));
+#pragma unroll
+        for (int l = 0; l < DVT; l += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(gp + l));
+      }
       const float *dt = dtab + (c % NS) * G::DT_STRIDE;
       float bi = 0.f;
       if (GATED) {  // the stage's decay table (published before the score MMA's inputs)
@@ -885,14 +911,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int Cp = chunk_len(c);
       const int ob = out_buf(c);
       const uint32_t oph = out_phase(c);
+      const int64_t otok = tok0(c) + i;  // natural token of this row (in reverse time, may precede the sequence)
       if (!wait_bar_warp(sy, G::B_OFULL + ob, oph, c)) return false;
       tc_fence_after();
-      const int64_t otok = tok0(c) + i;  // natural token of this row (in reverse time, may precede the sequence)
       const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
-#pragma unroll 1
-      for (int pass = 0; pass < DVT / 64; ++pass) {
+      // this thread's 32 output values of a pass (columns hf DVT/2 + 32 pass ...)
+      auto load_o = [&](int pass, float (&o)[32]) {
         uint32_t ra[32], re[32];
-        float o[32];
         if (vd_mode) {  // o = gamma^(i+1) O_inter + O_intra; no inter term without a prior state
           const bool inter = c > 0 || has_init;
           const uint32_t pair = lane_base + G::T_O + ob * 2 * DVT + pass * 32;
@@ -908,18 +933,53 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ra[e]) * fac;
         }
+      };
+      float rstd = 1.f;
+      if (NG) {  // output norm: the row's mean square over d_v (this thread and its other half, lane ^ 16)
+        float ss = 0.f;
+#pragma unroll 1
+        for (int pass = 0; pass < DVT / 64; ++pass) {
+          float o[32];
+          load_o(pass, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ss = fmaf(o[e], o[e], ss);
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+        rstd = rsqrtf(ss / (float)DVT + a.ng_eps);
+      }
+      auto do_pass = [&](int pass) {
+        float o[32];
+        load_o(pass, o);
         if (pass == DVT / 64 - 1) {
           tc_fence_before();
           mbar_arrive(bars + G::B_OEMPTY + ob);
         }
         if (lrow(i) < Cp) {
-          uint4 *dst = reinterpret_cast<uint4 *>(obase + 2 * (otok * a.o_st + hf * (DVT / 2) + pass * 32));
+          const int col = hf * (DVT / 2) + pass * 32;
+          if (NG) {  // y = o rstd w swish(gate)
+            const uint4 *gsrc = reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const uint8_t *>(a.ng_gate) +
+                2 * ((int64_t)bidx * a.ng_sb + (int64_t)h * a.ng_sh + otok * a.ng_st + col));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float gv[8];
+              unpack8(gsrc[q], gv);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int e = 8 * q + u;
+                o[e] = o[e] * rstd * ngw[col + e] * swish_fast(gv[u]);
+              }
+            }
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(obase + 2 * (otok * a.o_st + col));
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             dst[q] = make_uint4(pack2(o[8 * q], o[8 * q + 1]), pack2(o[8 * q + 2], o[8 * q + 3]),
                                 pack2(o[8 * q + 4], o[8 * q + 5]), pack2(o[8 * q + 6], o[8 * q + 7]));
         }
-      }
+      };
+#pragma unroll 1
+      for (int pass = 0; pass < DVT / 64; ++pass) do_pass(pass);
       return true;
     };
 
@@ -1115,7 +1175,7 @@ __global__ void seg_scan_kernel(float *ws_s, float *ws_z, const float *ws_g, con
   }
 }
 
-template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, bool GATED, bool REV>
+template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, bool GATED, bool REV, bool NG = false>
 cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   using G = Cfg<DK, DVT, C, NS>;
   CUtensorMap mq, mk, mv;
@@ -1149,6 +1209,12 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.ws_z = nullptr;
   t.ws_g = nullptr;
   t.order = nullptr;
+  t.ng_w = a.ng_w;
+  t.ng_gate = a.ng_gate.data;
+  t.ng_sb = a.ng_gate.sb;
+  t.ng_st = a.ng_gate.st;
+  t.ng_sh = a.ng_gate.sh;
+  t.ng_eps = a.ng_eps;
   const size_t ob = a.noseg ? 0 : order_bytes(a.n_seqs, a.cu_seqlens != nullptr);
   if (ob > 0 && workspace) {
     int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + seg_ws_bytes(plan, DK, DVT));
@@ -1158,7 +1224,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
     if (e != cudaSuccess) return e;
     t.order = order;
   }
-  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0, GATED, REV>;
+  auto kern = chunk_tc_kernel<DK, DVT, C, NS, NORM, ELU, 0, GATED, REV, NG>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   if (plan.G > 1) {
@@ -1202,6 +1268,9 @@ cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset
   return e;
 }
 
+// The output norm fuses into the epilogue when one CTA holds whole rows of d_v.
+bool tc_can_fuse_norm_gate(const ChunkArgs &a) { return a.dk == 128 && a.dv == tc_dvt(a.dk) && !a.g && !a.rev; }
+
 bool tc_supported(const ChunkArgs &a) {
   if (a.dtype != LA_BF16 || a.chunk != 64) return false;
   if (a.dk != 128 && a.dk != 256) return false;
@@ -1221,6 +1290,14 @@ size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64
 template <int DK, int DVT, int NS, bool GATED>
 cudaError_t launch_shape_gated(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
   // one instantiation per (normaliser, feature map, decay kind): each carries only its own code path
+  if (!GATED && DVT == 128 && a.ng_w) {  // output norm and gate fused into the epilogue
+    if (a.dv != DVT) return cudaErrorInvalidValue;
+    if (a.normalize)
+      return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true, false, false, true>(a, workspace, stream, why)
+                   : launch_cfg<DK, DVT, 64, NS, true, false, false, false, true>(a, workspace, stream, why);
+    return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, false, false, true>(a, workspace, stream, why)
+                 : launch_cfg<DK, DVT, 64, NS, false, false, false, false, true>(a, workspace, stream, why);
+  }
   if (a.normalize) {
     return a.phi ? launch_cfg<DK, DVT, 64, NS, true, true, GATED, false>(a, workspace, stream, why)
                  : launch_cfg<DK, DVT, 64, NS, true, false, GATED, false>(a, workspace, stream, why);

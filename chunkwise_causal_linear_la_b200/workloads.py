@@ -160,6 +160,15 @@ def make_dout(v: torch.Tensor, seed: int = 0) -> torch.Tensor:
     return torch.randn(v.shape, generator=g, device=v.device, dtype=torch.float32).to(v.dtype)
 
 
+def make_norm_gate(v: torch.Tensor, seed: int = 0):
+    """Gate (N(0, 1) * 2, like v) and norm weights (U[0.5, 1.5), [d_v]) for the output norm."""
+    g = torch.Generator(device=v.device)
+    g.manual_seed(seed + 3)
+    gate = (torch.randn(v.shape, generator=g, device=v.device) * 2.0).to(v.dtype)
+    w = torch.rand(v.shape[-1], generator=g, device=v.device) + 0.5
+    return gate, w
+
+
 def make_decode_inputs(N, H, d_k, d_v, scale, state_std, gamma, seed=0, device="cpu",
                        dtype=torch.float32):
     """Decode inputs: q, k [N,H,d_k], v [N,H,d_v], state [N,H,d_k,d_v] fp32, gamma [H]."""

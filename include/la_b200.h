@@ -176,6 +176,31 @@ LA_API la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
                                     int32_t flags, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * la_norm_gate -- the output norm and gate of a retention layer, on its own:
+ *     y[r] = o[r] / sqrt(mean_r' o[r']^2 + eps) * w[r] * gate[r] * sigmoid(gate[r])
+ * per (token, head) over the d_v values ("使用 FlashAttention 内核实现最先进的线性注意力":
+ * RMSNorm fused with a Swish gate; the formula is the plain reading of those
+ * two names).  o, gate, y [B, T, H, d_v], one dtype; y may alias o.  w device
+ * float[d_v], shared by all heads; eps >= 0.  fp32 arithmetic.
+ */
+LA_API la_status la_norm_gate(const la_tensor *o, const la_tensor *gate, const float *w, float eps,
+                              const la_tensor *y, void *stream);
+
+/*
+ * la_fwd_chunk_normgate -- la_fwd_chunk whose `out` receives la_norm_gate of
+ * the attention output (gate, w, eps as there).  On the tensor cores with
+ * d_k = d_v = 128 the norm and gate run in the kernel's epilogue (the output is
+ * written once); otherwise a second pass normalises `out` in place, and then
+ * rows of a packed batch outside every sequence are written too.  Other
+ * arguments, results and errors as for la_fwd_chunk.
+ */
+LA_API la_status la_fwd_chunk_normgate(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                       const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs,
+                                       int32_t chunk, int32_t phi, int32_t normalize, const la_tensor *gate,
+                                       const float *w, float eps, const la_tensor *out, float *final_state,
+                                       int32_t flags, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of workspace la_fwd_chunk needs for this problem: B, T, H, d_k, d_v
  * and n_seqs as they will be passed, has_cu_seqlens nonzero for a packed
  * batch.  Returns 0 when no workspace is needed and (size_t)-1 for arguments
