@@ -20,6 +20,8 @@ it follows, is stated in the C file's header:
 * ``step_norm`` -- one normalised decode token (state and z updated).
 * ``backward``  -- dq, dk, dv of sum_t dout_t . o_t (unnormalised; the adjoint
   of the recurrence, token by token).
+* ``gated_delta`` -- the gated delta rule (section Gated delta rule of the same
+  page), token by token, unit-norm keys.
 * ``norm_gate``  -- y = RMSNorm(o) * w * swish(g) per (token, head) over d_v.
 * ``recurrent_gated``, ``step_gated`` -- the same with a data-dependent decay
   alpha_t = exp(g_t) per token and head (section 状态空间模型与 Mamba of the
@@ -82,6 +84,8 @@ def _load():
         lib.oracle_backward.restype = i32
         lib.oracle_norm_gate.argtypes = [dp, vp, i32, i64, i64, dp, ctypes.c_double, dp, i32]
         lib.oracle_norm_gate.restype = i32
+        lib.oracle_gated_delta.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, dp, vp, i64, dp, dp, dp, i32]
+        lib.oracle_gated_delta.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -329,3 +333,25 @@ def norm_gate(o, g, w, eps=1e-5, nthreads=0):
     if rc != 0:
         raise ValueError("oracle_norm_gate rejected its arguments (code %d)" % rc)
     return y
+
+
+def gated_delta(q, k, v, g, beta, cu_seqlens=None, init=None, nthreads=0):
+    """Gated delta rule: S_t = exp(g_t) S_{t-1} (I - beta_t kt kt^T) + beta_t v_t kt^T, o_t = S_t q_t,
+    kt = k_t / |k_t|.  g, beta [B, T, H]; init None or [N, H, d_k, d_v] (S^T).
+
+    Returns (out [B,T,H,d_v], final_state [N,H,d_k,d_v]) in float64."""
+    q, k, v, dt, B, T, H, dk, dv, _, cu, n = _prep(q, k, v, np.ones(q.shape[2]), cu_seqlens)
+    gg = np.ascontiguousarray(np.asarray(g, dtype=np.float64))
+    bb = np.ascontiguousarray(np.asarray(beta, dtype=np.float64))
+    if gg.shape != (B, T, H) or bb.shape != (B, T, H):
+        raise ValueError("g and beta must be [B, T, H]")
+    ii = None if init is None else np.ascontiguousarray(np.asarray(init, dtype=np.float64))
+    if ii is not None and ii.shape != (n, H, dk, dv):
+        raise ValueError("init must be [N, H, d_k, d_v]")
+    out = np.zeros((B, T, H, dv), np.float64)
+    fs = np.zeros((n, H, dk, dv), np.float64)
+    rc = _load().oracle_gated_delta(_ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(gg), _ptr(bb), _ptr(cu),
+                                    n, _ptr(ii), _ptr(out), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_gated_delta rejected its arguments (code %d)" % rc)
+    return out, fs

@@ -33,6 +33,7 @@
  *   oracle_backward   -- dq, dk, dv of sum_t dout_t . o_t for the unnormalised
  *                        recurrence: the adjoint of the definition.
  *   oracle_norm_gate  -- RMSNorm over d_v times a Swish gate, per (token, head).
+ *   oracle_gated_delta -- the gated delta rule, token by token.
  *   oracle_recurrent_gated, oracle_step_gated -- the same with a per-token
  *                        (per decode step) decay alpha_t = exp(g_t) in place
  *                        of the per-head constant gamma.
@@ -613,6 +614,72 @@ int oracle_norm_gate(const double *o, const void *g, int dtype, int64_t rows, in
       const double gv = orc_load(g, dtype, row * dv + r);
       y[row * dv + r] = x[r] * rstd * w[r] * gv / (1.0 + exp(-gv));
     }
+  }
+  return 0;
+}
+
+/*
+ * Gated delta rule ("1.6 长上下文与高效注意力", section Gated delta rule, and its
+ * listing): with the key normalised to unit length, kt = k_t / max(|k_t|, 1e-12),
+ *     S_t = alpha_t S_{t-1} (I - beta_t kt kt^T) + beta_t v_t kt^T,   o_t = S_t q_t
+ * per (sequence, head), S (d_v x d_k) starting at init (or zero), alpha_t =
+ * exp(g_t).  q is used as given (no feature map), as in the listing.
+ *   g, beta [B, T, H] double; init NULL or [n_seqs, H, d_k, d_v] (S^T);
+ *   out [B, T, H, d_v]; final_state [n_seqs, H, d_k, d_v] (S^T) or NULL.
+ */
+int oracle_gated_delta(const void *q, const void *k, const void *v, int dtype, int64_t B, int64_t T,
+                       int64_t H, int64_t dk, int64_t dv, const double *g, const double *beta,
+                       const int32_t *cu_seqlens, int64_t n_seqs, const double *init, double *out,
+                       double *final_state, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, ORC_PHI_IDENTITY);
+  if (rc) return rc;
+  if (!g || !beta) return -10;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double));  /* S[r][c] */
+    double *kt = (double *)malloc((size_t)dk * sizeof(double));
+    double *u = (double *)malloc((size_t)dv * sizeof(double));
+    if (init)
+      for (int64_t c = 0; c < dk; ++c)
+        for (int64_t r = 0; r < dv; ++r) S[r * dk + c] = init[task * dk * dv + c * dv + r];
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      const double a = exp(g[row * H + h]), b = beta[row * H + h];
+      double nrm = 0.0;
+      for (int64_t c = 0; c < dk; ++c) {
+        kt[c] = orc_load(k, dtype, qk + c);
+        nrm += kt[c] * kt[c];
+      }
+      nrm = sqrt(nrm);
+      if (nrm < 1e-12) nrm = 1e-12;
+      for (int64_t c = 0; c < dk; ++c) kt[c] /= nrm;
+      for (int64_t r = 0; r < dv; ++r) {  /* u = S kt */
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * kt[c];
+        u[r] = acc;
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, vb + r);
+        double o = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          S[r * dk + c] = a * (S[r * dk + c] - b * u[r] * kt[c]) + b * vr * kt[c];
+          o += S[r * dk + c] * orc_load(q, dtype, qk + c);
+        }
+        out[vb + r] = o;
+      }
+    }
+    if (final_state)
+      for (int64_t c = 0; c < dk; ++c)
+        for (int64_t r = 0; r < dv; ++r) final_state[task * dk * dv + c * dv + r] = S[r * dk + c];
+    free(S);
+    free(kt);
+    free(u);
   }
   return 0;
 }
