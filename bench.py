@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 METRIC = "causal linear-attn fwd tokens/s and % of roofline (bf16, B200)"
 METRIC_BWD = "causal linear-attn bwd (dq, dk, dv) tokens/s and % of roofline (bf16, B200)"
 METRIC_NG = "causal linear-attn fwd + output RMSNorm/Swish gate tokens/s and % of roofline (bf16, B200)"
+METRIC_GD = "gated delta rule fwd tokens/s and % of roofline (bf16, B200)"
 
 
 def _peaks():
@@ -173,9 +174,11 @@ def _traffic(workload_name, units_scale):
     return None
 
 
-def _oracle_run(oracle, w, q, k, v, gamma, g=None, bwd=False):
-    """The oracle's recurrence for workload w (per-head gamma, or the per-token log decay g);
-    bwd: its adjoint for an all-ones output gradient."""
+def _oracle_run(oracle, w, q, k, v, gamma, g=None, bwd=False, beta=None):
+    """The oracle's recurrence for workload w (per-head gamma, or the per-token log decay g;
+    with beta, the gated delta rule); bwd: its adjoint for an all-ones output gradient."""
+    if beta is not None:
+        return oracle.gated_delta(q, k, v, g, beta)
     if bwd:
         import torch
 
@@ -197,25 +200,30 @@ def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1, bwd=False):
         nseq = 1
     q, k, v = (t[:nseq] for t in (x["q"], x["k"], x["v"]))
     gd = x["g"][:nseq] if "g" in x else None
+    bd = x["beta"][:nseq] if "beta" in x else None
     g = x["gamma"].double().cpu().numpy()
 
     def sample(n):
         qs, ks, vs = (t[:, :n].cpu().contiguous() for t in (q, k, v))
         return qs, ks, vs, None if gd is None else gd[:, :n].double().cpu().numpy()
 
+    def run(qs, ks, vs, gs, n):
+        b_ = None if bd is None else bd[:, :n].double().cpu().numpy()
+        _oracle_run(oracle, w, qs, ks, vs, g, gs, bwd, beta=b_)
+
     # calibrate on short prefixes (the second sized to about a second), then size the sample to the budget
     n = min(T, 64)
     for target in (1.0, budget_s):
         qs, ks, vs, gs = sample(n)
         t0 = time.perf_counter()
-        _oracle_run(oracle, w, qs, ks, vs, g, gs, bwd)
+        run(qs, ks, vs, gs, n)
         dt = max(time.perf_counter() - t0, 1e-4)
         n = int(min(T, max(n, n * target / dt)))
     if max_tokens:
         n = min(n, max_tokens)
     qs, ks, vs, gs = sample(n)
     t0 = time.perf_counter()
-    _oracle_run(oracle, w, qs, ks, vs, g, gs, bwd)
+    run(qs, ks, vs, gs, n)
     secs = time.perf_counter() - t0
     return nseq * n / secs, n, secs, oracle.max_threads()
 
@@ -386,8 +394,12 @@ def main():
 
         ng_gate, ng_w = make_norm_gate(v, seed=rank_seed(rank))
 
+    gbeta = x.get("beta")  # gated delta rule workloads
+
     def step():
-        if args.normgate:
+        if gbeta is not None:
+            la.la_fwd_gated_delta(q, k, v, gd, gbeta, cu_seqlens=cu, out=out, final_state=fs, stream=stream)
+        elif args.normgate:
             la.la_fwd_chunk_normgate(q, k, v, g, ng_gate, ng_w, eps=1e-5, cu_seqlens=cu, chunk=w.chunk, phi=w.phi,
                                      normalize=w.normalize, out=out, final_state=fs, workspace=wsbuf, stream=stream)
         elif args.bwd:
@@ -432,6 +444,8 @@ def main():
         [e_all0.elapsed_time(e_all1), statistics.mean(a.elapsed_time(b) for a, b in evs)], dev, dist)
     value = aggregate_rate(tokens, args.steps, ws, elapsed_ms)
     alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
+    if gbeta is not None:  # beta is read too
+        alg_bytes += tokens * w.H * 4
     if args.normgate:  # the gate is read too
         alg_bytes += tokens * w.H * (2 if w.dtype == "bf16" else 4) * w.d_v
     if args.bwd:  # read q, k, v, dout; write dq, dk, dv (no final state); three forward-shaped passes of flops
@@ -469,7 +483,8 @@ def main():
             if cu is None:
                 qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
                 gs = None if gd is None else gd[b:b + 1, :, h:h + 1].double().cpu().numpy()
-                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs)
+                bs = None if gbeta is None else gbeta[b:b + 1, :, h:h + 1].double().cpu().numpy()
+                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs, beta=bs)
                 if args.normgate:
                     ref = oracle.norm_gate(ref, ng_gate[b:b + 1, :, h:h + 1].cpu(), ng_w.double().cpu().numpy())
                 o = out[b:b + 1, :, h:h + 1].float().cpu().numpy()
@@ -478,7 +493,8 @@ def main():
                 s, e = int(cu[0]), int(cu[1])
                 qs, ks, vs = (t[:, s:e, h:h + 1].cpu() for t in (q, k, v))
                 gs = None if gd is None else gd[:, s:e, h:h + 1].double().cpu().numpy()
-                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs)
+                bs = None if gbeta is None else gbeta[:, s:e, h:h + 1].double().cpu().numpy()
+                ref, fref = _oracle_run(oracle, w, qs, ks, vs, [float(g[h])], gs, beta=bs)
                 o = out[:, s:e, h:h + 1].float().cpu().numpy()
                 f = fs[0:1, h:h + 1].cpu().numpy()
             worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))),
@@ -488,6 +504,8 @@ def main():
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     inputs = (q, k, v) if gd is None else (q, k, v, gd)
+    if gbeta is not None:
+        inputs = (q, k, v, gd, gbeta)
     if args.normgate:
         inputs = (q, k, v, ng_gate)
     if args.bwd:
@@ -536,18 +554,20 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC_BWD if args.bwd else (METRIC_NG if args.normgate else METRIC), "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "metric": METRIC_BWD if args.bwd else (METRIC_NG if args.normgate else (
+                METRIC_GD if gbeta is not None else METRIC)), "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype), "data": "synthetic",
             "config": _config(w, ws),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
-                         "traffic": None if (args.bwd or args.normgate) else _traffic(w.name, 1.0),
+                         "traffic": None if (args.bwd or args.normgate or gbeta is not None) else
+                         _traffic(w.name, 1.0),
                          "peak_kind": "%s (burst copy bandwidth)" % peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "launch_ms": launch_ms,
                          "kernel": "chunk_tc_kernel (3 passes: forward + 2 in reverse time)" if args.bwd
-                         else "chunk_tc_kernel"},
+                         else ("delta_kernel" if gbeta is not None else "chunk_tc_kernel")},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
             "parity": parity, "extra": extra,
         }

@@ -23,6 +23,7 @@ from .binding import (  # noqa: F401
     la_fwd_chunk_gated,
     la_fwd_chunk_normgate,
     la_fwd_chunk_z,
+    la_fwd_gated_delta,
     la_norm_gate,
     la_step,
     la_step_gated,

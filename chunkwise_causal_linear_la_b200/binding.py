@@ -29,7 +29,8 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 # Every function include/la_b200.h declares.
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
-           "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate")
+           "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
+           "la_fwd_gated_delta")
 
 
 class LaTensor(ctypes.Structure):
@@ -82,6 +83,8 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_chunk_normgate.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, ctypes.c_float, P, vp, i32,
                                           vp, sz, vp]
     lib.la_fwd_chunk_normgate.restype = i32
+    lib.la_fwd_gated_delta.argtypes = [P, P, P, vp, vp, vp, i64, vp, P, vp, vp]
+    lib.la_fwd_gated_delta.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -336,4 +339,28 @@ def la_fwd_chunk_normgate(q, k, v, gamma, gate, w, eps=1e-5, cu_seqlens=None, ch
         None if workspace is None else workspace.data_ptr(),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
     _check(lib, st, "la_fwd_chunk_normgate")
+    return out, final_state
+
+
+def la_fwd_gated_delta(q, k, v, g, beta, cu_seqlens=None, initial_state=None, out=None, final_state=None,
+                       return_final_state=True, stream=None):
+    """Gated delta rule (see la_fwd_gated_delta in include/la_b200.h).  g, beta float32 [B, T, H];
+    initial_state / final_state float32 [N, H, d_k, d_v] (S^T).  Returns (out, final_state)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("g", g), ("beta", beta)):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, T, H) or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous float32 [B, T, H] tensor" % name)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32, device=q.device)
+    t = [describe(x) for x in (q, k, v, out)]
+    st = lib.la_fwd_gated_delta(ctypes.byref(t[0]), ctypes.byref(t[1]), ctypes.byref(t[2]), g.data_ptr(),
+                                beta.data_ptr(), None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs,
+                                None if initial_state is None else initial_state.data_ptr(), ctypes.byref(t[3]),
+                                None if final_state is None else final_state.data_ptr(), _stream(stream))
+    _check(lib, st, "la_fwd_gated_delta")
     return out, final_state

@@ -352,6 +352,59 @@ la_status la_fwd_chunk_normgate(const la_tensor *q, const la_tensor *k, const la
                     flags, workspace, workspace_bytes, stream, ng);
 }
 
+la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int64_t n_seqs,
+                             const float *initial_state, const la_tensor *out, float *final_state, void *stream) {
+  la_status s;
+  const la_tensor *ts[4] = {q, k, v, out};
+  const char *names[4] = {"q", "k", "v", "out"};
+  for (int i = 0; i < 4; ++i)
+    if ((s = check_tensor(ts[i], names[i])) != LA_OK) return s;
+  for (int i = 1; i < 4; ++i) {
+    if (ts[i]->dtype != q->dtype) return fail(LA_ERR_INVALID_ARG, "%s must have q's dtype", names[i]);
+    if (ts[i]->B != q->B || ts[i]->T != q->T || ts[i]->H != q->H)
+      return fail(LA_ERR_INVALID_ARG, "%s disagrees with q on B, T or H", names[i]);
+  }
+  if (k->D != q->D || out->D != v->D) return fail(LA_ERR_INVALID_ARG, "head dims disagree");
+  if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
+  const int64_t rows = q->B * q->T * q->H;
+  if (rows > 0 && (!g || !beta)) return fail(LA_ERR_INVALID_ARG, "g or beta is NULL");
+  if (((uintptr_t)g) % 4 || ((uintptr_t)beta) % 4 || ((uintptr_t)initial_state) % 4 || ((uintptr_t)final_state) % 4)
+    return fail(LA_ERR_INVALID_ARG, "g, beta, initial_state and final_state must be 4-byte aligned");
+  if (cu_seqlens) {
+    if (q->B != 1) return fail(LA_ERR_INVALID_ARG, "packed batches (cu_seqlens) need B == 1");
+    if (n_seqs < 0) return fail(LA_ERR_INVALID_ARG, "n_seqs is negative");
+  } else if (n_seqs != q->B) {
+    return fail(LA_ERR_INVALID_ARG, "n_seqs must equal B when cu_seqlens is NULL");
+  }
+  if (!head_dim_ok(q->D) || !head_dim_ok(v->D))
+    return fail(LA_ERR_UNSUPPORTED, "head dims (%lld, %lld) not in {16, 32, 64, 128, 256}",
+                (long long)q->D, (long long)v->D);
+  DeltaArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.out = out->data;
+  a.o_sb = out->stride_b;
+  a.o_st = out->stride_t;
+  a.o_sh = out->stride_h;
+  a.g = g;
+  a.beta = beta;
+  a.init = initial_state;
+  a.final_state = final_state;
+  a.cu_seqlens = cu_seqlens;
+  a.T = q->T;
+  a.n_seqs = n_seqs;
+  a.H = (int)q->H;
+  a.dk = (int)q->D;
+  a.dv = (int)v->D;
+  a.dtype = q->dtype;
+  if (n_seqs == 0) return ok();
+  const cudaError_t err = launch_delta(a, (cudaStream_t)stream);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "gated delta kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
 la_status la_norm_gate(const la_tensor *o, const la_tensor *gate, const float *w, float eps, const la_tensor *y,
                        void *stream) {
   la_status s;

@@ -1,0 +1,183 @@
+// la_delta.cu -- the gated delta rule, token by token on CUDA cores (fp32).
+//
+// "1.6 长上下文与高效注意力", section Gated delta rule: with the key normalised
+// to unit length (kt = k_t / max(|k_t|, 1e-12), as in the section's listing),
+//     S_t = alpha_t S_{t-1} (I - beta_t kt kt^T) + beta_t v_t kt^T,   o_t = S_t q_t,
+// alpha_t = exp(g_t).  Row r of S (the state of value column r) evolves on its
+// own: with u_r = S[r, :] . kt,
+//     S[r, :] <- alpha S[r, :] + beta (v_r - alpha u_r) kt,    o_r = S[r, :] . q_t,
+// so the P adjacent lanes of a column each hold d_k / P of its state values in
+// registers, interleaved by 16-byte granules (lane p of a column holds the
+// granules p, p + P, ..., so the warp's broadcast loads of the key and query
+// hit distinct banks), and the dot products finish with log2 P shuffles and the columns of
+// a head are split over CTAs freely: 128 columns per CTA of 128 P threads.
+// Splitting d_k shortens each thread's per-token chain, which is what bounds
+// this token-by-token kernel.  Each CTA stages a tile of C tokens of q, the unit keys,
+// v, alpha and beta in shared memory (read by every thread as broadcasts) and
+// then walks the tile's tokens in order.
+#include <cuda_bf16.h>
+
+#include "la_common.cuh"
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+constexpr int kDeltaCols = 128;  // value columns per CTA
+constexpr int kDeltaTile = 64;
+
+// KP: state values per thread; P: threads per value column (KP * P = d_k)
+template <typename Tin, int KP, int P>
+__global__ void __launch_bounds__(kDeltaCols * P)
+delta_kernel(DeltaArgs a) {
+  extern __shared__ float sm[];
+  constexpr int kDeltaThreads = kDeltaCols * P;
+  constexpr int DK = KP * P;
+  constexpr int COLS = kDeltaCols;
+  float *qs = sm;                          // [C][DK]
+  float *ks = qs + kDeltaTile * DK;        // [C][DK] unit keys
+  float *vs = ks + kDeltaTile * DK;        // [C][COLS]
+  float *al = vs + kDeltaTile * COLS;      // [C] alpha
+  float *be = al + kDeltaTile;             // [C] beta
+
+  const int tid = threadIdx.x;
+  const int nsl = (a.dv + COLS - 1) / COLS;
+  const int64_t unit = blockIdx.x;
+  const int sl = (int)(unit % nsl);
+  const int h = (int)((unit / nsl) % a.H);
+  const int64_t n = unit / ((int64_t)nsl * a.H);
+  const int p = tid % P, col = tid / P;
+  const int r = sl * COLS + col;  // value column of this thread
+  const bool active = r < a.dv;
+  int64_t b, start, len;
+  if (a.cu_seqlens) {
+    b = 0;
+    start = a.cu_seqlens[n];
+    len = (int64_t)a.cu_seqlens[n + 1] - start;
+  } else {
+    b = n;
+    start = 0;
+    len = a.T;
+  }
+  const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + h * a.q.sh;
+  const Tin *K = (const Tin *)a.k.data + b * a.k.sb + h * a.k.sh;
+  const Tin *V = (const Tin *)a.v.data + b * a.v.sb + h * a.v.sh;
+  Tin *O = (Tin *)a.out + b * a.o_sb + h * a.o_sh;
+  const int64_t srow = b * a.T + start;  // first token row of the sequence in [B * T]
+
+  float S[KP];  // S[4 j + e] is state row 4 (p + P j) + e of column r
+  const int64_t sbase = ((int64_t)n * a.H + h) * (int64_t)DK * a.dv;
+  auto krow = [&](int c) -> int { return 4 * (p + P * (c >> 2)) + (c & 3); };
+#pragma unroll
+  for (int c = 0; c < KP; ++c) S[c] = (a.init && active) ? a.init[sbase + (int64_t)krow(c) * a.dv + r] : 0.f;
+
+  for (int64_t t0 = 0; t0 < len; t0 += kDeltaTile) {
+    const int Ct = (int)min((int64_t)kDeltaTile, len - t0);
+    __syncthreads();  // the previous tile is consumed
+    for (int e = tid; e < Ct * DK; e += kDeltaThreads) {
+      const int i = e / DK, c = e % DK;
+      const int64_t t = start + t0 + i;
+      qs[e] = to_f32<Tin>(Q[t * a.q.st + c]);
+      ks[e] = to_f32<Tin>(K[t * a.k.st + c]);
+    }
+    for (int e = tid; e < Ct * COLS; e += kDeltaThreads) {
+      const int i = e / COLS, cc = e % COLS, rr = sl * COLS + cc;
+      vs[e] = rr < a.dv ? to_f32<Tin>(V[(start + t0 + i) * a.v.st + rr]) : 0.f;
+    }
+    for (int i = tid; i < Ct; i += kDeltaThreads) {
+      const int64_t row = (srow + t0 + i) * a.H + h;
+      al[i] = expf(a.g[row]);
+      be[i] = a.beta[row];
+    }
+    __syncthreads();
+    // unit keys: one warp per row
+    for (int i = tid >> 5; i < Ct; i += kDeltaThreads / 32) {
+      float ss = 0.f;
+      for (int c = tid & 31; c < DK; c += 32) ss = fmaf(ks[i * DK + c], ks[i * DK + c], ss);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+      for (int c = tid & 31; c < DK; c += 32) ks[i * DK + c] *= inv;
+    }
+    __syncthreads();
+    for (int i = 0; i < Ct; ++i) {
+      const float *kt = ks + i * DK;
+      const float *qt = qs + i * DK;
+      static_assert(KP % 4 == 0, "16-byte broadcast loads of the key and query");
+      const float4 *kt4 = reinterpret_cast<const float4 *>(kt);
+      const float4 *qt4 = reinterpret_cast<const float4 *>(qt);
+      float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < KP; c += 4) {
+        const float4 kv = kt4[p + P * (c / 4)];
+        u0 = fmaf(S[c], kv.x, u0);
+        u1 = fmaf(S[c + 1], kv.y, u1);
+        u2 = fmaf(S[c + 2], kv.z, u2);
+        u3 = fmaf(S[c + 3], kv.w, u3);
+      }
+      float u = (u0 + u1) + (u2 + u3);
+#pragma unroll
+      for (int m = 1; m < P; m <<= 1) u += __shfl_xor_sync(0xffffffffu, u, m);
+      __syncwarp();  // reload kt below instead of keeping all of it in registers
+      const float alpha = al[i];
+      const float coef = be[i] * (vs[i * COLS + col] - alpha * u);
+      float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < KP; c += 4) {
+        const float4 kv = kt4[p + P * (c / 4)];
+        const float4 qv = qt4[p + P * (c / 4)];
+        S[c] = fmaf(alpha, S[c], coef * kv.x);
+        S[c + 1] = fmaf(alpha, S[c + 1], coef * kv.y);
+        S[c + 2] = fmaf(alpha, S[c + 2], coef * kv.z);
+        S[c + 3] = fmaf(alpha, S[c + 3], coef * kv.w);
+        o0 = fmaf(S[c], qv.x, o0);
+        o1 = fmaf(S[c + 1], qv.y, o1);
+        o2 = fmaf(S[c + 2], qv.z, o2);
+        o3 = fmaf(S[c + 3], qv.w, o3);
+      }
+      float o = (o0 + o1) + (o2 + o3);
+#pragma unroll
+      for (int m = 1; m < P; m <<= 1) o += __shfl_xor_sync(0xffffffffu, o, m);
+      if (p == 0 && active) O[(start + t0 + i) * a.o_st + r] = from_f32<Tin>(o);
+    }
+  }
+  if (a.final_state && active) {
+#pragma unroll
+    for (int c = 0; c < KP; ++c) a.final_state[sbase + (int64_t)krow(c) * a.dv + r] = S[c];
+  }
+}
+
+template <typename Tin, int KP, int P>
+cudaError_t launch_kp(const DeltaArgs &a, cudaStream_t stream) {
+  constexpr int COLS = kDeltaCols;
+  constexpr int kDeltaThreads = kDeltaCols * P;
+  const int64_t grid = a.n_seqs * a.H * ((a.dv + COLS - 1) / COLS);
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const size_t smem = (size_t)(2 * kDeltaTile * KP * P + kDeltaTile * COLS + 2 * kDeltaTile) * sizeof(float);
+  auto kern = delta_kernel<Tin, KP, P>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  kern<<<(unsigned)grid, kDeltaThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_dtype(const DeltaArgs &a, cudaStream_t stream) {
+  switch (a.dk) {
+    case 16: return launch_kp<Tin, 16, 1>(a, stream);
+    case 32: return launch_kp<Tin, 16, 2>(a, stream);
+    case 64: return launch_kp<Tin, 16, 4>(a, stream);
+    case 128: return launch_kp<Tin, 32, 4>(a, stream);
+    case 256: return launch_kp<Tin, 64, 4>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_delta(const DeltaArgs &a, cudaStream_t stream) {
+  return a.dtype == LA_F32 ? launch_dtype<float>(a, stream) : launch_dtype<__nv_bfloat16>(a, stream);
+}
+
+}  // namespace la

@@ -59,6 +59,18 @@ struct BwdArgs {
   int H, dk, dv, chunk, phi, dtype;
 };
 
+struct DeltaArgs {
+  TensorView q, k, v;
+  void *out;
+  int64_t o_sb, o_st, o_sh;
+  const float *g, *beta;      // [B * T][H] log decay and write strength
+  const float *init;          // NULL or [n_seqs, H, d_k, d_v] (S^T)
+  float *final_state;         // NULL or [n_seqs, H, d_k, d_v]; may alias init
+  const int32_t *cu_seqlens;  // NULL for dense batches
+  int64_t T, n_seqs;
+  int H, dk, dv, dtype;
+};
+
 // Sets the calling thread's la_last_error() message and returns `status`.
 la_status report_error(la_status status, const char *msg);
 
@@ -76,6 +88,7 @@ cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T,
 cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,
                              int64_t T, int64_t H, int dv, int dtype, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+cudaError_t launch_delta(const DeltaArgs &a, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 
 // One-token decode step.

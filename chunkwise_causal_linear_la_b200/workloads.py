@@ -12,7 +12,8 @@ CPU generator seeded the same way (``randint(lo, hi + 1, (n,))``), so the
 lengths do not depend on the device.  Decode workloads draw q, k, v of shape
 [N, H, d] and then the state [N, H, d_k, d_v] as ``state_std`` * N(0, 1).
 Workloads with a data-dependent decay then draw its log, g [B, T, H], uniform
-in [ln lo, ln hi] (``gate = (lo, hi)``), from a second generator seeded with seed + 1.
+in [ln lo, ln hi] (``gate = (lo, hi)``), from a second generator seeded with seed + 1,
+and gated-delta workloads a write strength beta [B, T, H] uniform in [0.1, 1) after it.
 """
 from __future__ import annotations
 
@@ -39,6 +40,7 @@ class Workload:
     chunk: int = 64
     varlen: Optional[tuple] = None  # (n_seqs, lo, hi) for packed batches
     gate: Optional[tuple] = None  # (lo, hi): per-token decays in [lo, hi] (log drawn uniform)
+    delta: bool = False  # gated delta rule: also a write strength beta per token, U[0.1, 1)
 
     @property
     def torch_dtype(self):
@@ -83,6 +85,11 @@ WORKLOADS = {
     "gated_T16384": Workload(
         "gated_B8_H16_d128_T16384", B=8, T=16384, H=16, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=(1.0,) * 16, phi="identity", normalize=False, gate=(0.9, 0.999),
+    ),
+    "gdelta_T16384": Workload(
+        "gated_delta_B8_H16_d128_T16384", B=8, T=16384, H=16, d_k=128, d_v=128, dtype="bf16",
+        scale=1.0 / math.sqrt(128), gamma=(1.0,) * 16, phi="identity", normalize=False, gate=(0.9, 0.999),
+        delta=True,
     ),
     "long_1m": Workload(
         "long_B1_H4_T1048576_d128", B=1, T=1 << 20, H=4, d_k=128, d_v=128, dtype="bf16",
@@ -150,6 +157,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", T: Optional[int] = Non
         gen = torch.Generator(device=device)
         gen.manual_seed(seed + 1)
         x["g"] = make_log_decay(Bq, Tq, w.H, w.gate[0], w.gate[1], gen, device)
+        if w.delta:
+            x["beta"] = torch.rand((Bq, Tq, w.H), generator=gen, device=device, dtype=torch.float32) * 0.9 + 0.1
     return x
 
 

@@ -176,6 +176,31 @@ LA_API la_status la_fwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
                                     int32_t flags, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * la_fwd_gated_delta -- the gated delta rule ("1.6 长上下文与高效注意力", section
+ * Gated delta rule, and its listing), token by token:
+ *     kt  = k_t / max(|k_t|, 1e-12)                       (unit key)
+ *     S_t = alpha_t S_{t-1} (I - beta_t kt kt^T) + beta_t v_t kt^T,   o_t = S_t q_t
+ * with alpha_t = exp(g_t), per (sequence, head); no feature map, no
+ * normaliser (as in the section).  One call covers prefill and decode (T = 1
+ * with the state passed in and out).
+ *   q, k [B, T, H, d_k]; v [B, T, H, d_v]; out [B, T, H, d_v]; one dtype.
+ *   g, beta     device float[B, T, H], contiguous: log decay (<= 0) and write
+ *               strength (in (0, 1]) of each token.
+ *   cu_seqlens, n_seqs  as for la_fwd_chunk.
+ *   initial_state  NULL (zero) or device float[n_seqs, H, d_k, d_v] holding S^T.
+ *   final_state    NULL or device float[n_seqs, H, d_k, d_v]: S^T after the last
+ *               token; may be the same buffer as initial_state (updated in place).
+ * CUDA cores, fp32 state and arithmetic: each thread keeps one value column's
+ * state in registers and walks the tokens in order (latency-bound, not a
+ * chunked kernel).  d_k, d_v in {16, 32, 64, 128, 256}.  Errors as for
+ * la_fwd_chunk.
+ */
+LA_API la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                                    const float *beta, const int32_t *cu_seqlens, int64_t n_seqs,
+                                    const float *initial_state, const la_tensor *out, float *final_state,
+                                    void *stream);
+
+/*
  * la_norm_gate -- the output norm and gate of a retention layer, on its own:
  *     y[r] = o[r] / sqrt(mean_r' o[r']^2 + eps) * w[r] * gate[r] * sigmoid(gate[r])
  * per (token, head) over the d_v values ("使用 FlashAttention 内核实现最先进的线性注意力":
