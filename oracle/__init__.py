@@ -86,6 +86,9 @@ def _load():
         lib.oracle_norm_gate.restype = i32
         lib.oracle_gated_delta.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, dp, vp, i64, dp, dp, dp, i32]
         lib.oracle_gated_delta.restype = i32
+        lib.oracle_gated_delta_chunked.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, dp, vp, i64, dp,
+                                                   i64, dp, dp, i32]
+        lib.oracle_gated_delta_chunked.restype = i32
         lib.oracle_step.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
@@ -354,4 +357,25 @@ def gated_delta(q, k, v, g, beta, cu_seqlens=None, init=None, nthreads=0):
                                     n, _ptr(ii), _ptr(out), _ptr(fs), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_gated_delta rejected its arguments (code %d)" % rc)
+    return out, fs
+
+
+def gated_delta_chunked(q, k, v, g, beta, chunk, cu_seqlens=None, init=None, nthreads=0):
+    """The gated delta rule regrouped into chunks of `chunk` tokens (float64): per chunk
+    the unit lower-triangular system for the writes u_i is solved by T = (I + A)^{-1}.
+    Same arguments and results as :func:`gated_delta`, equal to them up to rounding."""
+    q, k, v, dt, B, T, H, dk, dv, _, cu, n = _prep(q, k, v, np.ones(q.shape[2]), cu_seqlens)
+    gg = np.ascontiguousarray(np.asarray(g, dtype=np.float64))
+    bb = np.ascontiguousarray(np.asarray(beta, dtype=np.float64))
+    if gg.shape != (B, T, H) or bb.shape != (B, T, H):
+        raise ValueError("g and beta must be [B, T, H]")
+    ii = None if init is None else np.ascontiguousarray(np.asarray(init, dtype=np.float64))
+    if ii is not None and ii.shape != (n, H, dk, dv):
+        raise ValueError("init must be [N, H, d_k, d_v]")
+    out = np.zeros((B, T, H, dv), np.float64)
+    fs = np.zeros((n, H, dk, dv), np.float64)
+    rc = _load().oracle_gated_delta_chunked(_ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(gg), _ptr(bb),
+                                            _ptr(cu), n, _ptr(ii), int(chunk), _ptr(out), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_gated_delta_chunked rejected its arguments (code %d)" % rc)
     return out, fs

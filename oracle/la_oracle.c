@@ -34,6 +34,9 @@
  *                        recurrence: the adjoint of the definition.
  *   oracle_norm_gate  -- RMSNorm over d_v times a Swish gate, per (token, head).
  *   oracle_gated_delta -- the gated delta rule, token by token.
+ *   oracle_gated_delta_chunked -- the same rule regrouped into chunks (the
+ *                        WY / UT form of a chunked kernel), to pin that
+ *                        algebra against the token-by-token definition.
  *   oracle_recurrent_gated, oracle_step_gated -- the same with a per-token
  *                        (per decode step) decay alpha_t = exp(g_t) in place
  *                        of the per-head constant gamma.
@@ -680,6 +683,145 @@ int oracle_gated_delta(const void *q, const void *k, const void *v, int dtype, i
     free(S);
     free(kt);
     free(u);
+  }
+  return 0;
+}
+
+/*
+ * oracle_gated_delta_chunked -- the gated delta rule restated over chunks of
+ * C tokens (float64).  It checks the chunk algebra that a chunked kernel uses
+ * against the token-by-token definition; the pages give only the recurrence.
+ * Inside a chunk that starts from state S_0, let b_i be the sum of g over the
+ * chunk's tokens 0..i and write the update of token i as
+ *   S_i = alpha_i S_{i-1} + u_i kt_i^T,   u_i = beta_i (v_i - alpha_i S_{i-1} kt_i),
+ * so that S_i = e^{b_i} S_0 + sum_{j<=i} e^{b_i - b_j} u_j kt_j^T.  Putting that
+ * S_{i-1} into u_i gives a unit lower-triangular system for the rows u_i:
+ *   u_i + sum_{j<i} A_ij u_j = beta_i v_i - beta_i e^{b_i} S_0 kt_i,
+ *   A_ij = beta_i e^{b_i - b_j} (kt_i . kt_j)   (j < i),
+ * so with T = (I + A)^{-1}:  U = T diag(beta) V - T diag(beta e^b) Kt S_0^T.
+ * Then o_i = e^{b_i} S_0 q_i + sum_{j<=i} e^{b_i - b_j} (q_i . kt_j) u_j, and
+ * the next chunk starts from e^{b_last} S_0 + sum_j e^{b_last - b_j} u_j kt_j^T.
+ * T is formed column by column by forward substitution.  Arguments as for
+ * oracle_gated_delta, plus chunk >= 1.
+ */
+int oracle_gated_delta_chunked(const void *q, const void *k, const void *v, int dtype, int64_t B, int64_t T,
+                               int64_t H, int64_t dk, int64_t dv, const double *g, const double *beta,
+                               const int32_t *cu_seqlens, int64_t n_seqs, const double *init, int64_t chunk,
+                               double *out, double *final_state, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, ORC_PHI_IDENTITY);
+  if (rc) return rc;
+  if (!g || !beta) return -10;
+  if (chunk < 1) return -11;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+  const int64_t C = chunk;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double)); /* S[r][c] */
+    double *Kt = (double *)malloc((size_t)(C * dk) * sizeof(double));
+    double *Q = (double *)malloc((size_t)(C * dk) * sizeof(double));
+    double *V = (double *)malloc((size_t)(C * dv) * sizeof(double));
+    double *A = (double *)malloc((size_t)(C * C) * sizeof(double));
+    double *Ti = (double *)malloc((size_t)(C * C) * sizeof(double));
+    double *U = (double *)malloc((size_t)(C * dv) * sizeof(double));
+    double *X = (double *)malloc((size_t)(C * (dk > dv ? dk : dv)) * sizeof(double));
+    double *bcum = (double *)malloc((size_t)C * sizeof(double));
+    double *bet = (double *)malloc((size_t)C * sizeof(double));
+    if (init)
+      for (int64_t c = 0; c < dk; ++c)
+        for (int64_t r = 0; r < dv; ++r) S[r * dk + c] = init[task * dk * dv + c * dv + r];
+    for (int64_t t0 = 0; t0 < len; t0 += C) {
+      const int64_t Cp = len - t0 < C ? len - t0 : C;
+      double run = 0.0;
+      for (int64_t i = 0; i < Cp; ++i) {
+        const int64_t row = start + t0 + i;
+        const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+        run += g[row * H + h];
+        bcum[i] = run;
+        bet[i] = beta[row * H + h];
+        double nrm = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          Kt[i * dk + c] = orc_load(k, dtype, qk + c);
+          Q[i * dk + c] = orc_load(q, dtype, qk + c);
+          nrm += Kt[i * dk + c] * Kt[i * dk + c];
+        }
+        nrm = sqrt(nrm);
+        if (nrm < 1e-12) nrm = 1e-12;
+        for (int64_t c = 0; c < dk; ++c) Kt[i * dk + c] /= nrm;
+        for (int64_t r = 0; r < dv; ++r) V[i * dv + r] = orc_load(v, dtype, vb + r);
+      }
+      /* A, strictly lower */
+      for (int64_t i = 0; i < Cp; ++i)
+        for (int64_t j = 0; j < Cp; ++j) {
+          double a = 0.0;
+          if (j < i) {
+            for (int64_t c = 0; c < dk; ++c) a += Kt[i * dk + c] * Kt[j * dk + c];
+            a *= bet[i] * exp(bcum[i] - bcum[j]);
+          }
+          A[i * C + j] = a;
+        }
+      /* T = (I + A)^{-1}: column j solves (I + A) x = e_j */
+      for (int64_t j = 0; j < Cp; ++j)
+        for (int64_t i = 0; i < Cp; ++i) {
+          double x = i == j ? 1.0 : 0.0;
+          for (int64_t m = j; m < i; ++m) x -= A[i * C + m] * Ti[m * C + j];
+          Ti[i * C + j] = i < j ? 0.0 : x;
+        }
+      /* U = T diag(beta) V - T diag(beta e^b) (Kt S_0^T) */
+      for (int64_t i = 0; i < Cp; ++i) /* X = Kt S_0^T: X[i][r] = sum_c Kt[i][c] S[r][c] */
+        for (int64_t r = 0; r < dv; ++r) {
+          double acc = 0.0;
+          for (int64_t c = 0; c < dk; ++c) acc += Kt[i * dk + c] * S[r * dk + c];
+          X[i * dv + r] = acc;
+        }
+      for (int64_t i = 0; i < Cp; ++i)
+        for (int64_t r = 0; r < dv; ++r) {
+          double acc = 0.0;
+          for (int64_t j = 0; j <= i; ++j)
+            acc += Ti[i * C + j] * bet[j] * (V[j * dv + r] - exp(bcum[j]) * X[j * dv + r]);
+          U[i * dv + r] = acc;
+        }
+      /* outputs */
+      for (int64_t i = 0; i < Cp; ++i) {
+        const int64_t row = start + t0 + i;
+        const int64_t vb = (row * H + h) * dv;
+        for (int64_t r = 0; r < dv; ++r) {
+          double inter = 0.0;
+          for (int64_t c = 0; c < dk; ++c) inter += S[r * dk + c] * Q[i * dk + c];
+          double o = exp(bcum[i]) * inter;
+          for (int64_t j = 0; j <= i; ++j) {
+            double qk = 0.0;
+            for (int64_t c = 0; c < dk; ++c) qk += Q[i * dk + c] * Kt[j * dk + c];
+            o += exp(bcum[i] - bcum[j]) * qk * U[j * dv + r];
+          }
+          out[vb + r] = o;
+        }
+      }
+      /* next chunk's start state */
+      const double bl = bcum[Cp - 1];
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) {
+          double acc = exp(bl) * S[r * dk + c];
+          for (int64_t j = 0; j < Cp; ++j) acc += exp(bl - bcum[j]) * U[j * dv + r] * Kt[j * dk + c];
+          S[r * dk + c] = acc;
+        }
+    }
+    if (final_state)
+      for (int64_t c = 0; c < dk; ++c)
+        for (int64_t r = 0; r < dv; ++r) final_state[task * dk * dv + c * dv + r] = S[r * dk + c];
+    free(S);
+    free(Kt);
+    free(Q);
+    free(V);
+    free(A);
+    free(Ti);
+    free(U);
+    free(X);
+    free(bcum);
+    free(bet);
   }
   return 0;
 }

@@ -492,6 +492,54 @@ def test_gated_delta_beta_zero_decay_and_handover(oracle_mod):
         assert np.array_equal(pk[:, s_:e], o1) and np.array_equal(pf[n], f1[0])
 
 
+@pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100])
+def test_gated_delta_chunked_equals_recurrence(oracle_mod, chunk):
+    """The chunk (WY / UT) form of the gated delta rule: per chunk the writes solve
+    a unit lower-triangular system.  It must equal the token-by-token rule for
+    every chunk size, with a partial last chunk, strong and weak decay, beta
+    near 0 and 1, an initial state and a packed batch with an empty sequence."""
+    rng = np.random.default_rng(87 + chunk)
+    T, H, dk, dv = 100, 2, 7, 5
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=88 + chunk)
+    g = np.log(rng.uniform(0.05, 1.0, (1, T, H)))
+    g[0, :, 1] *= 0.01
+    b = rng.uniform(0.0, 1.0, (1, T, H))
+    b[0, ::5, 0] = 1.0
+    S0 = rng.standard_normal((1, H, dk, dv))
+    ref, fref = oracle_mod.gated_delta(q, k, v, g, b, init=S0)
+    out, fs = oracle_mod.gated_delta_chunked(q, k, v, g, b, chunk, init=S0)
+    assert rel(out, ref) < 1e-10 and rel(fs, fref) < 1e-10
+    cu = np.array([0, 37, 37, 38, 100], np.int32)
+    ref, fref = oracle_mod.gated_delta(q, k, v, g, b, cu_seqlens=cu)
+    out, fs = oracle_mod.gated_delta_chunked(q, k, v, g, b, chunk, cu_seqlens=cu)
+    assert rel(out, ref) < 1e-10 and rel(fs, fref) < 1e-10
+    assert not fs[1].any()
+
+
+def test_gated_delta_chunked_single_chunk_matrix_form(oracle_mod):
+    """One chunk holding the whole sequence, written out with numpy matrices from
+    the same derivation (A, T = (I + A)^{-1}, U, then O and the final state), and
+    the rule itself at alpha = 1: W = T diag(beta) Kt recovers plain delta-rule
+    outputs.  Catches a transposed Kt Kt^T, a missing beta or a decay on the wrong side."""
+    rng = np.random.default_rng(89)
+    T, dk, dv = 11, 4, 3
+    q, k, v = rand_qkv(1, T, 1, dk, dv, seed=90)
+    g = np.log(rng.uniform(0.3, 1.0, (1, T, 1)))
+    b = rng.uniform(0.1, 1.0, (1, T, 1))
+    out, fs = oracle_mod.gated_delta_chunked(q, k, v, g, b, T)
+    kt = k[0, :, 0] / np.linalg.norm(k[0, :, 0], axis=1, keepdims=True)
+    bc = np.cumsum(g[0, :, 0])
+    bt = b[0, :, 0]
+    D = np.exp(bc[:, None] - bc[None, :])
+    A = np.tril(bt[:, None] * D * (kt @ kt.T), -1)
+    U = np.linalg.solve(np.eye(T) + A, bt[:, None] * v[0, :, 0])
+    O = (np.tril(D) * (q[0, :, 0] @ kt.T)) @ U
+    Sf = (np.exp(bc[-1] - bc)[:, None] * kt).T @ U
+    assert rel(out[0, :, 0], O) < 1e-12 and rel(fs[0, 0], Sf) < 1e-12
+    ref, fref = oracle_mod.gated_delta(q, k, v, g, b)
+    assert rel(out, ref) < 1e-10 and rel(fs, fref) < 1e-10
+
+
 # ---------------------------------------------------------------- chunked form
 @pytest.mark.parametrize("chunk", [1, 2, 3, 7, 16, 64, 100, 130])
 @pytest.mark.parametrize("phi,normalize", [("identity", False), ("elu1", True)])
