@@ -395,10 +395,14 @@ def main():
         ng_gate, ng_w = make_norm_gate(v, seed=rank_seed(rank))
 
     gbeta = x.get("beta")  # gated delta rule workloads
+    if gbeta is not None:  # the chunked (WY) path keeps W and T diag(beta) V in its workspace
+        nws = la.gated_delta_workspace_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, q.dtype)
+        wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
 
     def step():
         if gbeta is not None:
-            la.la_fwd_gated_delta(q, k, v, gd, gbeta, cu_seqlens=cu, out=out, final_state=fs, stream=stream)
+            la.la_fwd_gated_delta_chunk(q, k, v, gd, gbeta, cu_seqlens=cu, out=out, final_state=fs,
+                                        workspace=wsbuf, stream=stream)
         elif args.normgate:
             la.la_fwd_chunk_normgate(q, k, v, g, ng_gate, ng_w, eps=1e-5, cu_seqlens=cu, chunk=w.chunk, phi=w.phi,
                                      normalize=w.normalize, out=out, final_state=fs, workspace=wsbuf, stream=stream)
@@ -458,6 +462,8 @@ def main():
     # (a packed batch with a workspace has its longest-first order computed first: 2 launches)
     launches_per_step = (7 if w.phi == "elu1" else 3) if args.bwd else (
         (2 if cu is not None else 3) if nws > 0 else 1)
+    if gbeta is not None:  # chunk offsets (packed batches), the per-chunk WY pass, the sequential pass
+        launches_per_step = (3 if cu is not None else 2) if nws > 0 else 1
     clocks = sampler.summary(t_wall0, t_wall1)
 
     # ---- parity on sampled (sequence, head) slices, float64 oracle (rank 0)
@@ -567,7 +573,8 @@ def main():
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "launch_ms": launch_ms,
                          "kernel": "chunk_tc_kernel (3 passes: forward + 2 in reverse time)" if args.bwd
-                         else ("delta_kernel" if gbeta is not None else "chunk_tc_kernel")},
+                         else ("gdn_prep_kernel + gdn_tc_kernel (whole step)" if gbeta is not None
+                               else "chunk_tc_kernel")},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
             "parity": parity, "extra": extra,
         }

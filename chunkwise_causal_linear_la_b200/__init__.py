@@ -24,6 +24,8 @@ from .binding import (  # noqa: F401
     la_fwd_chunk_normgate,
     la_fwd_chunk_z,
     la_fwd_gated_delta,
+    la_fwd_gated_delta_chunk,
+    gated_delta_workspace_size,
     la_norm_gate,
     la_step,
     la_step_gated,

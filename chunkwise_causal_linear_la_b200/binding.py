@@ -30,7 +30,7 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
            "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
-           "la_fwd_gated_delta")
+           "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size")
 
 
 class LaTensor(ctypes.Structure):
@@ -85,6 +85,10 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_chunk_normgate.restype = i32
     lib.la_fwd_gated_delta.argtypes = [P, P, P, vp, vp, vp, i64, vp, P, vp, vp]
     lib.la_fwd_gated_delta.restype = i32
+    lib.la_fwd_gated_delta_chunk.argtypes = [P, P, P, vp, vp, vp, i64, vp, P, vp, i32, vp, sz, vp]
+    lib.la_fwd_gated_delta_chunk.restype = i32
+    lib.la_fwd_gated_delta_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32]
+    lib.la_fwd_gated_delta_workspace_size.restype = sz
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -363,4 +367,46 @@ def la_fwd_gated_delta(q, k, v, g, beta, cu_seqlens=None, initial_state=None, ou
                                 None if initial_state is None else initial_state.data_ptr(), ctypes.byref(t[3]),
                                 None if final_state is None else final_state.data_ptr(), _stream(stream))
     _check(lib, st, "la_fwd_gated_delta")
+    return out, final_state
+
+
+def gated_delta_workspace_size(B, T, H, d_k, d_v, n_seqs, varlen, dtype=torch.bfloat16, flags=0) -> int:
+    """Bytes of workspace la_fwd_gated_delta_chunk needs (0: none)."""
+    lib = load_library()
+    n = lib.la_fwd_gated_delta_workspace_size(B, T, H, d_k, d_v, n_seqs, int(bool(varlen)), _DT[dtype], flags)
+    if n == ctypes.c_size_t(-1).value:
+        raise LaError(LA_ERR_INVALID_ARG, "la_fwd_gated_delta_workspace_size rejected the arguments")
+    return n
+
+
+def la_fwd_gated_delta_chunk(q, k, v, g, beta, cu_seqlens=None, initial_state=None, out=None, final_state=None,
+                             return_final_state=True, flags=0, workspace=None, stream=None):
+    """Gated delta rule in chunks (see la_fwd_gated_delta_chunk in include/la_b200.h): same
+    arguments and results as :func:`la_fwd_gated_delta`, plus flags and an optional
+    caller-owned workspace (allocated here when None)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("g", g), ("beta", beta)):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, T, H) or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous float32 [B, T, H] tensor" % name)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32, device=q.device)
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    need = gated_delta_workspace_size(B, T, H, dk, dv, n_seqs, cu_seqlens is not None, q.dtype, flags)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    t = [describe(x) for x in (q, k, v, out)]
+    st = lib.la_fwd_gated_delta_chunk(ctypes.byref(t[0]), ctypes.byref(t[1]), ctypes.byref(t[2]), g.data_ptr(),
+                                      beta.data_ptr(), None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                                      n_seqs, None if initial_state is None else initial_state.data_ptr(),
+                                      ctypes.byref(t[3]), None if final_state is None else final_state.data_ptr(),
+                                      int(flags), None if workspace is None else workspace.data_ptr(),
+                                      0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                      _stream(stream))
+    _check(lib, st, "la_fwd_gated_delta_chunk")
     return out, final_state

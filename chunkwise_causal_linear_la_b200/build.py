@@ -46,23 +46,25 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-# The tensor-core kernel re-splits its registers between warpgroups with
-# setmaxnreg (.dec to 120 and 152, .inc to 232), which is only valid if the
-# kernel launches with exactly this many registers per thread.
+# The warp-specialised tensor-core kernels re-split their registers between
+# warpgroups with setmaxnreg (.dec to 104, .inc to 232), which is only valid if
+# the kernel launches with exactly this many registers per thread.
 TC_LAUNCH_REGS = 168
+# source file -> kernel whose launch register count is checked
+TC_KERNELS = {"la_tc.cu": "chunk_tc_kernel", "la_gdn.cu": "gdn_tc_kernel"}
 
 
-def _check_tc_registers(ptxas_log: str) -> None:
+def _check_tc_registers(ptxas_log: str, kernel: str, src: str) -> None:
     regs, entry = [], None
     for line in ptxas_log.splitlines():
         if "Compiling entry function" in line:
             entry = line
-        elif "Used" in line and "registers" in line and entry and "chunk_tc_kernel" in entry:
+        elif "Used" in line and "registers" in line and entry and kernel in entry:
             regs.append(int(line.split("Used")[1].split("registers")[0]))
             entry = None
     if not regs or any(r != TC_LAUNCH_REGS for r in regs):
-        raise RuntimeError("tensor-core kernel launch registers %s != %d: the setmaxnreg split in la_tc.cu "
-                           "must be revised" % (regs, TC_LAUNCH_REGS))
+        raise RuntimeError("%s launch registers %s != %d: the setmaxnreg split in %s must be revised"
+                           % (kernel, regs, TC_LAUNCH_REGS, src))
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
@@ -77,7 +79,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
         objs.append(obj)
         cmd = [nv, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
-        if src.endswith("la_tc.cu"):
+        if os.path.basename(src) in TC_KERNELS:
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
@@ -90,8 +92,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
             sys.stderr.write(text)
         if p.returncode:
             failed.append(os.path.basename(src))
-        elif src.endswith("la_tc.cu"):
-            _check_tc_registers(text)
+        elif os.path.basename(src) in TC_KERNELS:
+            _check_tc_registers(text, TC_KERNELS[os.path.basename(src)], os.path.basename(src))
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
     tmp = LIB + ".tmp.%d" % os.getpid()

@@ -290,11 +290,12 @@ int32_t la_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
 la_status la_device_error(uint32_t *flags, uint32_t *detail, int32_t reset) {
   if (!flags || !detail) return fail(LA_ERR_INVALID_ARG, "flags and detail must not be NULL");
-  unsigned int f = 0, w = 0;
+  unsigned int f = 0, w = 0, f2 = 0, w2 = 0;
   cudaError_t err = tc_device_error(&f, &w, reset != 0);
+  if (err == cudaSuccess) err = gdn_device_error(&f2, &w2, reset != 0);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(err));
-  *flags = f;
-  *detail = w;
+  *flags = f | f2;
+  *detail = w ? w : w2;
   return ok();
 }
 
@@ -352,9 +353,14 @@ la_status la_fwd_chunk_normgate(const la_tensor *q, const la_tensor *k, const la
                     flags, workspace, workspace_bytes, stream, ng);
 }
 
-la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
-                             const float *beta, const int32_t *cu_seqlens, int64_t n_seqs,
-                             const float *initial_state, const la_tensor *out, float *final_state, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation shared by the two gated-delta entry points; fills `a`.
+la_status delta_setup(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                      const float *beta, const int32_t *cu_seqlens, int64_t n_seqs, const float *initial_state,
+                      const la_tensor *out, float *final_state, DeltaArgs &a) {
   la_status s;
   const la_tensor *ts[4] = {q, k, v, out};
   const char *names[4] = {"q", "k", "v", "out"};
@@ -380,7 +386,6 @@ la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_te
   if (!head_dim_ok(q->D) || !head_dim_ok(v->D))
     return fail(LA_ERR_UNSUPPORTED, "head dims (%lld, %lld) not in {16, 32, 64, 128, 256}",
                 (long long)q->D, (long long)v->D);
-  DeltaArgs a;
   a.q = view(q);
   a.k = view(k);
   a.v = view(v);
@@ -399,10 +404,61 @@ la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_te
   a.dk = (int)q->D;
   a.dv = (int)v->D;
   a.dtype = q->dtype;
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int64_t n_seqs,
+                             const float *initial_state, const la_tensor *out, float *final_state, void *stream) {
+  DeltaArgs a;
+  la_status s = delta_setup(q, k, v, g, beta, cu_seqlens, n_seqs, initial_state, out, final_state, a);
+  if (s != LA_OK) return s;
   if (n_seqs == 0) return ok();
   const cudaError_t err = launch_delta(a, (cudaStream_t)stream);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "gated delta kernel: %s", cudaGetErrorString(err));
   return ok();
+}
+
+la_status la_fwd_gated_delta_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *g,
+                                   const float *beta, const int32_t *cu_seqlens, int64_t n_seqs,
+                                   const float *initial_state, const la_tensor *out, float *final_state,
+                                   int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+  DeltaArgs a;
+  la_status s = delta_setup(q, k, v, g, beta, cu_seqlens, n_seqs, initial_state, out, final_state, a);
+  if (s != LA_OK) return s;
+  if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (n_seqs == 0) return ok();
+  cudaError_t err;
+  const bool states16 = ((uintptr_t)initial_state) % 16 == 0 && ((uintptr_t)final_state) % 16 == 0;
+  if (!(flags & LA_FLAG_SIMT) && gdn_tc_supported(a) && states16) {
+    const size_t need = gdn_workspace_bytes(q->B, q->T, q->H, a.dk, a.dv, n_seqs, cu_seqlens != nullptr);
+    if (workspace_bytes < need || (need > 0 && !workspace))
+      return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (la_fwd_gated_delta_workspace_size)",
+                  workspace_bytes, need);
+    if (((uintptr_t)workspace) % 256) return fail(LA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const char *why = nullptr;
+    err = launch_gdn_chunk(a, workspace, workspace_bytes, (cudaStream_t)stream, &why);
+    if (err != cudaSuccess)
+      return fail(LA_ERR_CUDA, "chunked gated delta: %s%s%s", cudaGetErrorString(err), why ? ": " : "",
+                  why ? why : "");
+    return ok();
+  }
+  err = launch_delta(a, (cudaStream_t)stream);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "gated delta kernel: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+size_t la_fwd_gated_delta_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                         int64_t n_seqs, int32_t has_cu_seqlens, int32_t dtype, int32_t flags) {
+  if (B < 0 || T < 0 || H <= 0 || n_seqs < 0 || !head_dim_ok(d_k) || !head_dim_ok(d_v)) return (size_t)-1;
+  if (dtype != LA_F32 && dtype != LA_BF16) return (size_t)-1;
+  if (flags & ~LA_FLAG_SIMT) return (size_t)-1;
+  if (dtype == LA_F32 || (flags & LA_FLAG_SIMT)) return 0;
+  return gdn_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0);
 }
 
 la_status la_norm_gate(const la_tensor *o, const la_tensor *gate, const float *w, float eps, const la_tensor *y,

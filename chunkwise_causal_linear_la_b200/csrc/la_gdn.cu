@@ -1,0 +1,964 @@
+// la_gdn.cu -- the gated delta rule in chunks, on the sm_100a tensor cores
+// (tcgen05 + TMA + TMEM), bf16 inputs, fp32 accumulation and state.
+//
+// The rule ("1.6 长上下文与高效注意力", section Gated delta rule): with unit keys
+// kt_t = k_t / max(|k_t|, 1e-12) and alpha_t = exp(g_t),
+//     S_t = alpha_t S_{t-1} (I - beta_t kt_t kt_t^T) + beta_t v_t kt_t^T,   o_t = S_t q_t.
+// Regrouped over a chunk of C tokens that starts from state S_0 (b_i = the sum
+// of g over the chunk's tokens 0..i), token i writes u_i kt_i^T with
+// u_i = beta_i (v_i - alpha_i S_{i-1} kt_i), so
+//     S_i = e^{b_i} S_0 + sum_{j<=i} e^{b_i - b_j} u_j kt_j^T.
+// Putting that S_{i-1} into u_i makes the rows u_i the solution of a unit
+// lower-triangular system.  With A_ij = beta_i e^{b_i - b_j} (kt_i . kt_j) for
+// j < i and T = (I + A)^{-1} (the "UT transform" of the chunk):
+//     U  = Ut - W S_0^T,     Ut = T diag(beta) V,     W = T diag(beta e^b) Kt,
+//     O  = diag(e^b) Q S_0^T + (tril(Q Kt^T) .* D) U,      D_ij = e^{b_i - b_j},
+//     S' = e^{b_last} S_0 + (diag(e^{b_last - b}) Kt)^T U.
+// Ut and W depend on the chunk's own inputs only; U, O and S' need the state.
+// Two kernels:
+//   gdn_prep_kernel  one CTA per (sequence, chunk, head), all independent: unit
+//                    keys; G = Kt Kt^T on the tensor cores; A from G; T by
+//                    forward substitution on the CUDA cores (fp32); then
+//                    [W | Ut] = T [diag(beta e^b) Kt | diag(beta) V] on the
+//                    tensor cores, stored as bf16 [B, T, H, 128] in the workspace.
+//   gdn_tc_kernel    one CTA per (sequence, head) walks its chunks in order with
+//                    the fp32 state S^T in registers, as the linear-attention
+//                    forward does.  Per chunk, five products:
+//                      MW  WS = W Sb                 (M=C, N=d_v, K=d_k)   Sb = bf16(S^T)
+//                      M1  A  = Q Kt^T               (M=C, N=C,   K=d_k)
+//                      M4  Us = Kd^T U               (M=d_k, N=d_v, K=C)   Kd = diag(e^{b_last-b}) Kt
+//                      M2  O  = Qd Sb                (M=C, N=d_v, K=d_k)   Qd = diag(e^b) Q
+//                      M3  O += P U                  (M=C, N=d_v, K=C)     P = tril(A) .* D
+//                    with U = Ut - WS between MW and M4 and S^T <- e^{b_last} S^T + Us after M4.
+//   Warp roles of gdn_tc_kernel (384 threads, as in the forward):
+//     warp 0      TMA producer: Q, K, W, Ut chunk tiles into a two-deep ring.
+//     warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
+//     warps 2-3   transform: unit keys Kt in place, decayed unit keys Kd, and
+//                 the chunk's table of b_i.
+//     warps 4-7   state: S^T update, the bf16 operand Sb, and U = Ut - WS in place.
+//     warps 8-11  output: score tile -> P, Qd in place, epilogue.
+// Every wait is bounded: on a timeout the CTA raises an abort flag, records the
+// failure in a device error word, drains and frees its tensor memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "la_common.cuh"
+#include "la_internal.h"
+#include "la_sm100.cuh"
+#include "la_tc_sync.cuh"
+
+namespace la {
+
+__device__ unsigned int g_gdn_error = 0;
+// First wait that gave up: 0x80000000 | chunk << 8 | barrier index.
+__device__ unsigned int g_gdn_where = 0;
+
+namespace {
+
+using namespace sm100;
+using namespace tcsync;
+
+constexpr int kC = 64;            // chunk length
+constexpr int kD = 128;           // d_k = d_v on this path
+constexpr int kSlab = kC * 128;   // one [C rows x 64 cols] bf16 slab, 128-byte swizzled
+constexpr int kTile = 2 * kSlab;  // one [C x 128] tile
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset of the 16-byte chunk holding logical columns [8p, 8p + 8) of row r
+// in a 128-byte-swizzled [rows x 64] slab.
+__device__ __forceinline__ int swz(int r, int p) { return r * 128 + ((p ^ (r & 7)) << 4); }
+
+// Start-address offset (16-byte units) of K step kk (16 columns) in a K-major
+// operand made of 64-column slabs.
+__device__ __forceinline__ uint32_t kmaj(int kk) { return (uint32_t)(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4); }
+
+// Sequence, first token and length of sequence n: dense batches hold B
+// sequences of T tokens; packed ones one row of sequences cut by cu_seqlens.
+struct SeqPos {
+  int64_t bidx, start, len;
+};
+__device__ __forceinline__ SeqPos seq_pos(const int32_t *cu, int64_t n, int64_t T) {
+  if (cu) return SeqPos{0, (int64_t)cu[n], (int64_t)cu[n + 1] - cu[n]};
+  return SeqPos{n, 0, T};
+}
+
+// ============================================================== prep kernel
+struct PrepArgs {
+  const float *g, *beta;      // [B * T][H]
+  const int32_t *cu_seqlens;  // NULL: dense
+  const int32_t *coff;        // packed: first chunk slot of each sequence, [n_seqs + 1]
+  __nv_bfloat16 *w, *ut;      // [B, T, H, 128] each
+  int64_t T, n_seqs;
+  int H;
+};
+
+struct PrepCfg {
+  static constexpr int OFF_K = 0;              // K, then unit keys, then diag(beta e^b) Kt
+  static constexpr int OFF_V = OFF_K + kTile;  // V, then diag(beta) V: [K | V] is one 4-slab operand
+  static constexpr int OFF_T = OFF_V + kTile;  // T = (I + A)^{-1}, bf16 [C x C] K-major
+  static constexpr int OFF_A = OFF_T + kSlab;  // A, fp32 [C][A_LD]
+  static constexpr int A_LD = kC + 4;          // rows 16-byte aligned for float4 reads
+  static constexpr int OFF_VEC = OFF_A + kC * A_LD * 4;  // b_i and beta_i, 2 x C floats
+  static constexpr int OFF_BAR = OFF_VEC + 2 * kC * 4;   // 0: tiles landed, 1: MMA done
+  static constexpr int OFF_MISC = OFF_BAR + 2 * 8;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
+  // More than a third of an SM's shared memory: at most two CTAs share an SM,
+  // so their two 256-column tensor-memory allocations always fit.
+  static constexpr int SMEM_BYTES = 80 * 1024;
+  static constexpr int T_COLS = 256;
+  static_assert(SMEM_USED + 1024 <= SMEM_BYTES, "prep shared memory");
+  static_assert(3 * SMEM_BYTES > 232448, "at most two prep CTAs per SM");
+};
+
+// Sequence start slots of a packed batch: coff[n] = sum_{m<n} ceil(len_m / C).
+// One block; the counts are scanned 1024 sequences at a time.
+__global__ void __launch_bounds__(1024) gdn_chunk_offsets_kernel(const int32_t *cu, int64_t n_seqs,
+                                                                 int32_t *coff) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry = 0;
+    coff[0] = 0;
+  }
+  __syncthreads();
+  for (int64_t base = 0; base < n_seqs; base += 1024) {
+    const int64_t n = base + tid;
+    int32_t x = n < n_seqs ? (int32_t)(((int64_t)cu[n + 1] - cu[n] + kC - 1) / kC) : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t s = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      warp_sums[lane] = s;
+    }
+    __syncthreads();
+    const int32_t incl = x + (warp > 0 ? warp_sums[warp - 1] : 0) + carry;
+    if (n < n_seqs) coff[n + 1] = incl;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                       const __grid_constant__ CUtensorMap tm_v,
+                                                       const PrepArgs a) {
+  using P = PrepCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = align1024(smem_raw);
+  float *As = reinterpret_cast<float *>(sm + P::OFF_A);
+  float *bvec = reinterpret_cast<float *>(sm + P::OFF_VEC);
+  float *betav = bvec + kC;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P::OFF_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P::OFF_MISC + 4);
+  const Sync sy{bars, abort_flag, &g_gdn_error, &g_gdn_where};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- this CTA's (sequence, chunk, head); heads vary fastest
+  const int h = (int)(blockIdx.x % a.H);
+  const int64_t slot = blockIdx.x / a.H;
+  int64_t n, c;
+  if (a.coff) {
+    if (slot >= a.coff[a.n_seqs]) return;  // past the last chunk (the grid is an upper bound)
+    int64_t lo = 0, hi = a.n_seqs - 1;     // last n with coff[n] <= slot
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (a.coff[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    c = slot - a.coff[n];
+  } else {
+    const int64_t nck = (a.T + kC - 1) / kC;
+    n = slot / nck;
+    c = slot % nck;
+  }
+  const SeqPos sp = seq_pos(a.cu_seqlens, n, a.T);
+  const int64_t t0 = sp.start + c * kC;  // first token of the chunk in its batch row
+  const int Cp = (int)min((int64_t)kC, sp.len - c * kC);
+
+  // ---- setup: barriers, tensor memory, the tile loads, b_i and beta_i
+  if (tid == 0) {
+    mbar_init(bars + 0, 1);
+    mbar_init(bars + 1, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bars + 0, 2 * kTile);
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_4d(sm + P::OFF_K + kb * kSlab, &tm_k, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
+      tma_load_4d(sm + P::OFF_V + kb * kSlab, &tm_v, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
+    }
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, P::T_COLS);
+  if (warp == 0) {  // b_i = sum_{t<=i} g_t over the chunk (rows past its end add 0 and get beta = 0)
+    const int64_t row0 = (sp.bidx * a.T + t0) * a.H + h;
+    float blo = lane < Cp ? a.g[row0 + (int64_t)lane * a.H] : 0.f;
+    float bhi = lane + 32 < Cp ? a.g[row0 + (int64_t)(lane + 32) * a.H] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y0 = __shfl_up_sync(0xffffffffu, blo, o);
+      const float y1 = __shfl_up_sync(0xffffffffu, bhi, o);
+      if (lane >= o) {
+        blo += y0;
+        bhi += y1;
+      }
+    }
+    bhi += __shfl_sync(0xffffffffu, blo, 31);
+    bvec[lane] = blo;
+    bvec[lane + 32] = bhi;
+    betav[lane] = lane < Cp ? a.beta[row0 + (int64_t)lane * a.H] : 0.f;
+    betav[lane + 32] = lane + 32 < Cp ? a.beta[row0 + (int64_t)(lane + 32) * a.H] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  bool ok = wait_bar_warp(sy, 0, 0);
+  int issued = 0;  // products committed on barrier 1 (thread 0)
+
+  // ---- unit keys in place; rows past the chunk end become zero (keys and values)
+  const int ri = tid >> 1, hh = tid & 1;  // row and 64-column half handled by this thread
+  uint8_t *krow = sm + P::OFF_K + hh * kSlab + ri * 128;
+  uint8_t *vrow = sm + P::OFF_V + hh * kSlab + ri * 128;
+  if (ok) {
+    uint4 x[8];
+    float ss = 0.f;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      x[p] = *reinterpret_cast<const uint4 *>(krow + p * 16);
+      float f[8];
+      unpack8(x[p], f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ss = fmaf(f[u], f[u], ss);
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const float inv = ri < Cp ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float f[8];
+      unpack8(x[p], f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] *= inv;
+      *reinterpret_cast<uint4 *>(krow + p * 16) = pack8(f);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  // G = Kt Kt^T (M = N = C, K = 128) into columns [0, C)
+  if (ok && tid == 0) {
+    tc_fence_after();
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + P::OFF_K), 16, 1024);
+    constexpr uint32_t ID_G = idesc_bf16_f32(kC, kC, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) umma_bf16(tbase, dk + kmaj(kk), dk + kmaj(kk), ID_G, kk > 0);
+    umma_commit(bars + 1);
+    issued = 1;
+  }
+  // diag(beta) V in place, while the product runs (it does not read V)
+  if (ok) {
+    const float bt = betav[ri];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint4 x = *reinterpret_cast<const uint4 *>(vrow + p * 16);
+      float f[8];
+      unpack8(x, f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = ri < Cp ? f[u] * bt : 0.f;
+      *reinterpret_cast<uint4 *>(vrow + p * 16) = pack8(f);
+    }
+  }
+  ok = ok && wait_bar_warp(sy, 1, 0);
+  tc_fence_after();
+  if (ok) {
+    // A_ij = beta_i e^{b_i - b_j} G_ij for j < i: this thread's row i and 32 columns
+    const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;
+    uint32_t r[32];
+    tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(warp * 32) << 16), r);
+    tmem_wait_ld();
+    const float bi = bvec[i], bt = betav[i];
+    float *arow = As + i * P::A_LD + hf * 32;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = hf * 32 + e;
+      arow[e] = j < i ? bt * expf(bi - bvec[j]) * __uint_as_float(r[e]) : 0.f;
+    }
+    // diag(beta e^b) Kt in place (the product above has read Kt)
+    const float wk = betav[ri] * expf(bvec[ri]);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint4 x = *reinterpret_cast<const uint4 *>(krow + p * 16);
+      float f[8];
+      unpack8(x, f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] *= wk;
+      *reinterpret_cast<uint4 *>(krow + p * 16) = pack8(f);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // ---- T = (I + A)^{-1} by forward substitution: thread j solves column j,
+  // x_i = [i == j] - sum_{m<i} A_im x_m (x_m = 0 for m < j), in fp32; all threads
+  // walk the same rows so every read of A is a broadcast.  The bf16 result goes
+  // to the K-major T tile (row i, column j).
+  if (ok && tid < kC) {
+    const int j = tid;
+    float x[kC];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) x[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+      const float4 *a4 = reinterpret_cast<const float4 *>(As + i * P::A_LD);
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int m = 0; m < i; m += 4) {  // A_im = 0 for m >= i and x_m = 0 beyond what is solved
+        const float4 av = a4[m >> 2];
+        s0 = fmaf(av.x, x[m], s0);
+        s1 = fmaf(av.y, x[m + 1], s1);
+        s2 = fmaf(av.z, x[m + 2], s2);
+        s3 = fmaf(av.w, x[m + 3], s3);
+      }
+      x[i] = i < j ? 0.f : (i == j ? 1.f : -((s0 + s1) + (s2 + s3)));
+    }
+    uint8_t *tt = sm + P::OFF_T;
+#pragma unroll
+    for (int i = 0; i < kC; ++i)
+      *reinterpret_cast<__nv_bfloat16 *>(tt + swz(i, j >> 3) + (j & 7) * 2) = __float2bfloat16_rn(x[i]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // [W | Ut] = T [diag(beta e^b) Kt | diag(beta) V]  (M = C, N = 256, K = C) into columns [0, 256)
+  if (ok && tid == 0) {
+    tc_fence_after();
+    const uint64_t dt = smem_desc_sw128(smem_u32(sm + P::OFF_T), 16, 1024);
+    const uint64_t dx = smem_desc_sw128(smem_u32(sm + P::OFF_K), kSlab, 1024);  // MN-major, 4 slabs
+    constexpr uint32_t ID_X = idesc_bf16_f32(kC, 256, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < kC / 16; ++kk) umma_bf16(tbase, dt + kmaj(kk), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
+    umma_commit(bars + 1);
+    issued = 2;
+  }
+  ok = ok && wait_bar_warp(sy, 1, 1);
+  tc_fence_after();
+  if (ok) {
+    // row i, columns [0, 128) (W) for lanes 0-15 and [128, 256) (Ut) for lanes 16-31
+    const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;
+    __nv_bfloat16 *dst = (hf ? a.ut : a.w) + ((sp.bidx * a.T + t0 + i) * a.H + h) * (int64_t)kD;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      uint32_t r[32];
+      tmem_ld_16x32bx2_x32<128>(tbase + ((uint32_t)(warp * 32) << 16) + pass * 32, r);
+      tmem_wait_ld();
+      if (i < Cp) {
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst + pass * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          d4[q] = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                             pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                             pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                             pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      }
+    }
+  }
+  // ---- teardown (after an abort, let the tile loads and products finish first)
+  if (*abort_flag && tid == 0) {
+    drain_bar(sy, 0, 0);
+    for (int u = 0; u < issued; ++u) drain_bar(sy, 1, u & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    tmem_dealloc(tbase, P::T_COLS);
+    tmem_relinquish();
+  }
+}
+
+// ============================================================== chunk kernel
+constexpr int kThreads = 384;
+
+struct GdnTcArgs {
+  void *out;
+  int64_t o_sb, o_st, o_sh;
+  const float *g;             // [B * T][H] log decay
+  const float *init;          // NULL or [n_seqs, H, 128, 128] (S^T)
+  float *final_state;         // NULL or [n_seqs, H, 128, 128]
+  const int32_t *cu_seqlens;  // NULL: dense
+  int64_t T;
+  int H;
+};
+
+template <int NS>
+struct GdnCfg {
+  // a stage: Q (then Qd), K (then Kt), W, Ut (then U), Kd; [C x 128] bf16 tiles
+  static constexpr int OFF_Q = 0, OFF_K = kTile, OFF_W = 2 * kTile, OFF_U = 3 * kTile, OFF_KD = 4 * kTile;
+  static constexpr int STAGE_BYTES = 5 * kTile;
+  static constexpr int LOAD_BYTES = 4 * kTile;  // Q, K, W, Ut arrive by TMA
+  static constexpr int SB_SLAB = kD * 128;      // [d_k rows x 64 cols] bf16
+  static constexpr int OFF_SB = NS * STAGE_BYTES;
+  static constexpr int OFF_P = OFF_SB + 2 * SB_SLAB;
+  static constexpr int OFF_DT = OFF_P + 2 * kSlab;  // per stage: b_i (i < C), b_last at [C]
+  static constexpr int DT_STRIDE = kC + 4;
+  static constexpr int OFF_BAR = OFF_DT + NS * DT_STRIDE * 4;
+  static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_QREADY = 3 * NS, B_AFULL = 4 * NS,
+                       B_PFULL = 4 * NS + 2, B_OFULL = 4 * NS + 4, B_OEMPTY = 4 * NS + 6, B_WSFULL = 4 * NS + 8,
+                       B_UREADY = 4 * NS + 9, B_UFULL = 4 * NS + 10, B_SBFULL = 4 * NS + 11,
+                       B_SBEMPTY = 4 * NS + 12, NBAR = 4 * NS + 13;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+  // tensor memory: Us / WS (time-shared), two score tiles, two output tiles
+  static constexpr int T_U = 0, T_A = 128, T_O = 256, T_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(OFF_BAR % 8 == 0, "barrier alignment");
+};
+
+// Thread roles and per-chunk protocol (chunk c, stage s = c % NS, b = c & 1;
+// "prev" = the chunk starts from a state: c > 0 or an initial state):
+//   MMA:       [prev: FULL, SBFULL] MW -> WSFULL;  [XFORM] M1 -> AFULL[b];
+//              [UREADY] M4 -> UFULL;  [OEMPTY[b], QREADY[s]] prev: M2 -> SBEMPTY;
+//              [PFULL[b]] M3 -> OFULL[b], EMPTY[s].
+//   state:     [UFULL(c-1)] S^T <- e^{b_last} S^T + Us;  [prev: SBEMPTY(c-1)] Sb -> SBFULL;
+//              [XFORM, prev: WSFULL] U = Ut - WS in place -> UREADY.
+//   output:    [AFULL[b], XFORM] P -> PFULL[b];  Qd in place -> QREADY[s];
+//              [OFULL[b-1]] epilogue of chunk c-1 -> OEMPTY.
+//   transform: [FULL] b table, Kt in place, Kd -> XFORM.
+template <int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
+              const GdnTcArgs a) {
+  using G = GdnCfg<NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = align1024(smem_raw);
+  float *dtab = reinterpret_cast<float *>(sm + G::OFF_DT);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + G::OFF_MISC + 4);
+  const Sync sy{bars, abort_flag, &g_gdn_error, &g_gdn_where};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int h = (int)(blockIdx.x % a.H);
+  const int64_t n = blockIdx.x / a.H;
+  const SeqPos sq = seq_pos(a.cu_seqlens, n, a.T);
+  const int nchunks = (int)((sq.len + kC - 1) / kC);
+  const bool has_init = a.init != nullptr;
+  auto chunk_len = [&](int c) -> int { return (int)min((int64_t)kC, sq.len - (int64_t)c * kC); };
+  auto prev = [&](int c) -> bool { return c > 0 || has_init; };
+  // index of chunk c among the chunks that start from a state (parity of SBFULL, WSFULL, SBEMPTY)
+  auto sbi = [&](int c) -> int { return c - 1 + (has_init ? 1 : 0); };
+  auto stage = [&](int s) { return sm + s * G::STAGE_BYTES; };
+
+  if (tid == 0) {
+    for (int i = 0; i < G::NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i >= G::B_XFORM && i < G::B_XFORM + NS) cnt = 64;
+      else if ((i >= G::B_QREADY && i < G::B_QREADY + NS) || (i >= G::B_PFULL && i < G::B_PFULL + 2) ||
+               (i >= G::B_OEMPTY && i < G::B_OEMPTY + 2) || i == G::B_UREADY || i == G::B_SBFULL)
+        cnt = 128;
+      mbar_init(bars + i, cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_u);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, G::T_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp < 4) {
+    reg_dealloc<104>();
+    if (warp == 0 && lane == 0) {
+      // ============================================================ TMA producer
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS;
+        if (!wait_bar(sy, G::B_EMPTY + s, (k & 1) ^ 1, c)) break;
+        mbar_arrive_expect_tx(bars + G::B_FULL + s, G::LOAD_BYTES);
+        const int t0 = (int)(sq.start + (int64_t)c * kC);
+        const int bi = (int)sq.bidx;
+        uint8_t *st = stage(s);
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_4d(st + G::OFF_Q + kb * kSlab, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bi);
+          tma_load_4d(st + G::OFF_K + kb * kSlab, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bi);
+          tma_load_4d(st + G::OFF_W + kb * kSlab, &tm_w, bars + G::B_FULL + s, kb * 64, h, t0, bi);
+          tma_load_4d(st + G::OFF_U + kb * kSlab, &tm_u, bars + G::B_FULL + s, kb * 64, h, t0, bi);
+        }
+        issued = c + 1;
+      }
+      if (*abort_flag) {  // let every issued copy land before the CTA exits
+        for (int c = max(0, issued - NS); c < issued; ++c) drain_bar(sy, G::B_FULL + c % NS, (c / NS) & 1);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ============================================================ MMA issuer
+      constexpr uint32_t ID_S = idesc_bf16_f32(kC, kC, 0, 0);   // scores
+      constexpr uint32_t ID_O = idesc_bf16_f32(kC, kD, 0, 1);   // WS, O
+      constexpr uint32_t ID_U = idesc_bf16_f32(kD, kD, 1, 1);   // state update
+      const uint64_t dsb = smem_desc_sw128(smem_u32(sm + G::OFF_SB), G::SB_SLAB, 1024);
+      // operand descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the
+      // start-address field (no carry: shared addresses are < 256 KB)
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_Q), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_K), 16, 1024);
+      const uint64_t dw0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_W), 16, 1024);
+      const uint64_t du0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_U), kSlab, 1024);   // MN-major
+      const uint64_t dkd0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_KD), kSlab, 1024); // MN-major
+      const uint64_t dp0 = smem_desc_sw128(smem_u32(sm + G::OFF_P), 16, 1024);
+      auto soff = [](int s) -> uint64_t { return (uint64_t)(s * (G::STAGE_BYTES >> 4)); };
+      int done = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS, b = c & 1;
+        const uint32_t o_acc = tbase + G::T_O + b * kD;
+        bool ok = true;
+        // MW: WS = W Sb
+        if (prev(c)) {
+          ok = wait_bar(sy, G::B_FULL + s, k & 1, c) && wait_bar(sy, G::B_SBFULL, sbi(c) & 1, c);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            umma_bf16(tbase + G::T_U, dw0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
+          umma_commit(bars + G::B_WSFULL);
+        }
+        // M1: A = Q Kt^T
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_bf16(tbase + G::T_A + b * kC, dq0 + soff(s) + kmaj(kk), dk0 + soff(s) + kmaj(kk), ID_S, kk > 0);
+        umma_commit(bars + G::B_AFULL + b);
+        // M4: Us = Kd^T U
+        if (!wait_bar(sy, G::B_UREADY, c & 1, c)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          umma_bf16(tbase + G::T_U, dkd0 + soff(s) + ((kk * 2048) >> 4), du0 + soff(s) + ((kk * 2048) >> 4), ID_U,
+                    kk > 0);
+        umma_commit(bars + G::B_UFULL);
+        // M2: O = Qd Sb.  Qd is waited for even without M2: the output warps write
+        // it in place, so the stage must not be released before they are done.
+        if (!wait_bar(sy, G::B_OEMPTY + b, ((c >> 1) & 1) ^ 1, c) || !wait_bar(sy, G::B_QREADY + s, k & 1, c))
+          break;
+        if (prev(c)) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            umma_bf16(o_acc, dq0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
+          umma_commit(bars + G::B_SBEMPTY);
+        }
+        // M3: O += P U
+        if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          umma_bf16(o_acc, dp0 + (uint64_t)(b * (kSlab >> 4)) + kmaj(kk), du0 + soff(s) + ((kk * 2048) >> 4),
+                    ID_O, (prev(c) || kk > 0) ? 1u : 0u);
+        umma_commit(bars + G::B_OFULL + b);
+        umma_commit(bars + G::B_EMPTY + s);
+        done = c + 1;
+      }
+      // the last commits arrive asynchronously: wait for them before tensor memory is freed
+      for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
+      if (done < nchunks && *abort_flag) {  // products of an aborted chunk may still be running
+        const int c = done;
+        drain_bar(sy, G::B_AFULL + (c & 1), (c >> 1) & 1);
+      }
+    } else if (warp >= 2) {
+      // ========================================================== transform
+      // 64 threads; thread tt owns the 16-byte vectors tt + 64 m (m < 8) of both
+      // 64-column slabs of the key tile: row tt/8 + 8 m, physical chunk tt mod 8.
+      // The 8 lanes holding a row differ in their low three bits.
+      const int tt = tid - 64, ln = tt & 31;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS, k = c / NS;
+        if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c)) break;
+        const int Cp = chunk_len(c);
+        // b_i over the chunk (rows past its end add 0): lane l holds b_l and b_{l+32}
+        const int64_t row0 = (sq.bidx * a.T + sq.start + (int64_t)c * kC) * a.H + h;
+        float blo = ln < Cp ? a.g[row0 + (int64_t)ln * a.H] : 0.f;
+        float bhi = ln + 32 < Cp ? a.g[row0 + (int64_t)(ln + 32) * a.H] : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y0 = __shfl_up_sync(0xffffffffu, blo, o);
+          const float y1 = __shfl_up_sync(0xffffffffu, bhi, o);
+          if (ln >= o) {
+            blo += y0;
+            bhi += y1;
+          }
+        }
+        bhi += __shfl_sync(0xffffffffu, blo, 31);
+        const float blast = __shfl_sync(0xffffffffu, Cp <= 32 ? blo : bhi, (Cp - 1) & 31);
+        if (tt < 32) {
+          float *dt = dtab + s * G::DT_STRIDE;
+          dt[ln] = blo;
+          dt[ln + 32] = bhi;
+          if (ln == 0) dt[kC] = blast;
+        }
+        uint8_t *kt = stage(s) + G::OFF_K;
+        uint8_t *kd = stage(s) + G::OFF_KD;
+#pragma unroll 1
+        for (int m = 0; m < 8; ++m) {
+          const int r = (tt >> 3) + 8 * m;
+          const int off = (tt + 64 * m) * 16;
+          uint4 x0 = *reinterpret_cast<const uint4 *>(kt + off);
+          uint4 x1 = *reinterpret_cast<const uint4 *>(kt + kSlab + off);
+          float f0[8], f1[8];
+          unpack8(x0, f0);
+          unpack8(x1, f1);
+          float ss = 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ss = fmaf(f0[u], f0[u], fmaf(f1[u], f1[u], ss));
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+          const float b0 = __shfl_sync(0xffffffffu, blo, r & 31);
+          const float b1 = __shfl_sync(0xffffffffu, bhi, r & 31);
+          const float br = r < 32 ? b0 : b1;
+          const float inv = r < Cp ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
+          const float wd = inv * exp_fast(blast - br);
+          float g0[8], g1[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            g0[u] = f0[u] * wd;
+            g1[u] = f1[u] * wd;
+            f0[u] *= inv;
+            f1[u] *= inv;
+          }
+          *reinterpret_cast<uint4 *>(kt + off) = pack8(f0);
+          *reinterpret_cast<uint4 *>(kt + kSlab + off) = pack8(f1);
+          *reinterpret_cast<uint4 *>(kd + off) = pack8(g0);
+          *reinterpret_cast<uint4 *>(kd + kSlab + off) = pack8(g1);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bars + G::B_XFORM + s);
+      }
+    }
+  } else if (warp < 8) {
+    // ================================================================ state
+    reg_alloc<232>();
+    const int sp = warp & 3;
+    const int kr = sp * 32 + lane;  // row of S^T (d_k index) held by this thread
+    const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
+    const int64_t sbase = (n * a.H + h) * (int64_t)kD * kD;
+    float S[kD];
+    if (has_init) {
+      const float4 *src = reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)kr * kD);
+#pragma unroll
+      for (int q = 0; q < kD / 4; ++q) {
+        const float4 x = src[q];
+        S[4 * q] = x.x;
+        S[4 * q + 1] = x.y;
+        S[4 * q + 2] = x.z;
+        S[4 * q + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kD; ++u) S[u] = 0.f;
+    }
+    // Sb = bf16(S^T): two [d_k x 64] slabs, MN-major (row kr, 128-byte swizzle)
+    auto write_sb = [&]() {
+#pragma unroll
+      for (int grp = 0; grp < kD / 32; ++grp) {
+        uint8_t *row = sm + G::OFF_SB + (grp >> 1) * G::SB_SLAB + kr * 128;
+        const int ch0 = (grp & 1) * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float *x = &S[grp * 32 + 8 * q];
+          *reinterpret_cast<uint4 *>(row + (((ch0 + q) ^ (kr & 7)) << 4)) =
+              make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + G::B_SBFULL);
+    };
+    const int i = sp * 16 + (lane & 15), hf = lane >> 4;  // U row and column half of this thread
+    float gdec = 1.f;  // e^{b_last} of the previous chunk
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int s = c % NS, k = c / NS;
+      ok = false;
+      if (c > 0) {  // S^T <- e^{b_last} S^T + Us of chunk c - 1
+        if (!wait_bar_warp(sy, G::B_UFULL, (c - 1) & 1, c)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int grp = 0; grp < kD / 32; ++grp) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(lane_base + G::T_U + grp * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) S[grp * 32 + e] = fmaf(gdec, S[grp * 32 + e], __uint_as_float(r[e]));
+        }
+      }
+      if (prev(c)) {  // Sb of chunk c, once the products of chunk c - 1 have read the previous one
+        if (sbi(c) >= 1 && !wait_bar_warp(sy, G::B_SBEMPTY, (sbi(c) - 1) & 1, c)) break;
+        write_sb();
+      }
+      if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c) || !wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) break;
+      const float blast = dtab[s * G::DT_STRIDE + kC];
+      const int Cp = chunk_len(c);
+      if (prev(c)) {
+        if (!wait_bar_warp(sy, G::B_WSFULL, sbi(c) & 1, c)) break;
+        tc_fence_after();
+      }
+      // U = Ut - WS on row i, columns [64 hf, 64 hf + 64), in place; zero past the chunk end
+      uint8_t *urow = stage(s) + G::OFF_U + hf * kSlab;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t r[32];
+        if (prev(c)) {
+          tmem_ld_16x32bx2_x32<64>(lane_base + G::T_U + pass * 32, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 *p4 = reinterpret_cast<uint4 *>(urow + swz(i, pass * 4 + q));
+          float f[8];
+          unpack8(*p4, f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = i < Cp ? f[u] - __uint_as_float(r[8 * q + u]) : 0.f;
+          *p4 = pack8(f);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + G::B_UREADY);
+      gdec = exp_fast(blast);
+      ok = true;
+    }
+    // the last chunk's update, then the final state (zero for an empty sequence)
+    if (ok && nchunks > 0 && wait_bar_warp(sy, G::B_UFULL, (nchunks - 1) & 1, nchunks)) {
+      tc_fence_after();
+#pragma unroll
+      for (int grp = 0; grp < kD / 32; ++grp) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(lane_base + G::T_U + grp * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) S[grp * 32 + e] = fmaf(gdec, S[grp * 32 + e], __uint_as_float(r[e]));
+      }
+    }
+    if (a.final_state && !*abort_flag) {
+      float4 *dst = reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)kr * kD);
+#pragma unroll
+      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+    }
+  } else {
+    // ================================================================ output
+    const int sp = warp & 3;
+    const int i = sp * 16 + (lane & 15), hf = lane >> 4;  // chunk row and column half of this thread
+    const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
+    uint8_t *obase = reinterpret_cast<uint8_t *>(a.out) + 2 * (sq.bidx * a.o_sb + (int64_t)h * a.o_sh);
+
+    // chunk c: P = tril(A) .* D into P[c & 1], then Qd = diag(e^b) Q in place
+    auto scores = [&](int c) -> bool {
+      const int s = c % NS, k = c / NS, b = c & 1;
+      const int Cp = chunk_len(c);
+      if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return false;
+      tc_fence_after();
+      if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c) || !wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) return false;
+      const float *dt = dtab + s * G::DT_STRIDE;
+      const float bi = dt[i];
+      uint32_t r[32];
+      tmem_ld_16x32bx2_x32<32>(lane_base + G::T_A + b * kC, r);
+      tmem_wait_ld();
+      float f[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = hf * 32 + e;
+        f[e] = (j <= i && i < Cp) ? __uint_as_float(r[e]) * exp_fast(bi - dt[j]) : 0.f;
+      }
+      uint8_t *prow = sm + G::OFF_P + b * kSlab;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(prow + swz(i, hf * 4 + q)) =
+            make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
+                       pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + G::B_PFULL + b);  // also tells the MMA issuer that A[b] has been read
+      // the score product has read Q: scale its row i by e^{b_i} for the inter-chunk product
+      const float qf = i < Cp ? exp_fast(bi) : 0.f;
+      uint8_t *qrow = stage(s) + G::OFF_Q + hf * kSlab + i * 128;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        uint4 *p4 = reinterpret_cast<uint4 *>(qrow + p * 16);
+        float x[8];
+        unpack8(*p4, x);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] *= qf;
+        *p4 = pack8(x);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bars + G::B_QREADY + s);
+      return true;
+    };
+
+    // epilogue of chunk c: O[c & 1] -> bf16 output rows
+    auto epilogue = [&](int c) -> bool {
+      const int b = c & 1;
+      const int Cp = chunk_len(c);
+      if (!wait_bar_warp(sy, G::B_OFULL + b, (c >> 1) & 1, c)) return false;
+      tc_fence_after();
+      const int64_t tok = sq.start + (int64_t)c * kC + i;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t r[32];
+        tmem_ld_16x32bx2_x32<64>(lane_base + G::T_O + b * kD + pass * 32, r);
+        tmem_wait_ld();
+        if (pass == 1) {
+          tc_fence_before();
+          mbar_arrive(bars + G::B_OEMPTY + b);
+        }
+        if (i < Cp) {
+          uint4 *dst = reinterpret_cast<uint4 *>(obase + 2 * (tok * a.o_st + hf * 64 + pass * 32));
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                                pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                                pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                                pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+        }
+      }
+      return true;
+    };
+
+    for (int t = 0; t <= nchunks; ++t) {
+      if (t < nchunks && !scores(t)) break;
+      if (t >= 1 && !epilogue(t - 1)) break;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    tmem_dealloc(tbase, G::T_COLS);
+    tmem_relinquish();
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+constexpr int kStages = 2;
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// W and Ut, bf16 [B, T, H, 128] each, then (packed batches) the chunk offsets
+size_t wu_bytes(int64_t B, int64_t T, int64_t H) { return align256((size_t)(B * T * H) * kD * 2); }
+
+}  // namespace
+
+bool gdn_tc_supported(const DeltaArgs &a) { return a.dtype == LA_BF16 && a.dk == kD && a.dv == kD; }
+
+size_t gdn_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen) {
+  if (dk != kD || dv != kD) return 0;
+  return 2 * wu_bytes(B, T, H) + (varlen ? align256((size_t)(n_seqs + 1) * 4) : 0);
+}
+
+cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                             const char **why) {
+  const int64_t B = a.cu_seqlens ? 1 : a.n_seqs;
+  const bool varlen = a.cu_seqlens != nullptr;
+  const size_t need = gdn_workspace_bytes(B, a.T, a.H, a.dk, a.dv, a.n_seqs, varlen);
+  if (!workspace || workspace_bytes < need) {
+    if (why) *why = "workspace too small for the chunked gated delta rule";
+    return cudaErrorInvalidValue;
+  }
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  __nv_bfloat16 *w = reinterpret_cast<__nv_bfloat16 *>(ws);
+  __nv_bfloat16 *ut = reinterpret_cast<__nv_bfloat16 *>(ws + wu_bytes(B, a.T, a.H));
+  int32_t *coff = varlen ? reinterpret_cast<int32_t *>(ws + 2 * wu_bytes(B, a.T, a.H)) : nullptr;
+  const TensorView wv{w, a.T * a.H * kD, (int64_t)a.H * kD, kD};
+  const TensorView uv{ut, a.T * a.H * kD, (int64_t)a.H * kD, kD};
+  CUtensorMap mq, mk, mv, mw, mu;
+  if (!make_map(&mq, a.q, B, a.T, a.H, kD, kC) || !make_map(&mk, a.k, B, a.T, a.H, kD, kC) ||
+      !make_map(&mv, a.v, B, a.T, a.H, kD, kC) || !make_map(&mw, wv, B, a.T, a.H, kD, kC) ||
+      !make_map(&mu, uv, B, a.T, a.H, kD, kC)) {
+    if (why) *why = "cuTensorMapEncodeTiled rejected a tensor";
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t err;
+  // 1. the per-chunk WY pass (grid: chunk slots x heads; packed batches bound the slot count)
+  const int64_t nck = (a.T + kC - 1) / kC;
+  const int64_t slots = varlen ? nck + a.n_seqs : a.n_seqs * nck;
+  if (slots * a.H > 0x7fffffffLL || a.n_seqs * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (slots > 0 && a.T > 0) {
+    if (varlen) {
+      gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.n_seqs, coff);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    PrepArgs p;
+    p.g = a.g;
+    p.beta = a.beta;
+    p.cu_seqlens = a.cu_seqlens;
+    p.coff = coff;
+    p.w = w;
+    p.ut = ut;
+    p.T = a.T;
+    p.n_seqs = a.n_seqs;
+    p.H = a.H;
+    err = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepCfg::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    gdn_prep_kernel<<<(unsigned)(slots * a.H), 128, PrepCfg::SMEM_BYTES, stream>>>(mk, mv, p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  // 2. the sequential pass, one CTA per (sequence, head)
+  GdnTcArgs t;
+  t.out = a.out;
+  t.o_sb = a.o_sb;
+  t.o_st = a.o_st;
+  t.o_sh = a.o_sh;
+  t.g = a.g;
+  t.init = a.init;
+  t.final_state = a.final_state;
+  t.cu_seqlens = a.cu_seqlens;
+  t.T = a.T;
+  t.H = a.H;
+  using G = GdnCfg<kStages>;
+  auto kern = gdn_tc_kernel<kStages>;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  kern<<<(unsigned)(a.n_seqs * a.H), kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mw, mu, t);
+  return cudaGetLastError();
+}
+
+cudaError_t gdn_device_error(unsigned int *flags, unsigned int *where, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_gdn_error, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(where, g_gdn_where, sizeof(unsigned int));
+  if (e == cudaSuccess && reset) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_gdn_error, &zero, sizeof(zero));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gdn_where, &zero, sizeof(zero));
+  }
+  return e;
+}
+
+}  // namespace la

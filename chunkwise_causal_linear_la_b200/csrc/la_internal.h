@@ -2,6 +2,7 @@
 // and the kernel files.  Not installed; not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -104,5 +105,18 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t workspac
                             cudaStream_t stream, const char **why);
 // Device error words of the tensor-core kernel (timeouts of bounded waits).
 cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset);
+
+// [B, T, H, D] bf16 view as a 4-D TMA map with dims (D, H, T, B) and a
+// (64, 1, C, 1) box, 128-byte swizzle: one box is a [C rows x 64 cols] slab.
+bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t H, int64_t D, int C);
+
+// Chunked gated delta rule on the tensor cores (bf16, d_k = d_v = 128): a
+// per-chunk WY pass into the workspace, then one sequential pass per
+// (sequence, head).
+bool gdn_tc_supported(const DeltaArgs &a);
+size_t gdn_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen);
+cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                             const char **why);
+cudaError_t gdn_device_error(unsigned int *flags, unsigned int *where, bool reset);
 
 }  // namespace la

@@ -53,8 +53,42 @@
 #include "la_common.cuh"
 #include "la_internal.h"
 #include "la_sm100.cuh"
+#include "la_tc_sync.cuh"
 
 namespace la {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, T, H, D] bf16 view as a 4-D TMA map with dims (D, H, T, B) and a
+// (64, 1, C, 1) box, 128-byte swizzle: one box is a [C rows x 64 cols] slab.
+bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t H, int64_t D, int C) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sh * 2, (cuuint64_t)t.st * 2, (cuuint64_t)t.sb * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (B == 1) strides[2] = (cuuint64_t)T * t.st * 2 > 0 ? ((cuuint64_t)T * t.st * 2 + 15) / 16 * 16 : 16;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(t.data), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 __device__ unsigned int g_tc_error = 0;
 // First wait that gave up: 0x80000000 | chunk << 8 | barrier index.
@@ -63,10 +97,9 @@ __device__ unsigned int g_tc_where = 0;
 namespace {
 
 using namespace sm100;
+using namespace tcsync;
 
 constexpr int kThreads = 384;
-constexpr long long kTimeoutCycles = 4000000000LL;  // about two seconds
-constexpr uint32_t kSuspendHintNs = 20000;
 constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64: below, value-decay mode
 
 struct TcArgs {
@@ -151,47 +184,6 @@ struct Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-struct Sync {
-  uint64_t *bar;
-  volatile int *abort;
-};
-
-// Waiting threads sleep in the barrier (suspend hint) instead of polling, so
-// they leave issue slots to the warps that share their SM sub-partition.
-__device__ __forceinline__ bool wait_bar(const Sync &sy, int idx, uint32_t parity, int chunk = 0) {
-  uint64_t *b = sy.bar + idx;
-  if (mbar_test(b, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_wait_hint(b, parity, kSuspendHintNs)) return true;
-    if (*sy.abort) return false;
-    if (clock64() - t0 > kTimeoutCycles) {
-      *sy.abort = 1;
-      atomicOr(&g_tc_error, 1u);
-      atomicCAS(&g_tc_where, 0u, 0x80000000u | ((uint32_t)(chunk & 0x7FFFFF) << 8) | (uint32_t)idx);
-      return false;
-    }
-  }
-}
-
-// Warp-uniform wait for warps that go on to execute warp-collective or
-// .sync.aligned instructions: every lane takes the same path even on abort.
-__device__ __forceinline__ bool wait_bar_warp(const Sync &sy, int idx, uint32_t parity, int chunk = 0) {
-  return __all_sync(0xffffffffu, wait_bar(sy, idx, parity, chunk));
-}
-
-// Wait that ignores the abort flag (used to drain asynchronous arrivals).
-__device__ __forceinline__ void drain_bar(const Sync &sy, int idx, uint32_t parity) {
-  uint64_t *b = sy.bar + idx;
-  const long long t0 = clock64();
-  while (!mbar_test(b, parity)) {
-    if (clock64() - t0 > kTimeoutCycles) {
-      atomicOr(&g_tc_error, 2u);
-      return;
-    }
-  }
-}
-
 // phi for the bf16 tensor-core operands: elu(x) + 1, with e^x = 2^(x log2 e)
 // on the PTX ex2.approx.ftz instruction (one multiply and one special-function
 // op; relative error ~2^-22, far below the bf16 rounding (2^-9) the operand
@@ -211,32 +203,6 @@ __device__ __forceinline__ float swish_fast(float x) {
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
   return x * fmaf(0.5f, t, 0.5f);
-}
-
-// e^x on the same instruction, for the data-dependent decay factors (x <= 0).
-__device__ __forceinline__ float exp_fast(float x) {
-  constexpr float kLog2e = 1.4426950408889634f;
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * kLog2e));
-  return e;
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&p);
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-  return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
 // Transform of one [C x 64k] tile by the 64 transform threads (bf16 in and out):
@@ -314,7 +280,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + G::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + G::OFF_MISC + 4);
-  const Sync sy{bars, abort_flag};
+  const Sync sy{bars, abort_flag, &g_tc_error, &g_tc_where};
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -1046,38 +1012,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// [B, T, H, D] bf16 view as a 4-D TMA map with dims (D, H, T, B) and a
-// (64, 1, C, 1) box, 128-byte swizzle: one box is a [C rows x 64 cols] slab.
-bool make_map(CUtensorMap *m, const TensorView &t, int64_t B, int64_t T, int64_t H, int64_t D, int C) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)t.sh * 2, (cuuint64_t)t.st * 2, (cuuint64_t)t.sb * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  if (B == 1) strides[2] = (cuuint64_t)T * t.st * 2 > 0 ? ((cuuint64_t)T * t.st * 2 + 15) / 16 * 16 : 16;
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(t.data), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
 
 // Segmentation plan for the tensor-core path: when a dense batch has too few
 // (sequence, head, value-slice) units to fill the GPU, every sequence is split

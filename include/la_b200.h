@@ -201,6 +201,44 @@ LA_API la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, cons
                                     void *stream);
 
 /*
+ * la_fwd_gated_delta_chunk -- the same rule as la_fwd_gated_delta (same
+ * arguments and results), computed in chunks of 64 tokens.  Inside a chunk
+ * the writes u_i = beta_i (v_i - alpha_i S_{i-1} kt_i) solve a unit
+ * lower-triangular system (the UT / WY form of the delta rule; the pages give
+ * the recurrence, the chunk form is its exact regrouping), so
+ *     U = T diag(beta) V - T diag(beta e^b) Kt S_0^T,   T = (I + A)^{-1},
+ *     A_ij = beta_i e^{b_i - b_j} kt_i . kt_j  (j < i),  b_i = sum of g over the chunk up to i,
+ * and outputs and the next chunk's state follow from U with matrix products.
+ * Tensor cores (tcgen05) for bf16 with d_k = d_v = 128 and 16-byte aligned
+ * initial_state / final_state: a parallel pass over all chunks writes
+ * W = T diag(beta e^b) Kt and T diag(beta) V (bf16) to the workspace, then one
+ * CTA per (sequence, head) walks its chunks with the fp32 state.  Every other
+ * case, and flags = LA_FLAG_SIMT, runs la_fwd_gated_delta's kernel (no
+ * workspace needed).
+ *   flags       LA_FLAG_NONE or LA_FLAG_SIMT.
+ *   workspace   device memory of la_fwd_gated_delta_workspace_size bytes,
+ *               256-byte aligned, owned by the caller; its contents are
+ *               scratch (nothing needs to be zero; nothing is kept).
+ * Errors as for la_fwd_chunk (LA_ERR_WORKSPACE when the workspace is short).
+ */
+LA_API la_status la_fwd_gated_delta_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                          const float *g, const float *beta, const int32_t *cu_seqlens,
+                                          int64_t n_seqs, const float *initial_state, const la_tensor *out,
+                                          float *final_state, int32_t flags, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace la_fwd_gated_delta_chunk needs: B, T, H, d_k, d_v,
+ * n_seqs, has_cu_seqlens, dtype and flags as they will be passed.  0 when the
+ * call needs none (the token-by-token kernel); (size_t)-1 for arguments the
+ * call would reject.  Host-only.  On the tensor cores: 2 B T H 128 bf16 values
+ * (W and T diag(beta) V) plus, for a packed batch, n_seqs + 1 chunk offsets.
+ */
+LA_API size_t la_fwd_gated_delta_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                                int64_t n_seqs, int32_t has_cu_seqlens, int32_t dtype,
+                                                int32_t flags);
+
+/*
  * la_norm_gate -- the output norm and gate of a retention layer, on its own:
  *     y[r] = o[r] / sqrt(mean_r' o[r']^2 + eps) * w[r] * gate[r] * sigmoid(gate[r])
  * per (token, head) over the d_v values ("使用 FlashAttention 内核实现最先进的线性注意力":

@@ -95,3 +95,111 @@ def test_gated_delta_decode_in_place(la, oracle_mod):
     for j, o in enumerate(outs):
         assert slice_rel_err(to_np(o), ref[:, T + j:T + j + 1], seq_slices(B, 1)) < 1e-4
     assert state_rel_err(to_np(state), fref) < 1e-4
+
+
+# ---------------------------------------------------------------- chunked (tensor-core) path
+def _check_chunk(la, oracle_mod, q, k, v, g, beta, cu=None, init=None, flags=0, garbage=False):
+    """la_fwd_gated_delta_chunk against the token-by-token oracle.  garbage: the
+    workspace starts filled with NaN bit patterns (nothing may read unwritten rows)."""
+    dev = torch.device("cuda")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n = B if cu is None else cu.numel() - 1
+    ws = None
+    need = la.gated_delta_workspace_size(B, T, H, dk, dv, n, cu is not None, q.dtype, flags)
+    if need:
+        ws = torch.full((need,), 0xFF if garbage else 0, dtype=torch.uint8, device=dev)
+    out, fs = la.la_fwd_gated_delta_chunk(q.to(dev), k.to(dev), v.to(dev), g.to(dev), beta.to(dev),
+                                          cu_seqlens=None if cu is None else cu.to(dev),
+                                          initial_state=None if init is None else init.to(dev), flags=flags,
+                                          workspace=ws)
+    torch.cuda.synchronize()
+    assert la.device_error(reset=True) == (0, 0)
+    ref, fref = oracle_mod.gated_delta(q, k, v, g.double().numpy(), beta.double().numpy(),
+                                       cu_seqlens=None if cu is None else cu.numpy(),
+                                       init=None if init is None else init.double().numpy())
+    tol = TOL[q.dtype]
+    e1 = slice_rel_err(to_np(out), ref, seq_slices(B, T, None if cu is None else cu.tolist()))
+    e2 = state_rel_err(to_np(fs), fref)
+    assert e1 < tol and e2 < tol, (e1, e2)
+    return out, fs
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
+@pytest.mark.parametrize("alo,blo", [(0.05, 0.01), (0.9, 0.5), (0.999, 0.99)])
+def test_gated_delta_chunk_lengths_and_gates(la, oracle_mod, T, alo, blo):
+    """Tensor-core path (bf16, d = 128): partial last chunks, strong and mild decay,
+    weak and full-strength writes."""
+    q, k, v, g, beta = _inputs(2, T, 3, 128, 128, torch.bfloat16, 1000 + T, alo, blo)
+    _check_chunk(la, oracle_mod, q, k, v, g, beta)
+
+
+def test_gated_delta_chunk_many_heads(la, oracle_mod):
+    """More (sequence, head) units than SMs in the sequential pass, and thousands of
+    chunk CTAs in the WY pass; only a few slices are compared in full."""
+    q, k, v, g, beta = _inputs(4, 700, 40, 128, 128, torch.bfloat16, 77)
+    dev = torch.device("cuda")
+    out, fs = la.la_fwd_gated_delta_chunk(q.to(dev), k.to(dev), v.to(dev), g.to(dev), beta.to(dev))
+    torch.cuda.synchronize()
+    pick = [(0, 0), (1, 17), (3, 39)]
+    for b, h in pick:
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        ref, fref = oracle_mod.gated_delta(q[sl], k[sl], v[sl], g[sl].double().numpy(), beta[sl].double().numpy())
+        assert slice_rel_err(to_np(out[sl]), ref, seq_slices(1, 700)) < TOL[torch.bfloat16]
+        assert state_rel_err(to_np(fs[b:b + 1, h:h + 1]), fref) < TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("garbage", [False, True])
+def test_gated_delta_chunk_varlen_and_initial_state(la, oracle_mod, garbage):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300, 7])
+    q, k, v, g, beta = _inputs(1, int(cu[-1]) + 5, 2, 128, 128, torch.bfloat16, 6)  # 5 rows after the last sequence
+    _check_chunk(la, oracle_mod, q, k, v, g, beta, cu=cu, garbage=garbage)
+    init = torch.randn((7, 2, 128, 128)) * 0.1
+    _, fs = _check_chunk(la, oracle_mod, q, k, v, g, beta, cu=cu, init=init, garbage=garbage)
+    assert torch.equal(fs[1].cpu(), init[1])  # an empty sequence hands its initial state through
+
+
+def test_gated_delta_chunk_prefill_then_decode(la, oracle_mod):
+    """Chunked prefill, then token steps on the state in place (la_fwd_gated_delta),
+    equals the oracle over all tokens."""
+    B, T, H, d = 2, 333, 2, 128
+    q, k, v, g, beta = _inputs(B, T + 2, H, d, d, torch.bfloat16, 13)
+    dev = torch.device("cuda")
+    qd, kd, vd, gd, bd = (x.to(dev) for x in (q, k, v, g, beta))
+    _, state = la.la_fwd_gated_delta_chunk(qd[:, :T].contiguous(), kd[:, :T].contiguous(), vd[:, :T].contiguous(),
+                                           gd[:, :T].contiguous(), bd[:, :T].contiguous())
+    outs = []
+    for t in range(T, T + 2):
+        o, _ = la.la_fwd_gated_delta(qd[:, t:t + 1].contiguous(), kd[:, t:t + 1].contiguous(),
+                                     vd[:, t:t + 1].contiguous(), gd[:, t:t + 1].contiguous(),
+                                     bd[:, t:t + 1].contiguous(), initial_state=state, final_state=state)
+        outs.append(o)
+    torch.cuda.synchronize()
+    ref, fref = oracle_mod.gated_delta(q, k, v, g.double().numpy(), beta.double().numpy())
+    for j, o in enumerate(outs):
+        assert slice_rel_err(to_np(o), ref[:, T + j:T + j + 1], seq_slices(B, 1)) < TOL[torch.bfloat16]
+    assert state_rel_err(to_np(state), fref) < TOL[torch.bfloat16]
+
+
+def test_gated_delta_chunk_state_in_place_and_fallbacks(la, oracle_mod):
+    """initial_state and final_state one buffer (chunked continuation); f32 and
+    LA_FLAG_SIMT take the token-by-token kernel through the same entry point."""
+    q, k, v, g, beta = _inputs(2, 260, 2, 128, 128, torch.bfloat16, 21)
+    dev = torch.device("cuda")
+    qd, kd, vd, gd, bd = (x.to(dev) for x in (q, k, v, g, beta))
+    _, st = la.la_fwd_gated_delta_chunk(qd[:, :100].contiguous(), kd[:, :100].contiguous(),
+                                        vd[:, :100].contiguous(), gd[:, :100].contiguous(), bd[:, :100].contiguous())
+    o2, _ = la.la_fwd_gated_delta_chunk(qd[:, 100:].contiguous(), kd[:, 100:].contiguous(), vd[:, 100:].contiguous(),
+                                        gd[:, 100:].contiguous(), bd[:, 100:].contiguous(), initial_state=st,
+                                        final_state=st)
+    torch.cuda.synchronize()
+    ref, fref = oracle_mod.gated_delta(q, k, v, g.double().numpy(), beta.double().numpy())
+    assert slice_rel_err(to_np(o2), ref[:, 100:], seq_slices(2, 160)) < TOL[torch.bfloat16]
+    assert state_rel_err(to_np(st), fref) < TOL[torch.bfloat16]
+    assert la.gated_delta_workspace_size(2, 260, 2, 128, 128, 2, False, torch.float32) == 0
+    _check_chunk(la, oracle_mod, q.float(), k.float(), v.float(), g, beta)
+    _check_chunk(la, oracle_mod, q, k, v, g, beta, flags=1)
+    q2, k2, v2, g2, b2 = _inputs(1, 90, 2, 64, 64, torch.bfloat16, 22)
+    _check_chunk(la, oracle_mod, q2, k2, v2, g2, b2)

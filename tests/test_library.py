@@ -68,6 +68,25 @@ def test_workspace_size_host_logic(lib):
     assert ws(8, 128, 16, 128, 128, 8, 0, 64, 1, 1) == 0  # forced SIMT
 
 
+def test_gated_delta_workspace_size(lib):
+    """The chunked gated delta rule keeps W and T diag(beta) V, bf16 [B, T, H, 128] each,
+    plus n_seqs + 1 chunk offsets for a packed batch (each region 256-byte aligned);
+    shapes that take the token-by-token kernel need nothing."""
+    ws = lib.la_fwd_gated_delta_workspace_size
+    bad = ctypes.c_size_t(-1).value
+    wu = 8 * 4096 * 16 * 128 * 2
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 0) == 2 * wu
+    assert ws(1, 1000, 3, 128, 128, 5, 1, 1, 0) == 2 * (1000 * 3 * 256 + 0) + 256  # 768000 B each, aligned
+    assert ws(1, 3, 1, 128, 128, 100, 1, 1, 0) == 2 * 768 + 512
+    assert ws(8, 4096, 16, 64, 64, 8, 0, 1, 0) == 0      # d = 64: token-by-token kernel
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 0, 0) == 0    # f32
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 1) == 0    # LA_FLAG_SIMT
+    assert ws(8, 4096, 16, 96, 128, 8, 0, 1, 0) == bad   # head dim
+    assert ws(8, 4096, 0, 128, 128, 8, 0, 1, 0) == bad   # H = 0
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 2, 0) == bad  # dtype
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 4) == bad  # flags
+
+
 def test_workspace_size_segment_plan(lib):
     """Segment states (S^T, the normaliser sum and the log decay of a
     data-dependent decay) are kept for all but the last segment of each unit,
