@@ -16,11 +16,12 @@
 //     S' = e^{b_last} S_0 + (diag(e^{b_last - b}) Kt)^T U.
 // Ut and W depend on the chunk's own inputs only; U, O and S' need the state.
 // Two kernels:
-//   gdn_prep_kernel  one CTA per (sequence, chunk, head), all independent: unit
-//                    keys; G = Kt Kt^T on the tensor cores; A from G; T by
-//                    forward substitution on the CUDA cores (fp32); then
-//                    [W | Ut] = T [diag(beta e^b) Kt | diag(beta) V] on the
-//                    tensor cores, stored as bf16 [B, T, H, 128] in the workspace.
+//   gdn_prep_kernel  one CTA per (sequence, chunk, head), all independent: G =
+//                    K K^T on the tensor cores; A from G and the key norms; T
+//                    by forward substitution on the CUDA cores (fp32); then
+//                    W = T diag(beta e^b) Kt and Ut = T diag(beta) V on the
+//                    tensor cores.  W, Ut and the unit keys Kt go to the
+//                    workspace as bf16 [B, T, H, 128], with the chunk's b_i.
 //   gdn_tc_kernel    one CTA per (sequence, head) walks its chunks in order with
 //                    the fp32 state S^T in registers, as the linear-attention
 //                    forward does.  Per chunk, five products:
@@ -31,10 +32,9 @@
 //                      M3  O += P U                  (M=C, N=d_v, K=C)     P = tril(A) .* D
 //                    with U = Ut - WS between MW and M4 and S^T <- e^{b_last} S^T + Us after M4.
 //   Warp roles of gdn_tc_kernel (384 threads, as in the forward):
-//     warp 0      TMA producer: Q, K, W, Ut chunk tiles into a two-deep ring.
+//     warp 0      TMA producer: Q, Kt, W, Ut chunk tiles and b_i into a two-deep ring.
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//     warps 2-3   transform: unit keys Kt in place, decayed unit keys Kd, and
-//                 the chunk's table of b_i.
+//     warps 2-3   transform: the decayed unit keys Kd.
 //     warps 4-7   state: S^T update, the bf16 operand Sb, and U = Ut - WS in place.
 //     warps 8-11  output: score tile -> P, Qd in place, epilogue.
 // Every wait is bounded: on a timeout the CTA raises an abort flag, records the
@@ -91,27 +91,26 @@ struct PrepArgs {
   const float *g, *beta;      // [B * T][H]
   const int32_t *cu_seqlens;  // NULL: dense
   const int32_t *coff;        // packed: first chunk slot of each sequence, [n_seqs + 1]
-  __nv_bfloat16 *w, *ut;      // [B, T, H, 128] each
+  __nv_bfloat16 *w, *ut, *kt;  // [B, T, H, 128] each: W, T diag(beta) V, unit keys
+  float *bt;                    // [chunk slot][H][C]: b_i of every chunk (rows past its end repeat b_last)
   int64_t T, n_seqs;
   int H;
 };
 
 struct PrepCfg {
-  static constexpr int OFF_K = 0;              // K, then unit keys, then diag(beta e^b) Kt
-  static constexpr int OFF_V = OFF_K + kTile;  // V, then diag(beta) V: [K | V] is one 4-slab operand
-  static constexpr int OFF_T = OFF_V + kTile;  // T = (I + A)^{-1}, bf16 [C x C] K-major
-  static constexpr int OFF_A = OFF_T + kSlab;  // A, fp32 [C][A_LD]
-  static constexpr int A_LD = kC + 4;          // rows 16-byte aligned for float4 reads
-  static constexpr int OFF_VEC = OFF_A + kC * A_LD * 4;  // b_i and beta_i, 2 x C floats
-  static constexpr int OFF_BAR = OFF_VEC + 2 * kC * 4;   // 0: tiles landed, 1: MMA done
+  static constexpr int OFF_K = 0;              // K, then diag(beta e^b / |k|) K
+  static constexpr int OFF_V = OFF_K + kTile;  // V, then diag(beta) V
+  static constexpr int OFF_A = OFF_V + kTile;  // A, fp32 [C][A_LD]; afterwards T^T, bf16 [C x C]
+  static constexpr int A_LD = kC + 4;          // rows 16-byte aligned for float4 access
+  static constexpr int OFF_VEC = OFF_A + kC * A_LD * 4;  // b_i, beta_i, 1/max(|k_i|, 1e-12): 3 x C floats
+  static constexpr int OFF_BAR = OFF_VEC + 3 * kC * 4;   // 0: tiles landed, 1: products done
   static constexpr int OFF_MISC = OFF_BAR + 2 * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
-  // More than a third of an SM's shared memory: at most two CTAs share an SM,
-  // so their two 256-column tensor-memory allocations always fit.
-  static constexpr int SMEM_BYTES = 80 * 1024;
-  static constexpr int T_COLS = 256;
-  static_assert(SMEM_USED + 1024 <= SMEM_BYTES, "prep shared memory");
-  static_assert(3 * SMEM_BYTES > 232448, "at most two prep CTAs per SM");
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+  static constexpr int T_COLS = 128;                   // four CTAs per SM fill the tensor memory
+  static_assert(4 * (SMEM_BYTES + 1024) <= 233472, "four prep CTAs per SM");
+  static_assert(5 * (SMEM_BYTES + 1024) > 233472, "at most four prep CTAs per SM (tensor memory)");
+  static_assert(OFF_A % 1024 == 0, "T^T tile alignment");
 };
 
 // Sequence start slots of a packed batch: coff[n] = sum_{m<n} ceil(len_m / C).
@@ -154,15 +153,46 @@ __global__ void __launch_bounds__(1024) gdn_chunk_offsets_kernel(const int32_t *
   }
 }
 
-__global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                                       const __grid_constant__ CUtensorMap tm_v,
-                                                       const PrepArgs a) {
+// Columns j of T = (I + A)^{-1} by forward substitution in fp32:
+// x_i = [i == j] - sum_{m<i} A_im x_m.  Every lane of a warp walks the same rows,
+// so each read of A is a broadcast; the sums use paired fp32 FMAs.  W0: the
+// warp's first column; rows and columns below it are zero for all its lanes.
+template <int W0>
+__device__ __forceinline__ void solve_column(const float *As, int j, float2 (&x2)[kC / 2]) {
+#pragma unroll
+  for (int q = 0; q < kC / 2; ++q) x2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = W0; i < kC; ++i) {
+    const float4 *a4 = reinterpret_cast<const float4 *>(As + i * PrepCfg::A_LD);
+    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int m = W0; m < i; m += 4) {  // A_im = 0 for m >= i, and x_m is still 0 there
+      const float4 av = a4[m >> 2];
+      s0 = __ffma2_rn(make_float2(av.x, av.y), x2[m >> 1], s0);
+      s1 = __ffma2_rn(make_float2(av.z, av.w), x2[(m >> 1) + 1], s1);
+    }
+    const float xi = i < j ? 0.f : (i == j ? 1.f : -((s0.x + s0.y) + (s1.x + s1.y)));
+    if (i & 1)
+      x2[i >> 1].y = xi;
+    else
+      x2[i >> 1].x = xi;
+  }
+}
+
+// One CTA per (sequence, chunk, head), four per SM.  Thread tt owns the
+// 16-byte vectors tt + 128 m (m < 8) of a [C x 128] tile: rows tt/8 + 16 m'
+// (m' < 4) in both 64-column slabs, physical chunk tt mod 8; the 8 lanes of a
+// row differ in their low three bits.
+__global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                          const __grid_constant__ CUtensorMap tm_v,
+                                                          const PrepArgs a) {
   using P = PrepCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = align1024(smem_raw);
   float *As = reinterpret_cast<float *>(sm + P::OFF_A);
   float *bvec = reinterpret_cast<float *>(sm + P::OFF_VEC);
   float *betav = bvec + kC;
+  float *invn = betav + kC;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P::OFF_MISC + 4);
@@ -175,10 +205,13 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
   int64_t n, c;
   if (a.coff) {
     if (slot >= a.coff[a.n_seqs]) return;  // past the last chunk (the grid is an upper bound)
-    int64_t lo = 0, hi = a.n_seqs - 1;     // last n with coff[n] <= slot
+    int64_t lo = 0, hi = a.n_seqs - 1;     // last n with coff[n] <= slot: never an empty sequence
     while (lo < hi) {
       const int64_t mid = (lo + hi + 1) >> 1;
-      if (a.coff[mid] <= slot) lo = mid; else hi = mid - 1;
+      if (a.coff[mid] <= slot)
+        lo = mid;
+      else
+        hi = mid - 1;
     }
     n = lo;
     c = slot - a.coff[n];
@@ -203,7 +236,12 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
       tma_load_4d(sm + P::OFF_V + kb * kSlab, &tm_v, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
     }
   }
-  if (warp == 1) tmem_alloc(tmem_slot, P::T_COLS);
+  // Give up the allocation permit at once: an SM takes no further CTA while one
+  // of its CTAs still holds the permit (measured), and four CTAs fill the tensor memory.
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, P::T_COLS);
+    tmem_relinquish();
+  }
   if (warp == 0) {  // b_i = sum_{t<=i} g_t over the chunk (rows past its end add 0 and get beta = 0)
     const int64_t row0 = (sp.bidx * a.T + t0) * a.H + h;
     float blo = lane < Cp ? a.g[row0 + (int64_t)lane * a.H] : 0.f;
@@ -220,6 +258,9 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
     bhi += __shfl_sync(0xffffffffu, blo, 31);
     bvec[lane] = blo;
     bvec[lane + 32] = bhi;
+    float *btab = a.bt + (slot * a.H + h) * kC;
+    btab[lane] = blo;
+    btab[lane + 32] = bhi;
     betav[lane] = lane < Cp ? a.beta[row0 + (int64_t)lane * a.H] : 0.f;
     betav[lane + 32] = lane + 32 < Cp ? a.beta[row0 + (int64_t)(lane + 32) * a.H] : 0.f;
   }
@@ -230,35 +271,8 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
   bool ok = wait_bar_warp(sy, 0, 0);
   int issued = 0;  // products committed on barrier 1 (thread 0)
 
-  // ---- unit keys in place; rows past the chunk end become zero (keys and values)
-  const int ri = tid >> 1, hh = tid & 1;  // row and 64-column half handled by this thread
-  uint8_t *krow = sm + P::OFF_K + hh * kSlab + ri * 128;
-  uint8_t *vrow = sm + P::OFF_V + hh * kSlab + ri * 128;
-  if (ok) {
-    uint4 x[8];
-    float ss = 0.f;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      x[p] = *reinterpret_cast<const uint4 *>(krow + p * 16);
-      float f[8];
-      unpack8(x[p], f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) ss = fmaf(f[u], f[u], ss);
-    }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    const float inv = ri < Cp ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      float f[8];
-      unpack8(x[p], f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] *= inv;
-      *reinterpret_cast<uint4 *>(krow + p * 16) = pack8(f);
-    }
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  // G = Kt Kt^T (M = N = C, K = 128) into columns [0, C)
+  // G = K K^T from the raw keys (M = N = C, K = 128) into columns [0, C); the
+  // norms are applied to G afterwards
   if (ok && tid == 0) {
     tc_fence_after();
     const uint64_t dk = smem_desc_sw128(smem_u32(sm + P::OFF_K), 16, 1024);
@@ -268,111 +282,143 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
     umma_commit(bars + 1);
     issued = 1;
   }
-  // diag(beta) V in place, while the product runs (it does not read V)
+  // while it runs: 1/|k_i| and diag(beta) V in place (rows past the chunk end: zero)
   if (ok) {
-    const float bt = betav[ri];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      uint4 x = *reinterpret_cast<const uint4 *>(vrow + p * 16);
-      float f[8];
-      unpack8(x, f);
+    for (int m = 0; m < 4; ++m) {
+      const int r = (tid >> 3) + 16 * m;
+      const int off = (tid + 128 * m) * 16;
+      float f0[8], f1[8];
+      unpack8(*reinterpret_cast<const uint4 *>(sm + P::OFF_K + off), f0);
+      unpack8(*reinterpret_cast<const uint4 *>(sm + P::OFF_K + kSlab + off), f1);
+      float ss = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] = ri < Cp ? f[u] * bt : 0.f;
-      *reinterpret_cast<uint4 *>(vrow + p * 16) = pack8(f);
+      for (int u = 0; u < 8; ++u) ss = fmaf(f0[u], f0[u], fmaf(f1[u], f1[u], ss));
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+      if ((tid & 7) == 0) invn[r] = r < Cp ? inv : 0.f;
+      if (r < Cp) {  // unit keys, bf16: physical chunk tid & 7 of row r holds logical columns 8 ((tid & 7) ^ (r & 7))
+        __nv_bfloat16 *kd = a.kt + ((sp.bidx * a.T + t0 + r) * a.H + h) * (int64_t)kD + 8 * ((tid & 7) ^ (r & 7));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          f0[u] *= inv;
+          f1[u] *= inv;
+        }
+        *reinterpret_cast<uint4 *>(kd) = pack8(f0);
+        *reinterpret_cast<uint4 *>(kd + 64) = pack8(f1);
+      }
+      const float bt = betav[r];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        uint4 *p4 = reinterpret_cast<uint4 *>(sm + P::OFF_V + sl * kSlab + off);
+        float f[8];
+        unpack8(*p4, f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] = r < Cp ? f[u] * bt : 0.f;
+        *p4 = pack8(f);
+      }
     }
   }
+  __syncthreads();  // 1/|k| of every row
   ok = ok && wait_bar_warp(sy, 1, 0);
   tc_fence_after();
   if (ok) {
-    // A_ij = beta_i e^{b_i - b_j} G_ij for j < i: this thread's row i and 32 columns
+    // A_ij = beta_i e^{b_i - b_j} kt_i . kt_j for j < i < C': row i, 32 columns
     const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;
     uint32_t r[32];
     tmem_ld_16x32bx2_x32<32>(tbase + ((uint32_t)(warp * 32) << 16), r);
     tmem_wait_ld();
-    const float bi = bvec[i], bt = betav[i];
-    float *arow = As + i * P::A_LD + hf * 32;
+    const float bi = bvec[i], wi = i < Cp ? betav[i] * invn[i] : 0.f;
+    float4 *arow = reinterpret_cast<float4 *>(As + i * P::A_LD + hf * 32);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = hf * 32 + e;
-      arow[e] = j < i ? bt * expf(bi - bvec[j]) * __uint_as_float(r[e]) : 0.f;
+    for (int q = 0; q < 8; ++q) {
+      float e4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = hf * 32 + 4 * q + u;
+        e4[u] = (j < i && i < Cp) ? wi * invn[j] * exp_fast(bi - bvec[j]) * __uint_as_float(r[4 * q + u]) : 0.f;
+      }
+      arow[q] = make_float4(e4[0], e4[1], e4[2], e4[3]);
     }
-    // diag(beta e^b) Kt in place (the product above has read Kt)
-    const float wk = betav[ri] * expf(bvec[ri]);
+    // diag(beta e^b / |k|) K in place (the product has read K)
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      uint4 x = *reinterpret_cast<const uint4 *>(krow + p * 16);
-      float f[8];
-      unpack8(x, f);
+    for (int m = 0; m < 4; ++m) {
+      const int rr = (tid >> 3) + 16 * m;
+      const float wk = betav[rr] * exp_fast(bvec[rr]) * invn[rr];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] *= wk;
-      *reinterpret_cast<uint4 *>(krow + p * 16) = pack8(f);
+      for (int sl = 0; sl < 2; ++sl) {
+        uint4 *p4 = reinterpret_cast<uint4 *>(sm + P::OFF_K + sl * kSlab + (tid + 128 * m) * 16);
+        float f[8];
+        unpack8(*p4, f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] = rr < Cp ? f[u] * wk : 0.f;
+        *p4 = pack8(f);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  // ---- T = (I + A)^{-1} by forward substitution: thread j solves column j,
-  // x_i = [i == j] - sum_{m<i} A_im x_m (x_m = 0 for m < j), in fp32; all threads
-  // walk the same rows so every read of A is a broadcast.  The bf16 result goes
-  // to the K-major T tile (row i, column j).
+  // ---- T = (I + A)^{-1}: thread j < C solves column j (warp 1 starts at row and column 32)
+  float2 x2[kC / 2];
   if (ok && tid < kC) {
-    const int j = tid;
-    float x[kC];
+    if (warp == 0)
+      solve_column<0>(As, tid, x2);
+    else
+      solve_column<32>(As, tid, x2);
+  }
+  __syncthreads();  // every read of A is done: T^T (bf16, row j = column j of T) replaces it
+  if (ok && tid < kC) {
+    uint8_t *trow = sm + P::OFF_A + tid * 128;
 #pragma unroll
-    for (int i = 0; i < kC; ++i) x[i] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      const float4 *a4 = reinterpret_cast<const float4 *>(As + i * P::A_LD);
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-      for (int m = 0; m < i; m += 4) {  // A_im = 0 for m >= i and x_m = 0 beyond what is solved
-        const float4 av = a4[m >> 2];
-        s0 = fmaf(av.x, x[m], s0);
-        s1 = fmaf(av.y, x[m + 1], s1);
-        s2 = fmaf(av.z, x[m + 2], s2);
-        s3 = fmaf(av.w, x[m + 3], s3);
-      }
-      x[i] = i < j ? 0.f : (i == j ? 1.f : -((s0 + s1) + (s2 + s3)));
-    }
-    uint8_t *tt = sm + P::OFF_T;
-#pragma unroll
-    for (int i = 0; i < kC; ++i)
-      *reinterpret_cast<__nv_bfloat16 *>(tt + swz(i, j >> 3) + (j & 7) * 2) = __float2bfloat16_rn(x[i]);
+    for (int p = 0; p < 8; ++p)
+      *reinterpret_cast<uint4 *>(trow + ((p ^ (tid & 7)) << 4)) =
+          make_uint4(pack2(x2[4 * p].x, x2[4 * p].y), pack2(x2[4 * p + 1].x, x2[4 * p + 1].y),
+                     pack2(x2[4 * p + 2].x, x2[4 * p + 2].y), pack2(x2[4 * p + 3].x, x2[4 * p + 3].y));
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-  // [W | Ut] = T [diag(beta e^b) Kt | diag(beta) V]  (M = C, N = 256, K = C) into columns [0, 256)
-  if (ok && tid == 0) {
-    tc_fence_after();
-    const uint64_t dt = smem_desc_sw128(smem_u32(sm + P::OFF_T), 16, 1024);
-    const uint64_t dx = smem_desc_sw128(smem_u32(sm + P::OFF_K), kSlab, 1024);  // MN-major, 4 slabs
-    constexpr uint32_t ID_X = idesc_bf16_f32(kC, 256, 0, 1);
-#pragma unroll
-    for (int kk = 0; kk < kC / 16; ++kk) umma_bf16(tbase, dt + kmaj(kk), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
-    umma_commit(bars + 1);
-    issued = 2;
-  }
-  ok = ok && wait_bar_warp(sy, 1, 1);
-  tc_fence_after();
-  if (ok) {
-    // row i, columns [0, 128) (W) for lanes 0-15 and [128, 256) (Ut) for lanes 16-31
-    const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;
-    __nv_bfloat16 *dst = (hf ? a.ut : a.w) + ((sp.bidx * a.T + t0 + i) * a.H + h) * (int64_t)kD;
+
+  // ---- W = T diag(beta e^b) Kt, then Ut = T diag(beta) V (M = C, N = 128, K = C), each into
+  // columns [0, 128) and stored as bf16 rows of the workspace
+  const uint64_t dtt = smem_desc_sw128(smem_u32(sm + P::OFF_A), kSlab, 1024);  // T^T: A operand, MN-major
+  constexpr uint32_t ID_X = idesc_bf16_f32(kC, kD, 1, 1);
+  const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;  // row and 64-column half read back
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-      uint32_t r[32];
-      tmem_ld_16x32bx2_x32<128>(tbase + ((uint32_t)(warp * 32) << 16) + pass * 32, r);
-      tmem_wait_ld();
-      if (i < Cp) {
-        uint4 *d4 = reinterpret_cast<uint4 *>(dst + pass * 32);
+  for (int part = 0; part < 2; ++part) {
+    if (ok && tid == 0) {
+      tc_fence_after();
+      const uint64_t dx = smem_desc_sw128(smem_u32(sm + (part ? P::OFF_V : P::OFF_K)), kSlab, 1024);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d4[q] = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                             pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                             pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                             pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      for (int kk = 0; kk < kC / 16; ++kk)
+        umma_bf16(tbase, dtt + ((kk * 2048) >> 4), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
+      umma_commit(bars + 1);
+      issued = 2 + part;
+    }
+    ok = ok && wait_bar_warp(sy, 1, (part + 1) & 1);
+    tc_fence_after();
+    if (ok) {
+      __nv_bfloat16 *dst = (part ? a.ut : a.w) + ((sp.bidx * a.T + t0 + i) * a.H + h) * (int64_t)kD + hf * 64;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t r[32];
+        tmem_ld_16x32bx2_x32<64>(tbase + ((uint32_t)(warp * 32) << 16) + pass * 32, r);
+        tmem_wait_ld();
+        if (i < Cp) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + pass * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            d4[q] = make_uint4(pack2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                               pack2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                               pack2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                               pack2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+        }
       }
     }
+    tc_fence_before();
+    __syncthreads();  // the columns are read before the next product overwrites them
   }
   // ---- teardown (after an abort, let the tile loads and products finish first)
   if (*abort_flag && tid == 0) {
@@ -382,10 +428,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const __grid_constant__ C
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
-    tmem_dealloc(tbase, P::T_COLS);
-    tmem_relinquish();
-  }
+  if (warp == 1) tmem_dealloc(tbase, P::T_COLS);
 }
 
 // ============================================================== chunk kernel
@@ -394,7 +437,9 @@ constexpr int kThreads = 384;
 struct GdnTcArgs {
   void *out;
   int64_t o_sb, o_st, o_sh;
-  const float *g;             // [B * T][H] log decay
+  const float *bt;            // [chunk slot][H][C]: b_i of every chunk, from the WY pass
+  const int32_t *coff;        // packed: first chunk slot of each sequence (dense: n * nck)
+  int64_t nck;                // chunks per sequence (dense)
   const float *init;          // NULL or [n_seqs, H, 128, 128] (S^T)
   float *final_state;         // NULL or [n_seqs, H, 128, 128]
   const int32_t *cu_seqlens;  // NULL: dense
@@ -404,15 +449,15 @@ struct GdnTcArgs {
 
 template <int NS>
 struct GdnCfg {
-  // a stage: Q (then Qd), K (then Kt), W, Ut (then U), Kd; [C x 128] bf16 tiles
+  // a stage: Q (then Qd), Kt, W, Ut (then U), Kd; [C x 128] bf16 tiles
   static constexpr int OFF_Q = 0, OFF_K = kTile, OFF_W = 2 * kTile, OFF_U = 3 * kTile, OFF_KD = 4 * kTile;
   static constexpr int STAGE_BYTES = 5 * kTile;
-  static constexpr int LOAD_BYTES = 4 * kTile;  // Q, K, W, Ut arrive by TMA
+  static constexpr int LOAD_BYTES = 4 * kTile + kC * 4;  // Q, Kt, W, Ut and the b table arrive by TMA
   static constexpr int SB_SLAB = kD * 128;      // [d_k rows x 64 cols] bf16
   static constexpr int OFF_SB = NS * STAGE_BYTES;
   static constexpr int OFF_P = OFF_SB + 2 * SB_SLAB;
-  static constexpr int OFF_DT = OFF_P + 2 * kSlab;  // per stage: b_i (i < C), b_last at [C]
-  static constexpr int DT_STRIDE = kC + 4;
+  static constexpr int OFF_DT = OFF_P + 2 * kSlab;  // per stage: b_i (i < C); b_last = b_{C-1}
+  static constexpr int DT_STRIDE = kC;
   static constexpr int OFF_BAR = OFF_DT + NS * DT_STRIDE * 4;
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_QREADY = 3 * NS, B_AFULL = 4 * NS,
                        B_PFULL = 4 * NS + 2, B_OFULL = 4 * NS + 4, B_OEMPTY = 4 * NS + 6, B_WSFULL = 4 * NS + 8,
@@ -436,7 +481,7 @@ struct GdnCfg {
 //              [XFORM, prev: WSFULL] U = Ut - WS in place -> UREADY.
 //   output:    [AFULL[b], XFORM] P -> PFULL[b];  Qd in place -> QREADY[s];
 //              [OFULL[b-1]] epilogue of chunk c-1 -> OEMPTY.
-//   transform: [FULL] b table, Kt in place, Kd -> XFORM.
+//   transform: [FULL] Kd -> XFORM.
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -499,6 +544,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t0 = (int)(sq.start + (int64_t)c * kC);
         const int bi = (int)sq.bidx;
         uint8_t *st = stage(s);
+        const int64_t slot = (a.coff ? (int64_t)a.coff[n] : n * a.nck) + c;
+        bulk_load(dtab + s * G::DT_STRIDE, a.bt + (slot * a.H + h) * kC, kC * 4, bars + G::B_FULL + s);
         for (int kb = 0; kb < 2; ++kb) {
           tma_load_4d(st + G::OFF_Q + kb * kSlab, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bi);
           tma_load_4d(st + G::OFF_K + kb * kSlab, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bi);
@@ -587,67 +634,29 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // ========================================================== transform
       // 64 threads; thread tt owns the 16-byte vectors tt + 64 m (m < 8) of both
       // 64-column slabs of the key tile: row tt/8 + 8 m, physical chunk tt mod 8.
-      // The 8 lanes holding a row differ in their low three bits.
-      const int tt = tid - 64, ln = tt & 31;
+      // Kd = diag(e^{b_last - b}) Kt, zero past the chunk end.
+      const int tt = tid - 64;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
         if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c)) break;
         const int Cp = chunk_len(c);
-        // b_i over the chunk (rows past its end add 0): lane l holds b_l and b_{l+32}
-        const int64_t row0 = (sq.bidx * a.T + sq.start + (int64_t)c * kC) * a.H + h;
-        float blo = ln < Cp ? a.g[row0 + (int64_t)ln * a.H] : 0.f;
-        float bhi = ln + 32 < Cp ? a.g[row0 + (int64_t)(ln + 32) * a.H] : 0.f;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float y0 = __shfl_up_sync(0xffffffffu, blo, o);
-          const float y1 = __shfl_up_sync(0xffffffffu, bhi, o);
-          if (ln >= o) {
-            blo += y0;
-            bhi += y1;
-          }
-        }
-        bhi += __shfl_sync(0xffffffffu, blo, 31);
-        const float blast = __shfl_sync(0xffffffffu, Cp <= 32 ? blo : bhi, (Cp - 1) & 31);
-        if (tt < 32) {
-          float *dt = dtab + s * G::DT_STRIDE;
-          dt[ln] = blo;
-          dt[ln + 32] = bhi;
-          if (ln == 0) dt[kC] = blast;
-        }
-        uint8_t *kt = stage(s) + G::OFF_K;
+        const float *dt = dtab + s * G::DT_STRIDE;
+        const float blast = dt[kC - 1];
+        const uint8_t *kt = stage(s) + G::OFF_K;
         uint8_t *kd = stage(s) + G::OFF_KD;
-#pragma unroll 1
+#pragma unroll 2
         for (int m = 0; m < 8; ++m) {
           const int r = (tt >> 3) + 8 * m;
           const int off = (tt + 64 * m) * 16;
-          uint4 x0 = *reinterpret_cast<const uint4 *>(kt + off);
-          uint4 x1 = *reinterpret_cast<const uint4 *>(kt + kSlab + off);
-          float f0[8], f1[8];
-          unpack8(x0, f0);
-          unpack8(x1, f1);
-          float ss = 0.f;
+          const float wd = r < Cp ? exp_fast(blast - dt[r]) : 0.f;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) ss = fmaf(f0[u], f0[u], fmaf(f1[u], f1[u], ss));
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-          const float b0 = __shfl_sync(0xffffffffu, blo, r & 31);
-          const float b1 = __shfl_sync(0xffffffffu, bhi, r & 31);
-          const float br = r < 32 ? b0 : b1;
-          const float inv = r < Cp ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
-          const float wd = inv * exp_fast(blast - br);
-          float g0[8], g1[8];
+          for (int sl = 0; sl < 2; ++sl) {
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(kt + sl * kSlab + off), f);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            g0[u] = f0[u] * wd;
-            g1[u] = f1[u] * wd;
-            f0[u] *= inv;
-            f1[u] *= inv;
+            for (int u = 0; u < 8; ++u) f[u] = r < Cp ? f[u] * wd : 0.f;
+            *reinterpret_cast<uint4 *>(kd + sl * kSlab + off) = pack8(f);
           }
-          *reinterpret_cast<uint4 *>(kt + off) = pack8(f0);
-          *reinterpret_cast<uint4 *>(kt + kSlab + off) = pack8(f1);
-          *reinterpret_cast<uint4 *>(kd + off) = pack8(g0);
-          *reinterpret_cast<uint4 *>(kd + kSlab + off) = pack8(g1);
         }
         fence_proxy_async_smem();
         mbar_arrive(bars + G::B_XFORM + s);
@@ -715,7 +724,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         write_sb();
       }
       if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c) || !wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) break;
-      const float blast = dtab[s * G::DT_STRIDE + kC];
+      const float blast = dtab[s * G::DT_STRIDE + kC - 1];
       const int Cp = chunk_len(c);
       if (prev(c)) {
         if (!wait_bar_warp(sy, G::B_WSFULL, sbi(c) & 1, c)) break;
@@ -801,11 +810,12 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(bars + G::B_PFULL + b);  // also tells the MMA issuer that A[b] has been read
       // the score product has read Q: scale its row i by e^{b_i} for the inter-chunk product
+      // (chunks in swizzled order, so that the rows of a warp spread over the banks)
       const float qf = i < Cp ? exp_fast(bi) : 0.f;
-      uint8_t *qrow = stage(s) + G::OFF_Q + hf * kSlab + i * 128;
+      uint8_t *qrow = stage(s) + G::OFF_Q + hf * kSlab;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        uint4 *p4 = reinterpret_cast<uint4 *>(qrow + p * 16);
+        uint4 *p4 = reinterpret_cast<uint4 *>(qrow + swz(i, p));
         float x[8];
         unpack8(*p4, x);
 #pragma unroll
@@ -871,8 +881,24 @@ constexpr int kStages = 2;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// W and Ut, bf16 [B, T, H, 128] each, then (packed batches) the chunk offsets
-size_t wu_bytes(int64_t B, int64_t T, int64_t H) { return align256((size_t)(B * T * H) * kD * 2); }
+// Workspace regions, in order: W, Ut and the unit keys (bf16 [B, T, H, 128]
+// each), the b tables ([chunk slot][H][C] fp32) and, for packed batches, the
+// first chunk slot of each sequence.  Packed batches bound their slot count by
+// ceil(T / C) + n_seqs (each sequence adds at most one partial chunk).
+struct WsPlan {
+  size_t wu, bt, coff, total;
+  int64_t nck, slots;
+};
+WsPlan ws_plan(int64_t B, int64_t T, int64_t H, int64_t n_seqs, bool varlen) {
+  WsPlan p;
+  p.nck = (T + kC - 1) / kC;
+  p.slots = varlen ? p.nck + n_seqs : n_seqs * p.nck;
+  p.wu = align256((size_t)(B * T * H) * kD * 2);
+  p.bt = align256((size_t)(p.slots * H) * kC * 4);
+  p.coff = varlen ? align256((size_t)(n_seqs + 1) * 4) : 0;
+  p.total = 3 * p.wu + p.bt + p.coff;
+  return p;
+}
 
 }  // namespace
 
@@ -880,37 +906,38 @@ bool gdn_tc_supported(const DeltaArgs &a) { return a.dtype == LA_BF16 && a.dk ==
 
 size_t gdn_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen) {
   if (dk != kD || dv != kD) return 0;
-  return 2 * wu_bytes(B, T, H) + (varlen ? align256((size_t)(n_seqs + 1) * 4) : 0);
+  return ws_plan(B, T, H, n_seqs, varlen).total;
 }
 
 cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspace_bytes, cudaStream_t stream,
                              const char **why) {
   const int64_t B = a.cu_seqlens ? 1 : a.n_seqs;
   const bool varlen = a.cu_seqlens != nullptr;
-  const size_t need = gdn_workspace_bytes(B, a.T, a.H, a.dk, a.dv, a.n_seqs, varlen);
-  if (!workspace || workspace_bytes < need) {
+  const WsPlan plan = ws_plan(B, a.T, a.H, a.n_seqs, varlen);
+  if (!workspace || workspace_bytes < plan.total) {
     if (why) *why = "workspace too small for the chunked gated delta rule";
     return cudaErrorInvalidValue;
   }
+  if (plan.slots * a.H > 0x7fffffffLL || a.n_seqs * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   __nv_bfloat16 *w = reinterpret_cast<__nv_bfloat16 *>(ws);
-  __nv_bfloat16 *ut = reinterpret_cast<__nv_bfloat16 *>(ws + wu_bytes(B, a.T, a.H));
-  int32_t *coff = varlen ? reinterpret_cast<int32_t *>(ws + 2 * wu_bytes(B, a.T, a.H)) : nullptr;
+  __nv_bfloat16 *ut = reinterpret_cast<__nv_bfloat16 *>(ws + plan.wu);
+  __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * plan.wu);
+  float *bt = reinterpret_cast<float *>(ws + 3 * plan.wu);
+  int32_t *coff = varlen ? reinterpret_cast<int32_t *>(ws + 3 * plan.wu + plan.bt) : nullptr;
   const TensorView wv{w, a.T * a.H * kD, (int64_t)a.H * kD, kD};
   const TensorView uv{ut, a.T * a.H * kD, (int64_t)a.H * kD, kD};
-  CUtensorMap mq, mk, mv, mw, mu;
+  const TensorView kv{kt, a.T * a.H * kD, (int64_t)a.H * kD, kD};
+  CUtensorMap mq, mk, mv, mw, mu, mkt;
   if (!make_map(&mq, a.q, B, a.T, a.H, kD, kC) || !make_map(&mk, a.k, B, a.T, a.H, kD, kC) ||
       !make_map(&mv, a.v, B, a.T, a.H, kD, kC) || !make_map(&mw, wv, B, a.T, a.H, kD, kC) ||
-      !make_map(&mu, uv, B, a.T, a.H, kD, kC)) {
+      !make_map(&mu, uv, B, a.T, a.H, kD, kC) || !make_map(&mkt, kv, B, a.T, a.H, kD, kC)) {
     if (why) *why = "cuTensorMapEncodeTiled rejected a tensor";
     return cudaErrorInvalidValue;
   }
   cudaError_t err;
-  // 1. the per-chunk WY pass (grid: chunk slots x heads; packed batches bound the slot count)
-  const int64_t nck = (a.T + kC - 1) / kC;
-  const int64_t slots = varlen ? nck + a.n_seqs : a.n_seqs * nck;
-  if (slots * a.H > 0x7fffffffLL || a.n_seqs * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (slots > 0 && a.T > 0) {
+  // 1. the per-chunk WY pass (grid: chunk slots x heads)
+  if (plan.slots > 0 && a.T > 0) {
     if (varlen) {
       gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.n_seqs, coff);
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -922,12 +949,14 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
     p.coff = coff;
     p.w = w;
     p.ut = ut;
+    p.kt = kt;
+    p.bt = bt;
     p.T = a.T;
     p.n_seqs = a.n_seqs;
     p.H = a.H;
     err = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepCfg::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    gdn_prep_kernel<<<(unsigned)(slots * a.H), 128, PrepCfg::SMEM_BYTES, stream>>>(mk, mv, p);
+    gdn_prep_kernel<<<(unsigned)(plan.slots * a.H), 128, PrepCfg::SMEM_BYTES, stream>>>(mk, mv, p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   // 2. the sequential pass, one CTA per (sequence, head)
@@ -936,7 +965,9 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   t.o_sb = a.o_sb;
   t.o_st = a.o_st;
   t.o_sh = a.o_sh;
-  t.g = a.g;
+  t.bt = bt;
+  t.coff = coff;
+  t.nck = plan.nck;
   t.init = a.init;
   t.final_state = a.final_state;
   t.cu_seqlens = a.cu_seqlens;
@@ -946,7 +977,7 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   auto kern = gdn_tc_kernel<kStages>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  kern<<<(unsigned)(a.n_seqs * a.H), kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mw, mu, t);
+  kern<<<(unsigned)(a.n_seqs * a.H), kThreads, G::SMEM_BYTES, stream>>>(mq, mkt, mw, mu, t);
   return cudaGetLastError();
 }
 

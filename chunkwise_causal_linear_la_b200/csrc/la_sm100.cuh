@@ -97,6 +97,17 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *tmap, 
       : "memory");
 }
 
+// Contiguous copy of `bytes` from global to shared memory (both addresses
+// 16-byte aligned, bytes a multiple of 16); completion is signalled on `bar`
+// as transaction bytes.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- TMEM
 // Allocation is warp-wide; the base address is written to shared memory.
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
