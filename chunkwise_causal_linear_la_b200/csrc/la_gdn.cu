@@ -100,7 +100,7 @@ struct PrepArgs {
 struct PrepCfg {
   static constexpr int OFF_K = 0;              // K, then diag(beta e^b / |k|) K
   static constexpr int OFF_V = OFF_K + kTile;  // V, then diag(beta) V
-  static constexpr int OFF_A = OFF_V + kTile;  // A, fp32 [C][A_LD]; afterwards T^T, bf16 [C x C]
+  static constexpr int OFF_A = OFF_V + kTile;  // A, fp32 [C][A_LD], inverted in place; then T, bf16 [C x C]
   static constexpr int A_LD = kC + 4;          // rows 16-byte aligned for float4 access
   static constexpr int OFF_VEC = OFF_A + kC * A_LD * 4;  // b_i, beta_i, 1/max(|k_i|, 1e-12): 3 x C floats
   static constexpr int OFF_BAR = OFF_VEC + 3 * kC * 4;   // 0: tiles landed, 1: products done
@@ -153,30 +153,105 @@ __global__ void __launch_bounds__(1024) gdn_chunk_offsets_kernel(const int32_t *
   }
 }
 
-// Columns j of T = (I + A)^{-1} by forward substitution in fp32:
-// x_i = [i == j] - sum_{m<i} A_im x_m.  Every lane of a warp walks the same rows,
-// so each read of A is a broadcast; the sums use paired fp32 FMAs.  W0: the
-// warp's first column; rows and columns below it are zero for all its lanes.
-template <int W0>
-__device__ __forceinline__ void solve_column(const float *As, int j, float2 (&x2)[kC / 2]) {
+// ---- T = (I + A)^{-1} for the strictly lower-triangular C x C matrix A (fp32,
+// leading dimension A_LD), in place, by blocks.  With L = I + A split into
+// halves, L = [L1 0; L21 L2] gives L^{-1} = [L1^{-1} 0; -L2^{-1} L21 L1^{-1} L2^{-1}],
+// and the same split of each 32 x 32 half into 16 x 16 blocks D_k = (I + A_kk)^{-1}:
+//   level 0  the four D_k by forward substitution (thread = one column of one block)
+//   level 1  the lower-left 16 x 16 block of each half, -D_1 A_10 D_0 and -D_3 A_32 D_2
+//   level 2  the lower-left 32 x 32 block, -L2^{-1} (L21 L1^{-1})
+// Products go through strips: a thread forms one row of 8 consecutive columns
+// with paired fp32 FMAs.  Intermediate blocks use the (zero) upper triangle.
+
+// out[e] = sum_{m in [m0, m1)} X[r][m] Y[m][c + e], e < 8 (X, Y fp32, leading dimension A_LD)
+template <int M0, int M1>
+__device__ __forceinline__ void strip_product(const float *X, const float *Y, int r, int c, float (&out)[8]) {
+  constexpr int LD = PrepCfg::A_LD;
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int q = 0; q < kC / 2; ++q) x2[q] = make_float2(0.f, 0.f);
+  for (int m = M0; m < M1; m += 4) {
+    const float4 xv = *reinterpret_cast<const float4 *>(X + r * LD + m);
+    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-  for (int i = W0; i < kC; ++i) {
-    const float4 *a4 = reinterpret_cast<const float4 *>(As + i * PrepCfg::A_LD);
-    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int m = W0; m < i; m += 4) {  // A_im = 0 for m >= i, and x_m is still 0 there
-      const float4 av = a4[m >> 2];
-      s0 = __ffma2_rn(make_float2(av.x, av.y), x2[m >> 1], s0);
-      s1 = __ffma2_rn(make_float2(av.z, av.w), x2[(m >> 1) + 1], s1);
+    for (int u = 0; u < 4; ++u) {
+      const float4 y0 = *reinterpret_cast<const float4 *>(Y + (m + u) * LD + c);
+      const float4 y1 = *reinterpret_cast<const float4 *>(Y + (m + u) * LD + c + 4);
+      const float2 xx = make_float2(xs[u], xs[u]);
+      acc[0] = __ffma2_rn(xx, make_float2(y0.x, y0.y), acc[0]);
+      acc[1] = __ffma2_rn(xx, make_float2(y0.z, y0.w), acc[1]);
+      acc[2] = __ffma2_rn(xx, make_float2(y1.x, y1.y), acc[2]);
+      acc[3] = __ffma2_rn(xx, make_float2(y1.z, y1.w), acc[3]);
     }
-    const float xi = i < j ? 0.f : (i == j ? 1.f : -((s0.x + s0.y) + (s1.x + s1.y)));
-    if (i & 1)
-      x2[i >> 1].y = xi;
-    else
-      x2[i >> 1].x = xi;
   }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    out[2 * q] = acc[q].x;
+    out[2 * q + 1] = acc[q].y;
+  }
+}
+
+__device__ __forceinline__ void store_strip(float *dst, const float (&v)[8], float sc) {
+  reinterpret_cast<float4 *>(dst)[0] = make_float4(sc * v[0], sc * v[1], sc * v[2], sc * v[3]);
+  reinterpret_cast<float4 *>(dst)[1] = make_float4(sc * v[4], sc * v[5], sc * v[6], sc * v[7]);
+}
+
+// Called by all 128 threads of the CTA (contains __syncthreads).
+__device__ __forceinline__ void invert_unit_lower(float *As, int tid) {
+  constexpr int LD = PrepCfg::A_LD;
+  const int warp = tid >> 5, lane = tid & 31;
+  // level 0: thread tid < 64 solves column j of block k: x_i = [i == j] - sum_{m<i} A_kk[i][m] x_m
+  float x[16];
+  const int k0 = tid >> 4, j0 = tid & 15;
+  if (tid < 64) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float *arow = As + (16 * k0 + i) * LD + 16 * k0;
+      float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < i; m += 4) {  // A_im = 0 for m >= i; x_m = 0 beyond what is solved
+        const float4 av = *reinterpret_cast<const float4 *>(arow + m);
+        s0 = __ffma2_rn(make_float2(av.x, av.y), make_float2(x[m], x[m + 1]), s0);
+        s1 = __ffma2_rn(make_float2(av.z, av.w), make_float2(x[m + 2], x[m + 3]), s1);
+      }
+      x[i] = i < j0 ? 0.f : (i == j0 ? 1.f : -((s0.x + s0.y) + (s1.x + s1.y)));
+    }
+  }
+  __syncthreads();  // the diagonal blocks of A are read: D_k replaces them
+  if (tid < 64) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) As[(16 * k0 + i) * LD + 16 * k0 + j0] = x[i];
+  }
+  __syncthreads();
+  // level 1: warp 0 the first half (blocks 0, 1), warp 1 the second (blocks 2, 3)
+  if (warp < 2) {
+    const int r = lane & 15, c = 8 * (lane >> 4), o = 32 * warp;  // strip (r, c) of a 16 x 16 block
+    float v[8];
+    // X = A_10 D_0 into the (zero) upper block (0, 1) of the half
+    strip_product<0, 16>(As + (o + 16) * LD + o, As + o * LD + o, r, c, v);
+    __syncwarp();
+    store_strip(As + (o + r) * LD + o + 16 + c, v, 1.f);
+    __syncwarp();
+    // -D_1 X over A_10; then the scratch block back to zero
+    strip_product<0, 16>(As + (o + 16) * LD + o + 16, As + o * LD + o + 16, r, c, v);
+    __syncwarp();
+    store_strip(As + (o + 16 + r) * LD + o + c, v, -1.f);
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    store_strip(As + (o + r) * LD + o + 16 + c, z, 1.f);
+  }
+  __syncthreads();
+  // level 2: Y = L21 L1^{-1} (32 x 32) into the upper-right quarter, then -L2^{-1} Y over L21
+  {
+    const int r = lane, c = 8 * warp;  // strip (r, c) of a 32 x 32 block
+    float v[8];
+    strip_product<0, 32>(As + 32 * LD, As, r, c, v);  // L1^{-1} is zero above its diagonal
+    store_strip(As + r * LD + 32 + c, v, 1.f);
+    __syncthreads();
+    strip_product<0, 32>(As + 32 * LD + 32, As + 32, r, c, v);
+    store_strip(As + (32 + r) * LD + c, v, -1.f);
+  }
+  __syncthreads();
 }
 
 // One CTA per (sequence, chunk, head), four per SM.  Thread tt owns the
@@ -360,22 +435,25 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
-  // ---- T = (I + A)^{-1}: thread j < C solves column j (warp 1 starts at row and column 32)
-  float2 x2[kC / 2];
-  if (ok && tid < kC) {
-    if (warp == 0)
-      solve_column<0>(As, tid, x2);
-    else
-      solve_column<32>(As, tid, x2);
-  }
-  __syncthreads();  // every read of A is done: T^T (bf16, row j = column j of T) replaces it
-  if (ok && tid < kC) {
-    uint8_t *trow = sm + P::OFF_A + tid * 128;
+  // ---- T = (I + A)^{-1} in place (fp32), then as bf16 [C x C] K-major over the start of A
+  // (every thread takes part, whatever `ok` says: the inverse synchronises the CTA)
+  invert_unit_lower(As, tid);
+  uint4 tpk[4];
+  {
+    const int ti = tid >> 1, th = tid & 1;  // row and 32-column half of T
+    const float4 *trow = reinterpret_cast<const float4 *>(As + ti * P::A_LD + th * 32);
 #pragma unroll
-    for (int p = 0; p < 8; ++p)
-      *reinterpret_cast<uint4 *>(trow + ((p ^ (tid & 7)) << 4)) =
-          make_uint4(pack2(x2[4 * p].x, x2[4 * p].y), pack2(x2[4 * p + 1].x, x2[4 * p + 1].y),
-                     pack2(x2[4 * p + 2].x, x2[4 * p + 2].y), pack2(x2[4 * p + 3].x, x2[4 * p + 3].y));
+    for (int q = 0; q < 4; ++q) {
+      const float4 a0 = trow[2 * q], a1 = trow[2 * q + 1];
+      const int j = th * 32 + 8 * q;  // zero above the diagonal (the upper triangle held scratch)
+      float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = j + u <= ti ? f[u] : 0.f;
+      tpk[q] = pack8(f);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(sm + P::OFF_A + swz(ti, th * 4 + q)) = tpk[q];
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -383,8 +461,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
 
   // ---- W = T diag(beta e^b) Kt, then Ut = T diag(beta) V (M = C, N = 128, K = C), each into
   // columns [0, 128) and stored as bf16 rows of the workspace
-  const uint64_t dtt = smem_desc_sw128(smem_u32(sm + P::OFF_A), kSlab, 1024);  // T^T: A operand, MN-major
-  constexpr uint32_t ID_X = idesc_bf16_f32(kC, kD, 1, 1);
+  const uint64_t dtt = smem_desc_sw128(smem_u32(sm + P::OFF_A), 16, 1024);  // T: A operand, K-major
+  constexpr uint32_t ID_X = idesc_bf16_f32(kC, kD, 0, 1);
   const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;  // row and 64-column half read back
 #pragma unroll 1
   for (int part = 0; part < 2; ++part) {
@@ -393,7 +471,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
       const uint64_t dx = smem_desc_sw128(smem_u32(sm + (part ? P::OFF_V : P::OFF_K)), kSlab, 1024);
 #pragma unroll
       for (int kk = 0; kk < kC / 16; ++kk)
-        umma_bf16(tbase, dtt + ((kk * 2048) >> 4), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
+        umma_bf16(tbase, dtt + kmaj(kk), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
       umma_commit(bars + 1);
       issued = 2 + part;
     }
@@ -474,9 +552,9 @@ struct GdnCfg {
 
 // Thread roles and per-chunk protocol (chunk c, stage s = c % NS, b = c & 1;
 // "prev" = the chunk starts from a state: c > 0 or an initial state):
-//   MMA:       [prev: FULL, SBFULL] MW -> WSFULL;  [XFORM] M1 -> AFULL[b];
-//              [UREADY] M4 -> UFULL;  [OEMPTY[b], QREADY[s]] prev: M2 -> SBEMPTY;
-//              [PFULL[b]] M3 -> OFULL[b], EMPTY[s].
+//   MMA:       [prev: FULL, SBFULL] MW -> WSFULL;  [UREADY] M4 -> UFULL;
+//              [OEMPTY[b], QREADY[s]] prev: M2 -> SBEMPTY;  [PFULL[b]] M3 -> OFULL[b], EMPTY[s];
+//              [XFORM(c+1)] M1 of chunk c + 1 -> AFULL[b ^ 1]  (M1 of chunk 0 before the loop).
 //   state:     [UFULL(c-1)] S^T <- e^{b_last} S^T + Us;  [prev: SBEMPTY(c-1)] Sb -> SBFULL;
 //              [XFORM, prev: WSFULL] U = Ut - WS in place -> UREADY.
 //   output:    [AFULL[b], XFORM] P -> PFULL[b];  Qd in place -> QREADY[s];
@@ -572,8 +650,23 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint64_t dkd0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_KD), kSlab, 1024); // MN-major
       const uint64_t dp0 = smem_desc_sw128(smem_u32(sm + G::OFF_P), 16, 1024);
       auto soff = [](int s) -> uint64_t { return (uint64_t)(s * (G::STAGE_BYTES >> 4)); };
-      int done = 0;
-      for (int c = 0; c < nchunks; ++c) {
+      int done = 0, m1_issued = 0;
+      // M1 of chunk c: A[c & 1] = Q Kt^T
+      auto issue_scores = [&](int c) -> bool {
+        const int s = c % NS, k = c / NS, b = c & 1;
+        if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_bf16(tbase + G::T_A + b * kC, dq0 + soff(s) + kmaj(kk), dk0 + soff(s) + kmaj(kk), ID_S, kk > 0);
+        umma_commit(bars + G::B_AFULL + b);
+        m1_issued = c + 1;
+        return true;
+      };
+      // Per chunk: MW, M4, M2, M3, then the next chunk's M1, so that its scores and Qd
+      // are ready before its M2 (which gates the next Sb write).
+      const bool started = nchunks == 0 || issue_scores(0);
+      for (int c = 0; c < nchunks && started; ++c) {
         const int s = c % NS, k = c / NS, b = c & 1;
         const uint32_t o_acc = tbase + G::T_O + b * kD;
         bool ok = true;
@@ -587,13 +680,6 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             umma_bf16(tbase + G::T_U, dw0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
           umma_commit(bars + G::B_WSFULL);
         }
-        // M1: A = Q Kt^T
-        if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          umma_bf16(tbase + G::T_A + b * kC, dq0 + soff(s) + kmaj(kk), dk0 + soff(s) + kmaj(kk), ID_S, kk > 0);
-        umma_commit(bars + G::B_AFULL + b);
         // M4: Us = Kd^T U
         if (!wait_bar(sy, G::B_UREADY, c & 1, c)) break;
         tc_fence_after();
@@ -623,11 +709,12 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         umma_commit(bars + G::B_OFULL + b);
         umma_commit(bars + G::B_EMPTY + s);
         done = c + 1;
+        if (c + 1 < nchunks && !issue_scores(c + 1)) break;
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
       for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
-      if (done < nchunks && *abort_flag) {  // products of an aborted chunk may still be running
-        const int c = done;
+      if (m1_issued > done) {  // a score product issued ahead of an aborted chunk
+        const int c = m1_issued - 1;
         drain_bar(sy, G::B_AFULL + (c & 1), (c >> 1) & 1);
       }
     } else if (warp >= 2) {
@@ -726,12 +813,16 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c) || !wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) break;
       const float blast = dtab[s * G::DT_STRIDE + kC - 1];
       const int Cp = chunk_len(c);
+      // U = Ut - WS on row i, columns [64 hf, 64 hf + 64), in place; zero past the chunk end.
+      // The Ut row is read while the product still runs.
+      uint8_t *urow = stage(s) + G::OFF_U + hf * kSlab;
+      uint4 ut[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) ut[p] = *reinterpret_cast<const uint4 *>(urow + swz(i, p));
       if (prev(c)) {
         if (!wait_bar_warp(sy, G::B_WSFULL, sbi(c) & 1, c)) break;
         tc_fence_after();
       }
-      // U = Ut - WS on row i, columns [64 hf, 64 hf + 64), in place; zero past the chunk end
-      uint8_t *urow = stage(s) + G::OFF_U + hf * kSlab;
 #pragma unroll
       for (int pass = 0; pass < 2; ++pass) {
         uint32_t r[32];
@@ -744,12 +835,11 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint4 *p4 = reinterpret_cast<uint4 *>(urow + swz(i, pass * 4 + q));
           float f[8];
-          unpack8(*p4, f);
+          unpack8(ut[pass * 4 + q], f);
 #pragma unroll
           for (int u = 0; u < 8; ++u) f[u] = i < Cp ? f[u] - __uint_as_float(r[8 * q + u]) : 0.f;
-          *p4 = pack8(f);
+          *reinterpret_cast<uint4 *>(urow + swz(i, pass * 4 + q)) = pack8(f);
         }
       }
       fence_proxy_async_smem();
