@@ -157,42 +157,45 @@ __global__ void __launch_bounds__(1024) gdn_chunk_offsets_kernel(const int32_t *
 // leading dimension A_LD), in place, by blocks.  With L = I + A split into
 // halves, L = [L1 0; L21 L2] gives L^{-1} = [L1^{-1} 0; -L2^{-1} L21 L1^{-1} L2^{-1}],
 // and the same split of each 32 x 32 half into 16 x 16 blocks D_k = (I + A_kk)^{-1}:
-//   level 0  the four D_k by forward substitution (thread = one column of one block)
+//   level 0  the four D_k by forward substitution in fp32 (thread = one column of one block)
 //   level 1  the lower-left 16 x 16 block of each half, -D_1 A_10 D_0 and -D_3 A_32 D_2
 //   level 2  the lower-left 32 x 32 block, -L2^{-1} (L21 L1^{-1})
-// Products go through strips: a thread forms one row of 8 consecutive columns
-// with paired fp32 FMAs.  Intermediate blocks use the (zero) upper triangle.
+// The block products run on the warp-level tensor-core instruction (mma.sync
+// m16n8k8, tf32 inputs rounded to nearest, fp32 accumulation): 16 x 8 tiles,
+// with operands loaded straight from the fp32 matrix (conflict-free at this
+// leading dimension).  Intermediate blocks use the (zero) upper triangle.
 
-// out[e] = sum_{m in [m0, m1)} X[r][m] Y[m][c + e], e < 8 (X, Y fp32, leading dimension A_LD)
-template <int M0, int M1>
-__device__ __forceinline__ void strip_product(const float *X, const float *Y, int r, int c, float (&out)[8]) {
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d = X[16 rows][K] Y[K][8 cols] for one warp (X, Y fp32, leading dimension A_LD).  Lane
+// l holds rows l / 4 and l / 4 + 8, columns 2 (l % 4) and 2 (l % 4) + 1.
+template <int K>
+__device__ __forceinline__ void tile_product(const float *X, const float *Y, int lane, float (&d)[4]) {
   constexpr int LD = PrepCfg::A_LD;
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  const int g = lane >> 2, t = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
 #pragma unroll
-  for (int m = M0; m < M1; m += 4) {
-    const float4 xv = *reinterpret_cast<const float4 *>(X + r * LD + m);
-    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 y0 = *reinterpret_cast<const float4 *>(Y + (m + u) * LD + c);
-      const float4 y1 = *reinterpret_cast<const float4 *>(Y + (m + u) * LD + c + 4);
-      const float2 xx = make_float2(xs[u], xs[u]);
-      acc[0] = __ffma2_rn(xx, make_float2(y0.x, y0.y), acc[0]);
-      acc[1] = __ffma2_rn(xx, make_float2(y0.z, y0.w), acc[1]);
-      acc[2] = __ffma2_rn(xx, make_float2(y1.x, y1.y), acc[2]);
-      acc[3] = __ffma2_rn(xx, make_float2(y1.z, y1.w), acc[3]);
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    out[2 * q] = acc[q].x;
-    out[2 * q + 1] = acc[q].y;
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const uint32_t a0 = to_tf32(X[g * LD + k0 + t]), a1 = to_tf32(X[(g + 8) * LD + k0 + t]);
+    const uint32_t a2 = to_tf32(X[g * LD + k0 + t + 4]), a3 = to_tf32(X[(g + 8) * LD + k0 + t + 4]);
+    const uint32_t b0 = to_tf32(Y[(k0 + t) * LD + g]), b1 = to_tf32(Y[(k0 + t + 4) * LD + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
 }
 
-__device__ __forceinline__ void store_strip(float *dst, const float (&v)[8], float sc) {
-  reinterpret_cast<float4 *>(dst)[0] = make_float4(sc * v[0], sc * v[1], sc * v[2], sc * v[3]);
-  reinterpret_cast<float4 *>(dst)[1] = make_float4(sc * v[4], sc * v[5], sc * v[6], sc * v[7]);
+__device__ __forceinline__ void store_tile(float *dst, const float (&d)[4], int lane, float sc) {
+  constexpr int LD = PrepCfg::A_LD;
+  const int g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2 *>(dst + g * LD + 2 * t) = make_float2(sc * d[0], sc * d[1]);
+  *reinterpret_cast<float2 *>(dst + (g + 8) * LD + 2 * t) = make_float2(sc * d[2], sc * d[3]);
 }
 
 // Called by all 128 threads of the CTA (contains __syncthreads).
@@ -226,30 +229,42 @@ __device__ __forceinline__ void invert_unit_lower(float *As, int tid) {
   __syncthreads();
   // level 1: warp 0 the first half (blocks 0, 1), warp 1 the second (blocks 2, 3)
   if (warp < 2) {
-    const int r = lane & 15, c = 8 * (lane >> 4), o = 32 * warp;  // strip (r, c) of a 16 x 16 block
-    float v[8];
+    const int o = 32 * warp;
+    float d[2][4];
     // X = A_10 D_0 into the (zero) upper block (0, 1) of the half
-    strip_product<0, 16>(As + (o + 16) * LD + o, As + o * LD + o, r, c, v);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) tile_product<16>(As + (o + 16) * LD + o, As + o * LD + o + 8 * nt, lane, d[nt]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) store_tile(As + o * LD + o + 16 + 8 * nt, d[nt], lane, 1.f);
     __syncwarp();
-    store_strip(As + (o + r) * LD + o + 16 + c, v, 1.f);
+    // -D_1 X over A_10
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+      tile_product<16>(As + (o + 16) * LD + o + 16, As + o * LD + o + 16 + 8 * nt, lane, d[nt]);
     __syncwarp();
-    // -D_1 X over A_10; then the scratch block back to zero
-    strip_product<0, 16>(As + (o + 16) * LD + o + 16, As + o * LD + o + 16, r, c, v);
-    __syncwarp();
-    store_strip(As + (o + 16 + r) * LD + o + c, v, -1.f);
-    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    store_strip(As + (o + r) * LD + o + 16 + c, z, 1.f);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) store_tile(As + (o + 16) * LD + o + 8 * nt, d[nt], lane, -1.f);
+    // the scratch block back to zero
+    const float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) store_tile(As + o * LD + o + 16 + 8 * nt, z, lane, 1.f);
   }
   __syncthreads();
-  // level 2: Y = L21 L1^{-1} (32 x 32) into the upper-right quarter, then -L2^{-1} Y over L21
+  // level 2: Y = L21 L1^{-1} (32 x 32) into the upper-right quarter, then -L2^{-1} Y over L21;
+  // warp w: row tile w % 2, column tiles 2 (w / 2) and 2 (w / 2) + 1
   {
-    const int r = lane, c = 8 * warp;  // strip (r, c) of a 32 x 32 block
-    float v[8];
-    strip_product<0, 32>(As + 32 * LD, As, r, c, v);  // L1^{-1} is zero above its diagonal
-    store_strip(As + r * LD + 32 + c, v, 1.f);
+    const int mt = warp & 1, n0 = 2 * (warp >> 1);
+    float d[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) tile_product<32>(As + (32 + 16 * mt) * LD, As + 8 * (n0 + u), lane, d[u]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) store_tile(As + 16 * mt * LD + 32 + 8 * (n0 + u), d[u], lane, 1.f);
     __syncthreads();
-    strip_product<0, 32>(As + 32 * LD + 32, As + 32, r, c, v);
-    store_strip(As + (32 + r) * LD + c, v, -1.f);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      tile_product<32>(As + (32 + 16 * mt) * LD + 32, As + 32 + 8 * (n0 + u), lane, d[u]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) store_tile(As + (32 + 16 * mt) * LD + 8 * (n0 + u), d[u], lane, -1.f);
   }
   __syncthreads();
 }
