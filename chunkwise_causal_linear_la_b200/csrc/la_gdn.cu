@@ -98,9 +98,10 @@ struct PrepArgs {
 };
 
 struct PrepCfg {
-  static constexpr int OFF_K = 0;              // K, then diag(beta e^b / |k|) K
-  static constexpr int OFF_V = OFF_K + kTile;  // V, then diag(beta) V
-  static constexpr int OFF_A = OFF_V + kTile;  // A, fp32 [C][A_LD], inverted in place; then T, bf16 [C x C]
+  static constexpr int OFF_K = 0;              // K (rows past the chunk end zeroed)
+  static constexpr int OFF_V = OFF_K + kTile;  // V (likewise)
+  // A, fp32 [C][A_LD], inverted in place; then T diag(beta) and T diag(beta e^b / |k|), bf16
+  static constexpr int OFF_A = OFF_V + kTile;
   static constexpr int A_LD = kC + 4;          // rows 16-byte aligned for float4 access
   static constexpr int OFF_VEC = OFF_A + kC * A_LD * 4;  // b_i, beta_i, 1/max(|k_i|, 1e-12): 3 x C floats
   static constexpr int OFF_BAR = OFF_VEC + 3 * kC * 4;   // 0: tiles landed, 1: products done
@@ -372,7 +373,9 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
     umma_commit(bars + 1);
     issued = 1;
   }
-  // while it runs: 1/|k_i| and diag(beta) V in place (rows past the chunk end: zero)
+  // while it runs: 1/|k_i| and the unit keys to the workspace.  Rows past the chunk end
+  // must not reach the products below (they may hold anything): V rows become zero here,
+  // K rows once G is done.
   if (ok) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -399,15 +402,9 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
         *reinterpret_cast<uint4 *>(kd) = pack8(f0);
         *reinterpret_cast<uint4 *>(kd + 64) = pack8(f1);
       }
-      const float bt = betav[r];
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        uint4 *p4 = reinterpret_cast<uint4 *>(sm + P::OFF_V + sl * kSlab + off);
-        float f[8];
-        unpack8(*p4, f);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) f[u] = r < Cp ? f[u] * bt : 0.f;
-        *p4 = pack8(f);
+      if (r >= Cp) {
+        *reinterpret_cast<uint4 *>(sm + P::OFF_V + off) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(sm + P::OFF_V + kSlab + off) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
@@ -432,61 +429,64 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
       }
       arow[q] = make_float4(e4[0], e4[1], e4[2], e4[3]);
     }
-    // diag(beta e^b / |k|) K in place (the product has read K)
+    // K rows past the chunk end to zero (the product has read K)
+    if (Cp < kC) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int rr = (tid >> 3) + 16 * m;
-      const float wk = betav[rr] * exp_fast(bvec[rr]) * invn[rr];
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        uint4 *p4 = reinterpret_cast<uint4 *>(sm + P::OFF_K + sl * kSlab + (tid + 128 * m) * 16);
-        float f[8];
-        unpack8(*p4, f);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) f[u] = rr < Cp ? f[u] * wk : 0.f;
-        *p4 = pack8(f);
+      for (int m = 0; m < 4; ++m) {
+        if ((tid >> 3) + 16 * m < Cp) continue;
+        *reinterpret_cast<uint4 *>(sm + P::OFF_K + (tid + 128 * m) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(sm + P::OFF_K + kSlab + (tid + 128 * m) * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  // ---- T = (I + A)^{-1} in place (fp32), then as bf16 [C x C] K-major over the start of A
+  // ---- T = (I + A)^{-1} in place (fp32).  The row scalings of the right-hand sides
+  // move onto the columns of T: W = (T diag(beta e^b / |k|)) K and Ut = (T diag(beta)) V,
+  // stored as two bf16 [C x C] tiles in the MN-major layout (row j = column j of T).
+  // Thread (j, hr) handles rows [32 hr, 32 hr + 32) of column j.
   // (every thread takes part, whatever `ok` says: the inverse synchronises the CTA)
   invert_unit_lower(As, tid);
-  uint4 tpk[4];
   {
-    const int ti = tid >> 1, th = tid & 1;  // row and 32-column half of T
-    const float4 *trow = reinterpret_cast<const float4 *>(As + ti * P::A_LD + th * 32);
+    const int j = tid & 63, hr = tid >> 6;
+    const float cu = betav[j], cw = cu * exp_fast(bvec[j]) * invn[j];
+    float tc[32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 a0 = trow[2 * q], a1 = trow[2 * q + 1];
-      const int j = th * 32 + 8 * q;  // zero above the diagonal (the upper triangle held scratch)
-      float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] = j + u <= ti ? f[u] : 0.f;
-      tpk[q] = pack8(f);
+    for (int u = 0; u < 32; ++u) {
+      const int i = 32 * hr + u;  // zero above the diagonal (the upper triangle held scratch)
+      tc[u] = i >= j ? As[i * P::A_LD + j] : 0.f;
     }
     __syncthreads();
+    uint8_t *tu = sm + P::OFF_A, *tw = sm + P::OFF_A + kSlab;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(sm + P::OFF_A + swz(ti, th * 4 + q)) = tpk[q];
+    for (int q = 0; q < 4; ++q) {
+      float fu[8], fw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        fu[u] = tc[8 * q + u] * cu;
+        fw[u] = tc[8 * q + u] * cw;
+      }
+      *reinterpret_cast<uint4 *>(tu + swz(j, 4 * hr + q)) = pack8(fu);
+      *reinterpret_cast<uint4 *>(tw + swz(j, 4 * hr + q)) = pack8(fw);
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
 
-  // ---- W = T diag(beta e^b) Kt, then Ut = T diag(beta) V (M = C, N = 128, K = C), each into
-  // columns [0, 128) and stored as bf16 rows of the workspace
-  const uint64_t dtt = smem_desc_sw128(smem_u32(sm + P::OFF_A), 16, 1024);  // T: A operand, K-major
-  constexpr uint32_t ID_X = idesc_bf16_f32(kC, kD, 0, 1);
+  // ---- W, then Ut (M = C, N = 128, K = C), each into columns [0, 128) and stored as bf16
+  // rows of the workspace
+  constexpr uint32_t ID_X = idesc_bf16_f32(kC, kD, 1, 1);  // A = T-tile, MN-major
   const int i = (warp & 3) * 16 + (lane & 15), hf = lane >> 4;  // row and 64-column half read back
 #pragma unroll 1
   for (int part = 0; part < 2; ++part) {
     if (ok && tid == 0) {
       tc_fence_after();
       const uint64_t dx = smem_desc_sw128(smem_u32(sm + (part ? P::OFF_V : P::OFF_K)), kSlab, 1024);
+      const uint64_t dt = smem_desc_sw128(smem_u32(sm + P::OFF_A + (part ? 0 : kSlab)), kSlab, 1024);
 #pragma unroll
       for (int kk = 0; kk < kC / 16; ++kk)
-        umma_bf16(tbase, dtt + kmaj(kk), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
+        umma_bf16(tbase, dt + ((kk * 2048) >> 4), dx + ((kk * 2048) >> 4), ID_X, kk > 0);
       umma_commit(bars + 1);
       issued = 2 + part;
     }
