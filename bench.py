@@ -150,7 +150,7 @@ def _algorithmic(w, n_seqs, tokens):
 
 def _kernel_sources_sha():
     h = hashlib.sha256()
-    for fn in ("la_tc.cu", "la_sm100.cuh", "la_common.cuh"):
+    for fn in ("la_tc.cu", "la_tc_sync.cuh", "la_sm100.cuh", "la_common.cuh"):
         with open(os.path.join(ROOT, "chunkwise_causal_linear_la_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
