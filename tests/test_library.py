@@ -143,6 +143,29 @@ def test_validation_rejects_bad_arguments_before_any_device_call(lib):
     assert _call(lib, q=null) == b.LA_ERR_INVALID_ARG
 
 
+def test_gated_delta_chunk_arguments_validated_on_host(lib):
+    """la_fwd_gated_delta_chunk rejects bad arguments, unknown flags and a short or
+    misaligned workspace before any device call (d = 128 bf16 takes the tensor cores)."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    q, k, v, o = _t(D=128), _t(D=128), _t(D=128), _t(D=128)
+    need = lib.la_fwd_gated_delta_workspace_size(1, 4, 2, 128, 128, 1, 0, 1, 0)
+    assert need > 0
+
+    def call(g=0x2000, beta=0x3000, n=1, flags=0, ws=0x100000, ws_bytes=None, qq=None):
+        return lib.la_fwd_gated_delta_chunk(ctypes.byref(qq or q), ctypes.byref(k), ctypes.byref(v), g, beta, None,
+                                            n, None, ctypes.byref(o), None, flags, ws,
+                                            need if ws_bytes is None else ws_bytes, None)
+    assert call(g=None) == b.LA_ERR_INVALID_ARG and b"beta" in lib.la_last_error()
+    assert call(beta=0x3002) == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()
+    assert call(n=2) == b.LA_ERR_INVALID_ARG
+    assert call(flags=2) == b.LA_ERR_INVALID_ARG and b"flags" in lib.la_last_error()
+    assert call(ws_bytes=need - 1) == b.LA_ERR_WORKSPACE
+    assert call(ws=None) == b.LA_ERR_WORKSPACE
+    assert call(ws=0x100010) == b.LA_ERR_INVALID_ARG and b"256" in lib.la_last_error()
+    assert call(qq=_t(D=96)) == b.LA_ERR_INVALID_ARG  # q and k head dims disagree
+
+
 def test_normaliser_state_arguments_validated_on_host(lib):
     """la_fwd_chunk_z needs normalize for final_z and a 16-byte aligned final_z;
     la_step_norm needs a z pointer.  All rejected before any device call."""
