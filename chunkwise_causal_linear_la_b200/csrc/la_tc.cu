@@ -425,12 +425,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         m1_issued = c + 1;
         return true;
       };
-      // Issue order per chunk c with three stages: M4(c), M1(c+1), M2(c), M3(c).
-      // The next chunk's scores are queued before waiting for this chunk's P
-      // tile, so the score step of chunk c+1 overlaps the P V product of chunk c.
-      // With two stages the tiles of chunk c+1 wait for the release of chunk
-      // c-1's stage, so M1(c+1) goes last: M4(c), M2(c), M3(c), M1(c+1).
-      constexpr bool kScoresAhead = NS >= 3;
       int done = 0;
       if (MODE == 1) {
         // state pass: U = kd^T V per chunk; the stage is released once the state
@@ -458,61 +452,160 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       const int sbo = has_init ? 1 : 0;  // an initial state adds one Sb hand-over before chunk 0
-      bool ok = MODE == 1 || nchunks == 0 || issue_scores(0);
-      for (int c = 0; c < nchunks && ok && MODE == 0; ++c) {
-        const int s = c % NS, b = c & 1;
-        const int ob = out_buf(c);
-        const uint32_t oph = out_phase(c);
-        const uint64_t dq = dq0 + stage_off(s);
-        const uint64_t dv = dv0 + stage_off(s);
-        const uint64_t dkd = dkm0 + stage_off(s);
-        // M4: this chunk's state update U = kd^T V (value decay: kh^T vd)
-        if (c > 0) {
-          if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
-          tc_fence_after();
-        }
-        const uint64_t dvu = vd_mode ? dvd : dv;
-#pragma unroll
-        for (int mb = 0; mb < G::MB; ++mb) {
-#pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk)
-            umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
-                      dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
-        }
-        umma_commit(bars + G::B_UFULL);
-        // M1 of the next chunk, ahead of M2 / M3 when three stages are in flight
-        if (kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
-        // M2 / M3: output accumulators
-        if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1, c)) break;
-        tc_fence_after();
-        const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
-        const uint32_t o_intra = vd_mode ? o_inter + DVT : o_inter;
-        if (c > 0 || has_init) {
-          if (!wait_bar(sy, G::B_SBFULL, (c - 1 + sbo) & 1, c)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-            umma_bf16(o_inter, dq + off, dsb + ((kk * 2048) >> 4), ID_M2, kk > 0);
+      if constexpr (NS < 3) {
+        // Two stages (d_k = 256): a fixed order per chunk, M4(c), M2(c), M3(c), M1(c+1):
+        // the tiles of chunk c+1 land only after chunk c-1's stage is released.
+        bool ok = MODE == 1 || nchunks == 0 || issue_scores(0);
+        for (int c = 0; c < nchunks && ok && MODE == 0; ++c) {
+          const int s = c % NS, b = c & 1;
+          const int ob = out_buf(c);
+          const uint32_t oph = out_phase(c);
+          const uint64_t dq = dq0 + stage_off(s);
+          const uint64_t dv = dv0 + stage_off(s);
+          const uint64_t dkd = dkm0 + stage_off(s);
+          // M4: this chunk's state update U = kd^T V (value decay: kh^T vd)
+          if (c > 0) {
+            if (!wait_bar(sy, G::B_UEMPTY, (c - 1) & 1, c)) break;
+            tc_fence_after();
           }
-          umma_commit(bars + G::B_SBEMPTY);
-        }
-        if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
-        tc_fence_after();
-        const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
+          const uint64_t dvu = vd_mode ? dvd : dv;
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-          umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
-                    ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+          for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+              umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
+                        dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
+          }
+          umma_commit(bars + G::B_UFULL);
+          // M2 / M3: output accumulators
+          if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1, c)) break;
+          tc_fence_after();
+          const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
+          const uint32_t o_intra = vd_mode ? o_inter + DVT : o_inter;
+          if (c > 0 || has_init) {
+            if (!wait_bar(sy, G::B_SBFULL, (c - 1 + sbo) & 1, c)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+              umma_bf16(o_inter, dq + off, dsb + ((kk * 2048) >> 4), ID_M2, kk > 0);
+            }
+            umma_commit(bars + G::B_SBEMPTY);
+          }
+          if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
+          tc_fence_after();
+          const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+            umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
+                      ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bars + G::B_OFULL + ob);
+          if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
+          umma_commit(bars + G::B_EMPTY + s);
+          done = c + 1;
+          if (c + 1 < nchunks && !issue_scores(c + 1)) break;
         }
-        umma_commit(bars + G::B_OFULL + ob);
-        if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
-        umma_commit(bars + G::B_EMPTY + s);
-        done = c + 1;
-        // with two stages, chunk c+1's tiles land only after chunk c-1's stage is
-        // released: its scores follow this chunk's products instead
-        if (!kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
+      } else {
+        // Output pass: an event loop.  The thread keeps the next chunk of each product
+        // (M1, M4, M2, M3) and of the stage release, and issues whichever product has
+        // its operands ready (probing the barriers without blocking), M2 and M4 first:
+        // they gate the state warps' serial chain (Sb -> M2 -> SBEMPTY -> next Sb, and
+        // M4 -> UFULL -> S update).  Issuing in a fixed order instead leaves the tensor
+        // pipe idle while one barrier is awaited and another product is ready.
+        //   M1(c): stage c transformed; A[c % 2] free once the scores of chunk c - 2 are
+        //          read (M3 of chunk c - 2 waited for them).
+        //   M4(c): after M1(c) (stage c transformed); T_U free (UEMPTY of chunk c - 1).
+        //   M2(c): after M1(c); its O buffer free (OEMPTY); Sb of chunk c (SBFULL).
+        //   M3(c): after M2(c) (accumulates onto it); P(c) (PFULL).
+        //   release of stage c: after all four (and, normalised or gated, ZFULL).
+        int c1 = 0, c4 = 0, c2 = 0, c3 = 0, ce = 0;
+        long long idle0 = clock64();
+        while (MODE == 0 && ce < nchunks) {
+          bool progress = false;
+          if (*abort_flag) break;
+          // M2(c2)
+          if (c2 < c1 && mbar_test(bars + G::B_OEMPTY + out_buf(c2), out_phase(c2) ^ 1) &&
+              (!(c2 > 0 || has_init) || mbar_test(bars + G::B_SBFULL, (c2 - 1 + sbo) & 1))) {
+            const int c = c2, s = c % NS, ob = out_buf(c);
+            if (c > 0 || has_init) {
+              tc_fence_after();
+              const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
+              const uint64_t dq = dq0 + stage_off(s);
+#pragma unroll
+              for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+                umma_bf16(o_inter, dq + off, dsb + ((kk * 2048) >> 4), ID_M2, kk > 0);
+              }
+              umma_commit(bars + G::B_SBEMPTY);
+            }
+            ++c2;
+            progress = true;
+          }
+          // M4(c4)
+          if (c4 < c1 && (c4 == 0 || mbar_test(bars + G::B_UEMPTY, (c4 - 1) & 1))) {
+            const int c = c4, s = c % NS;
+            tc_fence_after();
+            const uint64_t dvu = vd_mode ? dvd : dv0 + stage_off(s);
+            const uint64_t dkd = dkm0 + stage_off(s);
+#pragma unroll
+            for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
+              for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(tbase + G::T_U + mb * DVT, dkd + ((2 * mb * G::SLAB + kk * 2048) >> 4),
+                          dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
+            }
+            umma_commit(bars + G::B_UFULL);
+            ++c4;
+            progress = true;
+          }
+          // M3(c3)
+          if (c3 < c2 && mbar_test(bars + G::B_PFULL + (c3 & 1), (c3 >> 1) & 1)) {
+            const int c = c3, s = c % NS, b = c & 1, ob = out_buf(c);
+            tc_fence_after();
+            const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
+            const uint32_t o_intra = vd_mode ? o_inter + DVT : o_inter;
+            const uint64_t dv = dv0 + stage_off(s);
+            const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
+              umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
+                        ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bars + G::B_OFULL + ob);
+            ++c3;
+            progress = true;
+          }
+          // M1(c1)
+          if (c1 < nchunks && c1 <= c3 + 1 && mbar_test(bars + G::B_XFORM + c1 % NS, (c1 / NS) & 1)) {
+            if (!issue_scores(c1)) break;  // its wait returns at once
+            c1 = m1_issued;
+            progress = true;
+          }
+          // release of stage ce
+          if (ce < c3 && ce < c4 && (!(NORM || GATED) || mbar_test(bars + G::B_ZFULL + (ce & 1), (ce >> 1) & 1))) {
+            umma_commit(bars + G::B_EMPTY + ce % NS);
+            ++ce;
+            progress = true;
+          }
+          if (progress) {
+            idle0 = clock64();
+          } else if (clock64() - idle0 > kTimeoutCycles) {
+            *abort_flag = 1;
+            atomicOr(&g_tc_error, 1u);
+            atomicCAS(&g_tc_where, 0u, 0x80000000u | ((uint32_t)(ce & 0x7FFFFF) << 8) | 0xFFu);
+            break;
+          }
+        }
+        if (MODE == 0) done = ce;
+        if (*abort_flag) {  // products issued past the last released stage: let them finish
+          const long long t = clock64();
+          while (clock64() - t < 200000) {
+          }
+        }
+
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
       for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
