@@ -809,16 +809,20 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     for (int c = 0; c < nchunks && ok; ++c) {
       const int s = c % NS, k = c / NS;
       ok = false;
-      if (c > 0) {  // S^T <- e^{b_last} S^T + Us of chunk c - 1
+      if (c > 0) {  // S^T <- e^{b_last} S^T + Us of chunk c - 1 (two loads in flight per wait)
         if (!wait_bar_warp(sy, G::B_UFULL, (c - 1) & 1, c)) break;
         tc_fence_after();
 #pragma unroll
-        for (int grp = 0; grp < kD / 32; ++grp) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(lane_base + G::T_U + grp * 32, r);
+        for (int grp = 0; grp < kD / 32; grp += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(lane_base + G::T_U + grp * 32, r0);
+          tmem_ld_32x32b_x32(lane_base + G::T_U + grp * 32 + 32, r1);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) S[grp * 32 + e] = fmaf(gdec, S[grp * 32 + e], __uint_as_float(r[e]));
+          for (int e = 0; e < 32; ++e) {
+            S[grp * 32 + e] = fmaf(gdec, S[grp * 32 + e], __uint_as_float(r0[e]));
+            S[grp * 32 + 32 + e] = fmaf(gdec, S[grp * 32 + 32 + e], __uint_as_float(r1[e]));
+          }
         }
       }
       if (prev(c)) {  // Sb of chunk c, once the products of chunk c - 1 have read the previous one
