@@ -779,18 +779,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         gdec = exp_fast(bl);
         seg_log += bl;
       }
+      // two 32-column loads in flight per wait
 #pragma unroll
-      for (int mb = 0; mb < G::MB; ++mb) {
+      for (int g2 = 0; g2 < G::RPT / 64; ++g2) {
+        uint32_t r0[32], r1[32];
+        const uint32_t col = G::T_U + g2 * 64;  // state values [64 g2, 64 g2 + 64) of this thread
+        tmem_ld_32x32b_x32(tbase + ((uint32_t)(sp * 32) << 16) + col, r0);
+        tmem_ld_32x32b_x32(tbase + ((uint32_t)(sp * 32) << 16) + col + 32, r1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int grp = 0; grp < DVT / 32; ++grp) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tbase + ((uint32_t)(sp * 32) << 16) + G::T_U + mb * DVT + grp * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float &x = S[mb * DVT + grp * 32 + e];
-            x = fmaf(gdec, x, __uint_as_float(r[e]));
-          }
+        for (int e = 0; e < 32; ++e) {
+          S[g2 * 64 + e] = fmaf(gdec, S[g2 * 64 + e], __uint_as_float(r0[e]));
+          S[g2 * 64 + 32 + e] = fmaf(gdec, S[g2 * 64 + 32 + e], __uint_as_float(r1[e]));
         }
       }
       tc_fence_before();
