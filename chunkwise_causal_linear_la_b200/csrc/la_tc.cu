@@ -452,9 +452,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       const int sbo = has_init ? 1 : 0;  // an initial state adds one Sb hand-over before chunk 0
-      if constexpr (NS < 3) {
-        // Two stages (d_k = 256): a fixed order per chunk, M4(c), M2(c), M3(c), M1(c+1):
-        // the tiles of chunk c+1 land only after chunk c-1's stage is released.
+      if constexpr (!GATED) {
+        // A fixed order per chunk.  Three stages: M4(c), M1(c+1), M2(c), M3(c): the next
+        // chunk's scores are queued before waiting for this chunk's P tile, so the score
+        // step of chunk c+1 overlaps the P V product of chunk c.  Two stages (d_k = 256):
+        // M4(c), M2(c), M3(c), M1(c+1): chunk c+1's tiles land only after chunk c-1's
+        // stage is released.  (Measured faster than the event loop below here; the event
+        // loop wins with the data-dependent decay, whose chunks wait on more barriers.)
+        constexpr bool kScoresAhead = NS >= 3;
         bool ok = MODE == 1 || nchunks == 0 || issue_scores(0);
         for (int c = 0; c < nchunks && ok && MODE == 0; ++c) {
           const int s = c % NS, b = c & 1;
@@ -477,6 +482,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         dvu + ((kk * 2048) >> 4), ID_M4, kk > 0);
           }
           umma_commit(bars + G::B_UFULL);
+          // M1 of the next chunk, ahead of M2 / M3 when three stages are in flight
+          if (kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
           // M2 / M3: output accumulators
           if (!wait_bar(sy, G::B_OEMPTY + ob, oph ^ 1, c)) break;
           tc_fence_after();
@@ -505,7 +512,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
           umma_commit(bars + G::B_EMPTY + s);
           done = c + 1;
-          if (c + 1 < nchunks && !issue_scores(c + 1)) break;
+          if (!kScoresAhead && c + 1 < nchunks && !issue_scores(c + 1)) break;
         }
       } else {
         // Output pass: an event loop.  The thread keeps the next chunk of each product
