@@ -278,9 +278,10 @@ def _config(w, ws):
     }
 
 
-def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False):
-    """Times la_step (norm: la_step_norm, which also carries z) on the decode
-    workload: per-launch CUDA events, four state batches used in turn so that
+def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False, delta=False):
+    """Times la_step (norm: la_step_norm, which also carries z; delta: one token of
+    the gated delta rule, la_fwd_gated_delta with the state updated in place) on the
+    decode workload: per-launch CUDA events, four state batches used in turn so that
     each step's 67 MB state was last touched three steps (~200 MB of traffic)
     earlier and is not served from the 126 MB L2."""
     import torch
@@ -296,8 +297,16 @@ def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False):
     phi = "elu1" if norm else DECODE["phi"]
     zs = [torch.ones(st.shape[:3], dtype=torch.float32, device=dev) for _ in range(4)] if norm else None
 
+    if delta:  # [N, 1, H, d] views, per-(sequence, head) log decay and write strength
+        q4, k4, v4, o4 = dq.unsqueeze(1), dk_.unsqueeze(1), dv_.unsqueeze(1), do.unsqueeze(1)
+        lg = torch.log(dg).reshape(1, 1, -1).expand(dq.shape[0], 1, -1).contiguous()
+        bt = torch.full_like(lg, 0.5)
+
     def call(i):
-        if norm:
+        if delta:
+            la.la_fwd_gated_delta(q4, k4, v4, lg, bt, initial_state=states[i % 4], out=o4,
+                                  final_state=states[i % 4], stream=stream)
+        elif norm:
             la.la_step_norm(dq, dk_, dv_, dg, states[i % 4], zs[i % 4], out=do, phi=phi, stream=stream)
         else:
             la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=phi, stream=stream)
@@ -315,9 +324,13 @@ def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False):
     dbytes = 2 * st.numel() * 4 + (dq.numel() + dk_.numel() + dv_.numel() + do.numel()) * 4
     if norm:
         dbytes += 2 * zs[0].numel() * 4
-    return {"workload": DECODE["name"] + ("_normalised" if norm else ""), "us_per_step": us, "alg_bytes": dbytes,
+    if delta:
+        dbytes += 2 * lg.numel() * 4
+    name = DECODE["name"] + ("_normalised" if norm else "") + ("_gated_delta" if delta else "")
+    return {"workload": name, "us_per_step": us, "alg_bytes": dbytes,
             "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
-            "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "step_kernel", "launches": nrep,
+            "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "delta_kernel" if delta else "step_kernel",
+            "launches": nrep,
             "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
 
 
@@ -360,8 +373,10 @@ def main():
     if args.decode_only:
         res = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1))
         resn = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1), norm=True)
+        resd = _decode_leg(la, dev, stream, hbm_peak, rank, nrep=max(args.steps, 1), delta=True)
         if rank == 0:
-            print(json.dumps({"impl": "la", "decode": res, "decode_norm": resn, "peak_kind": peak_kind}), flush=True)
+            print(json.dumps({"impl": "la", "decode": res, "decode_norm": resn, "decode_gated_delta": resd,
+                              "peak_kind": peak_kind}), flush=True)
         if ws > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -548,6 +563,7 @@ def main():
     if not args.no_extra:
         extra["decode"] = _decode_leg(la, dev, stream, hbm_peak, rank)
         extra["decode_norm"] = _decode_leg(la, dev, stream, hbm_peak, rank, norm=True)
+        extra["decode_gated_delta"] = _decode_leg(la, dev, stream, hbm_peak, rank, delta=True)
 
     # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
     cpu = None

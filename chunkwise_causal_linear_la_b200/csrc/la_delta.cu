@@ -174,9 +174,149 @@ cudaError_t launch_dtype(const DeltaArgs &a, cudaStream_t stream) {
   }
 }
 
+// One token per sequence (decode): the state is read once and written once, so the
+// kernel is built for coalesced state traffic instead.  One CTA per (sequence,
+// head, 128 value columns), 512 threads: warp w holds rows [DK/16 w, DK/16 (w+1))
+// of S^T for the CTA's 128 columns, lane l the column quad 4l .. 4l + 3, loaded
+// and stored as float4 (a warp moves 512 contiguous bytes of one row at a time).
+// The two reductions over d_k (u = S kt and o = S q) go through shared memory.
+constexpr int kDecThreads = 512;
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kDecThreads) delta_decode_kernel(DeltaArgs a) {
+  constexpr int RW = DK / 16;  // rows of S^T per warp
+  __shared__ float kt[DK], qv[DK], part[16][kDeltaCols];
+  __shared__ float red[32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nsl = (a.dv + kDeltaCols - 1) / kDeltaCols;
+  const int64_t unit = blockIdx.x;
+  const int sl = (int)(unit % nsl);
+  const int h = (int)((unit / nsl) % a.H);
+  const int64_t n = unit / ((int64_t)nsl * a.H);
+  const int64_t b = n, t = 0;  // the sequence's one token
+  const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + t * a.q.st + h * a.q.sh;
+  const Tin *K = (const Tin *)a.k.data + b * a.k.sb + t * a.k.st + h * a.k.sh;
+  const Tin *V = (const Tin *)a.v.data + b * a.v.sb + t * a.v.st + h * a.v.sh;
+  const int64_t row = (b * a.T + t) * a.H + h;
+  const float alpha = expf(a.g[row]), beta = a.beta[row];
+  // unit key and query in shared memory
+  float ss = 0.f;
+  for (int c = tid; c < DK; c += kDecThreads) {
+    const float kv = to_f32<Tin>(K[c]);
+    kt[c] = kv;
+    qv[c] = to_f32<Tin>(Q[c]);
+    ss = fmaf(kv, kv, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (warp == 0) {
+    float x = lane < kDecThreads / 32 ? red[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) red[0] = 1.f / fmaxf(sqrtf(x), 1e-12f);
+  }
+  __syncthreads();
+  const float inv = red[0];
+  // this thread's state block: rows c0 .. c0 + RW - 1, columns r0 .. r0 + 3
+  const int c0 = warp * RW, r0 = sl * kDeltaCols + 4 * lane;
+  const bool active = r0 < a.dv;  // dv is a multiple of 4
+  const int64_t sbase = ((int64_t)n * a.H + h) * (int64_t)DK * a.dv;
+  float4 S[RW];
+#pragma unroll
+  for (int j = 0; j < RW; ++j)
+    S[j] = (a.init && active) ? *reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)(c0 + j) * a.dv + r0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  // u = S^T-contract kt over this thread's rows, then across the 16 warps
+  float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < RW; ++j) {
+    const float kc = kt[c0 + j] * inv;
+    u.x = fmaf(kc, S[j].x, u.x);
+    u.y = fmaf(kc, S[j].y, u.y);
+    u.z = fmaf(kc, S[j].z, u.z);
+    u.w = fmaf(kc, S[j].w, u.w);
+  }
+  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = u;
+  __syncthreads();
+  u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < 16; ++w) {
+    const float4 x = *reinterpret_cast<const float4 *>(&part[w][4 * lane]);
+    u.x += x.x;
+    u.y += x.y;
+    u.z += x.z;
+    u.w += x.w;
+  }
+  // S <- alpha (S - beta kt u^T) + beta kt v^T, i.e. S^T[c][r] += ... with coef_r = beta (v_r - alpha u_r)
+  float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) vv = make_float4(to_f32<Tin>(V[r0]), to_f32<Tin>(V[r0 + 1]), to_f32<Tin>(V[r0 + 2]), to_f32<Tin>(V[r0 + 3]));
+  const float4 coef = make_float4(beta * (vv.x - alpha * u.x), beta * (vv.y - alpha * u.y),
+                                  beta * (vv.z - alpha * u.z), beta * (vv.w - alpha * u.w));
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < RW; ++j) {
+    const float kc = kt[c0 + j] * inv, qc = qv[c0 + j];
+    S[j].x = fmaf(alpha, S[j].x, coef.x * kc);
+    S[j].y = fmaf(alpha, S[j].y, coef.y * kc);
+    S[j].z = fmaf(alpha, S[j].z, coef.z * kc);
+    S[j].w = fmaf(alpha, S[j].w, coef.w * kc);
+    o.x = fmaf(qc, S[j].x, o.x);
+    o.y = fmaf(qc, S[j].y, o.y);
+    o.z = fmaf(qc, S[j].z, o.z);
+    o.w = fmaf(qc, S[j].w, o.w);
+  }
+  if (a.final_state && active) {
+#pragma unroll
+    for (int j = 0; j < RW; ++j) *reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)(c0 + j) * a.dv + r0) = S[j];
+  }
+  __syncthreads();  // every warp has read the u partials
+  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = o;
+  __syncthreads();
+  if (warp == 0 && active) {
+    o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+      const float4 x = *reinterpret_cast<const float4 *>(&part[w][4 * lane]);
+      o.x += x.x;
+      o.y += x.y;
+      o.z += x.z;
+      o.w += x.w;
+    }
+    Tin *O = (Tin *)a.out + b * a.o_sb + t * a.o_st + h * a.o_sh + r0;
+    O[0] = from_f32<Tin>(o.x);
+    O[1] = from_f32<Tin>(o.y);
+    O[2] = from_f32<Tin>(o.z);
+    O[3] = from_f32<Tin>(o.w);
+  }
+}
+
+template <typename Tin>
+cudaError_t launch_decode(const DeltaArgs &a, cudaStream_t stream) {
+  const int64_t grid = a.n_seqs * a.H * ((a.dv + kDeltaCols - 1) / kDeltaCols);
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  switch (a.dk) {
+    case 64: delta_decode_kernel<Tin, 64><<<(unsigned)grid, kDecThreads, 0, stream>>>(a); break;
+    case 128: delta_decode_kernel<Tin, 128><<<(unsigned)grid, kDecThreads, 0, stream>>>(a); break;
+    case 256: delta_decode_kernel<Tin, 256><<<(unsigned)grid, kDecThreads, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// One token per sequence: a dense batch with T = 1 (the host cannot see the
+// lengths of a packed batch).
+bool decode_shape(const DeltaArgs &a) {
+  return !a.cu_seqlens && a.T == 1 && (a.dk == 64 || a.dk == 128 || a.dk == 256) && a.dv % 4 == 0 &&
+         ((uintptr_t)a.init) % 16 == 0 && ((uintptr_t)a.final_state) % 16 == 0;
+}
+
 }  // namespace
 
 cudaError_t launch_delta(const DeltaArgs &a, cudaStream_t stream) {
+  if (decode_shape(a))
+    return a.dtype == LA_F32 ? launch_decode<float>(a, stream) : launch_decode<__nv_bfloat16>(a, stream);
   return a.dtype == LA_F32 ? launch_dtype<float>(a, stream) : launch_dtype<__nv_bfloat16>(a, stream);
 }
 

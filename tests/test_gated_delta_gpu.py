@@ -75,6 +75,17 @@ def test_gated_delta_varlen_and_initial_state(la, oracle_mod):
     _check(la, oracle_mod, q, k, v, g, beta, cu=cu, init=init)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (256, 256), (128, 32), (64, 256)])
+def test_gated_delta_one_token_decode_kernel(la, oracle_mod, dtype, dk, dv):
+    """T = 1 takes the decode kernel (coalesced state, reductions across warps):
+    with and without an initial state, value slices narrower than 128 columns."""
+    q, k, v, g, beta = _inputs(5, 1, 3, dk, dv, dtype, dk + 7 * dv)
+    init = torch.randn((5, 3, dk, dv)) * 0.3
+    _check(la, oracle_mod, q, k, v, g, beta)
+    _check(la, oracle_mod, q, k, v, g, beta, init=init)
+
+
 def test_gated_delta_decode_in_place(la, oracle_mod):
     """Prefill T tokens, then one token at a time with the state updated in place,
     equals the oracle over all tokens."""
