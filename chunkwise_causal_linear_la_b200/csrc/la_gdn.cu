@@ -569,10 +569,11 @@ struct GdnCfg {
 // "prev" = the chunk starts from a state: c > 0 or an initial state):
 //   MMA:       [prev: FULL, SBFULL] MW -> WSFULL;  [UREADY] M4 -> UFULL;
 //              [OEMPTY[b], QREADY[s]] prev: M2 -> SBEMPTY;  [PFULL[b]] M3 -> OFULL[b], EMPTY[s];
-//              [XFORM(c+1)] M1 of chunk c + 1 -> AFULL[b ^ 1]  (M1 of chunk 0 before the loop).
+//              [FULL(c+1)] M1 of chunk c + 1 -> AFULL[b ^ 1], issued between MW and M4 when
+//              the tiles are in by then, else after M3 (M1 of chunk 0 before the loop).
 //   state:     [UFULL(c-1)] S^T <- e^{b_last} S^T + Us;  [prev: SBEMPTY(c-1)] Sb -> SBFULL;
 //              [XFORM, prev: WSFULL] U = Ut - WS in place -> UREADY.
-//   output:    [AFULL[b], XFORM] P -> PFULL[b];  Qd in place -> QREADY[s];
+//   output:    [AFULL[b], FULL] P -> PFULL[b];  Qd in place -> QREADY[s];
 //              [OFULL[b-1]] epilogue of chunk c-1 -> OEMPTY.
 //   transform: [FULL] Kd -> XFORM.
 template <int NS>
@@ -665,26 +666,46 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint64_t dkd0 = smem_desc_sw128(smem_u32(stage(0) + G::OFF_KD), kSlab, 1024); // MN-major
       const uint64_t dp0 = smem_desc_sw128(smem_u32(sm + G::OFF_P), 16, 1024);
       auto soff = [](int s) -> uint64_t { return (uint64_t)(s * (G::STAGE_BYTES >> 4)); };
-      int done = 0, m1_issued = 0;
+      int m1_issued = 0;
+      // The last commit: its arrival means every product issued before it has finished.
+      int last_bar = -1;
+      uint32_t last_par = 0;
+      auto commit = [&](int idx, uint32_t parity) {
+        umma_commit(bars + idx);
+        last_bar = idx;
+        last_par = parity;
+      };
       // M1 of chunk c: A[c & 1] = Q Kt^T
       auto issue_scores = [&](int c) -> bool {
         const int s = c % NS, k = c / NS, b = c & 1;
-        if (!wait_bar(sy, G::B_XFORM + s, k & 1, c)) return false;
+        if (!wait_bar(sy, G::B_FULL + s, k & 1, c)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_bf16(tbase + G::T_A + b * kC, dq0 + soff(s) + kmaj(kk), dk0 + soff(s) + kmaj(kk), ID_S, kk > 0);
-        umma_commit(bars + G::B_AFULL + b);
+        commit(G::B_AFULL + b, (c >> 1) & 1);
         m1_issued = c + 1;
         return true;
       };
-      // Per chunk: MW, M4, M2, M3, then the next chunk's M1, so that its scores and Qd
-      // are ready before its M2 (which gates the next Sb write).
+      constexpr bool kEarlyM2 = false;
+      // M2 of chunk c: O = Qd Sb
+      auto issue_m2 = [&](int c) {
+        const int s = c % NS, b = c & 1;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_bf16(tbase + G::T_O + b * kD, dq0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
+        commit(G::B_SBEMPTY, sbi(c) & 1);
+      };
+      // Per chunk: MW; then, while the state warps compute U, the next chunk's M1 as
+      // soon as its tiles have landed (the tensor pipe is idle there; issued later it
+      // would queue in front of the next MW); M4 at UREADY; M2, M3; the next M1 now if
+      // its tiles were late.
       const bool started = nchunks == 0 || issue_scores(0);
       for (int c = 0; c < nchunks && started; ++c) {
         const int s = c % NS, k = c / NS, b = c & 1;
         const uint32_t o_acc = tbase + G::T_O + b * kD;
-        bool ok = true;
+        bool ok = true, m2 = false;
         // MW: WS = W Sb
         if (prev(c)) {
           ok = wait_bar(sy, G::B_FULL + s, k & 1, c) && wait_bar(sy, G::B_SBFULL, sbi(c) & 1, c);
@@ -693,7 +714,20 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
             umma_bf16(tbase + G::T_U, dw0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
-          umma_commit(bars + G::B_WSFULL);
+          commit(G::B_WSFULL, sbi(c) & 1);
+        }
+        {
+          const int c1 = c + 1, s1 = c1 % NS, k1 = c1 / NS;
+          bool m1n = c1 >= nchunks;
+          const long long t0 = clock64();
+          while (!mbar_test(bars + G::B_UREADY, c & 1) && !*abort_flag && clock64() - t0 < kTimeoutCycles) {
+            if (!m1n && mbar_test(bars + G::B_FULL + s1, k1 & 1)) m1n = issue_scores(c1);
+            if (kEarlyM2 && prev(c) && !m2 && mbar_test(bars + G::B_OEMPTY + b, ((c >> 1) & 1) ^ 1) &&
+                mbar_test(bars + G::B_QREADY + s, k & 1)) {
+              issue_m2(c);
+              m2 = true;
+            }
+          }
         }
         // M4: Us = Kd^T U
         if (!wait_bar(sy, G::B_UREADY, c & 1, c)) break;
@@ -702,18 +736,12 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int kk = 0; kk < kC / 16; ++kk)
           umma_bf16(tbase + G::T_U, dkd0 + soff(s) + ((kk * 2048) >> 4), du0 + soff(s) + ((kk * 2048) >> 4), ID_U,
                     kk > 0);
-        umma_commit(bars + G::B_UFULL);
+        commit(G::B_UFULL, c & 1);
         // M2: O = Qd Sb.  Qd is waited for even without M2: the output warps write
         // it in place, so the stage must not be released before they are done.
         if (!wait_bar(sy, G::B_OEMPTY + b, ((c >> 1) & 1) ^ 1, c) || !wait_bar(sy, G::B_QREADY + s, k & 1, c))
           break;
-        if (prev(c)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk)
-            umma_bf16(o_acc, dq0 + soff(s) + kmaj(kk), dsb + ((kk * 2048) >> 4), ID_O, kk > 0);
-          umma_commit(bars + G::B_SBEMPTY);
-        }
+        if (prev(c) && !m2) issue_m2(c);
         // M3: O += P U
         if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
         tc_fence_after();
@@ -721,17 +749,12 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int kk = 0; kk < kC / 16; ++kk)
           umma_bf16(o_acc, dp0 + (uint64_t)(b * (kSlab >> 4)) + kmaj(kk), du0 + soff(s) + ((kk * 2048) >> 4),
                     ID_O, (prev(c) || kk > 0) ? 1u : 0u);
-        umma_commit(bars + G::B_OFULL + b);
-        umma_commit(bars + G::B_EMPTY + s);
-        done = c + 1;
-        if (c + 1 < nchunks && !issue_scores(c + 1)) break;
+        commit(G::B_OFULL + b, (c >> 1) & 1);
+        commit(G::B_EMPTY + s, k & 1);
+        if (m1_issued < c + 2 && c + 1 < nchunks && !issue_scores(c + 1)) break;
       }
       // the last commits arrive asynchronously: wait for them before tensor memory is freed
-      for (int c = max(0, done - NS); c < done; ++c) drain_bar(sy, G::B_EMPTY + c % NS, (c / NS) & 1);
-      if (m1_issued > done) {  // a score product issued ahead of an aborted chunk
-        const int c = m1_issued - 1;
-        drain_bar(sy, G::B_AFULL + (c & 1), (c >> 1) & 1);
-      }
+      if (last_bar >= 0) drain_bar(sy, last_bar, last_par);
     } else if (warp >= 2) {
       // ========================================================== transform
       // 64 threads; thread tt owns the 16-byte vectors tt + 64 m (m < 8) of both
@@ -897,7 +920,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int Cp = chunk_len(c);
       if (!wait_bar_warp(sy, G::B_AFULL + b, (c >> 1) & 1, c)) return false;
       tc_fence_after();
-      if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c) || !wait_bar_warp(sy, G::B_XFORM + s, k & 1, c)) return false;
+      if (!wait_bar_warp(sy, G::B_FULL + s, k & 1, c)) return false;
       const float *dt = dtab + s * G::DT_STRIDE;
       const float bi = dt[i];
       uint32_t r[32];
