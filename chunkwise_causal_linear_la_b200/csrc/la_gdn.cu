@@ -20,19 +20,21 @@
 //                    K K^T on the tensor cores; A from G and the key norms; T
 //                    by forward substitution on the CUDA cores (fp32); then
 //                    W = T diag(beta e^b) Kt and Ut = T diag(beta) V on the
-//                    tensor cores.  W, Ut and the unit keys Kt go to the
-//                    workspace as bf16 [B, T, H, 128], with the chunk's b_i.
+//                    tensor cores.  W and Ut go to the workspace as bf16
+//                    [B, T, H, 128], with the chunk's b_i and ln(1/|k_i|) - b_i.
 //   gdn_tc_kernel    one CTA per (sequence, head) walks its chunks in order with
 //                    the fp32 state S^T in registers, as the linear-attention
 //                    forward does.  Per chunk, five products:
 //                      MW  WS = W Sb                 (M=C, N=d_v, K=d_k)   Sb = bf16(S^T)
-//                      M1  A  = Q Kt^T               (M=C, N=C,   K=d_k)
+//                      M1  A  = Q K^T                (M=C, N=C,   K=d_k)   raw keys
 //                      M4  Us = Kd^T U               (M=d_k, N=d_v, K=C)   Kd = diag(e^{b_last-b}) Kt
 //                      M2  O  = Qd Sb                (M=C, N=d_v, K=d_k)   Qd = diag(e^b) Q
-//                      M3  O += P U                  (M=C, N=d_v, K=C)     P = tril(A) .* D
+//                      M3  O += P U                  (M=C, N=d_v, K=C)     P_ij = A_ij D_ij / |k_j|, j <= i
 //                    with U = Ut - WS between MW and M4 and S^T <- e^{b_last} S^T + Us after M4.
+//                    The key norms enter through the table c_j = ln(1/|k_j|) - b_j: P's
+//                    factor is e^{b_i + c_j}, Kd's row factor e^{b_last + c_j}.
 //   Warp roles of gdn_tc_kernel (384 threads, as in the forward):
-//     warp 0      TMA producer: Q, Kt, W, Ut chunk tiles and b_i into a two-deep ring.
+//     warp 0      TMA producer: Q, K, W, Ut chunk tiles and the chunk's table into a two-deep ring.
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
 //     warps 2-3   transform: the decayed unit keys Kd.
 //     warps 4-7   state: S^T update, the bf16 operand Sb, and U = Ut - WS in place.
@@ -91,8 +93,9 @@ struct PrepArgs {
   const float *g, *beta;      // [B * T][H]
   const int32_t *cu_seqlens;  // NULL: dense
   const int32_t *coff;        // packed: first chunk slot of each sequence, [n_seqs + 1]
-  __nv_bfloat16 *w, *ut, *kt;  // [B, T, H, 128] each: W, T diag(beta) V, unit keys
-  float *bt;                    // [chunk slot][H][C]: b_i of every chunk (rows past its end repeat b_last)
+  __nv_bfloat16 *w, *ut;  // [B, T, H, 128] each: W and T diag(beta) V
+  float *bt;               // [chunk slot][H][2][C]: b_i (rows past the chunk end repeat b_last), then
+                           // c_i = ln(1/|k_i|) - b_i (-inf there)
   int64_t T, n_seqs;
   int H;
 };
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
     bhi += __shfl_sync(0xffffffffu, blo, 31);
     bvec[lane] = blo;
     bvec[lane + 32] = bhi;
-    float *btab = a.bt + (slot * a.H + h) * kC;
+    float *btab = a.bt + (slot * a.H + h) * 2 * kC;
     btab[lane] = blo;
     btab[lane + 32] = bhi;
     betav[lane] = lane < Cp ? a.beta[row0 + (int64_t)lane * a.H] : 0.f;
@@ -373,9 +376,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
     umma_commit(bars + 1);
     issued = 1;
   }
-  // while it runs: 1/|k_i| and the unit keys to the workspace.  Rows past the chunk end
-  // must not reach the products below (they may hold anything): V rows become zero here,
-  // K rows once G is done.
+  // while it runs: 1/|k_i|.  Rows past the chunk end must not reach the products below
+  // (they may hold anything): V rows become zero here, K rows once G is done.
   if (ok) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -390,18 +392,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
       ss += __shfl_xor_sync(0xffffffffu, ss, 1);
       ss += __shfl_xor_sync(0xffffffffu, ss, 2);
       ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-      const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
-      if ((tid & 7) == 0) invn[r] = r < Cp ? inv : 0.f;
-      if (r < Cp) {  // unit keys, bf16: physical chunk tid & 7 of row r holds logical columns 8 ((tid & 7) ^ (r & 7))
-        __nv_bfloat16 *kd = a.kt + ((sp.bidx * a.T + t0 + r) * a.H + h) * (int64_t)kD + 8 * ((tid & 7) ^ (r & 7));
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          f0[u] *= inv;
-          f1[u] *= inv;
-        }
-        *reinterpret_cast<uint4 *>(kd) = pack8(f0);
-        *reinterpret_cast<uint4 *>(kd + 64) = pack8(f1);
-      }
+      if ((tid & 7) == 0) invn[r] = r < Cp ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
       if (r >= Cp) {
         *reinterpret_cast<uint4 *>(sm + P::OFF_V + off) = make_uint4(0u, 0u, 0u, 0u);
         *reinterpret_cast<uint4 *>(sm + P::OFF_V + kSlab + off) = make_uint4(0u, 0u, 0u, 0u);
@@ -409,6 +400,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
     }
   }
   __syncthreads();  // 1/|k| of every row
+  // for the chunk kernel: e^{b_i + c_j} = e^{b_i - b_j} / |k_j|, one exponential per factor
+  if (tid < kC) a.bt[(slot * a.H + h) * 2 * kC + kC + tid] = __logf(invn[tid]) - bvec[tid];
   ok = ok && wait_bar_warp(sy, 1, 0);
   tc_fence_after();
   if (ok) {
@@ -530,7 +523,7 @@ constexpr int kThreads = 384;
 struct GdnTcArgs {
   void *out;
   int64_t o_sb, o_st, o_sh;
-  const float *bt;            // [chunk slot][H][C]: b_i of every chunk, from the WY pass
+  const float *bt;            // [chunk slot][H][2][C]: b_i and ln(1/|k_i|) - b_i of every chunk, from the WY pass
   const int32_t *coff;        // packed: first chunk slot of each sequence (dense: n * nck)
   int64_t nck;                // chunks per sequence (dense)
   const float *init;          // NULL or [n_seqs, H, 128, 128] (S^T)
@@ -542,15 +535,15 @@ struct GdnTcArgs {
 
 template <int NS>
 struct GdnCfg {
-  // a stage: Q (then Qd), Kt, W, Ut (then U), Kd; [C x 128] bf16 tiles
+  // a stage: Q (then Qd), K, W, Ut (then U), Kd; [C x 128] bf16 tiles
   static constexpr int OFF_Q = 0, OFF_K = kTile, OFF_W = 2 * kTile, OFF_U = 3 * kTile, OFF_KD = 4 * kTile;
   static constexpr int STAGE_BYTES = 5 * kTile;
-  static constexpr int LOAD_BYTES = 4 * kTile + kC * 4;  // Q, Kt, W, Ut and the b table arrive by TMA
+  static constexpr int LOAD_BYTES = 4 * kTile + 2 * kC * 4;  // Q, K, W, Ut and the chunk's table arrive by TMA
   static constexpr int SB_SLAB = kD * 128;      // [d_k rows x 64 cols] bf16
   static constexpr int OFF_SB = NS * STAGE_BYTES;
   static constexpr int OFF_P = OFF_SB + 2 * SB_SLAB;
-  static constexpr int OFF_DT = OFF_P + 2 * kSlab;  // per stage: b_i (i < C); b_last = b_{C-1}
-  static constexpr int DT_STRIDE = kC;
+  static constexpr int OFF_DT = OFF_P + 2 * kSlab;  // per stage: b_i, then c_i (i < C); b_last = b_{C-1}
+  static constexpr int DT_STRIDE = 2 * kC;
   static constexpr int OFF_BAR = OFF_DT + NS * DT_STRIDE * 4;
   static constexpr int B_FULL = 0, B_EMPTY = NS, B_XFORM = 2 * NS, B_QREADY = 3 * NS, B_AFULL = 4 * NS,
                        B_PFULL = 4 * NS + 2, B_OFULL = 4 * NS + 4, B_OEMPTY = 4 * NS + 6, B_WSFULL = 4 * NS + 8,
@@ -639,7 +632,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int bi = (int)sq.bidx;
         uint8_t *st = stage(s);
         const int64_t slot = (a.coff ? (int64_t)a.coff[n] : n * a.nck) + c;
-        bulk_load(dtab + s * G::DT_STRIDE, a.bt + (slot * a.H + h) * kC, kC * 4, bars + G::B_FULL + s);
+        bulk_load(dtab + s * G::DT_STRIDE, a.bt + (slot * a.H + h) * G::DT_STRIDE, G::DT_STRIDE * 4,
+                  bars + G::B_FULL + s);
         for (int kb = 0; kb < 2; ++kb) {
           tma_load_4d(st + G::OFF_Q + kb * kSlab, &tm_q, bars + G::B_FULL + s, kb * 64, h, t0, bi);
           tma_load_4d(st + G::OFF_K + kb * kSlab, &tm_k, bars + G::B_FULL + s, kb * 64, h, t0, bi);
@@ -675,7 +669,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         last_bar = idx;
         last_par = parity;
       };
-      // M1 of chunk c: A[c & 1] = Q Kt^T
+      // M1 of chunk c: A[c & 1] = Q K^T (raw keys)
       auto issue_scores = [&](int c) -> bool {
         const int s = c % NS, k = c / NS, b = c & 1;
         if (!wait_bar(sy, G::B_FULL + s, k & 1, c)) return false;
@@ -759,7 +753,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // ========================================================== transform
       // 64 threads; thread tt owns the 16-byte vectors tt + 64 m (m < 8) of both
       // 64-column slabs of the key tile: row tt/8 + 8 m, physical chunk tt mod 8.
-      // Kd = diag(e^{b_last - b}) Kt, zero past the chunk end.
+      // Kd = diag(e^{b_last - b} / |k|) K (= diag(e^{b_last - b}) Kt), zero past the chunk end.
       const int tt = tid - 64;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
@@ -773,7 +767,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int m = 0; m < 8; ++m) {
           const int r = (tt >> 3) + 8 * m;
           const int off = (tt + 64 * m) * 16;
-          const float wd = r < Cp ? exp_fast(blast - dt[r]) : 0.f;
+          const float wd = r < Cp ? exp_fast(blast + dt[kC + r]) : 0.f;
 #pragma unroll
           for (int sl = 0; sl < 2; ++sl) {
             float f[8];
@@ -930,7 +924,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const int j = hf * 32 + e;
-        f[e] = (j <= i && i < Cp) ? __uint_as_float(r[e]) * exp_fast(bi - dt[j]) : 0.f;
+        f[e] = (j <= i && i < Cp) ? __uint_as_float(r[e]) * exp_fast(bi + dt[kC + j]) : 0.f;
       }
       uint8_t *prow = sm + G::OFF_P + b * kSlab;
 #pragma unroll
@@ -1013,8 +1007,8 @@ constexpr int kStages = 2;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace regions, in order: W, Ut and the unit keys (bf16 [B, T, H, 128]
-// each), the b tables ([chunk slot][H][C] fp32) and, for packed batches, the
+// Workspace regions, in order: W and Ut (bf16 [B, T, H, 128] each), the chunk
+// tables ([chunk slot][H][2][C] fp32: b_i, ln(1/|k_i|) - b_i) and, for packed batches, the
 // first chunk slot of each sequence.  Packed batches bound their slot count by
 // ceil(T / C) + n_seqs (each sequence adds at most one partial chunk).
 struct WsPlan {
@@ -1026,9 +1020,9 @@ WsPlan ws_plan(int64_t B, int64_t T, int64_t H, int64_t n_seqs, bool varlen) {
   p.nck = (T + kC - 1) / kC;
   p.slots = varlen ? p.nck + n_seqs : n_seqs * p.nck;
   p.wu = align256((size_t)(B * T * H) * kD * 2);
-  p.bt = align256((size_t)(p.slots * H) * kC * 4);
+  p.bt = align256((size_t)(p.slots * H) * 2 * kC * 4);
   p.coff = varlen ? align256((size_t)(n_seqs + 1) * 4) : 0;
-  p.total = 3 * p.wu + p.bt + p.coff;
+  p.total = 2 * p.wu + p.bt + p.coff;
   return p;
 }
 
@@ -1054,16 +1048,14 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   __nv_bfloat16 *w = reinterpret_cast<__nv_bfloat16 *>(ws);
   __nv_bfloat16 *ut = reinterpret_cast<__nv_bfloat16 *>(ws + plan.wu);
-  __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * plan.wu);
-  float *bt = reinterpret_cast<float *>(ws + 3 * plan.wu);
-  int32_t *coff = varlen ? reinterpret_cast<int32_t *>(ws + 3 * plan.wu + plan.bt) : nullptr;
+  float *bt = reinterpret_cast<float *>(ws + 2 * plan.wu);
+  int32_t *coff = varlen ? reinterpret_cast<int32_t *>(ws + 2 * plan.wu + plan.bt) : nullptr;
   const TensorView wv{w, a.T * a.H * kD, (int64_t)a.H * kD, kD};
   const TensorView uv{ut, a.T * a.H * kD, (int64_t)a.H * kD, kD};
-  const TensorView kv{kt, a.T * a.H * kD, (int64_t)a.H * kD, kD};
-  CUtensorMap mq, mk, mv, mw, mu, mkt;
+  CUtensorMap mq, mk, mv, mw, mu;
   if (!make_map(&mq, a.q, B, a.T, a.H, kD, kC) || !make_map(&mk, a.k, B, a.T, a.H, kD, kC) ||
       !make_map(&mv, a.v, B, a.T, a.H, kD, kC) || !make_map(&mw, wv, B, a.T, a.H, kD, kC) ||
-      !make_map(&mu, uv, B, a.T, a.H, kD, kC) || !make_map(&mkt, kv, B, a.T, a.H, kD, kC)) {
+      !make_map(&mu, uv, B, a.T, a.H, kD, kC)) {
     if (why) *why = "cuTensorMapEncodeTiled rejected a tensor";
     return cudaErrorInvalidValue;
   }
@@ -1081,7 +1073,6 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
     p.coff = coff;
     p.w = w;
     p.ut = ut;
-    p.kt = kt;
     p.bt = bt;
     p.T = a.T;
     p.n_seqs = a.n_seqs;
@@ -1109,7 +1100,7 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   auto kern = gdn_tc_kernel<kStages>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  kern<<<(unsigned)(a.n_seqs * a.H), kThreads, G::SMEM_BYTES, stream>>>(mq, mkt, mw, mu, t);
+  kern<<<(unsigned)(a.n_seqs * a.H), kThreads, G::SMEM_BYTES, stream>>>(mq, mk, mw, mu, t);
   return cudaGetLastError();
 }
 

@@ -211,9 +211,9 @@ LA_API la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, cons
  * and outputs and the next chunk's state follow from U with matrix products.
  * Tensor cores (tcgen05) for bf16 with d_k = d_v = 128 and 16-byte aligned
  * initial_state / final_state: a parallel pass over all chunks writes
- * W = T diag(beta e^b) Kt, T diag(beta) V and the unit keys Kt (bf16) and the
- * chunk's b_i (fp32) to the workspace, then one CTA per (sequence, head) walks
- * its chunks with the fp32 state.  Every other
+ * W = T diag(beta e^b) Kt and T diag(beta) V (bf16) and the chunk's b_i and
+ * ln(1/|k_i|) - b_i (fp32) to the workspace, then one CTA per (sequence, head)
+ * walks its chunks with the fp32 state.  Every other
  * case, and flags = LA_FLAG_SIMT, runs la_fwd_gated_delta's kernel (no
  * workspace needed).
  *   flags       LA_FLAG_NONE or LA_FLAG_SIMT.
@@ -232,8 +232,8 @@ LA_API la_status la_fwd_gated_delta_chunk(const la_tensor *q, const la_tensor *k
  * Bytes of workspace la_fwd_gated_delta_chunk needs: B, T, H, d_k, d_v,
  * n_seqs, has_cu_seqlens, dtype and flags as they will be passed.  0 when the
  * call needs none (the token-by-token kernel); (size_t)-1 for arguments the
- * call would reject.  Host-only.  On the tensor cores: 3 B T H 128 bf16 values
- * (W, T diag(beta) V, unit keys), 64 floats per (chunk, head) (b_i; a packed
+ * call would reject.  Host-only.  On the tensor cores: 2 B T H 128 bf16 values
+ * (W, T diag(beta) V), 128 floats per (chunk, head) (b_i, ln(1/|k_i|) - b_i; a packed
  * batch counts ceil(T / 64) + n_seqs chunks) and, for a packed batch,
  * n_seqs + 1 chunk offsets, each region rounded up to 256 bytes.
  */
