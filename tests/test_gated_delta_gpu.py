@@ -145,6 +145,18 @@ def test_gated_delta_chunk_lengths_and_gates(la, oracle_mod, T, alo, blo):
     _check_chunk(la, oracle_mod, q, k, v, g, beta)
 
 
+def test_gated_delta_chunk_zero_and_tiny_keys(la, oracle_mod):
+    """Keys that are exactly zero or far below the 1e-12 norm floor: the chunk kernel
+    reads the raw keys and takes 1/max(|k|, 1e-12) through the decay exponents, so
+    such rows must give what the unit-key definition gives (a zero or tiny kt)."""
+    q, k, v, g, beta = _inputs(2, 200, 3, 128, 128, torch.bfloat16, 31)
+    k[0, 5] = 0                       # every head of token 5
+    k[1, 64:70, 1] = 0                # the start of the second chunk, one head
+    k[0, 100:140, 2] = (k[0, 100:140, 2].float() * 1e-20).to(torch.bfloat16)  # |k| ~ 1e-20
+    k[1, 199] = 0                     # the last token of a partial chunk
+    _check_chunk(la, oracle_mod, q, k, v, g, beta)
+
+
 def test_gated_delta_chunk_many_heads(la, oracle_mod):
     """More (sequence, head) units than SMs in the sequential pass, and thousands of
     chunk CTAs in the WY pass; only a few slices are compared in full."""
