@@ -198,6 +198,16 @@ __global__ void __launch_bounds__(kDecThreads) delta_decode_kernel(DeltaArgs a) 
   const Tin *V = (const Tin *)a.v.data + b * a.v.sb + t * a.v.st + h * a.v.sh;
   const int64_t row = (b * a.T + t) * a.H + h;
   const float alpha = expf(a.g[row]), beta = a.beta[row];
+  // this thread's state block: rows c0 .. c0 + RW - 1, columns r0 .. r0 + 3, read once
+  // (streaming loads, issued first so that they overlap the key norm below)
+  const int c0 = warp * RW, r0 = sl * kDeltaCols + 4 * lane;
+  const bool active = r0 < a.dv;  // dv is a multiple of 4
+  const int64_t sbase = ((int64_t)n * a.H + h) * (int64_t)DK * a.dv;
+  float4 S[RW];
+#pragma unroll
+  for (int j = 0; j < RW; ++j)
+    S[j] = (a.init && active) ? __ldcs(reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)(c0 + j) * a.dv + r0))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
   // unit key and query in shared memory
   float ss = 0.f;
   for (int c = tid; c < DK; c += kDecThreads) {
@@ -218,15 +228,6 @@ __global__ void __launch_bounds__(kDecThreads) delta_decode_kernel(DeltaArgs a) 
   }
   __syncthreads();
   const float inv = red[0];
-  // this thread's state block: rows c0 .. c0 + RW - 1, columns r0 .. r0 + 3
-  const int c0 = warp * RW, r0 = sl * kDeltaCols + 4 * lane;
-  const bool active = r0 < a.dv;  // dv is a multiple of 4
-  const int64_t sbase = ((int64_t)n * a.H + h) * (int64_t)DK * a.dv;
-  float4 S[RW];
-#pragma unroll
-  for (int j = 0; j < RW; ++j)
-    S[j] = (a.init && active) ? *reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)(c0 + j) * a.dv + r0)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
   // u = S^T-contract kt over this thread's rows, then across the 16 warps
   float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(kDecThreads) delta_decode_kernel(DeltaArgs a) 
   }
   if (a.final_state && active) {
 #pragma unroll
-    for (int j = 0; j < RW; ++j) *reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)(c0 + j) * a.dv + r0) = S[j];
+    for (int j = 0; j < RW; ++j) __stcs(reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)(c0 + j) * a.dv + r0), S[j]);
   }
   __syncthreads();  // every warp has read the u partials
   *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = o;
