@@ -48,12 +48,21 @@ step_kernel(StepArgs a) {
   const Tin *Q = (const Tin *)a.q.data + n * a.q.sb + h * a.q.sh;
   const Tin *K = (const Tin *)a.k.data + n * a.k.sb + h * a.k.sh;
   const Tin *V = (const Tin *)a.v.data + n * a.v.sb + h * a.v.sh;
+  const int cg = tid % ncg, rg = tid / ncg;
+  float4 *S = (float4 *)(a.state + unit * (int64_t)dk * dv) + cg;
+  float4 s[kRowsUnroll];  // this thread's first state rows: in flight while q, k, v arrive
+  if (rg < nrg) {
+#pragma unroll
+    for (int u = 0; u < kRowsUnroll; ++u) {
+      const int c = rg + u * nrg;
+      if (c < dk) s[u] = __ldcs(S + (int64_t)c * ncg);
+    }
+  }
   for (int c = tid; c < dk; c += kStepThreads) {
     qh[c] = feature_map(to_f32<Tin>(Q[c]), a.phi);
     kh[c] = feature_map(to_f32<Tin>(K[c]), a.phi);
   }
   const float g = a.g ? expf(a.g[unit]) : a.gamma[h];  // data-dependent decay: exp(g[n][h])
-  const int cg = tid % ncg, rg = tid / ncg;
   float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
   if (rg < nrg) {
     vr.x = to_f32<Tin>(V[4 * cg + 0]);
@@ -78,13 +87,13 @@ step_kernel(StepArgs a) {
 
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   if (rg < nrg) {
-    float4 *S = (float4 *)(a.state + unit * (int64_t)dk * dv) + cg;
     for (int c0 = rg; c0 < dk; c0 += nrg * kRowsUnroll) {
-      float4 s[kRowsUnroll];
+      if (c0 != rg) {
 #pragma unroll
-      for (int u = 0; u < kRowsUnroll; ++u) {
-        const int c = c0 + u * nrg;
-        if (c < dk) s[u] = __ldcs(S + (int64_t)c * ncg);
+        for (int u = 0; u < kRowsUnroll; ++u) {
+          const int c = c0 + u * nrg;
+          if (c < dk) s[u] = __ldcs(S + (int64_t)c * ncg);
+        }
       }
 #pragma unroll
       for (int u = 0; u < kRowsUnroll; ++u) {
