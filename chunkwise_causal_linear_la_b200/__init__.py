@@ -16,6 +16,7 @@ this package is its Python binding:
 from .binding import (  # noqa: F401
     LA_FLAG_NONE,
     LA_FLAG_SIMT,
+    LA_FLAG_TEST_WAIT_TIMEOUT,
     LaError,
     device_error,
     la_bwd_chunk,

@@ -21,6 +21,7 @@ LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE, LA_ERR_CUDA = r
 LA_PHI_IDENTITY, LA_PHI_ELU1 = 0, 1
 LA_F32, LA_BF16 = 0, 1
 LA_FLAG_NONE, LA_FLAG_SIMT = 0, 1
+LA_FLAG_TEST_WAIT_TIMEOUT = 0x100  # tests of the failure path only (see include/la_b200.h)
 
 _PHI = {"identity": LA_PHI_IDENTITY, "elu1": LA_PHI_ELU1, LA_PHI_IDENTITY: LA_PHI_IDENTITY,
         LA_PHI_ELU1: LA_PHI_ELU1}

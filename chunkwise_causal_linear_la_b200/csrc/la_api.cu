@@ -430,7 +430,9 @@ la_status la_fwd_gated_delta_chunk(const la_tensor *q, const la_tensor *k, const
   DeltaArgs a;
   la_status s = delta_setup(q, k, v, g, beta, cu_seqlens, n_seqs, initial_state, out, final_state, a);
   if (s != LA_OK) return s;
-  if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(LA_FLAG_SIMT | LA_FLAG_TEST_WAIT_TIMEOUT))
+    return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  a.test_wait_timeout = (flags & LA_FLAG_TEST_WAIT_TIMEOUT) != 0;
   if (n_seqs == 0) return ok();
   cudaError_t err;
   const bool states16 = ((uintptr_t)initial_state) % 16 == 0 && ((uintptr_t)final_state) % 16 == 0;
@@ -456,7 +458,7 @@ size_t la_fwd_gated_delta_workspace_size(int64_t B, int64_t T, int64_t H, int64_
                                          int64_t n_seqs, int32_t has_cu_seqlens, int32_t dtype, int32_t flags) {
   if (B < 0 || T < 0 || H <= 0 || n_seqs < 0 || !head_dim_ok(d_k) || !head_dim_ok(d_v)) return (size_t)-1;
   if (dtype != LA_F32 && dtype != LA_BF16) return (size_t)-1;
-  if (flags & ~LA_FLAG_SIMT) return (size_t)-1;
+  if (flags & ~(LA_FLAG_SIMT | LA_FLAG_TEST_WAIT_TIMEOUT)) return (size_t)-1;
   if (dtype == LA_F32 || (flags & LA_FLAG_SIMT)) return 0;
   return gdn_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0);
 }

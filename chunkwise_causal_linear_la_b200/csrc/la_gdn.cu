@@ -98,6 +98,7 @@ struct PrepArgs {
                            // c_i = ln(1/|k_i|) - b_i (-inf there)
   int64_t T, n_seqs;
   int H;
+  int skip_load;  // testing the failure path: no tile load, so the first wait runs out
 };
 
 struct PrepCfg {
@@ -324,10 +325,12 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant_
     mbar_init(bars + 1, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    mbar_arrive_expect_tx(bars + 0, 2 * kTile);
-    for (int kb = 0; kb < 2; ++kb) {
-      tma_load_4d(sm + P::OFF_K + kb * kSlab, &tm_k, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
-      tma_load_4d(sm + P::OFF_V + kb * kSlab, &tm_v, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
+    if (!a.skip_load) {
+      mbar_arrive_expect_tx(bars + 0, 2 * kTile);
+      for (int kb = 0; kb < 2; ++kb) {
+        tma_load_4d(sm + P::OFF_K + kb * kSlab, &tm_k, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
+        tma_load_4d(sm + P::OFF_V + kb * kSlab, &tm_v, bars + 0, kb * 64, h, (int)t0, (int)sp.bidx);
+      }
     }
   }
   // Give up the allocation permit at once: an SM takes no further CTA while one
@@ -1077,6 +1080,7 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
     p.T = a.T;
     p.n_seqs = a.n_seqs;
     p.H = a.H;
+    p.skip_load = a.test_wait_timeout ? 1 : 0;
     err = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepCfg::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     gdn_prep_kernel<<<(unsigned)(plan.slots * a.H), 128, PrepCfg::SMEM_BYTES, stream>>>(mk, mv, p);

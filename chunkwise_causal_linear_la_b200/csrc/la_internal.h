@@ -70,6 +70,7 @@ struct DeltaArgs {
   const int32_t *cu_seqlens;  // NULL for dense batches
   int64_t T, n_seqs;
   int H, dk, dv, dtype;
+  bool test_wait_timeout = false;  // LA_FLAG_TEST_WAIT_TIMEOUT (chunked path)
 };
 
 // Sets the calling thread's la_last_error() message and returns `status`.

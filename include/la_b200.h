@@ -66,6 +66,13 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 /* Run the CUDA-core (SIMT, fp32 arithmetic) chunk kernel even where the
  * tensor-core kernel applies.  Both are CUDA kernels; there is no CPU path. */
 #define LA_FLAG_SIMT 1
+/* Testing the failure path, la_fwd_gated_delta_chunk on the tensor cores only:
+ * the WY pass issues no tile load, so its first wait runs out (bounded: about
+ * two seconds per CTA, plus as long again to drain), its CTAs raise their
+ * abort flags, free their tensor memory and return; la_device_error then
+ * reports the timeout (flags bit 0) and where it happened.  The call's
+ * outputs are undefined; the CUDA context stays usable. */
+#define LA_FLAG_TEST_WAIT_TIMEOUT 0x100
 
 /*
  * A strided 4-D activation tensor [B, T, H, D] in device memory.
@@ -216,7 +223,7 @@ LA_API la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, cons
  * walks its chunks with the fp32 state.  Every other
  * case, and flags = LA_FLAG_SIMT, runs la_fwd_gated_delta's kernel (no
  * workspace needed).
- *   flags       LA_FLAG_NONE or LA_FLAG_SIMT.
+ *   flags       LA_FLAG_NONE or LA_FLAG_SIMT; LA_FLAG_TEST_WAIT_TIMEOUT (tests only).
  *   workspace   device memory of la_fwd_gated_delta_workspace_size bytes,
  *               256-byte aligned, owned by the caller; its contents are
  *               scratch (nothing needs to be zero; nothing is kept).

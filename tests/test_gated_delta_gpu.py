@@ -157,6 +157,26 @@ def test_gated_delta_chunk_zero_and_tiny_keys(la, oracle_mod):
     _check_chunk(la, oracle_mod, q, k, v, g, beta)
 
 
+def test_gated_delta_chunk_wait_timeout_is_reported(la, oracle_mod):
+    """Failure detection without a GPU fault: with LA_FLAG_TEST_WAIT_TIMEOUT the WY pass
+    issues no tile load, so its first wait (bounded, about two seconds) runs out; the
+    CTA raises its abort flag, drains (again bounded), frees its tensor memory and
+    returns, and la_device_error reports the timeout and the barrier.  One CTA (one
+    chunk, one head) keeps the test short.  The next call on the same context is
+    correct again."""
+    q, k, v, g, beta = _inputs(1, 64, 1, 128, 128, torch.bfloat16, 5)
+    dev = torch.device("cuda")
+    assert la.device_error(reset=True) == (0, 0)
+    la.la_fwd_gated_delta_chunk(q.to(dev), k.to(dev), v.to(dev), g.to(dev), beta.to(dev),
+                                flags=la.LA_FLAG_TEST_WAIT_TIMEOUT)
+    torch.cuda.synchronize()
+    flags, where = la.device_error(reset=True)
+    assert flags & 1, (flags, hex(where))          # a wait ran out
+    assert where == 0x80000000, hex(where)         # chunk 0, barrier 0: the tile load
+    assert la.device_error(reset=True) == (0, 0)
+    _check_chunk(la, oracle_mod, q, k, v, g, beta)
+
+
 def test_gated_delta_chunk_many_heads(la, oracle_mod):
     """More (sequence, head) units than SMs in the sequential pass, and thousands of
     chunk CTAs in the WY pass; only a few slices are compared in full."""

@@ -87,6 +87,7 @@ def test_gated_delta_workspace_size(lib):
     assert ws(8, 4096, 0, 128, 128, 8, 0, 1, 0) == bad   # H = 0
     assert ws(8, 4096, 16, 128, 128, 8, 0, 2, 0) == bad  # dtype
     assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 4) == bad  # flags
+    assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 0x100) == 2 * wu + (8 * 64) * 16 * 512  # the test flag
 
 
 def test_workspace_size_segment_plan(lib):
