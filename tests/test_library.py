@@ -161,6 +161,8 @@ def test_gated_delta_chunk_arguments_validated_on_host(lib):
     assert call(beta=0x3002) == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()
     assert call(n=2) == b.LA_ERR_INVALID_ARG
     assert call(flags=2) == b.LA_ERR_INVALID_ARG and b"flags" in lib.la_last_error()
+    assert call(flags=0x200) == b.LA_ERR_INVALID_ARG and b"flags" in lib.la_last_error()
+    assert call(flags=b.LA_FLAG_TEST_WAIT_TIMEOUT, ws_bytes=need - 1) == b.LA_ERR_WORKSPACE  # flag accepted
     assert call(ws_bytes=need - 1) == b.LA_ERR_WORKSPACE
     assert call(ws=None) == b.LA_ERR_WORKSPACE
     assert call(ws=0x100010) == b.LA_ERR_INVALID_ARG and b"256" in lib.la_last_error()
