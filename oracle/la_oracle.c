@@ -32,6 +32,8 @@
  *                        place, o_t = S_t phi(q_t) / (z_t^T phi(q_t)).
  *   oracle_backward   -- dq, dk, dv of sum_t dout_t . o_t for the unnormalised
  *                        recurrence: the adjoint of the definition.
+ *   oracle_backward_gated -- the same for the per-token decay, plus the
+ *                        gradient of the log decays g.
  *   oracle_norm_gate  -- RMSNorm over d_v times a Swish gate, per (token, head).
  *   oracle_gated_delta -- the gated delta rule, token by token.
  *   oracle_gated_delta_chunked -- the same rule regrouped into chunks (the
@@ -586,6 +588,94 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
       }
     }
     free(S);
+    free(qh);
+    free(kh);
+  }
+  return 0;
+}
+
+/*
+ * Gradients of L = sum_t dout_t . o_t for the unnormalised recurrence with a
+ * per-token decay (oracle_recurrent_gated): the adjoint of that definition,
+ * with respect to q, k, v and the log decays g.  With alpha_t = exp(g_t):
+ *   forward   S_t = alpha_t S_{t-1} + v_t kh_t^T,  dqh_t = S_t^T dout_t;
+ *   backward  D_t = dout_t qh_t^T + alpha_{t+1} D_{t+1}   (D after the last token: 0),
+ *             dv_t = D_t kh_t,  dkh_t = D_t^T v_t,
+ *             dg_t = alpha_t <D_t, S_{t-1}>   (the Frobenius product; S_{-1} = 0),
+ * then dq = dqh phi'(q), dk = dkh phi'(k).  Every state S_{t-1} is kept for
+ * the dg step, so this is for test sizes (len * d_v * d_k doubles per task).
+ *   g, dg  [B, T, H] double.  Other arguments as for oracle_backward.
+ */
+int oracle_backward_gated(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                          int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                          const double *g, const int32_t *cu_seqlens, int64_t n_seqs, int phi,
+                          double *dq, double *dkk, double *dvv, double *dg, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (!g || !dg) return -10;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const size_t sz = (size_t)(dv * dk);
+    double *prev = (double *)calloc((size_t)(len > 0 ? len : 1) * sz, sizeof(double));  /* S_{t-1}, every t */
+    double *S = (double *)calloc(sz, sizeof(double));  /* S[r][c] */
+    double *D = (double *)calloc(sz, sizeof(double));
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    /* forward in time */
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;
+      const double a = exp(g[row * H + h]);
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      memcpy(prev + (size_t)t * sz, S, sz * sizeof(double));
+      for (int64_t c = 0; c < dk; ++c) kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, vb + r);
+        for (int64_t c = 0; c < dk; ++c) S[r * dk + c] = a * S[r * dk + c] + vr * kh[c];
+      }
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * orc_load(dout, dtype, vb + r);
+        dq[qk + c] = acc * orc_dphi(orc_load(q, dtype, qk + c), phi);
+      }
+    }
+    /* backward in time */
+    double a_next = 0.0;  /* alpha_{t+1}; D is zero before the last token anyway */
+    for (int64_t t = len - 1; t >= 0; --t) {
+      const int64_t row = start + t;
+      const double a = exp(g[row * H + h]);
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        const double d = orc_load(dout, dtype, vb + r);
+        for (int64_t c = 0; c < dk; ++c) D[r * dk + c] = a_next * D[r * dk + c] + d * qh[c];
+      }
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < dv; ++r) acc += D[r * dk + c] * orc_load(v, dtype, vb + r);
+        dkk[qk + c] = acc * orc_dphi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += D[r * dk + c] * kh[c];
+        dvv[vb + r] = acc;
+      }
+      const double *P = prev + (size_t)t * sz;
+      double inner = 0.0;
+      for (size_t e = 0; e < sz; ++e) inner += D[e] * P[e];
+      dg[row * H + h] = a * inner;
+      a_next = a;
+    }
+    free(prev);
+    free(S);
+    free(D);
     free(qh);
     free(kh);
   }

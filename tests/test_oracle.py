@@ -393,6 +393,99 @@ def test_backward_varlen_equals_independent_runs(oracle_mod):
         assert np.array_equal(gq[:, s_:e], a) and np.array_equal(gk[:, s_:e], b) and np.array_equal(gv[:, s_:e], c)
 
 
+def _rand_log_decay(B, T, H, seed, lo=0.3):
+    return np.log(np.random.default_rng(seed).uniform(lo, 1.0, (B, T, H)))
+
+
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+def test_backward_gated_matches_finite_differences(oracle_mod, phi):
+    """Central differences of L = sum(dout * o) through the per-token-decay forward
+    oracle, for q, k, v and the log decays g."""
+    B, T, H, dk, dv = 1, 6, 2, 3, 2
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=71)
+    dout = np.random.default_rng(72).standard_normal((B, T, H, dv))
+    g = _rand_log_decay(B, T, H, 73)
+    gq, gk, gv, gg = oracle_mod.backward_gated(q, k, v, dout, g, phi=phi)
+
+    def loss(q_, k_, v_, g_):
+        o, _, _ = oracle_mod.recurrent_gated(q_, k_, v_, g_, phi=phi)
+        return float(np.sum(o * dout))
+
+    eps = 1e-6
+    for x, gref, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2), (g, gg, 3)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v, g]
+            args_m = [q, k, v, g]
+            args_p[which], args_m[which] = xp, xm
+            fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert rel(gref, fd) < 1e-7, which
+
+
+def test_backward_gated_matches_autograd_of_masked_form(oracle_mod):
+    """torch autograd (float64) through O = ((phi(Q) phi(K)^T) .* M) V with the
+    cumulative-decay mask M_ij = exp(b_i - b_j) (i >= j), b = cumsum(g): a
+    different formula for the same outputs, including dg."""
+    T, H, dk, dv = 25, 2, 4, 3
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=74)
+    dout = np.random.default_rng(75).standard_normal((1, T, H, dv))
+    g = _rand_log_decay(1, T, H, 76)
+    for phi in ("identity", "elu1"):
+        gq, gk, gv, gg = oracle_mod.backward_gated(q, k, v, dout, g, phi=phi)
+        for h in range(H):
+            qt, kt, vt, lg = (torch.tensor(x[0, :, h], dtype=torch.float64, requires_grad=True) for x in (q, k, v, g))
+            f = (lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))) if phi == "elu1" \
+                else (lambda x: x)
+            b = torch.cumsum(lg, 0)
+            i = torch.arange(T)[:, None]
+            j = torch.arange(T)[None, :]
+            M = torch.where(i >= j, torch.exp(b[:, None] - b[None, :]), torch.zeros((), dtype=torch.float64))
+            O = ((f(qt) @ f(kt).T) * M) @ vt
+            (O * torch.tensor(dout[0, :, h])).sum().backward()
+            assert rel(gq[0, :, h], qt.grad.numpy()) < 1e-11
+            assert rel(gk[0, :, h], kt.grad.numpy()) < 1e-11
+            assert rel(gv[0, :, h], vt.grad.numpy()) < 1e-11
+            assert rel(gg[0, :, h], lg.grad.numpy()) < 1e-11
+
+
+def test_backward_gated_reduces_to_per_head_decay_and_dg_identity(oracle_mod):
+    """g constant over time per head: dq, dk, dv equal the per-head-decay backward
+    with gamma = exp(g).  And for any g (identity feature map), dg_t equals the
+    reverse cumulative sum over s >= t of q_s . dq_s - k_s . dk_s, which follows
+    from o_s = sum_{j<=s} exp(b_s - b_j) (q_s . k_j) v_j with b the prefix sum of g."""
+    B, T, H, dk, dv = 2, 40, 3, 5, 4
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=77)
+    dout = np.random.default_rng(78).standard_normal((B, T, H, dv))
+    lg = np.log(np.array([0.6, 0.95, 1.0]))
+    g = np.broadcast_to(lg, (B, T, H)).copy()
+    gq, gk, gv, _ = oracle_mod.backward_gated(q, k, v, dout, g, phi="elu1")
+    rq, rk, rv = oracle_mod.backward(q, k, v, dout, np.exp(lg), phi="elu1")
+    assert rel(gq, rq) < 1e-12 and rel(gk, rk) < 1e-12 and rel(gv, rv) < 1e-12
+    g = _rand_log_decay(B, T, H, 79)
+    gq, gk, _, gg = oracle_mod.backward_gated(q, k, v, dout, g, phi="identity")
+    per_t = np.sum(q * gq, axis=-1) - np.sum(k * gk, axis=-1)  # [B, T, H]
+    want = np.flip(np.cumsum(np.flip(per_t, axis=1), axis=1), axis=1)
+    assert rel(gg, want) < 1e-11
+
+
+def test_backward_gated_varlen_equals_independent_runs(oracle_mod):
+    lengths = [6, 0, 13, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 2, 4, 3
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=80)
+    dout = np.random.default_rng(81).standard_normal((1, Tt, H, dv))
+    g = _rand_log_decay(1, Tt, H, 82)
+    full = oracle_mod.backward_gated(q, k, v, dout, g, cu_seqlens=cu, phi="elu1")
+    for n in range(len(lengths)):
+        s_, e = cu[n], cu[n + 1]
+        part = oracle_mod.backward_gated(q[:, s_:e], k[:, s_:e], v[:, s_:e], dout[:, s_:e], g[:, s_:e], phi="elu1")
+        for a, b in zip(full, part):
+            assert np.array_equal(a[:, s_:e], b)
+
+
 # ---------------------------------------------------------------- output norm and gate
 def test_norm_gate_closed_forms(oracle_mod):
     """Constant rows: o = c * 1 gives y = sign(c) * w * swish(g) (up to eps); scaling

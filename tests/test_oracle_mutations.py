@@ -87,3 +87,64 @@ def test_mutant_is_caught(tmp_path, name):
     old, new = MUTATIONS[name]
     lib = _build(tmp_path, name, old, new)
     assert not _pins_pass(lib), name
+
+
+# ---------------------------------------------------------------- per-token-decay backward
+GATED_BWD_MUTATIONS = {
+    "dg without the decay's own factor": (
+        "dg[row * H + h] = a * inner;", "dg[row * H + h] = inner;"),
+    "reverse carry decayed by the current token's factor": (
+        "D[r * dk + c] = a_next * D[r * dk + c] + d * qh[c];", "D[r * dk + c] = a * D[r * dk + c] + d * qh[c];"),
+    "dg paired with the state after the token": (
+        "const double *P = prev + (size_t)t * sz;",
+        "const double *P = t + 1 < len ? prev + (size_t)(t + 1) * sz : S;"),
+}
+
+
+def _gated_bwd(lib, q, k, v, dout, g):
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.oracle_backward_gated.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, vp, vp, i64, i32,
+                                          vp, vp, vp, vp, i32]
+    lib.oracle_backward_gated.restype = i32
+    q, k, v, dout, g = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout, g))
+    outs = [np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape), np.zeros((B, T, H))]
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = lib.oracle_backward_gated(p(q), p(k), p(v), p(dout), 2, B, T, H, dk, dv, p(g), None, B, 0,
+                                   *(p(o) for o in outs), 1)
+    assert rc == 0
+    return outs
+
+
+def _gated_bwd_pin_passes(lib):
+    """The autograd pin of test_oracle.py: torch float64 gradients through the
+    masked form with the cumulative-decay mask."""
+    import torch
+
+    T, dk, dv = 12, 3, 2
+    q, k, v = rand_qkv(1, T, 1, dk, dv, seed=90)
+    rng = np.random.default_rng(91)
+    dout = rng.standard_normal((1, T, 1, dv))
+    g = np.log(rng.uniform(0.3, 1.0, (1, T, 1)))
+    got = _gated_bwd(lib, q, k, v, dout, g)
+    qt, kt, vt, lg = (torch.tensor(x[0, :, 0], dtype=torch.float64, requires_grad=True) for x in (q, k, v, g))
+    b = torch.cumsum(lg, 0)
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    M = torch.where(i >= j, torch.exp(b[:, None] - b[None, :]), torch.zeros((), dtype=torch.float64))
+    (((qt @ kt.T) * M) @ vt * torch.tensor(dout[0, :, 0])).sum().backward()
+    want = [qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy(), lg.grad.numpy()]
+    return all(rel(a[0, :, 0], w) < 1e-11 for a, w in zip(got, want))
+
+
+def test_unmutated_copy_passes_gated_backward_pin(tmp_path):
+    lib = _build(tmp_path, "none", "#define ROWS_PER_TASK 8", "#define ROWS_PER_TASK 8")
+    assert _gated_bwd_pin_passes(lib)
+
+
+@pytest.mark.parametrize("name", sorted(GATED_BWD_MUTATIONS))
+def test_gated_backward_mutant_is_caught(tmp_path, name):
+    old, new = GATED_BWD_MUTATIONS[name]
+    lib = _build(tmp_path, name, old, new)
+    assert not _gated_bwd_pin_passes(lib), name
