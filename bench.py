@@ -40,6 +40,9 @@ METRIC_BWD = "causal linear-attn bwd (dq, dk, dv) tokens/s and % of roofline (bf
 METRIC_NG = "causal linear-attn fwd + output RMSNorm/Swish gate tokens/s and % of roofline (bf16, B200)"
 METRIC_GD = "gated delta rule fwd tokens/s and % of roofline (bf16, B200)"
 
+# forward workloads timed and checked beside the main one in the default run
+EXTRA_FWD = ("sweep_T16384", "sweep_T4096", "sweep_T8192", "retnet_d256", "varlen", "long_1m")
+
 
 def _peaks():
     try:
@@ -272,13 +275,98 @@ def _config(w, ws):
     return {
         "workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "B_per_gpu": w.B, "H": w.H,
         "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk, "phi": w.phi, "normalize": w.normalize,
-        "gamma": ("per token: exp(g), g uniform in [ln %.3g, ln %.3g]" % w.gate) if w.gate else
-                 "evenly spaced in [%.3g, %.3g]" % (min(w.gamma), max(w.gamma)),
+        "gamma": w.gamma_rule or ("per head: %s" % ", ".join("%.6g" % x for x in w.gamma)),
         "parallelism": "dp%d" % ws, "l2": "inputs larger than L2 (no flush needed)",
     }
 
 
-def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False, delta=False):
+def _roofline(alg_bytes, alg_flops, launch_ms, hbm_peak, tc_peak):
+    """Roofline of one launch: the larger of the HBM time (bytes at the copy peak) and the
+    tensor time (flops at the bf16 peak) is the bound; frac = that time / the launch time."""
+    t_hbm = alg_bytes / (hbm_peak * 1e9)
+    t_tc = alg_flops / (tc_peak * 1e12)
+    s = launch_ms / 1e3
+    if t_hbm >= t_tc:
+        return {"bound": "hbm", "achieved": alg_bytes / s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "frac": t_hbm / s, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}
+    return {"bound": "tensor", "achieved": alg_flops / s / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+            "frac": t_tc / s, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}
+
+
+def _slice_err(got, ref):
+    import numpy as np
+
+    d = float(np.max(np.abs(ref)))
+    e = float(np.max(np.abs(got - ref)))
+    return e / d if d > 0 else e
+
+
+def _fwd_leg(la, w, dev, stream, hbm_peak, tc_peak, nrep=30, warm=5, parity=True):
+    """One forward workload other than the timed one: per-launch CUDA events over nrep
+    launches of la_fwd_chunk (all its kernels), the roofline, and parity of two full-length
+    (sequence, head) slices against the float64 oracle."""
+    import torch
+
+    from chunkwise_causal_linear_la_b200.workloads import make_inputs
+
+    x = make_inputs(w, seed=0, device=dev)
+    q, k, v, g, cu = x["q"], x["k"], x["v"], x["gamma"], x["cu_seqlens"]
+    B, T = q.shape[:2]
+    n_seqs = B if cu is None else cu.numel() - 1
+    tokens = B * T if cu is None else int(cu[-1])
+    out = torch.empty((B, T, w.H, w.d_v), dtype=q.dtype, device=dev)
+    fs = torch.empty((n_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
+    nws = la.workspace_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, w.chunk, q.dtype)
+    wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        la.la_fwd_chunk(q, k, v, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, normalize=w.normalize, out=out,
+                        final_state=fs, workspace=wsbuf, stream=stream)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nrep)]
+    for a_, b_ in ev:
+        a_.record(stream)
+        call()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ev)
+    alg_bytes, alg_flops = _algorithmic(w, n_seqs, tokens)
+    res = {"workload": w.name, "ms_per_launch": ms, "tokens_per_s": tokens / (ms / 1e3), "tokens": tokens,
+           "launches_per_call": (2 if cu is not None else 3) if nws > 0 else 1, "timed_calls": nrep,
+           "roofline": dict(_roofline(alg_bytes, alg_flops, ms, hbm_peak, tc_peak),
+                            alg_bytes_per_launch=alg_bytes, alg_flops_per_launch=alg_flops),
+           "config": _config(w, 1)}
+    if parity:
+        import oracle
+
+        oracle.build()
+        if cu is None:
+            sl = [(0, 0, T, 0), (B - 1, 0, T, w.H - 1)]
+            fidx = lambda b: b  # noqa: E731
+        else:
+            lens = (cu[1:] - cu[:-1]).tolist()
+            nl = max(range(n_seqs), key=lambda m: lens[m])
+            sl = [(0, int(cu[0]), int(cu[1]), 0), (0, int(cu[nl]), int(cu[nl + 1]), w.H - 1)]
+            seqs = [0, nl]
+        worst, names = 0.0, []
+        for m, (b, s0, e0, h) in enumerate(sl):
+            cut = lambda t: t[b:b + 1, s0:e0, h:h + 1].cpu()  # noqa: E731
+            ref, fref = oracle.recurrent(cut(q), cut(k), cut(v), [float(g[h])], phi=w.phi, normalize=w.normalize)
+            n_ = fidx(b) if cu is None else seqs[m]
+            worst = max(worst, _slice_err(cut(out).double().numpy(), ref),
+                        _slice_err(fs[n_:n_ + 1, h:h + 1].double().cpu().numpy(), fref))
+            names.append("(sequence %d, head %d, %d tokens)" % (n_, h, e0 - s0))
+        res["parity"] = {"max_rel_err": worst, "tolerance": 2e-2 if w.dtype == "bf16" else 1e-4,
+                         "slices": ", ".join(names) + " vs float64 oracle, outputs and final states"}
+    del x, q, k, v, out, fs, wsbuf
+    torch.cuda.empty_cache()
+    return res
+
+
+def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False, delta=False, check=False):
     """Times la_step (norm: la_step_norm, which also carries z; delta: one token of
     the gated delta rule, la_fwd_gated_delta with the state updated in place) on the
     decode workload: per-launch CUDA events, four state batches used in turn so that
@@ -311,6 +399,35 @@ def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False, delta=Fal
         else:
             la.la_step(dq, dk_, dv_, dg, states[i % 4], out=do, phi=phi, stream=stream)
 
+    # parity first: one call on state batch 0 against the oracle's step from the same state
+    parity = None
+    if check:
+        import numpy as np
+
+        import oracle
+
+        oracle.build()
+        st0 = states[0].double().cpu().numpy()
+        z0 = zs[0].double().cpu().numpy() if norm else None
+        call(0)
+        torch.cuda.synchronize()
+        if delta:
+            ref, fref = oracle.gated_delta(dq.unsqueeze(1).cpu(), dk_.unsqueeze(1).cpu(), dv_.unsqueeze(1).cpu(),
+                                           lg.double().cpu().numpy(), bt.double().cpu().numpy(), init=st0)
+            ref = ref[:, 0]
+        elif norm:
+            ref, fref, _ = oracle.step_norm(dq.cpu(), dk_.cpu(), dv_.cpu(), dg.double().cpu().numpy(), st0, z0,
+                                            phi=phi)
+        else:
+            ref, fref = oracle.step(dq.cpu(), dk_.cpu(), dv_.cpu(), dg.double().cpu().numpy(), st0, phi=phi)
+        got_o = do.double().cpu().numpy()
+        got_s = states[0].double().cpu().numpy()
+        e_o = max(_slice_err(got_o[n_, h_], ref[n_, h_]) for n_ in range(ref.shape[0]) for h_ in range(ref.shape[1]))
+        e_s = max(_slice_err(got_s[n_, h_], fref[n_, h_]) for n_ in range(ref.shape[0])
+                  for h_ in range(ref.shape[1]))
+        parity = {"max_rel_err_out": e_o, "max_rel_err_state": e_s, "tolerance": 1e-4,
+                  "slices": "every (sequence, head) of one call, fp32, vs the float64 oracle's step"}
+        del st0, got_s, fref
     for i in range(12):
         call(i)
     torch.cuda.synchronize()
@@ -330,7 +447,7 @@ def _decode_leg(la, dev, stream, hbm_peak, rank, nrep=400, norm=False, delta=Fal
     return {"workload": name, "us_per_step": us, "alg_bytes": dbytes,
             "achieved_gbs": dbytes / (us / 1e6) / 1e9, "peak_gbs": hbm_peak,
             "frac": dbytes / (us / 1e6) / 1e9 / hbm_peak, "kernel": "delta_kernel" if delta else "step_kernel",
-            "launches": nrep,
+            "launches": nrep, "parity": parity,
             "note": "per-launch CUDA events; four state batches in rotation (L2-cold)"}
 
 
@@ -471,7 +588,7 @@ def main():
         e_ = 2 if w.dtype == "bf16" else 4
         alg_bytes = tokens * w.H * e_ * (4 * w.d_k + 3 * w.d_v)
         alg_flops = 3 * alg_flops
-    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    roof = _roofline(alg_bytes, alg_flops, launch_ms, hbm_peak, tc_peak)
     # kernels launched per step: segmented sequences take a state pass, a scan and the output pass; the
     # backward takes three forward-shaped passes (plus four elementwise kernels with elu + 1)
     # (a packed batch with a workspace has its longest-first order computed first: 2 launches)
@@ -558,13 +675,6 @@ def main():
     e2e = {"value": aggregate_rate(tokens, args.e2e_steps, ws, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
-    # ---- decode step (la_step), HBM-bound: achieved GB/s
-    extra = {}
-    if not args.no_extra:
-        extra["decode"] = _decode_leg(la, dev, stream, hbm_peak, rank)
-        extra["decode_norm"] = _decode_leg(la, dev, stream, hbm_peak, rank, norm=True)
-        extra["decode_gated_delta"] = _decode_leg(la, dev, stream, hbm_peak, rank, delta=True)
-
     # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -574,6 +684,25 @@ def main():
                "sample": "%d sequence(s) of %s, all %d heads, first %d tokens each (float64 %s, %.1f s)"
                          % (nseq, w.name, w.H, n, "adjoint of the recurrence" if args.bwd else "recurrence", secs)}
 
+    # ---- decode step (la_step), HBM-bound: achieved GB/s
+    extra = {}
+    if not args.no_extra:
+        chk = rank == 0
+        extra["decode"] = _decode_leg(la, dev, stream, hbm_peak, rank, check=chk)
+        extra["decode_norm"] = _decode_leg(la, dev, stream, hbm_peak, rank, norm=True, check=chk)
+        extra["decode_gated_delta"] = _decode_leg(la, dev, stream, hbm_peak, rank, delta=True, check=chk)
+        # the other forward workloads, each timed and checked on its own (one GPU only: the
+        # multi-GPU run times the main workload alone)
+        if ws == 1 and not (args.bwd or args.normgate or gbeta is not None or gd is not None):
+            del out, fs, wsbuf, hosts, host_out
+            del x, q, k, v
+            torch.cuda.empty_cache()
+            for name in EXTRA_FWD:
+                if WORKLOADS[name].name == w.name:
+                    continue
+                extra[name] = _fwd_leg(la, WORKLOADS[name], dev, stream, hbm_peak, tc_peak,
+                                       nrep=20 if name == "long_1m" else 30)
+
     if rank == 0:
         line = {
             "metric": METRIC_BWD if args.bwd else (METRIC_NG if args.normgate else (
@@ -581,11 +710,13 @@ def main():
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype), "data": "synthetic",
             "config": _config(w, ws),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak,
+            "roofline": {"bound": roof["bound"], "achieved": roof["achieved"], "peak": roof["peak"],
+                         "unit": roof["unit"], "frac": roof["frac"],
+                         "t_hbm_us": roof["t_hbm_us"], "t_tensor_us": roof["t_tensor_us"],
                          "traffic": None if (args.bwd or args.normgate or gbeta is not None) else
                          _traffic(w.name, 1.0),
-                         "peak_kind": "%s (burst copy bandwidth)" % peak_kind,
+                         "peak_kind": "%s (burst: %s)" % (peak_kind, "copy bandwidth" if roof["bound"] == "hbm"
+                                                          else "cuBLAS bf16 GEMM"),
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "launch_ms": launch_ms,
                          "kernel": "chunk_tc_kernel (3 passes: forward + 2 in reverse time)" if args.bwd

@@ -41,6 +41,7 @@ class Workload:
     varlen: Optional[tuple] = None  # (n_seqs, lo, hi) for packed batches
     gate: Optional[tuple] = None  # (lo, hi): per-token decays in [lo, hi] (log drawn uniform)
     delta: bool = False  # gated delta rule: also a write strength beta per token, U[0.1, 1)
+    gamma_rule: str = ""  # how the per-head decays were chosen (a label for reports)
 
     @property
     def torch_dtype(self):
@@ -61,18 +62,19 @@ def _sweep(T: int) -> Workload:
     return Workload(
         f"sweep_B8_H16_d128_T{T}", B=8, T=T, H=16, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=linspace_gammas(16, 0.9, 0.999),
-        phi="identity", normalize=False,
+        phi="identity", normalize=False, gamma_rule="evenly spaced in [0.9, 0.999]",
     )
 
 
 WORKLOADS = {
     "tiny_f32": Workload(
         "tiny_f32_B1_H2_T256_d64", B=1, T=256, H=2, d_k=64, d_v=64, dtype="f32", scale=1.0,
-        gamma=(1.0, 1.0), phi="elu1", normalize=True,
+        gamma=(1.0, 1.0), phi="elu1", normalize=True, gamma_rule="1 (no decay)",
     ),
     "retnet_d256": Workload(
         "retnet_B32_H4_T2048_d256", B=32, T=2048, H=4, d_k=256, d_v=256, dtype="bf16",
         scale=1.0 / math.sqrt(256), gamma=retnet_gammas(4, 5), phi="identity", normalize=False,
+        gamma_rule="1 - 2^(-5-h), h = 0..3",
     ),
     "sweep_T4096": _sweep(4096),
     "sweep_T8192": _sweep(8192),
@@ -80,20 +82,22 @@ WORKLOADS = {
     "varlen": Workload(
         "varlen_64seqs_L128-2048_H8_d128", B=1, T=0, H=8, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=(1.0,) * 8, phi="elu1", normalize=True,
-        varlen=(64, 128, 2048),
+        varlen=(64, 128, 2048), gamma_rule="1 (no decay)",
     ),
     "gated_T16384": Workload(
         "gated_B8_H16_d128_T16384", B=8, T=16384, H=16, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=(1.0,) * 16, phi="identity", normalize=False, gate=(0.9, 0.999),
+        gamma_rule="per token: exp(g), g uniform in [ln 0.9, ln 0.999]",
     ),
     "gdelta_T16384": Workload(
         "gated_delta_B8_H16_d128_T16384", B=8, T=16384, H=16, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=(1.0,) * 16, phi="identity", normalize=False, gate=(0.9, 0.999),
-        delta=True,
+        delta=True, gamma_rule="per token: exp(g), g uniform in [ln 0.9, ln 0.999]; beta uniform in [0.1, 1)",
     ),
     "long_1m": Workload(
         "long_B1_H4_T1048576_d128", B=1, T=1 << 20, H=4, d_k=128, d_v=128, dtype="bf16",
         scale=1.0 / math.sqrt(128), gamma=retnet_gammas(4, 8), phi="identity", normalize=False,
+        gamma_rule="1 - 2^(-8-h), h = 0..3",
     ),
 }
 
