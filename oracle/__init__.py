@@ -101,6 +101,13 @@ def _load():
     return _lib
 
 
+def _oracle_error(name: str, rc: int) -> Exception:
+    """The exception for a non-zero return code of the C oracle."""
+    if rc == -20:
+        return MemoryError("%s could not allocate its working buffers on this host" % name)
+    return ValueError("%s rejected its arguments (code %d)" % (name, rc))
+
+
 def max_threads() -> int:
     return int(_load().oracle_max_threads())
 
@@ -171,7 +178,7 @@ def recurrent(q, k, v, gamma, cu_seqlens=None, phi="identity", normalize=False, 
         _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), int(nthreads),
     )
     if rc != 0:
-        raise ValueError("oracle_recurrent rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_recurrent", rc)
     return out, fs
 
 
@@ -185,7 +192,7 @@ def chunked(q, k, v, gamma, chunk, cu_seqlens=None, phi="identity", normalize=Fa
         _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), int(nthreads),
     )
     if rc != 0:
-        raise ValueError("oracle_chunked rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_chunked", rc)
     return out, fs
 
 
@@ -210,7 +217,7 @@ def step(q, k, v, gamma, state, phi="identity", nthreads=0):
         _ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(g), _ptr(st), _ptr(out), _PHI[phi], int(nthreads)
     )
     if rc != 0:
-        raise ValueError("oracle_step rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_step", rc)
     return out, st
 
 
@@ -235,7 +242,7 @@ def final_z(k, gamma, cu_seqlens=None, phi="identity", nthreads=0):
     z = np.zeros((n, H, dk), np.float64)
     rc = _load().oracle_final_z(_ptr(k), dt, B, T, H, dk, _ptr(g), _ptr(cu), n, _PHI[phi], _ptr(z), int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_final_z rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_final_z", rc)
     return z
 
 
@@ -259,7 +266,7 @@ def step_norm(q, k, v, gamma, state, z, phi="identity", nthreads=0):
     rc = _load().oracle_step_norm(_ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(g), _ptr(st), _ptr(zz),
                                   _ptr(out), _PHI[phi], int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_step_norm rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_step_norm", rc)
     return out, st, zz
 
 
@@ -281,7 +288,7 @@ def recurrent_gated(q, k, v, g, cu_seqlens=None, phi="identity", normalize=False
         _PHI[phi], int(bool(normalize)), _ptr(out), _ptr(fs), _ptr(fz), int(nthreads),
     )
     if rc != 0:
-        raise ValueError("oracle_recurrent_gated rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_recurrent_gated", rc)
     return out, fs, fz
 
 
@@ -303,7 +310,7 @@ def step_gated(q, k, v, g, state, z=None, phi="identity", nthreads=0):
     rc = _load().oracle_step_gated(_ptr(q), _ptr(k), _ptr(v), dq, N, H, dk, dv, _ptr(gg), _ptr(st), _ptr(zz),
                                    _ptr(out), _PHI[phi], int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_step_gated rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_step_gated", rc)
     return out, st, zz
 
 
@@ -321,7 +328,7 @@ def backward(q, k, v, dout, gamma, cu_seqlens=None, phi="identity", nthreads=0):
     rc = _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), dt, B, T, H, dk, dv, _ptr(g), _ptr(cu), n,
                                  _PHI[phi], 0, _ptr(gq), _ptr(gk), _ptr(gv), int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_backward rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_backward", rc)
     return gq, gk, gv
 
 
@@ -345,7 +352,7 @@ def backward_gated(q, k, v, dout, g, cu_seqlens=None, phi="identity", nthreads=0
     rc = _load().oracle_backward_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(do), dt, B, T, H, dk, dv, _ptr(gg), _ptr(cu),
                                        n, _PHI[phi], _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gd), int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_backward_gated rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_backward_gated", rc)
     return gq, gk, gv, gd
 
 
@@ -363,7 +370,7 @@ def norm_gate(o, g, w, eps=1e-5, nthreads=0):
     rc = _load().oracle_norm_gate(_ptr(oo), _ptr(gg), dt, oo.size // dv, dv, _ptr(ww), float(eps), _ptr(y),
                                   int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_norm_gate rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_norm_gate", rc)
     return y
 
 
@@ -385,7 +392,7 @@ def gated_delta(q, k, v, g, beta, cu_seqlens=None, init=None, nthreads=0):
     rc = _load().oracle_gated_delta(_ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(gg), _ptr(bb), _ptr(cu),
                                     n, _ptr(ii), _ptr(out), _ptr(fs), int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_gated_delta rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_gated_delta", rc)
     return out, fs
 
 
@@ -406,5 +413,5 @@ def gated_delta_chunked(q, k, v, g, beta, chunk, cu_seqlens=None, init=None, nth
     rc = _load().oracle_gated_delta_chunked(_ptr(q), _ptr(k), _ptr(v), dt, B, T, H, dk, dv, _ptr(gg), _ptr(bb),
                                             _ptr(cu), n, _ptr(ii), int(chunk), _ptr(out), _ptr(fs), int(nthreads))
     if rc != 0:
-        raise ValueError("oracle_gated_delta_chunked rejected its arguments (code %d)" % rc)
+        raise _oracle_error("oracle_gated_delta_chunked", rc)
     return out, fs

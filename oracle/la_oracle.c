@@ -55,6 +55,9 @@
  * Return value: 0 on success, a negative number for a bad argument.
  */
 #include <math.h>
+
+/* A task could not allocate its working buffers (inputs too large for this host). */
+#define ORC_ERR_NOMEM (-20)
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -140,6 +143,7 @@ int oracle_recurrent(const void *q, const void *k, const void *v, int dtype,
   const int64_t ntask = n_seqs * H * nblk;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < ntask; ++task) {
     const int64_t n = task / (H * nblk);
@@ -154,6 +158,12 @@ int oracle_recurrent(const void *q, const void *k, const void *v, int dtype,
     double *z = (double *)calloc((size_t)dk, sizeof(double));
     double *qh = (double *)malloc((size_t)dk * sizeof(double));
     double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    if (!S || !z || !qh || !kh) {
+      free(S); free(z); free(qh); free(kh);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
 
     for (int64_t t = 0; t < len; ++t) {
       const int64_t tok = start + t;
@@ -192,7 +202,7 @@ int oracle_recurrent(const void *q, const void *k, const void *v, int dtype,
     free(qh);
     free(kh);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -217,6 +227,7 @@ int oracle_chunked(const void *q, const void *k, const void *v, int dtype,
   if (chunk <= 0) return -9;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -230,6 +241,12 @@ int oracle_chunked(const void *q, const void *k, const void *v, int dtype,
     double *qh = (double *)malloc((size_t)(chunk * dk) * sizeof(double));
     double *kh = (double *)malloc((size_t)(chunk * dk) * sizeof(double));
     double *vv = (double *)malloc((size_t)(chunk * dv) * sizeof(double));
+    if (!S || !Sn || !z || !zn || !qh || !kh || !vv) {
+      free(S); free(Sn); free(z); free(zn); free(qh); free(kh); free(vv);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
 
     for (int64_t c0 = 0; c0 < len; c0 += chunk) {
       const int64_t Cp = len - c0 < chunk ? len - c0 : chunk;
@@ -293,7 +310,7 @@ int oracle_chunked(const void *q, const void *k, const void *v, int dtype,
     free(kh);
     free(vv);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -421,6 +438,7 @@ int oracle_recurrent_gated(const void *q, const void *k, const void *v, int dtyp
   if (!g) return -10;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -430,6 +448,12 @@ int oracle_recurrent_gated(const void *q, const void *k, const void *v, int dtyp
     double *z = (double *)calloc((size_t)dk, sizeof(double));
     double *qh = (double *)malloc((size_t)dk * sizeof(double));
     double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    if (!S || !z || !qh || !kh) {
+      free(S); free(z); free(qh); free(kh);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
     for (int64_t t = 0; t < len; ++t) {
       const int64_t row = start + t;  /* token row of the flattened [B * T] grid */
       const double a = exp(g[row * H + h]);
@@ -468,7 +492,7 @@ int oracle_recurrent_gated(const void *q, const void *k, const void *v, int dtyp
     free(qh);
     free(kh);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -537,6 +561,7 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
   if (normalize) return -11;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -546,6 +571,12 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
     double *S = (double *)calloc((size_t)(dv * dk), sizeof(double));  /* S[r][c] */
     double *qh = (double *)malloc((size_t)dk * sizeof(double));
     double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    if (!S || !qh || !kh) {
+      free(S); free(qh); free(kh);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
     /* forward in time: dqh_t = S_t^T dout_t */
     for (int64_t t = 0; t < len; ++t) {
       const int64_t row = start + t;
@@ -591,7 +622,7 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
     free(qh);
     free(kh);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -615,6 +646,7 @@ int oracle_backward_gated(const void *q, const void *k, const void *v, const voi
   if (!g || !dg) return -10;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -626,6 +658,12 @@ int oracle_backward_gated(const void *q, const void *k, const void *v, const voi
     double *D = (double *)calloc(sz, sizeof(double));
     double *qh = (double *)malloc((size_t)dk * sizeof(double));
     double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    if (!prev || !S || !D || !qh || !kh) {
+      free(prev); free(S); free(D); free(qh); free(kh);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
     /* forward in time */
     for (int64_t t = 0; t < len; ++t) {
       const int64_t row = start + t;
@@ -679,7 +717,7 @@ int oracle_backward_gated(const void *q, const void *k, const void *v, const voi
     free(qh);
     free(kh);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -729,6 +767,7 @@ int oracle_gated_delta(const void *q, const void *k, const void *v, int dtype, i
   if (!g || !beta) return -10;
   if (nthreads <= 0) nthreads = oracle_max_threads();
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -737,6 +776,12 @@ int oracle_gated_delta(const void *q, const void *k, const void *v, int dtype, i
     double *S = (double *)calloc((size_t)(dv * dk), sizeof(double));  /* S[r][c] */
     double *kt = (double *)malloc((size_t)dk * sizeof(double));
     double *u = (double *)malloc((size_t)dv * sizeof(double));
+    if (!S || !kt || !u) {
+      free(S); free(kt); free(u);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
     if (init)
       for (int64_t c = 0; c < dk; ++c)
         for (int64_t r = 0; r < dv; ++r) S[r * dk + c] = init[task * dk * dv + c * dv + r];
@@ -774,7 +819,7 @@ int oracle_gated_delta(const void *q, const void *k, const void *v, int dtype, i
     free(kt);
     free(u);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
 
 /*
@@ -805,6 +850,7 @@ int oracle_gated_delta_chunked(const void *q, const void *k, const void *v, int 
   if (nthreads <= 0) nthreads = oracle_max_threads();
   const int64_t C = chunk;
 
+  int oom = 0; /* set when a task could not allocate its buffers */
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
   for (int64_t task = 0; task < n_seqs * H; ++task) {
     const int64_t n = task / H, h = task % H;
@@ -820,6 +866,12 @@ int oracle_gated_delta_chunked(const void *q, const void *k, const void *v, int 
     double *X = (double *)malloc((size_t)(C * (dk > dv ? dk : dv)) * sizeof(double));
     double *bcum = (double *)malloc((size_t)C * sizeof(double));
     double *bet = (double *)malloc((size_t)C * sizeof(double));
+    if (!S || !Kt || !Q || !V || !A || !Ti || !U || !X || !bcum || !bet) {
+      free(S); free(Kt); free(Q); free(V); free(A); free(Ti); free(U); free(X); free(bcum); free(bet);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
     if (init)
       for (int64_t c = 0; c < dk; ++c)
         for (int64_t r = 0; r < dv; ++r) S[r * dk + c] = init[task * dk * dv + c * dv + r];
@@ -913,5 +965,5 @@ int oracle_gated_delta_chunked(const void *q, const void *k, const void *v, int 
     free(bcum);
     free(bet);
   }
-  return 0;
+  return oom ? ORC_ERR_NOMEM : 0;
 }
