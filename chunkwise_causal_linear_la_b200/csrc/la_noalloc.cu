@@ -14,6 +14,7 @@
 // slot the scan and the output pass read.  Two calls whose work overlaps on
 // the GPU (different streams, or different host threads on one device) race on
 // the array; callers must order them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -27,20 +28,47 @@ static_assert(LA_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size");
 // The scratch itself: every GPU that loads the library holds it until exit.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// cuCtxGetCurrent from the driver, looked up once through the runtime (no -lcuda).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void *g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch per device, with the context it was looked up
+// in: the array is placed anew whenever the device's context is recreated (after
+// cudaDeviceReset, for one), so an address is reused only in the context it came from.
+void *g_scratch_addr[kMaxDevices];
+CUcontext g_scratch_ctx[kMaxDevices];
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device memory:
-// the device address is looked up once per device, with that device current.
+// the device address is looked up with that device current, once per device and
+// context (the first call on a device, or the first after its context changed).
 cudaError_t scratch_address(int device, void **out) {
   if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return cudaErrorInitializationError;
+  CUcontext ctx = nullptr;  // NULL until the runtime has made a context current on this thread
+  if (get(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_addr[device]) {
+  if (!ctx || !g_scratch_addr[device] || g_scratch_ctx[device] != ctx) {
     void *p = nullptr;
-    const cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // sets the context up if needed
     if (err != cudaSuccess) return err;
+    if (!ctx && (get(&ctx) != CUDA_SUCCESS || !ctx)) return cudaErrorInitializationError;
     g_scratch_addr[device] = p;
+    g_scratch_ctx[device] = ctx;
   }
   *out = g_scratch_addr[device];
   return cudaSuccess;

@@ -384,8 +384,10 @@ LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_t
  *   than LA_NOALLOC_SCRATCH_BYTES of scratch (la_fwd_chunk_workspace_size tells;
  *   every problem the current kernels segment fits).
  *   Set-up: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and caches it together
+ *   with the device's current context; a call made in another context of that
+ *   device (after cudaDeviceReset, say) looks the address up again.  Make the
+ *   first call in each context before any stream capture.
  *   Sharing: all calls on a device use the same array and it keeps the previous
  *   call's contents (nothing in it needs to start at zero).  Calls whose work
  *   overlaps on the GPU (different streams, or several host threads on one
