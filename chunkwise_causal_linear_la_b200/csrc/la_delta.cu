@@ -175,126 +175,142 @@ cudaError_t launch_dtype(const DeltaArgs &a, cudaStream_t stream) {
 }
 
 // One token per sequence (decode): the state is read once and written once, so the
-// kernel is built for coalesced state traffic instead.  One CTA per (sequence,
-// head, 128 value columns), 512 threads: warp w holds rows [DK/16 w, DK/16 (w+1))
-// of S^T for the CTA's 128 columns, lane l the column quad 4l .. 4l + 3, loaded
-// and stored as float4 (a warp moves 512 contiguous bytes of one row at a time).
-// The two reductions over d_k (u = S kt and o = S q) go through shared memory.
-constexpr int kDecThreads = 512;
+// kernel is built for coalesced state traffic instead.  One CTA of 128 threads per
+// (sequence, head, 32 value columns): thread (row group rg, column quad cq) holds
+// rows rg, rg + 16, ... of S^T for columns 4 cq .. 4 cq + 3, all requested with
+// streaming loads before anything else (a warp moves 4 rows x 128 contiguous bytes
+// per instruction).  Both reductions over d_k come out of one pass over the old
+// state: with coef_r = beta (v_r - alpha u_r), the output of the updated state is
+// o = S_new q = alpha (S^T-contract q) + coef (kt . q), so u = S^T-contract kt and
+// p = S^T-contract q are summed over the 16 row groups together, behind a single
+// barrier.  Small CTAs keep the whole grid resident: the 512-thread CTAs used
+// before ran the [256, 4, 128, 128] state in 3.5 waves.
+constexpr int kDecThreads = 128;
+constexpr int kDecCols = 32;                       // value columns per CTA
+constexpr int kDecQuads = kDecCols / 4;            // float4 column quads
+constexpr int kDecGroups = kDecThreads / kDecQuads;  // row groups (16)
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(kDecThreads) delta_decode_kernel(DeltaArgs a) {
-  constexpr int RW = DK / 16;  // rows of S^T per warp
-  __shared__ float kt[DK], qv[DK], part[16][kDeltaCols];
-  __shared__ float red[32];
+  constexpr int RW = DK / kDecGroups;  // rows of S^T per thread
+  __shared__ float kt[DK], qv[DK];
+  __shared__ float4 pu[kDecGroups][kDecQuads], pq[kDecGroups][kDecQuads];
+  __shared__ float red[2][kDecThreads / 32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nsl = (a.dv + kDeltaCols - 1) / kDeltaCols;
+  const int cq = tid % kDecQuads, rg = tid / kDecQuads;
+  const int nsl = (a.dv + kDecCols - 1) / kDecCols;
   const int64_t unit = blockIdx.x;
   const int sl = (int)(unit % nsl);
   const int h = (int)((unit / nsl) % a.H);
   const int64_t n = unit / ((int64_t)nsl * a.H);
   const int64_t b = n, t = 0;  // the sequence's one token
-  const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + t * a.q.st + h * a.q.sh;
-  const Tin *K = (const Tin *)a.k.data + b * a.k.sb + t * a.k.st + h * a.k.sh;
-  const Tin *V = (const Tin *)a.v.data + b * a.v.sb + t * a.v.st + h * a.v.sh;
-  const int64_t row = (b * a.T + t) * a.H + h;
-  const float alpha = expf(a.g[row]), beta = a.beta[row];
-  // this thread's state block: rows c0 .. c0 + RW - 1, columns r0 .. r0 + 3, read once
-  // (streaming loads, issued first so that they overlap the key norm below)
-  const int c0 = warp * RW, r0 = sl * kDeltaCols + 4 * lane;
+  const int r0 = sl * kDecCols + 4 * cq;
   const bool active = r0 < a.dv;  // dv is a multiple of 4
   const int64_t sbase = ((int64_t)n * a.H + h) * (int64_t)DK * a.dv;
   float4 S[RW];
 #pragma unroll
   for (int j = 0; j < RW; ++j)
-    S[j] = (a.init && active) ? __ldcs(reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)(c0 + j) * a.dv + r0))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-  // unit key and query in shared memory
-  float ss = 0.f;
+    S[j] = (a.init && active)
+               ? __ldcs(reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)(rg + kDecGroups * j) * a.dv + r0))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + t * a.q.st + h * a.q.sh;
+  const Tin *K = (const Tin *)a.k.data + b * a.k.sb + t * a.k.st + h * a.k.sh;
+  const Tin *V = (const Tin *)a.v.data + b * a.v.sb + t * a.v.st + h * a.v.sh;
+  const int64_t row = (b * a.T + t) * a.H + h;
+  const float alpha = expf(a.g[row]), beta = a.beta[row];
+  // raw key and query in shared memory, |k|^2 and k . q
+  float ss = 0.f, kq = 0.f;
   for (int c = tid; c < DK; c += kDecThreads) {
-    const float kv = to_f32<Tin>(K[c]);
+    const float kv = to_f32<Tin>(K[c]), qq = to_f32<Tin>(Q[c]);
     kt[c] = kv;
-    qv[c] = to_f32<Tin>(Q[c]);
+    qv[c] = qq;
     ss = fmaf(kv, kv, ss);
+    kq = fmaf(kv, qq, kq);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) red[warp] = ss;
-  __syncthreads();
-  if (warp == 0) {
-    float x = lane < kDecThreads / 32 ? red[lane] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) red[0] = 1.f / fmaxf(sqrtf(x), 1e-12f);
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    kq += __shfl_xor_sync(0xffffffffu, kq, o);
   }
+  if (lane == 0) {
+    red[0][warp] = ss;
+    red[1][warp] = kq;
+  }
+  float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) vv = make_float4(to_f32<Tin>(V[r0]), to_f32<Tin>(V[r0 + 1]), to_f32<Tin>(V[r0 + 2]), to_f32<Tin>(V[r0 + 3]));
   __syncthreads();
-  const float inv = red[0];
-  // u = S^T-contract kt over this thread's rows, then across the 16 warps
-  float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+  // this thread's rows of u = sum_c k_c S^T[c][:] (raw key) and p = sum_c q_c S^T[c][:]
+  float4 u = make_float4(0.f, 0.f, 0.f, 0.f), p = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < RW; ++j) {
-    const float kc = kt[c0 + j] * inv;
+    const int c = rg + kDecGroups * j;
+    const float kc = kt[c], qc = qv[c];
     u.x = fmaf(kc, S[j].x, u.x);
     u.y = fmaf(kc, S[j].y, u.y);
     u.z = fmaf(kc, S[j].z, u.z);
     u.w = fmaf(kc, S[j].w, u.w);
+    p.x = fmaf(qc, S[j].x, p.x);
+    p.y = fmaf(qc, S[j].y, p.y);
+    p.z = fmaf(qc, S[j].z, p.z);
+    p.w = fmaf(qc, S[j].w, p.w);
   }
-  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = u;
+  pu[rg][cq] = u;
+  pq[rg][cq] = p;
   __syncthreads();
+  float sst = 0.f, kqt = 0.f;
+#pragma unroll
+  for (int w = 0; w < kDecThreads / 32; ++w) {
+    sst += red[0][w];
+    kqt += red[1][w];
+  }
+  const float inv = 1.f / fmaxf(sqrtf(sst), 1e-12f);  // kt = k inv, the listing's floor on |k|
   u = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int w = 0; w < 16; ++w) {
-    const float4 x = *reinterpret_cast<const float4 *>(&part[w][4 * lane]);
+  for (int r = 0; r < kDecGroups; ++r) {
+    const float4 x = pu[r][cq];
     u.x += x.x;
     u.y += x.y;
     u.z += x.z;
     u.w += x.w;
   }
-  // S <- alpha (S - beta kt u^T) + beta kt v^T, i.e. S^T[c][r] += ... with coef_r = beta (v_r - alpha u_r)
-  float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (active) vv = make_float4(to_f32<Tin>(V[r0]), to_f32<Tin>(V[r0 + 1]), to_f32<Tin>(V[r0 + 2]), to_f32<Tin>(V[r0 + 3]));
-  const float4 coef = make_float4(beta * (vv.x - alpha * u.x), beta * (vv.y - alpha * u.y),
-                                  beta * (vv.z - alpha * u.z), beta * (vv.w - alpha * u.w));
-  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < RW; ++j) {
-    const float kc = kt[c0 + j] * inv, qc = qv[c0 + j];
-    S[j].x = fmaf(alpha, S[j].x, coef.x * kc);
-    S[j].y = fmaf(alpha, S[j].y, coef.y * kc);
-    S[j].z = fmaf(alpha, S[j].z, coef.z * kc);
-    S[j].w = fmaf(alpha, S[j].w, coef.w * kc);
-    o.x = fmaf(qc, S[j].x, o.x);
-    o.y = fmaf(qc, S[j].y, o.y);
-    o.z = fmaf(qc, S[j].z, o.z);
-    o.w = fmaf(qc, S[j].w, o.w);
-  }
+  // S <- alpha (S - beta kt u^T) + beta kt v^T, i.e. S^T[c][r] = alpha S^T[c][r] + coef_r kt_c
+  // with u taken with the unit key and coef_r = beta (v_r - alpha u_r)
+  const float4 coef = make_float4(beta * (vv.x - alpha * u.x * inv), beta * (vv.y - alpha * u.y * inv),
+                                  beta * (vv.z - alpha * u.z * inv), beta * (vv.w - alpha * u.w * inv));
   if (a.final_state && active) {
 #pragma unroll
-    for (int j = 0; j < RW; ++j) __stcs(reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)(c0 + j) * a.dv + r0), S[j]);
-  }
-  __syncthreads();  // every warp has read the u partials
-  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = o;
-  __syncthreads();
-  if (warp == 0 && active) {
-    o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < 16; ++w) {
-      const float4 x = *reinterpret_cast<const float4 *>(&part[w][4 * lane]);
-      o.x += x.x;
-      o.y += x.y;
-      o.z += x.z;
-      o.w += x.w;
+    for (int j = 0; j < RW; ++j) {
+      const int c = rg + kDecGroups * j;
+      const float kc = kt[c] * inv;
+      float4 x = S[j];
+      x.x = fmaf(alpha, x.x, coef.x * kc);
+      x.y = fmaf(alpha, x.y, coef.y * kc);
+      x.z = fmaf(alpha, x.z, coef.z * kc);
+      x.w = fmaf(alpha, x.w, coef.w * kc);
+      __stcs(reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)c * a.dv + r0), x);
     }
+  }
+  if (rg == 0 && active) {  // o = alpha p + coef (kt . q)
+    p = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kDecGroups; ++r) {
+      const float4 x = pq[r][cq];
+      p.x += x.x;
+      p.y += x.y;
+      p.z += x.z;
+      p.w += x.w;
+    }
+    const float ktq = kqt * inv;
     Tin *O = (Tin *)a.out + b * a.o_sb + t * a.o_st + h * a.o_sh + r0;
-    O[0] = from_f32<Tin>(o.x);
-    O[1] = from_f32<Tin>(o.y);
-    O[2] = from_f32<Tin>(o.z);
-    O[3] = from_f32<Tin>(o.w);
+    O[0] = from_f32<Tin>(fmaf(alpha, p.x, coef.x * ktq));
+    O[1] = from_f32<Tin>(fmaf(alpha, p.y, coef.y * ktq));
+    O[2] = from_f32<Tin>(fmaf(alpha, p.z, coef.z * ktq));
+    O[3] = from_f32<Tin>(fmaf(alpha, p.w, coef.w * ktq));
   }
 }
 
 template <typename Tin>
 cudaError_t launch_decode(const DeltaArgs &a, cudaStream_t stream) {
-  const int64_t grid = a.n_seqs * a.H * ((a.dv + kDeltaCols - 1) / kDeltaCols);
+  const int64_t grid = a.n_seqs * a.H * ((a.dv + kDecCols - 1) / kDecCols);
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   switch (a.dk) {
