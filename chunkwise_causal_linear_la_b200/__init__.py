@@ -18,7 +18,10 @@ from .binding import (  # noqa: F401
     LA_FLAG_SIMT,
     LA_FLAG_TEST_WAIT_TIMEOUT,
     LaError,
+    LA_PATH_CUDA_CORE,
+    LA_PATH_TENSOR_CORE,
     device_error,
+    fwd_chunk_path,
     la_bwd_chunk,
     la_fwd_chunk,
     la_fwd_chunk_gated,

@@ -31,7 +31,8 @@ _DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk_workspace_size", "la_step",
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
            "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
-           "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size")
+           "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size",
+           "la_fwd_chunk_path")
 
 
 class LaTensor(ctypes.Structure):
@@ -90,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_gated_delta_chunk.restype = i32
     lib.la_fwd_gated_delta_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32]
     lib.la_fwd_gated_delta_workspace_size.restype = sz
+    lib.la_fwd_chunk_path.argtypes = [i64, i64, i64, i64, i32, i32, i32]
+    lib.la_fwd_chunk_path.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -134,6 +137,15 @@ def workspace_size(B, T, H, d_k, d_v, n_seqs, varlen, chunk, dtype=torch.bfloat1
     if n == ctypes.c_size_t(-1).value:
         raise LaError(LA_ERR_INVALID_ARG, "la_fwd_chunk_workspace_size rejected the arguments")
     return int(n)
+
+
+LA_PATH_TENSOR_CORE, LA_PATH_CUDA_CORE = 1, 2
+
+
+def fwd_chunk_path(d_k, d_v, T, H, chunk=64, dtype=torch.bfloat16, flags=LA_FLAG_NONE) -> int:
+    """Kernel la_fwd_chunk runs for this shape: LA_PATH_TENSOR_CORE, LA_PATH_CUDA_CORE,
+    or -1 for arguments it rejects (see la_fwd_chunk_path in include/la_b200.h)."""
+    return int(load_library().la_fwd_chunk_path(d_k, d_v, T, H, chunk, _DT[dtype], flags))
 
 
 def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", normalize=False,

@@ -310,6 +310,24 @@ size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k,
   return tc_workspace_bytes(B, T, H, (int)d_k, (int)d_v, n_seqs, has_cu_seqlens != 0, chunk);
 }
 
+int32_t la_fwd_chunk_path(int64_t d_k, int64_t d_v, int64_t T, int64_t H, int32_t chunk, int32_t dtype,
+                          int32_t flags) {
+  if (!head_dim_ok(d_k) || !head_dim_ok(d_v) || T < 0 || H <= 0) return -1;
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return -1;
+  if ((dtype != LA_F32 && dtype != LA_BF16) || (flags & ~LA_FLAG_SIMT)) return -1;
+  ChunkArgs a{};
+  a.dtype = dtype;
+  a.chunk = chunk;
+  a.dk = (int)d_k;
+  a.dv = (int)d_v;
+  a.T = T;
+  a.H = (int)H;
+  if (dtype == LA_BF16 && !(flags & LA_FLAG_SIMT) && tc_supported(a)) return LA_PATH_TENSOR_CORE;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) device = 0;
+  return simt_supported(a, device) ? LA_PATH_CUDA_CORE : -1;
+}
+
 la_status la_fwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
                        const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
                        int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,

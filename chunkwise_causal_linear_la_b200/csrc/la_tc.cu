@@ -110,7 +110,7 @@ struct TcArgs {
   float *final_state;
   float *final_z;  // NULL, or z after each sequence's last token (normalised only)
   int64_t T;
-  int H, dv, phi, normalize;
+  int H, dk, dv, phi, normalize;  // dk: the key head dim (64 in the d_k = 128 layout is zero padded)
   // Segmentation of long sequences (G = 1: none).  A sequence is split into G
   // segments of segC chunks.  The state pass (MODE 1, Gp = G - 1 CTAs per unit)
   // writes each segment's end state from a zero start to ws_s / ws_z; a scan
@@ -289,7 +289,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   constexpr bool kQByOutput = ELU && MODE == 0;
 
   // ---- the unit this CTA owns
-  const int NVT = a.dv / DVT;
+  // value slices; a d_v narrower than DVT (64 at d_k <= 128) runs in one slice whose
+  // columns past d_v read TMA zero fill and are never written out
+  const int NVT = (a.dv + DVT - 1) / DVT;
   const int unit = blockIdx.x / a.Gp;  // (sequence, head, value slice)
   const int seg = blockIdx.x % a.Gp;
   const int vt = unit % NVT;
@@ -626,7 +628,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // vector v sits in row (v mod 8C) / 8 of its [C x 64] slab.
       const int tt = tid - 64;
       constexpr bool elu = ELU;
-      constexpr int NV = G::QK_BYTES / 16 / 64;   // vectors per thread of a q or k tile
+      // vectors per thread of a q or k tile: 8 per 64-column slab; a d_k of 64 in the
+      // d_k = 128 layout transforms slab 0 only (slab 1 holds TMA zero fill, which
+      // must stay zero: phi(0) = 1 for elu + 1)
+      const int NV = 8 * (a.dk / 64);
       constexpr int NVV = G::V_BYTES / 16 / 64;   // ... of a v tile
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS, k = c / NS;
@@ -746,7 +751,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
         const int kr = mb * 128 + sp * 32 + lane;
-        zr[mb] = fmaf(gdec, zr[mb], ks[kr] + ks[DK + kr]);
+        zr[mb] = kr < a.dk ? fmaf(gdec, zr[mb], ks[kr] + ks[DK + kr]) : 0.f;
         zb[kr] = zr[mb];
       }
       return true;
@@ -823,22 +828,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       if (GATED && sp == 0 && lane == 0) a.ws_g[ws_slot] = seg_log;
     } else if (a.final_state && last_seg) {
-      F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)DK * a.dv + vt * DVT;
+      F = a.final_state + ((int64_t)n * a.H + h) * (int64_t)a.dk * a.dv + vt * DVT;
     }
     if (MODE == 0 && NORM && a.final_z && last_seg && vt == 0) {  // z after the last token
 #pragma unroll
-      for (int mb = 0; mb < G::MB; ++mb)
-        a.final_z[((int64_t)n * a.H + h) * DK + mb * 128 + sp * 32 + lane] = zr[mb];
+      for (int mb = 0; mb < G::MB; ++mb) {
+        const int kr = mb * 128 + sp * 32 + lane;
+        if (kr < a.dk) a.final_z[((int64_t)n * a.H + h) * a.dk + kr] = zr[mb];
+      }
     }
-    if (F) {
+    if (F) {  // workspace slots hold all DK x DVT values; the final state only d_k rows, d_v columns
+      const int rows = MODE == 1 ? DK : a.dk;
+      const int cols = MODE == 1 ? DVT : min(DVT, a.dv - vt * DVT);
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
         const int kr = mb * 128 + sp * 32 + lane;
         float4 *dst = reinterpret_cast<float4 *>(F + (int64_t)kr * ld);
+        if (kr < rows) {
 #pragma unroll
-        for (int q = 0; q < DVT / 4; ++q)
-          dst[q] = make_float4(S[mb * DVT + 4 * q], S[mb * DVT + 4 * q + 1], S[mb * DVT + 4 * q + 2],
-                               S[mb * DVT + 4 * q + 3]);
+          for (int q = 0; q < DVT / 4; ++q)
+            if (4 * q < cols)
+              dst[q] = make_float4(S[mb * DVT + 4 * q], S[mb * DVT + 4 * q + 1], S[mb * DVT + 4 * q + 2],
+                                   S[mb * DVT + 4 * q + 3]);
+        }
       }
     }
   } else {
@@ -1020,8 +1032,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc_fence_before();
           mbar_arrive(bars + G::B_OEMPTY + ob);
         }
-        if (lrow(i) < Cp) {
-          const int col = hf * (DVT / 2) + pass * 32;
+        const int col = hf * (DVT / 2) + pass * 32;
+        if (lrow(i) < Cp && vt * DVT + col < a.dv) {
           if (NG) {  // y = o rstd w swish(gate)
             const uint4 *gsrc = reinterpret_cast<const uint4 *>(
                 reinterpret_cast<const uint8_t *>(a.ng_gate) +
@@ -1055,7 +1067,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int s = c % NS;
       if (!wait_bar_warp(sy, G::B_FULL + s, (c / NS) & 1, c)) return false;
 #pragma unroll 1
-      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2); ++kb) {
+      for (int kb = hf * (G::KB / 2); kb < (hf + 1) * (G::KB / 2) && kb < a.dk / 64; ++kb) {
         uint8_t *row = q_tile(s) + kb * G::SLAB + i * 128;
         uint4 x[8];
 #pragma unroll
@@ -1127,8 +1139,12 @@ struct SegPlan {
 };
 
 // Value-slice width of the tensor-core kernel for a key head dim: the state
-// warpgroup holds d_k x DVT fp32 values, 128 per thread.
+// warpgroup holds d_k x DVT fp32 values, 128 per thread.  d_k = 64 runs in the
+// d_k = 128 layout (key and query columns 64 .. 127 are TMA zero fill).
 constexpr int tc_dvt(int dk) { return dk == 256 ? 64 : 128; }
+constexpr int tc_dk(int dk) { return dk == 256 ? 256 : 128; }
+// Value slices of a d_v: a d_v of 64 in a 128-wide slice counts as one.
+inline int tc_nvt(int dk, int dv) { return (dv + tc_dvt(dk) - 1) / tc_dvt(dk); }
 
 SegPlan seg_plan(int64_t n_seqs, int64_t T, int64_t H, int nvt, bool varlen, int chunk) {
   SegPlan p;
@@ -1230,11 +1246,13 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.g = a.g;
   t.T = a.T;
   t.H = a.H;
+  t.dk = a.dk;
   t.dv = a.dv;
   t.phi = a.phi;
   t.normalize = a.normalize;
-  const SegPlan plan = a.noseg ? SegPlan{1, 0, 0} : seg_plan(a.n_seqs, a.T, a.H, a.dv / DVT, a.cu_seqlens != nullptr, C);
-  const int64_t units = a.n_seqs * a.H * (a.dv / DVT);
+  const int nvt = (a.dv + DVT - 1) / DVT;
+  const SegPlan plan = a.noseg ? SegPlan{1, 0, 0} : seg_plan(a.n_seqs, a.T, a.H, nvt, a.cu_seqlens != nullptr, C);
+  const int64_t units = a.n_seqs * a.H * nvt;
   if (units == 0) return cudaSuccess;
   if (units * plan.G > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   t.G = plan.G;
@@ -1280,7 +1298,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
     const int elems_s = DK * DVT, elems_z = NORM ? DK : 0;
     dim3 sgrid((unsigned)((elems_s + elems_z + 255) / 256), (unsigned)units);
     seg_scan_kernel<<<sgrid, 256, 0, stream>>>(t.ws_s, t.ws_z, t.ws_g, a.gamma, plan.G, (int64_t)plan.segC * C,
-                                               a.H, a.dv / DVT, elems_s, elems_z);
+                                               a.H, nvt, elems_s, elems_z);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   // output pass: every segment, seeded with its start state
@@ -1303,22 +1321,30 @@ cudaError_t tc_device_error(unsigned int *flags, unsigned int *where, bool reset
 }
 
 // The output norm fuses into the epilogue when one CTA holds whole rows of d_v.
-bool tc_can_fuse_norm_gate(const ChunkArgs &a) { return a.dk == 128 && a.dv == tc_dvt(a.dk) && !a.g && !a.rev; }
+bool tc_can_fuse_norm_gate(const ChunkArgs &a) {
+  return (a.dk == 64 || a.dk == 128) && a.dv == tc_dvt(a.dk) && !a.g && !a.rev;
+}
+
+// Head dims the tensor-core kernel takes: d_k in {64, 128} with d_v = 64 or a
+// multiple of 128, and d_k = 256 with d_v a multiple of 64.
+bool tc_shape(int dk, int dv) {
+  if (dk == 64 || dk == 128) return dv == 64 || (dv > 0 && dv % 128 == 0);
+  if (dk == 256) return dv > 0 && dv % 64 == 0;
+  return false;
+}
 
 bool tc_supported(const ChunkArgs &a) {
   if (a.dtype != LA_BF16 || a.chunk != 64) return false;
-  if (a.dk != 128 && a.dk != 256) return false;
-  if (a.dv < tc_dvt(a.dk) || a.dv % tc_dvt(a.dk) != 0) return false;
+  if (!tc_shape(a.dk, a.dv)) return false;
   if (a.T > 0x7fffffffLL || a.H > 0xffff) return false;
   return encode_fn() != nullptr;
 }
 
 size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen, int chunk) {
   (void)B;
-  if (chunk != 64 || (dk != 128 && dk != 256) || dv < tc_dvt(dk) || dv % tc_dvt(dk) != 0)
-    return 0;  // not a tensor-core shape
-  const int dvt = tc_dvt(dk);
-  return seg_ws_bytes(seg_plan(n_seqs, T, H, dv / dvt, varlen, chunk), dk, dvt) + order_bytes(n_seqs, varlen);
+  if (chunk != 64 || !tc_shape(dk, dv)) return 0;  // not a tensor-core shape
+  return seg_ws_bytes(seg_plan(n_seqs, T, H, tc_nvt(dk, dv), varlen, chunk), tc_dk(dk), tc_dvt(dk)) +
+         order_bytes(n_seqs, varlen);
 }
 
 template <int DK, int DVT, int NS, bool GATED>

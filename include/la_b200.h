@@ -123,9 +123,11 @@ typedef struct {
  *               Its contents need not be initialised and are undefined after.
  *   stream      cudaStream_t as void*.
  *
- * Kernels: bf16 with chunk 64 and d_k = 128 (d_v = 128 or 256) or d_k = 256
- * (d_v = 64, 128 or 256) runs on the tensor cores; every other valid shape,
- * f32, and LA_FLAG_SIMT run on the CUDA-core kernel.
+ * Kernels: bf16 with chunk 64 and d_k in {64, 128} (d_v = 64, 128 or 256) or
+ * d_k = 256 (d_v = 64, 128 or 256) runs on the tensor cores; every other valid
+ * shape, f32, and LA_FLAG_SIMT run on the CUDA-core kernel, which computes in
+ * fp32 and is roughly ten times slower.  la_fwd_chunk_path tells which one a
+ * shape takes.
  *
  * Arithmetic: bf16 inputs are read as bf16, phi is evaluated in fp32 and the
  * tensor-core operands (phi(q), phi(k), decayed phi(k) or decayed v, the masked
@@ -285,6 +287,21 @@ LA_API la_status la_fwd_chunk_normgate(const la_tensor *q, const la_tensor *k, c
 LA_API size_t la_fwd_chunk_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
                                    int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk,
                                    int32_t dtype, int32_t flags);
+
+/*
+ * la_fwd_chunk_path -- which kernel la_fwd_chunk (and la_fwd_chunk_z,
+ * la_fwd_chunk_gated, la_fwd_chunk_normgate, the noalloc variant) runs for a
+ * problem with these head dims, length, heads, chunk, dtype and flags on the
+ * current device: LA_PATH_TENSOR_CORE (the tcgen05 kernel) or
+ * LA_PATH_CUDA_CORE (fp32 CUDA-core kernel: every other valid shape, much
+ * slower); -1 for arguments la_fwd_chunk rejects (LA_ERR_INVALID_ARG or
+ * LA_ERR_UNSUPPORTED).  An addition of this library (the pages have no
+ * counterpart): it lets a caller see a fall back to the slow kernel before
+ * timing it.  Host-only; reads device attributes but launches nothing.
+ */
+typedef enum { LA_PATH_TENSOR_CORE = 1, LA_PATH_CUDA_CORE = 2 } la_path;
+LA_API int32_t la_fwd_chunk_path(int64_t d_k, int64_t d_v, int64_t T, int64_t H, int32_t chunk, int32_t dtype,
+                                 int32_t flags);
 
 /*
  * la_step -- one decode token per sequence: the recurrence applied once.

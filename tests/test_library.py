@@ -94,7 +94,7 @@ def test_workspace_size_segment_plan(lib):
     """Segment states (S^T, the normaliser sum and the log decay of a
     data-dependent decay) are kept for all but the last segment of each unit,
     one unit per (sequence, head, value slice); value slices are 128 columns
-    wide at d_k = 128 and 64 at d_k = 256."""
+    wide at d_k <= 128 and 64 at d_k = 256."""
     ws = lib.la_fwd_chunk_workspace_size
     # d_k = 128: 2 units, 79 chunks -> G = min(148 // 2, 79 // 16) = 4 segments of 20 chunks
     assert ws(1, 5000, 2, 128, 128, 1, 0, 64, 1, 0) == 2 * 3 * (128 * 128 + 128 + 1) * 4
@@ -108,7 +108,9 @@ def test_workspace_size_segment_plan(lib):
     assert ws(1, 77431, 8, 128, 128, 64, 1, 64, 1, 0) == 256
     assert ws(1, 77431, 8, 128, 128, 65, 1, 64, 1, 0) == 512
     assert ws(1, 77431, 8, 128, 128, 5000, 1, 64, 1, 0) == 0
-    assert ws(1, 5000, 2, 64, 64, 1, 0, 64, 1, 0) == 0
+    # d_k = d_v = 64 runs in the d_k = 128 layout (zero-padded keys, a 128-wide value slice)
+    assert ws(1, 5000, 2, 64, 64, 1, 0, 64, 1, 0) == 2 * 3 * (128 * 128 + 128 + 1) * 4
+    assert ws(1, 5000, 2, 32, 32, 1, 0, 64, 1, 0) == 0  # CUDA-core kernel: no workspace
 
 
 def _t(B=1, T=4, H=2, D=64, dtype=1, ptr=0x1000):
@@ -188,3 +190,24 @@ def test_normaliser_state_arguments_validated_on_host(lib):
     st = lib.la_step_norm(ctypes.byref(q1), ctypes.byref(k1), ctypes.byref(v1), 0x2000, 0x5000, 0x6008,
                           ctypes.byref(o1), 1, None)
     assert st == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()
+
+
+def test_path_query_host_logic(lib):
+    """la_fwd_chunk_path: -1 where la_fwd_chunk rejects the arguments, the CUDA-core
+    kernel for f32, LA_FLAG_SIMT and bf16 shapes the tensor cores do not take (the
+    tensor-core answer itself needs a GPU driver; tests/test_tc_d64_gpu.py checks it)."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    path = lib.la_fwd_chunk_path
+    assert path(96, 128, 100, 4, 64, b.LA_BF16, 0) == -1  # head dim
+    assert path(128, 128, 100, 4, 48, b.LA_BF16, 0) == -1  # chunk
+    assert path(128, 128, 100, 0, 64, b.LA_BF16, 0) == -1  # heads
+    assert path(128, 128, -1, 4, 64, b.LA_BF16, 0) == -1  # length
+    assert path(128, 128, 100, 4, 64, 7, 0) == -1  # dtype
+    assert path(128, 128, 100, 4, 64, b.LA_BF16, 4) == -1  # flags
+    assert path(128, 128, 100, 4, 64, b.LA_F32, 0) == 2
+    assert path(128, 128, 100, 4, 64, b.LA_BF16, b.LA_FLAG_SIMT) == 2
+    for chunk in (16, 32, 128):
+        assert path(128, 128, 100, 4, chunk, b.LA_BF16, 0) == 2
+    assert path(32, 32, 100, 4, 64, b.LA_BF16, 0) == 2
+    assert path(128, 128, 100, 4, 64, b.LA_BF16, 0) in (1, 2)
