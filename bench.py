@@ -640,7 +640,10 @@ def main():
         parity = {"max_rel_err": worst, "tolerance": 2e-2 if w.dtype == "bf16" else 1e-4,
                   "slices": "(sequence, head) = %s vs float64 oracle, full length" % sl}
 
-    # ---- end to end: pinned host buffers, copies inside the timed region
+    # ---- end to end: pinned host buffers, copies inside the timed region.  The plain forward
+    # goes through the C-ABI call that takes host buffers (la_fwd_chunk_host: copies in, forward,
+    # copies out, one stream); the other legs copy through torch around their device call.
+    plain = not (args.bwd or args.normgate or gbeta is not None or gd is not None)
     inputs = (q, k, v) if gd is None else (q, k, v, gd)
     if gbeta is not None:
         inputs = (q, k, v, gd, gbeta)
@@ -648,11 +651,21 @@ def main():
         inputs = (q, k, v, ng_gate)
     if args.bwd:
         inputs = (q, k, v, dout)
+    if plain:
+        inputs = (q, k, v, g) + (() if cu is None else (cu,))
     outputs = grads if args.bwd else (out, fs)
     hosts = [t.cpu().pin_memory() for t in inputs]
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outputs]
+    if plain:
+        arena = torch.empty(la.host_arena_size(B, T, w.H, w.d_k, w.d_v, n_seqs, cu is not None, w.chunk, q.dtype),
+                            dtype=torch.uint8, device=dev)
 
     def e2e_step():
+        if plain:
+            la.la_fwd_chunk_host(hosts[0], hosts[1], hosts[2], hosts[3], cu_seqlens=hosts[4] if cu is not None else None,
+                                 chunk=w.chunk, phi=w.phi, normalize=w.normalize, out=host_out[0],
+                                 final_state=host_out[1], arena=arena, stream=stream)
+            return
         for dst, src in zip(inputs, hosts):
             dst.copy_(src, non_blocking=True)
         step()
@@ -673,7 +686,8 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in inputs)
     d2h = sum(t.numel() * t.element_size() for t in outputs)
     e2e = {"value": aggregate_rate(tokens, args.e2e_steps, ws, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+           "call": "la_fwd_chunk_host (C ABI, host buffers)" if plain else "torch copies around the device call"}
 
     # ---- CPU baseline: the float64 oracle on host cores, rank 0 at N=1 only
     cpu = None
@@ -694,7 +708,7 @@ def main():
         # the other forward workloads, each timed and checked on its own (one GPU only: the
         # multi-GPU run times the main workload alone)
         if ws == 1 and not (args.bwd or args.normgate or gbeta is not None or gd is not None):
-            del out, fs, wsbuf, hosts, host_out
+            del out, fs, wsbuf, hosts, host_out, arena
             del x, q, k, v
             torch.cuda.empty_cache()
             for name in EXTRA_FWD:

@@ -22,6 +22,8 @@ from .binding import (  # noqa: F401
     LA_PATH_TENSOR_CORE,
     device_error,
     fwd_chunk_path,
+    host_arena_size,
+    la_fwd_chunk_host,
     la_bwd_chunk,
     la_fwd_chunk,
     la_fwd_chunk_gated,

@@ -32,7 +32,7 @@ EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
            "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
            "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size",
-           "la_fwd_chunk_path")
+           "la_fwd_chunk_path", "la_fwd_chunk_host", "la_fwd_chunk_host_arena_size")
 
 
 class LaTensor(ctypes.Structure):
@@ -93,6 +93,10 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_gated_delta_workspace_size.restype = sz
     lib.la_fwd_chunk_path.argtypes = [i64, i64, i64, i64, i32, i32, i32]
     lib.la_fwd_chunk_path.restype = i32
+    lib.la_fwd_chunk_host_arena_size.argtypes = [i64, i64, i64, i64, i64, i64, i32, i32, i32, i32, i32]
+    lib.la_fwd_chunk_host_arena_size.restype = sz
+    lib.la_fwd_chunk_host.argtypes = [P, P, P, vp, vp, i64, i32, i32, i32, P, vp, i32, vp, sz, vp]
+    lib.la_fwd_chunk_host.restype = i32
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -158,6 +162,49 @@ def la_fwd_chunk(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", norm
     """
     out, final_state, _ = _fwd(q, k, v, gamma, cu_seqlens, chunk, phi, normalize, out, final_state,
                                return_final_state, None, flags, workspace, stream)
+    return out, final_state
+
+
+def host_arena_size(B, T, H, d_k, d_v, n_seqs, varlen, chunk=64, dtype=torch.bfloat16, flags=0,
+                    final_state=True) -> int:
+    """Device bytes la_fwd_chunk_host needs as its arena."""
+    n = load_library().la_fwd_chunk_host_arena_size(B, T, H, d_k, d_v, n_seqs, int(bool(varlen)), chunk, _DT[dtype],
+                                                     flags, int(bool(final_state)))
+    if n == ctypes.c_size_t(-1).value:
+        raise LaError(LA_ERR_INVALID_ARG, "la_fwd_chunk_host_arena_size rejected the arguments")
+    return int(n)
+
+
+def la_fwd_chunk_host(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", normalize=False, out=None,
+                      final_state=None, return_final_state=True, flags=LA_FLAG_NONE, arena=None, stream=None):
+    """la_fwd_chunk on host tensors (see la_fwd_chunk_host in include/la_b200.h): q, k, v, gamma,
+    cu_seqlens, out and final_state are CPU tensors (pin them for asynchronous copies); the arena is a
+    device uint8 tensor (allocated here if None).  The copies and the forward are enqueued on the
+    stream; synchronise it before reading out / final_state.  Returns (out, final_state or None)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("gamma", gamma)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous host tensor" % name)
+    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or cu_seqlens.device.type != "cpu"):
+        raise TypeError("cu_seqlens must be a host int32 tensor")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    need = host_arena_size(B, T, H, dk, dv, n_seqs, cu_seqlens is not None, chunk, q.dtype, flags,
+                           final_state is not None)
+    if arena is None or arena.numel() * arena.element_size() < need:
+        arena = torch.empty(need, dtype=torch.uint8, device="cuda")
+    tq, tk, tv, to = describe(q), describe(k), describe(v), describe(out)
+    st = lib.la_fwd_chunk_host(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), gamma.data_ptr(),
+                               None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
+                               int(bool(normalize)), ctypes.byref(to),
+                               None if final_state is None else final_state.data_ptr(), int(flags),
+                               arena.data_ptr(), arena.numel() * arena.element_size(), _stream(stream))
+    _check(lib, st, "la_fwd_chunk_host")
     return out, final_state
 
 

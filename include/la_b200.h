@@ -304,6 +304,42 @@ LA_API int32_t la_fwd_chunk_path(int64_t d_k, int64_t d_v, int64_t T, int64_t H,
                                  int32_t flags);
 
 /*
+ * la_fwd_chunk_host -- la_fwd_chunk on host buffers, end to end: the inputs
+ * are copied into a device arena, the forward runs there, and the output and
+ * final state are copied back, all enqueued on `stream` in that order (one
+ * cudaMemcpyAsync per buffer); the call returns before they complete, so
+ * synchronise the stream before reading `out` or `final_state`.  An addition
+ * of this library (the pages have no counterpart): for callers whose
+ * activations are in host memory and who want the whole round trip measured
+ * or scheduled as one call.
+ *
+ *   q, k, v, out  la_tensors whose data pointers are HOST memory, each
+ *                 contiguous [B, T, H, D] (stride_h = D, stride_t = H D,
+ *                 stride_b = T H D).  Page-locked memory lets the copies run
+ *                 asynchronously; pageable memory works, but then each copy
+ *                 waits for the host.
+ *   gamma         host float[H]; cu_seqlens host int32[n_seqs + 1] or NULL;
+ *   final_state   host float[n_seqs, H, d_k, d_v] or NULL.
+ *   arena         device memory the caller owns, 256-byte aligned, of at
+ *                 least la_fwd_chunk_host_arena_size(...) bytes (with
+ *                 has_final_state = final_state != NULL): it receives the device
+ *                 copies of every buffer and la_fwd_chunk's workspace.  Its
+ *                 contents are undefined after the call.
+ *   Every other argument, the results and the arithmetic are la_fwd_chunk's.
+ * Errors: LA_ERR_INVALID_ARG for a non-contiguous host tensor, a NULL pointer
+ * or a misaligned arena; LA_ERR_UNSUPPORTED for a shape la_fwd_chunk rejects;
+ * LA_ERR_WORKSPACE for a missing or short arena; LA_ERR_CUDA if a copy cannot
+ * be enqueued; la_fwd_chunk's own errors otherwise.  Nothing is allocated.
+ */
+LA_API size_t la_fwd_chunk_host_arena_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                           int64_t n_seqs, int32_t has_cu_seqlens, int32_t chunk, int32_t dtype,
+                                           int32_t flags, int32_t has_final_state);
+LA_API la_status la_fwd_chunk_host(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma,
+                                   const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                                   int32_t normalize, const la_tensor *out, float *final_state, int32_t flags,
+                                   void *arena, size_t arena_bytes, void *stream);
+
+/*
  * la_step -- one decode token per sequence: the recurrence applied once.
  *   q, k   [N, 1, H, d_k]; v [N, 1, H, d_v] (la_tensor with T = 1); f32 or
  *          bf16, one dtype for all three.

@@ -211,3 +211,30 @@ def test_path_query_host_logic(lib):
         assert path(128, 128, 100, 4, chunk, b.LA_BF16, 0) == 2
     assert path(32, 32, 100, 4, 64, b.LA_BF16, 0) == 2
     assert path(128, 128, 100, 4, 64, b.LA_BF16, 0) in (1, 2)
+
+
+def test_host_arena_size_and_validation(lib):
+    """la_fwd_chunk_host_arena_size lays out q, k, v, out, the final state, gamma,
+    cu_seqlens and the workspace at 256-byte boundaries; la_fwd_chunk_host rejects
+    non-contiguous host tensors and a missing arena before touching a device."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, T, H, dk, dv = 2, 100, 3, 128, 64
+    tok = B * T * H
+    want = up(tok * dk * 2) * 2 + up(tok * dv * 2) * 2 + up(B * H * dk * dv * 4) + up(H * 4)
+    assert lib.la_fwd_chunk_host_arena_size(B, T, H, dk, dv, B, 0, 64, b.LA_BF16, 0, 1) == want
+    assert lib.la_fwd_chunk_host_arena_size(B, T, H, dk, dv, B, 0, 64, b.LA_BF16, 0, 0) == want - up(B * H * dk * dv * 4)
+    # a packed batch adds cu_seqlens (and its longest-first order in the workspace)
+    packed = lib.la_fwd_chunk_host_arena_size(1, 500, H, dk, dv, 5, 1, 64, b.LA_BF16, 0, 0)
+    assert packed == (up(500 * H * dk * 2) * 2 + up(500 * H * dv * 2) * 2 + up(H * 4) + up(6 * 4)
+                      + lib.la_fwd_chunk_workspace_size(1, 500, H, dk, dv, 5, 1, 64, b.LA_BF16, 0))
+    assert lib.la_fwd_chunk_host_arena_size(B, T, H, 96, dv, B, 0, 64, b.LA_BF16, 0, 1) == ctypes.c_size_t(-1).value
+    t = _t(B=1, T=4, H=2, D=64)
+    strided = b.LaTensor(0x1000, 1, 1, 4, 2, 64, 4 * 2 * 128, 2 * 128, 128)
+    call = lambda q, arena, nbytes: lib.la_fwd_chunk_host(  # noqa: E731
+        ctypes.byref(q), ctypes.byref(t), ctypes.byref(t), 0x2000, None, 1, 64, 0, 0, ctypes.byref(t), None, 0,
+        arena, nbytes, None)
+    assert call(strided, 0x4000, 1 << 20) == b.LA_ERR_INVALID_ARG
+    assert call(t, None, 0) == b.LA_ERR_WORKSPACE
+    assert call(t, 0x4010, 1 << 20) == b.LA_ERR_INVALID_ARG  # arena not 256-byte aligned
