@@ -529,11 +529,14 @@ struct GdnTcArgs {
   const float *bt;            // [chunk slot][H][2][C]: b_i and ln(1/|k_i|) - b_i of every chunk, from the WY pass
   const int32_t *coff;        // packed: first chunk slot of each sequence (dense: n * nck)
   int64_t nck;                // chunks per sequence (dense)
-  const float *init;          // NULL or [n_seqs, H, 128, 128] (S^T)
-  float *final_state;         // NULL or [n_seqs, H, 128, 128]
+  const float *init;          // NULL or [n_seqs, H, d_k, d_v] (S^T)
+  float *final_state;         // NULL or [n_seqs, H, d_k, d_v]
   const int32_t *cu_seqlens;  // NULL: dense
   int64_t T;
   int H;
+  // head dims: 64 or 128 each; a 64 runs in the 128 layout, its extra key, query and
+  // value columns read as TMA zero fill (zero rows and columns of S), never written out
+  int dk, dv;
 };
 
 template <int NS>
@@ -790,13 +793,13 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int sp = warp & 3;
     const int kr = sp * 32 + lane;  // row of S^T (d_k index) held by this thread
     const uint32_t lane_base = tbase + ((uint32_t)(sp * 32) << 16);
-    const int64_t sbase = (n * a.H + h) * (int64_t)kD * kD;
+    const int64_t sbase = (n * a.H + h) * (int64_t)a.dk * a.dv;
     float S[kD];
     if (has_init) {
-      const float4 *src = reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)kr * kD);
+      const float4 *src = reinterpret_cast<const float4 *>(a.init + sbase + (int64_t)kr * a.dv);
 #pragma unroll
       for (int q = 0; q < kD / 4; ++q) {
-        const float4 x = src[q];
+        const float4 x = (kr < a.dk && 4 * q < a.dv) ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
         S[4 * q] = x.x;
         S[4 * q + 1] = x.y;
         S[4 * q + 2] = x.z;
@@ -899,10 +902,11 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int e = 0; e < 32; ++e) S[grp * 32 + e] = fmaf(gdec, S[grp * 32 + e], __uint_as_float(r[e]));
       }
     }
-    if (a.final_state && !*abort_flag) {
-      float4 *dst = reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)kr * kD);
+    if (a.final_state && !*abort_flag && kr < a.dk) {
+      float4 *dst = reinterpret_cast<float4 *>(a.final_state + sbase + (int64_t)kr * a.dv);
 #pragma unroll
-      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+      for (int q = 0; q < kD / 4; ++q)
+        if (4 * q < a.dv) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
     }
   } else {
     // ================================================================ output
@@ -972,7 +976,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           tc_fence_before();
           mbar_arrive(bars + G::B_OEMPTY + b);
         }
-        if (i < Cp) {
+        if (i < Cp && hf * 64 + pass * 32 < a.dv) {
           uint4 *dst = reinterpret_cast<uint4 *>(obase + 2 * (tok * a.o_st + hf * 64 + pass * 32));
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -1031,10 +1035,13 @@ WsPlan ws_plan(int64_t B, int64_t T, int64_t H, int64_t n_seqs, bool varlen) {
 
 }  // namespace
 
-bool gdn_tc_supported(const DeltaArgs &a) { return a.dtype == LA_BF16 && a.dk == kD && a.dv == kD; }
+// Head dims of the tensor-core path: 64 or 128 each (a 64 in the 128 layout, zero padded).
+bool gdn_shape(int dk, int dv) { return (dk == 64 || dk == kD) && (dv == 64 || dv == kD); }
+
+bool gdn_tc_supported(const DeltaArgs &a) { return a.dtype == LA_BF16 && gdn_shape(a.dk, a.dv); }
 
 size_t gdn_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs, bool varlen) {
-  if (dk != kD || dv != kD) return 0;
+  if (!gdn_shape(dk, dv)) return 0;
   return ws_plan(B, T, H, n_seqs, varlen).total;
 }
 
@@ -1056,8 +1063,9 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   const TensorView wv{w, a.T * a.H * kD, (int64_t)a.H * kD, kD};
   const TensorView uv{ut, a.T * a.H * kD, (int64_t)a.H * kD, kD};
   CUtensorMap mq, mk, mv, mw, mu;
-  if (!make_map(&mq, a.q, B, a.T, a.H, kD, kC) || !make_map(&mk, a.k, B, a.T, a.H, kD, kC) ||
-      !make_map(&mv, a.v, B, a.T, a.H, kD, kC) || !make_map(&mw, wv, B, a.T, a.H, kD, kC) ||
+  // q, k, v maps have the tensors' own head dims: columns past them read as zero fill
+  if (!make_map(&mq, a.q, B, a.T, a.H, a.dk, kC) || !make_map(&mk, a.k, B, a.T, a.H, a.dk, kC) ||
+      !make_map(&mv, a.v, B, a.T, a.H, a.dv, kC) || !make_map(&mw, wv, B, a.T, a.H, kD, kC) ||
       !make_map(&mu, uv, B, a.T, a.H, kD, kC)) {
     if (why) *why = "cuTensorMapEncodeTiled rejected a tensor";
     return cudaErrorInvalidValue;
@@ -1100,6 +1108,8 @@ cudaError_t launch_gdn_chunk(const DeltaArgs &a, void *workspace, size_t workspa
   t.cu_seqlens = a.cu_seqlens;
   t.T = a.T;
   t.H = a.H;
+  t.dk = a.dk;
+  t.dv = a.dv;
   using G = GdnCfg<kStages>;
   auto kern = gdn_tc_kernel<kStages>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);

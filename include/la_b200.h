@@ -218,7 +218,7 @@ LA_API la_status la_fwd_gated_delta(const la_tensor *q, const la_tensor *k, cons
  *     U = T diag(beta) V - T diag(beta e^b) Kt S_0^T,   T = (I + A)^{-1},
  *     A_ij = beta_i e^{b_i - b_j} kt_i . kt_j  (j < i),  b_i = sum of g over the chunk up to i,
  * and outputs and the next chunk's state follow from U with matrix products.
- * Tensor cores (tcgen05) for bf16 with d_k = d_v = 128 and 16-byte aligned
+ * Tensor cores (tcgen05) for bf16 with d_k, d_v in {64, 128} and 16-byte aligned
  * initial_state / final_state: a parallel pass over all chunks writes
  * W = T diag(beta e^b) Kt and T diag(beta) V (bf16) and the chunk's b_i and
  * ln(1/|k_i|) - b_i (fp32) to the workspace, then one CTA per (sequence, head)

@@ -246,3 +246,24 @@ def test_gated_delta_chunk_state_in_place_and_fallbacks(la, oracle_mod):
     _check_chunk(la, oracle_mod, q, k, v, g, beta, flags=1)
     q2, k2, v2, g2, b2 = _inputs(1, 90, 2, 64, 64, torch.bfloat16, 22)
     _check_chunk(la, oracle_mod, q2, k2, v2, g2, b2)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 65, 300])
+def test_gated_delta_chunk_d64(la, oracle_mod, dk, dv, T):
+    """64-wide heads on the tensor-core path: the d = 128 layout with the extra key,
+    query and value columns read as TMA zero fill (zero rows and columns of the
+    state, outputs and final state clipped to d_v), with and without an initial state."""
+    assert la.gated_delta_workspace_size(2, T, 2, dk, dv, 2, False, torch.bfloat16) > 0
+    q, k, v, g, beta = _inputs(2, T, 2, dk, dv, torch.bfloat16, 40 + dk + dv + T)
+    _check_chunk(la, oracle_mod, q, k, v, g, beta)
+    init = torch.randn((2, 2, dk, dv)) * 0.2
+    _check_chunk(la, oracle_mod, q, k, v, g, beta, init=init)
+
+
+def test_gated_delta_chunk_d64_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300, 7])
+    q, k, v, g, beta = _inputs(1, int(cu[-1]), 2, 64, 64, torch.bfloat16, 61)
+    _check_chunk(la, oracle_mod, q, k, v, g, beta, cu=cu, garbage=True)

@@ -72,15 +72,16 @@ def test_gated_delta_workspace_size(lib):
     """The chunked gated delta rule keeps W and T diag(beta) V, bf16 [B, T, H, 128]
     each, the 64 prefix sums b_i and key norms 1/|k_i| of every (chunk slot, head) in fp32, and
     n_seqs + 1 chunk offsets for a packed batch, whose slot count is bounded by
-    ceil(T / 64) + n_seqs (each region 256-byte aligned); shapes that take the
-    token-by-token kernel need nothing."""
+    ceil(T / 64) + n_seqs (each region 256-byte aligned); head dims of 64 use the
+    same 128-wide layout; shapes that take the token-by-token kernel need nothing."""
     ws = lib.la_fwd_gated_delta_workspace_size
     bad = ctypes.c_size_t(-1).value
     wu = 8 * 4096 * 16 * 128 * 2
     assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 0) == 2 * wu + (8 * 64) * 16 * 512
     assert ws(1, 1000, 3, 128, 128, 5, 1, 1, 0) == 2 * 768000 + (16 + 5) * 3 * 512 + 256
     assert ws(1, 3, 1, 128, 128, 100, 1, 1, 0) == 2 * 768 + 101 * 512 + 512
-    assert ws(8, 4096, 16, 64, 64, 8, 0, 1, 0) == 0      # d = 64: token-by-token kernel
+    assert ws(8, 4096, 16, 64, 64, 8, 0, 1, 0) == 2 * wu + (8 * 64) * 16 * 512  # d = 64: the 128 layout
+    assert ws(8, 4096, 16, 256, 256, 8, 0, 1, 0) == 0    # d = 256: token-by-token kernel
     assert ws(8, 4096, 16, 128, 128, 8, 0, 0, 0) == 0    # f32
     assert ws(8, 4096, 16, 128, 128, 8, 0, 1, 1) == 0    # LA_FLAG_SIMT
     assert ws(8, 4096, 16, 96, 128, 8, 0, 1, 0) == bad   # head dim
