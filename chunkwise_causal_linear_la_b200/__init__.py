@@ -25,6 +25,7 @@ from .binding import (  # noqa: F401
     host_arena_size,
     la_fwd_chunk_host,
     la_bwd_chunk,
+    la_bwd_chunk_gated,
     la_fwd_chunk,
     la_fwd_chunk_gated,
     la_fwd_chunk_normgate,

@@ -498,10 +498,13 @@ la_status la_norm_gate(const la_tensor *o, const la_tensor *gate, const float *w
   return ok();
 }
 
-la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
-                       const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
-                       const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
-                       void *stream) {
+// The backward of la_fwd_chunk (g == NULL: per-head decay gamma) or of
+// la_fwd_chunk_gated's unnormalised form (g: per-token log decay; dg receives
+// its gradient).
+static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                            const float *gamma, const float *g, float *dg, const int32_t *cu_seqlens, int64_t n_seqs,
+                            int32_t chunk, int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv,
+                            int32_t flags, void *stream) {
   la_status s;
   const la_tensor *ts[7] = {q, k, v, dout, dq, dk, dv};
   const char *names[7] = {"q", "k", "v", "dout", "dq", "dk", "dv"};
@@ -515,7 +518,9 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
   if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
-  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!gamma && !g) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (g && (!dg || ((uintptr_t)g) % 4 || ((uintptr_t)dg) % 4))
+    return fail(LA_ERR_INVALID_ARG, "g and dg must be non-NULL, 4-byte aligned [B, T, H] float arrays");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
   if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (cu_seqlens) {
@@ -562,7 +567,7 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
   const bool elu = phi == LA_PHI_ELU1;
   ChunkArgs f;
   f.gamma = gamma;
-  f.g = nullptr;
+  f.g = g;
   f.cu_seqlens = cu_seqlens;
   f.final_state = nullptr;
   f.final_z = nullptr;
@@ -602,30 +607,58 @@ la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *
       return launch_chunk_tc(f, nullptr, 0, st, &why);
     };
     const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D;
+    // per-token decay: dg_t = sum_{s>=t} (phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s), the row
+    // dot products taken while the gradients are still those of phi(q), phi(k)
+    auto grad_of_x = [&](const la_tensor *x, const la_tensor *gx, float sign, bool accumulate) -> cudaError_t {
+      if (g) return launch_dg_terms(view(x), view(gx), dg, B, T, H, Dk, sign, phi, accumulate, elu, q->dtype, st);
+      return elu ? launch_mul_dphi(view(x), view(gx), B, T, H, Dk, q->dtype, st) : cudaSuccess;
+    };
     if (elu) {
       if ((err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
           (err = run(v, dout, dq, dk, 0, 1)) != cudaSuccess ||
-          (err = launch_mul_dphi(view(k), view(dk), B, T, H, Dk, q->dtype, st)) != cudaSuccess ||
+          (err = grad_of_x(k, dk, -1.f, false)) != cudaSuccess ||
           (err = launch_phi_copy(view(k), view(dv), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
           (err = run(dout, v, dv, dq, 0, 0)) != cudaSuccess ||
-          (err = launch_mul_dphi(view(q), view(dq), B, T, H, Dk, q->dtype, st)) != cudaSuccess ||
+          (err = grad_of_x(q, dq, 1.f, true)) != cudaSuccess ||
           (err = run(k, q, dout, dv, 1, 1)) != cudaSuccess)
         return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
                     why ? why : "");
     } else {
       if ((err = run(v, dout, q, dk, 0, 1)) != cudaSuccess || (err = run(dout, v, k, dq, 0, 0)) != cudaSuccess ||
-          (err = run(k, q, dout, dv, 0, 1)) != cudaSuccess)
+          (err = run(k, q, dout, dv, 0, 1)) != cudaSuccess || (err = grad_of_x(k, dk, -1.f, false)) != cudaSuccess ||
+          (err = grad_of_x(q, dq, 1.f, true)) != cudaSuccess)
         return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
                     why ? why : "");
     }
+    if (g && (err = launch_dg_rev_cumsum(dg, cu_seqlens, n_seqs, T, H, st)) != cudaSuccess)
+      return fail(LA_ERR_CUDA, "backward (log decay gradient): %s", cudaGetErrorString(err));
     return ok();
   }
+  if (g)
+    return fail(LA_ERR_UNSUPPORTED, "the per-token-decay backward runs on the tensor cores only: bf16, chunk 64, "
+                "d_k in {64, 128, 256} with d_v as la_fwd_chunk_path allows (d_k = d_v with elu + 1)");
   if (!bwd_supported(a, device))
     return fail(LA_ERR_UNSUPPORTED, "d_k %d x d_v %d does not fit the backward kernel's shared memory", a.dk,
                 a.dv);
   err = launch_bwd(a, st);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(err));
   return ok();
+}
+
+la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                       const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                       const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
+                       void *stream) {
+  return bwd_common(q, k, v, dout, gamma, nullptr, nullptr, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags,
+                    stream);
+}
+
+la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                             const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                             const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, float *dg, int32_t flags,
+                             void *stream) {
+  if (!g) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  return bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags, stream);
 }
 
 la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,

@@ -77,6 +77,86 @@ __global__ void __launch_bounds__(kEwThreads) mul_dphi_kernel(TensorView x, Tens
   }
 }
 
+// Gradient of the log decays (per-token decay backward), first step.  With b the
+// prefix sum of the log decays g, the loss depends on b_s through the weights
+// exp(b_i - b_j) of o_i = sum_{j<=i} exp(b_i - b_j) (qh_i . kh_j) v_j, so
+// dL/db_s = qh_s . dqh_s - kh_s . dkh_s (the gradients with respect to qh = phi(q),
+// kh = phi(k)), and dg_t = sum_{s>=t} dL/db_s.  This kernel adds
+// sign * phi(x_row) . grad_row to dg[row] (or stores it), and with apply_dphi
+// turns grad (with respect to phi(x)) into the gradient with respect to x in
+// place (times phi'(x) = 1 for x > 0, e^x otherwise).  LPR lanes share a row,
+// each with one 16-byte vector; rows are ordered (b, t, h) like dg [B, T, H].
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) dg_terms_kernel(TensorView x, TensorView grad, float *dg, int64_t T_,
+                                                               int64_t H, int D, int64_t rows, float sign, int phi,
+                                                               int accumulate, int apply_dphi) {
+  constexpr int VW = Vec<T>::VW;
+  const int lpr = D / VW;  // lanes per row (a power of two dividing 32)
+  const int lane = threadIdx.x & 31, sub = lane % lpr;
+  const int64_t rows_per_step = (int64_t)gridDim.x * (kEwThreads / lpr);
+  for (int64_t row0 = blockIdx.x * (int64_t)(kEwThreads / lpr); row0 < rows; row0 += rows_per_step) {
+    const int64_t row = row0 + threadIdx.x / lpr;
+    float acc = 0.f;
+    if (row < rows) {
+      const int64_t h = row % H, bt = row / H, t = bt % T_, b = bt / T_;
+      const uint4 xr = *reinterpret_cast<const uint4 *>((const T *)x.data + b * x.sb + t * x.st + h * x.sh + sub * VW);
+      uint4 *gp = reinterpret_cast<uint4 *>((T *)grad.data + b * grad.sb + t * grad.st + h * grad.sh + sub * VW);
+      uint4 gr = *gp;
+      const T *xv = reinterpret_cast<const T *>(&xr);
+      T *gv = reinterpret_cast<T *>(&gr);
+#pragma unroll
+      for (int u = 0; u < VW; ++u) {
+        const float xf = to_f32<T>(xv[u]), gf = to_f32<T>(gv[u]);
+        acc = fmaf(feature_map(xf, phi), gf, acc);
+        if (apply_dphi) gv[u] = from_f32<T>(gf * (xf > 0.f ? 1.f : expf(xf)));
+      }
+      if (apply_dphi) *gp = gr;
+    }
+    for (int o = lpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (row < rows && sub == 0) dg[row] = (accumulate ? dg[row] : 0.f) + sign * acc;
+  }
+}
+
+// Second step: dg_t <- sum_{s >= t} dg_s over each sequence, in place.  One CTA
+// per (sequence, head) walks the sequence from its end in tiles of kEwThreads
+// tokens: a block-wide inclusive scan in reversed order plus the running total.
+__global__ void __launch_bounds__(kEwThreads) dg_rev_cumsum_kernel(float *dg, const int32_t *cu, int64_t T_,
+                                                                    int64_t H) {
+  __shared__ float wsum[kEwThreads / 32];
+  const int64_t unit = blockIdx.x;
+  const int64_t h = unit % H, n = unit / H;
+  int64_t row0, len;  // token row of the sequence's first token in the [B * T] grid, and its length
+  if (cu) {
+    row0 = cu[n];
+    len = (int64_t)cu[n + 1] - cu[n];
+  } else {
+    row0 = n * T_;
+    len = T_;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float carry = 0.f;
+  for (int64_t k0 = 0; k0 < len; k0 += kEwThreads) {
+    const int64_t k = k0 + tid;  // k-th token from the end
+    const int64_t t = len - 1 - k;
+    float x = k < len ? dg[(row0 + t) * H + h] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    float before = carry;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    float tile = 0.f;
+#pragma unroll
+    for (int w = 0; w < kEwThreads / 32; ++w) tile += wsum[w];
+    if (k < len) dg[(row0 + t) * H + h] = x + before;
+    carry += tile;
+    __syncthreads();  // wsum is rewritten by the next tile
+  }
+}
+
 unsigned ew_grid(int64_t n) {
   const int64_t blocks = (n + kEwThreads - 1) / kEwThreads;
   return (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
@@ -109,6 +189,36 @@ cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T,
     mul_dphi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
   else
     mul_dphi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
+  return cudaGetLastError();
+}
+
+// dg[row] (+)= sign * phi(x_row) . grad_row, grad optionally times phi'(x) in place
+// (rows of 16-byte aligned vectors; D / VW a power of two, at most 32).
+cudaError_t launch_dg_terms(TensorView x, TensorView grad, float *dg, int64_t B, int64_t T, int64_t H, int64_t D,
+                            float sign, int phi, bool accumulate, bool apply_dphi, int dtype, cudaStream_t stream) {
+  const int vw = dtype == LA_F32 ? 4 : 8;
+  const int lpr = (int)(D / vw);
+  if (D % vw || lpr < 1 || lpr > 32 || (lpr & (lpr - 1))) return cudaErrorInvalidValue;
+  const int64_t rows = B * T * H;
+  if (rows == 0) return cudaSuccess;
+  const int64_t blocks = (rows + kEwThreads / lpr - 1) / (kEwThreads / lpr);
+  const unsigned grid = (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
+  if (dtype == LA_F32)
+    dg_terms_kernel<float><<<grid, kEwThreads, 0, stream>>>(x, grad, dg, T, H, (int)D, rows, sign, phi, accumulate,
+                                                             apply_dphi);
+  else
+    dg_terms_kernel<__nv_bfloat16><<<grid, kEwThreads, 0, stream>>>(x, grad, dg, T, H, (int)D, rows, sign, phi,
+                                                                     accumulate, apply_dphi);
+  return cudaGetLastError();
+}
+
+// dg_t <- sum_{s >= t} dg_s within each sequence (dense batch, or packed by cu_seqlens).
+cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,
+                                 cudaStream_t stream) {
+  const int64_t units = n_seqs * H;
+  if (units == 0 || T == 0) return cudaSuccess;
+  if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dg_rev_cumsum_kernel<<<(unsigned)units, kEwThreads, 0, stream>>>(dg, cu_seqlens, T, H);
   return cudaGetLastError();
 }
 

@@ -87,6 +87,10 @@ cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T
                             int dtype, cudaStream_t stream);
 cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
                             cudaStream_t stream);
+cudaError_t launch_dg_terms(TensorView x, TensorView grad, float *dg, int64_t B, int64_t T, int64_t H, int64_t D,
+                            float sign, int phi, bool accumulate, bool apply_dphi, int dtype, cudaStream_t stream);
+cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,
+                                 cudaStream_t stream);
 cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,
                              int64_t T, int64_t H, int dv, int dtype, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);

@@ -262,14 +262,19 @@ __device__ __forceinline__ void xform_tile(const uint8_t *src, uint8_t *dst, int
 // formula of the forward then holds in the primed indices (valid rows
 // i' < C', causal j' <= i'); the tiles stay in natural row order, so the
 // products need no change.  This runs the anti-causal sums of the backward
-// pass (sum over i >= j) on the same kernel.
+// pass (sum over i >= j) on the same kernel.  With a per-token decay the
+// anti-causal weight exp(b_i - b_j), i >= j, is the product of the decays of
+// tokens j+1 .. i; in reversed positions that is the forward's weight for the
+// decays shifted by one token, g''(i') = g(token of i' + 1), which is what
+// the transform warps load (zero for the last token of the sequence, whose
+// reversed predecessor state is zero).
 // NG: the output RMSNorm with a Swish gate in the epilogue (d_v == DVT).
 template <int DK, int DVT, int C, int NS, bool NORM, bool ELU, int MODE, bool GATED, bool REV, bool NG = false>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
   using G = Cfg<DK, DVT, C, NS>;
-  static_assert(!(REV && (NORM || GATED)), "reverse time is built for the unnormalised per-head decay");
+  static_assert(!(REV && NORM), "reverse time is built for the unnormalised forms");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *z = reinterpret_cast<float *>(sm + G::OFF_Z);
@@ -646,9 +651,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float blo = 0.f, bhi = 0.f, blast = 0.f;
         if (GATED) {
           const int ln = tt & 31;
-          const int64_t row0 = (int64_t)bidx * a.T + start + (int64_t)c * C;
-          blo = ln < Cp ? a.g[(row0 + ln) * a.H + h] : 0.f;
-          bhi = ln + 32 < Cp ? a.g[(row0 + ln + 32) * a.H + h] : 0.f;
+          if (REV) {  // position p: the decay of the token after it (reversed order), none after the last
+            const int64_t after0 = (int64_t)bidx * a.T + rend - (int64_t)c * C;  // token after position 0
+            blo = (ln < Cp && (c > 0 || ln > 0)) ? a.g[(after0 - ln) * a.H + h] : 0.f;
+            bhi = ln + 32 < Cp ? a.g[(after0 - ln - 32) * a.H + h] : 0.f;
+          } else {
+            const int64_t row0 = (int64_t)bidx * a.T + start + (int64_t)c * C;
+            blo = ln < Cp ? a.g[(row0 + ln) * a.H + h] : 0.f;
+            bhi = ln + 32 < Cp ? a.g[(row0 + ln + 32) * a.H + h] : 0.f;
+          }
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const float y0 = __shfl_up_sync(0xffffffffu, blo, o);
@@ -673,10 +684,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             const int j = (tt >> 3) + 8 * m;
-            if (GATED) {
-              const float b0 = __shfl_sync(0xffffffffu, blo, j & 31);
-              const float b1 = __shfl_sync(0xffffffffu, bhi, j & 31);
-              wv[m] = j < Cp ? exp_fast(blast - (j < 32 ? b0 : b1)) : 0.f;
+            if (GATED) {  // the table is indexed by position (reversed order in reverse time)
+              const int jp = lrow(j);
+              const float b0 = __shfl_sync(0xffffffffu, blo, jp & 31);
+              const float b1 = __shfl_sync(0xffffffffu, bhi, jp & 31);
+              wv[m] = jp < Cp ? exp_fast(blast - (jp < 32 ? b0 : b1)) : 0.f;
             } else {
               const int jl = lrow(j);
               wv[m] = jl < Cp ? pw[Cp - 1 - jl] : 0.f;
@@ -918,7 +930,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float bi = 0.f;
       if (GATED) {  // the stage's decay table (published before the score MMA's inputs)
         if (!wait_bar_warp(sy, G::B_XFORM + c % NS, (c / NS) & 1, c)) return 0.f;
-        bi = dt[i];
+        bi = dt[lrow(i)];
         gi = exp_fast(bi);
       } else {
         gi = pw[lrow(i) + 1];
@@ -939,6 +951,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!vd_mode) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) f[e] = (hf * 32 + e >= i && row_ok) ? __uint_as_float(r[e]) : 0.f;
+        } else if (GATED) {  // P_ij = A_ij exp(b''_i' - b''_j') over reversed positions
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = hf * 32 + e;
+            f[e] = (j >= i && row_ok) ? __uint_as_float(r[e]) * exp_fast(bi - dt[lrow(j)]) : 0.f;
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -1368,8 +1386,11 @@ cudaError_t launch_shape_gated(const ChunkArgs &a, void *workspace, cudaStream_t
 
 template <int DK, int DVT, int NS>
 cudaError_t launch_shape(const ChunkArgs &a, void *workspace, cudaStream_t stream, const char **why) {
-  if (a.rev) {  // reverse time (the backward pass): unnormalised, per-head decay
-    if (a.normalize || a.g) return cudaErrorInvalidValue;
+  if (a.rev) {  // reverse time (the backward pass): unnormalised, per-head or per-token decay
+    if (a.normalize) return cudaErrorInvalidValue;
+    if (a.g)
+      return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, true, true>(a, workspace, stream, why)
+                   : launch_cfg<DK, DVT, 64, NS, false, false, true, true>(a, workspace, stream, why);
     return a.phi ? launch_cfg<DK, DVT, 64, NS, false, true, false, true>(a, workspace, stream, why)
                  : launch_cfg<DK, DVT, 64, NS, false, false, false, true>(a, workspace, stream, why);
   }

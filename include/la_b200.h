@@ -412,13 +412,42 @@ LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_
  * in fp32; it needs the d_k x d_v fp32 state and one chunk's tiles to fit in
  * shared memory (d_k = d_v = 128 fits; 256 does not: LA_ERR_UNSUPPORTED).
  * Tokens outside every sequence of a packed batch may be overwritten in dq,
- * dk, dv.  The normalised forward has no backward here.  Other errors as for
- * la_fwd_chunk.
+ * dk, dv.  The normalised forward has no backward here (the per-token decay's
+ * is la_bwd_chunk_gated).  Other errors as for la_fwd_chunk.
  */
 LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                               const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
                               int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv,
                               int32_t flags, void *stream);
+
+/*
+ * la_bwd_chunk_gated -- backward of la_fwd_chunk_gated's unnormalised forward
+ * (the data-dependent decay of "1.6 长上下文与高效注意力", section 状态空间模型与
+ * Mamba: alpha_t = exp(g_t) per token and head), including the gradient of the
+ * log decays.  With b the prefix sum of g over each sequence,
+ *     o_i = sum_{j<=i} exp(b_i - b_j) (phi(q_i) . phi(k_j)) v_j,
+ * so the gradients of phi(q), phi(k), v have la_bwd_chunk's three sums with
+ * exp(b_i - b_j) in place of gamma^(i-j), and, because the loss sees b_s only
+ * through those weights,
+ *     dg_t = sum_{s >= t} (phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s).
+ *   q, k, v, cu_seqlens, n_seqs, chunk, phi  as for la_fwd_chunk_gated.
+ *   g           device float[B, T, H], the forward's log decays (<= 0).
+ *   dout        [B, T, H, d_v], q's dtype: the gradient at `out`.
+ *   dq, dk, dv  as for la_bwd_chunk.
+ *   dg          device float[B, T, H]: the gradient with respect to g (fp32
+ *               arithmetic: row dot products, then a reverse cumulative sum per
+ *               sequence and head); 4-byte aligned.
+ * Kernels: the tensor cores only: bf16, chunk 64, head dims for which
+ * la_fwd_chunk_path reports LA_PATH_TENSOR_CORE (with elu + 1 also
+ * d_k == d_v); the two reverse-time passes take, at each reversed position,
+ * the decay of the token after it.  Other shapes, f32 and LA_FLAG_SIMT return
+ * LA_ERR_UNSUPPORTED.  Other errors as for la_bwd_chunk.
+ */
+LA_API la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                    const la_tensor *dout, const float *g, const int32_t *cu_seqlens,
+                                    int64_t n_seqs, int32_t chunk, int32_t phi, const la_tensor *dq,
+                                    const la_tensor *dk, const la_tensor *dv, float *dg, int32_t flags,
+                                    void *stream);
 
 /*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device

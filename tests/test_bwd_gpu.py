@@ -131,3 +131,113 @@ def test_bwd_tc_matches_simt(la):
 
 def test_bwd_device_error_word_clear(la):
     assert la.device_error(reset=True) == (0, 0)
+
+
+# ---------------------------------------------------------------- per-token decay backward
+# la_bwd_chunk_gated against oracle.backward_gated (dq, dk, dv and dg, the gradient of
+# the log decays): bf16 on the tensor cores, three passes with the per-token decay
+# (the two reverse-time ones taking each position's following decay), then dg from
+# the row dot products and a reverse cumulative sum per sequence and head.
+def _check_gated(la, oracle_mod, q, k, v, dout, g, cu=None, phi="identity"):
+    dev = torch.device("cuda")
+    dq, dk, dv, dg = la.la_bwd_chunk_gated(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), g.to(dev),
+                                           cu_seqlens=None if cu is None else cu.to(dev), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_error(reset=True) == (0, 0)
+    rq, rk, rv, rg = oracle_mod.backward_gated(q, k, v, dout, g.double().numpy(),
+                                               cu_seqlens=None if cu is None else cu.numpy(), phi=phi)
+    B, T = q.shape[:2]
+    sl = seq_slices(B, T, None if cu is None else cu.tolist())
+    errs = [slice_rel_err(to_np(x), r, sl) for x, r in ((dq, rq), (dk, rk), (dv, rv))]
+    errs.append(_dg_err(to_np(dg), rg, q, k, rq, rk, phi, sl))
+    assert all(np.isfinite(to_np(x)).all() for x in (dq, dk, dv, dg))
+    assert max(errs) < TOL[torch.bfloat16], errs
+    return errs
+
+
+def _dg_err(dg, rg, q, k, rq, rk, phi, slices):
+    """dg_t is a reverse cumulative sum of the row terms phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s,
+    and is exactly 0 at a sequence's first token (its decay multiplies the zero initial state), so
+    a slice can be all zero (one token), and a single term can cancel to far below its parts.  Per
+    (sequence, head) slice the error is taken relative to the larger of max |dg_ref| and the largest
+    single-token absolute sum sum_c |phi(q)_c dphi(q)_c| + |phi(k)_c dphi(k)_c| (the scale of a dot
+    product's rounding error), rebuilt in float64 from the oracle's dq, dk (dphi(x) = dx / phi'(x),
+    phi' > 0).  On sequences longer than a few tokens max |dg_ref| is the larger."""
+    qf, kf = q.double().numpy(), k.double().numpy()
+    if phi == "elu1":
+        fq, fk = np.where(qf > 0, qf + 1, np.exp(np.minimum(qf, 0))), np.where(kf > 0, kf + 1, np.exp(np.minimum(kf, 0)))
+        dfq, dfk = rq / np.where(qf > 0, 1.0, np.exp(np.minimum(qf, 0))), rk / np.where(kf > 0, 1.0, np.exp(np.minimum(kf, 0)))
+    else:
+        fq, fk, dfq, dfk = qf, kf, rq, rk
+    term = np.sum(np.abs(fq * dfq), -1) + np.sum(np.abs(fk * dfk), -1)  # [B, T, H]
+    worst = 0.0
+    for b, s0, e0 in slices:
+        if e0 <= s0:
+            continue
+        for h in range(rg.shape[2]):
+            scale = max(np.max(np.abs(rg[b, s0:e0, h])), np.max(term[b, s0:e0, h]))
+            worst = max(worst, float(np.max(np.abs(dg[b, s0:e0, h] - rg[b, s0:e0, h])) / scale))
+    return worst
+
+
+def _log_decay(B, T, H, lo, hi, seed):
+    from chunkwise_causal_linear_la_b200.workloads import make_log_decay
+
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    return make_log_decay(B, T, H, lo, hi, gen)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("T", [1, 65, 300])
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+def test_bwd_gated_shapes(la, oracle_mod, d, T, phi):
+    q, k, v, dout = _inputs(2, T, 2, d, d, torch.bfloat16, 500 + T + d)
+    g = _log_decay(2, T, 2, 0.9, 0.999, 600 + T)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, phi=phi)
+
+
+@pytest.mark.parametrize("lo,hi", [(0.05, 0.5), (0.5, 0.99), (0.999, 1.0)])
+def test_bwd_gated_decay_ranges(la, oracle_mod, lo, hi):
+    """Strong decays (a 64-token chunk's decay underflows), mild ones and none at all."""
+    q, k, v, dout = _inputs(1, 400, 3, 128, 128, torch.bfloat16, 31)
+    g = _log_decay(1, 400, 3, lo, hi, 32)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, phi="elu1")
+
+
+def test_bwd_gated_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 2, 128, 128, torch.bfloat16, 33)
+    g = _log_decay(1, int(cu[-1]), 2, 0.8, 0.999, 34)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, cu=cu)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, cu=cu, phi="elu1")
+
+
+def test_bwd_gated_long_sequence_dg(la, oracle_mod):
+    """A 4000-token sequence: dg sums up to 4000 row terms per head in fp32."""
+    q, k, v, dout = _inputs(1, 4000, 2, 128, 128, torch.bfloat16, 35)
+    g = _log_decay(1, 4000, 2, 0.95, 0.999, 36)
+    _check_gated(la, oracle_mod, q, k, v, dout, g)
+
+
+def test_bwd_gated_constant_decay_equals_per_head_backward(la):
+    """A per-token decay constant in time gives la_bwd_chunk's dq, dk, dv for gamma = exp(g)."""
+    dev = torch.device("cuda")
+    q, k, v, dout = (x.to(dev) for x in _inputs(2, 300, 2, 128, 128, torch.bfloat16, 37))
+    lg = torch.log(torch.tensor([0.97, 0.999]))
+    g = lg.reshape(1, 1, 2).expand(2, 300, 2).contiguous().to(dev)
+    a = la.la_bwd_chunk_gated(q, k, v, dout, g, phi="elu1")[:3]
+    b = la.la_bwd_chunk(q, k, v, dout, torch.exp(lg).to(dev), phi="elu1")
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert slice_rel_err(to_np(x), to_np(y), seq_slices(2, 300)) < TOL[torch.bfloat16]
+
+
+def test_bwd_gated_unsupported_shapes(la):
+    dev = torch.device("cuda")
+    q, k, v, dout = (x.to(dev) for x in _inputs(1, 50, 2, 128, 128, torch.float32, 39))
+    g = _log_decay(1, 50, 2, 0.9, 0.99, 40).to(dev)
+    with pytest.raises(la.LaError):
+        la.la_bwd_chunk_gated(q, k, v, dout, g)  # f32: the tensor cores only
