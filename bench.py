@@ -185,6 +185,8 @@ def _oracle_run(oracle, w, q, k, v, gamma, g=None, bwd=False, beta=None):
     if bwd:
         import torch
 
+        if g is not None:
+            return oracle.backward_gated(q, k, v, torch.ones_like(v), g, phi=w.phi)
         return oracle.backward(q, k, v, torch.ones_like(v), gamma, phi=w.phi)
     if g is not None:
         return oracle.recurrent_gated(q, k, v, g, phi=w.phi, normalize=w.normalize)[:2]
@@ -512,12 +514,14 @@ def main():
 
     gd = x.get("g")  # data-dependent log decay (gated workloads)
     if args.bwd:
-        if gd is not None or w.normalize:
-            raise SystemExit("--bwd covers the unnormalised per-head-decay workloads")
+        if w.normalize or x.get("beta") is not None:
+            raise SystemExit("--bwd covers the unnormalised forwards (per-head or per-token decay)")
         from chunkwise_causal_linear_la_b200.workloads import make_dout
 
         dout = make_dout(v, seed=rank_seed(rank))
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        if gd is not None:  # the per-token decay's backward also returns dg
+            grads = grads + (torch.empty_like(gd),)
 
     if args.normgate:
         if gd is not None or args.bwd:
@@ -538,6 +542,9 @@ def main():
         elif args.normgate:
             la.la_fwd_chunk_normgate(q, k, v, g, ng_gate, ng_w, eps=1e-5, cu_seqlens=cu, chunk=w.chunk, phi=w.phi,
                                      normalize=w.normalize, out=out, final_state=fs, workspace=wsbuf, stream=stream)
+        elif args.bwd and gd is not None:
+            la.la_bwd_chunk_gated(q, k, v, dout, gd, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0],
+                                  dk=grads[1], dv=grads[2], dg=grads[3], stream=stream)
         elif args.bwd:
             la.la_bwd_chunk(q, k, v, dout, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0], dk=grads[1],
                             dv=grads[2], stream=stream)
@@ -587,13 +594,18 @@ def main():
     if args.bwd:  # read q, k, v, dout; write dq, dk, dv (no final state); three forward-shaped passes of flops
         e_ = 2 if w.dtype == "bf16" else 4
         alg_bytes = tokens * w.H * e_ * (4 * w.d_k + 3 * w.d_v)
+        if gd is not None:  # read g, write dg (fp32 per token and head)
+            alg_bytes += tokens * w.H * 8
         alg_flops = 3 * alg_flops
     roof = _roofline(alg_bytes, alg_flops, launch_ms, hbm_peak, tc_peak)
-    # kernels launched per step: segmented sequences take a state pass, a scan and the output pass; the
-    # backward takes three forward-shaped passes (plus four elementwise kernels with elu + 1)
+    # kernels launched per step: segmented sequences take a state pass, a scan and the output pass
     # (a packed batch with a workspace has its longest-first order computed first: 2 launches)
-    launches_per_step = (7 if w.phi == "elu1" else 3) if args.bwd else (
+    # (backward: three tensor-core passes, two phi copies with elu + 1, and with a per-token decay the
+    # reverse cumulative sum of dg, whose row terms the passes' epilogues add)
+    launches_per_step = (5 if w.phi == "elu1" else 3) if args.bwd else (
         (2 if cu is not None else 3) if nws > 0 else 1)
+    if args.bwd and gd is not None:
+        launches_per_step += 1
     if gbeta is not None:  # chunk offsets (packed batches), the per-chunk WY pass, the sequential pass
         launches_per_step = (3 if cu is not None else 2) if nws > 0 else 1
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -613,9 +625,13 @@ def main():
             s0, e0_ = (0, T) if cu is None else (int(cu[0]), int(cu[1]))
             bb = b if cu is None else 0
             cut = lambda t: t[bb:bb + 1, s0:e0_, h:h + 1].cpu()  # noqa: E731
-            refs = oracle.backward(cut(q), cut(k), cut(v), cut(dout), [float(g[h])], phi=w.phi)
+            if gd is not None:
+                refs = oracle.backward_gated(cut(q), cut(k), cut(v), cut(dout),
+                                             gd[bb:bb + 1, s0:e0_, h:h + 1].double().cpu().numpy(), phi=w.phi)
+            else:
+                refs = oracle.backward(cut(q), cut(k), cut(v), cut(dout), [float(g[h])], phi=w.phi)
             for got, ref in zip(grads, refs):
-                o = cut(got).float().numpy()
+                o = (cut(got) if got.dim() == 4 else got[bb:bb + 1, s0:e0_, h:h + 1].cpu()).double().numpy()
                 worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))))
         for b, h in [] if args.bwd else sl:
             if cu is None:
@@ -650,7 +666,7 @@ def main():
     if args.normgate:
         inputs = (q, k, v, ng_gate)
     if args.bwd:
-        inputs = (q, k, v, dout)
+        inputs = (q, k, v, dout) if gd is None else (q, k, v, dout, gd)
     if plain:
         inputs = (q, k, v, g) + (() if cu is None else (cu,))
     outputs = grads if args.bwd else (out, fs)

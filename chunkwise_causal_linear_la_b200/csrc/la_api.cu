@@ -157,6 +157,10 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
   a.dtype = q->dtype;
   a.rev = 0;
   a.noseg = 0;
+  a.ex = TensorView{nullptr, 0, 0, 0};
+  a.edg = nullptr;
+  a.esign = 0.f;
+  a.ephi = a.edphi = 0;
   a.ng_w = nullptr;
   a.ng_gate = TensorView{nullptr, 0, 0, 0};
   a.ng_eps = 0.f;
@@ -582,6 +586,10 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   f.ng_w = nullptr;
   f.ng_gate = TensorView{nullptr, 0, 0, 0};
   f.ng_eps = 0.f;
+  f.ex = TensorView{nullptr, 0, 0, 0};
+  f.edg = nullptr;
+  f.esign = 0.f;
+  f.ephi = f.edphi = 0;
   auto setup = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
                    int rev) {
     f.q = view(qq);
@@ -601,32 +609,39 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   if (tc) tc = setup(v, dout, q, dk, 0, 1) && setup(dout, v, k, dq, 0, 0) && setup(k, q, dout, dv, 1, 1);
   if (tc) {
     const char *why = nullptr;
+    // x: the forward input whose gradient this pass produces (k for dphi(k), q for dphi(q)); the
+    // pass's epilogue then scales by phi'(x) (elu + 1) and, with a per-token decay, adds the row
+    // term of dg_t = sum_{s>=t} (phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s), both from the fp32
+    // accumulators before rounding
     auto run = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
-                   int rev) -> cudaError_t {
+                   int rev, const la_tensor *x = nullptr, float sign = 0.f) -> cudaError_t {
       setup(qq, kk, vv, oo, ph, rev);
-      return launch_chunk_tc(f, nullptr, 0, st, &why);
+      f.ex = x ? view(x) : TensorView{nullptr, 0, 0, 0};
+      f.edg = x && g ? dg : nullptr;
+      f.esign = sign;
+      f.ephi = phi;
+      f.edphi = elu ? 1 : 0;
+      const cudaError_t e = launch_chunk_tc(f, nullptr, 0, st, &why);
+      f.ex = TensorView{nullptr, 0, 0, 0};
+      f.edg = nullptr;
+      return e;
     };
     const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D;
-    // per-token decay: dg_t = sum_{s>=t} (phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s), the row
-    // dot products taken while the gradients are still those of phi(q), phi(k)
-    auto grad_of_x = [&](const la_tensor *x, const la_tensor *gx, float sign, bool accumulate) -> cudaError_t {
-      if (g) return launch_dg_terms(view(x), view(gx), dg, B, T, H, Dk, sign, phi, accumulate, elu, q->dtype, st);
-      return elu ? launch_mul_dphi(view(x), view(gx), B, T, H, Dk, q->dtype, st) : cudaSuccess;
-    };
+    const bool epi = g || elu;  // the dk and dq passes need x in their epilogue
+    if (g && (err = cudaMemsetAsync(dg, 0, (size_t)(B * T * H) * sizeof(float), st)) != cudaSuccess)
+      return fail(LA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     if (elu) {
       if ((err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
-          (err = run(v, dout, dq, dk, 0, 1)) != cudaSuccess ||
-          (err = grad_of_x(k, dk, -1.f, false)) != cudaSuccess ||
+          (err = run(v, dout, dq, dk, 0, 1, k, -1.f)) != cudaSuccess ||
           (err = launch_phi_copy(view(k), view(dv), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess ||
-          (err = run(dout, v, dv, dq, 0, 0)) != cudaSuccess ||
-          (err = grad_of_x(q, dq, 1.f, true)) != cudaSuccess ||
+          (err = run(dout, v, dv, dq, 0, 0, q, 1.f)) != cudaSuccess ||
           (err = run(k, q, dout, dv, 1, 1)) != cudaSuccess)
         return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
                     why ? why : "");
     } else {
-      if ((err = run(v, dout, q, dk, 0, 1)) != cudaSuccess || (err = run(dout, v, k, dq, 0, 0)) != cudaSuccess ||
-          (err = run(k, q, dout, dv, 0, 1)) != cudaSuccess || (err = grad_of_x(k, dk, -1.f, false)) != cudaSuccess ||
-          (err = grad_of_x(q, dq, 1.f, true)) != cudaSuccess)
+      if ((err = run(v, dout, q, dk, 0, 1, epi ? k : nullptr, -1.f)) != cudaSuccess ||
+          (err = run(dout, v, k, dq, 0, 0, epi ? q : nullptr, 1.f)) != cudaSuccess ||
+          (err = run(k, q, dout, dv, 0, 1)) != cudaSuccess)
         return fail(LA_ERR_CUDA, "backward (tensor cores): %s%s%s", cudaGetErrorString(err), why ? ": " : "",
                     why ? why : "");
     }

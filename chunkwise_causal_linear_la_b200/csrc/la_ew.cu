@@ -1,11 +1,12 @@
-// la_ew.cu -- elementwise kernels: the steps of the backward pass with
-// phi = elu + 1, and the output RMSNorm with a Swish gate.
+// la_ew.cu -- elementwise kernels: the steps of the backward pass outside the
+// tensor-core passes, and the output RMSNorm with a Swish gate.
 //
-// The backward runs on the forward kernel (see la_bwd_chunk): operands that
-// the forward kernel reads untransformed must hold phi(x) already, and the
-// gradients of phi(q), phi(k) are turned into those of q, k by phi'(x) = 1 for
-// x > 0 and e^x otherwise ("1.6 长上下文与高效注意力", section 线性注意力:
-// phi(x) = elu(x) + 1).  Both kernels stream a [B, T, H, D] tensor once.
+// The backward runs on the forward kernel (see la_bwd_chunk): with phi = elu + 1
+// the operands that kernel reads untransformed must hold phi(x) already
+// ("1.6 长上下文与高效注意力", section 线性注意力: phi(x) = elu(x) + 1), which
+// phi_kernel writes in one pass over a [B, T, H, D] tensor (the passes' epilogues
+// apply phi'); the per-token decay's log-decay gradient ends in a reverse
+// cumulative sum per sequence and head.
 #include <cuda_bf16.h>
 
 #include "la_common.cuh"
@@ -54,70 +55,12 @@ __global__ void __launch_bounds__(kEwThreads) phi_kernel(TensorView src, TensorV
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kEwThreads) mul_dphi_kernel(TensorView x, TensorView grad, int64_t T_, int64_t H,
-                                                               int64_t D, int64_t nvec) {
-  constexpr int VW = Vec<T>::VW;
-  const int64_t nvr = D / VW;
-  for (int64_t e = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; e < nvec; e += (int64_t)gridDim.x * kEwThreads) {
-    int64_t b, t, h;
-    int col;
-    row_of<T>(e, nvr, T_, H, b, t, h, col);
-    const uint4 xr = *reinterpret_cast<const uint4 *>((const T *)x.data + b * x.sb + t * x.st + h * x.sh + col);
-    uint4 *gp = reinterpret_cast<uint4 *>((T *)grad.data + b * grad.sb + t * grad.st + h * grad.sh + col);
-    uint4 gr = *gp;
-    const T *xv = reinterpret_cast<const T *>(&xr);
-    T *gv = reinterpret_cast<T *>(&gr);
-#pragma unroll
-    for (int u = 0; u < VW; ++u) {
-      const float xf = to_f32<T>(xv[u]);
-      gv[u] = from_f32<T>(to_f32<T>(gv[u]) * (xf > 0.f ? 1.f : expf(xf)));
-    }
-    *gp = gr;
-  }
-}
-
-// Gradient of the log decays (per-token decay backward), first step.  With b the
-// prefix sum of the log decays g, the loss depends on b_s through the weights
-// exp(b_i - b_j) of o_i = sum_{j<=i} exp(b_i - b_j) (qh_i . kh_j) v_j, so
-// dL/db_s = qh_s . dqh_s - kh_s . dkh_s (the gradients with respect to qh = phi(q),
-// kh = phi(k)), and dg_t = sum_{s>=t} dL/db_s.  This kernel adds
-// sign * phi(x_row) . grad_row to dg[row] (or stores it), and with apply_dphi
-// turns grad (with respect to phi(x)) into the gradient with respect to x in
-// place (times phi'(x) = 1 for x > 0, e^x otherwise).  LPR lanes share a row,
-// each with one 16-byte vector; rows are ordered (b, t, h) like dg [B, T, H].
-template <typename T>
-__global__ void __launch_bounds__(kEwThreads) dg_terms_kernel(TensorView x, TensorView grad, float *dg, int64_t T_,
-                                                               int64_t H, int D, int64_t rows, float sign, int phi,
-                                                               int accumulate, int apply_dphi) {
-  constexpr int VW = Vec<T>::VW;
-  const int lpr = D / VW;  // lanes per row (a power of two dividing 32)
-  const int lane = threadIdx.x & 31, sub = lane % lpr;
-  const int64_t rows_per_step = (int64_t)gridDim.x * (kEwThreads / lpr);
-  for (int64_t row0 = blockIdx.x * (int64_t)(kEwThreads / lpr); row0 < rows; row0 += rows_per_step) {
-    const int64_t row = row0 + threadIdx.x / lpr;
-    float acc = 0.f;
-    if (row < rows) {
-      const int64_t h = row % H, bt = row / H, t = bt % T_, b = bt / T_;
-      const uint4 xr = *reinterpret_cast<const uint4 *>((const T *)x.data + b * x.sb + t * x.st + h * x.sh + sub * VW);
-      uint4 *gp = reinterpret_cast<uint4 *>((T *)grad.data + b * grad.sb + t * grad.st + h * grad.sh + sub * VW);
-      uint4 gr = *gp;
-      const T *xv = reinterpret_cast<const T *>(&xr);
-      T *gv = reinterpret_cast<T *>(&gr);
-#pragma unroll
-      for (int u = 0; u < VW; ++u) {
-        const float xf = to_f32<T>(xv[u]), gf = to_f32<T>(gv[u]);
-        acc = fmaf(feature_map(xf, phi), gf, acc);
-        if (apply_dphi) gv[u] = from_f32<T>(gf * (xf > 0.f ? 1.f : expf(xf)));
-      }
-      if (apply_dphi) *gp = gr;
-    }
-    for (int o = lpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (row < rows && sub == 0) dg[row] = (accumulate ? dg[row] : 0.f) + sign * acc;
-  }
-}
-
-// Second step: dg_t <- sum_{s >= t} dg_s over each sequence, in place.  One CTA
+// Gradient of the log decays (per-token decay backward).  With b the prefix sum of
+// the log decays g, the loss sees b_s only through the weights exp(b_i - b_j) of
+// o_i = sum_{j<=i} exp(b_i - b_j) (qh_i . kh_j) v_j, so dL/db_s = qh_s . dqh_s -
+// kh_s . dkh_s and dg_t = sum_{s>=t} dL/db_s.  The backward passes' epilogues add
+// the row terms into dg (chunk_tc_kernel); this kernel finishes the sum.
+// dg_t <- sum_{s >= t} dg_s over each sequence, in place.  One CTA
 // per (sequence, head) walks the sequence from its end in tiles of kEwThreads
 // tokens: a block-wide inclusive scan in reversed order plus the running total.
 __global__ void __launch_bounds__(kEwThreads) dg_rev_cumsum_kernel(float *dg, const int32_t *cu, int64_t T_,
@@ -176,39 +119,6 @@ cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T
     phi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
   else
     phi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
-                            cudaStream_t stream) {
-  const int vw = dtype == LA_F32 ? 4 : 8;
-  if (D % vw) return cudaErrorInvalidValue;
-  const int64_t n = B * T * H * (D / vw);
-  if (n == 0) return cudaSuccess;
-  if (dtype == LA_F32)
-    mul_dphi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
-  else
-    mul_dphi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(x, grad, T, H, D, n);
-  return cudaGetLastError();
-}
-
-// dg[row] (+)= sign * phi(x_row) . grad_row, grad optionally times phi'(x) in place
-// (rows of 16-byte aligned vectors; D / VW a power of two, at most 32).
-cudaError_t launch_dg_terms(TensorView x, TensorView grad, float *dg, int64_t B, int64_t T, int64_t H, int64_t D,
-                            float sign, int phi, bool accumulate, bool apply_dphi, int dtype, cudaStream_t stream) {
-  const int vw = dtype == LA_F32 ? 4 : 8;
-  const int lpr = (int)(D / vw);
-  if (D % vw || lpr < 1 || lpr > 32 || (lpr & (lpr - 1))) return cudaErrorInvalidValue;
-  const int64_t rows = B * T * H;
-  if (rows == 0) return cudaSuccess;
-  const int64_t blocks = (rows + kEwThreads / lpr - 1) / (kEwThreads / lpr);
-  const unsigned grid = (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
-  if (dtype == LA_F32)
-    dg_terms_kernel<float><<<grid, kEwThreads, 0, stream>>>(x, grad, dg, T, H, (int)D, rows, sign, phi, accumulate,
-                                                             apply_dphi);
-  else
-    dg_terms_kernel<__nv_bfloat16><<<grid, kEwThreads, 0, stream>>>(x, grad, dg, T, H, (int)D, rows, sign, phi,
-                                                                     accumulate, apply_dphi);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,14 @@ struct ChunkArgs {
   float ng_eps;
   int rev;    // 1: reverse time (tensor-core kernel only; used by the backward pass)
   int noseg;  // 1: never split sequences into segments (no workspace)
+  // Backward-pass epilogue (tensor-core kernel): with ex.data set, each output row o
+  // (fp32, before rounding) meets the row x of ex at the same token, head and
+  // columns (q's dtype): edg[row] += esign * phi(x) . o when edg is set (phi =
+  // ephi), and with edphi the row written is o * phi'(x) (elu + 1).  ex.data NULL: off.
+  TensorView ex;
+  float *edg;
+  float esign;
+  int ephi, edphi;
 };
 
 struct StepArgs {
@@ -85,10 +93,6 @@ bool simt_supported(const ChunkArgs &a, int device);
 bool bwd_supported(const BwdArgs &a, int device);
 cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T, int64_t H, int64_t D, int phi,
                             int dtype, cudaStream_t stream);
-cudaError_t launch_mul_dphi(TensorView x, TensorView grad, int64_t B, int64_t T, int64_t H, int64_t D, int dtype,
-                            cudaStream_t stream);
-cudaError_t launch_dg_terms(TensorView x, TensorView grad, float *dg, int64_t B, int64_t T, int64_t H, int64_t D,
-                            float sign, int phi, bool accumulate, bool apply_dphi, int dtype, cudaStream_t stream);
 cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,
                                  cudaStream_t stream);
 cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,

@@ -129,6 +129,14 @@ struct TcArgs {
   const void *ng_gate;
   int64_t ng_sb, ng_st, ng_sh;
   float ng_eps;
+  // Backward epilogue: the row x of ex (bf16, element strides) at each output row's token:
+  // edg[token][h] += esign * phi(x) . o (fp32 o, before rounding) when edg is set, and
+  // the row written is o * phi'(x) with edphi.  ex NULL: off.
+  const void *ex;
+  int64_t ex_sb, ex_st, ex_sh;
+  float *edg;
+  float esign;
+  int ephi, edphi;
 };
 
 template <int DK, int DVT, int C, int NS>
@@ -1043,6 +1051,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ss += __shfl_xor_sync(0xffffffffu, ss, 16);
         rstd = rsqrtf(ss / (float)DVT + a.ng_eps);
       }
+      float edot = 0.f;  // backward epilogue: this thread's part of phi(x) . o
       auto do_pass = [&](int pass) {
         float o[32];
         load_o(pass, o);
@@ -1052,6 +1061,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         const int col = hf * (DVT / 2) + pass * 32;
         if (lrow(i) < Cp && vt * DVT + col < a.dv) {
+          if (!NG && a.ex) {  // the row of x at this token: the dot takes o before phi' scales it
+            const uint4 *xs = reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const uint8_t *>(a.ex) +
+                2 * ((int64_t)bidx * a.ex_sb + otok * a.ex_st + (int64_t)h * a.ex_sh + vt * DVT + col));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float xf[8];
+              unpack8(xs[q], xf);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float xv = xf[u];
+                edot = fmaf(a.ephi ? phi_fast(xv) : xv, o[8 * q + u], edot);
+                if (a.edphi) o[8 * q + u] *= xv > 0.f ? 1.f : exp_fast(xv);
+              }
+            }
+          }
           if (NG) {  // y = o rstd w swish(gate)
             const uint4 *gsrc = reinterpret_cast<const uint4 *>(
                 reinterpret_cast<const uint8_t *>(a.ng_gate) +
@@ -1076,6 +1101,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
 #pragma unroll 1
       for (int pass = 0; pass < DVT / 64; ++pass) do_pass(pass);
+      if (!NG && a.edg) {  // the row's two halves, then one thread adds the row's term
+        edot += __shfl_xor_sync(0xffffffffu, edot, 16);
+        if (hf == 0 && lrow(i) < Cp) atomicAdd(a.edg + ((int64_t)bidx * a.T + otok) * a.H + h, a.esign * edot);
+      }
       return true;
     };
 
@@ -1285,6 +1314,14 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.ng_st = a.ng_gate.st;
   t.ng_sh = a.ng_gate.sh;
   t.ng_eps = a.ng_eps;
+  t.ex = a.ex.data;
+  t.ex_sb = a.ex.sb;
+  t.ex_st = a.ex.st;
+  t.ex_sh = a.ex.sh;
+  t.edg = a.edg;
+  t.esign = a.esign;
+  t.ephi = a.ephi;
+  t.edphi = a.edphi;
   const size_t ob = a.noseg ? 0 : order_bytes(a.n_seqs, a.cu_seqlens != nullptr);
   if (ob > 0 && workspace) {
     int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + seg_ws_bytes(plan, DK, DVT));
