@@ -22,6 +22,8 @@ it follows, is stated in the C file's header:
   of the recurrence, token by token).
 * ``backward_gated`` -- the same for the per-token decay, plus dg (the log
   decays' gradient); keeps every state, so for test sizes.
+* ``backward_norm`` -- dq, dk, dv of sum_t dout_t . o_t through the normalised
+  recurrence (o_t divided by z_t . phi(q_t)), token by token.
 * ``gated_delta`` -- the gated delta rule (section Gated delta rule of the same
   page), token by token, unit-norm keys.
 * ``norm_gate``  -- y = RMSNorm(o) * w * swish(g) per (token, head) over d_v.
@@ -84,6 +86,9 @@ def _load():
         lib.oracle_backward.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, i32,
                                         dp, dp, dp, i32]
         lib.oracle_backward.restype = i32
+        lib.oracle_backward_norm.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32, dp, dp,
+                                             dp, i32]
+        lib.oracle_backward_norm.restype = i32
         lib.oracle_backward_gated.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32,
                                               dp, dp, dp, dp, i32]
         lib.oracle_backward_gated.restype = i32
@@ -329,6 +334,24 @@ def backward(q, k, v, dout, gamma, cu_seqlens=None, phi="identity", nthreads=0):
                                  _PHI[phi], 0, _ptr(gq), _ptr(gk), _ptr(gv), int(nthreads))
     if rc != 0:
         raise _oracle_error("oracle_backward", rc)
+    return gq, gk, gv
+
+
+def backward_norm(q, k, v, dout, gamma, cu_seqlens=None, phi="elu1", nthreads=0):
+    """Gradients of L = sum(dout * o) for the normalised recurrence (o_t = S_t qh_t / z_t . qh_t).
+
+    Returns (dq [B,T,H,d_k], dk [B,T,H,d_k], dv [B,T,H,d_v]) in float64."""
+    q, k, v, dt, B, T, H, dk, dv, g, cu, n = _prep(q, k, v, gamma, cu_seqlens)
+    do, ddt = _as_input(dout)
+    if ddt != dt or do.shape != v.shape:
+        raise ValueError("dout must be [B, T, H, d_v] of the inputs' dtype")
+    gq = np.zeros(q.shape, np.float64)
+    gk = np.zeros(k.shape, np.float64)
+    gv = np.zeros(v.shape, np.float64)
+    rc = _load().oracle_backward_norm(_ptr(q), _ptr(k), _ptr(v), _ptr(do), dt, B, T, H, dk, dv, _ptr(g), _ptr(cu),
+                                      n, _PHI[phi], _ptr(gq), _ptr(gk), _ptr(gv), int(nthreads))
+    if rc != 0:
+        raise _oracle_error("oracle_backward_norm", rc)
     return gq, gk, gv
 
 

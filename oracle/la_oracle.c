@@ -626,6 +626,113 @@ int oracle_backward(const void *q, const void *k, const void *v, const void *dou
 }
 
 /*
+ * Backward of the normalised recurrence (per-head gamma), the adjoint of the
+ * definition token by token ("1.6 长上下文与高效注意力", section 线性注意力: the
+ * output divided by z_t^T phi(q_t)).  With L = sum_t dout_t . o_t:
+ *   forward:   S_t = gamma S_{t-1} + v_t kh_t^T,   z_t = gamma z_{t-1} + kh_t,
+ *              num_t = S_t qh_t,   den_t = z_t . qh_t,   o_t = num_t / den_t
+ *   u_t    = dL/dnum_t = dout_t / den_t
+ *   e_t    = dL/dden_t = -(dout_t . o_t) / den_t
+ *   dqh_t  = S_t^T u_t + e_t z_t
+ *   G_t    = dL/dS_t = u_t qh_t^T + gamma G_{t+1},   g_t = dL/dz_t = e_t qh_t + gamma g_{t+1}
+ *   dkh_t  = G_t^T v_t + g_t,   dv_t = G_t kh_t
+ *   dq = dqh * phi'(q),   dk = dkh * phi'(k).
+ * The forward sweep keeps u_t and e_t of every token of the task (len * (d_v + 1)
+ * doubles) for the backward sweep.  Arguments as for oracle_backward.
+ */
+int oracle_backward_norm(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                         int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                         const double *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int phi,
+                         double *dq, double *dkk, double *dvv, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+  int oom = 0; /* set when a task could not allocate its buffers */
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const double g = gamma[h];
+    const size_t nl = (size_t)(len > 0 ? len : 1);
+    double *S = (double *)calloc((size_t)(dv * dk), sizeof(double)); /* S[r][c] */
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    double *U = (double *)malloc(nl * (size_t)dv * sizeof(double)); /* u_t, every t */
+    double *E = (double *)malloc(nl * sizeof(double));               /* e_t, every t */
+    double *num = (double *)malloc((size_t)dv * sizeof(double));
+    if (!S || !z || !qh || !kh || !U || !E || !num) {
+      free(S); free(z); free(qh); free(kh); free(U); free(E); free(num);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
+    /* forward in time: the outputs' adjoints and dqh */
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      }
+      double den = 0.0;
+      for (int64_t c = 0; c < dk; ++c) {
+        z[c] = kh[c] + g * z[c];
+        den += z[c] * qh[c];
+      }
+      double dot = 0.0; /* dout_t . o_t */
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, vb + r);
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          S[r * dk + c] = g * S[r * dk + c] + vr * kh[c];
+          acc += S[r * dk + c] * qh[c];
+        }
+        num[r] = acc;
+        dot += orc_load(dout, dtype, vb + r) * (acc / den);
+      }
+      double *u = U + (size_t)t * dv;
+      for (int64_t r = 0; r < dv; ++r) u[r] = orc_load(dout, dtype, vb + r) / den;
+      E[t] = -dot / den;
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = E[t] * z[c];
+        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * u[r];
+        dq[qk + c] = acc * orc_dphi(orc_load(q, dtype, qk + c), phi);
+      }
+    }
+    /* backward in time: G (in S's buffer) and g (in z's) */
+    memset(S, 0, (size_t)(dv * dk) * sizeof(double));
+    memset(z, 0, (size_t)dk * sizeof(double));
+    for (int64_t t = len - 1; t >= 0; --t) {
+      const int64_t row = start + t;
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+      }
+      const double *u = U + (size_t)t * dv;
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) S[r * dk + c] = g * S[r * dk + c] + u[r] * qh[c];
+      for (int64_t c = 0; c < dk; ++c) z[c] = g * z[c] + E[t] * qh[c];
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = z[c];
+        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * orc_load(v, dtype, vb + r);
+        dkk[qk + c] = acc * orc_dphi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * kh[c];
+        dvv[vb + r] = acc;
+      }
+    }
+    free(S); free(z); free(qh); free(kh); free(U); free(E); free(num);
+  }
+  return oom ? ORC_ERR_NOMEM : 0;
+}
+
+/*
  * Gradients of L = sum_t dout_t . o_t for the unnormalised recurrence with a
  * per-token decay (oracle_recurrent_gated): the adjoint of that definition,
  * with respect to q, k, v and the log decays g.  With alpha_t = exp(g_t):

@@ -393,6 +393,80 @@ def test_backward_varlen_equals_independent_runs(oracle_mod):
         assert np.array_equal(gq[:, s_:e], a) and np.array_equal(gk[:, s_:e], b) and np.array_equal(gv[:, s_:e], c)
 
 
+# ---------------------------------------------------------------- normalised backward
+# elu + 1 keeps every denominator positive (phi > 0, positive weights); the identity
+# map with the normaliser can make it vanish, so the pins use elu + 1 (and one
+# identity case on positive inputs).
+@pytest.mark.parametrize("gamma", [1.0, 0.8])
+def test_backward_norm_matches_finite_differences(oracle_mod, gamma):
+    """Central differences of L = sum(dout * o) through the normalised forward oracle."""
+    B, T, H, dk, dv = 1, 7, 2, 3, 2
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=91)
+    dout = np.random.default_rng(92).standard_normal((B, T, H, dv))
+    gam = [gamma, 0.5]
+    gq, gk, gv = oracle_mod.backward_norm(q, k, v, dout, gam, phi="elu1")
+
+    def loss(q_, k_, v_):
+        o, _ = oracle_mod.recurrent(q_, k_, v_, gam, phi="elu1", normalize=True)
+        return float(np.sum(o * dout))
+
+    eps = 1e-6
+    for x, gref, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert rel(gref, fd) < 1e-7, which
+
+
+def test_backward_norm_matches_autograd_of_masked_form(oracle_mod):
+    """torch autograd (float64) through the normalised quadratic masked form,
+    O = ((phi(Q) phi(K)^T * M) V) / rowsum(phi(Q) phi(K)^T * M): a different formula."""
+    T, H, dk, dv = 30, 2, 5, 4
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=93)
+    dout = np.random.default_rng(94).standard_normal((1, T, H, dv))
+    gam = [0.9, 1.0]
+    cases = [("elu1", q, k)]
+    cases.append(("identity", np.abs(q) + 0.1, np.abs(k) + 0.1))  # positive keys and queries: den > 0
+    for phi, qq, kk in cases:
+        gq, gk, gv = oracle_mod.backward_norm(qq, kk, v, dout, gam, phi=phi)
+        for h in range(H):
+            qt, kt, vt = (torch.tensor(x[0, :, h], dtype=torch.float64, requires_grad=True) for x in (qq, kk, v))
+            f = (lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))) if phi == "elu1" \
+                else (lambda x: x)
+            A = f(qt) @ f(kt).T
+            i = torch.arange(T)[:, None]
+            j = torch.arange(T)[None, :]
+            M = torch.where(i >= j, torch.tensor(gam[h], dtype=torch.float64) ** (i - j).clamp(min=0).double(),
+                            torch.zeros((), dtype=torch.float64))
+            P = A * M
+            O = (P @ vt) / P.sum(dim=1, keepdim=True)
+            (O * torch.tensor(dout[0, :, h])).sum().backward()
+            assert rel(gq[0, :, h], qt.grad.numpy()) < 1e-11
+            assert rel(gk[0, :, h], kt.grad.numpy()) < 1e-11
+            assert rel(gv[0, :, h], vt.grad.numpy()) < 1e-11
+
+
+def test_backward_norm_varlen_equals_independent_runs(oracle_mod):
+    lengths = [5, 0, 17, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 2, 4, 3
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=95)
+    dout = np.random.default_rng(96).standard_normal((1, Tt, H, dv))
+    gam = [0.7, 1.0]
+    full = oracle_mod.backward_norm(q, k, v, dout, gam, cu_seqlens=cu, phi="elu1")
+    for n in range(len(lengths)):
+        s_, e = cu[n], cu[n + 1]
+        part = oracle_mod.backward_norm(q[:, s_:e], k[:, s_:e], v[:, s_:e], dout[:, s_:e], gam, phi="elu1")
+        for a, b in zip(full, part):
+            assert np.array_equal(a[:, s_:e], b)
+
+
 def _rand_log_decay(B, T, H, seed, lo=0.3):
     return np.log(np.random.default_rng(seed).uniform(lo, 1.0, (B, T, H)))
 

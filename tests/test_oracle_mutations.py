@@ -148,3 +148,68 @@ def test_gated_backward_mutant_is_caught(tmp_path, name):
     old, new = GATED_BWD_MUTATIONS[name]
     lib = _build(tmp_path, name, old, new)
     assert not _gated_bwd_pin_passes(lib), name
+
+
+NORM_BWD_MUTATIONS = {
+    "dq without the denominator's term e_t z_t": (
+        "        double acc = E[t] * z[c];\n        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * u[r];",
+        "        double acc = 0.0;\n        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * u[r];"),
+    "dk without the z adjoint g_t": (
+        "        double acc = z[c];\n        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * orc_load(v, dtype, vb + r);",
+        "        double acc = 0.0;\n        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * orc_load(v, dtype, vb + r);"),
+    "denominator's adjoint with the wrong sign": (
+        "E[t] = -dot / den;", "E[t] = dot / den;"),
+    "z adjoint not decayed": (
+        "for (int64_t c = 0; c < dk; ++c) z[c] = g * z[c] + E[t] * qh[c];",
+        "for (int64_t c = 0; c < dk; ++c) z[c] = z[c] + E[t] * qh[c];"),
+}
+
+
+def _norm_bwd(lib, q, k, v, dout, gamma):
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.oracle_backward_norm.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, vp, vp, i64, i32,
+                                         vp, vp, vp, i32]
+    lib.oracle_backward_norm.restype = i32
+    q, k, v, dout, gamma = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout, gamma))
+    outs = [np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)]
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = lib.oracle_backward_norm(p(q), p(k), p(v), p(dout), 2, B, T, H, dk, dv, p(gamma), None, B, 1,
+                                  *(p(o) for o in outs), 1)
+    assert rc == 0
+    return outs
+
+
+def _norm_bwd_pin_passes(lib):
+    """The autograd pin of test_oracle.py: torch float64 gradients through the
+    normalised masked form with elu + 1."""
+    import torch
+
+    T, dk, dv = 12, 3, 2
+    q, k, v = rand_qkv(1, T, 1, dk, dv, seed=97)
+    dout = np.random.default_rng(98).standard_normal((1, T, 1, dv))
+    gam = 0.85
+    got = _norm_bwd(lib, q, k, v, dout, np.array([gam]))
+    qt, kt, vt = (torch.tensor(x[0, :, 0], dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    f = lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))  # noqa: E731
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    M = torch.where(i >= j, torch.tensor(gam, dtype=torch.float64) ** (i - j).clamp(min=0).double(),
+                    torch.zeros((), dtype=torch.float64))
+    P = (f(qt) @ f(kt).T) * M
+    ((P @ vt) / P.sum(dim=1, keepdim=True) * torch.tensor(dout[0, :, 0])).sum().backward()
+    want = [qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()]
+    return all(rel(a[0, :, 0], w) < 1e-11 for a, w in zip(got, want))
+
+
+def test_unmutated_copy_passes_norm_backward_pin(tmp_path):
+    lib = _build(tmp_path, "none", "#define ROWS_PER_TASK 8", "#define ROWS_PER_TASK 8")
+    assert _norm_bwd_pin_passes(lib)
+
+
+@pytest.mark.parametrize("name", sorted(NORM_BWD_MUTATIONS))
+def test_norm_backward_mutant_is_caught(tmp_path, name):
+    old, new = NORM_BWD_MUTATIONS[name]
+    lib = _build(tmp_path, name, old, new)
+    assert not _norm_bwd_pin_passes(lib), name
