@@ -187,10 +187,27 @@ def _oracle_run(oracle, w, q, k, v, gamma, g=None, bwd=False, beta=None):
 
         if g is not None:
             return oracle.backward_gated(q, k, v, torch.ones_like(v), g, phi=w.phi)
+        if w.normalize:
+            return oracle.backward_norm(q, k, v, torch.ones_like(v), gamma, phi=w.phi)
         return oracle.backward(q, k, v, torch.ones_like(v), gamma, phi=w.phi)
     if g is not None:
         return oracle.recurrent_gated(q, k, v, g, phi=w.phi, normalize=w.normalize)[:2]
     return oracle.recurrent(q, k, v, gamma, phi=w.phi, normalize=w.normalize)
+
+
+def _norm_bwd_terms(oracle, q, k, v, dout, gamma, phi):
+    """|numerator| and |denominator| terms of the normalised dq and dk for one (sequence, head):
+    the unnormalised adjoints for (v, dout / den) and for (1, e), e_t = -(dout_t . o_t) / den_t."""
+    import numpy as np
+    import torch
+
+    q, k, v = q.double(), k.double(), v.double()
+    ones = torch.ones(v.shape[:3] + (1,), dtype=torch.float64)
+    den = torch.from_numpy(oracle.recurrent(q, k, ones, [gamma], phi=phi, normalize=False)[0])
+    o = torch.from_numpy(oracle.recurrent(q, k, v, [gamma], phi=phi, normalize=True)[0])
+    a = oracle.backward(q, k, v, dout.double() / den, [gamma], phi=phi)
+    b = oracle.backward(q, k, ones, -(dout.double() * o).sum(-1, keepdim=True) / den, [gamma], phi=phi)
+    return [np.maximum(np.abs(a[0]), np.abs(b[0])), np.maximum(np.abs(a[1]), np.abs(b[1])), None]
 
 
 def _oracle_rate(w, x, budget_s, max_tokens=None, nseq=1, bwd=False):
@@ -514,14 +531,18 @@ def main():
 
     gd = x.get("g")  # data-dependent log decay (gated workloads)
     if args.bwd:
-        if w.normalize or x.get("beta") is not None:
-            raise SystemExit("--bwd covers the unnormalised forwards (per-head or per-token decay)")
+        if x.get("beta") is not None or (w.normalize and gd is not None) or w.dtype != "bf16" and w.normalize:
+            raise SystemExit("--bwd covers the per-head-decay forwards (normalised in bf16) and the "
+                             "unnormalised per-token decay")
         from chunkwise_causal_linear_la_b200.workloads import make_dout
 
         dout = make_dout(v, seed=rank_seed(rank))
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
         if gd is not None:  # the per-token decay's backward also returns dg
             grads = grads + (torch.empty_like(gd),)
+        if w.normalize:  # the normalised backward keeps [v, 1, 1], [u, e_hi, e_lo] and phi(k) in its workspace
+            nws = la.bwd_norm_workspace_size(B, T, w.H, w.d_k, w.d_v, w.chunk, q.dtype)
+            wsbuf = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
 
     if args.normgate:
         if gd is not None or args.bwd:
@@ -545,6 +566,9 @@ def main():
         elif args.bwd and gd is not None:
             la.la_bwd_chunk_gated(q, k, v, dout, gd, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0],
                                   dk=grads[1], dv=grads[2], dg=grads[3], stream=stream)
+        elif args.bwd and w.normalize:
+            la.la_bwd_chunk_norm(q, k, v, dout, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0],
+                                 dk=grads[1], dv=grads[2], workspace=wsbuf, stream=stream)
         elif args.bwd:
             la.la_bwd_chunk(q, k, v, dout, g, cu_seqlens=cu, chunk=w.chunk, phi=w.phi, dq=grads[0], dk=grads[1],
                             dv=grads[2], stream=stream)
@@ -601,11 +625,14 @@ def main():
     # kernels launched per step: segmented sequences take a state pass, a scan and the output pass
     # (a packed batch with a workspace has its longest-first order computed first: 2 launches)
     # (backward: three tensor-core passes, two phi copies with elu + 1, and with a per-token decay the
-    # reverse cumulative sum of dg, whose row terms the passes' epilogues add)
+    # reverse cumulative sum of dg, whose row terms the passes' epilogues add; the normalised backward
+    # adds [v, 1, 1], the forward of the widened values and the [u, e] row pass)
     launches_per_step = (5 if w.phi == "elu1" else 3) if args.bwd else (
         (2 if cu is not None else 3) if nws > 0 else 1)
     if args.bwd and gd is not None:
         launches_per_step += 1
+    if args.bwd and w.normalize:
+        launches_per_step += 3
     if gbeta is not None:  # chunk offsets (packed batches), the per-chunk WY pass, the sequential pass
         launches_per_step = (3 if cu is not None else 2) if nws > 0 else 1
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -628,11 +655,18 @@ def main():
             if gd is not None:
                 refs = oracle.backward_gated(cut(q), cut(k), cut(v), cut(dout),
                                              gd[bb:bb + 1, s0:e0_, h:h + 1].double().cpu().numpy(), phi=w.phi)
+            elif w.normalize:
+                refs = oracle.backward_norm(cut(q), cut(k), cut(v), cut(dout), [float(g[h])], phi=w.phi)
             else:
                 refs = oracle.backward(cut(q), cut(k), cut(v), cut(dout), [float(g[h])], phi=w.phi)
-            for got, ref in zip(grads, refs):
+            # the normalised dq, dk are differences of a numerator and a denominator term that
+            # cancel: their error is measured against the larger of the two as well
+            terms = (_norm_bwd_terms(oracle, cut(q), cut(k), cut(v), cut(dout), float(g[h]), w.phi)
+                     if w.normalize else [None, None, None])
+            for got, ref, sc in zip(grads, refs, terms):
                 o = (cut(got) if got.dim() == 4 else got[bb:bb + 1, s0:e0_, h:h + 1].cpu()).double().numpy()
-                worst = max(worst, float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))))
+                den = np.max(np.abs(ref)) if sc is None else max(np.max(np.abs(ref)), np.max(sc))
+                worst = max(worst, float(np.max(np.abs(o - ref)) / den))
         for b, h in [] if args.bwd else sl:
             if cu is None:
                 qs, ks, vs = (t[b:b + 1, :, h:h + 1].cpu() for t in (q, k, v))
@@ -749,7 +783,13 @@ def main():
                                                           else "cuBLAS bf16 GEMM"),
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "launch_ms": launch_ms,
-                         "kernel": "chunk_tc_kernel (3 passes: forward + 2 in reverse time)" if args.bwd
+                         # the launch time scaled to the maximum SM clock by the median sampled clock, so that
+                         # settling under the power cap shows (time x median MHz / max MHz)
+                         "launch_ms_at_max_clock": (launch_ms * clocks["sm_mhz"] / clocks["sm_max_mhz"]
+                                                    if clocks.get("sm_mhz") and clocks.get("sm_max_mhz") else None),
+                         "kernel": ("chunk_tc_kernel (4 passes: forward of [v, 1, 1], forward + 2 in reverse time)"
+                                    if w.normalize else "chunk_tc_kernel (3 passes: forward + 2 in reverse time)")
+                         if args.bwd
                          else ("gdn_prep_kernel + gdn_tc_kernel (whole step)" if gbeta is not None
                                else "chunk_tc_kernel")},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * launches_per_step, "clocks": clocks,

@@ -26,6 +26,8 @@ from .binding import (  # noqa: F401
     la_fwd_chunk_host,
     la_bwd_chunk,
     la_bwd_chunk_gated,
+    la_bwd_chunk_norm,
+    bwd_norm_workspace_size,
     la_fwd_chunk,
     la_fwd_chunk_gated,
     la_fwd_chunk_normgate,

@@ -32,7 +32,8 @@ EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk
            "la_step_norm", "la_step_gated", "la_status_string", "la_last_error", "la_version", "la_device_error",
            "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
            "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size",
-           "la_fwd_chunk_path", "la_fwd_chunk_host", "la_fwd_chunk_host_arena_size", "la_bwd_chunk_gated")
+           "la_fwd_chunk_path", "la_fwd_chunk_host", "la_fwd_chunk_host_arena_size", "la_bwd_chunk_gated",
+           "la_bwd_chunk_norm", "la_bwd_chunk_norm_workspace_size")
 
 
 class LaTensor(ctypes.Structure):
@@ -99,6 +100,10 @@ def load_library(path: str = LIB_PATH):
     lib.la_fwd_chunk_host.restype = i32
     lib.la_bwd_chunk_gated.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, vp, i32, vp]
     lib.la_bwd_chunk_gated.restype = i32
+    lib.la_bwd_chunk_norm.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, i32, vp, sz, vp]
+    lib.la_bwd_chunk_norm.restype = i32
+    lib.la_bwd_chunk_norm_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32, i32]
+    lib.la_bwd_chunk_norm_workspace_size.restype = sz
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -383,6 +388,38 @@ def la_bwd_chunk_gated(q, k, v, dout, g, cu_seqlens=None, chunk=64, phi="identit
                                 *[ctypes.byref(x) for x in t[4:]], dg.data_ptr(), int(flags), _stream(stream))
     _check(lib, st, "la_bwd_chunk_gated")
     return dq, dk, dv, dg
+
+
+def bwd_norm_workspace_size(B, T, H, d_k, d_v, chunk=64, dtype=torch.bfloat16, flags=LA_FLAG_NONE) -> int:
+    """Bytes of workspace la_bwd_chunk_norm needs; -1 for arguments it rejects."""
+    n = load_library().la_bwd_chunk_norm_workspace_size(B, T, H, d_k, d_v, int(chunk), _DT[dtype], int(flags))
+    return -1 if n == ctypes.c_size_t(-1).value else int(n)
+
+
+def la_bwd_chunk_norm(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="elu1", dq=None, dk=None, dv=None,
+                      flags=LA_FLAG_NONE, workspace=None, stream=None):
+    """Gradients of la_fwd_chunk's normalised forward (see la_bwd_chunk_norm in
+    include/la_b200.h): returns (dq, dk, dv)."""
+    lib = load_library()
+    B, T, H, d_k = q.shape
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if gamma.dtype != torch.float32 or gamma.numel() != H:
+        raise TypeError("gamma must be float32 with H entries")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_norm_workspace_size(B, T, H, d_k, v.shape[3], chunk, q.dtype, flags)
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    t = [describe(x) for x in (q, k, v, dout, dq, dk, dv)]
+    st = lib.la_bwd_chunk_norm(*[ctypes.byref(x) for x in t[:4]], gamma.data_ptr(),
+                               None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk), _PHI[phi],
+                               *[ctypes.byref(x) for x in t[4:]], int(flags),
+                               None if workspace is None else workspace.data_ptr(),
+                               0 if workspace is None else workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+    _check(lib, st, "la_bwd_chunk_norm")
+    return dq, dk, dv
 
 
 def la_norm_gate(o, gate, w, eps=1e-5, y=None, stream=None):

@@ -676,6 +676,166 @@ la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
   return bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags, stream);
 }
 
+// The backward of la_fwd_chunk's normalised form (o_t = num_t / den_t), on the
+// tensor cores through the unnormalised backward of an augmented problem.  With
+// the value rows widened to v'_t = [v_t, 1, 1, 0...] the unnormalised forward of
+// (q, k, v') returns [num_t, den_t, den_t, 0...], and the gradient reaching it is
+// u'_t = [u_t, e_t, 0...] with u_t = dout_t / den_t and e_t = -(u_t . num_t) / den_t
+// (the denominator's adjoint), e_t carried as a bf16 pair over the two columns of
+// ones.  The unnormalised backward of (q, k, v', u') then gives dq and dk of the
+// normalised recurrence, and dv as the first d_v columns of dv'.
+// Steps: v' (elementwise), forward of (q, k, v') into F', F' -> u' in place
+// (one row pass), then the three backward passes of la_bwd_chunk with u' as the
+// output gradient; the dv pass reads only u''s first d_v columns.
+namespace {
+
+// Widths of the augmented value rows: d_v + 2 rounded up to a tensor-core value width.
+int64_t norm_aug_width(int64_t dv) { return dv == 64 ? 128 : dv == 128 ? 256 : -1; }
+
+struct NormBwdWs {
+  size_t vp, up, kh, total;  // byte offsets of v', F' / u', phi(k); total size
+};
+
+bool norm_bwd_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int32_t chunk, int32_t dtype,
+                   int32_t flags, NormBwdWs *w) {
+  const int64_t dvp = norm_aug_width(dv);
+  if (dtype != LA_BF16 || chunk != 64 || (flags & LA_FLAG_SIMT) || dvp < 0 || B < 0 || T < 0 || H <= 0)
+    return false;
+  if (!tc_shape((int)dk, (int)dvp) || !tc_shape((int)dvp, (int)dk) || !tc_shape((int)dk, (int)dv)) return false;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t rows = (size_t)(B * T * H);
+  w->vp = 0;
+  w->up = up(rows * dvp * 2);
+  w->kh = w->up + up(rows * dvp * 2);
+  w->total = w->kh + up(rows * dk * 2);
+  return true;
+}
+
+}  // namespace
+
+size_t la_bwd_chunk_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v, int32_t chunk,
+                                        int32_t dtype, int32_t flags) {
+  NormBwdWs w;
+  return norm_bwd_plan(B, T, H, d_k, d_v, chunk, dtype, flags, &w) ? w.total : (size_t)-1;
+}
+
+la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                            const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                            const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+  la_status s;
+  const la_tensor *ts[7] = {q, k, v, dout, dq, dk, dv};
+  const char *names[7] = {"q", "k", "v", "dout", "dq", "dk", "dv"};
+  for (int i = 0; i < 7; ++i)
+    if ((s = check_tensor(ts[i], names[i])) != LA_OK) return s;
+  for (int i = 1; i < 7; ++i) {
+    if (ts[i]->dtype != q->dtype) return fail(LA_ERR_INVALID_ARG, "%s must have q's dtype", names[i]);
+    if (ts[i]->B != q->B || ts[i]->T != q->T || ts[i]->H != q->H)
+      return fail(LA_ERR_INVALID_ARG, "%s disagrees with q on B, T or H", names[i]);
+  }
+  if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
+  if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
+  if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
+  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
+  if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (cu_seqlens) {
+    if (q->B != 1) return fail(LA_ERR_INVALID_ARG, "packed batches (cu_seqlens) need B == 1");
+    if (n_seqs < 0) return fail(LA_ERR_INVALID_ARG, "n_seqs is negative");
+  } else if (n_seqs != q->B) {
+    return fail(LA_ERR_INVALID_ARG, "n_seqs must equal B when cu_seqlens is NULL");
+  }
+  NormBwdWs w;
+  if (!norm_bwd_plan(q->B, q->T, q->H, q->D, v->D, chunk, q->dtype, flags, &w))
+    return fail(LA_ERR_UNSUPPORTED, "the normalised backward runs on the tensor cores only: bf16, chunk 64, "
+                "d_v in {64, 128}, d_k in {64, 128, 256}");
+  if (!workspace || workspace_bytes < w.total)
+    return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if (((uintptr_t)workspace) % 256 != 0) return fail(LA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (n_seqs == 0 || q->T == 0 || q->B == 0) return ok();
+
+  const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D, Dv = v->D, Dvp = norm_aug_width(Dv);
+  uint8_t *base = static_cast<uint8_t *>(workspace);
+  // contiguous [B, T, H, D] bf16 buffers in the workspace
+  auto buf = [&](size_t off, int64_t D) {
+    la_tensor t;
+    t.data = base + off;
+    t.dtype = q->dtype;
+    t.B = B;
+    t.T = T;
+    t.H = H;
+    t.D = D;
+    t.stride_h = D;
+    t.stride_t = H * D;
+    t.stride_b = T * H * D;
+    return t;
+  };
+  const la_tensor vp = buf(w.vp, Dvp), up = buf(w.up, Dvp), kh = buf(w.kh, Dk);
+  la_tensor u_head = up;  // u' seen as its first d_v columns: dout / den
+  u_head.D = Dv;
+  const bool elu = phi == LA_PHI_ELU1;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  ChunkArgs f;
+  f.gamma = gamma;
+  f.g = nullptr;
+  f.cu_seqlens = cu_seqlens;
+  f.final_state = nullptr;
+  f.final_z = nullptr;
+  f.B = B;
+  f.T = T;
+  f.n_seqs = n_seqs;
+  f.H = (int)H;
+  f.chunk = 64;
+  f.normalize = 0;
+  f.dtype = q->dtype;
+  f.noseg = 1;
+  f.ng_w = nullptr;
+  f.ng_gate = TensorView{nullptr, 0, 0, 0};
+  f.ng_eps = 0.f;
+  f.edg = nullptr;
+  f.esign = 0.f;
+  const char *why = nullptr;
+  // one tensor-core pass: out = fwd or rev(qq, kk, vv) with feature map ph on qq and kk; x (the
+  // input whose gradient this pass produces) makes the epilogue scale by phi'(x)
+  auto run = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
+                 int rev, const la_tensor *x) -> cudaError_t {
+    f.q = view(qq);
+    f.k = view(kk);
+    f.v = view(vv);
+    f.out = oo->data;
+    f.o_sb = oo->stride_b;
+    f.o_st = oo->stride_t;
+    f.o_sh = oo->stride_h;
+    f.dk = (int)qq->D;
+    f.dv = (int)vv->D;
+    f.phi = ph;
+    f.rev = rev;
+    f.ex = x && elu ? view(x) : TensorView{nullptr, 0, 0, 0};
+    f.ephi = phi;
+    f.edphi = x && elu ? 1 : 0;
+    if (!tc_supported(f)) return cudaErrorInvalidValue;
+    return launch_chunk_tc(f, nullptr, 0, st, &why);
+  };
+  cudaError_t err;
+  if ((err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess ||
+      (err = run(q, k, &vp, &up, phi, 0, nullptr)) != cudaSuccess ||
+      (err = launch_norm_grad_out(view(dout), up.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess)
+    return fail(LA_ERR_CUDA, "normalised backward (forward and output gradient): %s%s%s", cudaGetErrorString(err),
+                why ? ": " : "", why ? why : "");
+  // dphi(k) = rev(v', u', phi(q)); dphi(q) = fwd(u', v', phi(k)); dv = rev(phi(k), phi(q), u'[:d_v]).
+  // With elu + 1, phi(q) is staged in dq (written after it is read) and phi(k) in the workspace.
+  const la_tensor *qh = elu ? dq : q, *khp = elu ? &kh : k;
+  if ((elu && (err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess) ||
+      (err = run(&vp, &up, qh, dk, 0, 1, k)) != cudaSuccess ||
+      (elu && (err = launch_phi_copy(view(k), view(&kh), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess) ||
+      (err = run(&up, &vp, khp, dq, 0, 0, q)) != cudaSuccess ||
+      (err = run(k, q, &u_head, dv, phi, 1, nullptr)) != cudaSuccess)
+    return fail(LA_ERR_CUDA, "normalised backward (tensor cores): %s%s%s", cudaGetErrorString(err),
+                why ? ": " : "", why ? why : "");
+  return ok();
+}
+
 la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,
                   const la_tensor *out, int32_t phi, void *stream) {
   return step_common("la_step", q, k, v, gamma, nullptr, state, nullptr, out, phi, stream);

@@ -93,6 +93,10 @@ bool simt_supported(const ChunkArgs &a, int device);
 bool bwd_supported(const BwdArgs &a, int device);
 cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T, int64_t H, int64_t D, int phi,
                             int dtype, cudaStream_t stream);
+cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+                         cudaStream_t stream);
+cudaError_t launch_norm_grad_out(TensorView dout, void *up, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+                                 cudaStream_t stream);
 cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,
                                  cudaStream_t stream);
 cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,
@@ -108,6 +112,7 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 // Tensor-core (tcgen05 / TMA / TMEM) chunked forward for bf16.
 bool tc_supported(const ChunkArgs &a);
 bool tc_can_fuse_norm_gate(const ChunkArgs &a);
+bool tc_shape(int dk, int dv);  // head dims the tensor-core kernel takes
 size_t tc_workspace_bytes(int64_t B, int64_t T, int64_t H, int dk, int dv, int64_t n_seqs,
                           bool varlen, int chunk);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, void *workspace, size_t workspace_bytes,

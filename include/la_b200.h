@@ -412,8 +412,8 @@ LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_
  * in fp32; it needs the d_k x d_v fp32 state and one chunk's tiles to fit in
  * shared memory (d_k = d_v = 128 fits; 256 does not: LA_ERR_UNSUPPORTED).
  * Tokens outside every sequence of a packed batch may be overwritten in dq,
- * dk, dv.  The normalised forward has no backward here (the per-token decay's
- * is la_bwd_chunk_gated).  Other errors as for la_fwd_chunk.
+ * dk, dv.  The normalised forward's backward is la_bwd_chunk_norm, the per-token
+ * decay's la_bwd_chunk_gated.  Other errors as for la_fwd_chunk.
  */
 LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                               const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
@@ -448,6 +448,47 @@ LA_API la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
                                     int64_t n_seqs, int32_t chunk, int32_t phi, const la_tensor *dq,
                                     const la_tensor *dk, const la_tensor *dv, float *dg, int32_t flags,
                                     void *stream);
+
+/*
+ * la_bwd_chunk_norm -- backward of la_fwd_chunk with normalize = 1, the
+ * normalised linear attention of "1.6 长上下文与高效注意力", section 线性注意力:
+ *     o_t = num_t / den_t,  num_t = sum_{j<=t} gamma^(t-j) (phi(q_t) . phi(k_j)) v_j,
+ *                           den_t = sum_{j<=t} gamma^(t-j)  phi(q_t) . phi(k_j).
+ * With L = sum_t dout_t . o_t, the gradient reaching num_t is u_t = dout_t / den_t
+ * and the one reaching den_t is e_t = -(dout_t . num_t) / den_t^2; so
+ *     dphi(q)_t = sum_{j<=t} gamma^(t-j) (u_t . v_j + e_t) phi(k_j),
+ *     dphi(k)_j = sum_{t>=j} gamma^(t-j) (u_t . v_j + e_t) phi(q_t),
+ *     dv_j      = sum_{t>=j} gamma^(t-j) (phi(q_t) . phi(k_j)) u_t,
+ * which are la_bwd_chunk's three sums for the values [v_j, 1] and the output
+ * gradient [u_t, e_t]; dq and dk then take phi' (elu + 1) as in la_bwd_chunk.
+ *   q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi  as for la_fwd_chunk.
+ *   dout, dq, dk, dv  as for la_bwd_chunk.
+ *   workspace   device memory of la_bwd_chunk_norm_workspace_size bytes,
+ *               256-byte aligned, owned by the caller; it holds [v, 1, 1, 0...],
+ *               the forward's [num, den, den, 0...] turned in place into
+ *               [u, e_hi, e_lo, 0...] (bf16, d_v + 2 rounded up to 128 or 256
+ *               columns) and, with elu + 1, phi(k).  Nothing in it need start
+ *               at zero.
+ * Kernels: one elementwise pass, the tensor-core forward of (q, k, [v, 1, 1]),
+ * one row pass, then the three tensor-core backward passes (plus two
+ * feature-map copies with elu + 1).  Rounding: the sums u_t . v_j + e_t cancel
+ * (for a one-token sequence exactly, since o_1 = v_1), so the row pass takes e_t
+ * from the bf16-rounded u_t (the exact gradient for an output gradient within
+ * one bf16 rounding of dout) and stores it as a bf16 pair e_hi + e_lo.
+ * Shapes: bf16, chunk 64, d_v in {64, 128}, d_k in {64, 128, 256}; anything
+ * else, f32 and LA_FLAG_SIMT return LA_ERR_UNSUPPORTED.  den_t = 0 gives
+ * non-finite gradients, as it gives a non-finite forward output.
+ * LA_ERR_WORKSPACE if workspace is NULL or short.  Other errors as for
+ * la_bwd_chunk.  la_bwd_chunk_norm_workspace_size returns (size_t)-1 for
+ * shapes, chunks, dtypes or flags that la_bwd_chunk_norm rejects.
+ */
+LA_API size_t la_bwd_chunk_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                               int32_t chunk, int32_t dtype, int32_t flags);
+LA_API la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                   const la_tensor *dout, const float *gamma, const int32_t *cu_seqlens,
+                                   int64_t n_seqs, int32_t chunk, int32_t phi, const la_tensor *dq,
+                                   const la_tensor *dk, const la_tensor *dv, int32_t flags, void *workspace,
+                                   size_t workspace_bytes, void *stream);
 
 /*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device

@@ -14,8 +14,12 @@ import torch
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 
-def slice_rel_err(x, ref, seq_slices):
-    """x, ref: [B, T, H, D] arrays; seq_slices: list of (b, start, end)."""
+def slice_rel_err(x, ref, seq_slices, scale=None):
+    """x, ref: [B, T, H, D] arrays; seq_slices: list of (b, start, end).
+
+    scale (optional, ref's shape): where ref is a difference of terms that cancel,
+    the size of one of those terms; a slice's denominator is then the larger of
+    max|ref| and max|scale| over it."""
     worst = 0.0
     H = ref.shape[2]
     for b, s, e in seq_slices:
@@ -24,6 +28,8 @@ def slice_rel_err(x, ref, seq_slices):
         for h in range(H):
             r = ref[b, s:e, h]
             d = np.max(np.abs(r))
+            if scale is not None:
+                d = max(d, np.max(np.abs(scale[b, s:e, h])))
             err = np.max(np.abs(x[b, s:e, h] - r))
             worst = max(worst, float(err / d) if d > 0 else float(err))
     return worst

@@ -241,3 +241,116 @@ def test_bwd_gated_unsupported_shapes(la):
     g = _log_decay(1, 50, 2, 0.9, 0.99, 40).to(dev)
     with pytest.raises(la.LaError):
         la.la_bwd_chunk_gated(q, k, v, dout, g)  # f32: the tensor cores only
+
+
+# ---- backward of the normalised forward (la_bwd_chunk_norm) ----
+
+def _norm_bwd_scales(oracle_mod, q, k, v, dout, gamma, cu, phi, slices):
+    """Error scales for dq and dk of the normalised backward (from the oracle).
+
+    With u = dout / den and e_t = -(dout_t . o_t) / den_t the denominator's adjoint,
+        dphi(q)_t = sum_{j<=t} w_tj (u_t . v_j) phi(k_j) + e_t sum_{j<=t} w_tj phi(k_j) = A + B
+    (dphi(k) likewise): two sums that cancel, the more so as the sequence grows,
+    since a normalised average does not move with the part of phi(k) common to all
+    tokens.  In bf16 each of A and B carries its own rounding (the inter-chunk
+    state enters the tensor cores in bf16), so the error is measured against
+    max(|dq|, |A|, |B|) per slice.  A one-token sequence cancels inside the dot
+    products themselves (o_1 = v_1 whatever q and k: exact dq = dk = 0); there the
+    scale is the same sums with every term by its absolute value."""
+    q64, k64, v64 = q.double(), k.double(), v.double()
+    ones = torch.ones(v.shape[:3] + (1,), dtype=torch.float64)
+    den, _ = oracle_mod.recurrent(q64, k64, ones, gamma, cu_seqlens=cu, phi=phi, normalize=False)
+    o, _ = oracle_mod.recurrent(q64, k64, v64, gamma, cu_seqlens=cu, phi=phi, normalize=True)
+    den, o, do = torch.from_numpy(den), torch.from_numpy(o), dout.double()
+    u = do / den
+    e = -(do * o).sum(-1, keepdim=True) / den
+    aq, ak, _ = oracle_mod.backward(q64, k64, v64, u, gamma, cu_seqlens=cu, phi=phi)
+    bq, bk, _ = oracle_mod.backward(q64, k64, ones, e, gamma, cu_seqlens=cu, phi=phi)
+    xq, xk, _ = oracle_mod.backward(q64, k64, torch.cat([v64.abs(), ones], -1), torch.cat([u.abs(), e.abs()], -1),
+                                    gamma, cu_seqlens=cu, phi=phi)
+    scales = []
+    for a, b, x in ((aq, bq, xq), (ak, bk, xk)):
+        sc = np.maximum(np.abs(a), np.abs(b))
+        for bb, s0, e0 in slices:
+            if e0 - s0 == 1:
+                sc[bb, s0:e0] = np.abs(x[bb, s0:e0])
+        scales.append(sc)
+    return scales
+
+
+def _check_norm(la, oracle_mod, q, k, v, dout, gamma, cu=None, phi="elu1"):
+    dev = torch.device("cuda")
+    dq, dk, dv = la.la_bwd_chunk_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), gamma.to(dev),
+                                      cu_seqlens=None if cu is None else cu.to(dev), phi=phi)
+    torch.cuda.synchronize()
+    g64, cu_np = gamma.double().numpy(), None if cu is None else cu.numpy()
+    refs = oracle_mod.backward_norm(q, k, v, dout, g64, cu_seqlens=cu_np, phi=phi)
+    B, T = q.shape[:2]
+    sl = seq_slices(B, T, None if cu is None else cu.tolist())
+    sq, sk = _norm_bwd_scales(oracle_mod, q, k, v, dout, g64, cu_np, phi, sl)
+    assert all(np.isfinite(to_np(x)).all() for x in (dq, dk, dv))
+    errs = [slice_rel_err(to_np(x), r, sl, scale=s) for x, r, s in zip((dq, dk, dv), refs, (sq, sk, None))]
+    assert max(errs) < TOL[torch.bfloat16], errs
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64), (256, 128)])
+@pytest.mark.parametrize("T", [1, 65, 300])
+def test_bwd_norm_shapes(la, oracle_mod, dk, dv, T):
+    q, k, v, dout = _inputs(2, T, 2, dk, dv, torch.bfloat16, dk + dv + T)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.9]))
+
+
+@pytest.mark.parametrize("gamma", [0.0, 0.3, 0.9, 0.999, 1.0])
+def test_bwd_norm_gammas(la, oracle_mod, gamma):
+    """gamma <= 0.3 takes the value-decay path of each pass, the others the decayed-key path."""
+    q, k, v, dout = _inputs(1, 200, 2, 128, 128, torch.bfloat16, 41)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([gamma, 1.0]))
+
+
+def test_bwd_norm_identity_positive_features(la, oracle_mod):
+    """The identity feature map with positive q, k (den > 0), as the normalised form asks."""
+    q, k, v, dout = _inputs(2, 150, 2, 64, 64, torch.bfloat16, 43)
+    _check_norm(la, oracle_mod, q.abs(), k.abs(), v, dout, torch.tensor([1.0, 0.95]), phi="identity")
+
+
+def test_bwd_norm_varlen(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 300, 17])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 3, 128, 128, torch.bfloat16, 47)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.97, 0.5]), cu=cu)
+
+
+def test_bwd_norm_long_sequence(la, oracle_mod):
+    q, k, v, dout = _inputs(1, 4096, 2, 128, 128, torch.bfloat16, 53)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.999]))
+
+
+def test_bwd_norm_caller_workspace_reused(la, oracle_mod):
+    """A caller-owned workspace left dirty by an earlier call gives the same gradients."""
+    dev = torch.device("cuda")
+    q, k, v, dout = _inputs(1, 257, 2, 128, 128, torch.bfloat16, 59)
+    gamma = torch.tensor([1.0, 0.9])
+    need = la.bwd_norm_workspace_size(1, 257, 2, 128, 128)
+    ws = torch.full((need,), 0x7F, dtype=torch.uint8, device=dev)
+    args = [x.to(dev) for x in (q, k, v, dout, gamma)]
+    a = la.la_bwd_chunk_norm(*args, workspace=ws)
+    b = la.la_bwd_chunk_norm(*args, workspace=ws)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    refs = oracle_mod.backward_norm(q, k, v, dout, gamma.double().numpy())
+    sl = seq_slices(1, 257)
+    scales = _norm_bwd_scales(oracle_mod, q, k, v, dout, gamma.double().numpy(), None, "elu1", sl) + [None]
+    assert max(slice_rel_err(to_np(x), r, sl, scale=sc) for x, r, sc in zip(a, refs, scales)) < TOL[torch.bfloat16]
+
+
+def test_bwd_norm_unsupported(la):
+    dev = torch.device("cuda")
+    assert la.bwd_norm_workspace_size(1, 64, 2, 128, 256) == -1
+    assert la.bwd_norm_workspace_size(1, 64, 2, 128, 128, dtype=torch.float32) == -1
+    q, k, v, dout = _inputs(1, 64, 2, 128, 256, torch.bfloat16, 61)
+    with pytest.raises(la.LaError) as e:
+        la.la_bwd_chunk_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), torch.ones(2, device=dev))
+    assert e.value.status == la.binding.LA_ERR_UNSUPPORTED
+    assert la.device_error(reset=True) == (0, 0)

@@ -239,3 +239,46 @@ def test_host_arena_size_and_validation(lib):
     assert call(strided, 0x4000, 1 << 20) == b.LA_ERR_INVALID_ARG
     assert call(t, None, 0) == b.LA_ERR_WORKSPACE
     assert call(t, 0x4010, 1 << 20) == b.LA_ERR_INVALID_ARG  # arena not 256-byte aligned
+
+
+def test_bwd_norm_workspace_and_validation_on_host(lib):
+    """la_bwd_chunk_norm_workspace_size: the augmented value rows ([v, 1, 1] rounded up
+    to 128 or 256 columns) twice, plus phi(k), each at a 256-byte boundary; -1 for
+    what la_bwd_chunk_norm rejects.  Bad arguments and a short or misaligned
+    workspace are rejected before any device call."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    ws = lib.la_bwd_chunk_norm_workspace_size
+    bad = ctypes.c_size_t(-1).value
+    rows = 3 * 100 * 5
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert ws(3, 100, 5, 128, 128, 64, 1, 0) == 2 * up(rows * 256 * 2) + up(rows * 128 * 2)
+    assert ws(3, 100, 5, 64, 64, 64, 1, 0) == 2 * up(rows * 128 * 2) + up(rows * 64 * 2)
+    assert ws(3, 100, 5, 256, 128, 64, 1, 0) == 2 * up(rows * 256 * 2) + up(rows * 256 * 2)
+    assert ws(3, 100, 5, 128, 256, 64, 1, 0) == bad  # d_v + 2 does not fit 256 columns
+    assert ws(3, 100, 5, 128, 128, 32, 1, 0) == bad  # chunk
+    assert ws(3, 100, 5, 128, 128, 64, 0, 0) == bad  # f32
+    assert ws(3, 100, 5, 128, 128, 64, 1, 1) == bad  # LA_FLAG_SIMT
+    assert ws(3, 100, 5, 32, 128, 64, 1, 0) == bad  # d_k
+    assert ws(3, 100, 0, 128, 128, 64, 1, 0) == bad  # H = 0
+
+    need = ws(1, 4, 2, 128, 128, 64, 1, 0)
+    q, k, v, do, dq, dk, dv = (_t(D=128) for _ in range(7))
+
+    def call(gamma=0x2000, phi=1, ws_ptr=0x100000, ws_bytes=None, qq=None, vv=None, flags=0):
+        return lib.la_bwd_chunk_norm(ctypes.byref(qq or q), ctypes.byref(k), ctypes.byref(vv or v), ctypes.byref(do),
+                                     gamma, None, 1, 64, phi, ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv),
+                                     flags, ws_ptr, need if ws_bytes is None else ws_bytes, None)
+    assert call(gamma=None) == b.LA_ERR_INVALID_ARG and b"gamma" in lib.la_last_error()
+    assert call(phi=5) == b.LA_ERR_INVALID_ARG
+    assert call(flags=8) == b.LA_ERR_INVALID_ARG and b"flags" in lib.la_last_error()
+    assert call(qq=_t(D=64)) == b.LA_ERR_INVALID_ARG  # q and k disagree
+    assert call(qq=_t(D=128, ptr=0x1008)) == b.LA_ERR_INVALID_ARG  # misaligned
+    assert call(ws_bytes=need - 1) == b.LA_ERR_WORKSPACE
+    assert call(ws_ptr=None) == b.LA_ERR_WORKSPACE
+    assert call(ws_ptr=0x100010) == b.LA_ERR_INVALID_ARG and b"256" in lib.la_last_error()
+    assert call(flags=1) == b.LA_ERR_UNSUPPORTED and b"tensor cores" in lib.la_last_error()
+    f32 = [_t(D=128, dtype=0) for _ in range(7)]
+    st = lib.la_bwd_chunk_norm(*[ctypes.byref(x) for x in f32[:4]], 0x2000, None, 1, 64, 1,
+                               *[ctypes.byref(x) for x in f32[4:]], 0, 0x100000, need, None)
+    assert st == b.LA_ERR_UNSUPPORTED

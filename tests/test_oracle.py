@@ -758,3 +758,25 @@ def test_oracle_is_independent_of_the_product():
     src = open(os.path.join(os.path.dirname(__file__), "..", "oracle", "__init__.py")).read()
     src += open(os.path.join(os.path.dirname(__file__), "..", "oracle", "la_oracle.c")).read()
     assert "chunkwise_causal_linear_la_b200" not in src
+
+
+def test_backward_norm_splits_into_numerator_and_denominator_adjoints(oracle_mod):
+    """The normalised adjoint is the unnormalised one twice: once for the numerator
+    (values v, output gradient dout / den) and once for the denominator (values 1,
+    output gradient e_t = -(dout_t . o_t) / den_t), with den and o from the forward."""
+    gen = torch.Generator()
+    gen.manual_seed(71)
+    B, T, H, dk, dv = 2, 37, 2, 5, 4
+    q, k, v, do = (torch.randn((B, T, H, d), generator=gen, dtype=torch.float64) for d in (dk, dk, dv, dv))
+    gamma = np.array([1.0, 0.85])
+    for phi in ("elu1",):
+        ones = torch.ones((B, T, H, 1), dtype=torch.float64)
+        den, _ = oracle_mod.recurrent(q, k, ones, gamma, phi=phi, normalize=False)
+        o, _ = oracle_mod.recurrent(q, k, v, gamma, phi=phi, normalize=True)
+        den, o = torch.from_numpy(den), torch.from_numpy(o)
+        a = oracle_mod.backward(q, k, v, do / den, gamma, phi=phi)
+        b = oracle_mod.backward(q, k, ones, -(do * o).sum(-1, keepdim=True) / den, gamma, phi=phi)
+        ref = oracle_mod.backward_norm(q, k, v, do, gamma, phi=phi)
+        for x, y, r in zip(a[:2], b[:2], ref[:2]):
+            np.testing.assert_allclose(x + y, r, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(a[2], ref[2], rtol=1e-10, atol=1e-12)
