@@ -161,6 +161,7 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
   a.edg = nullptr;
   a.esign = 0.f;
   a.ephi = a.edphi = 0;
+  a.den_out = nullptr;
   a.ng_w = nullptr;
   a.ng_gate = TensorView{nullptr, 0, 0, 0};
   a.ng_eps = 0.f;
@@ -590,6 +591,7 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   f.edg = nullptr;
   f.esign = 0.f;
   f.ephi = f.edphi = 0;
+  f.den_out = nullptr;
   auto setup = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
                    int rev) {
     f.q = view(qq);
@@ -678,22 +680,21 @@ la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
 
 // The backward of la_fwd_chunk's normalised form (o_t = num_t / den_t), on the
 // tensor cores through the unnormalised backward of an augmented problem.  With
-// the value rows widened to v'_t = [v_t, 1, 1, 0...] the unnormalised forward of
-// (q, k, v') returns [num_t, den_t, den_t, 0...], and the gradient reaching it is
-// u'_t = [u_t, e_t, 0...] with u_t = dout_t / den_t and e_t = -(u_t . num_t) / den_t
-// (the denominator's adjoint), e_t carried as a bf16 pair over the two columns of
-// ones.  The unnormalised backward of (q, k, v', u') then gives dq and dk of the
-// normalised recurrence, and dv as the first d_v columns of dv'.
-// Steps: v' (elementwise), forward of (q, k, v') into F', F' -> u' in place
-// (one row pass), then the three backward passes of la_bwd_chunk with u' as the
-// output gradient; the dv pass reads only u''s first d_v columns.
+// the value rows widened to v'_t = [v_t, 1, 1, 0...] and the output gradient to
+// u'_t = [u_t, e_t, 0...], u_t = dout_t / den_t and e_t = -(u_t . o_t) (the
+// denominator's adjoint, carried as a bf16 pair over the two columns of ones),
+// the unnormalised backward of (q, k, v', u') gives dq and dk of the normalised
+// recurrence, and dv as the first d_v columns of dv'.
+// Steps: v' (elementwise), the normalised forward (o and den_t), u' (one row
+// pass), then the three backward passes of la_bwd_chunk with u' as the output
+// gradient; the dv pass reads only u''s first d_v columns.
 namespace {
 
-// Widths of the augmented value rows: d_v + 2 rounded up to a tensor-core value width.
+// Widths of the augmented value rows: d_v + 2 rounded up to a tensor-core key width.
 int64_t norm_aug_width(int64_t dv) { return dv == 64 ? 128 : dv == 128 ? 256 : -1; }
 
 struct NormBwdWs {
-  size_t vp, up, kh, total;  // byte offsets of v', F' / u', phi(k); total size
+  size_t vp, up, o, den, kh, total;  // byte offsets of v', u', o, den, phi(k); total size
 };
 
 bool norm_bwd_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int32_t chunk, int32_t dtype,
@@ -701,12 +702,14 @@ bool norm_bwd_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int3
   const int64_t dvp = norm_aug_width(dv);
   if (dtype != LA_BF16 || chunk != 64 || (flags & LA_FLAG_SIMT) || dvp < 0 || B < 0 || T < 0 || H <= 0)
     return false;
-  if (!tc_shape((int)dk, (int)dvp) || !tc_shape((int)dvp, (int)dk) || !tc_shape((int)dk, (int)dv)) return false;
+  if (!tc_shape((int)dvp, (int)dk) || !tc_shape((int)dk, (int)dv)) return false;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t rows = (size_t)(B * T * H);
   w->vp = 0;
   w->up = up(rows * dvp * 2);
-  w->kh = w->up + up(rows * dvp * 2);
+  w->o = w->up + up(rows * dvp * 2);
+  w->den = w->o + up(rows * dv * 2);
+  w->kh = w->den + up(rows * 4);
   w->total = w->kh + up(rows * dk * 2);
   return true;
 }
@@ -770,7 +773,8 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     t.stride_b = T * H * D;
     return t;
   };
-  const la_tensor vp = buf(w.vp, Dvp), up = buf(w.up, Dvp), kh = buf(w.kh, Dk);
+  const la_tensor vp = buf(w.vp, Dvp), up = buf(w.up, Dvp), o = buf(w.o, Dv), kh = buf(w.kh, Dk);
+  float *den = reinterpret_cast<float *>(base + w.den);
   la_tensor u_head = up;  // u' seen as its first d_v columns: dout / den
   u_head.D = Dv;
   const bool elu = phi == LA_PHI_ELU1;
@@ -795,6 +799,7 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   f.ng_eps = 0.f;
   f.edg = nullptr;
   f.esign = 0.f;
+  f.den_out = nullptr;
   const char *why = nullptr;
   // one tensor-core pass: out = fwd or rev(qq, kk, vv) with feature map ph on qq and kk; x (the
   // input whose gradient this pass produces) makes the epilogue scale by phi'(x)
@@ -818,9 +823,16 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     return launch_chunk_tc(f, nullptr, 0, st, &why);
   };
   cudaError_t err;
-  if ((err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess ||
-      (err = run(q, k, &vp, &up, phi, 0, nullptr)) != cudaSuccess ||
-      (err = launch_norm_grad_out(view(dout), up.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess)
+  // the normalised forward (o, and den_t from its epilogue), then u'
+  f.normalize = 1;
+  f.den_out = den;
+  err = run(q, k, v, &o, phi, 0, nullptr);
+  f.normalize = 0;
+  f.den_out = nullptr;
+  if (err != cudaSuccess ||
+      (err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess ||
+      (err = launch_norm_grad_out(view(dout), o.data, den, up.data, B, T, H, (int)Dv, (int)Dvp, st)) !=
+          cudaSuccess)
     return fail(LA_ERR_CUDA, "normalised backward (forward and output gradient): %s%s%s", cudaGetErrorString(err),
                 why ? ": " : "", why ? why : "");
   // dphi(k) = rev(v', u', phi(q)); dphi(q) = fwd(u', v', phi(k)); dv = rev(phi(k), phi(q), u'[:d_v]).

@@ -25,28 +25,29 @@ struct Vec {
   static constexpr int VW = 16 / sizeof(T);
 };
 
-template <typename T>
-__device__ __forceinline__ void row_of(int64_t e, int64_t nvr, int64_t T_, int64_t H, int64_t &b, int64_t &t,
-                                       int64_t &h, int &col) {
-  const int64_t row = e / nvr;
-  col = (int)(e - row * nvr) * Vec<T>::VW;
+// Token row r of a [B, T, H] grid (rows ordered (b, t, h)) in the index type I:
+// 32-bit whenever the launch's element count fits (the divisions are then a few
+// instructions instead of a 64-bit division's long sequence).
+template <typename I>
+__device__ __forceinline__ void split_row(I row, I T_, I H, I &b, I &t, I &h) {
   h = row % H;
-  const int64_t bt = row / H;
+  const I bt = row / H;
   t = bt % T_;
   b = bt / T_;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kEwThreads) phi_kernel(TensorView src, TensorView dst, int64_t T_, int64_t H,
-                                                          int64_t D, int64_t nvec, int phi) {
+template <typename T, typename I>
+__global__ void __launch_bounds__(kEwThreads) phi_kernel(TensorView src, TensorView dst, I T_, I H, I D, I nvec,
+                                                          int phi) {
   constexpr int VW = Vec<T>::VW;
-  const int64_t nvr = D / VW;
-  for (int64_t e = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; e < nvec; e += (int64_t)gridDim.x * kEwThreads) {
-    int64_t b, t, h;
-    int col;
-    row_of<T>(e, nvr, T_, H, b, t, h, col);
-    const T *s = (const T *)src.data + b * src.sb + t * src.st + h * src.sh + col;
-    T *o = (T *)dst.data + b * dst.sb + t * dst.st + h * dst.sh + col;
+  const I nvr = D / VW;
+  for (I e = blockIdx.x * (I)kEwThreads + threadIdx.x; e < nvec; e += (I)gridDim.x * kEwThreads) {
+    const I row = e / nvr;
+    const int col = (int)(e - row * nvr) * VW;
+    I b, t, h;
+    split_row<I>(row, T_, H, b, t, h);
+    const T *s = (const T *)src.data + (int64_t)b * src.sb + (int64_t)t * src.st + (int64_t)h * src.sh + col;
+    T *o = (T *)dst.data + (int64_t)b * dst.sb + (int64_t)t * dst.st + (int64_t)h * dst.sh + col;
     uint4 x = *reinterpret_cast<const uint4 *>(s);
     T *xv = reinterpret_cast<T *>(&x);
 #pragma unroll
@@ -55,11 +56,6 @@ __global__ void __launch_bounds__(kEwThreads) phi_kernel(TensorView src, TensorV
   }
 }
 
-// Gradient of the log decays (per-token decay backward).  With b the prefix sum of
-// the log decays g, the loss sees b_s only through the weights exp(b_i - b_j) of
-// o_i = sum_{j<=i} exp(b_i - b_j) (qh_i . kh_j) v_j, so dL/db_s = qh_s . dqh_s -
-// kh_s . dkh_s and dg_t = sum_{s>=t} dL/db_s.  The backward passes' epilogues add
-// the row terms into dg (chunk_tc_kernel); this kernel finishes the sum.
 __device__ __forceinline__ void unpack_bf16x8(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -80,82 +76,95 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&f)[8]) {
 }
 
 // Backward of the normalised forward (see la_bwd_chunk_norm).  With v' = [v, 1, 1, 0...]
-// the unnormalised forward returns [num, den, den, 0...] per row (den_t = sum_{j<=t}
-// gamma^(t-j) phi(q_t) . phi(k_j) is a value column of ones), and with
-// u' = [u, e_hi, e_lo, 0...], u_t = dout_t / den_t and e_t = -(u_t . num_t) / den_t
-// (the denominator's adjoint) split into a bf16 pair e_hi + e_lo, the unnormalised
-// backward of (q, k, v', u') is the normalised one's.
+// and u' = [u, e_hi, e_lo, 0...], u_t = dout_t / den_t and e_t = -(u_t . o_t) (the
+// denominator's adjoint, o_t = num_t / den_t) split into a bf16 pair e_hi + e_lo,
+// the unnormalised backward of (q, k, v', u') is the normalised one's.
 //
 // Rounding: the sums u_t . v_j + e_t that the backward forms cancel (for a one-token
 // sequence exactly: o_1 = v_1 whatever q and k).  e_t is therefore taken from the
 // bf16-rounded u_t, so that u' is the exact gradient for an output gradient within
 // one bf16 rounding of dout, and carried to about 16 bits by the pair.
 //
-// v' rows in a contiguous [rows][dvp] bf16 buffer: thread e writes the 16-byte
-// vector e mod (dvp / 8) of row e / (dvp / 8); dv is a multiple of 8.
-__global__ void __launch_bounds__(kEwThreads) aug_v_kernel(TensorView v, __nv_bfloat16 *vp, int64_t T_, int64_t H,
-                                                            int dv, int dvp, int64_t nvec) {
-  const int nvr = dvp / 8;
-  for (int64_t e = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; e < nvec; e += (int64_t)gridDim.x * kEwThreads) {
-    const int64_t row = e / nvr;
-    const int col = (int)(e - row * nvr) * 8;
-    const int64_t h = row % H, bt = row / H, t = bt % T_, b = bt / T_;
+// Both kernels write contiguous [rows][dvp] bf16 rows, one thread per 16-byte
+// vector (lpr = dvp / 8 vectors per row, a power of two, so a row's vectors sit
+// in one warp); dv is a multiple of 8 below dvp.
+template <typename I>
+__global__ void __launch_bounds__(kEwThreads) aug_v_kernel(TensorView v, __nv_bfloat16 *vp, I T_, I H, int dv,
+                                                            int lpr_log2, I nvec) {
+  const int lpr = 1 << lpr_log2;
+  for (I e = blockIdx.x * (I)kEwThreads + threadIdx.x; e < nvec; e += (I)gridDim.x * kEwThreads) {
+    const I row = e >> lpr_log2;
+    const int col = (int)(e & (I)(lpr - 1)) * 8;
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (col < dv)
-      x = *reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)v.data + b * v.sb + t * v.st + h * v.sh + col);
-    else if (col == dv)
+    if (col < dv) {
+      I b, t, h;
+      split_row<I>(row, T_, H, b, t, h);
+      x = *reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)v.data + (int64_t)b * v.sb +
+                                           (int64_t)t * v.st + (int64_t)h * v.sh + col);
+    } else if (col == dv) {
       x.x = 0x3F803F80u;  // bf16 1.0 in columns dv and dv + 1
-    *reinterpret_cast<uint4 *>(vp + row * dvp + col) = x;
+    }
+    *reinterpret_cast<uint4 *>(vp + (int64_t)row * (8 << lpr_log2) + col) = x;
   }
 }
 
-// up rows ([rows][dvp] bf16): [num, den, den, 0...] in, [u, e_hi, e_lo, 0...] out
-// (fp32 arithmetic), dout rows read through their strides.  lpr = dvp / 8 lanes per
-// row, one vector each.
-__global__ void __launch_bounds__(kEwThreads) norm_grad_out_kernel(TensorView dout, __nv_bfloat16 *up, int64_t T_,
-                                                                    int64_t H, int dv, int dvp, int64_t rows) {
-  const int lpr = dvp / 8;
-  const int lane = threadIdx.x & 31, sub = lane % lpr;
-  const int col = sub * 8;
-  const int den_lane = (lane - sub) + dv / 8;  // the lane of this row holding column dv
-  const int64_t rows_per_step = (int64_t)gridDim.x * (kEwThreads / lpr);
-  for (int64_t row0 = blockIdx.x * (int64_t)(kEwThreads / lpr); row0 < rows; row0 += rows_per_step) {
-    const int64_t row = row0 + threadIdx.x / lpr;
-    const bool live = row < rows;
-    float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint4 *p = reinterpret_cast<uint4 *>(up + (live ? row : 0) * dvp + col);
-    if (live) {
-      unpack_bf16x8(*p, f);
-      if (col < dv) {
-        const int64_t h = row % H, bt = row / H, t = bt % T_, b = bt / T_;
-        unpack_bf16x8(*reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)dout.data + b * dout.sb +
-                                                        t * dout.st + h * dout.sh + col), d);
-      }
+// u' rows from the normalised forward's o ([rows][dv] bf16, contiguous) and den
+// ([rows] fp32), and dout (through its strides); fp32 arithmetic.
+template <typename I>
+__global__ void __launch_bounds__(kEwThreads) norm_grad_out_kernel(TensorView dout, const __nv_bfloat16 *o,
+                                                                    const float *den, __nv_bfloat16 *up, I T_, I H,
+                                                                    int dv, int lpr_log2, I nvec) {
+  const int lpr = 1 << lpr_log2;
+  for (I e0 = blockIdx.x * (I)kEwThreads; e0 < nvec; e0 += (I)gridDim.x * kEwThreads) {
+    const I e = e0 + threadIdx.x;  // rows are whole within a warp and the loop bound is warp-uniform
+    const bool live = e < nvec;
+    const I row = live ? e >> lpr_log2 : 0;
+    const int col = (int)(e & (I)(lpr - 1)) * 8;
+    float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float inv = 0.f;
+    if (live && col < dv) {
+      I b, t, h;
+      split_row<I>(row, T_, H, b, t, h);
+      unpack_bf16x8(*reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)dout.data + (int64_t)b * dout.sb +
+                                                      (int64_t)t * dout.st + (int64_t)h * dout.sh + col), d);
+      unpack_bf16x8(*reinterpret_cast<const uint4 *>(o + (int64_t)row * dv + col), f);
     }
-    const float den = __shfl_sync(0xffffffffu, f[0], den_lane);
-    const float inv = 1.f / den;
+    if (live) inv = 1.f / den[row];
     float y[8], dot = 0.f;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      y[u] = col + u < dv ? __bfloat162float(__float2bfloat16_rn(d[u] * inv)) : 0.f;  // u as stored
-      dot = fmaf(y[u], f[u], dot);  // u . num (zero past dv)
+      y[u] = col < dv ? __bfloat162float(__float2bfloat16_rn(d[u] * inv)) : 0.f;  // u as stored
+      dot = fmaf(y[u], f[u], dot);                               // u . o
     }
-    for (int o = lpr / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    for (int s = lpr / 2; s > 0; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
     if (!live) continue;
     if (col == dv) {
-      const float e = -dot * inv;
-      y[0] = __bfloat162float(__float2bfloat16_rn(e));
-      y[1] = e - y[0];
+      y[0] = __bfloat162float(__float2bfloat16_rn(-dot));
+      y[1] = -dot - y[0];
     }
-    *p = pack_bf16x8(y);
+    *reinterpret_cast<uint4 *>(up + (int64_t)row * (8 << lpr_log2) + col) = pack_bf16x8(y);
   }
 }
 
 unsigned ew_grid(int64_t n) {
   const int64_t blocks = (n + kEwThreads - 1) / kEwThreads;
-  return (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
+  return (unsigned)(blocks < 148 * 64 ? blocks : 148 * 64);
 }
 
+// 32-bit indices when every element index of a launch fits.
+bool fits32(int64_t n) { return n < 0x7fffffffLL - 148 * 64 * kEwThreads; }
+
+int log2_exact(int x) {
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return (1 << l) == x ? l : -1;
+}
+
+// Gradient of the log decays (per-token decay backward).  With b the prefix sum of
+// the log decays g, the loss sees b_s only through the weights exp(b_i - b_j) of
+// o_i = sum_{j<=i} exp(b_i - b_j) (qh_i . kh_j) v_j, so dL/db_s = qh_s . dqh_s -
+// kh_s . dkh_s and dg_t = sum_{s>=t} dL/db_s.  The backward passes' epilogues add
+// the row terms into dg (chunk_tc_kernel); this kernel finishes the sum.
 // dg_t <- sum_{s >= t} dg_s over each sequence, in place.  One CTA
 // per (sequence, head) walks the sequence from its end in tiles of kEwThreads
 // tokens: a block-wide inclusive scan in reversed order plus the running total.
@@ -207,10 +216,18 @@ cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T
   if (D % vw) return cudaErrorInvalidValue;
   const int64_t n = B * T * H * (D / vw);
   if (n == 0) return cudaSuccess;
-  if (dtype == LA_F32)
-    phi_kernel<float><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
-  else
-    phi_kernel<__nv_bfloat16><<<ew_grid(n), kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
+  const unsigned grid = ew_grid(n);
+  if (fits32(n)) {
+    const uint32_t T32 = (uint32_t)T, H32 = (uint32_t)H, D32 = (uint32_t)D, n32 = (uint32_t)n;
+    if (dtype == LA_F32)
+      phi_kernel<float, uint32_t><<<grid, kEwThreads, 0, stream>>>(src, dst, T32, H32, D32, n32, phi);
+    else
+      phi_kernel<__nv_bfloat16, uint32_t><<<grid, kEwThreads, 0, stream>>>(src, dst, T32, H32, D32, n32, phi);
+  } else if (dtype == LA_F32) {
+    phi_kernel<float, int64_t><<<grid, kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
+  } else {
+    phi_kernel<__nv_bfloat16, int64_t><<<grid, kEwThreads, 0, stream>>>(src, dst, T, H, D, n, phi);
+  }
   return cudaGetLastError();
 }
 
@@ -224,26 +241,37 @@ cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n
   return cudaGetLastError();
 }
 
-// v' = [v, 1, 1, 0...] into a contiguous [B * T * H][dvp] bf16 buffer (dv a multiple of 8, dvp > dv).
+// v' = [v, 1, 1, 0...] into a contiguous [B * T * H][dvp] bf16 buffer (dv a multiple
+// of 8 below dvp, dvp / 8 a power of two up to 32).
 cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp,
                          cudaStream_t stream) {
-  if (dv % 8 || dvp % 8 || dvp <= dv) return cudaErrorInvalidValue;
+  const int l = log2_exact(dvp / 8);
+  if (dv % 8 || dvp % 8 || dvp <= dv || l < 0 || l > 5) return cudaErrorInvalidValue;
   const int64_t n = B * T * H * (dvp / 8);
   if (n == 0) return cudaSuccess;
-  aug_v_kernel<<<ew_grid(n), kEwThreads, 0, stream>>>(v, static_cast<__nv_bfloat16 *>(vp), T, H, dv, dvp, n);
+  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(vp);
+  if (fits32(n))
+    aug_v_kernel<uint32_t><<<ew_grid(n), kEwThreads, 0, stream>>>(v, out, (uint32_t)T, (uint32_t)H, dv, l,
+                                                                    (uint32_t)n);
+  else
+    aug_v_kernel<int64_t><<<ew_grid(n), kEwThreads, 0, stream>>>(v, out, T, H, dv, l, n);
   return cudaGetLastError();
 }
 
-// [num, den, den, 0...] -> [u, e_hi, e_lo, 0...] in place, per row of up (see norm_grad_out_kernel).
-cudaError_t launch_norm_grad_out(TensorView dout, void *up, int64_t B, int64_t T, int64_t H, int dv, int dvp,
-                                 cudaStream_t stream) {
-  const int lpr = dvp / 8;
-  if (dv % 8 || dvp <= dv || lpr > 32 || (lpr & (lpr - 1))) return cudaErrorInvalidValue;
-  const int64_t rows = B * T * H;
-  if (rows == 0) return cudaSuccess;
-  const int64_t blocks = (rows + kEwThreads / lpr - 1) / (kEwThreads / lpr);
-  const unsigned grid = (unsigned)(blocks < 148 * 16 ? blocks : 148 * 16);
-  norm_grad_out_kernel<<<grid, kEwThreads, 0, stream>>>(dout, static_cast<__nv_bfloat16 *>(up), T, H, dv, dvp, rows);
+// u' = [dout / den, e_hi, e_lo, 0...] per row from o, den and dout (see norm_grad_out_kernel).
+cudaError_t launch_norm_grad_out(TensorView dout, const void *o, const float *den, void *up, int64_t B, int64_t T,
+                                 int64_t H, int dv, int dvp, cudaStream_t stream) {
+  const int l = log2_exact(dvp / 8);
+  if (dv % 8 || dvp % 8 || dvp <= dv || l < 0 || l > 5) return cudaErrorInvalidValue;
+  const int64_t n = B * T * H * (dvp / 8);
+  if (n == 0) return cudaSuccess;
+  const __nv_bfloat16 *ob = static_cast<const __nv_bfloat16 *>(o);
+  __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(up);
+  if (fits32(n))
+    norm_grad_out_kernel<uint32_t><<<ew_grid(n), kEwThreads, 0, stream>>>(dout, ob, den, u, (uint32_t)T,
+                                                                            (uint32_t)H, dv, l, (uint32_t)n);
+  else
+    norm_grad_out_kernel<int64_t><<<ew_grid(n), kEwThreads, 0, stream>>>(dout, ob, den, u, T, H, dv, l, n);
   return cudaGetLastError();
 }
 

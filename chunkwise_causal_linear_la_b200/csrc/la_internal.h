@@ -46,6 +46,9 @@ struct ChunkArgs {
   float *edg;
   float esign;
   int ephi, edphi;
+  // Normalised forward on the tensor cores: den_t per (token, head), [B * T][H] fp32
+  // (the backward of the normalised form reads it).  NULL: not written.
+  float *den_out;
 };
 
 struct StepArgs {
@@ -95,8 +98,8 @@ cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T
                             int dtype, cudaStream_t stream);
 cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp,
                          cudaStream_t stream);
-cudaError_t launch_norm_grad_out(TensorView dout, void *up, int64_t B, int64_t T, int64_t H, int dv, int dvp,
-                                 cudaStream_t stream);
+cudaError_t launch_norm_grad_out(TensorView dout, const void *o, const float *den, void *up, int64_t B, int64_t T,
+                                 int64_t H, int dv, int dvp, cudaStream_t stream);
 cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,
                                  cudaStream_t stream);
 cudaError_t launch_norm_gate(TensorView o, TensorView g, TensorView y, const float *w, float eps, int64_t B,

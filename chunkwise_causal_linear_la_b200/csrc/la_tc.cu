@@ -137,6 +137,9 @@ struct TcArgs {
   float *edg;
   float esign;
   int ephi, edphi;
+  // Normalised: den_t per (token, head), [B * T][H] fp32, written by the first value
+  // slice's epilogue (NULL: not written).
+  float *den_out;
 };
 
 template <int DK, int DVT, int C, int NS>
@@ -1105,6 +1108,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         edot += __shfl_xor_sync(0xffffffffu, edot, 16);
         if (hf == 0 && lrow(i) < Cp) atomicAdd(a.edg + ((int64_t)bidx * a.T + otok) * a.H + h, a.esign * edot);
       }
+      // the row's denominator: fac is 1 / den, or in decayed-key mode 1 / (den gamma^(C'-1-i))
+      if (NORM && a.den_out && vt == 0 && hf == 0 && lrow(i) < Cp)
+        a.den_out[((int64_t)bidx * a.T + otok) * a.H + h] =
+            vd_mode ? 1.f / fac : 1.f / (fac * pw[Cp - 1 - lrow(i)]);
       return true;
     };
 
@@ -1322,6 +1329,7 @@ cudaError_t launch_cfg(const ChunkArgs &a, void *workspace, cudaStream_t stream,
   t.esign = a.esign;
   t.ephi = a.ephi;
   t.edphi = a.edphi;
+  t.den_out = a.den_out;
   const size_t ob = a.noseg ? 0 : order_bytes(a.n_seqs, a.cu_seqlens != nullptr);
   if (ob > 0 && workspace) {
     int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + seg_ws_bytes(plan, DK, DVT));

@@ -464,17 +464,17 @@ LA_API la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
  *   q, k, v, gamma, cu_seqlens, n_seqs, chunk, phi  as for la_fwd_chunk.
  *   dout, dq, dk, dv  as for la_bwd_chunk.
  *   workspace   device memory of la_bwd_chunk_norm_workspace_size bytes,
- *               256-byte aligned, owned by the caller; it holds [v, 1, 1, 0...],
- *               the forward's [num, den, den, 0...] turned in place into
- *               [u, e_hi, e_lo, 0...] (bf16, d_v + 2 rounded up to 128 or 256
- *               columns) and, with elu + 1, phi(k).  Nothing in it need start
- *               at zero.
- * Kernels: one elementwise pass, the tensor-core forward of (q, k, [v, 1, 1]),
- * one row pass, then the three tensor-core backward passes (plus two
- * feature-map copies with elu + 1).  Rounding: the sums u_t . v_j + e_t cancel
- * (for a one-token sequence exactly, since o_1 = v_1), so the row pass takes e_t
- * from the bf16-rounded u_t (the exact gradient for an output gradient within
- * one bf16 rounding of dout) and stores it as a bf16 pair e_hi + e_lo.
+ *               256-byte aligned, owned by the caller; it holds [v, 1, 1, 0...]
+ *               and [u, e_hi, e_lo, 0...] (bf16, d_v + 2 rounded up to 128 or
+ *               256 columns), the forward's o (bf16) and den (fp32) and, with
+ *               elu + 1, phi(k).  Nothing in it need start at zero.
+ * Kernels: the tensor-core normalised forward (which also writes den_t), two
+ * row passes ([v, 1, 1] and [u, e]), then the three tensor-core backward
+ * passes (plus two feature-map copies with elu + 1).  Rounding: the sums
+ * u_t . v_j + e_t cancel (for a one-token sequence exactly, since o_1 = v_1),
+ * so e_t = -(u_t . o_t) is taken from the bf16-rounded u_t (the exact gradient
+ * for an output gradient within one bf16 rounding of dout) and stored as a
+ * bf16 pair e_hi + e_lo.
  * Shapes: bf16, chunk 64, d_v in {64, 128}, d_k in {64, 128, 256}; anything
  * else, f32 and LA_FLAG_SIMT return LA_ERR_UNSUPPORTED.  den_t = 0 gives
  * non-finite gradients, as it gives a non-finite forward output.

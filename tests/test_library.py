@@ -243,8 +243,8 @@ def test_host_arena_size_and_validation(lib):
 
 def test_bwd_norm_workspace_and_validation_on_host(lib):
     """la_bwd_chunk_norm_workspace_size: the augmented value rows ([v, 1, 1] rounded up
-    to 128 or 256 columns) twice, plus phi(k), each at a 256-byte boundary; -1 for
-    what la_bwd_chunk_norm rejects.  Bad arguments and a short or misaligned
+    to 128 or 256 columns) twice, the forward's o (bf16) and den (fp32), and phi(k),
+    each at a 256-byte boundary; -1 for what la_bwd_chunk_norm rejects.  Bad arguments and a short or misaligned
     workspace are rejected before any device call."""
     from chunkwise_causal_linear_la_b200 import binding as b
 
@@ -252,9 +252,12 @@ def test_bwd_norm_workspace_and_validation_on_host(lib):
     bad = ctypes.c_size_t(-1).value
     rows = 3 * 100 * 5
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert ws(3, 100, 5, 128, 128, 64, 1, 0) == 2 * up(rows * 256 * 2) + up(rows * 128 * 2)
-    assert ws(3, 100, 5, 64, 64, 64, 1, 0) == 2 * up(rows * 128 * 2) + up(rows * 64 * 2)
-    assert ws(3, 100, 5, 256, 128, 64, 1, 0) == 2 * up(rows * 256 * 2) + up(rows * 256 * 2)
+    def expect(dk, dv, dvp):
+        return 2 * up(rows * dvp * 2) + up(rows * dv * 2) + up(rows * 4) + up(rows * dk * 2)
+    assert ws(3, 100, 5, 128, 128, 64, 1, 0) == expect(128, 128, 256)
+    assert ws(3, 100, 5, 64, 64, 64, 1, 0) == expect(64, 64, 128)
+    assert ws(3, 100, 5, 256, 128, 64, 1, 0) == expect(256, 128, 256)
+    assert ws(3, 100, 5, 128, 64, 64, 1, 0) == expect(128, 64, 128)
     assert ws(3, 100, 5, 128, 256, 64, 1, 0) == bad  # d_v + 2 does not fit 256 columns
     assert ws(3, 100, 5, 128, 128, 32, 1, 0) == bad  # chunk
     assert ws(3, 100, 5, 128, 128, 64, 0, 0) == bad  # f32
