@@ -678,39 +678,56 @@ la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
   return bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags, stream);
 }
 
-// The backward of la_fwd_chunk's normalised form (o_t = num_t / den_t), on the
-// tensor cores through the unnormalised backward of an augmented problem.  With
-// the value rows widened to v'_t = [v_t, 1, 1, 0...] and the output gradient to
-// u'_t = [u_t, e_t, 0...], u_t = dout_t / den_t and e_t = -(u_t . o_t) (the
-// denominator's adjoint, carried as a bf16 pair over the two columns of ones),
-// the unnormalised backward of (q, k, v', u') gives dq and dk of the normalised
-// recurrence, and dv as the first d_v columns of dv'.
-// Steps: v' (elementwise), the normalised forward (o and den_t), u' (one row
-// pass), then the three backward passes of la_bwd_chunk with u' as the output
-// gradient; the dv pass reads only u''s first d_v columns.
+// The backward of la_fwd_chunk's normalised form (o_t = num_t / den_t) through the
+// unnormalised backward of an augmented problem.  With the value rows widened to
+// v'_t = [v_t, 1, 1, 0...] and the output gradient to u'_t = [u_t, e_t, 0...],
+// u_t = dout_t / den_t and e_t = -(u_t . o_t) (the denominator's adjoint, carried
+// as a pair e_hi + e_lo over the two columns of ones), the unnormalised backward
+// of (q, k, v', u') gives dq and dk of the normalised recurrence, and dv as the
+// first d_v columns of dv'.
+//   Tensor cores (bf16, chunk 64): the normalised forward (o, and den_t from its
+//   epilogue), v' and u' (row passes), then the three passes of la_bwd_chunk with
+//   u' as the output gradient; the dv pass reads only u''s first d_v columns.
+//   CUDA cores (f32, other chunks, LA_FLAG_SIMT): the unnormalised forward of
+//   (q, k, v') gives [num, den, den, 0...], turned into u' in place; the backward
+//   kernel on (q, k, v', u') writes dv' to the workspace, and a copy takes dv.
 namespace {
 
-// Widths of the augmented value rows: d_v + 2 rounded up to a tensor-core key width.
-int64_t norm_aug_width(int64_t dv) { return dv == 64 ? 128 : dv == 128 ? 256 : -1; }
+// Widths of the augmented value rows: d_v + 2 rounded up to a head dim the
+// kernels take (tensor cores: 128 or 256 as the key width of the widened passes).
+int64_t norm_aug_width(int64_t dv) { return dv >= 16 && dv <= 128 && (dv & (dv - 1)) == 0 ? 2 * dv : -1; }
 
 struct NormBwdWs {
-  size_t vp, up, o, den, kh, total;  // byte offsets of v', u', o, den, phi(k); total size
+  bool tc;  // the tensor-core route
+  // byte offsets: v', u' (both routes); o, den, phi(k) (tensor cores); dv' (CUDA cores); total size
+  size_t vp, up, o, den, kh, dvw, total;
 };
 
 bool norm_bwd_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int32_t chunk, int32_t dtype,
                    int32_t flags, NormBwdWs *w) {
   const int64_t dvp = norm_aug_width(dv);
-  if (dtype != LA_BF16 || chunk != 64 || (flags & LA_FLAG_SIMT) || dvp < 0 || B < 0 || T < 0 || H <= 0)
+  if ((dtype != LA_BF16 && dtype != LA_F32) || dvp < 0 || B < 0 || T < 0 || H <= 0 || (flags & ~LA_FLAG_SIMT))
     return false;
-  if (!tc_shape((int)dvp, (int)dk) || !tc_shape((int)dk, (int)dv)) return false;
+  if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return false;
+  if (!head_dim_ok(dk) || !head_dim_ok(dvp)) return false;
+  w->tc = dtype == LA_BF16 && chunk == 64 && !(flags & LA_FLAG_SIMT) && tc_shape((int)dvp, (int)dk) &&
+          tc_shape((int)dk, (int)dv);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  const size_t rows = (size_t)(B * T * H);
+  const size_t rows = (size_t)(B * T * H), es = dtype == LA_F32 ? 4 : 2;
   w->vp = 0;
-  w->up = up(rows * dvp * 2);
-  w->o = w->up + up(rows * dvp * 2);
-  w->den = w->o + up(rows * dv * 2);
-  w->kh = w->den + up(rows * 4);
-  w->total = w->kh + up(rows * dk * 2);
+  w->up = up(rows * dvp * es);
+  const size_t end = w->up + up(rows * dvp * es);
+  if (w->tc) {
+    w->o = end;
+    w->den = w->o + up(rows * dv * es);
+    w->kh = w->den + up(rows * 4);
+    w->total = w->kh + up(rows * dk * es);
+    w->dvw = 0;
+  } else {
+    w->dvw = end;
+    w->total = w->dvw + up(rows * dvp * es);
+    w->o = w->den = w->kh = 0;
+  }
   return true;
 }
 
@@ -750,16 +767,19 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   }
   NormBwdWs w;
   if (!norm_bwd_plan(q->B, q->T, q->H, q->D, v->D, chunk, q->dtype, flags, &w))
-    return fail(LA_ERR_UNSUPPORTED, "the normalised backward runs on the tensor cores only: bf16, chunk 64, "
-                "d_v in {64, 128}, d_k in {64, 128, 256}");
+    return fail(LA_ERR_UNSUPPORTED, "the normalised backward takes d_v in {16, 32, 64, 128}, d_k in "
+                "{16, 32, 64, 128, 256} and chunk in {16, 32, 64, 128}");
   if (!workspace || workspace_bytes < w.total)
     return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
   if (((uintptr_t)workspace) % 256 != 0) return fail(LA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  int device = 0;
+  cudaError_t err = cudaGetDevice(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
   if (n_seqs == 0 || q->T == 0 || q->B == 0) return ok();
 
   const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D, Dv = v->D, Dvp = norm_aug_width(Dv);
   uint8_t *base = static_cast<uint8_t *>(workspace);
-  // contiguous [B, T, H, D] bf16 buffers in the workspace
+  // contiguous [B, T, H, D] buffers of q's dtype in the workspace
   auto buf = [&](size_t off, int64_t D) {
     la_tensor t;
     t.data = base + off;
@@ -773,10 +793,7 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     t.stride_b = T * H * D;
     return t;
   };
-  const la_tensor vp = buf(w.vp, Dvp), up = buf(w.up, Dvp), o = buf(w.o, Dv), kh = buf(w.kh, Dk);
-  float *den = reinterpret_cast<float *>(base + w.den);
-  la_tensor u_head = up;  // u' seen as its first d_v columns: dout / den
-  u_head.D = Dv;
+  const la_tensor vp = buf(w.vp, Dvp), up = buf(w.up, Dvp);
   const bool elu = phi == LA_PHI_ELU1;
   cudaStream_t st = (cudaStream_t)stream;
 
@@ -790,21 +807,20 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   f.T = T;
   f.n_seqs = n_seqs;
   f.H = (int)H;
-  f.chunk = 64;
+  f.chunk = chunk;
   f.normalize = 0;
   f.dtype = q->dtype;
+  f.rev = 0;
   f.noseg = 1;
   f.ng_w = nullptr;
   f.ng_gate = TensorView{nullptr, 0, 0, 0};
   f.ng_eps = 0.f;
+  f.ex = TensorView{nullptr, 0, 0, 0};
   f.edg = nullptr;
   f.esign = 0.f;
+  f.ephi = f.edphi = 0;
   f.den_out = nullptr;
-  const char *why = nullptr;
-  // one tensor-core pass: out = fwd or rev(qq, kk, vv) with feature map ph on qq and kk; x (the
-  // input whose gradient this pass produces) makes the epilogue scale by phi'(x)
-  auto run = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
-                 int rev, const la_tensor *x) -> cudaError_t {
+  auto set_io = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo) {
     f.q = view(qq);
     f.k = view(kk);
     f.v = view(vv);
@@ -814,6 +830,57 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     f.o_sh = oo->stride_h;
     f.dk = (int)qq->D;
     f.dv = (int)vv->D;
+  };
+
+  if (!w.tc) {  // ---- CUDA cores
+    const la_tensor dvw = buf(w.dvw, Dvp);
+    set_io(q, k, &vp, &up);
+    f.phi = phi;
+    BwdArgs b;
+    b.q = view(q);
+    b.k = view(k);
+    b.v = view(&vp);
+    b.dout = view(&up);
+    b.dq = view(dq);
+    b.dk_ = view(dk);
+    b.dv_ = view(&dvw);
+    b.gamma = gamma;
+    b.cu_seqlens = cu_seqlens;
+    b.T = T;
+    b.n_seqs = n_seqs;
+    b.H = (int)H;
+    b.dk = (int)Dk;
+    b.dv = (int)Dvp;
+    b.chunk = chunk;
+    b.phi = phi;
+    b.dtype = q->dtype;
+    if (!simt_supported(f, device) || !bwd_supported(b, device))
+      return fail(LA_ERR_UNSUPPORTED, "d_k %lld x widened d_v %lld does not fit the CUDA-core kernels' shared "
+                  "memory", (long long)Dk, (long long)Dvp);
+    la_tensor dv_head = dvw;  // dv' seen as its first d_v columns
+    dv_head.D = Dv;
+    if ((err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, q->dtype, st)) != cudaSuccess ||
+        (err = launch_chunk_simt(f, st)) != cudaSuccess ||
+        (err = launch_norm_grad_num(view(dout), up.data, B, T, H, (int)Dv, (int)Dvp, q->dtype, st)) !=
+            cudaSuccess ||
+        (err = launch_bwd(b, st)) != cudaSuccess ||
+        (err = launch_phi_copy(view(&dv_head), view(dv), B, T, H, Dv, LA_PHI_IDENTITY, q->dtype, st)) !=
+            cudaSuccess)
+      return fail(LA_ERR_CUDA, "normalised backward (CUDA cores): %s", cudaGetErrorString(err));
+    return ok();
+  }
+
+  // ---- tensor cores
+  const la_tensor o = buf(w.o, Dv), kh = buf(w.kh, Dk);
+  float *den = reinterpret_cast<float *>(base + w.den);
+  la_tensor u_head = up;  // u' seen as its first d_v columns: dout / den
+  u_head.D = Dv;
+  const char *why = nullptr;
+  // one tensor-core pass: out = fwd or rev(qq, kk, vv) with feature map ph on qq and kk; x (the
+  // input whose gradient this pass produces) makes the epilogue scale by phi'(x)
+  auto run = [&](const la_tensor *qq, const la_tensor *kk, const la_tensor *vv, const la_tensor *oo, int ph,
+                 int rev, const la_tensor *x) -> cudaError_t {
+    set_io(qq, kk, vv, oo);
     f.phi = ph;
     f.rev = rev;
     f.ex = x && elu ? view(x) : TensorView{nullptr, 0, 0, 0};
@@ -822,7 +889,6 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     if (!tc_supported(f)) return cudaErrorInvalidValue;
     return launch_chunk_tc(f, nullptr, 0, st, &why);
   };
-  cudaError_t err;
   // the normalised forward (o, and den_t from its epilogue), then u'
   f.normalize = 1;
   f.den_out = den;
@@ -830,7 +896,7 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   f.normalize = 0;
   f.den_out = nullptr;
   if (err != cudaSuccess ||
-      (err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, st)) != cudaSuccess ||
+      (err = launch_aug_v(view(v), vp.data, B, T, H, (int)Dv, (int)Dvp, q->dtype, st)) != cudaSuccess ||
       (err = launch_norm_grad_out(view(dout), o.data, den, up.data, B, T, H, (int)Dv, (int)Dvp, st)) !=
           cudaSuccess)
     return fail(LA_ERR_CUDA, "normalised backward (forward and output gradient): %s%s%s", cudaGetErrorString(err),

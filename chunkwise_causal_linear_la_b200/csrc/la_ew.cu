@@ -88,23 +88,82 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&f)[8]) {
 // Both kernels write contiguous [rows][dvp] bf16 rows, one thread per 16-byte
 // vector (lpr = dvp / 8 vectors per row, a power of two, so a row's vectors sit
 // in one warp); dv is a multiple of 8 below dvp.
-template <typename I>
-__global__ void __launch_bounds__(kEwThreads) aug_v_kernel(TensorView v, __nv_bfloat16 *vp, I T_, I H, int dv,
-                                                            int lpr_log2, I nvec) {
+template <typename T, typename I>
+__global__ void __launch_bounds__(kEwThreads) aug_v_kernel(TensorView v, T *vp, I T_, I H, int dv, int lpr_log2,
+                                                            I nvec) {
+  constexpr int VW = Vec<T>::VW;
   const int lpr = 1 << lpr_log2;
   for (I e = blockIdx.x * (I)kEwThreads + threadIdx.x; e < nvec; e += (I)gridDim.x * kEwThreads) {
     const I row = e >> lpr_log2;
-    const int col = (int)(e & (I)(lpr - 1)) * 8;
+    const int col = (int)(e & (I)(lpr - 1)) * VW;
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
     if (col < dv) {
       I b, t, h;
       split_row<I>(row, T_, H, b, t, h);
-      x = *reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)v.data + (int64_t)b * v.sb +
-                                           (int64_t)t * v.st + (int64_t)h * v.sh + col);
-    } else if (col == dv) {
-      x.x = 0x3F803F80u;  // bf16 1.0 in columns dv and dv + 1
+      x = *reinterpret_cast<const uint4 *>((const T *)v.data + (int64_t)b * v.sb + (int64_t)t * v.st +
+                                           (int64_t)h * v.sh + col);
+    } else if (col == dv) {  // ones in columns dv and dv + 1
+      T *xv = reinterpret_cast<T *>(&x);
+      xv[0] = xv[1] = from_f32<T>(1.f);
     }
-    *reinterpret_cast<uint4 *>(vp + (int64_t)row * (8 << lpr_log2) + col) = x;
+    *reinterpret_cast<uint4 *>(vp + (int64_t)row * (VW << lpr_log2) + col) = x;
+  }
+}
+
+// The CUDA-core route: rows of the unnormalised forward of (q, k, v'), [num, den,
+// den, 0...], turned into [u, e_hi, e_lo, 0...] in place (e_t = -(u_t . num_t) /
+// den_t from u_t as stored); dout through its strides; T is the rows' element type.
+template <typename T, typename I>
+__global__ void __launch_bounds__(kEwThreads) norm_grad_num_kernel(TensorView dout, T *up, I T_, I H, int dv,
+                                                                    int lpr_log2, I nvec) {
+  constexpr int VW = Vec<T>::VW;
+  const int lpr = 1 << lpr_log2;
+  const int lane = threadIdx.x & 31;
+  const int den_lane = (lane & ~(lpr - 1)) + dv / VW;  // the lane of this row holding column dv
+  for (I e0 = blockIdx.x * (I)kEwThreads; e0 < nvec; e0 += (I)gridDim.x * kEwThreads) {
+    const I e = e0 + threadIdx.x;  // rows are whole within a warp and the loop bound is warp-uniform
+    const bool live = e < nvec;
+    const I row = live ? e >> lpr_log2 : 0;
+    const int col = (int)(e & (I)(lpr - 1)) * VW;
+    T *p = up + (int64_t)row * (VW << lpr_log2) + col;
+    float f[VW], d[VW];
+#pragma unroll
+    for (int u = 0; u < VW; ++u) f[u] = d[u] = 0.f;
+    if (live) {
+      const uint4 x = *reinterpret_cast<const uint4 *>(p);
+      const T *xv = reinterpret_cast<const T *>(&x);
+#pragma unroll
+      for (int u = 0; u < VW; ++u) f[u] = to_f32<T>(xv[u]);
+      if (col < dv) {
+        I b, t, h;
+        split_row<I>(row, T_, H, b, t, h);
+        const uint4 y = *reinterpret_cast<const uint4 *>((const T *)dout.data + (int64_t)b * dout.sb +
+                                                         (int64_t)t * dout.st + (int64_t)h * dout.sh + col);
+        const T *yv = reinterpret_cast<const T *>(&y);
+#pragma unroll
+        for (int u = 0; u < VW; ++u) d[u] = to_f32<T>(yv[u]);
+      }
+    }
+    const float den = __shfl_sync(0xffffffffu, f[0], den_lane);
+    const float inv = 1.f / den;
+    float y[VW], dot = 0.f;
+#pragma unroll
+    for (int u = 0; u < VW; ++u) {
+      y[u] = col < dv ? to_f32<T>(from_f32<T>(d[u] * inv)) : 0.f;  // u as stored
+      dot = fmaf(y[u], f[u], dot);                                   // u . num
+    }
+    for (int s = lpr / 2; s > 0; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
+    if (!live) continue;
+    if (col == dv) {
+      const float ev = -dot * inv;
+      y[0] = to_f32<T>(from_f32<T>(ev));
+      y[1] = ev - y[0];
+    }
+    uint4 o;
+    T *ov = reinterpret_cast<T *>(&o);
+#pragma unroll
+    for (int u = 0; u < VW; ++u) ov[u] = from_f32<T>(y[u]);
+    *reinterpret_cast<uint4 *>(p) = o;
   }
 }
 
@@ -241,20 +300,58 @@ cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n
   return cudaGetLastError();
 }
 
-// v' = [v, 1, 1, 0...] into a contiguous [B * T * H][dvp] bf16 buffer (dv a multiple
-// of 8 below dvp, dvp / 8 a power of two up to 32).
-cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+// v' = [v, 1, 1, 0...] into a contiguous [B * T * H][dvp] buffer of v's dtype (dv a
+// multiple of the vector width below dvp, dvp / width a power of two up to 32).
+cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp, int dtype,
                          cudaStream_t stream) {
-  const int l = log2_exact(dvp / 8);
-  if (dv % 8 || dvp % 8 || dvp <= dv || l < 0 || l > 5) return cudaErrorInvalidValue;
-  const int64_t n = B * T * H * (dvp / 8);
+  const int vw = dtype == LA_F32 ? 4 : 8;
+  const int l = log2_exact(dvp / vw);
+  if (dv % vw || dvp % vw || dvp <= dv || l < 0 || l > 5) return cudaErrorInvalidValue;
+  const int64_t n = B * T * H * (dvp / vw);
   if (n == 0) return cudaSuccess;
-  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(vp);
-  if (fits32(n))
-    aug_v_kernel<uint32_t><<<ew_grid(n), kEwThreads, 0, stream>>>(v, out, (uint32_t)T, (uint32_t)H, dv, l,
-                                                                    (uint32_t)n);
-  else
-    aug_v_kernel<int64_t><<<ew_grid(n), kEwThreads, 0, stream>>>(v, out, T, H, dv, l, n);
+  const unsigned grid = ew_grid(n);
+  if (dtype == LA_F32) {
+    float *out = static_cast<float *>(vp);
+    if (fits32(n))
+      aug_v_kernel<float, uint32_t><<<grid, kEwThreads, 0, stream>>>(v, out, (uint32_t)T, (uint32_t)H, dv, l,
+                                                                      (uint32_t)n);
+    else
+      aug_v_kernel<float, int64_t><<<grid, kEwThreads, 0, stream>>>(v, out, T, H, dv, l, n);
+  } else {
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(vp);
+    if (fits32(n))
+      aug_v_kernel<__nv_bfloat16, uint32_t><<<grid, kEwThreads, 0, stream>>>(v, out, (uint32_t)T, (uint32_t)H, dv,
+                                                                              l, (uint32_t)n);
+    else
+      aug_v_kernel<__nv_bfloat16, int64_t><<<grid, kEwThreads, 0, stream>>>(v, out, T, H, dv, l, n);
+  }
+  return cudaGetLastError();
+}
+
+// [num, den, den, 0...] -> [u, e_hi, e_lo, 0...] in place (see norm_grad_num_kernel).
+cudaError_t launch_norm_grad_num(TensorView dout, void *up, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+                                 int dtype, cudaStream_t stream) {
+  const int vw = dtype == LA_F32 ? 4 : 8;
+  const int l = log2_exact(dvp / vw);
+  if (dv % vw || dvp % vw || dvp <= dv || l < 0 || l > 5) return cudaErrorInvalidValue;
+  const int64_t n = B * T * H * (dvp / vw);
+  if (n == 0) return cudaSuccess;
+  const unsigned grid = ew_grid(n);
+  if (dtype == LA_F32) {
+    float *u = static_cast<float *>(up);
+    if (fits32(n))
+      norm_grad_num_kernel<float, uint32_t><<<grid, kEwThreads, 0, stream>>>(dout, u, (uint32_t)T, (uint32_t)H, dv,
+                                                                              l, (uint32_t)n);
+    else
+      norm_grad_num_kernel<float, int64_t><<<grid, kEwThreads, 0, stream>>>(dout, u, T, H, dv, l, n);
+  } else {
+    __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(up);
+    if (fits32(n))
+      norm_grad_num_kernel<__nv_bfloat16, uint32_t><<<grid, kEwThreads, 0, stream>>>(
+          dout, u, (uint32_t)T, (uint32_t)H, dv, l, (uint32_t)n);
+    else
+      norm_grad_num_kernel<__nv_bfloat16, int64_t><<<grid, kEwThreads, 0, stream>>>(dout, u, T, H, dv, l, n);
+  }
   return cudaGetLastError();
 }
 

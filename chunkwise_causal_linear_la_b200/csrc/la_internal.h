@@ -96,8 +96,10 @@ bool simt_supported(const ChunkArgs &a, int device);
 bool bwd_supported(const BwdArgs &a, int device);
 cudaError_t launch_phi_copy(TensorView src, TensorView dst, int64_t B, int64_t T, int64_t H, int64_t D, int phi,
                             int dtype, cudaStream_t stream);
-cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+cudaError_t launch_aug_v(TensorView v, void *vp, int64_t B, int64_t T, int64_t H, int dv, int dvp, int dtype,
                          cudaStream_t stream);
+cudaError_t launch_norm_grad_num(TensorView dout, void *up, int64_t B, int64_t T, int64_t H, int dv, int dvp,
+                                 int dtype, cudaStream_t stream);
 cudaError_t launch_norm_grad_out(TensorView dout, const void *o, const float *den, void *up, int64_t B, int64_t T,
                                  int64_t H, int dv, int dvp, cudaStream_t stream);
 cudaError_t launch_dg_rev_cumsum(float *dg, const int32_t *cu_seqlens, int64_t n_seqs, int64_t T, int64_t H,

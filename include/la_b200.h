@@ -465,19 +465,25 @@ LA_API la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, cons
  *   dout, dq, dk, dv  as for la_bwd_chunk.
  *   workspace   device memory of la_bwd_chunk_norm_workspace_size bytes,
  *               256-byte aligned, owned by the caller; it holds [v, 1, 1, 0...]
- *               and [u, e_hi, e_lo, 0...] (bf16, d_v + 2 rounded up to 128 or
- *               256 columns), the forward's o (bf16) and den (fp32) and, with
- *               elu + 1, phi(k).  Nothing in it need start at zero.
- * Kernels: the tensor-core normalised forward (which also writes den_t), two
- * row passes ([v, 1, 1] and [u, e]), then the three tensor-core backward
- * passes (plus two feature-map copies with elu + 1).  Rounding: the sums
+ *               and [u, e_hi, e_lo, 0...] (q's dtype, 2 d_v columns) and, on
+ *               the tensor cores, the forward's o and den (fp32) and, with
+ *               elu + 1, phi(k); on the CUDA cores the widened dv as well.
+ *               Nothing in it need start at zero.
+ * Kernels: bf16 with chunk 64, d_v in {64, 128} and d_k in {64, 128, 256} run
+ * on the tensor cores: the normalised forward (which also writes den_t), two
+ * row passes ([v, 1, 1] and [u, e]), then the three backward passes (plus two
+ * feature-map copies with elu + 1).  f32, the other chunks, d_v in {16, 32}
+ * and LA_FLAG_SIMT run on the CUDA-core kernels in fp32: the unnormalised
+ * forward of (q, k, [v, 1, 1]) gives [num, den], a row pass turns it into
+ * [u, e], the backward kernel runs on the widened values, and a copy takes dv;
+ * shapes whose widened rows do not fit that kernel's shared memory (d_k = 128
+ * with d_v = 128, say) return LA_ERR_UNSUPPORTED.  Rounding: the sums
  * u_t . v_j + e_t cancel (for a one-token sequence exactly, since o_1 = v_1),
- * so e_t = -(u_t . o_t) is taken from the bf16-rounded u_t (the exact gradient
- * for an output gradient within one bf16 rounding of dout) and stored as a
- * bf16 pair e_hi + e_lo.
- * Shapes: bf16, chunk 64, d_v in {64, 128}, d_k in {64, 128, 256}; anything
- * else, f32 and LA_FLAG_SIMT return LA_ERR_UNSUPPORTED.  den_t = 0 gives
- * non-finite gradients, as it gives a non-finite forward output.
+ * so e_t = -(u_t . o_t) is taken from u_t as stored (the exact gradient for an
+ * output gradient within one rounding of dout) and kept as a pair
+ * e_hi + e_lo.  d_v = 256 (widened past 256 columns), other chunks and head
+ * dims return LA_ERR_UNSUPPORTED.  den_t = 0 gives non-finite gradients, as
+ * it gives a non-finite forward output.
  * LA_ERR_WORKSPACE if workspace is NULL or short.  Other errors as for
  * la_bwd_chunk.  la_bwd_chunk_norm_workspace_size returns (size_t)-1 for
  * shapes, chunks, dtypes or flags that la_bwd_chunk_norm rejects.

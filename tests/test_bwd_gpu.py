@@ -278,10 +278,11 @@ def _norm_bwd_scales(oracle_mod, q, k, v, dout, gamma, cu, phi, slices):
     return scales
 
 
-def _check_norm(la, oracle_mod, q, k, v, dout, gamma, cu=None, phi="elu1"):
+def _check_norm(la, oracle_mod, q, k, v, dout, gamma, cu=None, phi="elu1", chunk=64, flags=0):
     dev = torch.device("cuda")
     dq, dk, dv = la.la_bwd_chunk_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), gamma.to(dev),
-                                      cu_seqlens=None if cu is None else cu.to(dev), phi=phi)
+                                      cu_seqlens=None if cu is None else cu.to(dev), phi=phi, chunk=chunk,
+                                      flags=flags)
     torch.cuda.synchronize()
     g64, cu_np = gamma.double().numpy(), None if cu is None else cu.numpy()
     refs = oracle_mod.backward_norm(q, k, v, dout, g64, cu_seqlens=cu_np, phi=phi)
@@ -290,7 +291,7 @@ def _check_norm(la, oracle_mod, q, k, v, dout, gamma, cu=None, phi="elu1"):
     sq, sk = _norm_bwd_scales(oracle_mod, q, k, v, dout, g64, cu_np, phi, sl)
     assert all(np.isfinite(to_np(x)).all() for x in (dq, dk, dv))
     errs = [slice_rel_err(to_np(x), r, sl, scale=s) for x, r, s in zip((dq, dk, dv), refs, (sq, sk, None))]
-    assert max(errs) < TOL[torch.bfloat16], errs
+    assert max(errs) < TOL[q.dtype], errs
 
 
 @pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64), (256, 128)])
@@ -345,10 +346,37 @@ def test_bwd_norm_caller_workspace_reused(la, oracle_mod):
     assert max(slice_rel_err(to_np(x), r, sl, scale=sc) for x, r, sc in zip(a, refs, scales)) < TOL[torch.bfloat16]
 
 
+@pytest.mark.parametrize("T", [1, 100, 256])
+def test_bwd_norm_f32_cuda_cores(la, oracle_mod, T):
+    """f32 (the tiny workload's dtype: d = 64, elu + 1, normaliser, gamma = 1) runs on
+    the CUDA-core kernels in fp32."""
+    q, k, v, dout = _inputs(1, T, 2, 64, 64, torch.float32, 67 + T)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.9]))
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 128])
+def test_bwd_norm_other_chunks(la, oracle_mod, chunk):
+    """bf16 with a chunk other than 64 takes the CUDA-core route."""
+    q, k, v, dout = _inputs(2, 3 * chunk + 5, 2, 64, 64, torch.bfloat16, 71 + chunk)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.95]), chunk=chunk)
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 16), (64, 32), (128, 64)])
+def test_bwd_norm_cuda_core_shapes(la, oracle_mod, dk, dv):
+    """Small heads (no tensor-core shape) and LA_FLAG_SIMT; packed batch with f32."""
+    q, k, v, dout = _inputs(1, 150, 2, dk, dv, torch.bfloat16, dk + dv)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.8]), flags=la.LA_FLAG_SIMT)
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([70, 0, 1, 64, 15])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 2, dk, dv, torch.float32, dk * dv)
+    _check_norm(la, oracle_mod, q, k, v, dout, torch.tensor([1.0, 0.9]), cu=cu)
+
+
 def test_bwd_norm_unsupported(la):
     dev = torch.device("cuda")
     assert la.bwd_norm_workspace_size(1, 64, 2, 128, 256) == -1
-    assert la.bwd_norm_workspace_size(1, 64, 2, 128, 128, dtype=torch.float32) == -1
+    assert la.bwd_norm_workspace_size(1, 64, 2, 128, 128, chunk=48) == -1
     q, k, v, dout = _inputs(1, 64, 2, 128, 256, torch.bfloat16, 61)
     with pytest.raises(la.LaError) as e:
         la.la_bwd_chunk_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), torch.ones(2, device=dev))

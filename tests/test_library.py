@@ -242,35 +242,46 @@ def test_host_arena_size_and_validation(lib):
 
 
 def test_bwd_norm_workspace_and_validation_on_host(lib):
-    """la_bwd_chunk_norm_workspace_size: the augmented value rows ([v, 1, 1] rounded up
-    to 128 or 256 columns) twice, the forward's o (bf16) and den (fp32), and phi(k),
-    each at a 256-byte boundary; -1 for what la_bwd_chunk_norm rejects.  Bad arguments and a short or misaligned
-    workspace are rejected before any device call."""
+    """la_bwd_chunk_norm_workspace_size, each region at a 256-byte boundary: on the
+    tensor-core route (bf16, chunk 64, d_v in {64, 128}) the augmented rows ([v, 1, 1]
+    rounded up to 2 d_v columns) twice, the forward's o (bf16) and den (fp32), and
+    phi(k); on the CUDA-core route (f32, other chunks, LA_FLAG_SIMT, d_v of 16 or 32)
+    the augmented rows three times (v', u', dv'); -1 for what la_bwd_chunk_norm
+    rejects.  Bad arguments and a short or misaligned workspace are rejected before
+    any device call."""
     from chunkwise_causal_linear_la_b200 import binding as b
 
     ws = lib.la_bwd_chunk_norm_workspace_size
     bad = ctypes.c_size_t(-1).value
     rows = 3 * 100 * 5
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    def expect(dk, dv, dvp):
-        return 2 * up(rows * dvp * 2) + up(rows * dv * 2) + up(rows * 4) + up(rows * dk * 2)
-    assert ws(3, 100, 5, 128, 128, 64, 1, 0) == expect(128, 128, 256)
-    assert ws(3, 100, 5, 64, 64, 64, 1, 0) == expect(64, 64, 128)
-    assert ws(3, 100, 5, 256, 128, 64, 1, 0) == expect(256, 128, 256)
-    assert ws(3, 100, 5, 128, 64, 64, 1, 0) == expect(128, 64, 128)
+
+    def tc(dk, dv):
+        return 2 * up(rows * 2 * dv * 2) + up(rows * dv * 2) + up(rows * 4) + up(rows * dk * 2)
+
+    def cc(dv, es):
+        return 3 * up(rows * 2 * dv * es)
+    assert ws(3, 100, 5, 128, 128, 64, 1, 0) == tc(128, 128)
+    assert ws(3, 100, 5, 64, 64, 64, 1, 0) == tc(64, 64)
+    assert ws(3, 100, 5, 256, 128, 64, 1, 0) == tc(256, 128)
+    assert ws(3, 100, 5, 128, 64, 64, 1, 0) == tc(128, 64)
+    assert ws(3, 100, 5, 128, 128, 32, 1, 0) == cc(128, 2)  # chunk 32: CUDA cores
+    assert ws(3, 100, 5, 128, 128, 64, 1, 1) == cc(128, 2)  # LA_FLAG_SIMT
+    assert ws(3, 100, 5, 64, 64, 64, 0, 0) == cc(64, 4)  # f32
+    assert ws(3, 100, 5, 32, 32, 16, 0, 0) == cc(32, 4)
+    assert ws(3, 100, 5, 64, 16, 64, 1, 0) == cc(16, 2)  # d_v = 16: widened to 32, no tensor-core shape
     assert ws(3, 100, 5, 128, 256, 64, 1, 0) == bad  # d_v + 2 does not fit 256 columns
-    assert ws(3, 100, 5, 128, 128, 32, 1, 0) == bad  # chunk
-    assert ws(3, 100, 5, 128, 128, 64, 0, 0) == bad  # f32
-    assert ws(3, 100, 5, 128, 128, 64, 1, 1) == bad  # LA_FLAG_SIMT
-    assert ws(3, 100, 5, 32, 128, 64, 1, 0) == bad  # d_k
+    assert ws(3, 100, 5, 128, 128, 48, 1, 0) == bad  # chunk
+    assert ws(3, 100, 5, 96, 128, 64, 1, 0) == bad  # d_k
+    assert ws(3, 100, 5, 128, 128, 64, 1, 4) == bad  # unknown flag
     assert ws(3, 100, 0, 128, 128, 64, 1, 0) == bad  # H = 0
 
     need = ws(1, 4, 2, 128, 128, 64, 1, 0)
     q, k, v, do, dq, dk, dv = (_t(D=128) for _ in range(7))
 
-    def call(gamma=0x2000, phi=1, ws_ptr=0x100000, ws_bytes=None, qq=None, vv=None, flags=0):
+    def call(gamma=0x2000, phi=1, ws_ptr=0x100000, ws_bytes=None, qq=None, vv=None, flags=0, chunk=64):
         return lib.la_bwd_chunk_norm(ctypes.byref(qq or q), ctypes.byref(k), ctypes.byref(vv or v), ctypes.byref(do),
-                                     gamma, None, 1, 64, phi, ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv),
+                                     gamma, None, 1, chunk, phi, ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv),
                                      flags, ws_ptr, need if ws_bytes is None else ws_bytes, None)
     assert call(gamma=None) == b.LA_ERR_INVALID_ARG and b"gamma" in lib.la_last_error()
     assert call(phi=5) == b.LA_ERR_INVALID_ARG
@@ -280,8 +291,9 @@ def test_bwd_norm_workspace_and_validation_on_host(lib):
     assert call(ws_bytes=need - 1) == b.LA_ERR_WORKSPACE
     assert call(ws_ptr=None) == b.LA_ERR_WORKSPACE
     assert call(ws_ptr=0x100010) == b.LA_ERR_INVALID_ARG and b"256" in lib.la_last_error()
-    assert call(flags=1) == b.LA_ERR_UNSUPPORTED and b"tensor cores" in lib.la_last_error()
-    f32 = [_t(D=128, dtype=0) for _ in range(7)]
-    st = lib.la_bwd_chunk_norm(*[ctypes.byref(x) for x in f32[:4]], 0x2000, None, 1, 64, 1,
-                               *[ctypes.byref(x) for x in f32[4:]], 0, 0x100000, need, None)
+    assert call(chunk=48) == b.LA_ERR_UNSUPPORTED and b"chunk" in lib.la_last_error()
+    assert call(flags=1, ws_bytes=ws(1, 4, 2, 128, 128, 64, 1, 1) - 1) == b.LA_ERR_WORKSPACE  # CUDA-core route
+    big = [_t(D=128), _t(D=128), _t(D=256), _t(D=256), _t(D=128), _t(D=128), _t(D=256)]
+    st = lib.la_bwd_chunk_norm(*[ctypes.byref(x) for x in big[:4]], 0x2000, None, 1, 64, 1,
+                               *[ctypes.byref(x) for x in big[4:]], 0, 0x100000, 1 << 30, None)
     assert st == b.LA_ERR_UNSUPPORTED
