@@ -548,6 +548,8 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   a.dk_ = view(dk);
   a.dv_ = view(dv);
   a.gamma = gamma;
+  a.g = g;
+  a.dg = g ? dg : nullptr;
   a.cu_seqlens = cu_seqlens;
   a.T = q->T;
   a.n_seqs = n_seqs;
@@ -651,14 +653,15 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
       return fail(LA_ERR_CUDA, "backward (log decay gradient): %s", cudaGetErrorString(err));
     return ok();
   }
-  if (g)
-    return fail(LA_ERR_UNSUPPORTED, "the per-token-decay backward runs on the tensor cores only: bf16, chunk 64, "
-                "d_k in {64, 128, 256} with d_v as la_fwd_chunk_path allows (d_k = d_v with elu + 1)");
   if (!bwd_supported(a, device))
     return fail(LA_ERR_UNSUPPORTED, "d_k %d x d_v %d does not fit the backward kernel's shared memory", a.dk,
                 a.dv);
+  if (g && (err = cudaMemsetAsync(dg, 0, (size_t)(q->B * q->T * q->H) * sizeof(float), st)) != cudaSuccess)
+    return fail(LA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
   err = launch_bwd(a, st);
   if (err != cudaSuccess) return fail(LA_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(err));
+  if (g && (err = launch_dg_rev_cumsum(dg, cu_seqlens, n_seqs, q->T, q->H, st)) != cudaSuccess)
+    return fail(LA_ERR_CUDA, "backward (log decay gradient): %s", cudaGetErrorString(err));
   return ok();
 }
 
@@ -854,6 +857,8 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     b.chunk = chunk;
     b.phi = phi;
     b.dtype = q->dtype;
+    b.g = nullptr;
+    b.dg = nullptr;
     if (!simt_supported(f, device) || !bwd_supported(b, device))
       return fail(LA_ERR_UNSUPPORTED, "d_k %lld x widened d_v %lld does not fit the CUDA-core kernels' shared "
                   "memory", (long long)Dk, (long long)Dvp);

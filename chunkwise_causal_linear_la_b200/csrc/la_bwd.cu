@@ -17,6 +17,18 @@
 // One CTA owns one (sequence, head): a forward sweep over its chunks writes dq,
 // a backward sweep writes dk and dv.  S^T, then R^T, lives in shared memory
 // ([d_k][d_v] fp32) next to the chunk's tiles; every product is fp32.
+//
+// Per-token decay (g set: alpha_t = exp(g_t), "1.6 长上下文与高效注意力", section
+// 状态空间模型与 Mamba): with b_i the chunk's prefix sums of g, gamma^(i-j) becomes
+// exp(b_i - b_j), gamma^(i+1) exp(b_i), and the state update's weights
+// exp(b_last - b_j) and exp(b_last).  The backward carry is kept as
+// Rt = alpha(next chunk's first token) R, so that
+//   dv_j, dkh_j inter terms:  exp(b_last - b_j) Rt kh_j,  exp(b_last - b_j) Rt^T v_j
+//   Rt <- exp(b_last) Rt + sum_i exp(b_i) dout_i qh_i^T
+// (with b_i = (i + 1) ln gamma this is the per-head recursion above).  The loss
+// sees b only through those weights, so dL/db_s = qh_s . dqh_s - kh_s . dkh_s;
+// the sweeps add these row terms into dg (zeroed by the caller, fp32 atomics
+// after a warp reduction) and a later kernel takes the reverse cumulative sum.
 #include <cuda_bf16.h>
 
 #include "la_common.cuh"
@@ -30,7 +42,7 @@ constexpr int kBwdThreads = 256;
 struct BwdLayout {
   int C;
   size_t smem;
-  int off_s, off_q, off_k, off_v, off_d, off_a, off_b, off_pw;  // float offsets
+  int off_s, off_q, off_k, off_v, off_d, off_a, off_b, off_pw, off_bt;  // float offsets
 };
 
 BwdLayout bwd_layout(int dk, int dv, int C) {
@@ -45,6 +57,7 @@ BwdLayout bwd_layout(int dk, int dv, int C) {
   L.off_a = o; o += C * (C + 1);
   L.off_b = o; o += C * (C + 1);
   L.off_pw = o; o += C + 1;
+  L.off_bt = o; o += C + 1;
   L.smem = (size_t)o * sizeof(float);
   return L;
 }
@@ -65,6 +78,7 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
   float *A = sm + L.off_a;     // [C][C+1]  gamma^(i-j) dout_i . v_j   (j <= i)
   float *Bm = sm + L.off_b;    // [C][C+1]  gamma^(i-j) qh_i . kh_j    (j <= i)
   float *pw = sm + L.off_pw;   // [C+1]     gamma^n
+  float *bt = sm + L.off_bt;   // [C]       per-token decay: prefix sums of g over the chunk
 
   const int tid = threadIdx.x;
   const int C = L.C, dk = a.dk, dv = a.dv;
@@ -81,7 +95,8 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
     start = 0;
     len = a.T;
   }
-  const float g = a.gamma[h];
+  const bool gated = a.g != nullptr;
+  const float g = gated ? 1.f : a.gamma[h];
   const Tin *Q = (const Tin *)a.q.data + b * a.q.sb + h * a.q.sh;
   const Tin *K = (const Tin *)a.k.data + b * a.k.sb + h * a.k.sh;
   const Tin *V = (const Tin *)a.v.data + b * a.v.sb + h * a.v.sh;
@@ -119,24 +134,51 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
       dd[i * (dv + 1) + r] = y;
     }
   };
+  // per-token decay: prefix sums b_i of the chunk's log decays (one thread; the
+  // caller synchronises before use)
+  auto load_decay = [&](int64_t c0, int Cp) {
+    if (gated && tid == 0) {
+      float acc = 0.f;
+      const float *gp = a.g + (b * a.T + start + c0) * a.H + h;
+      for (int i = 0; i < C; ++i) {
+        if (i < Cp) acc += gp[(int64_t)i * a.H];
+        bt[i] = acc;
+      }
+    }
+  };
+  // decay factors: D(i, j) = gamma^(i-j), E(i) = gamma^(i+1), W(j) = gamma^(Cp-1-j),
+  // F(Cp) = gamma^Cp (per-token: differences of the prefix sums)
+  auto Dij = [&](int i, int j) { return gated ? expf(bt[i] - bt[j]) : pw[i - j]; };
+  auto Ei = [&](int i) { return gated ? expf(bt[i]) : pw[i + 1]; };
+  auto Wj = [&](int j, int Cp) { return gated ? expf(bt[Cp - 1] - bt[j]) : pw[Cp - 1 - j]; };
+  auto Fc = [&](int Cp) { return gated ? expf(bt[Cp - 1]) : pw[Cp]; };
   // decayed score tiles of the chunk (lower triangle, diagonal included)
   auto scores = [&](int Cp, bool with_b) {
     for (int e = tid; e < C * C; e += kBwdThreads) {
       const int i = e / C, j = e % C;
       float sa = 0.f, sb = 0.f;
       if (j <= i && i < Cp) {
+        const float dij = Dij(i, j);
         const float *di = dd + i * (dv + 1), *vj = vv + j * (dv + 1);
         for (int r = 0; r < dv; ++r) sa = fmaf(di[r], vj[r], sa);
-        sa *= pw[i - j];
+        sa *= dij;
         if (with_b) {
           const float *qi = qh + i * (dk + 1), *kj = kh + j * (dk + 1);
           for (int c = 0; c < dk; ++c) sb = fmaf(qi[c], kj[c], sb);
-          sb *= pw[i - j];
+          sb *= dij;
         }
       }
       A[i * (C + 1) + j] = sa;
       if (with_b) Bm[i * (C + 1) + j] = sb;
     }
+  };
+  // dg row term x at row i of the chunk: reduced over the row's lanes (a row's d_k
+  // elements are consecutive e; d_k >= 16 divides 32 or is a multiple of it), then
+  // one atomic add per row.  Called by every thread with the same trip count.
+  const int lane = tid & 31, rw = dk < 32 ? dk : 32;
+  auto add_dg = [&](bool live, int64_t row, float x) {
+    for (int o = rw / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (live && lane % rw == 0) atomicAdd(a.dg + (b * a.T + row) * a.H + h, x);
   };
   __syncthreads();
 
@@ -144,25 +186,33 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
   for (int64_t c0 = 0; c0 < len; c0 += C) {
     const int Cp = (int)min((int64_t)C, len - c0);
     load_chunk(c0, Cp);
+    load_decay(c0, Cp);
     __syncthreads();
     scores(Cp, false);
     __syncthreads();
-    for (int e = tid; e < Cp * dk; e += kBwdThreads) {
-      const int i = e / dk, c = e % dk;
-      float intra = 0.f, inter = 0.f;
-      for (int j = 0; j <= i; ++j) intra = fmaf(A[i * (C + 1) + j], kh[j * (dk + 1) + c], intra);
-      const float *di = dd + i * (dv + 1), *sc = St + c * ds;
-      for (int r = 0; r < dv; ++r) inter = fmaf(sc[r], di[r], inter);
-      const float dqh = fmaf(pw[i + 1], inter, intra);
-      DQ[(start + c0 + i) * a.dq.st + c] = from_f32<Tin>(dqh * dphi_from_phi(qh[i * (dk + 1) + c], a.phi));
+    for (int e0 = 0; e0 < Cp * dk; e0 += kBwdThreads) {
+      const int e = e0 + tid;
+      const bool live = e < Cp * dk;
+      const int i = live ? e / dk : 0, c = e % dk;
+      float dqh = 0.f;
+      if (live) {
+        float intra = 0.f, inter = 0.f;
+        for (int j = 0; j <= i; ++j) intra = fmaf(A[i * (C + 1) + j], kh[j * (dk + 1) + c], intra);
+        const float *di = dd + i * (dv + 1), *sc = St + c * ds;
+        for (int r = 0; r < dv; ++r) inter = fmaf(sc[r], di[r], inter);
+        dqh = fmaf(Ei(i), inter, intra);
+        DQ[(start + c0 + i) * a.dq.st + c] = from_f32<Tin>(dqh * dphi_from_phi(qh[i * (dk + 1) + c], a.phi));
+      }
+      if (gated) add_dg(live, start + c0 + i, qh[i * (dk + 1) + c] * dqh);
     }
     __syncthreads();
     // S^T <- gamma^C' S^T + sum_j gamma^(C'-1-j) kh_j v_j^T
+    const float fc = Fc(Cp);
     for (int e = tid; e < dk * dv; e += kBwdThreads) {
       const int c = e / dv, r = e % dv;
       float acc = 0.f;
-      for (int j = 0; j < Cp; ++j) acc = fmaf(pw[Cp - 1 - j] * kh[j * (dk + 1) + c], vv[j * (dv + 1) + r], acc);
-      St[c * ds + r] = fmaf(pw[Cp], St[c * ds + r], acc);
+      for (int j = 0; j < Cp; ++j) acc = fmaf(Wj(j, Cp) * kh[j * (dk + 1) + c], vv[j * (dv + 1) + r], acc);
+      St[c * ds + r] = fmaf(fc, St[c * ds + r], acc);
     }
     __syncthreads();
   }
@@ -175,9 +225,12 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
     const int Cp = (int)min((int64_t)C, len - c0);
     __syncthreads();
     load_chunk(c0, Cp);
+    load_decay(c0, Cp);
     __syncthreads();
     scores(Cp, true);
     __syncthreads();
+    // inter-chunk weight of row j: gamma^(C'-j) on R (per-token: exp(b_last - b_j) on Rt)
+    auto Ij = [&](int j) { return gated ? expf(bt[Cp - 1] - bt[j]) : pw[Cp - j]; };
     // dv_j = sum_{i>=j} B_ij dout_i + gamma^(C'-j) R kh_j
     for (int e = tid; e < Cp * dv; e += kBwdThreads) {
       const int j = e / dv, r = e % dv;
@@ -185,25 +238,34 @@ bwd_simt_kernel(BwdArgs a, BwdLayout L) {
       for (int i = j; i < Cp; ++i) intra = fmaf(Bm[i * (C + 1) + j], dd[i * (dv + 1) + r], intra);
       const float *kj = kh + j * (dk + 1);
       for (int c = 0; c < dk; ++c) inter = fmaf(St[c * ds + r], kj[c], inter);
-      DV[(start + c0 + j) * a.dv_.st + r] = from_f32<Tin>(fmaf(pw[Cp - j], inter, intra));
+      DV[(start + c0 + j) * a.dv_.st + r] = from_f32<Tin>(fmaf(Ij(j), inter, intra));
     }
     // dkh_j = sum_{i>=j} A_ij qh_i + gamma^(C'-j) R^T v_j
-    for (int e = tid; e < Cp * dk; e += kBwdThreads) {
-      const int j = e / dk, c = e % dk;
-      float intra = 0.f, inter = 0.f;
-      for (int i = j; i < Cp; ++i) intra = fmaf(A[i * (C + 1) + j], qh[i * (dk + 1) + c], intra);
-      const float *vj = vv + j * (dv + 1), *sc = St + c * ds;
-      for (int r = 0; r < dv; ++r) inter = fmaf(sc[r], vj[r], inter);
-      const float dkh = fmaf(pw[Cp - j], inter, intra);
-      DK[(start + c0 + j) * a.dk_.st + c] = from_f32<Tin>(dkh * dphi_from_phi(kh[j * (dk + 1) + c], a.phi));
+    for (int e0 = 0; e0 < Cp * dk; e0 += kBwdThreads) {
+      const int e = e0 + tid;
+      const bool live = e < Cp * dk;
+      const int j = live ? e / dk : 0, c = e % dk;
+      float dkh = 0.f;
+      if (live) {
+        float intra = 0.f, inter = 0.f;
+        for (int i = j; i < Cp; ++i) intra = fmaf(A[i * (C + 1) + j], qh[i * (dk + 1) + c], intra);
+        const float *vj = vv + j * (dv + 1), *sc = St + c * ds;
+        for (int r = 0; r < dv; ++r) inter = fmaf(sc[r], vj[r], inter);
+        dkh = fmaf(Ij(j), inter, intra);
+        DK[(start + c0 + j) * a.dk_.st + c] = from_f32<Tin>(dkh * dphi_from_phi(kh[j * (dk + 1) + c], a.phi));
+      }
+      if (gated) add_dg(live, start + c0 + j, -kh[j * (dk + 1) + c] * dkh);
     }
     __syncthreads();
     // R^T <- gamma^C' R^T + sum_i gamma^i qh_i dout_i^T
+    // (per-token: Rt^T <- exp(b_last) Rt^T + sum_i exp(b_i) qh_i dout_i^T)
+    const float fc = Fc(Cp);
     for (int e = tid; e < dk * dv; e += kBwdThreads) {
       const int c = e / dv, r = e % dv;
       float acc = 0.f;
-      for (int i = 0; i < Cp; ++i) acc = fmaf(pw[i] * qh[i * (dk + 1) + c], dd[i * (dv + 1) + r], acc);
-      St[c * ds + r] = fmaf(pw[Cp], St[c * ds + r], acc);
+      for (int i = 0; i < Cp; ++i)
+        acc = fmaf((gated ? expf(bt[i]) : pw[i]) * qh[i * (dk + 1) + c], dd[i * (dv + 1) + r], acc);
+      St[c * ds + r] = fmaf(fc, St[c * ds + r], acc);
     }
   }
 }

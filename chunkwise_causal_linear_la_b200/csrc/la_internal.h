@@ -66,6 +66,11 @@ struct StepArgs {
 struct BwdArgs {
   TensorView q, k, v, dout, dq, dk_, dv_;
   const float *gamma;
+  // per-token decay (NULL: gamma): log decays [B * T][H]; dg receives the row terms
+  // of the log decays' gradient (zeroed by the caller; a reverse cumulative sum
+  // per sequence finishes it)
+  const float *g;
+  float *dg;
   const int32_t *cu_seqlens;  // NULL for dense batches
   int64_t T, n_seqs;
   int H, dk, dv, chunk, phi, dtype;

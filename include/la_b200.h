@@ -437,11 +437,13 @@ LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_t
  *   dg          device float[B, T, H]: the gradient with respect to g (fp32
  *               arithmetic: row dot products, then a reverse cumulative sum per
  *               sequence and head); 4-byte aligned.
- * Kernels: the tensor cores only: bf16, chunk 64, head dims for which
- * la_fwd_chunk_path reports LA_PATH_TENSOR_CORE (with elu + 1 also
- * d_k == d_v); the two reverse-time passes take, at each reversed position,
- * the decay of the token after it.  Other shapes, f32 and LA_FLAG_SIMT return
- * LA_ERR_UNSUPPORTED.  Other errors as for la_bwd_chunk.
+ * Kernels: bf16 with chunk 64 and head dims for which la_fwd_chunk_path
+ * reports LA_PATH_TENSOR_CORE (with elu + 1 also d_k == d_v) run on the
+ * tensor cores; the two reverse-time passes take, at each reversed position,
+ * the decay of the token after it.  f32, other chunks and shapes and
+ * LA_FLAG_SIMT run la_bwd_chunk's CUDA-core kernel with the per-token decay
+ * (fp32; LA_ERR_UNSUPPORTED where its shared memory does not fit).  Other
+ * errors as for la_bwd_chunk.
  */
 LA_API la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_tensor *v,
                                     const la_tensor *dout, const float *g, const int32_t *cu_seqlens,

@@ -138,10 +138,11 @@ def test_bwd_device_error_word_clear(la):
 # the log decays): bf16 on the tensor cores, three passes with the per-token decay
 # (the two reverse-time ones taking each position's following decay), then dg from
 # the row dot products and a reverse cumulative sum per sequence and head.
-def _check_gated(la, oracle_mod, q, k, v, dout, g, cu=None, phi="identity"):
+def _check_gated(la, oracle_mod, q, k, v, dout, g, cu=None, phi="identity", chunk=64, flags=0):
     dev = torch.device("cuda")
     dq, dk, dv, dg = la.la_bwd_chunk_gated(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), g.to(dev),
-                                           cu_seqlens=None if cu is None else cu.to(dev), phi=phi)
+                                           cu_seqlens=None if cu is None else cu.to(dev), phi=phi, chunk=chunk,
+                                           flags=flags)
     torch.cuda.synchronize()
     assert la.device_error(reset=True) == (0, 0)
     rq, rk, rv, rg = oracle_mod.backward_gated(q, k, v, dout, g.double().numpy(),
@@ -151,7 +152,7 @@ def _check_gated(la, oracle_mod, q, k, v, dout, g, cu=None, phi="identity"):
     errs = [slice_rel_err(to_np(x), r, sl) for x, r in ((dq, rq), (dk, rk), (dv, rv))]
     errs.append(_dg_err(to_np(dg), rg, q, k, rq, rk, phi, sl))
     assert all(np.isfinite(to_np(x)).all() for x in (dq, dk, dv, dg))
-    assert max(errs) < TOL[torch.bfloat16], errs
+    assert max(errs) < TOL[q.dtype], errs
     return errs
 
 
@@ -235,12 +236,46 @@ def test_bwd_gated_constant_decay_equals_per_head_backward(la):
         assert slice_rel_err(to_np(x), to_np(y), seq_slices(2, 300)) < TOL[torch.bfloat16]
 
 
-def test_bwd_gated_unsupported_shapes(la):
+@pytest.mark.parametrize("T", [1, 37, 200])
+@pytest.mark.parametrize("phi", ["identity", "elu1"])
+def test_bwd_gated_f32_cuda_cores(la, oracle_mod, T, phi):
+    """f32 runs the CUDA-core backward with the per-token decay (fp32 throughout)."""
+    q, k, v, dout = _inputs(2, T, 2, 64, 64, torch.float32, 79 + T)
+    g = _log_decay(2, T, 2, 0.5, 0.999, 80 + T)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, phi=phi)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 128])
+def test_bwd_gated_other_chunks(la, oracle_mod, chunk):
+    q, k, v, dout = _inputs(1, 2 * chunk + 9, 2, 64, 64, torch.bfloat16, 83 + chunk)
+    g = _log_decay(1, 2 * chunk + 9, 2, 0.8, 0.999, 84 + chunk)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, phi="elu1", chunk=chunk)
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (128, 64)])
+def test_bwd_gated_cuda_core_shapes(la, oracle_mod, dk, dv):
+    """Shapes off the tensor cores, LA_FLAG_SIMT, and a packed batch in f32."""
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    q, k, v, dout = _inputs(1, 130, 2, dk, dv, torch.bfloat16, dk + 3 * dv)
+    g = _log_decay(1, 130, 2, 0.9, 0.99, dk + dv)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, flags=la.LA_FLAG_SIMT)
+    cu = cu_seqlens_from_lengths([70, 0, 1, 33, 64])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 2, dk, dv, torch.float32, 2 * dk + dv)
+    g = _log_decay(1, int(cu[-1]), 2, 0.7, 0.999, dk * dv)
+    _check_gated(la, oracle_mod, q, k, v, dout, g, cu=cu, phi="elu1")
+
+
+def test_bwd_gated_simt_matches_tc(la):
+    """The CUDA-core and tensor-core backward of the same bf16 problem agree to bf16 rounding."""
     dev = torch.device("cuda")
-    q, k, v, dout = (x.to(dev) for x in _inputs(1, 50, 2, 128, 128, torch.float32, 39))
-    g = _log_decay(1, 50, 2, 0.9, 0.99, 40).to(dev)
-    with pytest.raises(la.LaError):
-        la.la_bwd_chunk_gated(q, k, v, dout, g)  # f32: the tensor cores only
+    q, k, v, dout = (x.to(dev) for x in _inputs(1, 300, 2, 128, 128, torch.bfloat16, 89))
+    g = _log_decay(1, 300, 2, 0.9, 0.999, 90).to(dev)
+    a = la.la_bwd_chunk_gated(q, k, v, dout, g, phi="elu1")
+    b = la.la_bwd_chunk_gated(q, k, v, dout, g, phi="elu1", flags=la.LA_FLAG_SIMT)
+    torch.cuda.synchronize()
+    for x, y in zip(a[:3], b[:3]):
+        assert (x.float() - y.float()).abs().max() <= 2e-2 * y.float().abs().max()
 
 
 # ---- backward of the normalised forward (la_bwd_chunk_norm) ----
