@@ -100,6 +100,10 @@ using namespace sm100;
 using namespace tcsync;
 
 constexpr int kThreads = 384;
+// The masked score tile P stays in tensor memory: the output warps overwrite the
+// first C/2 columns of the fp32 score tile with its bf16 pairs, and the P V product
+// reads its A operand from there (no shared-memory P tile).
+constexpr bool kPTmem = true;
 constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64: below, value-decay mode
 
 struct TcArgs {
@@ -523,8 +527,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-            umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
-                      ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+            const uint32_t acc = ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u;
+            if (kPTmem)
+              umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3, acc);
+            else
+              umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3, acc);
           }
           umma_commit(bars + G::B_OFULL + ob);
           if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
@@ -596,8 +603,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-              umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3,
-                        ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
+              const uint32_t acc = ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u;
+              if (kPTmem)
+                umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3, acc);
+              else
+                umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3, acc);
             }
             umma_commit(bars + G::B_OFULL + ob);
             ++c3;
@@ -991,14 +1001,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           f[e] = (j <= i && row_ok) ? __uint_as_float(r[e]) * pw[i - j] : 0.f;
         }
       }
-      uint8_t *prow = p_tile(b) + i * 128;
+      if (kPTmem) {  // P row i, columns [32 hf, 32 hf + 32) as bf16 pairs in score columns [16 hf, 16 hf + 16)
+        uint32_t pk[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
-                                   pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
-        *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
+        for (int e = 0; e < 16; ++e) pk[e] = pack2(f[2 * e], f[2 * e + 1]);
+        tmem_st_16x32bx2_x16<16>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, pk);
+        tmem_wait_st();
+      } else {
+        uint8_t *prow = p_tile(b) + i * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
+                                     pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
+          *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bars + G::B_PFULL + b);  // also tells the MMA issuer that A[b] has been read
       ok = true;
