@@ -34,13 +34,14 @@
 //   warps 2-3   transform: phi(q) and the decayed keys, in place.
 //   warps 4-7   state: S <- gamma^C' S + U (U from tensor memory), the bf16
 //               operand Sb for the next chunk, and the final state.
-//   warps 8-11  output: score tile -> P (one chunk ahead), then the epilogue
-//               (row factor, cast, store) of the previous chunk.
+//   warps 8-11  output: score tile -> P (one chunk ahead, in tensor memory),
+//               then the epilogue (row factor, cast, store) of the previous chunk.
 // Per chunk, four MMAs:
 //   M1  A = qh kd^T          (M=C, N=C,   K=d_k)     -> A[c%2]
 //   M4  U = kd^T V           (M=128 per d_k block, N=DVT, K=C)  [value decay: kh^T vd]
 //   M2  O = qh Sb^T          (M=C, N=DVT, K=d_k)     [skipped on chunk 0]
-//   M3  O += P V             (M=C, N=DVT, K=C)       -> O[c%2]
+//   M3  O += P V             (M=C, N=DVT, K=C)       -> O[c%2]; P (bf16) is read from
+//                            tensor memory, where the output warps wrote it over A[c%2]
 //
 // Every wait is bounded: on a timeout the CTA raises an abort flag, records
 // the failure in a device error word, drains and frees its tensor memory.
@@ -100,10 +101,6 @@ using namespace sm100;
 using namespace tcsync;
 
 constexpr int kThreads = 384;
-// The masked score tile P stays in tensor memory: the output warps overwrite the
-// first C/2 columns of the fp32 score tile with its bf16 pairs, and the P V product
-// reads its A operand from there (no shared-memory P tile).
-constexpr bool kPTmem = true;
 constexpr float kSmallGammaLimit = 5.421010862427522e-20f;  // 2^-64: below, value-decay mode
 
 struct TcArgs {
@@ -155,14 +152,12 @@ struct Cfg {
   static constexpr int QK_BYTES = KB * SLAB;
   static constexpr int V_BYTES = VB * SLAB;
   static constexpr int STAGE_BYTES = 2 * QK_BYTES + V_BYTES;
-  static constexpr int P_BYTES = (C / 64) * SLAB;  // [C rows x C cols] bf16, K-major
   static constexpr int SB_SLAB = DK * 128;         // [DK rows x 64 cols] bf16
   static constexpr int SB_BYTES = VB * SB_SLAB;
 
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_VD = NS * STAGE_BYTES;  // decayed values (value-decay mode)
-  static constexpr int OFF_P = OFF_VD + V_BYTES;
-  static constexpr int OFF_SB = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_SB = OFF_VD + V_BYTES;
   static constexpr int OFF_Z = OFF_SB + SB_BYTES;  // normaliser key sums z, two buffers of DK floats
   static constexpr int OFF_KSUM = OFF_Z + 2 * DK * 4;  // per stage, per transform warp: chunk key column sums
   // data-dependent decay, per stage: b_i = sum_{t<=i} log alpha_t over the chunk, i < C, and b_last at [C]
@@ -389,7 +384,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto v_tile = [&](int s) { return sm + G::OFF_STAGE + s * G::STAGE_BYTES + 2 * G::QK_BYTES; };
   uint8_t *vd_tile = sm + G::OFF_VD;
   uint8_t *sb_tile = sm + G::OFF_SB;
-  auto p_tile = [&](int b) { return sm + G::OFF_P + b * G::P_BYTES; };
 
   if (warp < 4) {
     reg_dealloc<104>();
@@ -426,7 +420,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t dkm0 = smem_desc_sw128(smem_u32(k_tile(0)), G::SLAB, 1024);    // MN-major (state update)
       const uint64_t dv0 = smem_desc_sw128(smem_u32(v_tile(0)), G::SLAB, 1024);
       const uint64_t dvd = smem_desc_sw128(smem_u32(vd_tile), G::SLAB, 1024);
-      const uint64_t dp0 = smem_desc_sw128(smem_u32(p_tile(0)), 16, 1024);
       auto stage_off = [](int s) -> uint64_t { return (uint64_t)(s * (G::STAGE_BYTES >> 4)); };
       int m1_issued = 0;
       // M1 of chunk c: scores A[c%2] = qh kd^T
@@ -523,16 +516,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           if (!wait_bar(sy, G::B_PFULL + b, (c >> 1) & 1, c)) break;
           tc_fence_after();
-          const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-            const uint32_t acc = ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u;
-            if (kPTmem)
-              umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3, acc);
-            else
-              umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3, acc);
-          }
+          for (int kk = 0; kk < C / 16; ++kk)  // A = P from tensor memory, K = 16 per product (8 columns)
+            umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3,
+                         ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
           umma_commit(bars + G::B_OFULL + ob);
           if ((NORM || GATED) && !wait_bar(sy, G::B_ZFULL + (c & 1), (c >> 1) & 1, c)) break;  // state warps done
           umma_commit(bars + G::B_EMPTY + s);
@@ -599,16 +586,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t o_inter = tbase + G::T_O + ob * (vd_mode ? 2 : 1) * DVT;
             const uint32_t o_intra = vd_mode ? o_inter + DVT : o_inter;
             const uint64_t dv = dv0 + stage_off(s);
-            const uint64_t dp = dp0 + (uint64_t)(b * (G::P_BYTES >> 4));
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * G::SLAB + (kk & 3) * 32) >> 4;
-              const uint32_t acc = ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u;
-              if (kPTmem)
-                umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3, acc);
-              else
-                umma_bf16(o_intra, dp + off, dv + ((kk * 2048) >> 4), ID_M3, acc);
-            }
+            for (int kk = 0; kk < C / 16; ++kk)  // A = P from tensor memory
+              umma_bf16_ts(o_intra, tbase + G::T_A + b * C + kk * 8, dv + ((kk * 2048) >> 4), ID_M3,
+                           ((!vd_mode && (c > 0 || has_init)) || kk > 0) ? 1u : 0u);
             umma_commit(bars + G::B_OFULL + ob);
             ++c3;
             progress = true;
@@ -1001,21 +982,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           f[e] = (j <= i && row_ok) ? __uint_as_float(r[e]) * pw[i - j] : 0.f;
         }
       }
-      if (kPTmem) {  // P row i, columns [32 hf, 32 hf + 32) as bf16 pairs in score columns [16 hf, 16 hf + 16)
+      {  // P in tensor memory, in place: row i's columns [32 hf, 32 hf + 32) as bf16 pairs in score
+         // columns [16 hf, 16 hf + 16) (the M = 64 layout: row 16 w + l at lane 32 w + l); this
+         // warp has read its lanes of the fp32 tile already
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack2(f[2 * e], f[2 * e + 1]);
         tmem_st_16x32bx2_x16<16>(tbase + ((uint32_t)(sp * 32) << 16) + G::T_A + b * C, pk);
         tmem_wait_st();
-      } else {
-        uint8_t *prow = p_tile(b) + i * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = make_uint4(pack2(f[8 * q], f[8 * q + 1]), pack2(f[8 * q + 2], f[8 * q + 3]),
-                                     pack2(f[8 * q + 4], f[8 * q + 5]), pack2(f[8 * q + 6], f[8 * q + 7]));
-          *reinterpret_cast<uint4 *>(prow + (((hf * 4 + q) ^ (i & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
       }
       tc_fence_before();
       mbar_arrive(bars + G::B_PFULL + b);  // also tells the MMA issuer that A[b] has been read
