@@ -11,6 +11,10 @@ this package is its Python binding:
     out, final_state, z = la_fwd_chunk_z(q, k, v, gamma, phi="elu1")
     o = la_step_norm(q1, k1, v1, gamma, final_state, z, phi="elu1")
 
+    # training: the forward and its backward as one differentiable call
+    from chunkwise_causal_linear_la_b200.autograd import chunk_linear_attention
+    o = chunk_linear_attention(q, k, v, gamma, phi="elu1", normalize=True)
+
 ``workloads`` draws the seeded synthetic inputs of the standard workloads.
 """
 from .binding import (  # noqa: F401

@@ -73,6 +73,12 @@ int sm_count(int device) {
   return v;
 }
 
+cudaError_t bind_device(int *device) {
+  cudaError_t e = cudaGetDevice(device);
+  if (e == cudaSuccess) e = cudaSetDevice(*device);
+  return e;
+}
+
 int max_smem_optin(int device) {
   if (device < 0 || device >= kMaxDevices) return 232448;
   int v = g_smem_optin[device].load(std::memory_order_relaxed);
@@ -182,8 +188,8 @@ la_status fwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v,
 
   cudaStream_t st = (cudaStream_t)stream;
   int device = 0;
-  cudaError_t err = cudaGetDevice(&device);
-  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  cudaError_t err = bind_device(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice / cudaSetDevice: %s", cudaGetErrorString(err));
 
   // No token to process: only the final states (all zero) remain to be written.
   if (a.n_seqs == 0) return ok();
@@ -465,6 +471,9 @@ la_status la_fwd_gated_delta_chunk(const la_tensor *q, const la_tensor *k, const
       return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (la_fwd_gated_delta_workspace_size)",
                   workspace_bytes, need);
     if (((uintptr_t)workspace) % 256) return fail(LA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    int device = 0;
+    if ((err = bind_device(&device)) != cudaSuccess)
+      return fail(LA_ERR_CUDA, "cudaGetDevice / cudaSetDevice: %s", cudaGetErrorString(err));
     const char *why = nullptr;
     err = launch_gdn_chunk(a, workspace, workspace_bytes, (cudaStream_t)stream, &why);
     if (err != cudaSuccess)
@@ -560,8 +569,8 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   a.phi = phi;
   a.dtype = q->dtype;
   int device = 0;
-  cudaError_t err = cudaGetDevice(&device);
-  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  cudaError_t err = bind_device(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice / cudaSetDevice: %s", cudaGetErrorString(err));
   if (a.n_seqs == 0 || a.T == 0 || q->B == 0) return ok();
   cudaStream_t st = (cudaStream_t)stream;
 
@@ -776,8 +785,8 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
   if (((uintptr_t)workspace) % 256 != 0) return fail(LA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
   int device = 0;
-  cudaError_t err = cudaGetDevice(&device);
-  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  cudaError_t err = bind_device(&device);
+  if (err != cudaSuccess) return fail(LA_ERR_CUDA, "cudaGetDevice / cudaSetDevice: %s", cudaGetErrorString(err));
   if (n_seqs == 0 || q->T == 0 || q->B == 0) return ok();
 
   const int64_t B = q->B, T = q->T, H = q->H, Dk = q->D, Dv = v->D, Dvp = norm_aug_width(Dv);

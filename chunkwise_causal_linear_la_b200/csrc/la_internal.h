@@ -92,6 +92,12 @@ struct DeltaArgs {
 // Sets the calling thread's la_last_error() message and returns `status`.
 la_status report_error(la_status status, const char *msg);
 
+// The current device, with its primary context made current on the calling thread
+// (cudaSetDevice): the driver's tensor-map encoder works in the thread's current
+// context, which a thread that has made no call binding one yet (torch's autograd
+// worker thread, say) lacks.  Every entry point that launches a TMA kernel calls it.
+cudaError_t bind_device(int *device);
+
 // Per-device properties, cached on first use.
 int sm_count(int device);
 int max_smem_optin(int device);
