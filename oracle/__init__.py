@@ -24,6 +24,8 @@ it follows, is stated in the C file's header:
   decays' gradient); keeps every state, so for test sizes.
 * ``backward_norm`` -- dq, dk, dv of sum_t dout_t . o_t through the normalised
   recurrence (o_t divided by z_t . phi(q_t)), token by token.
+* ``backward_gated_norm`` -- dq, dk, dv and dg through the normalised recurrence
+  with the per-token decay; keeps every state, so for test sizes.
 * ``gated_delta`` -- the gated delta rule (section Gated delta rule of the same
   page), token by token, unit-norm keys.
 * ``norm_gate``  -- y = RMSNorm(o) * w * swish(g) per (token, head) over d_v.
@@ -92,6 +94,9 @@ def _load():
         lib.oracle_backward_gated.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32,
                                               dp, dp, dp, dp, i32]
         lib.oracle_backward_gated.restype = i32
+        lib.oracle_backward_gated_norm.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, vp, i64, i32,
+                                                   dp, dp, dp, dp, i32]
+        lib.oracle_backward_gated_norm.restype = i32
         lib.oracle_norm_gate.argtypes = [dp, vp, i32, i64, i64, dp, ctypes.c_double, dp, i32]
         lib.oracle_norm_gate.restype = i32
         lib.oracle_gated_delta.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, dp, dp, vp, i64, dp, dp, dp, i32]
@@ -376,6 +381,31 @@ def backward_gated(q, k, v, dout, g, cu_seqlens=None, phi="identity", nthreads=0
                                        n, _PHI[phi], _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gd), int(nthreads))
     if rc != 0:
         raise _oracle_error("oracle_backward_gated", rc)
+    return gq, gk, gv, gd
+
+
+def backward_gated_norm(q, k, v, dout, g, cu_seqlens=None, phi="elu1", nthreads=0):
+    """Gradients of L = sum(dout * o) for the normalised recurrence with the per-token
+    decay exp(g[b, t, h]) (o_t = S_t qh_t / z_t . qh_t).
+
+    Returns (dq, dk, dv, dg) in float64; dg [B, T, H] is the gradient of the log decays."""
+    q, k, v, dt, B, T, H, dk, dv, _, cu, n = _prep(q, k, v, np.ones(q.shape[2] if hasattr(q, "shape") else 1),
+                                                    cu_seqlens)
+    do, ddt = _as_input(dout)
+    if ddt != dt or do.shape != v.shape:
+        raise ValueError("dout must be [B, T, H, d_v] of the inputs' dtype")
+    gg = np.ascontiguousarray(np.asarray(g, dtype=np.float64))
+    if gg.shape != (B, T, H):
+        raise ValueError("g must be [B, T, H]")
+    gq = np.zeros(q.shape, np.float64)
+    gk = np.zeros(k.shape, np.float64)
+    gv = np.zeros(v.shape, np.float64)
+    gd = np.zeros((B, T, H), np.float64)
+    rc = _load().oracle_backward_gated_norm(_ptr(q), _ptr(k), _ptr(v), _ptr(do), dt, B, T, H, dk, dv, _ptr(gg),
+                                            _ptr(cu), n, _PHI[phi], _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gd),
+                                            int(nthreads))
+    if rc != 0:
+        raise _oracle_error("oracle_backward_gated_norm", rc)
     return gq, gk, gv, gd
 
 

@@ -34,6 +34,8 @@
  *                        recurrence: the adjoint of the definition.
  *   oracle_backward_gated -- the same for the per-token decay, plus the
  *                        gradient of the log decays g.
+ *   oracle_backward_gated_norm -- the normalised per-token-decay forward's
+ *                        adjoint (dq, dk, dv, dg).
  *   oracle_norm_gate  -- RMSNorm over d_v times a Swish gate, per (token, head).
  *   oracle_gated_delta -- the gated delta rule, token by token.
  *   oracle_gated_delta_chunked -- the same rule regrouped into chunks (the
@@ -823,6 +825,126 @@ int oracle_backward_gated(const void *q, const void *k, const void *v, const voi
     free(D);
     free(qh);
     free(kh);
+  }
+  return oom ? ORC_ERR_NOMEM : 0;
+}
+
+/*
+ * Adjoint of the normalised recurrence with the per-token decay alpha_t =
+ * exp(g_t) ("1.6 长上下文与高效注意力", section 状态空间模型与 Mamba, with the
+ * normaliser of section 线性注意力):
+ *   S_t = alpha_t S_{t-1} + v_t kh_t^T,  z_t = alpha_t z_{t-1} + kh_t,
+ *   num_t = S_t qh_t,  den_t = z_t . qh_t,  o_t = num_t / den_t.
+ * With L = sum_t dout_t . o_t, u_t = dout_t / den_t reaches num_t and
+ * e_t = -(dout_t . o_t) / den_t reaches den_t, so
+ *   dqh_t = S_t^T u_t + e_t z_t,
+ *   G_t = u_t qh_t^T + alpha_{t+1} G_{t+1},   gz_t = e_t qh_t + alpha_{t+1} gz_{t+1},
+ *   dkh_t = G_t^T v_t + gz_t,   dv_t = G_t kh_t,
+ *   dg_t = alpha_t (<G_t, S_{t-1}> + gz_t . z_{t-1})   (the loss sees g_t only
+ *          through alpha_t's two products).
+ * The forward sweep keeps every S_{t-1}, z_{t-1}, u_t and e_t of the task.
+ */
+int oracle_backward_gated_norm(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                               int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                               const double *g, const int32_t *cu_seqlens, int64_t n_seqs, int phi,
+                               double *dq, double *dkk, double *dvv, double *dg, int nthreads) {
+  int rc = orc_check(dtype, B, T, H, dk, dv, cu_seqlens, n_seqs, phi);
+  if (rc) return rc;
+  if (!g || !dg) return -10;
+  if (nthreads <= 0) nthreads = oracle_max_threads();
+
+  int oom = 0; /* set when a task could not allocate its buffers */
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int64_t task = 0; task < n_seqs * H; ++task) {
+    const int64_t n = task / H, h = task % H;
+    int64_t start, len;
+    orc_seq(cu_seqlens, T, n, &start, &len);
+    const size_t sz = (size_t)(dv * dk), L1 = (size_t)(len > 0 ? len : 1);
+    double *prevS = (double *)calloc(L1 * sz, sizeof(double));        /* S_{t-1} */
+    double *prevz = (double *)calloc(L1 * (size_t)dk, sizeof(double)); /* z_{t-1} */
+    double *U = (double *)calloc(L1 * (size_t)dv, sizeof(double));     /* u_t */
+    double *E = (double *)calloc(L1, sizeof(double));                  /* e_t */
+    double *S = (double *)calloc(sz, sizeof(double));
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *G = (double *)calloc(sz, sizeof(double));
+    double *gz = (double *)calloc((size_t)dk, sizeof(double));
+    double *qh = (double *)malloc((size_t)dk * sizeof(double));
+    double *kh = (double *)malloc((size_t)dk * sizeof(double));
+    double *num = (double *)malloc((size_t)dv * sizeof(double));
+    if (!prevS || !prevz || !U || !E || !S || !z || !G || !gz || !qh || !kh || !num) {
+      free(prevS); free(prevz); free(U); free(E); free(S); free(z); free(G); free(gz); free(qh); free(kh);
+      free(num);
+#pragma omp atomic write
+      oom = 1;
+      continue;
+    }
+    /* forward in time: the state, the normaliser, u_t, e_t and dq */
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t row = start + t;
+      const double a = exp(g[row * H + h]);
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      memcpy(prevS + (size_t)t * sz, S, sz * sizeof(double));
+      memcpy(prevz + (size_t)t * dk, z, (size_t)dk * sizeof(double));
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+        z[c] = a * z[c] + kh[c];
+      }
+      double den = 0.0;
+      for (int64_t c = 0; c < dk; ++c) den += z[c] * qh[c];
+      double dot = 0.0;  /* dout . o */
+      for (int64_t r = 0; r < dv; ++r) {
+        const double vr = orc_load(v, dtype, vb + r);
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) {
+          S[r * dk + c] = a * S[r * dk + c] + vr * kh[c];
+          acc += S[r * dk + c] * qh[c];
+        }
+        num[r] = acc;
+        dot += orc_load(dout, dtype, vb + r) * (acc / den);
+      }
+      double *u = U + (size_t)t * dv;
+      for (int64_t r = 0; r < dv; ++r) u[r] = orc_load(dout, dtype, vb + r) / den;
+      E[t] = -(dot / den);
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = z[c] * E[t];
+        for (int64_t r = 0; r < dv; ++r) acc += S[r * dk + c] * u[r];
+        dq[qk + c] = acc * orc_dphi(orc_load(q, dtype, qk + c), phi);
+      }
+    }
+    /* backward in time: G, gz, dk, dv and dg */
+    double a_next = 0.0;  /* alpha_{t+1}; G and gz are zero before the last token anyway */
+    for (int64_t t = len - 1; t >= 0; --t) {
+      const int64_t row = start + t;
+      const double a = exp(g[row * H + h]);
+      const int64_t qk = (row * H + h) * dk, vb = (row * H + h) * dv;
+      const double *u = U + (size_t)t * dv;
+      for (int64_t c = 0; c < dk; ++c) {
+        qh[c] = orc_phi(orc_load(q, dtype, qk + c), phi);
+        kh[c] = orc_phi(orc_load(k, dtype, qk + c), phi);
+        gz[c] = a_next * gz[c] + E[t] * qh[c];
+      }
+      for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) G[r * dk + c] = a_next * G[r * dk + c] + u[r] * qh[c];
+      for (int64_t c = 0; c < dk; ++c) {
+        double acc = gz[c];
+        for (int64_t r = 0; r < dv; ++r) acc += G[r * dk + c] * orc_load(v, dtype, vb + r);
+        dkk[qk + c] = acc * orc_dphi(orc_load(k, dtype, qk + c), phi);
+      }
+      for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += G[r * dk + c] * kh[c];
+        dvv[vb + r] = acc;
+      }
+      const double *P = prevS + (size_t)t * sz, *Z = prevz + (size_t)t * dk;
+      double inner = 0.0;
+      for (size_t e = 0; e < sz; ++e) inner += G[e] * P[e];
+      for (int64_t c = 0; c < dk; ++c) inner += gz[c] * Z[c];
+      dg[row * H + h] = inner * a;
+      a_next = a;
+    }
+    free(prevS); free(prevz); free(U); free(E); free(S); free(z); free(G); free(gz); free(qh); free(kh);
+    free(num);
   }
   return oom ? ORC_ERR_NOMEM : 0;
 }

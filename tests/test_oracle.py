@@ -780,3 +780,88 @@ def test_backward_norm_splits_into_numerator_and_denominator_adjoints(oracle_mod
         for x, y, r in zip(a[:2], b[:2], ref[:2]):
             np.testing.assert_allclose(x + y, r, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(a[2], ref[2], rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- normalised backward, per-token decay
+def test_backward_gated_norm_matches_finite_differences(oracle_mod):
+    """Central differences of L = sum(dout * o) through the normalised per-token-decay
+    forward oracle, for q, k, v and the log decays g."""
+    B, T, H, dk, dv = 1, 6, 2, 3, 2
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=101)
+    dout = np.random.default_rng(102).standard_normal((B, T, H, dv))
+    g = _rand_log_decay(B, T, H, 103)
+    gq, gk, gv, gg = oracle_mod.backward_gated_norm(q, k, v, dout, g, phi="elu1")
+
+    def loss(q_, k_, v_, g_):
+        o, _, _ = oracle_mod.recurrent_gated(q_, k_, v_, g_, phi="elu1", normalize=True)
+        return float(np.sum(o * dout))
+
+    eps = 1e-6
+    for x, gref, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2), (g, gg, 3)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v, g]
+            args_m = [q, k, v, g]
+            args_p[which], args_m[which] = xp, xm
+            fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert rel(gref, fd) < 1e-7, which
+
+
+def test_backward_gated_norm_matches_autograd_of_masked_form(oracle_mod):
+    """torch autograd (float64) through O = ((phi(Q) phi(K)^T .* M) V) / rowsum(phi(Q) phi(K)^T .* M)
+    with the cumulative-decay mask M_ij = exp(b_i - b_j) (i >= j), b = cumsum(g)."""
+    T, H, dk, dv = 25, 2, 4, 3
+    q, k, v = rand_qkv(1, T, H, dk, dv, seed=104)
+    dout = np.random.default_rng(105).standard_normal((1, T, H, dv))
+    g = _rand_log_decay(1, T, H, 106)
+    cases = [("elu1", q, k), ("identity", np.abs(q) + 0.1, np.abs(k) + 0.1)]
+    for phi, qq, kk in cases:
+        gq, gk, gv, gg = oracle_mod.backward_gated_norm(qq, kk, v, dout, g, phi=phi)
+        for h in range(H):
+            qt, kt, vt, lg = (torch.tensor(x[0, :, h], dtype=torch.float64, requires_grad=True)
+                              for x in (qq, kk, v, g))
+            f = (lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))) if phi == "elu1" \
+                else (lambda x: x)
+            b = torch.cumsum(lg, 0)
+            i = torch.arange(T)[:, None]
+            j = torch.arange(T)[None, :]
+            M = torch.where(i >= j, torch.exp(b[:, None] - b[None, :]), torch.zeros((), dtype=torch.float64))
+            P = (f(qt) @ f(kt).T) * M
+            O = (P @ vt) / P.sum(dim=1, keepdim=True)
+            (O * torch.tensor(dout[0, :, h])).sum().backward()
+            assert rel(gq[0, :, h], qt.grad.numpy()) < 1e-11
+            assert rel(gk[0, :, h], kt.grad.numpy()) < 1e-11
+            assert rel(gv[0, :, h], vt.grad.numpy()) < 1e-11
+            assert rel(gg[0, :, h], lg.grad.numpy()) < 1e-10
+
+
+def test_backward_gated_norm_reduces_to_per_head_decay(oracle_mod):
+    """g constant over time per head: dq, dk, dv equal the normalised per-head-decay
+    backward with gamma = exp(g)."""
+    B, T, H, dk, dv = 2, 30, 3, 4, 3
+    q, k, v = rand_qkv(B, T, H, dk, dv, seed=107)
+    dout = np.random.default_rng(108).standard_normal((B, T, H, dv))
+    lg = np.log(np.array([0.6, 0.95, 1.0]))
+    g = np.broadcast_to(lg, (B, T, H)).copy()
+    gq, gk, gv, _ = oracle_mod.backward_gated_norm(q, k, v, dout, g, phi="elu1")
+    rq, rk, rv = oracle_mod.backward_norm(q, k, v, dout, np.exp(lg), phi="elu1")
+    assert rel(gq, rq) < 1e-12 and rel(gk, rk) < 1e-12 and rel(gv, rv) < 1e-12
+
+
+def test_backward_gated_norm_varlen_equals_independent_runs(oracle_mod):
+    lengths = [6, 0, 13, 1]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Tt, H, dk, dv = int(cu[-1]), 2, 4, 3
+    q, k, v = rand_qkv(1, Tt, H, dk, dv, seed=109)
+    dout = np.random.default_rng(110).standard_normal((1, Tt, H, dv))
+    g = _rand_log_decay(1, Tt, H, 111)
+    full = oracle_mod.backward_gated_norm(q, k, v, dout, g, cu_seqlens=cu, phi="elu1")
+    for n in range(len(lengths)):
+        s_, e = cu[n], cu[n + 1]
+        part = oracle_mod.backward_gated_norm(q[:, s_:e], k[:, s_:e], v[:, s_:e], dout[:, s_:e], g[:, s_:e],
+                                              phi="elu1")
+        for a, b in zip(full, part):
+            assert np.array_equal(a[:, s_:e], b)

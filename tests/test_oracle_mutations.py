@@ -213,3 +213,65 @@ def test_norm_backward_mutant_is_caught(tmp_path, name):
     old, new = NORM_BWD_MUTATIONS[name]
     lib = _build(tmp_path, name, old, new)
     assert not _norm_bwd_pin_passes(lib), name
+
+
+GATED_NORM_BWD_MUTATIONS = {
+    "dg without the normaliser's term gz . z_{t-1}": (
+        "      for (int64_t c = 0; c < dk; ++c) inner += gz[c] * Z[c];\n", ""),
+    "z adjoint gz not decayed": (
+        "gz[c] = a_next * gz[c] + E[t] * qh[c];", "gz[c] = gz[c] + E[t] * qh[c];"),
+    "denominator's adjoint with the wrong sign (per-token decay)": (
+        "E[t] = -(dot / den);", "E[t] = dot / den;"),
+    "dg paired with z after the token": (
+        "*Z = prevz + (size_t)t * dk;", "*Z = t + 1 < len ? prevz + (size_t)(t + 1) * dk : z;"),
+}
+
+
+def _gated_norm_bwd(lib, q, k, v, dout, g):
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.oracle_backward_gated_norm.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, vp, vp, i64, i32,
+                                               vp, vp, vp, vp, i32]
+    lib.oracle_backward_gated_norm.restype = i32
+    q, k, v, dout, g = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout, g))
+    outs = [np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape), np.zeros(g.shape)]
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = lib.oracle_backward_gated_norm(p(q), p(k), p(v), p(dout), 2, B, T, H, dk, dv, p(g), None, B, 1,
+                                        *(p(o) for o in outs), 1)
+    assert rc == 0
+    return outs
+
+
+def _gated_norm_bwd_pin_passes(lib):
+    """The autograd pin of test_oracle.py: torch float64 gradients (dq, dk, dv, dg)
+    through the normalised masked form with the cumulative-decay mask and elu + 1."""
+    import torch
+
+    T, dk, dv = 12, 3, 2
+    q, k, v = rand_qkv(1, T, 1, dk, dv, seed=112)
+    dout = np.random.default_rng(113).standard_normal((1, T, 1, dv))
+    g = np.log(np.random.default_rng(114).uniform(0.3, 1.0, (1, T, 1)))
+    got = _gated_norm_bwd(lib, q, k, v, dout, g)
+    qt, kt, vt, lg = (torch.tensor(x[0, :, 0], dtype=torch.float64, requires_grad=True) for x in (q, k, v, g))
+    f = lambda x: torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))  # noqa: E731
+    b = torch.cumsum(lg, 0)
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    M = torch.where(i >= j, torch.exp(b[:, None] - b[None, :]), torch.zeros((), dtype=torch.float64))
+    P = (f(qt) @ f(kt).T) * M
+    ((P @ vt) / P.sum(dim=1, keepdim=True) * torch.tensor(dout[0, :, 0])).sum().backward()
+    want = [qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy(), lg.grad.numpy()]
+    return all(rel(a[0, :, 0], w) < 1e-10 for a, w in zip(got, want))
+
+
+def test_unmutated_copy_passes_gated_norm_backward_pin(tmp_path):
+    lib = _build(tmp_path, "none", "#define ROWS_PER_TASK 8", "#define ROWS_PER_TASK 8")
+    assert _gated_norm_bwd_pin_passes(lib)
+
+
+@pytest.mark.parametrize("name", sorted(GATED_NORM_BWD_MUTATIONS))
+def test_gated_norm_backward_mutant_is_caught(tmp_path, name):
+    old, new = GATED_NORM_BWD_MUTATIONS[name]
+    lib = _build(tmp_path, name, old, new)
+    assert not _gated_norm_bwd_pin_passes(lib), name
