@@ -31,6 +31,7 @@ from .binding import (  # noqa: F401
     la_bwd_chunk,
     la_bwd_chunk_gated,
     la_bwd_chunk_norm,
+    la_bwd_chunk_gated_norm,
     bwd_norm_workspace_size,
     la_fwd_chunk,
     la_fwd_chunk_gated,

@@ -38,19 +38,19 @@ class _ChunkLinearAttention(torch.autograd.Function):
 
 class _ChunkGatedLinearAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, g, cu_seqlens, chunk, phi):
+    def forward(ctx, q, k, v, g, cu_seqlens, chunk, phi, normalize):
         out, _, _ = binding.la_fwd_chunk_gated(q, k, v, g, cu_seqlens=cu_seqlens, chunk=chunk, phi=phi,
-                                               normalize=False)
+                                               normalize=normalize)
         ctx.save_for_backward(q, k, v, g, cu_seqlens)
-        ctx.chunk, ctx.phi = chunk, phi
+        ctx.chunk, ctx.phi, ctx.normalize = chunk, phi, normalize
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, g, cu = ctx.saved_tensors
-        dq, dk, dv, dg = binding.la_bwd_chunk_gated(q, k, v, dout.contiguous(), g, cu_seqlens=cu, chunk=ctx.chunk,
-                                                    phi=ctx.phi)
-        return dq, dk, dv, dg, None, None, None
+        bwd = binding.la_bwd_chunk_gated_norm if ctx.normalize else binding.la_bwd_chunk_gated
+        dq, dk, dv, dg = bwd(q, k, v, dout.contiguous(), g, cu_seqlens=cu, chunk=ctx.chunk, phi=ctx.phi)
+        return dq, dk, dv, dg, None, None, None, None
 
 
 def chunk_linear_attention(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="identity", normalize=False):
@@ -59,7 +59,7 @@ def chunk_linear_attention(q, k, v, gamma, cu_seqlens=None, chunk=64, phi="ident
     return _ChunkLinearAttention.apply(q, k, v, gamma, cu_seqlens, chunk, phi, normalize)
 
 
-def chunk_gated_linear_attention(q, k, v, g, cu_seqlens=None, chunk=64, phi="identity"):
-    """Differentiable la_fwd_chunk_gated (unnormalised): the decay exp(g[b, t, h]) per
-    token and head; gradients reach q, k, v and the log decays g."""
-    return _ChunkGatedLinearAttention.apply(q, k, v, g, cu_seqlens, chunk, phi)
+def chunk_gated_linear_attention(q, k, v, g, cu_seqlens=None, chunk=64, phi="identity", normalize=False):
+    """Differentiable la_fwd_chunk_gated: the decay exp(g[b, t, h]) per token and head,
+    optionally normalised; gradients reach q, k, v and the log decays g."""
+    return _ChunkGatedLinearAttention.apply(q, k, v, g, cu_seqlens, chunk, phi, normalize)

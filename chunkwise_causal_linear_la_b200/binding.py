@@ -33,7 +33,8 @@ EXPORTS = ("la_fwd_chunk", "la_fwd_chunk_z", "la_fwd_chunk_gated", "la_fwd_chunk
            "la_fwd_chunk_noalloc", "la_bwd_chunk", "la_norm_gate", "la_fwd_chunk_normgate",
            "la_fwd_gated_delta", "la_fwd_gated_delta_chunk", "la_fwd_gated_delta_workspace_size",
            "la_fwd_chunk_path", "la_fwd_chunk_host", "la_fwd_chunk_host_arena_size", "la_bwd_chunk_gated",
-           "la_bwd_chunk_norm", "la_bwd_chunk_norm_workspace_size")
+           "la_bwd_chunk_norm", "la_bwd_chunk_norm_workspace_size", "la_bwd_chunk_gated_norm",
+           "la_bwd_chunk_gated_norm_workspace_size")
 
 
 class LaTensor(ctypes.Structure):
@@ -104,6 +105,10 @@ def load_library(path: str = LIB_PATH):
     lib.la_bwd_chunk_norm.restype = i32
     lib.la_bwd_chunk_norm_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32, i32]
     lib.la_bwd_chunk_norm_workspace_size.restype = sz
+    lib.la_bwd_chunk_gated_norm.argtypes = [P, P, P, P, vp, vp, i64, i32, i32, P, P, P, vp, i32, vp, sz, vp]
+    lib.la_bwd_chunk_gated_norm.restype = i32
+    lib.la_bwd_chunk_gated_norm_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32, i32]
+    lib.la_bwd_chunk_gated_norm_workspace_size.restype = sz
     lib.la_status_string.argtypes = [i32]
     lib.la_status_string.restype = ctypes.c_char_p
     lib.la_last_error.argtypes = []
@@ -420,6 +425,33 @@ def la_bwd_chunk_norm(q, k, v, dout, gamma, cu_seqlens=None, chunk=64, phi="elu1
                                _stream(stream))
     _check(lib, st, "la_bwd_chunk_norm")
     return dq, dk, dv
+
+
+def la_bwd_chunk_gated_norm(q, k, v, dout, g, cu_seqlens=None, chunk=64, phi="elu1", dq=None, dk=None, dv=None,
+                            dg=None, flags=LA_FLAG_NONE, workspace=None, stream=None):
+    """Gradients of la_fwd_chunk_gated's normalised forward (see la_bwd_chunk_gated_norm in
+    include/la_b200.h): returns (dq, dk, dv, dg), dg float32 [B, T, H] for the log decays g."""
+    lib = load_library()
+    B, T, H, d_k = q.shape
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if g.dtype != torch.float32 or tuple(g.shape) != (B, T, H) or not g.is_contiguous():
+        raise TypeError("g must be a contiguous float32 [B, T, H] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dg = torch.empty_like(g) if dg is None else dg
+    need = bwd_norm_workspace_size(B, T, H, d_k, v.shape[3], chunk, q.dtype, flags)
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    t = [describe(x) for x in (q, k, v, dout, dq, dk, dv)]
+    st = lib.la_bwd_chunk_gated_norm(*[ctypes.byref(x) for x in t[:4]], g.data_ptr(),
+                                     None if cu_seqlens is None else cu_seqlens.data_ptr(), n_seqs, int(chunk),
+                                     _PHI[phi], *[ctypes.byref(x) for x in t[4:]], dg.data_ptr(), int(flags),
+                                     None if workspace is None else workspace.data_ptr(),
+                                     0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    _check(lib, st, "la_bwd_chunk_gated_norm")
+    return dq, dk, dv, dg
 
 
 def la_norm_gate(o, gate, w, eps=1e-5, y=None, stream=None):

@@ -751,10 +751,15 @@ size_t la_bwd_chunk_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t
   return norm_bwd_plan(B, T, H, d_k, d_v, chunk, dtype, flags, &w) ? w.total : (size_t)-1;
 }
 
-la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
-                            const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
-                            const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
-                            void *workspace, size_t workspace_bytes, void *stream) {
+// Shared by la_bwd_chunk_norm (g == NULL: per-head decay gamma) and
+// la_bwd_chunk_gated_norm (g: per-token log decays; dg receives their gradient,
+// which the widened backward passes give as for la_bwd_chunk_gated: the loss sees
+// g only through the weights of num and den, both outputs of the widened problem).
+static la_status norm_bwd_common(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                                 const float *gamma, const float *g, float *dg, const int32_t *cu_seqlens,
+                                 int64_t n_seqs, int32_t chunk, int32_t phi, const la_tensor *dq, const la_tensor *dk,
+                                 const la_tensor *dv, int32_t flags, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
   la_status s;
   const la_tensor *ts[7] = {q, k, v, dout, dq, dk, dv};
   const char *names[7] = {"q", "k", "v", "dout", "dq", "dk", "dv"};
@@ -768,7 +773,9 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
   if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
-  if (!gamma) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!gamma && !g) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (g && (!dg || ((uintptr_t)g) % 4 || ((uintptr_t)dg) % 4))
+    return fail(LA_ERR_INVALID_ARG, "g and dg must be non-NULL, 4-byte aligned [B, T, H] float arrays");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
   if (flags & ~LA_FLAG_SIMT) return fail(LA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (cu_seqlens) {
@@ -811,7 +818,7 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
 
   ChunkArgs f;
   f.gamma = gamma;
-  f.g = nullptr;
+  f.g = g;
   f.cu_seqlens = cu_seqlens;
   f.final_state = nullptr;
   f.final_z = nullptr;
@@ -866,8 +873,8 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     b.chunk = chunk;
     b.phi = phi;
     b.dtype = q->dtype;
-    b.g = nullptr;
-    b.dg = nullptr;
+    b.g = g;
+    b.dg = g ? dg : nullptr;
     if (!simt_supported(f, device) || !bwd_supported(b, device))
       return fail(LA_ERR_UNSUPPORTED, "d_k %lld x widened d_v %lld does not fit the CUDA-core kernels' shared "
                   "memory", (long long)Dk, (long long)Dvp);
@@ -877,9 +884,11 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
         (err = launch_chunk_simt(f, st)) != cudaSuccess ||
         (err = launch_norm_grad_num(view(dout), up.data, B, T, H, (int)Dv, (int)Dvp, q->dtype, st)) !=
             cudaSuccess ||
+        (g && (err = cudaMemsetAsync(dg, 0, (size_t)(B * T * H) * sizeof(float), st)) != cudaSuccess) ||
         (err = launch_bwd(b, st)) != cudaSuccess ||
         (err = launch_phi_copy(view(&dv_head), view(dv), B, T, H, Dv, LA_PHI_IDENTITY, q->dtype, st)) !=
-            cudaSuccess)
+            cudaSuccess ||
+        (g && (err = launch_dg_rev_cumsum(dg, cu_seqlens, n_seqs, T, H, st)) != cudaSuccess))
       return fail(LA_ERR_CUDA, "normalised backward (CUDA cores): %s", cudaGetErrorString(err));
     return ok();
   }
@@ -897,11 +906,18 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
     set_io(qq, kk, vv, oo);
     f.phi = ph;
     f.rev = rev;
-    f.ex = x && elu ? view(x) : TensorView{nullptr, 0, 0, 0};
+    // x: the input whose gradient this pass produces; the epilogue scales by phi'(x) (elu + 1)
+    // and, with a per-token decay, adds the row term sign * phi(x) . dphi(x) to dg
+    f.ex = x && (elu || g) ? view(x) : TensorView{nullptr, 0, 0, 0};
+    f.edg = x && g ? dg : nullptr;
+    f.esign = x == k ? -1.f : 1.f;
     f.ephi = phi;
     f.edphi = x && elu ? 1 : 0;
     if (!tc_supported(f)) return cudaErrorInvalidValue;
-    return launch_chunk_tc(f, nullptr, 0, st, &why);
+    const cudaError_t e = launch_chunk_tc(f, nullptr, 0, st, &why);
+    f.ex = TensorView{nullptr, 0, 0, 0};
+    f.edg = nullptr;
+    return e;
   };
   // the normalised forward (o, and den_t from its epilogue), then u'
   f.normalize = 1;
@@ -918,14 +934,38 @@ la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_ten
   // dphi(k) = rev(v', u', phi(q)); dphi(q) = fwd(u', v', phi(k)); dv = rev(phi(k), phi(q), u'[:d_v]).
   // With elu + 1, phi(q) is staged in dq (written after it is read) and phi(k) in the workspace.
   const la_tensor *qh = elu ? dq : q, *khp = elu ? &kh : k;
-  if ((elu && (err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess) ||
+  if ((g && (err = cudaMemsetAsync(dg, 0, (size_t)(B * T * H) * sizeof(float), st)) != cudaSuccess) ||
+      (elu && (err = launch_phi_copy(view(q), view(dq), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess) ||
       (err = run(&vp, &up, qh, dk, 0, 1, k)) != cudaSuccess ||
       (elu && (err = launch_phi_copy(view(k), view(&kh), B, T, H, Dk, 1, q->dtype, st)) != cudaSuccess) ||
       (err = run(&up, &vp, khp, dq, 0, 0, q)) != cudaSuccess ||
-      (err = run(k, q, &u_head, dv, phi, 1, nullptr)) != cudaSuccess)
+      (err = run(k, q, &u_head, dv, phi, 1, nullptr)) != cudaSuccess ||
+      (g && (err = launch_dg_rev_cumsum(dg, cu_seqlens, n_seqs, T, H, st)) != cudaSuccess))
     return fail(LA_ERR_CUDA, "normalised backward (tensor cores): %s%s%s", cudaGetErrorString(err),
                 why ? ": " : "", why ? why : "");
   return ok();
+}
+
+la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                            const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
+                            const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, int32_t flags,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+  return norm_bwd_common(q, k, v, dout, gamma, nullptr, nullptr, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags,
+                         workspace, workspace_bytes, stream);
+}
+
+la_status la_bwd_chunk_gated_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
+                                  const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
+                                  int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, float *dg,
+                                  int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!g) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  return norm_bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags,
+                         workspace, workspace_bytes, stream);
+}
+
+size_t la_bwd_chunk_gated_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                              int32_t chunk, int32_t dtype, int32_t flags) {
+  return la_bwd_chunk_norm_workspace_size(B, T, H, d_k, d_v, chunk, dtype, flags);
 }
 
 la_status la_step(const la_tensor *q, const la_tensor *k, const la_tensor *v, const float *gamma, float *state,

@@ -499,6 +499,33 @@ LA_API la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const
                                    size_t workspace_bytes, void *stream);
 
 /*
+ * la_bwd_chunk_gated_norm -- backward of la_fwd_chunk_gated with normalize = 1
+ * (the data-dependent decay of "1.6 长上下文与高效注意力", section 状态空间模型与
+ * Mamba, with the normaliser of section 线性注意力): with b the prefix sums of g,
+ *     o_t = num_t / den_t,  num_t = sum_{j<=t} exp(b_t - b_j) (phi(q_t) . phi(k_j)) v_j,
+ *                           den_t = sum_{j<=t} exp(b_t - b_j)  phi(q_t) . phi(k_j).
+ * The same widening as la_bwd_chunk_norm ([v, 1] values, [u, e] output
+ * gradient) turns it into la_bwd_chunk_gated's problem, whose dg is this one's:
+ * the loss sees g only through the weights of num and den, both outputs of the
+ * widened problem.
+ *   q, k, v, g, cu_seqlens, n_seqs, chunk, phi  as for la_fwd_chunk_gated.
+ *   dout, dq, dk, dv  as for la_bwd_chunk; dg as for la_bwd_chunk_gated.
+ *   workspace   as for la_bwd_chunk_norm (la_bwd_chunk_gated_norm_workspace_size
+ *               returns the same size).
+ * Kernels: as for la_bwd_chunk_norm, with the per-token decay in every pass
+ * (the tensor-core route's forward is the normalised la_fwd_chunk_gated
+ * kernel, which also writes den_t).  Errors as for la_bwd_chunk_norm; g or dg
+ * NULL or not 4-byte aligned: LA_ERR_INVALID_ARG.
+ */
+LA_API size_t la_bwd_chunk_gated_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                                     int32_t chunk, int32_t dtype, int32_t flags);
+LA_API la_status la_bwd_chunk_gated_norm(const la_tensor *q, const la_tensor *k, const la_tensor *v,
+                                         const la_tensor *dout, const float *g, const int32_t *cu_seqlens,
+                                         int64_t n_seqs, int32_t chunk, int32_t phi, const la_tensor *dq,
+                                         const la_tensor *dk, const la_tensor *dv, float *dg, int32_t flags,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * la_fwd_chunk_noalloc -- la_fwd_chunk for callers that cannot allocate device
  * memory.  (An addition of this library; the pages have no counterpart.)
  *

@@ -138,3 +138,22 @@ def test_entry_points_from_a_fresh_thread(la):
         t.join()
         assert "e" not in got, (name, got.get("e"))
         assert torch.equal(got["x"], want), name
+
+
+def test_autograd_gated_normalised(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.autograd import chunk_gated_linear_attention
+    from chunkwise_causal_linear_la_b200.workloads import make_log_decay
+
+    dev = torch.device("cuda")
+    q, k, v, dout = _inputs(1, 150, 2, 64, 47)
+    gen = torch.Generator()
+    gen.manual_seed(48)
+    g = make_log_decay(1, 150, 2, 0.9, 0.999, gen)
+    ql, kl, vl, gl = _leaf(q, dev), _leaf(k, dev), _leaf(v, dev), g.to(dev).requires_grad_(True)
+    o = chunk_gated_linear_attention(ql, kl, vl, gl, phi="elu1", normalize=True)
+    o.backward(dout.to(dev))
+    want = la.la_bwd_chunk_gated_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), g.to(dev), phi="elu1")
+    torch.cuda.synchronize()
+    for x, r in zip((ql, kl, vl), want[:3]):
+        assert torch.equal(x.grad, r)
+    assert torch.allclose(gl.grad, want[3], rtol=1e-5, atol=1e-6 * want[3].abs().max().item())

@@ -417,3 +417,89 @@ def test_bwd_norm_unsupported(la):
         la.la_bwd_chunk_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), torch.ones(2, device=dev))
     assert e.value.status == la.binding.LA_ERR_UNSUPPORTED
     assert la.device_error(reset=True) == (0, 0)
+
+
+# ---- backward of the normalised per-token-decay forward (la_bwd_chunk_gated_norm) ----
+
+def _gated_norm_scales(oracle_mod, q, k, v, dout, g, cu, phi, slices):
+    """Error scales for dq, dk and dg (from the oracle), as _norm_bwd_scales with the
+    per-token decay: dq and dk against max(|dq|, |A|, |B|) (numerator and denominator
+    terms; one-token sequences: the same sums by absolute value); dg, a reverse
+    cumulative sum of the row terms phi(q_s) . dphi(q)_s - phi(k_s) . dphi(k)_s whose
+    numerator and denominator parts cancel (the q part exactly: a normalised row
+    does not move with the scale of phi(q_s)), against the larger of max|dg| and the
+    largest single-token sum of those parts' sizes |phi(x) . A_x| + |phi(x) . B_x|."""
+    q64, k64, v64 = q.double(), k.double(), v.double()
+    ones = torch.ones(v.shape[:3] + (1,), dtype=torch.float64)
+    den, _, _ = oracle_mod.recurrent_gated(q64, k64, ones, g, cu_seqlens=cu, phi=phi, normalize=False)
+    o, _, _ = oracle_mod.recurrent_gated(q64, k64, v64, g, cu_seqlens=cu, phi=phi, normalize=True)
+    den, o, do = torch.from_numpy(den), torch.from_numpy(o), dout.double()
+    u = do / den
+    e = -(do * o).sum(-1, keepdim=True) / den
+    aq, ak, _, _ = oracle_mod.backward_gated(q64, k64, v64, u, g, cu_seqlens=cu, phi=phi)
+    bq, bk, _, _ = oracle_mod.backward_gated(q64, k64, ones, e, g, cu_seqlens=cu, phi=phi)
+    xq, xk, _, _ = oracle_mod.backward_gated(q64, k64, torch.cat([v64.abs(), ones], -1),
+                                             torch.cat([u.abs(), e.abs()], -1), g, cu_seqlens=cu, phi=phi)
+    sq, sk = np.maximum(np.abs(aq), np.abs(bq)), np.maximum(np.abs(ak), np.abs(bk))
+    for bb, s0, e0 in slices:
+        if e0 - s0 == 1:
+            sq[bb, s0:e0], sk[bb, s0:e0] = np.abs(xq[bb, s0:e0]), np.abs(xk[bb, s0:e0])
+    qf, kf = q64.numpy(), k64.numpy()
+    if phi == "elu1":
+        fq, fk = np.where(qf > 0, qf + 1, np.exp(np.minimum(qf, 0))), np.where(kf > 0, kf + 1, np.exp(np.minimum(kf, 0)))
+        pq, pk = np.where(qf > 0, 1.0, np.exp(np.minimum(qf, 0))), np.where(kf > 0, 1.0, np.exp(np.minimum(kf, 0)))
+    else:
+        fq, fk, pq, pk = qf, kf, np.ones_like(qf), np.ones_like(kf)
+    row = (np.abs(np.sum(fq * aq / pq, -1)) + np.abs(np.sum(fq * bq / pq, -1)) +
+           np.abs(np.sum(fk * ak / pk, -1)) + np.abs(np.sum(fk * bk / pk, -1)))  # [B, T, H]
+    return sq, sk, row
+
+
+def _check_gated_norm(la, oracle_mod, q, k, v, dout, g, cu=None, phi="elu1", chunk=64, flags=0):
+    dev = torch.device("cuda")
+    dq, dk, dv, dg = la.la_bwd_chunk_gated_norm(q.to(dev), k.to(dev), v.to(dev), dout.to(dev), g.to(dev),
+                                                cu_seqlens=None if cu is None else cu.to(dev), phi=phi, chunk=chunk,
+                                                flags=flags)
+    torch.cuda.synchronize()
+    assert la.device_error(reset=True) == (0, 0)
+    g64, cu_np = g.double().numpy(), None if cu is None else cu.numpy()
+    refs = oracle_mod.backward_gated_norm(q, k, v, dout, g64, cu_seqlens=cu_np, phi=phi)
+    B, T = q.shape[:2]
+    sl = seq_slices(B, T, None if cu is None else cu.tolist())
+    sq, sk, sg = _gated_norm_scales(oracle_mod, q, k, v, dout, g64, cu_np, phi, sl)
+    assert all(np.isfinite(to_np(x)).all() for x in (dq, dk, dv, dg))
+    errs = [slice_rel_err(to_np(x), r, sl, scale=s) for x, r, s in zip((dq, dk, dv), refs[:3], (sq, sk, None))]
+    errs.append(slice_rel_err(to_np(dg)[..., None], refs[3][..., None], sl, scale=sg[..., None]))
+    assert max(errs) < TOL[q.dtype], errs
+    return errs
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 65, 300])
+def test_bwd_gated_norm_shapes(la, oracle_mod, d, T):
+    q, k, v, dout = _inputs(2, T, 2, d, d, torch.bfloat16, 3 * d + T)
+    g = _log_decay(2, T, 2, 0.8, 0.999, 5 * d + T)
+    _check_gated_norm(la, oracle_mod, q, k, v, dout, g)
+
+
+def test_bwd_gated_norm_varlen_and_identity(la, oracle_mod):
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    cu = cu_seqlens_from_lengths([130, 0, 1, 64, 65, 17])
+    q, k, v, dout = _inputs(1, int(cu[-1]), 2, 128, 128, torch.bfloat16, 61)
+    g = _log_decay(1, int(cu[-1]), 2, 0.7, 0.999, 62)
+    _check_gated_norm(la, oracle_mod, q, k, v, dout, g, cu=cu)
+    q, k, v, dout = _inputs(1, 150, 2, 64, 64, torch.bfloat16, 63)
+    _check_gated_norm(la, oracle_mod, q.abs(), k.abs(), v, dout, _log_decay(1, 150, 2, 0.9, 0.99, 64), phi="identity")
+
+
+@pytest.mark.parametrize("T", [1, 100])
+def test_bwd_gated_norm_f32_and_simt(la, oracle_mod, T):
+    """f32 (fp32 CUDA-core kernels, 1e-4) and bf16 with LA_FLAG_SIMT or another chunk."""
+    q, k, v, dout = _inputs(2, T, 2, 64, 64, torch.float32, 65 + T)
+    g = _log_decay(2, T, 2, 0.6, 0.999, 66 + T)
+    _check_gated_norm(la, oracle_mod, q, k, v, dout, g)
+    q, k, v, dout = _inputs(1, T + 37, 2, 64, 32, torch.bfloat16, 67 + T)
+    g = _log_decay(1, T + 37, 2, 0.8, 0.999, 68 + T)
+    _check_gated_norm(la, oracle_mod, q, k, v, dout, g, flags=la.LA_FLAG_SIMT)
+    _check_gated_norm(la, oracle_mod, q, k, v, dout, g, chunk=32)
