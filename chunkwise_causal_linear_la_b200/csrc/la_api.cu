@@ -532,7 +532,7 @@ static la_status bwd_common(const la_tensor *q, const la_tensor *k, const la_ten
   if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
   if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
-  if (!gamma && !g) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!gamma && !g && q->B * q->T * q->H > 0) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
   if (g && (!dg || ((uintptr_t)g) % 4 || ((uintptr_t)dg) % 4))
     return fail(LA_ERR_INVALID_ARG, "g and dg must be non-NULL, 4-byte aligned [B, T, H] float arrays");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
@@ -686,7 +686,7 @@ la_status la_bwd_chunk_gated(const la_tensor *q, const la_tensor *k, const la_te
                              const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk, int32_t phi,
                              const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, float *dg, int32_t flags,
                              void *stream) {
-  if (!g) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  if (!g && q && q->B * q->T * q->H > 0) return fail(LA_ERR_INVALID_ARG, "g is NULL");
   return bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags, stream);
 }
 
@@ -773,7 +773,7 @@ static la_status norm_bwd_common(const la_tensor *q, const la_tensor *k, const l
   if (k->D != q->D || dq->D != q->D || dk->D != q->D) return fail(LA_ERR_INVALID_ARG, "d_k disagrees");
   if (dout->D != v->D || dv->D != v->D) return fail(LA_ERR_INVALID_ARG, "d_v disagrees");
   if (q->H <= 0) return fail(LA_ERR_INVALID_ARG, "H must be positive");
-  if (!gamma && !g) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
+  if (!gamma && !g && q->B * q->T * q->H > 0) return fail(LA_ERR_INVALID_ARG, "gamma is NULL");
   if (g && (!dg || ((uintptr_t)g) % 4 || ((uintptr_t)dg) % 4))
     return fail(LA_ERR_INVALID_ARG, "g and dg must be non-NULL, 4-byte aligned [B, T, H] float arrays");
   if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1) return fail(LA_ERR_INVALID_ARG, "phi %d unknown", phi);
@@ -788,7 +788,7 @@ static la_status norm_bwd_common(const la_tensor *q, const la_tensor *k, const l
   if (!norm_bwd_plan(q->B, q->T, q->H, q->D, v->D, chunk, q->dtype, flags, &w))
     return fail(LA_ERR_UNSUPPORTED, "the normalised backward takes d_v in {16, 32, 64, 128}, d_k in "
                 "{16, 32, 64, 128, 256} and chunk in {16, 32, 64, 128}");
-  if (!workspace || workspace_bytes < w.total)
+  if (w.total > 0 && (!workspace || workspace_bytes < w.total))  // an empty problem needs none
     return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
   if (((uintptr_t)workspace) % 256 != 0) return fail(LA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
   int device = 0;
@@ -958,7 +958,7 @@ la_status la_bwd_chunk_gated_norm(const la_tensor *q, const la_tensor *k, const 
                                   const float *g, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
                                   int32_t phi, const la_tensor *dq, const la_tensor *dk, const la_tensor *dv, float *dg,
                                   int32_t flags, void *workspace, size_t workspace_bytes, void *stream) {
-  if (!g) return fail(LA_ERR_INVALID_ARG, "g is NULL");
+  if (!g && q && q->B * q->T * q->H > 0) return fail(LA_ERR_INVALID_ARG, "g is NULL");
   return norm_bwd_common(q, k, v, dout, nullptr, g, dg, cu_seqlens, n_seqs, chunk, phi, dq, dk, dv, flags,
                          workspace, workspace_bytes, stream);
 }

@@ -515,7 +515,8 @@ LA_API la_status la_bwd_chunk_norm(const la_tensor *q, const la_tensor *k, const
  * Kernels: as for la_bwd_chunk_norm, with the per-token decay in every pass
  * (the tensor-core route's forward is the normalised la_fwd_chunk_gated
  * kernel, which also writes den_t).  Errors as for la_bwd_chunk_norm; g or dg
- * NULL or not 4-byte aligned: LA_ERR_INVALID_ARG.
+ * NULL (with tokens to process) or not 4-byte aligned: LA_ERR_INVALID_ARG.
+ * A problem without tokens needs no workspace and returns LA_OK.
  */
 LA_API size_t la_bwd_chunk_gated_norm_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
                                                      int32_t chunk, int32_t dtype, int32_t flags);

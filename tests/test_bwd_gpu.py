@@ -503,3 +503,25 @@ def test_bwd_gated_norm_f32_and_simt(la, oracle_mod, T):
     g = _log_decay(1, T + 37, 2, 0.8, 0.999, 68 + T)
     _check_gated_norm(la, oracle_mod, q, k, v, dout, g, flags=la.LA_FLAG_SIMT)
     _check_gated_norm(la, oracle_mod, q, k, v, dout, g, chunk=32)
+
+
+def test_bwd_empty_inputs(la):
+    """No token to process: every backward returns without error (T = 0, B = 0, and a
+    packed batch of empty sequences), and with a per-token decay dg stays zero."""
+    from chunkwise_causal_linear_la_b200.workloads import cu_seqlens_from_lengths
+
+    dev = torch.device("cuda")
+    for B, T in ((1, 0), (0, 5)):
+        q, k, v, dout = (torch.zeros((B, T, 2, 64), dtype=torch.bfloat16, device=dev) for _ in range(4))
+        g = torch.zeros((B, T, 2), device=dev)
+        la.la_bwd_chunk(q, k, v, dout, torch.ones(2, device=dev))
+        la.la_bwd_chunk_norm(q, k, v, dout, torch.ones(2, device=dev))
+        la.la_bwd_chunk_gated(q, k, v, dout, g)
+        la.la_bwd_chunk_gated_norm(q, k, v, dout, g)
+    cu = cu_seqlens_from_lengths([0, 0, 0]).to(dev)
+    q, k, v, dout = (torch.randn((1, 4, 2, 64), device=dev).to(torch.bfloat16) for _ in range(4))
+    g = torch.zeros((1, 4, 2), device=dev)
+    dq, dk, dv, dg = la.la_bwd_chunk_gated_norm(q, k, v, dout, g, cu_seqlens=cu)
+    dq2, dk2, dv2 = la.la_bwd_chunk_norm(q, k, v, dout, torch.ones(2, device=dev), cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert la.device_error(reset=True) == (0, 0)
