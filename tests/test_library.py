@@ -297,3 +297,24 @@ def test_bwd_norm_workspace_and_validation_on_host(lib):
     st = lib.la_bwd_chunk_norm(*[ctypes.byref(x) for x in big[:4]], 0x2000, None, 1, 64, 1,
                                *[ctypes.byref(x) for x in big[4:]], 0, 0x100000, 1 << 30, None)
     assert st == b.LA_ERR_UNSUPPORTED
+
+
+def test_bwd_gated_norm_host_logic(lib):
+    """la_bwd_chunk_gated_norm takes la_bwd_chunk_norm's workspace; NULL or misaligned
+    decays and gradients are rejected before any device call when there are tokens."""
+    from chunkwise_causal_linear_la_b200 import binding as b
+
+    for args in ((3, 100, 5, 128, 128, 64, 1, 0), (3, 100, 5, 64, 32, 32, 0, 0), (3, 100, 5, 128, 256, 64, 1, 0)):
+        assert lib.la_bwd_chunk_gated_norm_workspace_size(*args) == lib.la_bwd_chunk_norm_workspace_size(*args)
+    need = lib.la_bwd_chunk_norm_workspace_size(1, 4, 2, 128, 128, 64, 1, 0)
+    t = [_t(D=128) for _ in range(7)]
+
+    def call(g=0x2000, dg=0x3000):
+        return lib.la_bwd_chunk_gated_norm(*[ctypes.byref(x) for x in t[:4]], g, None, 1, 64, 1,
+                                           *[ctypes.byref(x) for x in t[4:]], dg, 0, 0x100000, need, None)
+    assert call(g=None) == b.LA_ERR_INVALID_ARG and b"g is NULL" in lib.la_last_error()
+    assert call(dg=None) == b.LA_ERR_INVALID_ARG and b"dg" in lib.la_last_error()
+    assert call(g=0x2002) == b.LA_ERR_INVALID_ARG and b"aligned" in lib.la_last_error()
+    st = lib.la_bwd_chunk_gated(*[ctypes.byref(x) for x in t[:4]], None, None, 1, 64, 1,
+                                *[ctypes.byref(x) for x in t[4:]], 0x3000, 0, None)
+    assert st == b.LA_ERR_INVALID_ARG and b"g is NULL" in lib.la_last_error()
