@@ -413,7 +413,8 @@ LA_API la_status la_step_gated(const la_tensor *q, const la_tensor *k, const la_
  * shared memory (d_k = d_v = 128 fits; 256 does not: LA_ERR_UNSUPPORTED).
  * Tokens outside every sequence of a packed batch may be overwritten in dq,
  * dk, dv.  The normalised forward's backward is la_bwd_chunk_norm, the per-token
- * decay's la_bwd_chunk_gated.  Other errors as for la_fwd_chunk.
+ * decay's la_bwd_chunk_gated (la_bwd_chunk_gated_norm when normalised).  Other
+ * errors as for la_fwd_chunk.
  */
 LA_API la_status la_bwd_chunk(const la_tensor *q, const la_tensor *k, const la_tensor *v, const la_tensor *dout,
                               const float *gamma, const int32_t *cu_seqlens, int64_t n_seqs, int32_t chunk,
